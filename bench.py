@@ -1,0 +1,441 @@
+#!/usr/bin/env python3
+"""Benchmark of one paged decode step: kv_append + paged_attention_decode.
+
+Default workload: the Llama-3.2-1B-shaped single-layer decode step (batch 1,
+32 query / 8 KV heads, head_dim 64, 2048 cached tokens + 1 appended, block
+size 16, 4096-block shuffled pool, bf16).  ``--config N`` picks another of
+the five named workloads.  Metric: achieved HBM GB/s of the step's
+algorithmic bytes (K/V of every context token + q + out), with seq-steps/s
+alongside.
+
+Timing: W warm-up steps, then exactly K timed steps, each bracketed by CUDA
+events on the launch stream; L2 is flushed (a 512 MiB memset) before every
+step, outside the events.  Under torchrun every rank runs its own copy of the
+workload (weak scaling, no collective on the data path); the step time is
+the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload instead
+(rank 0 only); it is the deliberately slow definition the CUDA path is
+checked against, not an optimised baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode-attention achieved HBM GB/s (% of B200 peak); seq-steps/sec"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 512 << 20
+DEFAULT_CONFIG = 2
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--simt", action="store_true", help="bf16: CUDA-core decode kernel")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local, backend="nccl"):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        kw = dict(backend=backend, timeout=datetime.timedelta(seconds=120))
+        if backend == "nccl":
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(**kw)
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def esize(dt):
+    return 2 if dt == torch.bfloat16 else 4
+
+
+def step_bytes(w, out_dtype) -> int:
+    """Algorithmic bytes of one decode call: every context token's K and V
+    row once per KV head, plus q read and out written."""
+    L = int(w.decode_lens.to(torch.int64).sum().item())
+    kv = L * w.Hkv * w.d * 2 * esize(w.dtype)
+    qo = w.B * w.Hq * w.d * (esize(w.dtype) + esize(out_dtype))
+    return kv + qo
+
+
+def load_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_484_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(cfg: int):
+    """DRAM bytes per decode launch from the committed ncu capture, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    ent = rec.get("configs", {}).get(str(cfg))
+    return None if ent is None else ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML (read only) while the
+    timed region runs."""
+
+    REASONS = {
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def config_block(cfg, w, out_dtype, P, NP, simt):
+    from paged_kv_cache_484_b200 import workloads as W
+    s = W.config_summary(cfg)
+    return {
+        "workload": W.CONFIG_NAMES[cfg],
+        "batch_seqs": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
+        "context": s["ctx"], "tokens_decoded": int(w.decode_lens.to(torch.int64).sum().item()),
+        "block_size": w.block_size, "pool_blocks": w.num_blocks,
+        "kv_dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "out_dtype": "bf16" if out_dtype == torch.bfloat16 else "f32",
+        "partition_tokens": P, "max_partitions": NP,
+        "decode_kernel": "simt" if (simt or w.dtype == torch.float32) else "mma_bf16",
+        "l2": f"flushed before every step ({FLUSH_BYTES >> 20} MiB memset, outside the events)",
+    }
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def time_oracle(w, seconds: float, nthreads: int):
+    """Oracle append + decode of the whole workload (or a bounded subset of
+    sequences for the big ones), repeated until ~``seconds`` of CPU time."""
+    import oracle
+    from paged_kv_cache_484_b200.workloads import extract_sequences
+
+    order = list(range(w.B))
+    # bounded sample: whole sequences until the sample holds <= 8M context tokens
+    lens = w.decode_lens.cpu().tolist()
+    seqs, tok = [], 0
+    for b in order:
+        if seqs and tok + lens[b] > 8_000_000:
+            break
+        seqs.append(b)
+        tok += lens[b]
+    sub = extract_sequences(w, seqs)
+    frac_bytes = sum(lens[b] for b in seqs) / max(1, sum(lens))
+    reps, t_total = 0, 0.0
+    while t_total < seconds or reps == 0:
+        q = sub.q.clone()
+        kc, vc = sub.k_cache.clone(), sub.v_cache.clone()
+        t0 = time.perf_counter()
+        oracle.kv_append(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions, sub.slots, kc, vc,
+                         sub.theta)
+        oracle.paged_attention_decode(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
+                                      nthreads=nthreads)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    return t_total / reps, seqs, frac_bytes, reps
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    from paged_kv_cache_484_b200 import workloads as W
+    out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+    w = W.make_config(args.config, device="cpu")
+    nthreads = os.cpu_count() or 1
+    per_step, seqs, frac, reps = time_oracle(w, max(1.0, min(args.cpu_seconds, 60.0)), nthreads)
+    bytes_sample = step_bytes(w, out_dtype) * frac
+    value = bytes_sample / per_step / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": reps, "warmup": 0,
+        "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "seq_steps_per_s": round(len(seqs) / per_step, 3),
+        "config": config_block(args.config, w, out_dtype, None, None, False),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads,
+                         "kind": "oracle",
+                         "sample": f"{len(seqs)} of {w.B} sequences, full append+decode step, "
+                                   f"{reps} repetitions"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- CUDA arm
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, local)
+
+    import paged_kv_cache_484_b200 as pkv
+    from paged_kv_cache_484_b200 import workloads as W
+
+    pkv.load_library()
+    out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+    w = W.make_config(args.config, device=device)
+    host_inputs = None
+    if not args.no_e2e:
+        # pristine copies of the per-step inputs, in pinned host memory
+        host_inputs = {k: v.cpu().pin_memory() for k, v in dict(
+            q=w.q, k_new=w.k_new, v_new=w.v_new, positions=w.positions,
+            slot_mapping=w.slot_mapping, block_tables=w.block_tables,
+            decode_lens=w.decode_lens).items()}
+
+    P = args.partition_tokens or pkv.decode_partition_tokens(w.B, w.Hq, w.Hkv, w.d, w.max_blocks,
+                                                              kv_dtype=w.dtype)
+    NP = math.ceil(w.max_blocks * w.block_size / P)
+    ws_bytes = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=w.dtype,
+                                         partition_tokens=P)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    launches_per_step = 2 + (1 if NP > 1 else 0)
+
+    def append():
+        pkv.kv_append(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
+                      w.rope_theta, device_error=err)
+
+    def decode():
+        pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
+                                   w.scale, out, workspace=ws, partition_tokens=P,
+                                   force_simt=args.simt, device_error=err)
+
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        append()
+        decode()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error flag {int(err.item()):#x} during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    torch.cuda.synchronize()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for k in range(K):
+            flush.zero_()
+            ev[k][0].record(stream)
+            append()
+            ev[k][1].record(stream)
+            decode()
+            ev[k][2].record(stream)
+        torch.cuda.synchronize()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / K
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    step_ms_max = max_over_ranks(step_ms, world, device)
+    decode_ms_max = max_over_ranks(decode_ms, world, device)
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error flag {int(err.item()):#x} during timing")
+
+    nbytes = step_bytes(w, out_dtype)
+    value = world * nbytes / (step_ms_max * 1e-3) / 1e9
+    peak, peak_src = load_peak()
+    achieved = nbytes / (decode_ms_max * 1e-3) / 1e9
+
+    # end to end: pinned host inputs -> device, the two calls, out -> pinned host
+    e2e = None
+    if host_inputs is not None:
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dev_in = {k: getattr(w, k) for k in host_inputs}
+        h2d = sum(t.numel() * t.element_size() for t in host_inputs.values())
+        d2h = out.numel() * out.element_size()
+        Ke = max(1, min(K, 500))
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+        for k in range(Ke + 3):
+            flush.zero_()
+            if k >= 3:
+                evs[k - 3][0].record(stream)
+            for name, t in host_inputs.items():
+                dev_in[name].copy_(t, non_blocking=True)
+            append()
+            decode()
+            out_host.copy_(out, non_blocking=True)
+            if k >= 3:
+                evs[k - 3][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / Ke, world, device)
+        e2e = {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wc = W.make_config(args.config, device="cpu") if args.config in (1, 2, 3) else None
+        if wc is None:
+            # big workloads: the oracle reads a bounded subset copied from the device
+            wc = w
+        nthreads = os.cpu_count() or 1
+        per_step, seqs, frac, reps = time_oracle(wc, args.cpu_seconds, nthreads)
+        cpu = {"value": round(nbytes * frac / per_step / 1e9, 4), "unit": "GB/s",
+               "cores": nthreads, "kind": "oracle",
+               "sample": f"{len(seqs)} of {w.B} sequences, full append+decode step in fp64, "
+                         f"{reps} repetitions ({per_step * 1e3:.1f} ms each)"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": max(3, args.warmup), "ms_per_step": round(step_ms_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "pct_of_hbm_peak": round(100.0 * value / (world * peak), 2),
+        "seq_steps_per_s": round(world * w.B / (step_ms_max * 1e-3), 1),
+        "config": config_block(args.config, w, out_dtype, P, NP, args.simt),
+        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode call (decode"
+                     + (" + combine" if NP > 1 else "") + ")",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                     "decode_ms": round(decode_ms_max, 5),
+                     "traffic": recorded_traffic(args.config)},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "device": torch.cuda.get_device_name(device),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

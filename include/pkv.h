@@ -1,0 +1,232 @@
+/*
+ * pkv.h -- C ABI of the B200 (sm_100a) paged-KV decode library.
+ *
+ * Two operations make up one decode step of one attention layer over a
+ * block-structured ("paged") KV cache, the data structure the pages build
+ * their serving engines around:
+ *
+ *   pkv_kv_append               RoPE on the new token's q (in place) and k,
+ *                               then k and v written into the token's slot.
+ *   pkv_paged_attention_decode  single-query attention softmax(q K^T scale) V
+ *                               for every sequence and query head, reading K/V
+ *                               through the sequence's block table.
+ *
+ * Sources (page title, section):
+ *   "Inference From Scratch" (book intro), "What you will build" and the
+ *     chapter table: ch. 4 KV cache, ch. 8 online softmax / flash attention,
+ *     ch. 9 continuous batching, ch. 10 paged attention and block tables,
+ *     ch. 11 prefix caching by block reuse;
+ *   "The Project: Serve Your Own LLM", milestones M2 (MHA/GQA/MQA choice of
+ *     n_kv_heads), M10 (paged_gather kernel and its coalescing), M13b/M13c
+ *     (paged greedy decode equals full recompute; a block pool smaller than
+ *     the worst case);
+ *   "LLM Inference from Scratch", Architecture overview (Llama-style decoder
+ *     with RoPE and causal attention; M1 KV cache, prefill/decode
+ *     equivalence);
+ *   "warpllama", Milestones (static KV cache + single-token decode; fused
+ *     RoPE kernel; fused attention hot path in CUDA).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.   Every tensor pointer is a DEVICE pointer (cudaMalloc, the
+ *             PyTorch caching allocator, ...) unless stated otherwise.  The
+ *             caller owns every buffer, including the workspace; the library
+ *             never allocates device memory and keeps no pointer after a call
+ *             returns.
+ * Layout.     Row-major and contiguous ("[A, B, C]" means C is innermost):
+ *               q            [num_tokens or num_seqs, Hq, head_dim]
+ *               k_new, v_new [num_tokens, Hkv, head_dim]
+ *               k/v cache    [num_blocks, Hkv, block_size, head_dim]
+ *               block_tables [num_seqs, max_blocks_per_seq]  int32
+ *               out          [num_seqs, Hq, head_dim]
+ *             Token t of sequence b lives in physical block
+ *             block_tables[b][t / block_size], row t % block_size.  A slot
+ *             s names physical block s / block_size, row s % block_size.
+ * Heads.      Hq must be a multiple of Hkv; query head h reads KV head
+ *             h / (Hq / Hkv) (contiguous groups).
+ * Supported.  head_dim in {64, 128}; block_size 16; Hq / Hkv in {1, 2, 4, 8};
+ *             storage dtype fp32 or bf16 (PKV_DTYPE_*), the same for q, the
+ *             new k/v and the cache.
+ * Alignment.  q, k_new, v_new, caches, out and workspace: 16-byte aligned.
+ * Streams.    `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *             work is enqueued asynchronously on it; a call returns as soon as
+ *             its kernels are launched.
+ * Errors.     Arguments are validated on the host before anything is
+ *             launched; a bad argument returns a status and launches nothing.
+ *             The library never reads device-resident values (slots, block
+ *             ids, context lengths) on the host.  Kernels check those values
+ *             themselves: an out-of-range value sets a bit in the optional
+ *             device word `device_error` (PKV_DEVERR_*, OR-ed in, never
+ *             cleared by the library) and the offending access is skipped --
+ *             a kernel never traps and never faults on such input.  Every
+ *             wait inside a kernel is bounded; a wait that runs out sets
+ *             PKV_DEVERR_TIMEOUT and the kernel returns.
+ * Threads.    Entry points are thread-safe; calls on one stream run in order.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape */
+    PKV_ERR_UNSUPPORTED = 2, /* valid, but outside the supported set above */
+    PKV_ERR_WORKSPACE = 3,   /* workspace smaller than required */
+    PKV_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+} pkv_status;
+
+typedef enum pkv_dtype {
+    PKV_DTYPE_F32 = 0,
+    PKV_DTYPE_BF16 = 1
+} pkv_dtype;
+
+/* Bits OR-ed into *device_error by the kernels. */
+#define PKV_DEVERR_SLOT 0x1u        /* slot_mapping[t] >= num_blocks * block_size  */
+#define PKV_DEVERR_BLOCK_ID 0x2u    /* block table entry outside [0, num_blocks)   */
+#define PKV_DEVERR_CONTEXT_LEN 0x4u /* context_lens[b] < 0 or > max_blocks * bs    */
+#define PKV_DEVERR_TIMEOUT 0x8u     /* a bounded in-kernel wait ran out            */
+
+/* Decode flags. */
+#define PKV_DECODE_FORCE_SIMT 0x1u  /* bf16: use the CUDA-core kernel instead of the
+                                       tensor-core one (same result within tolerance) */
+
+/* Upper limits of one call. */
+#define PKV_MAX_SEQS_PER_CALL 4096
+#define PKV_MAX_PARTITION_TOKENS 8192
+
+/*
+ * pkv_kv_append -- rotate the new tokens' q and k, write k and v into the cache.
+ *
+ * Source: "warpllama", Milestones (static KV cache + single-token decode,
+ * fused RoPE); "LLM Inference from Scratch", Architecture overview (RoPE);
+ * "Inference From Scratch", ch. 10 (block tables: a token's K/V go to the
+ * physical slot its sequence's table assigns).
+ *
+ * For every token t < num_tokens, with p = positions[t]:
+ *   q[t, h, :]   <- rope(q[t, h, :], p)                   (in place, all h < Hq)
+ *   if s = slot_mapping[t] >= 0:
+ *     k_cache[s / bs, h, s % bs, :] <- rope(k_new[t, h, :], p)   (h < Hkv)
+ *     v_cache[s / bs, h, s % bs, :] <- v_new[t, h, :]            (bit copy)
+ * rope() turns each pair (x[i], x[i + d/2]), i < d/2, by the angle
+ * p * rope_theta^(-2i/d); the angle and the rotation are computed in fp64 and
+ * the result is rounded once to the storage type (bf16: nearest, ties to
+ * even).  A negative slot skips the cache write for that token (padding).
+ *
+ * Arguments
+ *   q             device, [num_tokens, Hq, head_dim], dtype; read and written
+ *   k_new, v_new  device, [num_tokens, Hkv, head_dim], dtype; read only
+ *   positions     device, [num_tokens] int64, >= 0
+ *   slot_mapping  device, [num_tokens] int64; < 0 = skip,
+ *                 >= num_blocks * block_size sets PKV_DEVERR_SLOT and skips
+ *   k_cache, v_cache  device, [num_blocks, Hkv, block_size, head_dim], dtype
+ *   dtype         PKV_DTYPE_F32 or PKV_DTYPE_BF16
+ *   rope_theta    RoPE base (> 0)
+ *   device_error  device int32 or NULL
+ *   stream        cudaStream_t
+ * Two tokens with the same slot race; the caller gives each token its own.
+ * num_tokens == 0 returns PKV_OK and launches nothing.
+ */
+pkv_status pkv_kv_append(void* q, const void* k_new, const void* v_new,
+                         const int64_t* positions, const int64_t* slot_mapping,
+                         void* k_cache, void* v_cache,
+                         int64_t num_tokens, int64_t num_q_heads, int64_t num_kv_heads,
+                         int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                         int32_t dtype, double rope_theta,
+                         int32_t* device_error, void* stream);
+
+/*
+ * pkv_decode_workspace_size -- bytes of workspace pkv_paged_attention_decode
+ * needs for these shapes (0 when no context is split).
+ *
+ * The workspace holds the per-partition partial results (running max, sum
+ * and un-normalised output) of the split-context ("flash-decoding") path:
+ * num_seqs * Hq * max_partitions * (head_dim + 2) floats, where
+ * max_partitions = ceil(max_blocks_per_seq * block_size / P) and P is the
+ * partition length the decode call will use (partition_tokens, or the
+ * library's choice for the current device when it is 0).  Pass the same
+ * shapes, dtype and partition_tokens to both calls.  Host only; no device
+ * memory is touched.  Returns 0 for invalid arguments.
+ */
+size_t pkv_decode_workspace_size(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                 int64_t head_dim, int64_t max_blocks_per_seq,
+                                 int64_t block_size, int32_t kv_dtype, int32_t partition_tokens);
+
+/*
+ * pkv_decode_partition_tokens -- the partition length P (tokens, a multiple of
+ * block_size) that a decode call with these shapes uses when its
+ * partition_tokens argument is 0.  Host only.  Returns 0 for invalid
+ * arguments.
+ */
+int32_t pkv_decode_partition_tokens(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                    int64_t head_dim, int64_t max_blocks_per_seq,
+                                    int64_t block_size, int32_t kv_dtype);
+
+/*
+ * pkv_paged_attention_decode -- one query token per sequence attends to its
+ * whole cached context through its block table.
+ *
+ * Source: "Inference From Scratch", ch. 8 (online softmax, flash attention)
+ * and ch. 10 (paged attention over block tables); "The Project: Serve Your
+ * Own LLM", M2 (GQA) and M13b (paged decode equals the full-recompute
+ * reference); "LLM Inference from Scratch", M1 (decode equals the last row
+ * of the full-prefix causal pass, so causal attention of the newest token
+ * covers every cached token and needs no mask inside the context).
+ *
+ * For b < num_seqs, h < Hq, with L = context_lens[b], kvh = h / (Hq / Hkv):
+ *   s_t = scale * <q[b, h, :], K_b[t]>, t < L, K_b[t] the cache row of token t
+ *   out[b, h, :] = sum_t exp(s_t - max s) V_b[t] / sum_t exp(s_t - max s)
+ * and out[b, h, :] = 0 when L == 0.  Arithmetic is fp32 (bf16 inputs widen
+ * exactly); the result is rounded once to out_dtype.
+ *
+ * Arguments
+ *   q             device, [num_seqs, Hq, head_dim], kv_dtype
+ *   k_cache, v_cache  device, [num_blocks, Hkv, block_size, head_dim], kv_dtype
+ *   block_tables  device, [num_seqs, max_blocks_per_seq] int32; only the first
+ *                 ceil(L / block_size) entries of a row are read
+ *   context_lens  device, [num_seqs] int32 in [0, max_blocks_per_seq * block_size]
+ *   out           device, [num_seqs, Hq, head_dim], out_dtype (f32 or bf16)
+ *   workspace     device, >= pkv_decode_workspace_size(...) bytes (may be NULL
+ *                 when that size is 0); contents need no initialisation and
+ *                 are clobbered; two calls in flight at once need two
+ *                 workspaces
+ *   partition_tokens  0 = library choice, else a multiple of block_size in
+ *                 [block_size, PKV_MAX_PARTITION_TOKENS]: each sequence is cut
+ *                 into ceil(L / P) partitions that run in parallel and are
+ *                 merged by a log-sum-exp combine (any P gives the same
+ *                 result up to rounding)
+ *   flags         0 or PKV_DECODE_FORCE_SIMT
+ *   device_error  device int32 or NULL
+ *   stream        cudaStream_t
+ * num_seqs == 0 returns PKV_OK and launches nothing; num_seqs is at most
+ * PKV_MAX_SEQS_PER_CALL.
+ */
+pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* context_lens,
+                                      void* out, void* workspace, size_t workspace_bytes,
+                                      int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                      int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                                      int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                      int32_t out_dtype, float scale, int32_t partition_tokens,
+                                      uint32_t flags, int32_t* device_error, void* stream);
+
+/* Short text for a status code (static storage). */
+const char* pkv_status_string(int32_t status);
+
+/* Detail of the last non-OK status returned on the calling thread (static,
+ * thread-local storage; empty when none). */
+const char* pkv_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

@@ -1,0 +1,28 @@
+"""B200-native (sm_100a) decode step over a paged KV cache.
+
+The product is the C-ABI CUDA library ``_lib/libpkv.so`` (declared in
+``include/pkv.h``); this package is its thin Python binding with the same
+operation names:
+
+* ``kv_append(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_theta, stream)``
+* ``paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, stream)``
+
+plus ``decode_workspace_size`` / ``decode_partition_tokens`` for planning.
+PyTorch is used for device memory and streams only; the library is loaded on
+first use and its absence is an error, never a fallback.
+"""
+from ._binding import (  # noqa: F401
+    BLOCK_SIZE,
+    DEVERR_BLOCK_ID,
+    DEVERR_CONTEXT_LEN,
+    DEVERR_SLOT,
+    DEVERR_TIMEOUT,
+    LIB_PATH,
+    PkvError,
+    decode_partition_tokens,
+    decode_workspace_size,
+    kv_append,
+    load_library,
+    paged_attention_decode,
+    version,
+)

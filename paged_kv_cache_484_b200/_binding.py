@@ -1,0 +1,192 @@
+"""ctypes marshalling for the C ABI in include/pkv.h.
+
+Every function here only checks tensor metadata, turns tensors into raw
+device pointers plus sizes, and calls the library; all arithmetic of the
+decode step runs in the CUDA kernels of ``_lib/libpkv.so``.  If that library
+is missing the call raises -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libpkv.so")
+
+PKV_DTYPE_F32 = 0
+PKV_DTYPE_BF16 = 1
+PKV_DECODE_FORCE_SIMT = 0x1
+DEVERR_SLOT = 0x1
+DEVERR_BLOCK_ID = 0x2
+DEVERR_CONTEXT_LEN = 0x4
+DEVERR_TIMEOUT = 0x8
+BLOCK_SIZE = 16
+
+_lock = threading.Lock()
+_lib = None
+
+
+class PkvError(RuntimeError):
+    """A non-OK status from the C ABI (``status`` holds the pkv_status code)."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libpkv.so (built by ``paged_kv_cache_484_b200.build``); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {LIB_PATH} is not built; run "
+                "`python -m paged_kv_cache_484_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32
+        lib.pkv_kv_append.argtypes = [vp, vp, vp, vp, vp, vp, vp,
+                                      i64, i64, i64, i64, i64, i64, i32, ctypes.c_double, vp, vp]
+        lib.pkv_kv_append.restype = ctypes.c_int
+        lib.pkv_decode_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32]
+        lib.pkv_decode_workspace_size.restype = ctypes.c_size_t
+        lib.pkv_decode_partition_tokens.argtypes = [i64, i64, i64, i64, i64, i64, i32]
+        lib.pkv_decode_partition_tokens.restype = i32
+        lib.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                                   i64, i64, i64, i64, i64, i64, i64,
+                                                   i32, i32, ctypes.c_float, i32, u32, vp, vp]
+        lib.pkv_paged_attention_decode.restype = ctypes.c_int
+        lib.pkv_status_string.argtypes = [i32]
+        lib.pkv_status_string.restype = ctypes.c_char_p
+        lib.pkv_last_error.argtypes = []
+        lib.pkv_last_error.restype = ctypes.c_char_p
+        lib.pkv_version.argtypes = []
+        lib.pkv_version.restype = i32
+        _lib = lib
+        return lib
+
+
+def _raise(status: int, lib, what: str):
+    if status != 0:
+        detail = lib.pkv_last_error().decode()
+        raise PkvError(status, f"{what}: {lib.pkv_status_string(status).decode()}"
+                               + (f" ({detail})" if detail else ""))
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return PKV_DTYPE_F32
+    if dt == torch.bfloat16:
+        return PKV_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {dt} (float32 or bfloat16)")
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def kv_append(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_theta,
+              stream=None, *, device_error=None) -> None:
+    """RoPE on q (in place) and k_new; write k and v into their cache slots.
+
+    q [T, Hq, d], k_new/v_new [T, Hkv, d], k_cache/v_cache [NB, Hkv, 16, d]
+    (one dtype, float32 or bfloat16), positions/slot_mapping int64 [T]
+    (slot < 0: skip the write).  See include/pkv.h, pkv_kv_append.
+    """
+    lib = load_library()
+    dt = _dtype_code(q.dtype)
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q dtype {q.dtype}")
+    T, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if k_new.shape != (T, Hkv, d) or v_new.shape != (T, Hkv, d) or v_cache.shape != k_cache.shape \
+            or d2 != d or positions.shape != (T,) or slot_mapping.shape != (T,):
+        raise ValueError("inconsistent kv_append shapes")
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_kv_append(
+        _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+        _dev(positions, "positions", torch.int64), _dev(slot_mapping, "slot_mapping", torch.int64),
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), err, _stream_ptr(stream, q.device))
+    _raise(st, lib, "kv_append")
+
+
+def decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                            kv_dtype=torch.bfloat16, block_size=BLOCK_SIZE) -> int:
+    """Partition length the decode call picks when ``partition_tokens`` is 0."""
+    lib = load_library()
+    return int(lib.pkv_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                               max_blocks_per_seq, block_size,
+                                               _dtype_code(kv_dtype)))
+
+
+def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                          kv_dtype=torch.bfloat16, partition_tokens=0,
+                          block_size=BLOCK_SIZE) -> int:
+    """Bytes of workspace ``paged_attention_decode`` needs for these shapes."""
+    lib = load_library()
+    return int(lib.pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                             max_blocks_per_seq, block_size,
+                                             _dtype_code(kv_dtype), int(partition_tokens)))
+
+
+def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                           stream=None, *, workspace=None, partition_tokens=0, force_simt=False,
+                           device_error=None) -> torch.Tensor:
+    """Single-query attention over the paged cache; writes and returns ``out``.
+
+    q [B, Hq, d] and caches [NB, Hkv, 16, d] share a dtype (float32 or
+    bfloat16); block_tables int32 [B, MB]; context_lens int32 [B];
+    out [B, Hq, d] float32 or bfloat16.  ``workspace`` (uint8 CUDA tensor of
+    at least ``decode_workspace_size`` bytes) is allocated from PyTorch's
+    caching allocator when not given.  See include/pkv.h.
+    """
+    lib = load_library()
+    kv_dt = _dtype_code(k_cache.dtype)
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share one dtype")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, Hq, d) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("inconsistent paged_attention_decode shapes")
+    out_dt = _dtype_code(out.dtype)
+    need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_paged_attention_decode(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale), int(partition_tokens),
+        PKV_DECODE_FORCE_SIMT if force_simt else 0, err, _stream_ptr(stream, q.device))
+    _raise(st, lib, "paged_attention_decode")
+    return out
+
+
+def version() -> int:
+    return int(load_library().pkv_version())

@@ -1,0 +1,937 @@
+// paged_decode.cu -- single-query attention over a paged KV cache on sm_100a.
+//
+// What it computes ("Inference From Scratch", ch. 8 online softmax and ch. 10
+// paged attention / block tables; "The Project: Serve Your Own LLM", M2 GQA):
+// for every sequence b and query head h, softmax(q K^T * scale) V over the
+// context_lens[b] tokens that block_tables[b] lists, in fp32.
+//
+// Work decomposition.  A work item is (sequence, kv head, partition): the
+// partition is P consecutive tokens of the sequence (P chosen on the host),
+// and one item serves all G = Hq / Hkv query heads of the kv head, so every
+// K/V page is read from HBM once per step.  The grid is persistent (a
+// multiple of the SM count); every CTA first turns context_lens into an
+// exclusive prefix of partition counts in shared memory, then walks items
+// i = blockIdx.x, blockIdx.x + gridDim.x, ...  Sequences that need one
+// partition write their output directly; longer ones write a partial
+// (running max, sum, normalised output) that the combine kernel merges
+// ("flash-decoding" split-K; the pages do not describe it, the log-sum-exp
+// merge below is exact up to rounding).
+//
+// Inside a CTA.  One producer warp reads the block-table entries (one lane
+// per page, prefetched a chunk ahead), and issues TMA tensor loads of each
+// 16-token K page and V page into a ring of shared-memory stages, signalled
+// by mbarriers with transaction counts; the q rows of the item ride along
+// with the item's first stage as a bulk copy.  Four consumer warps each take
+// one page per stage:
+//   * bf16 (default): S = Q K^T and O += P V on the tensor cores with
+//     mma.sync m16n8k16 (bf16 in, fp32 accumulate).  The G query heads are
+//     rows of the 16-row A tile; rows G..2G-1 repeat them so that the same
+//     MMA yields a second copy of the scores, which those rows turn into the
+//     low part of a two-term bf16 split of P (p = hi + lo, |p - hi - lo| <=
+//     2^-17 p), keeping P V accurate to fp32 level although the MMA takes
+//     bf16 operands.  K/V are read with ldmatrix from 128-byte-swizzled
+//     pages (bank-conflict free).
+//   * fp32 inputs, or bf16 with PKV_DECODE_FORCE_SIMT: CUDA cores; lanes of a
+//     token group each hold 16 bytes of the row, q.k partial sums are reduced
+//     with warp shuffles, and each token group keeps its own online softmax.
+// At the end of an item the consumer warps merge their (max, sum, output)
+// triples through shared memory and write the result.
+//
+// Every wait is bounded (PKV_DEVERR_TIMEOUT); block ids and context lengths
+// are range-checked (PKV_DEVERR_BLOCK_ID / _CONTEXT_LEN) and the bad page or
+// length is skipped or clamped instead of being dereferenced.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <type_traits>
+
+#include "pkv_device.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int NW = kConsumerWarps;
+constexpr float kNegInf = -__builtin_huge_valf();
+
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+template <typename T, int D, int G>
+struct Layout {
+    static constexpr int ESZ = sizeof(T);
+    static constexpr bool SWZ = std::is_same<T, bf16>::value;  // 128B-swizzled bf16 pages
+    static constexpr int ROW_BYTES = D * ESZ;
+    static constexpr int PAGE_BYTES = kPageRows * ROW_BYTES;
+    static constexpr int BOXES = SWZ ? D / 64 : 1;  // TMA boxes per page
+    static constexpr int BOX_BYTES = PAGE_BYTES / BOXES;
+    static constexpr int STAGE_BYTES = 2 * NW * PAGE_BYTES;  // NW K pages then NW V pages
+    static constexpr int STAGES = cmax(2, cmin(6, 65536 / STAGE_BYTES));
+    static constexpr int Q_COPY = G * D * ESZ;
+    static constexpr int Q_BYTES = round_up(Q_COPY, 128);
+    static constexpr int MERGE_FLOATS = NW * G * (D + 2);
+    // byte offsets from the 1024-aligned base
+    static constexpr int OFF_Q = STAGES * STAGE_BYTES;
+    static constexpr int OFF_MERGE = OFF_Q + STAGES * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_MERGE + 2 * MERGE_FLOATS * 4;
+    static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
+    static constexpr int OFF_MISC = OFF_MASK + STAGES * 4;  // abort flag + 8 scan slots
+    static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;       // s_len[B], s_pre[B + 1]
+    static size_t smem_bytes(int B) { return 1024 + OFF_SEQ + (size_t)(2 * B + 1) * 4; }
+};
+
+struct DecodeParams {
+    const void* q;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    void* out;
+    float* part_o;
+    float* part_ml;
+    int32_t* err;
+    int B, Hq, Hkv, MB, P, NP;
+    int num_blocks;
+    float scale_log2;
+    int out_bf16;
+};
+
+struct Item {
+    int b, h, part, t0, t1, npages, np;
+};
+
+__device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const int* s_len,
+                                            const int* s_pre) {
+    Item it;
+    const int j = i / p.Hkv;
+    it.h = i - j * p.Hkv;
+    int lo = 0, hi = p.B - 1;  // largest b with s_pre[b] <= j
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] <= j) lo = mid;
+        else hi = mid - 1;
+    }
+    it.b = lo;
+    it.part = j - s_pre[lo];
+    it.np = s_pre[lo + 1] - s_pre[lo];
+    it.t0 = it.part * p.P;
+    it.t1 = min(s_len[lo], it.t0 + p.P);
+    it.npages = (it.t1 - it.t0 + kPageRows - 1) / kPageRows;
+    return it;
+}
+
+// Byte offset of 16-byte chunk `c` of token row `tok` inside a staged page.
+template <typename T, int D>
+__device__ __forceinline__ uint32_t chunk_offset(int tok, int c) {
+    if constexpr (std::is_same<T, bf16>::value) {
+        // TMA SWIZZLE_128B: chunk index XOR (row % 8) inside each 128-byte row;
+        // D = 128 pages are two 64-column boxes of 2 KiB each.
+        if constexpr (D == 64) {
+            return tok * 128 + ((c ^ (tok & 7)) << 4);
+        } else {
+            return (c >> 3) * 2048 + tok * 128 + (((c & 7) ^ (tok & 7)) << 4);
+        }
+    } else {
+        return tok * (D * (int)sizeof(T)) + (c << 4);
+    }
+}
+
+__device__ __forceinline__ void store_out(void* out, size_t idx, float v, int out_bf16) {
+    if (out_bf16)
+        reinterpret_cast<bf16*>(out)[idx] = __float2bfloat16_rn(v);
+    else
+        reinterpret_cast<float*>(out)[idx] = v;
+}
+
+// ---------------------------------------------------------------- producer
+
+template <typename T, int D, int G>
+__device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
+                             const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
+                             uint64_t* empty, uint32_t* masks, volatile int* s_abort,
+                             const int* s_len, const int* s_pre, int W) {
+    using L = Layout<T, D, G>;
+    const int lane = threadIdx.x & 31;
+    int item = blockIdx.x;
+    if (item >= W) return;
+
+    auto entry = [&](const Item& it, int page) -> int {
+        if (page >= it.npages) return -1;
+        const int jb = it.t0 / kPageRows + page;
+        const int v = p.block_tables[(size_t)it.b * p.MB + jb];
+        if (v < 0 || v >= p.num_blocks) {
+            report_error(p.err, PKV_DEVERR_BLOCK_ID);
+            return -1;
+        }
+        return v;
+    };
+
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_parity[8];  // parity of the last issue into each stage
+    uint32_t issued_any = 0;
+    Item cur = decode_item(item, p, s_len, s_pre);
+    int c0 = 0;
+    int cur_ent = entry(cur, lane);
+    bool abort = false;
+
+    while (!abort) {
+        // prefetch the block-table entries of the next chunk of 32 pages
+        int nitem = item, nc0 = c0 + 32;
+        Item nxt = cur;
+        if (nc0 >= cur.npages) {
+            nitem = item + gridDim.x;
+            nc0 = 0;
+            if (nitem < W) nxt = decode_item(nitem, p, s_len, s_pre);
+        }
+        const int nxt_ent = (nitem < W) ? entry(nxt, nc0 + lane) : -1;
+
+        const int cend = min(cur.npages, c0 + 32);
+        for (int s0 = c0; s0 < cend; s0 += NW) {
+            const int npg = min(NW, cur.npages - s0);
+            const int k = lane - (s0 - c0);
+            const bool mine = k >= 0 && k < npg && cur_ent >= 0;
+            const uint32_t vmask = __ballot_sync(0xffffffffu, mine) >> (s0 - c0);
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1) && !*s_abort;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                abort = true;
+                break;
+            }
+            uint8_t* kdst = base + stage * L::STAGE_BYTES;
+            uint8_t* vdst = kdst + NW * L::PAGE_BYTES;
+            const bool first = (s0 == 0);
+            if (lane == 0) {
+                masks[stage] = vmask;
+                const uint32_t bytes =
+                    __popc(vmask) * 2u * L::PAGE_BYTES + (first ? (uint32_t)L::Q_COPY : 0u);
+                mbar_arrive_expect_tx(&full[stage], bytes);
+            }
+            __syncwarp();
+            if (mine) {
+                const int row0 = (cur_ent * p.Hkv + cur.h) * kPageRows;
+#pragma unroll
+                for (int bx = 0; bx < L::BOXES; ++bx) {
+                    tma_load_2d(kdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmk, bx * 64, row0,
+                                &full[stage]);
+                    tma_load_2d(vdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmv, bx * 64, row0,
+                                &full[stage]);
+                }
+            }
+            if (first && lane == 0) {
+                const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
+                                      ((size_t)cur.b * p.Hq + (size_t)cur.h * G) * D * L::ESZ;
+                bulk_load(base + L::OFF_Q + stage * L::Q_BYTES, qsrc, L::Q_COPY, &full[stage]);
+            }
+            issued_parity[stage] = phase;
+            issued_any |= 1u << stage;
+            if (++stage == L::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+        if (abort || nitem >= W) break;
+        item = nitem;
+        c0 = nc0;
+        cur = nxt;
+        cur_ent = nxt_ent;
+    }
+    if (abort) {
+        *s_abort = 1;
+        if (lane == 0) {
+            report_error(p.err, PKV_DEVERR_TIMEOUT);
+            // let every copy this warp started land before the CTA can exit
+            for (int s = 0; s < L::STAGES; ++s)
+                if (issued_any & (1u << s)) (void)mbar_wait(&full[s], issued_parity[s]);
+        }
+        __syncwarp();
+    }
+}
+
+// ------------------------------------------------------------ item merge
+
+// All consumer warps have written (o, m, l) per head into `mb`; merge them
+// and write the output row or the partition partial.
+template <int D, int G>
+__device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Item& it,
+                                                const float* mb) {
+    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+        const int g = idx / D, dim = idx - (idx / D) * D;
+        float M = kNegInf;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, mb[(w * G + g) * (D + 2) + D]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float* row = mb + (w * G + g) * (D + 2);
+            const float f = row[D] == kNegInf ? 0.f : fast_exp2(row[D] - M);
+            num += f * row[dim];
+            den += f * row[D + 1];
+        }
+        const size_t hq = (size_t)it.b * p.Hq + (size_t)it.h * G + g;
+        // den == 0 only if every page of the item was rejected (bad block ids)
+        const float val = den > 0.f ? num / den : 0.f;
+        if (it.np == 1) {
+            store_out(p.out, hq * D + dim, val, p.out_bf16);
+        } else {
+            const size_t slot = hq * p.NP + it.part;
+            p.part_o[slot * D + dim] = val;
+            if (dim == 0) {
+                p.part_ml[slot * 2] = M;
+                p.part_ml[slot * 2 + 1] = den;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------- tensor-core consumer (bf16)
+
+template <int D, int G>
+__device__ void run_consumer_mma(const DecodeParams& p, uint8_t* base, uint64_t* full,
+                                 uint64_t* empty, uint64_t* merge_bar, const uint32_t* masks,
+                                 volatile int* s_abort, const int* s_len, const int* s_pre, int W) {
+    using L = Layout<bf16, D, G>;
+    constexpr int KS = D / 16;  // k-steps of the score MMA
+    constexpr int NT = D / 8;   // n-tiles of the output MMA
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, cq = lane & 3;
+    // Which query head (and which part of the P split) this lane's A rows carry.
+    //   G == 8: rows r (c0,c1) are the high part of head r, rows r+8 the low part.
+    //   G <= 4: row r < G high part of head r, G <= r < 2G low part of head r-G.
+    const int head_a = (G == 8) ? r : (r < 2 * G ? r % G : -1);  // head in A row r
+    const int head_b = (G == 8) ? r : -1;                        // head in A row r+8
+    const bool row_is_lo = (G < 8) && (r >= G) && (r < 2 * G);
+    const bool row_used = (G == 8) || (r < 2 * G);
+
+    int stage = 0;
+    uint32_t phase = 0, mphase = 0;
+    int mbuf = 0;
+    float* merge = reinterpret_cast<float*>(base + L::OFF_MERGE);
+
+    for (int item = blockIdx.x; item < W; item += gridDim.x) {
+        const Item it = decode_item(item, p, s_len, s_pre);
+        float o[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+        float m_run = kNegInf, l_run = 0.f;
+        uint32_t qa[KS][4];
+
+        const int nst = (it.npages + NW - 1) / NW;
+        bool ok = true;
+        for (int s = 0; s < nst; ++s) {
+            ok = mbar_wait(&full[stage], phase) && !*s_abort;
+            if (!ok) break;
+            if (s == 0) {
+                // A fragments of Q: rows = query heads (see qrow_*), cols = dims.
+                const uint8_t* qs = base + L::OFF_Q + stage * L::Q_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < KS; ++kk) {
+                    const int col = kk * 16 + 2 * cq;
+                    uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+                    if (head_a >= 0) {
+                        const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_a * D * 2);
+                        a0 = qr[col / 2];
+                        a2 = qr[(col + 8) / 2];
+                    }
+                    if (head_b >= 0) {
+                        const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_b * D * 2);
+                        a1 = qr[col / 2];
+                        a3 = qr[(col + 8) / 2];
+                    }
+                    qa[kk][0] = a0;  // row r,   cols col, col+1
+                    qa[kk][1] = a1;  // row r+8
+                    qa[kk][2] = a2;  // row r,   cols col+8, col+9
+                    qa[kk][3] = a3;  // row r+8
+                }
+            }
+            const int j = s * NW + warp;
+            if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
+                const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
+                const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
+                const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
+                const int mi = lane >> 3, ri = lane & 7;
+
+                // S^T tile: 16 rows (heads) x 16 tokens, as two n-tiles of 8 tokens
+                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int kk = 0; kk < KS; ++kk) {
+                    const int tok = ri + ((mi >> 1) << 3);
+                    const int ch = 2 * kk + (mi & 1);
+                    uint32_t b00, b01, b10, b11;
+                    ldsm_x4(kbase + chunk_offset<bf16, D>(tok, ch), b00, b01, b10, b11);
+                    mma_bf16_16816(sc[0], qa[kk], b00, b01);
+                    mma_bf16_16816(sc[1], qa[kk], b10, b11);
+                }
+                // online softmax in the log2 domain; rows r carry c0, c1
+                float x[2][2];
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int tk = n * 8 + 2 * cq + e;
+                        x[n][e] = tk < valid ? sc[n][e] * p.scale_log2 : kNegInf;
+                    }
+                float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float m_new = fmaxf(m_run, mx);
+                const float alpha = fast_exp2(m_run - m_new);
+                float pr[2][2];
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) pr[n][e] = fast_exp2(x[n][e] - m_new);
+                l_run = l_run * alpha + ((pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
+                m_run = m_new;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    o[n][0] *= alpha;
+                    o[n][1] *= alpha;
+                    o[n][2] *= alpha;
+                    o[n][3] *= alpha;
+                }
+                // P as the A operand of the output MMA: two-term bf16 split
+                uint32_t pa[4];
+                {
+                    const uint32_t hi0 = pack_bf16(pr[0][0], pr[0][1]);
+                    const uint32_t hi1 = pack_bf16(pr[1][0], pr[1][1]);
+                    const uint32_t lo0 = pack_bf16(pr[0][0] - bf16lo(hi0), pr[0][1] - bf16hi(hi0));
+                    const uint32_t lo1 = pack_bf16(pr[1][0] - bf16lo(hi1), pr[1][1] - bf16hi(hi1));
+                    if (G == 8) {
+                        pa[0] = hi0;
+                        pa[1] = lo0;
+                        pa[2] = hi1;
+                        pa[3] = lo1;
+                    } else {
+                        pa[0] = row_used ? (row_is_lo ? lo0 : hi0) : 0u;
+                        pa[2] = row_used ? (row_is_lo ? lo1 : hi1) : 0u;
+                        pa[1] = 0u;
+                        pa[3] = 0u;
+                    }
+                }
+                // O += P V over the page's 16 tokens
+                uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
+                if (valid < kPageRows) {
+                    const int k0 = 2 * cq;
+                    vmask_lo = (k0 < valid ? 0x0000ffffu : 0u) | (k0 + 1 < valid ? 0xffff0000u : 0u);
+                    vmask_hi = (k0 + 8 < valid ? 0x0000ffffu : 0u) |
+                               (k0 + 9 < valid ? 0xffff0000u : 0u);
+                }
+#pragma unroll
+                for (int c = 0; c < NT; c += 2) {
+                    const int tok = ri + ((mi & 1) << 3);
+                    const int ch = c + (mi >> 1);
+                    uint32_t v0, v1, v2, v3;
+                    ldsm_x4_trans(vbase + chunk_offset<bf16, D>(tok, ch), v0, v1, v2, v3);
+                    mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
+                    mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == L::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+        if (!ok) {
+            *s_abort = 1;
+            if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
+            return;
+        }
+
+        // per-warp result for each real head: add the low-part rows
+        float of[NT][2];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            if (G == 8) {
+                of[n][0] = o[n][0] + o[n][2];
+                of[n][1] = o[n][1] + o[n][3];
+            } else {
+                of[n][0] = o[n][0] + __shfl_down_sync(0xffffffffu, o[n][0], 4 * G);
+                of[n][1] = o[n][1] + __shfl_down_sync(0xffffffffu, o[n][1], 4 * G);
+            }
+        }
+        float lsum = l_run;
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+        float* mb = merge + mbuf * L::MERGE_FLOATS;
+        if (r < G) {
+            float* row = mb + (warp * G + r) * (D + 2);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                row[n * 8 + 2 * cq] = of[n][0];
+                row[n * 8 + 2 * cq + 1] = of[n][1];
+            }
+            if (cq == 0) {
+                row[D] = m_run;
+                row[D + 1] = lsum;
+            }
+        }
+        // every consumer thread arrives once its rows are written; bounded wait
+        mbar_arrive(merge_bar);
+        if (!mbar_wait(merge_bar, mphase)) {
+            *s_abort = 1;
+            report_error(p.err, PKV_DEVERR_TIMEOUT);
+            return;
+        }
+        mphase ^= 1;
+        merge_and_store<D, G>(p, it, mb);
+        mbuf ^= 1;
+    }
+}
+
+// ------------------------------------------------------- CUDA-core consumer
+
+template <typename T, int D, int G>
+__device__ void run_consumer_simt(const DecodeParams& p, uint8_t* base, uint64_t* full,
+                                  uint64_t* empty, uint64_t* merge_bar, const uint32_t* masks,
+                                  volatile int* s_abort, const int* s_len, const int* s_pre,
+                                  int W) {
+    using L = Layout<T, D, G>;
+    constexpr bool IS_BF16 = std::is_same<T, bf16>::value;
+    constexpr int EPL = 16 / (int)sizeof(T);  // elements per lane (one 16-byte chunk)
+    constexpr int TPL = D / EPL;              // lanes per token row
+    constexpr int TPW = 32 / TPL;             // tokens per warp pass
+    constexpr int PASSES = kPageRows / TPW;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = lane % TPL, tg = lane / TPL;
+
+    int stage = 0;
+    uint32_t phase = 0, mphase = 0;
+    int mbuf = 0;
+    float* merge = reinterpret_cast<float*>(base + L::OFF_MERGE);
+
+    auto load16 = [&](uint32_t addr, float (&f)[EPL]) {
+        uint32_t w0, w1, w2, w3;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                     : "r"(addr)
+                     : "memory");
+        if constexpr (IS_BF16) {
+            f[0] = bf16lo(w0); f[1] = bf16hi(w0); f[2] = bf16lo(w1); f[3] = bf16hi(w1);
+            f[4] = bf16lo(w2); f[5] = bf16hi(w2); f[6] = bf16lo(w3); f[7] = bf16hi(w3);
+        } else {
+            f[0] = __uint_as_float(w0); f[1] = __uint_as_float(w1);
+            f[2] = __uint_as_float(w2); f[3] = __uint_as_float(w3);
+        }
+    };
+
+    for (int item = blockIdx.x; item < W; item += gridDim.x) {
+        const Item it = decode_item(item, p, s_len, s_pre);
+        float qf[G][EPL], o[G][EPL], m[G], l[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            m[g] = kNegInf;
+            l[g] = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
+        }
+        const int nst = (it.npages + NW - 1) / NW;
+        bool ok = true;
+        for (int s = 0; s < nst; ++s) {
+            ok = mbar_wait(&full[stage], phase) && !*s_abort;
+            if (!ok) break;
+            if (s == 0) {
+                const uint32_t qs = smem_addr(base + L::OFF_Q + stage * L::Q_BYTES);
+#pragma unroll
+                for (int g = 0; g < G; ++g) load16(qs + g * D * (int)sizeof(T) + c * 16, qf[g]);
+            }
+            const int j = s * NW + warp;
+            if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
+                const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
+                const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
+                const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
+#pragma unroll 2
+                for (int ps = 0; ps < PASSES; ++ps) {
+                    const int tk = ps * TPW + tg;
+                    float kv[EPL];
+                    load16(kbase + chunk_offset<T, D>(tk, c), kv);
+                    float sdot[G];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) acc = fmaf(qf[g][e], kv[e], acc);
+                        sdot[g] = acc;
+                    }
+#pragma unroll
+                    for (int off = 1; off < TPL; off <<= 1)
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            sdot[g] += __shfl_xor_sync(0xffffffffu, sdot[g], off);
+                    if (tk < valid) {
+                        float vv[EPL];
+                        load16(vbase + chunk_offset<T, D>(tk, c), vv);
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            const float x = sdot[g] * p.scale_log2;
+                            const float mn = fmaxf(m[g], x);
+                            const float a = fast_exp2(m[g] - mn);
+                            const float pe = fast_exp2(x - mn);
+                            l[g] = l[g] * a + pe;
+#pragma unroll
+                            for (int e = 0; e < EPL; ++e) o[g][e] = fmaf(pe, vv[e], o[g][e] * a);
+                            m[g] = mn;
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == L::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+        if (!ok) {
+            *s_abort = 1;
+            if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
+            return;
+        }
+        // merge the token groups of this warp
+#pragma unroll
+        for (int off = TPL; off < 32; off <<= 1) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float m2 = __shfl_xor_sync(0xffffffffu, m[g], off);
+                const float l2 = __shfl_xor_sync(0xffffffffu, l[g], off);
+                const float M = fmaxf(m[g], m2);
+                const float a = m[g] == kNegInf ? 0.f : fast_exp2(m[g] - M);
+                const float a2 = m2 == kNegInf ? 0.f : fast_exp2(m2 - M);
+                l[g] = l[g] * a + l2 * a2;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) {
+                    const float o2 = __shfl_xor_sync(0xffffffffu, o[g][e], off);
+                    o[g][e] = o[g][e] * a + o2 * a2;
+                }
+                m[g] = M;
+            }
+        }
+        float* mb = merge + mbuf * L::MERGE_FLOATS;
+        if (tg == 0) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float* row = mb + (warp * G + g) * (D + 2);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) row[c * EPL + e] = o[g][e];
+                if (c == 0) {
+                    row[D] = m[g];
+                    row[D + 1] = l[g];
+                }
+            }
+        }
+        // every consumer thread arrives once its rows are written; bounded wait
+        mbar_arrive(merge_bar);
+        if (!mbar_wait(merge_bar, mphase)) {
+            *s_abort = 1;
+            report_error(p.err, PKV_DEVERR_TIMEOUT);
+            return;
+        }
+        mphase ^= 1;
+        merge_and_store<D, G>(p, it, mb);
+        mbuf ^= 1;
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <typename T, int D, int G, bool MMA>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+    paged_decode_kernel(const __grid_constant__ DecodeParams p,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v) {
+    using L = Layout<T, D, G>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
+    uint64_t* empty = full + L::STAGES;
+    uint64_t* merge_bar = empty + L::STAGES;
+    uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
+    int* misc = reinterpret_cast<int*>(base + L::OFF_MISC);
+    volatile int* s_abort = misc;
+    int* s_warp_tot = misc + 8;
+    int* s_len = reinterpret_cast<int*>(base + L::OFF_SEQ);
+    int* s_pre = s_len + p.B;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < L::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NW);
+        }
+        mbar_init(merge_bar, NW * 32);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == NW && lane == 0) {
+        prefetch_tensor_map(&tm_k);
+        prefetch_tensor_map(&tm_v);
+    }
+
+    // Everything below reads inputs a previous kernel may have written.
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    // Partition counts per sequence and their exclusive prefix (block scan).
+    const int B = p.B;
+    const int maxlen = p.MB * kPageRows;
+    const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
+    const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
+    int local = 0;
+    for (int b = b0; b < b1; ++b) {
+        int Lb = p.context_lens[b];
+        if (Lb < 0 || Lb > maxlen) {
+            report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
+            Lb = Lb < 0 ? 0 : maxlen;
+        }
+        s_len[b] = Lb;
+        const int npb = (Lb + p.P - 1) / p.P;
+        s_pre[b] = npb;
+        local += npb;
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) s_warp_tot[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w = 0; w < warp; ++w) run += s_warp_tot[w];
+    for (int b = b0; b < b1; ++b) {
+        const int cnt = s_pre[b];
+        s_pre[b] = run;
+        run += cnt;
+    }
+    if (tid == kDecodeThreads - 1) s_pre[B] = run;
+    __syncthreads();
+    const int W = s_pre[B] * p.Hkv;
+
+    if (warp == NW) {
+        run_producer<T, D, G>(p, &tm_k, &tm_v, base, full, empty, masks, s_abort, s_len, s_pre, W);
+        return;
+    }
+    // zero the output of empty contexts (spread over the CTAs)
+    for (int b = blockIdx.x; b < B; b += gridDim.x) {
+        if (s_len[b] != 0) continue;
+        for (int idx = tid; idx < p.Hq * D; idx += NW * 32)
+            store_out(p.out, (size_t)b * p.Hq * D + idx, 0.f, p.out_bf16);
+    }
+    if constexpr (MMA) {
+        run_consumer_mma<D, G>(p, base, full, empty, merge_bar, masks, s_abort, s_len, s_pre, W);
+    } else {
+        run_consumer_simt<T, D, G>(p, base, full, empty, merge_bar, masks, s_abort, s_len, s_pre,
+                                   W);
+    }
+}
+
+// ----------------------------------------------------------------- combine
+
+struct CombineParams {
+    const int32_t* context_lens;
+    const float* part_o;
+    const float* part_ml;
+    void* out;
+    int Hq, MB, P, NP;
+    int out_bf16;
+};
+
+// out[b, h*G+g, :] = sum_p w_p o_p with w_p = l_p 2^(m_p - M) / sum_q l_q 2^(m_q - M),
+// the exact log-sum-exp merge of the partition partials.
+template <int D, int G>
+__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ CombineParams p) {
+    extern __shared__ float w[];  // [G][np]
+    grid_dependency_wait();
+    const int b = blockIdx.y, h = blockIdx.x;
+    int Lb = p.context_lens[b];
+    const int maxlen = p.MB * kPageRows;
+    Lb = Lb < 0 ? 0 : (Lb > maxlen ? maxlen : Lb);
+    const int np = (Lb + p.P - 1) / p.P;
+    if (np <= 1) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int g = warp; g < G; g += 4) {
+        const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
+        const float* ml = p.part_ml + hq * p.NP * 2;
+        float M = kNegInf;
+        for (int k = lane; k < np; k += 32) M = fmaxf(M, ml[2 * k]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float S = 0.f;
+        for (int k = lane; k < np; k += 32) {
+            const float e = ml[2 * k] == kNegInf ? 0.f : fast_exp2(ml[2 * k] - M) * ml[2 * k + 1];
+            w[g * np + k] = e;
+            S += e;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(0xffffffffu, S, off);
+        const float inv = S > 0.f ? 1.f / S : 0.f;
+        for (int k = lane; k < np; k += 32) w[g * np + k] *= inv;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D, dim = idx - (idx / D) * D;
+        const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
+        const float* po = p.part_o + hq * p.NP * D + dim;
+        float acc = 0.f;
+        for (int k = 0; k < np; ++k) acc = fmaf(w[g * np + k], po[(size_t)k * D], acc);
+        store_out(p.out, hq * D + dim, acc, p.out_bf16);
+    }
+}
+
+// ------------------------------------------------------------------- host
+
+int current_device() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+
+template <typename K>
+cudaError_t prepare_kernel(K kern, size_t smem, int* ctas_per_sm) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, size_t>, int> cache;
+    const int dev = current_device();
+    const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), dev, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        *ctas_per_sm = it->second;
+        return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    cache[key] = n;
+    *ctas_per_sm = n;
+    return cudaSuccess;
+}
+
+template <typename T, int D, int G, bool MMA>
+cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
+                                const CUtensorMap& tmv) {
+    using L = Layout<T, D, G>;
+    auto kern = paged_decode_kernel<T, D, G, MMA>;
+    const size_t smem = L::smem_bytes((int)a.B);
+    int occ = 0;
+    cudaError_t e = prepare_kernel(kern, smem, &occ);
+    if (e != cudaSuccess) return e;
+
+    DecodeParams p;
+    p.q = a.q;
+    p.block_tables = a.block_tables;
+    p.context_lens = a.context_lens;
+    p.out = a.out;
+    p.part_o = a.part_o;
+    p.part_ml = a.part_ml;
+    p.err = a.device_error;
+    p.B = (int)a.B;
+    p.Hq = (int)a.Hq;
+    p.Hkv = (int)a.Hkv;
+    p.MB = (int)a.MB;
+    p.P = a.partition_tokens;
+    p.NP = a.max_partitions;
+    p.num_blocks = (int)a.num_blocks;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.out_bf16 = a.out_dtype == PKV_DTYPE_BF16;
+
+    const int64_t upper = a.B * a.Hkv * (int64_t)a.max_partitions;
+    const int64_t resident = (int64_t)device_sm_count() * occ;
+    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min(upper, resident));
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv);
+    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+
+    CombineParams cp;
+    cp.context_lens = a.context_lens;
+    cp.part_o = a.part_o;
+    cp.part_ml = a.part_ml;
+    cp.out = a.out;
+    cp.Hq = (int)a.Hq;
+    cp.MB = (int)a.MB;
+    cp.P = a.partition_tokens;
+    cp.NP = a.max_partitions;
+    cp.out_bf16 = p.out_bf16;
+    auto ckern = combine_kernel<D, G>;
+    const size_t csmem = (size_t)G * a.max_partitions * sizeof(float);
+    cudaLaunchConfig_t cc = cfg;
+    cc.gridDim = dim3((unsigned)a.Hkv, (unsigned)a.B);
+    cc.blockDim = dim3(128);
+    cc.dynamicSmemBytes = csmem;
+    return cudaLaunchKernelEx(&cc, ckern, cp);
+}
+
+template <typename T, int D, bool MMA>
+cudaError_t dispatch_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v) {
+    switch (a.Hq / a.Hkv) {
+        case 1: return launch_decode_typed<T, D, 1, MMA>(a, k, v);
+        case 2: return launch_decode_typed<T, D, 2, MMA>(a, k, v);
+        case 4: return launch_decode_typed<T, D, 4, MMA>(a, k, v);
+        case 8: return launch_decode_typed<T, D, 8, MMA>(a, k, v);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks, int64_t Hkv,
+                             int64_t D, int32_t dtype);
+
+cudaError_t launch_paged_decode(const DecodeArgs& a) {
+    CUtensorMap tmk, tmv;
+    cudaError_t e = encode_cache_map(&tmk, a.k_cache, a.num_blocks, a.Hkv, a.D, a.kv_dtype);
+    if (e != cudaSuccess) return e;
+    e = encode_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D, a.kv_dtype);
+    if (e != cudaSuccess) return e;
+    if (a.kv_dtype == PKV_DTYPE_F32) {
+        return a.D == 64 ? dispatch_g<float, 64, false>(a, tmk, tmv)
+                         : dispatch_g<float, 128, false>(a, tmk, tmv);
+    }
+    if (a.force_simt) {
+        return a.D == 64 ? dispatch_g<bf16, 64, false>(a, tmk, tmv)
+                         : dispatch_g<bf16, 128, false>(a, tmk, tmv);
+    }
+    return a.D == 64 ? dispatch_g<bf16, 64, true>(a, tmk, tmv)
+                     : dispatch_g<bf16, 128, true>(a, tmk, tmv);
+}
+
+int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_t num_seqs) {
+    // Estimate from the shared-memory footprint (the occupancy query needs a
+    // device; this is used for host-side planning only).
+    size_t smem = 0;
+    const int B = (int)num_seqs;
+    auto pick = [&](auto tag) { smem = decltype(tag)::smem_bytes(B); };
+    if (kv_dtype == PKV_DTYPE_F32) {
+        if (D == 64) pick(Layout<float, 64, 8>{});
+        else pick(Layout<float, 128, 8>{});
+    } else {
+        if (D == 64) pick(Layout<bf16, 64, 8>{});
+        else pick(Layout<bf16, 128, 8>{});
+    }
+    (void)G;
+    (void)simt;
+    const size_t per_sm = 228 * 1024;
+    int n = (int)(per_sm / (smem + 1024));
+    return std::max(1, std::min(n, 3));
+}
+
+}  // namespace pkv

@@ -1,0 +1,379 @@
+// pkv_api.cu -- the library's C ABI: argument validation, launch planning
+// (partition length, workspace layout), TMA descriptor encoding, and error
+// reporting.  No entry point allocates device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "pkv_internal.h"
+
+namespace pkv {
+
+namespace {
+thread_local char g_last_error[512] = "";
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+}  // namespace
+
+void set_last_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+}
+
+int device_sm_count() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// ---- TMA descriptors -------------------------------------------------------
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+}  // namespace
+
+// The cache [num_blocks, Hkv, 16, D] viewed as a 2-D tensor of num_blocks*Hkv*16
+// rows of D elements; one box is one 16-row page (bf16: 64 columns per box,
+// 128-byte swizzle; fp32: the whole row, no swizzle).
+cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks, int64_t Hkv,
+                             int64_t D, int32_t dtype) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const bool bf = dtype == PKV_DTYPE_BF16;
+    const cuuint64_t rows = (cuuint64_t)(num_blocks * Hkv * kPageRows);
+    cuuint64_t dims[2] = {(cuuint64_t)D, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(D * (bf ? 2 : 4))};
+    cuuint32_t box[2] = {(cuuint32_t)(bf ? 64 : D), (cuuint32_t)kPageRows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                    const_cast<void*>(cache), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    bf ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// ---- shared validation -----------------------------------------------------
+
+namespace {
+pkv_status check_heads(int64_t Hq, int64_t Hkv, int64_t D, int64_t bs) {
+    if (Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0) {
+        set_last_error("head counts, head_dim and block_size must be positive");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (Hq % Hkv != 0) {
+        set_last_error("num_q_heads (%lld) is not a multiple of num_kv_heads (%lld)",
+                       (long long)Hq, (long long)Hkv);
+        return PKV_ERR_INVALID_ARG;
+    }
+    const int64_t G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) {
+        set_last_error("group size Hq/Hkv = %lld not in {1, 2, 4, 8}", (long long)G);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (D != 64 && D != 128) {
+        set_last_error("head_dim %lld not in {64, 128}", (long long)D);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (bs != kPageRows) {
+        set_last_error("block_size %lld unsupported (16 only)", (long long)bs);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (Hkv > 256 || Hq > 2048) {
+        set_last_error("too many heads");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    return PKV_OK;
+}
+
+bool valid_dtype(int32_t t) { return t == PKV_DTYPE_F32 || t == PKV_DTYPE_BF16; }
+
+// Partition length: aim for ~16 items per resident CTA if every sequence had
+// the maximum length, in whole stages (64 tokens), at most 1024 tokens, and
+// never more than kMaxPartitions partitions.
+int32_t auto_partition(int64_t B, int64_t Hkv, int64_t D, int64_t MB, int32_t kv_dtype) {
+    const int64_t maxlen = MB * kPageRows;
+    const int64_t resident = (int64_t)device_sm_count() * decode_ctas_per_sm(D, 0, kv_dtype, false, B);
+    const int64_t target_items = 16 * resident;
+    int64_t P = ceil_div(std::max<int64_t>(1, maxlen * B * Hkv), target_items);
+    P = ceil_div(P, kStageTokens) * kStageTokens;
+    P = std::max<int64_t>(kStageTokens, std::min<int64_t>(P, 1024));
+    const int64_t floor_np = ceil_div(ceil_div(maxlen, kMaxPartitions), kStageTokens) * kStageTokens;
+    P = std::max(P, floor_np);
+    return (int32_t)P;
+}
+
+struct WorkspacePlan {
+    int32_t P;
+    int32_t NP;
+    size_t off_ml;
+    size_t bytes;
+};
+
+pkv_status plan_workspace(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t MB,
+                          int32_t kv_dtype, int32_t partition_tokens, WorkspacePlan* out) {
+    int32_t P = partition_tokens;
+    if (P == 0) {
+        P = auto_partition(B, Hkv, D, MB, kv_dtype);
+    } else if (P < kPageRows || P % kPageRows != 0 || P > PKV_MAX_PARTITION_TOKENS) {
+        set_last_error("partition_tokens %d must be a multiple of 16 in [16, %d]", P,
+                       PKV_MAX_PARTITION_TOKENS);
+        return PKV_ERR_INVALID_ARG;
+    }
+    const int64_t NP = std::max<int64_t>(1, ceil_div(MB * kPageRows, P));
+    if (NP > kMaxPartitions) {
+        set_last_error("max_blocks_per_seq*16 / partition_tokens = %lld partitions > %d",
+                       (long long)NP, kMaxPartitions);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    out->P = P;
+    out->NP = (int32_t)NP;
+    if (NP <= 1) {
+        out->off_ml = 0;
+        out->bytes = 0;
+        return PKV_OK;
+    }
+    const size_t slots = (size_t)B * Hq * NP;
+    out->off_ml = align_up(slots * D * sizeof(float));
+    out->bytes = out->off_ml + align_up(slots * 2 * sizeof(float));
+    return PKV_OK;
+}
+
+pkv_status cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return PKV_OK;
+    set_last_error("%s: %s", what, cudaGetErrorString(e));
+    return PKV_ERR_CUDA;
+}
+}  // namespace
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+pkv_status pkv_kv_append(void* q, const void* k_new, const void* v_new, const int64_t* positions,
+                         const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                         int64_t num_tokens, int64_t num_q_heads, int64_t num_kv_heads,
+                         int64_t head_dim, int64_t num_blocks, int64_t block_size, int32_t dtype,
+                         double rope_theta, int32_t* device_error, void* stream) {
+    set_last_error("");
+    if (num_tokens < 0) {
+        set_last_error("num_tokens < 0");
+        return PKV_ERR_INVALID_ARG;
+    }
+    pkv_status st = check_heads(num_q_heads, num_kv_heads, head_dim, block_size);
+    if (st != PKV_OK) return st;
+    if (!valid_dtype(dtype)) {
+        set_last_error("dtype %d unsupported", dtype);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (!(rope_theta > 0.0)) {
+        set_last_error("rope_theta must be > 0");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (num_blocks <= 0 || num_blocks * num_kv_heads * kPageRows > INT32_MAX) {
+        set_last_error("num_blocks %lld out of range", (long long)num_blocks);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (num_tokens > INT32_MAX) {
+        set_last_error("num_tokens too large");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (num_tokens == 0) return PKV_OK;
+    if (!q || !k_new || !v_new || !positions || !slot_mapping || !k_cache || !v_cache) {
+        set_last_error("null tensor pointer");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || !aligned8(positions) || !aligned8(slot_mapping) ||
+        (device_error && !aligned4(device_error))) {
+        set_last_error("misaligned tensor pointer (16 bytes for q/k/v/caches)");
+        return PKV_ERR_INVALID_ARG;
+    }
+    AppendArgs a;
+    a.q = q;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.positions = positions;
+    a.slot_mapping = slot_mapping;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.num_tokens = num_tokens;
+    a.Hq = num_q_heads;
+    a.Hkv = num_kv_heads;
+    a.D = head_dim;
+    a.num_blocks = num_blocks;
+    a.dtype = dtype;
+    a.theta = rope_theta;
+    a.device_error = device_error;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return cuda_status(launch_kv_append(a), "kv_append launch");
+}
+
+int32_t pkv_decode_partition_tokens(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                    int64_t head_dim, int64_t max_blocks_per_seq,
+                                    int64_t block_size, int32_t kv_dtype) {
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || !valid_dtype(kv_dtype)) return 0;
+    if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
+    WorkspacePlan w;
+    if (plan_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, kv_dtype,
+                       0, &w) != PKV_OK)
+        return 0;
+    return w.P;
+}
+
+size_t pkv_decode_workspace_size(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                 int64_t head_dim, int64_t max_blocks_per_seq, int64_t block_size,
+                                 int32_t kv_dtype, int32_t partition_tokens) {
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || !valid_dtype(kv_dtype)) return 0;
+    if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
+    WorkspacePlan w;
+    if (plan_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, kv_dtype,
+                       partition_tokens, &w) != PKV_OK)
+        return 0;
+    return w.bytes;
+}
+
+pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* context_lens,
+                                      void* out, void* workspace, size_t workspace_bytes,
+                                      int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                      int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                                      int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                      int32_t out_dtype, float scale, int32_t partition_tokens,
+                                      uint32_t flags, int32_t* device_error, void* stream) {
+    set_last_error("");
+    if (num_seqs < 0 || max_blocks_per_seq < 0) {
+        set_last_error("negative num_seqs or max_blocks_per_seq");
+        return PKV_ERR_INVALID_ARG;
+    }
+    pkv_status st = check_heads(num_q_heads, num_kv_heads, head_dim, block_size);
+    if (st != PKV_OK) return st;
+    if (!valid_dtype(kv_dtype) || !valid_dtype(out_dtype)) {
+        set_last_error("kv_dtype/out_dtype unsupported");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if ((flags & ~PKV_DECODE_FORCE_SIMT) != 0) {
+        set_last_error("unknown flags 0x%x", flags);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (num_seqs > PKV_MAX_SEQS_PER_CALL) {
+        set_last_error("num_seqs %lld > %d", (long long)num_seqs, PKV_MAX_SEQS_PER_CALL);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (num_blocks <= 0 || num_blocks * num_kv_heads * kPageRows > INT32_MAX) {
+        set_last_error("num_blocks %lld out of range", (long long)num_blocks);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (max_blocks_per_seq * kPageRows > INT32_MAX / 2) {
+        set_last_error("max_blocks_per_seq too large");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) {
+        set_last_error("scale must be finite");
+        return PKV_ERR_INVALID_ARG;
+    }
+    WorkspacePlan w;
+    st = plan_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                        kv_dtype, partition_tokens, &w);
+    if (st != PKV_OK) return st;
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) {
+        set_last_error("null tensor pointer");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (max_blocks_per_seq == 0) {
+        set_last_error("max_blocks_per_seq must be > 0 when num_seqs > 0");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        !aligned4(block_tables) || !aligned4(context_lens) ||
+        (device_error && !aligned4(device_error))) {
+        set_last_error("misaligned tensor pointer (16 bytes for q/caches/out)");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (workspace_bytes < w.bytes || (w.bytes > 0 && (!workspace || !aligned16(workspace)))) {
+        set_last_error("workspace of %zu bytes given, %zu needed (16-byte aligned)",
+                       workspace_bytes, w.bytes);
+        return PKV_ERR_WORKSPACE;
+    }
+    DecodeArgs a;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.out = out;
+    a.part_o = w.bytes ? static_cast<float*>(workspace) : nullptr;
+    a.part_ml = w.bytes ? reinterpret_cast<float*>(static_cast<char*>(workspace) + w.off_ml) : nullptr;
+    a.B = num_seqs;
+    a.Hq = num_q_heads;
+    a.Hkv = num_kv_heads;
+    a.D = head_dim;
+    a.num_blocks = num_blocks;
+    a.MB = max_blocks_per_seq;
+    a.kv_dtype = kv_dtype;
+    a.out_dtype = out_dtype;
+    a.partition_tokens = w.P;
+    a.max_partitions = w.NP;
+    a.scale = scale;
+    a.force_simt = (flags & PKV_DECODE_FORCE_SIMT) != 0;
+    a.device_error = device_error;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return cuda_status(launch_paged_decode(a), "paged_attention_decode launch");
+}
+
+const char* pkv_status_string(int32_t status) {
+    switch (status) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_INVALID_ARG: return "invalid argument";
+        case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case PKV_ERR_WORKSPACE: return "workspace too small";
+        case PKV_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char* pkv_last_error(void) { return g_last_error; }
+
+int32_t pkv_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// pkv_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pkv.h"
+
+namespace pkv {
+
+constexpr int kPageRows = 16;      // tokens per cache block (block_size)
+constexpr int kConsumerWarps = 4;  // decode: warps that compute
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kStageTokens = kConsumerWarps * kPageRows;   // one page per consumer warp
+constexpr int kMaxPartitions = 1024;
+
+// Per-thread detail of the last failing call (returned by pkv_last_error).
+void set_last_error(const char* fmt, ...);
+
+struct AppendArgs {
+    void* q;
+    const void* k_new;
+    const void* v_new;
+    const int64_t* positions;
+    const int64_t* slot_mapping;
+    void* k_cache;
+    void* v_cache;
+    int64_t num_tokens, Hq, Hkv, D, num_blocks;
+    int32_t dtype;
+    double theta;
+    int32_t* device_error;
+    cudaStream_t stream;
+};
+cudaError_t launch_kv_append(const AppendArgs& a);
+
+struct DecodeArgs {
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    void* out;
+    float* part_o;   // [B, Hq, NP, D]
+    float* part_ml;  // [B, Hq, NP, 2]
+    int64_t B, Hq, Hkv, D, num_blocks, MB;
+    int32_t kv_dtype, out_dtype;
+    int32_t partition_tokens;  // P (resolved, multiple of 16)
+    int32_t max_partitions;    // NP = ceil(MB * 16 / P)
+    float scale;
+    bool force_simt;
+    int32_t* device_error;
+    cudaStream_t stream;
+};
+cudaError_t launch_paged_decode(const DecodeArgs& a);
+
+// Resident decode CTAs per SM for these shapes (occupancy query, cached).
+int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_t num_seqs);
+int device_sm_count();
+
+}  // namespace pkv

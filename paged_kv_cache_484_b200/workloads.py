@@ -213,3 +213,49 @@ def config_summary(cfg: int) -> dict:
                 dtype="bf16"),
         5: dict(B=16, Hq=32, Hkv=8, d=128, ctx="131072, 1% keys x8", dtype="bf16"),
     }[cfg]
+
+
+@dataclass
+class SequenceSubset:
+    """CPU copy of the inputs that some sequences of a workload need: their
+    pages gathered into a compact pool, block tables and slots renumbered to
+    it.  Pure data movement; physical ids carry no meaning of their own."""
+    seqs: list
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    tables: torch.Tensor
+    q: torch.Tensor
+    k_new: torch.Tensor
+    v_new: torch.Tensor
+    positions: torch.Tensor
+    slots: torch.Tensor
+    decode_lens: torch.Tensor
+    theta: float
+    scale: float
+
+
+def extract_sequences(w: Workload, seqs) -> SequenceSubset:
+    """Copy the inputs of sequences ``seqs`` to the host (read before any step
+    modifies the workload's tensors)."""
+    seqs = list(seqs)
+    bs = w.block_size
+    rows = []
+    for b in seqs:
+        n = (int(w.cached_lens[b]) + 1 + bs - 1) // bs
+        rows.append(w.block_tables[b, :n].to(torch.int64))
+    ids = torch.cat(rows)
+    uniq, inv = torch.unique(ids, return_inverse=True)
+    MB = max(r.numel() for r in rows)
+    tables = torch.full((len(seqs), MB), -1, dtype=torch.int32)
+    off = 0
+    for i, r in enumerate(rows):
+        tables[i, :r.numel()] = inv[off:off + r.numel()].to(torch.int32).cpu()
+        off += r.numel()
+    sel = torch.tensor(seqs, device=w.q.device)
+    cached = w.cached_lens[sel].cpu().to(torch.int64)
+    slots = tables[torch.arange(len(seqs)), (cached // bs)].to(torch.int64) * bs + cached % bs
+    return SequenceSubset(
+        seqs=seqs, k_cache=w.k_cache[uniq].cpu(), v_cache=w.v_cache[uniq].cpu(), tables=tables,
+        q=w.q[sel].cpu(), k_new=w.k_new[sel].cpu(), v_new=w.v_new[sel].cpu(),
+        positions=w.positions[sel].cpu(), slots=slots, decode_lens=w.decode_lens[sel].cpu(),
+        theta=w.rope_theta, scale=w.scale)

@@ -1,0 +1,133 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/pkv.h declares, and rejects bad arguments on the host with the
+documented status before any launch (no compute call is made here)."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_484_b200 as pkv
+from paged_kv_cache_484_b200 import build as lib_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+F32, BF16 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lib_build.build()
+    return pkv.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"pkv_kv_append", "pkv_paged_attention_decode", "pkv_decode_workspace_size"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in pkv.h but not exported"
+
+
+def test_library_is_built_for_sm100a():
+    log = os.path.join(lib_build.BUILD_DIR, "paged_decode.cu.log")
+    assert os.path.exists(lib_build.LIB)
+    assert "arch=compute_100a,code=sm_100a" in open(log).read()
+
+
+def test_version_and_status_strings(lib):
+    assert lib.pkv_version() >= 100
+    assert lib.pkv_status_string(0) == b"ok"
+    assert lib.pkv_status_string(3) == b"workspace too small"
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def _append(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, slot=FAKE, kc=FAKE, vc=FAKE, T=1, Hq=8, Hkv=2, d=64,
+             NB=4, bs=16, dtype=BF16, theta=1e4, err=None)
+    a.update(kw)
+    return lib.pkv_kv_append(a["q"], a["k"], a["v"], a["pos"], a["slot"], a["kc"], a["vc"], a["T"],
+                             a["Hq"], a["Hkv"], a["d"], a["NB"], a["bs"], a["dtype"], a["theta"],
+                             a["err"], None)
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, out=FAKE, ws=None, wsb=0, B=2, Hq=8, Hkv=2,
+             d=64, NB=4, bs=16, MB=4, kvdt=BF16, odt=BF16, scale=0.125, P=0, flags=0, err=None)
+    a.update(kw)
+    return lib.pkv_paged_attention_decode(a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"],
+                                          a["ws"], a["wsb"], a["B"], a["Hq"], a["Hkv"], a["d"],
+                                          a["NB"], a["bs"], a["MB"], a["kvdt"], a["odt"],
+                                          a["scale"], a["P"], a["flags"], a["err"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=48), UNSUPPORTED),
+    (dict(Hq=6, Hkv=2), UNSUPPORTED),     # group size 3
+    (dict(Hq=7, Hkv=2), INVALID),         # not a multiple
+    (dict(bs=32), UNSUPPORTED),
+    (dict(dtype=7), UNSUPPORTED),
+    (dict(theta=0.0), INVALID),
+    (dict(T=-1), INVALID),
+    (dict(q=None), INVALID),
+    (dict(kc=FAKE + 8), INVALID),          # misaligned
+    (dict(NB=0), INVALID),
+    (dict(T=0, q=None, k=None), OK),       # empty: nothing to do, nothing launched
+])
+def test_kv_append_rejects_bad_arguments(lib, kw, status):
+    assert _append(lib, **kw) == status
+    if status != OK:
+        assert lib.pkv_last_error() != b""
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(Hq=16, Hkv=1), UNSUPPORTED),     # group size 16
+    (dict(bs=8), UNSUPPORTED),
+    (dict(kvdt=2), UNSUPPORTED),
+    (dict(odt=5), UNSUPPORTED),
+    (dict(B=-1), INVALID),
+    (dict(B=5000), UNSUPPORTED),           # over PKV_MAX_SEQS_PER_CALL
+    (dict(flags=0x10), INVALID),
+    (dict(scale=math.inf), INVALID),
+    (dict(P=24), INVALID),                 # not a multiple of 16
+    (dict(P=16, MB=2000), UNSUPPORTED),    # more than 1024 partitions
+    (dict(out=None), INVALID),
+    (dict(bt=FAKE + 2), INVALID),
+    (dict(MB=0), INVALID),
+    (dict(P=16, MB=4), WORKSPACE),         # split path needs a workspace
+    (dict(B=0, q=None, out=None), OK),
+])
+def test_decode_rejects_bad_arguments(lib, kw, status):
+    assert _decode(lib, **kw) == status
+
+
+def test_workspace_size_formula(lib):
+    # 16 sequences, 32/8 heads, d 128, contexts up to 8193 blocks, P = 1024
+    n = lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, BF16, 1024)
+    NP = math.ceil(8193 * 16 / 1024)
+    slots = 16 * 32 * NP
+    a = lambda x: (x + 255) // 256 * 256
+    assert n == a(slots * 128 * 4) + a(slots * 2 * 4)
+    # a single partition needs no workspace
+    assert lib.pkv_decode_workspace_size(4, 8, 2, 64, 4, 16, BF16, 64) == 0
+    assert lib.pkv_decode_workspace_size(4, 8, 2, 64, 4, 16, BF16, 24) == 0  # invalid P -> 0
+
+
+def test_auto_partition_is_a_whole_number_of_stages(lib):
+    for (B, MB) in ((1, 129), (64, 257), (256, 2049), (16, 8193), (4096, 3)):
+        P = lib.pkv_decode_partition_tokens(B, 32, 8, 64, MB, 16, BF16)
+        assert P % 64 == 0 and 64 <= P
+        assert math.ceil(MB * 16 / P) <= 1024
