@@ -71,7 +71,7 @@ struct Layout {
     static constexpr int BOXES = SWZ ? D / 64 : 1;  // TMA boxes per page
     static constexpr int BOX_BYTES = PAGE_BYTES / BOXES;
     static constexpr int STAGE_BYTES = 2 * NW * PAGE_BYTES;  // NW K pages then NW V pages
-    static constexpr int STAGES = cmax(2, cmin(6, 65536 / STAGE_BYTES));
+    static constexpr int STAGES = cmax(2, cmin(6, 49152 / STAGE_BYTES));
     static constexpr int Q_COPY = G * D * ESZ;
     static constexpr int Q_BYTES = round_up(Q_COPY, 128);
     static constexpr int MERGE_FLOATS = NW * G * (D + 2);
@@ -744,10 +744,20 @@ struct CombineParams {
 };
 
 // out[b, h*G+g, :] = sum_p w_p o_p with w_p = l_p 2^(m_p - M) / sum_q l_q 2^(m_q - M),
-// the exact log-sum-exp merge of the partition partials.
+// the exact log-sum-exp merge of the partition partials.  One CTA per
+// (kv head, sequence): a warp per query head turns (m_p, l_p) into weights,
+// then every thread owns one float4 column chunk of one partition group and
+// accumulates all G heads at once, so all partial loads are independent;
+// the partition groups are summed through shared memory.
+constexpr int kCombineThreads = 256;
+
 template <int D, int G>
-__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ CombineParams p) {
-    extern __shared__ float w[];  // [G][np]
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_constant__ CombineParams p) {
+    constexpr int CH = D / 4;                   // float4 chunks per row
+    constexpr int PG = kCombineThreads / CH;    // partition groups
+    extern __shared__ float4 smem4[];
+    float4* red = smem4;                                       // [PG][CH]
+    float* w = reinterpret_cast<float*>(smem4 + PG * CH);      // [G][np]
     grid_dependency_wait();
     const int b = blockIdx.y, h = blockIdx.x;
     int Lb = p.context_lens[b];
@@ -756,16 +766,17 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ Co
     const int np = (Lb + p.P - 1) / p.P;
     if (np <= 1) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int g = warp; g < G; g += 4) {
+    for (int g = warp; g < G; g += kCombineThreads / 32) {
         const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
-        const float* ml = p.part_ml + hq * p.NP * 2;
+        const float2* ml = reinterpret_cast<const float2*>(p.part_ml + hq * p.NP * 2);
         float M = kNegInf;
-        for (int k = lane; k < np; k += 32) M = fmaxf(M, ml[2 * k]);
+        for (int k = lane; k < np; k += 32) M = fmaxf(M, ml[k].x);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float S = 0.f;
         for (int k = lane; k < np; k += 32) {
-            const float e = ml[2 * k] == kNegInf ? 0.f : fast_exp2(ml[2 * k] - M) * ml[2 * k + 1];
+            const float2 v = ml[k];
+            const float e = v.x == kNegInf ? 0.f : fast_exp2(v.x - M) * v.y;
             w[g * np + k] = e;
             S += e;
         }
@@ -775,13 +786,43 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ Co
         for (int k = lane; k < np; k += 32) w[g * np + k] *= inv;
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int g = idx / D, dim = idx - (idx / D) * D;
-        const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
-        const float* po = p.part_o + hq * p.NP * D + dim;
-        float acc = 0.f;
-        for (int k = 0; k < np; ++k) acc = fmaf(w[g * np + k], po[(size_t)k * D], acc);
-        store_out(p.out, hq * D + dim, acc, p.out_bf16);
+    const int ch = threadIdx.x % CH, pg = threadIdx.x / CH;
+    float4 acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const size_t hq0 = (size_t)b * p.Hq + (size_t)h * G;
+#pragma unroll 2
+    for (int k = pg; k < np; k += PG) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float4 v = reinterpret_cast<const float4*>(p.part_o + ((hq0 + g) * p.NP + k) * D)[ch];
+            const float wk = w[g * np + k];
+            acc[g].x = fmaf(wk, v.x, acc[g].x);
+            acc[g].y = fmaf(wk, v.y, acc[g].y);
+            acc[g].z = fmaf(wk, v.z, acc[g].z);
+            acc[g].w = fmaf(wk, v.w, acc[g].w);
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        red[pg * CH + ch] = acc[g];
+        __syncthreads();
+        if (threadIdx.x < CH) {
+            float4 s = red[threadIdx.x];
+            for (int q = 1; q < PG; ++q) {
+                const float4 v = red[q * CH + threadIdx.x];
+                s.x += v.x;
+                s.y += v.y;
+                s.z += v.z;
+                s.w += v.w;
+            }
+            const size_t o = (hq0 + g) * D + threadIdx.x * 4;
+            store_out(p.out, o, s.x, p.out_bf16);
+            store_out(p.out, o + 1, s.y, p.out_bf16);
+            store_out(p.out, o + 2, s.z, p.out_bf16);
+            store_out(p.out, o + 3, s.w, p.out_bf16);
+        }
+        __syncthreads();
     }
 }
 
@@ -872,10 +913,10 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     cp.NP = a.max_partitions;
     cp.out_bf16 = p.out_bf16;
     auto ckern = combine_kernel<D, G>;
-    const size_t csmem = (size_t)G * a.max_partitions * sizeof(float);
+    const size_t csmem = (size_t)kCombineThreads * 16 + (size_t)G * a.max_partitions * sizeof(float);
     cudaLaunchConfig_t cc = cfg;
     cc.gridDim = dim3((unsigned)a.Hkv, (unsigned)a.B);
-    cc.blockDim = dim3(128);
+    cc.blockDim = dim3(kCombineThreads);
     cc.dynamicSmemBytes = csmem;
     return cudaLaunchKernelEx(&cc, ckern, cp);
 }
