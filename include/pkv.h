@@ -215,6 +215,49 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
                                       int32_t out_dtype, float scale, int32_t partition_tokens,
                                       uint32_t flags, int32_t* device_error, void* stream);
 
+/* Bytes of the built-in scratch behind pkv_paged_attention_decode_noalloc.
+ * Every GPU that loads the library holds this much device memory until the
+ * process exits. */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * pkv_paged_attention_decode_noalloc -- pkv_paged_attention_decode for callers
+ * that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot hand the library a workspace.  Typical examples: a serving
+ * engine that has reserved nearly all device memory for its KV block pool and
+ * may not allocate on the decode path; a plugin interface that passes only
+ * input and output buffers; a C host without a device allocator, for which a
+ * cudaMalloc per step would also synchronise the device.
+ *
+ * Same arguments, layout, result and errors as pkv_paged_attention_decode,
+ * minus the workspace.  The split-context scratch lives in one file-scope
+ * device array of PKV_NOALLOC_SCRATCH_BYTES per GPU instead; this call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   * Shapes whose scratch need (pkv_decode_workspace_size) exceeds
+ *     PKV_NOALLOC_SCRATCH_BYTES are rejected with PKV_ERR_WORKSPACE before any
+ *     launch; a larger partition_tokens lowers the need.
+ *   * The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture.
+ *   * Every call on a device shares the one array, and it keeps the last
+ *     call's contents.  Nothing in it has to start at zero.  Calls that can
+ *     overlap on the GPU (other streams, other host threads) race on it:
+ *     serialise them, or give each its own workspace through
+ *     pkv_paged_attention_decode.
+ */
+pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache,
+                                              const void* v_cache, const int32_t* block_tables,
+                                              const int32_t* context_lens, void* out,
+                                              int64_t num_seqs, int64_t num_q_heads,
+                                              int64_t num_kv_heads, int64_t head_dim,
+                                              int64_t num_blocks, int64_t block_size,
+                                              int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                              int32_t out_dtype, float scale,
+                                              int32_t partition_tokens, uint32_t flags,
+                                              int32_t* device_error, void* stream);
+
 /* Short text for a status code (static storage). */
 const char* pkv_status_string(int32_t status);
 

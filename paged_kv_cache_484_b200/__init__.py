@@ -18,11 +18,13 @@ from ._binding import (  # noqa: F401
     DEVERR_SLOT,
     DEVERR_TIMEOUT,
     LIB_PATH,
+    NOALLOC_SCRATCH_BYTES,
     PkvError,
     decode_partition_tokens,
     decode_workspace_size,
     kv_append,
     load_library,
     paged_attention_decode,
+    paged_attention_decode_noalloc,
     version,
 )

@@ -24,6 +24,7 @@ DEVERR_BLOCK_ID = 0x2
 DEVERR_CONTEXT_LEN = 0x4
 DEVERR_TIMEOUT = 0x8
 BLOCK_SIZE = 16
+NOALLOC_SCRATCH_BYTES = 16 << 20   # PKV_NOALLOC_SCRATCH_BYTES in include/pkv.h
 
 _lock = threading.Lock()
 _lib = None
@@ -60,6 +61,11 @@ def load_library() -> ctypes.CDLL:
                                                    i64, i64, i64, i64, i64, i64, i64,
                                                    i32, i32, ctypes.c_float, i32, u32, vp, vp]
         lib.pkv_paged_attention_decode.restype = ctypes.c_int
+        lib.pkv_paged_attention_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp,
+                                                           i64, i64, i64, i64, i64, i64, i64,
+                                                           i32, i32, ctypes.c_float, i32, u32,
+                                                           vp, vp]
+        lib.pkv_paged_attention_decode_noalloc.restype = ctypes.c_int
         lib.pkv_status_string.argtypes = [i32]
         lib.pkv_status_string.restype = ctypes.c_char_p
         lib.pkv_last_error.argtypes = []
@@ -185,6 +191,39 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale), int(partition_tokens),
         PKV_DECODE_FORCE_SIMT if force_simt else 0, err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                                   stream=None, *, partition_tokens=0, force_simt=False,
+                                   device_error=None) -> torch.Tensor:
+    """``paged_attention_decode`` for callers that cannot allocate device memory.
+
+    Same arguments and result, but no workspace: the split-context scratch is
+    the library's built-in per-GPU array of NOALLOC_SCRATCH_BYTES, shared by
+    every call on the device (calls that overlap on the GPU race on it).
+    Shapes that need more scratch raise PkvError (status 3) before any launch.
+    See include/pkv.h, pkv_paged_attention_decode_noalloc.
+    """
+    lib = load_library()
+    kv_dt = _dtype_code(k_cache.dtype)
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share one dtype")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, Hq, d) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("inconsistent paged_attention_decode_noalloc shapes")
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_paged_attention_decode_noalloc(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+        B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(scale),
+        int(partition_tokens), PKV_DECODE_FORCE_SIMT if force_simt else 0, err,
+        _stream_ptr(stream, q.device))
+    _raise(st, lib, "paged_attention_decode_noalloc")
     return out
 
 
