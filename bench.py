@@ -9,8 +9,10 @@ algorithmic bytes (K/V of every context token + q + out), with seq-steps/s
 alongside.
 
 Timing: W warm-up steps, then exactly K timed steps, each bracketed by CUDA
-events on the launch stream; L2 is flushed (a 512 MiB memset) before every
-step, outside the events.  Under torchrun every rank runs its own copy of the
+events on the launch stream.  Before every step, outside the events, L2 is
+flushed: a 512 MiB buffer is written, then a second 256 MiB buffer is read, so
+that the dirty lines of the write are written back before the step starts
+instead of inside it.  Under torchrun every rank runs its own copy of the
 workload (weak scaling, no collective on the data path); the step time is
 the max over ranks.
 
@@ -51,6 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--simt", action="store_true", help="bf16: CUDA-core decode kernel")
+    ap.add_argument("--two-calls", action="store_true",
+                    help="time kv_append + paged_attention_decode as two launches instead of "
+                         "the single-launch decode_step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
@@ -204,7 +209,7 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def config_block(cfg, w, out_dtype, P, NP, simt):
+def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
     from paged_kv_cache_484_b200 import workloads as W
     s = W.config_summary(cfg)
     return {
@@ -216,7 +221,10 @@ def config_block(cfg, w, out_dtype, P, NP, simt):
         "out_dtype": "bf16" if out_dtype == torch.bfloat16 else "f32",
         "partition_tokens": P, "max_partitions": NP,
         "decode_kernel": "simt" if (simt or w.dtype == torch.float32) else "mma_bf16",
-        "l2": f"flushed before every step ({FLUSH_BYTES >> 20} MiB memset, outside the events)",
+        "step": "two calls (kv_append, paged_attention_decode)" if two_calls
+                else "one launch (decode_step: append fused into the decode kernel)",
+        "l2": f"flushed before every step outside the events ({FLUSH_BYTES >> 20} MiB written, "
+              f"then {FLUSH_BYTES >> 21} MiB read so no dirty lines remain)",
     }
 
 
@@ -314,21 +322,36 @@ def run_ours(args):
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
     out = torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
-    launches_per_step = 2 + (1 if NP > 1 else 0)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush_r = torch.ones(FLUSH_BYTES // 2, dtype=torch.uint8, device=device)
+
+    def flush_l2():
+        flush_w.zero_()      # evict: write more than L2 holds
+        flush_r.max()        # then read more than L2 holds, so no dirty line is left
+
+    fused = not args.two_calls
+    kernels_per_decode = 1 + (1 if NP > 1 else 0)      # decode (+ split-context combine)
+    launches_per_step = kernels_per_decode + (0 if fused else 1)
 
     def append():
-        pkv.kv_append(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
-                      w.rope_theta, device_error=err)
+        if not fused:
+            pkv.kv_append(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                          w.v_cache, w.rope_theta, device_error=err)
 
     def decode():
-        pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
-                                   w.scale, out, workspace=ws, partition_tokens=P,
-                                   force_simt=args.simt, device_error=err)
+        if fused:
+            pkv.decode_step(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                            w.v_cache, w.block_tables, w.decode_lens, w.rope_theta, w.scale, out,
+                            workspace=ws, partition_tokens=P, force_simt=args.simt,
+                            device_error=err)
+        else:
+            pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
+                                       w.scale, out, workspace=ws, partition_tokens=P,
+                                       force_simt=args.simt, device_error=err)
 
     stream = torch.cuda.current_stream(device)
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush_l2()
         append()
         decode()
     torch.cuda.synchronize()
@@ -342,7 +365,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         for k in range(K):
-            flush.zero_()
+            flush_l2()
             ev[k][0].record(stream)
             append()
             ev[k][1].record(stream)
@@ -373,7 +396,7 @@ def run_ours(args):
         Ke = max(1, min(K, 500))
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
         for k in range(Ke + 3):
-            flush.zero_()
+            flush_l2()
             if k >= 3:
                 evs[k - 3][0].record(stream)
             for name, t in host_inputs.items():
@@ -409,9 +432,10 @@ def run_ours(args):
         "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "pct_of_hbm_peak": round(100.0 * value / (world * peak), 2),
         "seq_steps_per_s": round(world * w.B / (step_ms_max * 1e-3), 1),
-        "config": config_block(args.config, w, out_dtype, P, NP, args.simt),
-        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode call (decode"
-                     + (" + combine" if NP > 1 else "") + ")",
+        "config": config_block(args.config, w, out_dtype, P, NP, args.simt, args.two_calls),
+        "roofline": {"bound": "hbm",
+                     "kernel": ("decode_step" if fused else "paged_attention_decode")
+                     + " call: paged_decode_kernel" + (" + combine_kernel" if NP > 1 else ""),
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "decode_ms": round(decode_ms_max, 5),

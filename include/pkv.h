@@ -215,6 +215,49 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
                                       int32_t out_dtype, float scale, int32_t partition_tokens,
                                       uint32_t flags, int32_t* device_error, void* stream);
 
+/*
+ * pkv_decode_step -- one whole decode step in ONE launch: the effect of
+ * pkv_kv_append (one new token per sequence) followed by
+ * pkv_paged_attention_decode.
+ *
+ * Source: "warpllama", Milestones (static KV cache + single-token decode;
+ * fused RoPE; the attention hot path as one hand-written CUDA kernel);
+ * "Inference From Scratch", ch. 4 and ch. 10 (the new token's K/V go into its
+ * sequence's cache block, then the token attends to the whole cache).
+ *
+ * Token b of the append is sequence b's new token.  Every warp of the decode
+ * kernel rotates the q elements it feeds to its own MMA fragments (fp64, as
+ * pkv_kv_append computes them, rounded to the storage type), and the CTA that
+ * holds a sequence's last cache page rotates the new k, writes k and v into
+ * the slot and patches them into the staged page, so no separate append
+ * launch and no extra pass over memory is needed.  q itself is only read:
+ * unlike pkv_kv_append, the step does not store the rotated q (it is used
+ * inside the kernel only), so q can be shared by all partitions at once.
+ *
+ * Precondition: the new token is the last token of its context, i.e.
+ * context_lens[b] >= 1 and slot_mapping[b] is the slot that block_tables[b]
+ * gives token context_lens[b] - 1.  A sequence whose slot_mapping[b] is
+ * negative is not appended (its cached context is attended as is); one whose
+ * slot differs from that table slot gets PKV_DEVERR_SLOT and is not appended
+ * either.  A context of length 0 gives an all-zero output row and the token
+ * is appended as pkv_kv_append would.
+ *
+ * Arguments: those of the two calls (q [num_seqs, Hq, d], read only;
+ * k_new, v_new [num_seqs, Hkv, d]; positions, slot_mapping
+ * [num_seqs] int64), one dtype for q, the new rows and the cache.  The
+ * workspace is sized and owned exactly as for pkv_paged_attention_decode.
+ */
+pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new,
+                           const int64_t* positions, const int64_t* slot_mapping,
+                           void* k_cache, void* v_cache, const int32_t* block_tables,
+                           const int32_t* context_lens, void* out, void* workspace,
+                           size_t workspace_bytes, int64_t num_seqs, int64_t num_q_heads,
+                           int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                           int64_t block_size, int64_t max_blocks_per_seq, int32_t kv_dtype,
+                           int32_t out_dtype, double rope_theta, float scale,
+                           int32_t partition_tokens, uint32_t flags, int32_t* device_error,
+                           void* stream);
+
 /* Bytes of the built-in scratch behind pkv_paged_attention_decode_noalloc.
  * Every GPU that loads the library holds this much device memory until the
  * process exits. */

@@ -7,7 +7,8 @@ operation names:
 * ``kv_append(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_theta, stream)``
 * ``paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, stream)``
 
-plus ``decode_workspace_size`` / ``decode_partition_tokens`` for planning.
+plus ``decode_step`` (both in one launch), ``paged_attention_decode_noalloc``
+and ``decode_workspace_size`` / ``decode_partition_tokens`` for planning.
 PyTorch is used for device memory and streams only; the library is loaded on
 first use and its absence is an error, never a fallback.
 """
@@ -21,6 +22,7 @@ from ._binding import (  # noqa: F401
     NOALLOC_SCRATCH_BYTES,
     PkvError,
     decode_partition_tokens,
+    decode_step,
     decode_workspace_size,
     kv_append,
     load_library,

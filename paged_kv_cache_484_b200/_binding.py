@@ -61,6 +61,11 @@ def load_library() -> ctypes.CDLL:
                                                    i64, i64, i64, i64, i64, i64, i64,
                                                    i32, i32, ctypes.c_float, i32, u32, vp, vp]
         lib.pkv_paged_attention_decode.restype = ctypes.c_int
+        lib.pkv_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                        ctypes.c_size_t, i64, i64, i64, i64, i64, i64, i64,
+                                        i32, i32, ctypes.c_double, ctypes.c_float, i32, u32,
+                                        vp, vp]
+        lib.pkv_decode_step.restype = ctypes.c_int
         lib.pkv_paged_attention_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp,
                                                            i64, i64, i64, i64, i64, i64, i64,
                                                            i32, i32, ctypes.c_float, i32, u32,
@@ -191,6 +196,46 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale), int(partition_tokens),
         PKV_DECODE_FORCE_SIMT if force_simt else 0, err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode")
+    return out
+
+
+def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
+                context_lens, rope_theta, scale, out, stream=None, *, workspace=None,
+                partition_tokens=0, force_simt=False, device_error=None) -> torch.Tensor:
+    """``kv_append`` (one new token per sequence) then ``paged_attention_decode``,
+    in one launch.  The new token must be the last token of its context
+    (context_lens[b] - 1, at the slot block_tables gives it).  q is read only:
+    the rotated q is used inside the kernel and not stored.  See include/pkv.h,
+    pkv_decode_step.
+    """
+    lib = load_library()
+    kv_dt = _dtype_code(k_cache.dtype)
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("v_cache", v_cache)):
+        if t.dtype != k_cache.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from the cache dtype {k_cache.dtype}")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, Hq, d) \
+            or k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d) \
+            or positions.shape != (B,) or slot_mapping.shape != (B,) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("inconsistent decode_step shapes")
+    need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_decode_step(
+        _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+        _dev(positions, "positions", torch.int64), _dev(slot_mapping, "slot_mapping", torch.int64),
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(rope_theta), float(scale),
+        int(partition_tokens), PKV_DECODE_FORCE_SIMT if force_simt else 0, err,
+        _stream_ptr(stream, q.device))
+    _raise(st, lib, "decode_step")
     return out
 
 

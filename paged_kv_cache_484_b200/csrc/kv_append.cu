@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_kernel(
     const bool live0 = idx0 < total && (idx0 < nq || write_kv);
     for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
         double s, c;
-        sincos((double)pos * fr.f[i], &s, &c);
+        sincos(reduce_two_pi((double)pos * fr.f[i]), &s, &c);
         s_cos[i] = c;
         s_sin[i] = s;
     }

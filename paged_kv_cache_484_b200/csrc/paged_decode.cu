@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cmath>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -74,14 +75,20 @@ struct Layout {
     static constexpr int STAGES = cmax(2, cmin(6, 49152 / STAGE_BYTES));
     static constexpr int Q_COPY = G * D * ESZ;
     static constexpr int Q_BYTES = round_up(Q_COPY, 128);
+    static constexpr int ROW_COPY = D * ESZ;           // one k or v row
+    static constexpr int NEWKV_BYTES = 2 * ROW_COPY;   // fused step: raw new k row, new v row
     static constexpr int MERGE_FLOATS = NW * G * (D + 2);
     // byte offsets from the 1024-aligned base
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
-    static constexpr int OFF_MERGE = OFF_Q + STAGES * Q_BYTES;
+    static constexpr int OFF_NEWKV = OFF_Q + STAGES * Q_BYTES;
+    // fused step: one cos[D/2], sin[D/2] fp64 table per consumer warp
+    static constexpr int OFF_ROPE = OFF_NEWKV + STAGES * NEWKV_BYTES;
+    static constexpr int OFF_MERGE = OFF_ROPE + NW * D * 8;
     static constexpr int OFF_BAR = OFF_MERGE + 2 * MERGE_FLOATS * 4;
     static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
-    static constexpr int OFF_MISC = OFF_MASK + STAGES * 4;  // abort flag + 8 scan slots
-    static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;       // s_len[B], s_pre[B + 1]
+    static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
+    static constexpr int OFF_MISC = OFF_PATCH + STAGES * 8;  // abort flag + 8 scan slots
+    static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;        // s_len[B], s_pre[B + 1]
     static size_t smem_bytes(int B) { return 1024 + OFF_SEQ + (size_t)(2 * B + 1) * 4; }
 };
 
@@ -97,6 +104,17 @@ struct DecodeParams {
     int num_blocks;
     float scale_log2;
     int out_bf16;
+    // fused step only: the new token of every sequence
+    const void* k_new;            // [B, Hkv, D]
+    const void* v_new;            // [B, Hkv, D]
+    const int64_t* positions;     // [B]
+    const int64_t* slot_mapping;  // [B]
+    void* k_cache;                // cache bases for the new rows
+    void* v_cache;
+};
+
+struct RopeFreq {
+    double f[64];  // theta^(-2i/d), i < d/2 (fused step)
 };
 
 struct Item {
@@ -146,9 +164,120 @@ __device__ __forceinline__ void store_out(void* out, size_t idx, float v, int ou
         reinterpret_cast<float*>(out)[idx] = v;
 }
 
+
+// ---- fused step: RoPE on the new token inside the decode kernel ------------
+// Same arithmetic as kv_append.cu: fp64 angle, sine/cosine and rotation, one
+// rounding to the storage type.
+
+template <typename T>
+__device__ __forceinline__ double to_d(T x);
+template <>
+__device__ __forceinline__ double to_d<float>(float x) { return (double)x; }
+template <>
+__device__ __forceinline__ double to_d<bf16>(bf16 x) { return (double)__bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_d(double x);
+template <>
+__device__ __forceinline__ float from_d<float>(double x) { return __double2float_rn(x); }
+template <>
+__device__ __forceinline__ bf16 from_d<bf16>(double x) {
+    const uint16_t b = double_to_bf16_bits(x);
+    return *reinterpret_cast<const bf16*>(&b);
+}
+
+// Fused step: one warp's cos/sin table of a position, tab[i] = cos(pos f_i),
+// tab[D/2 + i] = sin(pos f_i) for i < D/2 (fp64, angle reduced first).
+template <int D>
+__device__ __forceinline__ void warp_rope_table(double pos, const RopeFreq& fr, double* tab) {
+    for (int i = threadIdx.x & 31; i < D / 2; i += 32) {
+        double sn, cs;
+        sincos(reduce_two_pi(pos * fr.f[i]), &sn, &cs);
+        tab[i] = cs;
+        tab[D / 2 + i] = sn;
+    }
+    __syncwarp();
+}
+
+// Element `col` of the rotated row (row in storage type T): the pair partner is
+// col +- D/2; fp64 rotation, as kv_append computes it.
+template <typename T, int D>
+__device__ __forceinline__ double rotated_elem(const T* row, int col, const double* tab) {
+    constexpr int HALF = D / 2;
+    const int i = col < HALF ? col : col - HALF;
+    const double x = to_d<T>(row[col]);
+    const double y = to_d<T>(row[col < HALF ? col + HALF : col - HALF]);
+    return col < HALF ? x * tab[i] - y * tab[HALF + i] : x * tab[i] + y * tab[HALF + i];
+}
+
+// One warp writes the new token's rotated k row and raw v row into row r of
+// the staged K and V pages (overwriting what the TMA brought) and into the
+// cache rows in global memory; then orders its shared-memory writes before
+// any later TMA write into the same stage.
+template <typename T, int D>
+__device__ void patch_new_row(uint8_t* kpage, uint8_t* vpage, const uint8_t* newkv, int r,
+                              const double* tab, T* kglob, T* vglob) {
+    const double* rc = tab;
+    const double* rs = tab + D / 2;
+    constexpr int HALF = D / 2, E = 16 / (int)sizeof(T), CH = D * (int)sizeof(T) / 16;
+    const int lane = threadIdx.x & 31;
+    const T* kn = reinterpret_cast<const T*>(newkv);
+    const uint8_t* vn = newkv + D * sizeof(T);
+    for (int i = lane; i < HALF; i += 32) {
+        const double x0 = to_d<T>(kn[i]), x1 = to_d<T>(kn[i + HALF]);
+        const T y0 = from_d<T>(x0 * rc[i] - x1 * rs[i]);
+        const T y1 = from_d<T>(x1 * rc[i] + x0 * rs[i]);
+        const int i1 = i + HALF;
+        *reinterpret_cast<T*>(kpage + chunk_offset<T, D>(r, i / E) + (i % E) * sizeof(T)) = y0;
+        *reinterpret_cast<T*>(kpage + chunk_offset<T, D>(r, i1 / E) + (i1 % E) * sizeof(T)) = y1;
+        kglob[i] = y0;
+        kglob[i1] = y1;
+    }
+    for (int c = lane; c < CH; c += 32) {
+        const uint4 v = *reinterpret_cast<const uint4*>(vn + c * 16);
+        *reinterpret_cast<uint4*>(vpage + chunk_offset<T, D>(r, c)) = v;
+        reinterpret_cast<uint4*>(vglob)[c] = v;
+    }
+    __syncwarp();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Fused step, context length 0: no attention, but the new token's k (rotated)
+// and v still go into a valid slot, as kv_append would put them.  Run by the
+// consumer threads of one CTA.
+template <typename T, int D>
+__device__ void append_only(const DecodeParams& p, const RopeFreq& fr, int b) {
+    constexpr int HALF = D / 2;
+    const double pos = (double)p.positions[b];
+    const int64_t slot = p.slot_mapping[b];
+    const int64_t num_slots = (int64_t)p.num_blocks * kPageRows;
+    const bool write_kv = slot >= 0 && slot < num_slots;
+    if (slot >= num_slots && threadIdx.x == 0) report_error(p.err, PKV_DEVERR_SLOT);
+    const T* kn = reinterpret_cast<const T*>(p.k_new) + (size_t)b * p.Hkv * D;
+    const T* vn = reinterpret_cast<const T*>(p.v_new) + (size_t)b * p.Hkv * D;
+    const int64_t blk = write_kv ? slot / kPageRows : 0, row = write_kv ? slot % kPageRows : 0;
+    const int nk = write_kv ? p.Hkv * HALF : 0;
+    for (int idx = threadIdx.x; idx < nk; idx += NW * 32) {
+        const int h = idx / HALF, i = idx % HALF;
+        const T* src = kn + h * D;
+        T* dst = reinterpret_cast<T*>(p.k_cache) + ((blk * p.Hkv + h) * kPageRows + row) * D;
+        double sn, cs;
+        sincos(reduce_two_pi(pos * fr.f[i]), &sn, &cs);
+        const double x0 = to_d<T>(src[i]), x1 = to_d<T>(src[i + HALF]);
+        dst[i] = from_d<T>(x0 * cs - x1 * sn);
+        dst[i + HALF] = from_d<T>(x1 * cs + x0 * sn);
+    }
+    if (write_kv) {
+        for (int idx = threadIdx.x; idx < p.Hkv * D; idx += NW * 32) {
+            const int h = idx / D, i = idx % D;
+            reinterpret_cast<T*>(p.v_cache)[((blk * p.Hkv + h) * kPageRows + row) * D + i] = vn[h * D + i];
+        }
+    }
+}
+
 // ---------------------------------------------------------------- producer
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool FUSED>
 __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
                              const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
                              uint64_t* empty, uint32_t* masks, volatile int* s_abort,
@@ -176,6 +305,9 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
     Item cur = decode_item(item, p, s_len, s_pre);
     int c0 = 0;
     int cur_ent = entry(cur, lane);
+    // fused step: the new token's slot, read together with the block table
+    int64_t cur_slot = FUSED ? p.slot_mapping[cur.b] : -1;
+    int* patch = reinterpret_cast<int*>(base + L::OFF_PATCH);
     bool abort = false;
 
     while (!abort) {
@@ -188,6 +320,8 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
             if (nitem < W) nxt = decode_item(nitem, p, s_len, s_pre);
         }
         const int nxt_ent = (nitem < W) ? entry(nxt, nc0 + lane) : -1;
+        const int64_t nxt_slot =
+            (FUSED && nitem != item && nitem < W) ? p.slot_mapping[nxt.b] : cur_slot;
 
         const int cend = min(cur.npages, c0 + 32);
         for (int s0 = c0; s0 < cend; s0 += NW) {
@@ -205,10 +339,33 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
             uint8_t* kdst = base + stage * L::STAGE_BYTES;
             uint8_t* vdst = kdst + NW * L::PAGE_BYTES;
             const bool first = (s0 == 0);
+            // fused step: the sequence's last page gets the new token's row;
+            // only when its slot is the one the block table gives that token
+            int patch_row = -1, patch_blk = 0;
+            if constexpr (FUSED) {
+                if (s0 + NW >= cur.npages && cur.part == cur.np - 1) {
+                    const int lastpage = cur.npages - 1;
+                    const int phys = __shfl_sync(0xffffffffu, cur_ent, lastpage - c0);
+                    const int row = (s_len[cur.b] - 1) % kPageRows;
+                    if (cur_slot >= 0) {
+                        if (phys >= 0 && cur_slot == (int64_t)phys * kPageRows + row) {
+                            patch_row = row;
+                            patch_blk = phys;
+                        } else if (lane == 0) {
+                            report_error(p.err, PKV_DEVERR_SLOT);
+                        }
+                    }
+                }
+            }
             if (lane == 0) {
                 masks[stage] = vmask;
-                const uint32_t bytes =
-                    __popc(vmask) * 2u * L::PAGE_BYTES + (first ? (uint32_t)L::Q_COPY : 0u);
+                if constexpr (FUSED) {
+                    patch[2 * stage] = patch_row;
+                    patch[2 * stage + 1] = patch_blk;
+                }
+                const uint32_t bytes = __popc(vmask) * 2u * L::PAGE_BYTES +
+                                       (first ? (uint32_t)L::Q_COPY : 0u) +
+                                       (patch_row >= 0 ? (uint32_t)L::NEWKV_BYTES : 0u);
                 mbar_arrive_expect_tx(&full[stage], bytes);
             }
             __syncwarp();
@@ -227,6 +384,14 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
                                       ((size_t)cur.b * p.Hq + (size_t)cur.h * G) * D * L::ESZ;
                 bulk_load(base + L::OFF_Q + stage * L::Q_BYTES, qsrc, L::Q_COPY, &full[stage]);
             }
+            if (FUSED && patch_row >= 0 && lane == 1) {
+                const size_t row_off = ((size_t)cur.b * p.Hkv + cur.h) * L::ROW_COPY;
+                uint8_t* nk = base + L::OFF_NEWKV + stage * L::NEWKV_BYTES;
+                bulk_load(nk, reinterpret_cast<const uint8_t*>(p.k_new) + row_off, L::ROW_COPY,
+                          &full[stage]);
+                bulk_load(nk + L::ROW_COPY, reinterpret_cast<const uint8_t*>(p.v_new) + row_off,
+                          L::ROW_COPY, &full[stage]);
+            }
             issued_parity[stage] = phase;
             issued_any |= 1u << stage;
             if (++stage == L::STAGES) {
@@ -239,6 +404,7 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
         c0 = nc0;
         cur = nxt;
         cur_ent = nxt_ent;
+        cur_slot = nxt_slot;
     }
     if (abort) {
         *s_abort = 1;
@@ -288,12 +454,45 @@ __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Ite
     }
 }
 
+// Bounded barrier of the consumer warps (every consumer thread arrives).
+__device__ __forceinline__ bool consumer_sync(const DecodeParams& p, uint64_t* bar,
+                                              uint32_t& phase, volatile int* s_abort) {
+    mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, phase);
+    phase ^= 1;
+    if (!ok) {
+        *s_abort = 1;
+        report_error(p.err, PKV_DEVERR_TIMEOUT);
+    }
+    return ok;
+}
+
+// Fused step, page that holds the sequence's newest token: patch it in.
+template <typename T, int D, int G, bool FUSED>
+__device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Item& it, int j,
+                                                int stage, uint8_t* base, const double* tab) {
+    if constexpr (FUSED) {
+        using L = Layout<T, D, G>;
+        const int* pt = reinterpret_cast<const int*>(base + L::OFF_PATCH) + 2 * stage;
+        if (pt[0] >= 0 && j == it.npages - 1) {
+            const int row = pt[0];
+            const size_t grow = (((size_t)pt[1] * p.Hkv + it.h) * kPageRows + row) * D;
+            uint8_t* kpage = base + stage * L::STAGE_BYTES + (threadIdx.x >> 5) * L::PAGE_BYTES;
+            patch_new_row<T, D>(kpage, kpage + NW * L::PAGE_BYTES,
+                                base + L::OFF_NEWKV + stage * L::NEWKV_BYTES, row, tab,
+                                reinterpret_cast<T*>(p.k_cache) + grow,
+                                reinterpret_cast<T*>(p.v_cache) + grow);
+        }
+    }
+}
+
 // ------------------------------------------------- tensor-core consumer (bf16)
 
-template <int D, int G>
-__device__ void run_consumer_mma(const DecodeParams& p, uint8_t* base, uint64_t* full,
-                                 uint64_t* empty, uint64_t* merge_bar, const uint32_t* masks,
-                                 volatile int* s_abort, const int* s_len, const int* s_pre, int W) {
+template <int D, int G, bool FUSED>
+__device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
+                                 uint64_t* full, uint64_t* empty, uint64_t* merge_bar,
+                                 const uint32_t* masks, volatile int* s_abort, const int* s_len,
+                                 const int* s_pre, int W) {
     using L = Layout<bf16, D, G>;
     constexpr int KS = D / 16;  // k-steps of the score MMA
     constexpr int NT = D / 8;   // n-tiles of the output MMA
@@ -311,9 +510,22 @@ __device__ void run_consumer_mma(const DecodeParams& p, uint8_t* base, uint64_t*
     uint32_t phase = 0, mphase = 0;
     int mbuf = 0;
     float* merge = reinterpret_cast<float*>(base + L::OFF_MERGE);
+    // fused step: this warp's rope table and the sequence it was built for
+    double* tab = reinterpret_cast<double*>(base + L::OFF_ROPE) + warp * D;
+    int tab_b = -1;
+    int64_t pos_next = (FUSED && blockIdx.x < W) ? p.positions[decode_item(blockIdx.x, p, s_len, s_pre).b] : 0;
 
     for (int item = blockIdx.x; item < W; item += gridDim.x) {
         const Item it = decode_item(item, p, s_len, s_pre);
+        if constexpr (FUSED) {
+            const int64_t pos = pos_next;
+            const int nitem = item + gridDim.x;
+            if (nitem < W) pos_next = p.positions[decode_item(nitem, p, s_len, s_pre).b];
+            if (it.b != tab_b) {
+                warp_rope_table<D>((double)pos, fr, tab);
+                tab_b = it.b;
+            }
+        }
         float o[NT][4];
 #pragma unroll
         for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -326,18 +538,35 @@ __device__ void run_consumer_mma(const DecodeParams& p, uint8_t* base, uint64_t*
             ok = mbar_wait(&full[stage], phase) && !*s_abort;
             if (!ok) break;
             if (s == 0) {
-                // A fragments of Q: rows = query heads (see qrow_*), cols = dims.
+                // A fragments of Q: rows = query heads (see head_a/head_b), cols = dims.
                 const uint8_t* qs = base + L::OFF_Q + stage * L::Q_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < KS; ++kk) {
                     const int col = kk * 16 + 2 * cq;
                     uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-                    if (head_a >= 0) {
+                    if (FUSED) {
+                        // the staged q is the raw (unrotated) input: rotate the
+                        // lane's own elements on the way into the fragment
+                        auto pair = [&](int head, int c) -> uint32_t {
+                            const bf16* row = reinterpret_cast<const bf16*>(qs + head * D * 2);
+                            return (uint32_t)double_to_bf16_bits(rotated_elem<bf16, D>(row, c, tab)) |
+                                   ((uint32_t)double_to_bf16_bits(
+                                        rotated_elem<bf16, D>(row, c + 1, tab)) << 16);
+                        };
+                        if (head_a >= 0) {
+                            a0 = pair(head_a, col);
+                            a2 = pair(head_a, col + 8);
+                        }
+                        if (head_b >= 0) {
+                            a1 = pair(head_b, col);
+                            a3 = pair(head_b, col + 8);
+                        }
+                    } else if (head_a >= 0) {
                         const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_a * D * 2);
                         a0 = qr[col / 2];
                         a2 = qr[(col + 8) / 2];
                     }
-                    if (head_b >= 0) {
+                    if (!FUSED && head_b >= 0) {
                         const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_b * D * 2);
                         a1 = qr[col / 2];
                         a3 = qr[(col + 8) / 2];
@@ -351,6 +580,7 @@ __device__ void run_consumer_mma(const DecodeParams& p, uint8_t* base, uint64_t*
             const int j = s * NW + warp;
             if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
                 const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
+                item_patch_page<bf16, D, G, FUSED>(p, it, j, stage, base, tab);
                 const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
                 const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
                 const int mi = lane >> 3, ri = lane & 7;
@@ -487,11 +717,11 @@ __device__ void run_consumer_mma(const DecodeParams& p, uint8_t* base, uint64_t*
 
 // ------------------------------------------------------- CUDA-core consumer
 
-template <typename T, int D, int G>
-__device__ void run_consumer_simt(const DecodeParams& p, uint8_t* base, uint64_t* full,
-                                  uint64_t* empty, uint64_t* merge_bar, const uint32_t* masks,
-                                  volatile int* s_abort, const int* s_len, const int* s_pre,
-                                  int W) {
+template <typename T, int D, int G, bool FUSED>
+__device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
+                                  uint64_t* full, uint64_t* empty, uint64_t* merge_bar,
+                                  const uint32_t* masks, volatile int* s_abort, const int* s_len,
+                                  const int* s_pre, int W) {
     using L = Layout<T, D, G>;
     constexpr bool IS_BF16 = std::is_same<T, bf16>::value;
     constexpr int EPL = 16 / (int)sizeof(T);  // elements per lane (one 16-byte chunk)
@@ -521,8 +751,22 @@ __device__ void run_consumer_simt(const DecodeParams& p, uint8_t* base, uint64_t
         }
     };
 
+    // fused step: this warp's rope table and the sequence it was built for
+    double* tab = reinterpret_cast<double*>(base + L::OFF_ROPE) + warp * D;
+    int tab_b = -1;
+    int64_t pos_next = (FUSED && blockIdx.x < W) ? p.positions[decode_item(blockIdx.x, p, s_len, s_pre).b] : 0;
+
     for (int item = blockIdx.x; item < W; item += gridDim.x) {
         const Item it = decode_item(item, p, s_len, s_pre);
+        if constexpr (FUSED) {
+            const int64_t pos = pos_next;
+            const int nitem = item + gridDim.x;
+            if (nitem < W) pos_next = p.positions[decode_item(nitem, p, s_len, s_pre).b];
+            if (it.b != tab_b) {
+                warp_rope_table<D>((double)pos, fr, tab);
+                tab_b = it.b;
+            }
+        }
         float qf[G][EPL], o[G][EPL], m[G], l[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -537,13 +781,26 @@ __device__ void run_consumer_simt(const DecodeParams& p, uint8_t* base, uint64_t
             ok = mbar_wait(&full[stage], phase) && !*s_abort;
             if (!ok) break;
             if (s == 0) {
-                const uint32_t qs = smem_addr(base + L::OFF_Q + stage * L::Q_BYTES);
+                if constexpr (FUSED) {
+                    // raw q staged: rotate the lane's slice (rounded to T as an
+                    // appended q would be)
+                    const T* qrow0 = reinterpret_cast<const T*>(base + L::OFF_Q + stage * L::Q_BYTES);
 #pragma unroll
-                for (int g = 0; g < G; ++g) load16(qs + g * D * (int)sizeof(T) + c * 16, qf[g]);
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e)
+                            qf[g][e] = (float)to_d<T>(from_d<T>(
+                                rotated_elem<T, D>(qrow0 + g * D, c * EPL + e, tab)));
+                } else {
+                    const uint32_t qs = smem_addr(base + L::OFF_Q + stage * L::Q_BYTES);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) load16(qs + g * D * (int)sizeof(T) + c * 16, qf[g]);
+                }
             }
             const int j = s * NW + warp;
             if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
                 const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
+                item_patch_page<T, D, G, FUSED>(p, it, j, stage, base, tab);
                 const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
                 const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
 #pragma unroll 2
@@ -640,11 +897,12 @@ __device__ void run_consumer_simt(const DecodeParams& p, uint8_t* base, uint64_t
 
 // ------------------------------------------------------------------ kernel
 
-template <typename T, int D, int G, bool MMA>
+template <typename T, int D, int G, bool MMA, bool FUSED>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
     paged_decode_kernel(const __grid_constant__ DecodeParams p,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ RopeFreq fr) {
     using L = Layout<T, D, G>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -677,6 +935,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     // Everything below reads inputs a previous kernel may have written.
     grid_dependency_wait();
     grid_launch_dependents();
+
+    // Warm L2 with the block-table entries of this CTA's first item, guessed
+    // as if every sequence had NP partitions (exact for uniform batches; a
+    // wrong guess only costs a prefetch), while the lengths are scanned.
+    if (warp == NW && lane < 2) {
+        const int j = blockIdx.x / p.Hkv;
+        const int bs = j / p.NP, ps = j - (j / p.NP) * p.NP;
+        const int jb = ps * (p.P / kPageRows) + lane * 31;
+        if (bs < p.B && jb < p.MB)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.block_tables + (size_t)bs * p.MB + jb));
+    }
 
     // Partition counts per sequence and their exclusive prefix (block scan).
     const int B = p.B;
@@ -715,20 +984,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     const int W = s_pre[B] * p.Hkv;
 
     if (warp == NW) {
-        run_producer<T, D, G>(p, &tm_k, &tm_v, base, full, empty, masks, s_abort, s_len, s_pre, W);
+        run_producer<T, D, G, FUSED>(p, &tm_k, &tm_v, base, full, empty, masks, s_abort, s_len,
+                                     s_pre, W);
         return;
     }
-    // zero the output of empty contexts (spread over the CTAs)
+    // zero the output of empty contexts (spread over the CTAs); in the fused
+    // step their new token is still appended
     for (int b = blockIdx.x; b < B; b += gridDim.x) {
         if (s_len[b] != 0) continue;
         for (int idx = tid; idx < p.Hq * D; idx += NW * 32)
             store_out(p.out, (size_t)b * p.Hq * D + idx, 0.f, p.out_bf16);
+        if constexpr (FUSED) append_only<T, D>(p, fr, b);
     }
     if constexpr (MMA) {
-        run_consumer_mma<D, G>(p, base, full, empty, merge_bar, masks, s_abort, s_len, s_pre, W);
+        run_consumer_mma<D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks, s_abort, s_len,
+                                      s_pre, W);
     } else {
-        run_consumer_simt<T, D, G>(p, base, full, empty, merge_bar, masks, s_abort, s_len, s_pre,
-                                   W);
+        run_consumer_simt<T, D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks, s_abort,
+                                          s_len, s_pre, W);
     }
 }
 
@@ -857,11 +1130,11 @@ cudaError_t prepare_kernel(K kern, size_t smem, int* ctas_per_sm) {
     return cudaSuccess;
 }
 
-template <typename T, int D, int G, bool MMA>
+template <typename T, int D, int G, bool MMA, bool FUSED>
 cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
                                 const CUtensorMap& tmv) {
     using L = Layout<T, D, G>;
-    auto kern = paged_decode_kernel<T, D, G, MMA>;
+    auto kern = paged_decode_kernel<T, D, G, MMA, FUSED>;
     const size_t smem = L::smem_bytes((int)a.B);
     int occ = 0;
     cudaError_t e = prepare_kernel(kern, smem, &occ);
@@ -884,6 +1157,14 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     p.num_blocks = (int)a.num_blocks;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out_bf16 = a.out_dtype == PKV_DTYPE_BF16;
+    p.k_new = a.k_new;
+    p.v_new = a.v_new;
+    p.positions = a.positions;
+    p.slot_mapping = a.slot_mapping;
+    p.k_cache = const_cast<void*>(a.k_cache);
+    p.v_cache = const_cast<void*>(a.v_cache);
+    RopeFreq fr;
+    for (int i = 0; i < 64; ++i) fr.f[i] = (FUSED && i < D / 2) ? std::pow(a.theta, -(2.0 * i) / D) : 0.0;
 
     const int64_t upper = a.B * a.Hkv * (int64_t)a.max_partitions;
     const int64_t resident = (int64_t)device_sm_count() * occ;
@@ -899,7 +1180,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv);
+    e = cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv, fr);
     if (e != cudaSuccess || a.max_partitions <= 1) return e;
 
     CombineParams cp;
@@ -921,15 +1202,29 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     return cudaLaunchKernelEx(&cc, ckern, cp);
 }
 
-template <typename T, int D, bool MMA>
+template <typename T, int D, bool MMA, bool FUSED>
 cudaError_t dispatch_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v) {
     switch (a.Hq / a.Hkv) {
-        case 1: return launch_decode_typed<T, D, 1, MMA>(a, k, v);
-        case 2: return launch_decode_typed<T, D, 2, MMA>(a, k, v);
-        case 4: return launch_decode_typed<T, D, 4, MMA>(a, k, v);
-        case 8: return launch_decode_typed<T, D, 8, MMA>(a, k, v);
+        case 1: return launch_decode_typed<T, D, 1, MMA, FUSED>(a, k, v);
+        case 2: return launch_decode_typed<T, D, 2, MMA, FUSED>(a, k, v);
+        case 4: return launch_decode_typed<T, D, 4, MMA, FUSED>(a, k, v);
+        case 8: return launch_decode_typed<T, D, 8, MMA, FUSED>(a, k, v);
     }
     return cudaErrorInvalidValue;
+}
+
+template <bool FUSED>
+cudaError_t dispatch_all(const DecodeArgs& a, const CUtensorMap& tmk, const CUtensorMap& tmv) {
+    if (a.kv_dtype == PKV_DTYPE_F32) {
+        return a.D == 64 ? dispatch_g<float, 64, false, FUSED>(a, tmk, tmv)
+                         : dispatch_g<float, 128, false, FUSED>(a, tmk, tmv);
+    }
+    if (a.force_simt) {
+        return a.D == 64 ? dispatch_g<bf16, 64, false, FUSED>(a, tmk, tmv)
+                         : dispatch_g<bf16, 128, false, FUSED>(a, tmk, tmv);
+    }
+    return a.D == 64 ? dispatch_g<bf16, 64, true, FUSED>(a, tmk, tmv)
+                     : dispatch_g<bf16, 128, true, FUSED>(a, tmk, tmv);
 }
 
 }  // namespace
@@ -943,16 +1238,7 @@ cudaError_t launch_paged_decode(const DecodeArgs& a) {
     if (e != cudaSuccess) return e;
     e = encode_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D, a.kv_dtype);
     if (e != cudaSuccess) return e;
-    if (a.kv_dtype == PKV_DTYPE_F32) {
-        return a.D == 64 ? dispatch_g<float, 64, false>(a, tmk, tmv)
-                         : dispatch_g<float, 128, false>(a, tmk, tmv);
-    }
-    if (a.force_simt) {
-        return a.D == 64 ? dispatch_g<bf16, 64, false>(a, tmk, tmv)
-                         : dispatch_g<bf16, 128, false>(a, tmk, tmv);
-    }
-    return a.D == 64 ? dispatch_g<bf16, 64, true>(a, tmk, tmv)
-                     : dispatch_g<bf16, 128, true>(a, tmk, tmv);
+    return a.fused ? dispatch_all<true>(a, tmk, tmv) : dispatch_all<false>(a, tmk, tmv);
 }
 
 int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_t num_seqs) {

@@ -272,15 +272,27 @@ size_t pkv_decode_workspace_size(int64_t num_seqs, int64_t num_q_heads, int64_t 
     return w.bytes;
 }
 
-pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
-                                      const int32_t* block_tables, const int32_t* context_lens,
-                                      void* out, void* workspace, size_t workspace_bytes,
-                                      int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
-                                      int64_t head_dim, int64_t num_blocks, int64_t block_size,
-                                      int64_t max_blocks_per_seq, int32_t kv_dtype,
-                                      int32_t out_dtype, float scale, int32_t partition_tokens,
-                                      uint32_t flags, int32_t* device_error, void* stream) {
-    set_last_error("");
+}  // extern "C"
+
+namespace {
+
+struct StepExtras {
+    const void* k_new;
+    const void* v_new;
+    const int64_t* positions;
+    const int64_t* slot_mapping;
+    double theta;
+};
+
+// Shared by the decode call and the fused step: validate, plan, launch.
+pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, void* out,
+                         void* workspace, size_t workspace_bytes, int64_t num_seqs,
+                         int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                         int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq,
+                         int32_t kv_dtype, int32_t out_dtype, float scale,
+                         int32_t partition_tokens, uint32_t flags, int32_t* device_error,
+                         void* stream, const StepExtras* step) {
     if (num_seqs < 0 || max_blocks_per_seq < 0) {
         set_last_error("negative num_seqs or max_blocks_per_seq");
         return PKV_ERR_INVALID_ARG;
@@ -311,6 +323,10 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
         set_last_error("scale must be finite");
         return PKV_ERR_INVALID_ARG;
     }
+    if (step && !(step->theta > 0.0)) {
+        set_last_error("rope_theta must be > 0");
+        return PKV_ERR_INVALID_ARG;
+    }
     WorkspacePlan w;
     st = plan_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                         kv_dtype, partition_tokens, &w);
@@ -320,14 +336,20 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
         set_last_error("null tensor pointer");
         return PKV_ERR_INVALID_ARG;
     }
+    if (step && (!step->k_new || !step->v_new || !step->positions || !step->slot_mapping)) {
+        set_last_error("null tensor pointer");
+        return PKV_ERR_INVALID_ARG;
+    }
     if (max_blocks_per_seq == 0) {
         set_last_error("max_blocks_per_seq must be > 0 when num_seqs > 0");
         return PKV_ERR_INVALID_ARG;
     }
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         !aligned4(block_tables) || !aligned4(context_lens) ||
-        (device_error && !aligned4(device_error))) {
-        set_last_error("misaligned tensor pointer (16 bytes for q/caches/out)");
+        (device_error && !aligned4(device_error)) ||
+        (step && (!aligned16(step->k_new) || !aligned16(step->v_new) ||
+                  !aligned8(step->positions) || !aligned8(step->slot_mapping)))) {
+        set_last_error("misaligned tensor pointer (16 bytes for q/k/v/caches/out)");
         return PKV_ERR_INVALID_ARG;
     }
     if (workspace_bytes < w.bytes || (w.bytes > 0 && (!workspace || !aligned16(workspace)))) {
@@ -335,7 +357,7 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
                        workspace_bytes, w.bytes);
         return PKV_ERR_WORKSPACE;
     }
-    DecodeArgs a;
+    DecodeArgs a = {};
     a.q = q;
     a.k_cache = k_cache;
     a.v_cache = v_cache;
@@ -358,7 +380,52 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     a.force_simt = (flags & PKV_DECODE_FORCE_SIMT) != 0;
     a.device_error = device_error;
     a.stream = static_cast<cudaStream_t>(stream);
-    return cuda_status(launch_paged_decode(a), "paged_attention_decode launch");
+    a.fused = step != nullptr;
+    if (step) {
+        a.k_new = step->k_new;
+        a.v_new = step->v_new;
+        a.positions = step->positions;
+        a.slot_mapping = step->slot_mapping;
+        a.theta = step->theta;
+    }
+    return cuda_status(launch_paged_decode(a), step ? "decode_step launch"
+                                                    : "paged_attention_decode launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* context_lens,
+                                      void* out, void* workspace, size_t workspace_bytes,
+                                      int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                                      int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                                      int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                      int32_t out_dtype, float scale, int32_t partition_tokens,
+                                      uint32_t flags, int32_t* device_error, void* stream) {
+    set_last_error("");
+    return decode_common(q, k_cache, v_cache, block_tables, context_lens, out, workspace,
+                         workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                         num_blocks, block_size, max_blocks_per_seq, kv_dtype, out_dtype, scale,
+                         partition_tokens, flags, device_error, stream, nullptr);
+}
+
+pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new, const int64_t* positions,
+                           const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, void* out,
+                           void* workspace, size_t workspace_bytes, int64_t num_seqs,
+                           int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                           int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq,
+                           int32_t kv_dtype, int32_t out_dtype, double rope_theta, float scale,
+                           int32_t partition_tokens, uint32_t flags, int32_t* device_error,
+                           void* stream) {
+    set_last_error("");
+    const StepExtras step = {k_new, v_new, positions, slot_mapping, rope_theta};
+    return decode_common(q, k_cache, v_cache, block_tables, context_lens, out, workspace,
+                         workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                         num_blocks, block_size, max_blocks_per_seq, kv_dtype, out_dtype, scale,
+                         partition_tokens, flags, device_error, stream, &step);
 }
 
 const char* pkv_status_string(int32_t status) {

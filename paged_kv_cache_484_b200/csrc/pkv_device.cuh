@@ -161,4 +161,21 @@ __device__ __forceinline__ uint16_t double_to_bf16_bits(double x) {
     return r;
 }
 
+// RoPE angle reduction: x - k*2pi with k = rint(x / 2pi), by Cody and
+// Waite's method with 2pi split into three doubles (2pi = C1 + C2 + C3 to
+// ~160 bits; constants computed here from a high-precision 2pi) and one fused
+// multiply-add per part.  For the angles RoPE produces (|x| < 2^31) the result
+// lies in [-pi, pi] with an absolute error near 2^-51, so the sine and cosine
+// that follow stay on their short-argument path.
+__device__ __forceinline__ double reduce_two_pi(double x) {
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    constexpr double kC1 = 6.283185307179586;          // 0x1.921fb54442d18p+2
+    constexpr double kC2 = 2.4492935982947064e-16;     // 0x1.1a62633145c07p-52
+    constexpr double kC3 = -5.989539619436679e-33;     // -0x1.f1976b7ed8fbcp-108
+    const double k = rint(x * kInvTwoPi);
+    double r = fma(-k, kC1, x);
+    r = fma(-k, kC2, r);
+    return fma(-k, kC3, r);
+}
+
 }  // namespace pkv

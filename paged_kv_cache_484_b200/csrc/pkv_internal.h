@@ -50,6 +50,13 @@ struct DecodeArgs {
     bool force_simt;
     int32_t* device_error;
     cudaStream_t stream;
+    // fused step (append inside the decode kernel); q is rotated in place
+    bool fused;
+    const void* k_new;
+    const void* v_new;
+    const int64_t* positions;
+    const int64_t* slot_mapping;
+    double theta;
 };
 cudaError_t launch_paged_decode(const DecodeArgs& a);
 

@@ -45,11 +45,18 @@ class SubProblem:
 
 
 def gpu_step(w: Workload, out_dtype=torch.float32, partition_tokens=0, force_simt=False,
-             device_error=None):
-    """kv_append then paged_attention_decode on the workload (in place)."""
+             device_error=None, fused=False):
+    """One decode step on the workload (in place): kv_append then
+    paged_attention_decode, or the single-launch decode_step when ``fused``."""
+    out = torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=w.q.device)
+    if fused:
+        pkv.decode_step(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
+                        w.block_tables, w.decode_lens, w.rope_theta, w.scale, out,
+                        partition_tokens=partition_tokens, force_simt=force_simt,
+                        device_error=device_error)
+        return out
     pkv.kv_append(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
                   w.rope_theta, device_error=device_error)
-    out = torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=w.q.device)
     pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens, w.scale,
                                out, partition_tokens=partition_tokens, force_simt=force_simt,
                                device_error=device_error)

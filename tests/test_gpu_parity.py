@@ -20,8 +20,10 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _placement_and_append(w, before_k, before_v, sub, q_gpu, q_or, kc_or, vc_or):
-    """Exactly the slot rows changed; v bit copy; k and q within one bf16 ulp."""
+def _placement_and_append(w, before_k, before_v, sub, q_gpu, q_or, kc_or, vc_or, q_in=None):
+    """Exactly the slot rows changed; v bit copy; k within one bf16 ulp; q
+    rotated in place within one bf16 ulp (two calls) or untouched (one-launch
+    step, ``q_in`` given)."""
     bs = w.block_size
     itype = torch.int16 if w.dtype == torch.bfloat16 else torch.int32
     changed = (w.k_cache.view(itype) != before_k.view(itype)).any(-1) | \
@@ -45,7 +47,10 @@ def _placement_and_append(w, before_k, before_v, sub, q_gpu, q_or, kc_or, vc_or)
         ov = vc_or[so // bs, :, so % bs]
         assert torch.equal(gv.view(itype), ov.view(itype)), f"v bits, seq {b}"
         check_within_one_bf16_ulp(gk, ok_, f"appended k, seq {b}")
-        check_within_one_bf16_ulp(q_gpu[b].cpu(), q_or[i], f"rotated q, seq {b}")
+        if q_in is None:
+            check_within_one_bf16_ulp(q_gpu[b].cpu(), q_or[i], f"rotated q, seq {b}")
+    if q_in is not None:
+        assert torch.equal(q_gpu, q_in), "decode_step must leave q untouched"
 
 
 def _seq_sample(cfg, w):
@@ -60,10 +65,12 @@ def _seq_sample(cfg, w):
     return sorted(pick)
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "one_launch"])
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
-def test_named_workload_step(cfg):
+def test_named_workload_step(cfg, fused):
     """One full step (append + decode) of each named workload, at full size,
-    in the launch configuration the benchmark times."""
+    in the launch configuration the benchmark times: as the two calls, and as
+    the single-launch decode_step."""
     w = W.make_config(cfg, device=DEV)
     seqs = _seq_sample(cfg, w)
     sub = SubProblem(w, seqs)
@@ -73,10 +80,13 @@ def test_named_workload_step(cfg):
     before_v = w.v_cache.clone()
     q_in = w.q.clone()
 
-    out32 = gpu_step(w, out_dtype=torch.float32)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out32 = gpu_step(w, out_dtype=torch.float32, fused=fused, device_error=err)
     torch.cuda.synchronize()
+    assert int(err.item()) == 0
     q_or, kc_or, vc_or, ref = sub.oracle_step(nthreads=16, pairs=pairs)
-    _placement_and_append(w, before_k, before_v, sub, w.q, q_or, kc_or, vc_or)
+    _placement_and_append(w, before_k, before_v, sub, w.q, q_or, kc_or, vc_or,
+                          q_in=q_in if fused else None)
     del before_k, before_v
 
     sel = torch.tensor(seqs)
@@ -89,10 +99,17 @@ def test_named_workload_step(cfg):
         check_decode(g, r, w.dtype, f"cfg{cfg} f32 out (sampled)")
 
     if w.dtype == torch.bfloat16:
-        # the benchmark's output dtype: same cache state, same rotated q
+        # the benchmark's output dtype, on the same state: the two-call path
+        # decodes again with the rotated q; the one-launch step runs again (it
+        # rewrites the same new rows and leaves q as it was)
         out16 = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=DEV)
-        pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
-                                   w.scale, out16)
+        if fused:
+            pkv.decode_step(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                            w.v_cache, w.block_tables, w.decode_lens, w.rope_theta, w.scale,
+                            out16)
+        else:
+            pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
+                                       w.scale, out16)
         got16 = out16.cpu()[sel]
         if pairs is None:
             check_decode_bf16_out(got16, ref, f"cfg{cfg} bf16 out")
@@ -115,20 +132,29 @@ LENS = [1, 15, 16, 17, 63, 64, 65, 127, 129, 300, 1000, 2049]
     (torch.bfloat16, 64, 4, True), (torch.bfloat16, 128, 8, True), (torch.bfloat16, 64, 1, True),
 ])
 @pytest.mark.parametrize("P", [0, 16, 64, 512])
-def test_shapes_and_partitions(dtype, d, G, simt, P):
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "one_launch"])
+def test_shapes_and_partitions(dtype, d, G, simt, P, fused):
     Hkv = 2
     lens = [L - 1 for L in LENS]
     w = W.build_workload("shapes", lens, G * Hkv, Hkv, d, dtype, 1e4, seed=100 + d + G, device=DEV,
                          pool_factor=1.3)
-    # one empty context: its output must be zeros
-    w.decode_lens[5] = 0
+    if not fused:
+        # one empty context: its output must be zeros (the fused step's
+        # precondition excludes it; tested separately)
+        w.decode_lens[5] = 0
     sub = SubProblem(w, range(w.B))
-    out = gpu_step(w, out_dtype=torch.float32, partition_tokens=P, force_simt=simt)
+    q_in = w.q.clone()
+    out = gpu_step(w, out_dtype=torch.float32, partition_tokens=P, force_simt=simt, fused=fused)
     torch.cuda.synchronize()
-    _, _, _, ref = sub.oracle_step()
-    ref[5].zero_()
-    check_decode(out, ref, dtype, f"{dtype} d{d} G{G} simt={simt} P={P}")
-    assert torch.equal(out[5].cpu(), torch.zeros_like(out[5].cpu()))
+    q_or, kc_or, _, ref = sub.oracle_step()
+    if not fused:
+        ref[5].zero_()
+    check_decode(out, ref, dtype, f"{dtype} d{d} G{G} simt={simt} P={P} fused={fused}")
+    if not fused:
+        assert torch.equal(out[5].cpu(), torch.zeros_like(out[5].cpu()))
+        check_within_one_bf16_ulp(w.q.cpu(), q_or, "rotated q")
+    else:
+        assert torch.equal(w.q, q_in)
 
 
 def test_partition_length_does_not_change_result():
@@ -196,3 +222,41 @@ def test_empty_batch_is_a_no_op():
                   torch.empty((0,), dtype=torch.int64, device=DEV),
                   torch.empty((0,), dtype=torch.int64, device=DEV), kc, kc, 1e4)
     torch.cuda.synchronize()
+
+
+def test_fused_step_edge_cases():
+    """decode_step with a padding slot (-1), a slot that is not the last
+    token's table slot, and an empty context, against the oracle's append +
+    decode of the same intent."""
+    d, Hkv, G = 64, 2, 4
+    w = W.build_workload("edges", [40, 40, 40, 0, 33], G * Hkv, Hkv, d, torch.bfloat16, 5e5, seed=21,
+                         device=DEV, pool_factor=1.5)
+    bs = 16
+    # sequence 0: padding slot -> not appended, cached context attended as is
+    w.slot_mapping[0] = -1
+    # sequence 1: a slot that is not its last token's slot -> flagged, not appended
+    good1 = int(w.slot_mapping[1])
+    w.slot_mapping[1] = int(w.block_tables[1][0]) * bs + 3
+    # sequence 3: context length 0 -> zero output, token appended as kv_append would
+    w.decode_lens[3] = 0
+    sub = SubProblem(w, range(w.B))
+    sub.slots[0] = -1          # the oracle sees "not appended" for sequences 0 and 1 too
+    sub.slots[1] = -1
+    k_before = w.k_cache.clone()
+    q_in = w.q.clone()
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = gpu_step(w, out_dtype=torch.float32, fused=True, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pkv.DEVERR_SLOT
+    q_or, kc_or, vc_or, ref = sub.oracle_step()
+    ref[3].zero_()
+    check_decode(out, ref, torch.bfloat16, "fused edge cases")
+    assert torch.equal(w.q, q_in)
+    # sequence 1's intended slot and the bogus one were left untouched
+    for s_ in (good1, int(w.block_tables[1][0]) * bs + 3):
+        assert torch.equal(w.k_cache[s_ // bs, :, s_ % bs], k_before[s_ // bs, :, s_ % bs])
+    # sequence 3 (empty context) was appended
+    s3 = int(w.slot_mapping[3])
+    so3 = int(sub.slots[3])
+    check_within_one_bf16_ulp(w.k_cache[s3 // bs, :, s3 % bs].cpu(), kc_or[so3 // bs, :, so3 % bs],
+                              "appended k of the empty context")
