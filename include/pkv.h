@@ -226,11 +226,13 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
  * sequence's cache block, then the token attends to the whole cache).
  *
  * Token b of the append is sequence b's new token.  Every warp of the decode
- * kernel rotates the q elements it feeds to its own MMA fragments (fp64, as
- * pkv_kv_append computes them, rounded to the storage type), and the CTA that
- * holds a sequence's last cache page rotates the new k, writes k and v into
- * the slot and patches them into the staged page, so no separate append
- * launch and no extra pass over memory is needed.  q itself is only read:
+ * kernel rotates the q elements it feeds to its own MMA fragments, and the
+ * CTA that holds a sequence's last cache page rotates the new k, writes k and
+ * v into the slot and patches them into the staged page, so no separate
+ * append launch and no extra pass over memory is needed.  Here the angle is
+ * reduced mod 2pi in fp64 but its sine, cosine and the rotation are fp32,
+ * rounded once to the storage type: within one storage ulp of the fp64 result
+ * pkv_kv_append produces (bit-equal in the vast majority of elements).  q itself is only read:
  * unlike pkv_kv_append, the step does not store the rotated q (it is used
  * inside the kernel only), so q can be shared by all partitions at once.
  *

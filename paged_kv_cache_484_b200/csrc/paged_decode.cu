@@ -81,9 +81,11 @@ struct Layout {
     // byte offsets from the 1024-aligned base
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
     static constexpr int OFF_NEWKV = OFF_Q + STAGES * Q_BYTES;
-    // fused step: one cos[D/2], sin[D/2] fp64 table per consumer warp
+    // fused step: per stage, cos[D/2], sin[D/2] (fp32) of the item's position,
+    // written by the producer with the item's first stage
+    static constexpr int ROPE_BYTES = D * 4;
     static constexpr int OFF_ROPE = OFF_NEWKV + STAGES * NEWKV_BYTES;
-    static constexpr int OFF_MERGE = OFF_ROPE + NW * D * 8;
+    static constexpr int OFF_MERGE = OFF_ROPE + STAGES * ROPE_BYTES;
     static constexpr int OFF_BAR = OFF_MERGE + 2 * MERGE_FLOATS * 4;
     static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
     static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
@@ -186,29 +188,36 @@ __device__ __forceinline__ bf16 from_d<bf16>(double x) {
     return *reinterpret_cast<const bf16*>(&b);
 }
 
-// Fused step: one warp's cos/sin table of a position, tab[i] = cos(pos f_i),
-// tab[D/2 + i] = sin(pos f_i) for i < D/2 (fp64, angle reduced first).
+// Fused step: a warp writes the cos/sin table of a position, tab[i] =
+// cos(pos f_i), tab[D/2 + i] = sin(pos f_i), i < D/2: angle in fp64, reduced
+// mod 2pi in fp64, then sine and cosine in fp32 of the reduced angle.
 template <int D>
-__device__ __forceinline__ void warp_rope_table(double pos, const RopeFreq& fr, double* tab) {
+__device__ __forceinline__ void warp_rope_table(double pos, const RopeFreq& fr, float* tab) {
     for (int i = threadIdx.x & 31; i < D / 2; i += 32) {
-        double sn, cs;
-        sincos(reduce_two_pi(pos * fr.f[i]), &sn, &cs);
+        float sn, cs;
+        sincosf((float)reduce_two_pi(pos * fr.f[i]), &sn, &cs);
         tab[i] = cs;
         tab[D / 2 + i] = sn;
     }
-    __syncwarp();
 }
 
-// Element `col` of the rotated row (row in storage type T): the pair partner is
-// col +- D/2; fp64 rotation, as kv_append computes it.
+// Element `col` of the rotated row (row in storage type T); the pair partner
+// is col +- D/2.  fp32 arithmetic (the result is rounded to T by the caller).
 template <typename T, int D>
-__device__ __forceinline__ double rotated_elem(const T* row, int col, const double* tab) {
+__device__ __forceinline__ float rotated_elem(const T* row, int col, const float* tab) {
     constexpr int HALF = D / 2;
     const int i = col < HALF ? col : col - HALF;
-    const double x = to_d<T>(row[col]);
-    const double y = to_d<T>(row[col < HALF ? col + HALF : col - HALF]);
-    return col < HALF ? x * tab[i] - y * tab[HALF + i] : x * tab[i] + y * tab[HALF + i];
+    const float x = (float)to_d<T>(row[col]);
+    const float y = (float)to_d<T>(row[col < HALF ? col + HALF : col - HALF]);
+    return col < HALF ? fmaf(x, tab[i], -y * tab[HALF + i]) : fmaf(x, tab[i], y * tab[HALF + i]);
 }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
 
 // One warp writes the new token's rotated k row and raw v row into row r of
 // the staged K and V pages (overwriting what the TMA brought) and into the
@@ -216,18 +225,15 @@ __device__ __forceinline__ double rotated_elem(const T* row, int col, const doub
 // any later TMA write into the same stage.
 template <typename T, int D>
 __device__ void patch_new_row(uint8_t* kpage, uint8_t* vpage, const uint8_t* newkv, int r,
-                              const double* tab, T* kglob, T* vglob) {
-    const double* rc = tab;
-    const double* rs = tab + D / 2;
+                              const float* tab, T* kglob, T* vglob) {
     constexpr int HALF = D / 2, E = 16 / (int)sizeof(T), CH = D * (int)sizeof(T) / 16;
     const int lane = threadIdx.x & 31;
     const T* kn = reinterpret_cast<const T*>(newkv);
     const uint8_t* vn = newkv + D * sizeof(T);
     for (int i = lane; i < HALF; i += 32) {
-        const double x0 = to_d<T>(kn[i]), x1 = to_d<T>(kn[i + HALF]);
-        const T y0 = from_d<T>(x0 * rc[i] - x1 * rs[i]);
-        const T y1 = from_d<T>(x1 * rc[i] + x0 * rs[i]);
         const int i1 = i + HALF;
+        const T y0 = from_f<T>(rotated_elem<T, D>(kn, i, tab));
+        const T y1 = from_f<T>(rotated_elem<T, D>(kn, i1, tab));
         *reinterpret_cast<T*>(kpage + chunk_offset<T, D>(r, i / E) + (i % E) * sizeof(T)) = y0;
         *reinterpret_cast<T*>(kpage + chunk_offset<T, D>(r, i1 / E) + (i1 % E) * sizeof(T)) = y1;
         kglob[i] = y0;
@@ -278,7 +284,7 @@ __device__ void append_only(const DecodeParams& p, const RopeFreq& fr, int b) {
 // ---------------------------------------------------------------- producer
 
 template <typename T, int D, int G, bool FUSED>
-__device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
+__device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CUtensorMap* tmk,
                              const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
                              uint64_t* empty, uint32_t* masks, volatile int* s_abort,
                              const int* s_len, const int* s_pre, int W) {
@@ -305,8 +311,10 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
     Item cur = decode_item(item, p, s_len, s_pre);
     int c0 = 0;
     int cur_ent = entry(cur, lane);
-    // fused step: the new token's slot, read together with the block table
+    // fused step: the new token's slot and position, read together with the
+    // block table
     int64_t cur_slot = FUSED ? p.slot_mapping[cur.b] : -1;
+    int64_t cur_pos = FUSED ? p.positions[cur.b] : 0;
     int* patch = reinterpret_cast<int*>(base + L::OFF_PATCH);
     bool abort = false;
 
@@ -320,8 +328,9 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
             if (nitem < W) nxt = decode_item(nitem, p, s_len, s_pre);
         }
         const int nxt_ent = (nitem < W) ? entry(nxt, nc0 + lane) : -1;
-        const int64_t nxt_slot =
-            (FUSED && nitem != item && nitem < W) ? p.slot_mapping[nxt.b] : cur_slot;
+        const bool new_item = FUSED && nitem != item && nitem < W;
+        const int64_t nxt_slot = new_item ? p.slot_mapping[nxt.b] : cur_slot;
+        const int64_t nxt_pos = new_item ? p.positions[nxt.b] : cur_pos;
 
         const int cend = min(cur.npages, c0 + 32);
         for (int s0 = c0; s0 < cend; s0 += NW) {
@@ -355,6 +364,16 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
                             report_error(p.err, PKV_DEVERR_SLOT);
                         }
                     }
+                }
+            }
+            if constexpr (FUSED) {
+                // the rope table rides with the item's first stage and with
+                // the stage that carries the new token
+                if (first || patch_row >= 0) {
+                    warp_rope_table<D>((double)cur_pos, fr,
+                                       reinterpret_cast<float*>(base + L::OFF_ROPE +
+                                                                stage * L::ROPE_BYTES));
+                    __syncwarp();
                 }
             }
             if (lane == 0) {
@@ -405,6 +424,7 @@ __device__ void run_producer(const DecodeParams& p, const CUtensorMap* tmk,
         cur = nxt;
         cur_ent = nxt_ent;
         cur_slot = nxt_slot;
+        cur_pos = nxt_pos;
     }
     if (abort) {
         *s_abort = 1;
@@ -470,9 +490,10 @@ __device__ __forceinline__ bool consumer_sync(const DecodeParams& p, uint64_t* b
 // Fused step, page that holds the sequence's newest token: patch it in.
 template <typename T, int D, int G, bool FUSED>
 __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Item& it, int j,
-                                                int stage, uint8_t* base, const double* tab) {
+                                                int stage, uint8_t* base) {
     if constexpr (FUSED) {
         using L = Layout<T, D, G>;
+        const float* tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
         const int* pt = reinterpret_cast<const int*>(base + L::OFF_PATCH) + 2 * stage;
         if (pt[0] >= 0 && j == it.npages - 1) {
             const int row = pt[0];
@@ -510,22 +531,11 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
     uint32_t phase = 0, mphase = 0;
     int mbuf = 0;
     float* merge = reinterpret_cast<float*>(base + L::OFF_MERGE);
-    // fused step: this warp's rope table and the sequence it was built for
-    double* tab = reinterpret_cast<double*>(base + L::OFF_ROPE) + warp * D;
-    int tab_b = -1;
-    int64_t pos_next = (FUSED && blockIdx.x < W) ? p.positions[decode_item(blockIdx.x, p, s_len, s_pre).b] : 0;
+    // fused step: the item's rope table, staged by the producer with its first stage
+    const float* tab = nullptr;
 
     for (int item = blockIdx.x; item < W; item += gridDim.x) {
         const Item it = decode_item(item, p, s_len, s_pre);
-        if constexpr (FUSED) {
-            const int64_t pos = pos_next;
-            const int nitem = item + gridDim.x;
-            if (nitem < W) pos_next = p.positions[decode_item(nitem, p, s_len, s_pre).b];
-            if (it.b != tab_b) {
-                warp_rope_table<D>((double)pos, fr, tab);
-                tab_b = it.b;
-            }
-        }
         float o[NT][4];
 #pragma unroll
         for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -538,6 +548,7 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
             ok = mbar_wait(&full[stage], phase) && !*s_abort;
             if (!ok) break;
             if (s == 0) {
+                tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
                 // A fragments of Q: rows = query heads (see head_a/head_b), cols = dims.
                 const uint8_t* qs = base + L::OFF_Q + stage * L::Q_BYTES;
 #pragma unroll
@@ -549,9 +560,8 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
                         // lane's own elements on the way into the fragment
                         auto pair = [&](int head, int c) -> uint32_t {
                             const bf16* row = reinterpret_cast<const bf16*>(qs + head * D * 2);
-                            return (uint32_t)double_to_bf16_bits(rotated_elem<bf16, D>(row, c, tab)) |
-                                   ((uint32_t)double_to_bf16_bits(
-                                        rotated_elem<bf16, D>(row, c + 1, tab)) << 16);
+                            return pack_bf16(rotated_elem<bf16, D>(row, c, tab),
+                                             rotated_elem<bf16, D>(row, c + 1, tab));
                         };
                         if (head_a >= 0) {
                             a0 = pair(head_a, col);
@@ -580,7 +590,7 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
             const int j = s * NW + warp;
             if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
                 const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
-                item_patch_page<bf16, D, G, FUSED>(p, it, j, stage, base, tab);
+                item_patch_page<bf16, D, G, FUSED>(p, it, j, stage, base);
                 const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
                 const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
                 const int mi = lane >> 3, ri = lane & 7;
@@ -751,22 +761,11 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
         }
     };
 
-    // fused step: this warp's rope table and the sequence it was built for
-    double* tab = reinterpret_cast<double*>(base + L::OFF_ROPE) + warp * D;
-    int tab_b = -1;
-    int64_t pos_next = (FUSED && blockIdx.x < W) ? p.positions[decode_item(blockIdx.x, p, s_len, s_pre).b] : 0;
+    // fused step: the item's rope table, staged by the producer with its first stage
+    const float* tab = nullptr;
 
     for (int item = blockIdx.x; item < W; item += gridDim.x) {
         const Item it = decode_item(item, p, s_len, s_pre);
-        if constexpr (FUSED) {
-            const int64_t pos = pos_next;
-            const int nitem = item + gridDim.x;
-            if (nitem < W) pos_next = p.positions[decode_item(nitem, p, s_len, s_pre).b];
-            if (it.b != tab_b) {
-                warp_rope_table<D>((double)pos, fr, tab);
-                tab_b = it.b;
-            }
-        }
         float qf[G][EPL], o[G][EPL], m[G], l[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -781,6 +780,7 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
             ok = mbar_wait(&full[stage], phase) && !*s_abort;
             if (!ok) break;
             if (s == 0) {
+                tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
                 if constexpr (FUSED) {
                     // raw q staged: rotate the lane's slice (rounded to T as an
                     // appended q would be)
@@ -789,7 +789,7 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
                     for (int g = 0; g < G; ++g)
 #pragma unroll
                         for (int e = 0; e < EPL; ++e)
-                            qf[g][e] = (float)to_d<T>(from_d<T>(
+                            qf[g][e] = (float)to_d<T>(from_f<T>(
                                 rotated_elem<T, D>(qrow0 + g * D, c * EPL + e, tab)));
                 } else {
                     const uint32_t qs = smem_addr(base + L::OFF_Q + stage * L::Q_BYTES);
@@ -800,7 +800,7 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
             const int j = s * NW + warp;
             if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
                 const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
-                item_patch_page<T, D, G, FUSED>(p, it, j, stage, base, tab);
+                item_patch_page<T, D, G, FUSED>(p, it, j, stage, base);
                 const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
                 const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
 #pragma unroll 2
@@ -897,8 +897,14 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
 
 // ------------------------------------------------------------------ kernel
 
+// Register budget: the d = 64 tensor-core kernels must fit three CTAs per SM
+// (their shared-memory ring allows it), i.e. at most 128 registers a thread;
+// the others are limited to two CTAs by shared memory anyway.
+template <bool MMA, int D>
+constexpr int decode_max_regs() { return (MMA && D == 64) ? 128 : 168; }
+
 template <typename T, int D, int G, bool MMA, bool FUSED>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+__global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<MMA, D>()))
     paged_decode_kernel(const __grid_constant__ DecodeParams p,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
@@ -984,8 +990,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     const int W = s_pre[B] * p.Hkv;
 
     if (warp == NW) {
-        run_producer<T, D, G, FUSED>(p, &tm_k, &tm_v, base, full, empty, masks, s_abort, s_len,
-                                     s_pre, W);
+        run_producer<T, D, G, FUSED>(p, fr, &tm_k, &tm_v, base, full, empty, masks, s_abort,
+                                     s_len, s_pre, W);
         return;
     }
     // zero the output of empty contexts (spread over the CTAs); in the fused
