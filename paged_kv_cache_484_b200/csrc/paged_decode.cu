@@ -1024,58 +1024,115 @@ struct CombineParams {
 
 // out[b, h*G+g, :] = sum_p w_p o_p with w_p = l_p 2^(m_p - M) / sum_q l_q 2^(m_q - M),
 // the exact log-sum-exp merge of the partition partials.  One CTA per
-// (kv head, sequence): a warp per query head turns (m_p, l_p) into weights,
-// then every thread owns one float4 column chunk of one partition group and
-// accumulates all G heads at once, so all partial loads are independent;
-// the partition groups are summed through shared memory.
+// (kv head, sequence); written for latency, since it sits at the end of every
+// split decode:
+//   * the context length and the (m, l) pairs of all NP possible partitions
+//     are loaded together (pairs past the sequence's own count are ignored);
+//   * every thread owns one float4 column chunk of one partition group and
+//     loads its first partials before the weights are known;
+//   * all heads' column sums meet in shared memory once, then are reduced.
 constexpr int kCombineThreads = 256;
 
 template <int D, int G>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_constant__ CombineParams p) {
     constexpr int CH = D / 4;                   // float4 chunks per row
     constexpr int PG = kCombineThreads / CH;    // partition groups
+    constexpr int kCombineUnroll = G >= 8 ? 1 : 8 / G;  // partitions in flight per head
     extern __shared__ float4 smem4[];
-    float4* red = smem4;                                       // [PG][CH]
-    float* w = reinterpret_cast<float*>(smem4 + PG * CH);      // [G][np]
+    float4* red = smem4;                                        // [G][PG][CH]
+    float* w = reinterpret_cast<float*>(smem4 + G * PG * CH);   // [G][NP]
     grid_dependency_wait();
     const int b = blockIdx.y, h = blockIdx.x;
-    int Lb = p.context_lens[b];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t hq0 = (size_t)b * p.Hq + (size_t)h * G;
     const int maxlen = p.MB * kPageRows;
+    int Lb = p.context_lens[b];
+    // (m, l) of this warp's head, all NP slots, issued with the length load
+    constexpr int MLR = 8;                      // slots per lane kept in registers
+    float2 ml[MLR];
+    const int g_w = warp;                       // warps 0..G-1 own one head each
+    if (g_w < G) {
+        const float2* src = reinterpret_cast<const float2*>(p.part_ml + (hq0 + g_w) * p.NP * 2);
+#pragma unroll
+        for (int r = 0; r < MLR; ++r) {
+            const int k = lane + 32 * r;
+            ml[r] = k < p.NP ? src[k] : make_float2(kNegInf, 0.f);
+        }
+    }
     Lb = Lb < 0 ? 0 : (Lb > maxlen ? maxlen : Lb);
     const int np = (Lb + p.P - 1) / p.P;
     if (np <= 1) return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int g = warp; g < G; g += kCombineThreads / 32) {
-        const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
-        const float2* ml = reinterpret_cast<const float2*>(p.part_ml + hq * p.NP * 2);
+
+    // first partials of this thread, independent of the weights
+    const int ch = threadIdx.x % CH, pg = threadIdx.x / CH;
+    float4 v0[G][kCombineUnroll];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int u = 0; u < kCombineUnroll; ++u) {
+            const int k = pg + u * PG;
+            v0[g][u] = k < np ? reinterpret_cast<const float4*>(
+                                    p.part_o + ((hq0 + g) * p.NP + k) * D)[ch]
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+
+    // weights: warp g turns head g's (m, l) pairs into normalised weights
+    if (g_w < G) {
+        const float2* src = reinterpret_cast<const float2*>(p.part_ml + (hq0 + g_w) * p.NP * 2);
         float M = kNegInf;
-        for (int k = lane; k < np; k += 32) M = fmaxf(M, ml[k].x);
+#pragma unroll
+        for (int r = 0; r < MLR; ++r)
+            if (lane + 32 * r < np) M = fmaxf(M, ml[r].x);
+        for (int k = lane + 32 * MLR; k < np; k += 32) M = fmaxf(M, src[k].x);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float S = 0.f;
-        for (int k = lane; k < np; k += 32) {
-            const float2 v = ml[k];
-            const float e = v.x == kNegInf ? 0.f : fast_exp2(v.x - M) * v.y;
-            w[g * np + k] = e;
-            S += e;
+        float e[MLR];
+#pragma unroll
+        for (int r = 0; r < MLR; ++r) {
+            const int k = lane + 32 * r;
+            e[r] = (k < np && ml[r].x != kNegInf) ? fast_exp2(ml[r].x - M) * ml[r].y : 0.f;
+            S += e[r];
+        }
+        for (int k = lane + 32 * MLR; k < np; k += 32) {
+            const float2 v = src[k];
+            const float ek = v.x == kNegInf ? 0.f : fast_exp2(v.x - M) * v.y;
+            w[g_w * p.NP + k] = ek;
+            S += ek;
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(0xffffffffu, S, off);
         const float inv = S > 0.f ? 1.f / S : 0.f;
-        for (int k = lane; k < np; k += 32) w[g * np + k] *= inv;
+#pragma unroll
+        for (int r = 0; r < MLR; ++r) {
+            const int k = lane + 32 * r;
+            if (k < np) w[g_w * p.NP + k] = e[r] * inv;
+        }
+        for (int k = lane + 32 * MLR; k < np; k += 32) w[g_w * p.NP + k] *= inv;
     }
     __syncthreads();
-    const int ch = threadIdx.x % CH, pg = threadIdx.x / CH;
+
     float4 acc[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const size_t hq0 = (size_t)b * p.Hq + (size_t)h * G;
+    for (int g = 0; g < G; ++g) {
+        acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < kCombineUnroll; ++u) {
+            const int k = pg + u * PG;
+            const float wk = k < np ? w[g * p.NP + k] : 0.f;
+            acc[g].x = fmaf(wk, v0[g][u].x, acc[g].x);
+            acc[g].y = fmaf(wk, v0[g][u].y, acc[g].y);
+            acc[g].z = fmaf(wk, v0[g][u].z, acc[g].z);
+            acc[g].w = fmaf(wk, v0[g][u].w, acc[g].w);
+        }
+    }
+    // partitions beyond the first kCombineUnroll rounds (long contexts)
 #pragma unroll 2
-    for (int k = pg; k < np; k += PG) {
+    for (int k = pg + kCombineUnroll * PG; k < np; k += PG) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             const float4 v = reinterpret_cast<const float4*>(p.part_o + ((hq0 + g) * p.NP + k) * D)[ch];
-            const float wk = w[g * np + k];
+            const float wk = w[g * p.NP + k];
             acc[g].x = fmaf(wk, v.x, acc[g].x);
             acc[g].y = fmaf(wk, v.y, acc[g].y);
             acc[g].z = fmaf(wk, v.z, acc[g].z);
@@ -1083,25 +1140,23 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_c
         }
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        red[pg * CH + ch] = acc[g];
-        __syncthreads();
-        if (threadIdx.x < CH) {
-            float4 s = red[threadIdx.x];
-            for (int q = 1; q < PG; ++q) {
-                const float4 v = red[q * CH + threadIdx.x];
-                s.x += v.x;
-                s.y += v.y;
-                s.z += v.z;
-                s.w += v.w;
-            }
-            const size_t o = (hq0 + g) * D + threadIdx.x * 4;
-            store_out(p.out, o, s.x, p.out_bf16);
-            store_out(p.out, o + 1, s.y, p.out_bf16);
-            store_out(p.out, o + 2, s.z, p.out_bf16);
-            store_out(p.out, o + 3, s.w, p.out_bf16);
+    for (int g = 0; g < G; ++g) red[(g * PG + pg) * CH + ch] = acc[g];
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * CH; idx += kCombineThreads) {
+        const int g = idx / CH, c = idx - (idx / CH) * CH;
+        float4 sum = red[(g * PG) * CH + c];
+        for (int q = 1; q < PG; ++q) {
+            const float4 v = red[(g * PG + q) * CH + c];
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
         }
-        __syncthreads();
+        const size_t o = (hq0 + g) * D + c * 4;
+        store_out(p.out, o, sum.x, p.out_bf16);
+        store_out(p.out, o + 1, sum.y, p.out_bf16);
+        store_out(p.out, o + 2, sum.z, p.out_bf16);
+        store_out(p.out, o + 3, sum.w, p.out_bf16);
     }
 }
 
@@ -1200,7 +1255,19 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     cp.NP = a.max_partitions;
     cp.out_bf16 = p.out_bf16;
     auto ckern = combine_kernel<D, G>;
-    const size_t csmem = (size_t)kCombineThreads * 16 + (size_t)G * a.max_partitions * sizeof(float);
+    {
+        static std::mutex mu;
+        static size_t set_bytes[64] = {0};
+        const int dev = current_device();
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev >= 0 && dev < 64 && set_bytes[dev] < (size_t)(G * kCombineThreads * 16 + G * kMaxPartitions * 4)) {
+            e = cudaFuncSetAttribute(ckern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     G * kCombineThreads * 16 + G * kMaxPartitions * 4);
+            if (e != cudaSuccess) return e;
+            set_bytes[dev] = (size_t)(G * kCombineThreads * 16 + G * kMaxPartitions * 4);
+        }
+    }
+    const size_t csmem = (size_t)G * kCombineThreads * 16 + (size_t)G * a.max_partitions * sizeof(float);
     cudaLaunchConfig_t cc = cfg;
     cc.gridDim = dim3((unsigned)a.Hkv, (unsigned)a.B);
     cc.blockDim = dim3(kCombineThreads);
