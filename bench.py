@@ -319,7 +319,7 @@ def run_ours(args):
     NP = math.ceil(w.max_blocks * w.block_size / P)
     ws_bytes = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=w.dtype,
                                          partition_tokens=P)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    ws = pkv.new_workspace(ws_bytes, device)
     out = torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)

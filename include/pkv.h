@@ -142,16 +142,19 @@ pkv_status pkv_kv_append(void* q, const void* k_new, const void* v_new,
 
 /*
  * pkv_decode_workspace_size -- bytes of workspace pkv_paged_attention_decode
- * needs for these shapes (0 when no context is split).
+ * needs for these shapes.
  *
- * The workspace holds the per-partition partial results (running max, sum
- * and un-normalised output) of the split-context ("flash-decoding") path:
- * num_seqs * Hq * max_partitions * (head_dim + 2) floats, where
- * max_partitions = ceil(max_blocks_per_seq * block_size / P) and P is the
- * partition length the decode call will use (partition_tokens, or the
- * library's choice for the current device when it is 0).  Pass the same
- * shapes, dtype and partition_tokens to both calls.  Host only; no device
- * memory is touched.  Returns 0 for invalid arguments.
+ * Layout: 256 bytes of work-scheduler counters, then, when contexts are
+ * split, the per-partition partial results (running max, sum and output) of
+ * the split-context ("flash-decoding") path: num_seqs * Hq * max_partitions *
+ * (head_dim + 2) floats, where max_partitions = ceil(max_blocks_per_seq *
+ * block_size / P) and P is the partition length the decode call will use
+ * (partition_tokens, or the library's choice for the current device when it
+ * is 0).  Pass the same shapes, dtype and partition_tokens to both calls.
+ * The counters let CTAs that finish early claim more work items; they must
+ * be zero before a workspace's first call (zero the first 256 bytes once,
+ * e.g. with cudaMemset at allocation) and every call leaves them zero.  Host
+ * only; no device memory is touched.  Returns 0 for invalid arguments.
  */
 size_t pkv_decode_workspace_size(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
                                  int64_t head_dim, int64_t max_blocks_per_seq,
@@ -191,10 +194,12 @@ int32_t pkv_decode_partition_tokens(int64_t num_seqs, int64_t num_q_heads, int64
  *                 ceil(L / block_size) entries of a row are read
  *   context_lens  device, [num_seqs] int32 in [0, max_blocks_per_seq * block_size]
  *   out           device, [num_seqs, Hq, head_dim], out_dtype (f32 or bf16)
- *   workspace     device, >= pkv_decode_workspace_size(...) bytes (may be NULL
- *                 when that size is 0); contents need no initialisation and
- *                 are clobbered; two calls in flight at once need two
- *                 workspaces
+ *   workspace     device, >= pkv_decode_workspace_size(...) bytes, 16-byte
+ *                 aligned; its first 256 bytes zero before its first call
+ *                 (each call leaves them zero), the rest is clobbered.  Two
+ *                 calls in flight at once need two workspaces.  May be NULL
+ *                 when max_partitions is 1 (no context is split): the work
+ *                 items are then dealt out round-robin instead of claimed
  *   partition_tokens  0 = library choice, else a multiple of block_size in
  *                 [block_size, PKV_MAX_PARTITION_TOKENS]: each sequence is cut
  *                 into ceil(L / P) partitions that run in parallel and are
@@ -286,11 +291,11 @@ pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new,
  *   * The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress); make that first call before any stream
  *     capture.
- *   * Every call on a device shares the one array, and it keeps the last
- *     call's contents.  Nothing in it has to start at zero.  Calls that can
- *     overlap on the GPU (other streams, other host threads) race on it:
- *     serialise them, or give each its own workspace through
- *     pkv_paged_attention_decode.
+ *   * Every call on a device shares the one array.  Its scheduler counters
+ *     start at zero (static storage) and every call leaves them zero; the
+ *     rest keeps the last call's partials.  Calls that can overlap on the GPU
+ *     (other streams, other host threads) race on it: serialise them, or
+ *     give each its own workspace through pkv_paged_attention_decode.
  */
 pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache,
                                               const void* v_cache, const int32_t* block_tables,

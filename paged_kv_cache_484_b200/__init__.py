@@ -8,7 +8,8 @@ operation names:
 * ``paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, stream)``
 
 plus ``decode_step`` (both in one launch), ``paged_attention_decode_noalloc``
-and ``decode_workspace_size`` / ``decode_partition_tokens`` for planning.
+and ``decode_workspace_size`` / ``decode_partition_tokens`` / ``new_workspace``
+for planning.
 PyTorch is used for device memory and streams only; the library is loaded on
 first use and its absence is an error, never a fallback.
 """
@@ -21,11 +22,13 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     NOALLOC_SCRATCH_BYTES,
     PkvError,
+    SCHED_BYTES,
     decode_partition_tokens,
     decode_step,
     decode_workspace_size,
     kv_append,
     load_library,
+    new_workspace,
     paged_attention_decode,
     paged_attention_decode_noalloc,
     version,

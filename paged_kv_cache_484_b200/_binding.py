@@ -162,6 +162,18 @@ def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blo
                                              _dtype_code(kv_dtype), int(partition_tokens)))
 
 
+SCHED_BYTES = 256  # scheduler counters at the head of a decode workspace
+
+
+def new_workspace(nbytes, device) -> torch.Tensor:
+    """A decode workspace of ``nbytes`` on ``device`` with its scheduler
+    counters zeroed (the rest needs no initialisation); reusable by later
+    calls, which leave the counters zero."""
+    ws = torch.empty(max(int(nbytes), SCHED_BYTES), dtype=torch.uint8, device=device)
+    ws[:SCHED_BYTES].zero_()
+    return ws
+
+
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out,
                            stream=None, *, workspace=None, partition_tokens=0, force_simt=False,
                            device_error=None) -> torch.Tensor:
@@ -170,8 +182,10 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     q [B, Hq, d] and caches [NB, Hkv, 16, d] share a dtype (float32 or
     bfloat16); block_tables int32 [B, MB]; context_lens int32 [B];
     out [B, Hq, d] float32 or bfloat16.  ``workspace`` (uint8 CUDA tensor of
-    at least ``decode_workspace_size`` bytes) is allocated from PyTorch's
-    caching allocator when not given.  See include/pkv.h.
+    at least ``decode_workspace_size`` bytes, see ``new_workspace``) is
+    allocated from PyTorch's caching allocator when not given; an empty tensor
+    passes none, which is allowed when no context is split (the work items
+    are then dealt out round-robin).  See include/pkv.h.
     """
     lib = load_library()
     kv_dt = _dtype_code(k_cache.dtype)
@@ -186,7 +200,7 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     out_dt = _dtype_code(out.dtype)
     need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
     if workspace is None:
-        workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+        workspace = new_workspace(int(need), q.device)
     err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
     st = lib.pkv_paged_attention_decode(
         _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
@@ -223,7 +237,7 @@ def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, bloc
         raise ValueError("inconsistent decode_step shapes")
     need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
     if workspace is None:
-        workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+        workspace = new_workspace(int(need), q.device)
     err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
     st = lib.pkv_decode_step(
         _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),

@@ -78,8 +78,10 @@ extern "C" pkv_status pkv_paged_attention_decode_noalloc(
             return PKV_ERR_CUDA;
         }
     }
-    // Nothing in the scratch has to start at zero: every partial that a call
-    // reads was written earlier in the same call.
+    // The scheduler counters at the head of the scratch start at zero (device
+    // statics are zero-initialised when the module loads) and every call
+    // leaves them zero; every partial that a call reads was written earlier
+    // in the same call.
     return pkv_paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, out,
                                       scratch, need > 0 ? (size_t)PKV_NOALLOC_SCRATCH_BYTES : 0,
                                       num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,

@@ -71,13 +71,22 @@ struct Layout {
     static constexpr int PAGE_BYTES = kPageRows * ROW_BYTES;
     static constexpr int BOXES = SWZ ? D / 64 : 1;  // TMA boxes per page
     static constexpr int BOX_BYTES = PAGE_BYTES / BOXES;
-    static constexpr int STAGE_BYTES = 2 * NW * PAGE_BYTES;  // NW K pages then NW V pages
-    static constexpr int STAGES = cmax(2, cmin(6, 49152 / STAGE_BYTES));
+    // Pages each consumer warp takes per stage: two for the d = 64 bf16
+    // tensor-core path with G <= 4 (a 32-token tile: longer independent MMA
+    // chains and half the softmax bookkeeping per token), else one.
+    static constexpr int PPW = (SWZ && D == 64 && G <= 4) ? 2 : 1;
+    static constexpr int STAGE_PAGES = NW * PPW;
+    static constexpr int STAGE_BYTES = 2 * STAGE_PAGES * PAGE_BYTES;  // K pages, then V pages
+    static constexpr int STAGES = cmax(2, cmin(6, 65536 / STAGE_BYTES));
     static constexpr int Q_COPY = G * D * ESZ;
     static constexpr int Q_BYTES = round_up(Q_COPY, 128);
     static constexpr int ROW_COPY = D * ESZ;           // one k or v row
     static constexpr int NEWKV_BYTES = 2 * ROW_COPY;   // fused step: raw new k row, new v row
-    static constexpr int MERGE_FLOATS = NW * G * (D + 2);
+    // Item merge: each warp leaves (o[D], m, l) per head in its own K and V
+    // page slots of the item's last stage (free once it has read its pages).
+    static constexpr int MERGE_ROW_BYTES = (D + 2) * 4;
+    static constexpr int MERGE_ROWS_PER_SLOT = PPW * PAGE_BYTES / MERGE_ROW_BYTES;
+    static_assert(2 * MERGE_ROWS_PER_SLOT >= G, "merge rows do not fit a warp's page slots");
     // byte offsets from the 1024-aligned base
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
     static constexpr int OFF_NEWKV = OFF_Q + STAGES * Q_BYTES;
@@ -85,11 +94,11 @@ struct Layout {
     // written by the producer with the item's first stage
     static constexpr int ROPE_BYTES = D * 4;
     static constexpr int OFF_ROPE = OFF_NEWKV + STAGES * NEWKV_BYTES;
-    static constexpr int OFF_MERGE = OFF_ROPE + STAGES * ROPE_BYTES;
-    static constexpr int OFF_BAR = OFF_MERGE + 2 * MERGE_FLOATS * 4;
+    static constexpr int OFF_BAR = OFF_ROPE + STAGES * ROPE_BYTES;
     static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
     static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
-    static constexpr int OFF_MISC = OFF_PATCH + STAGES * 8;  // abort flag + 8 scan slots
+    static constexpr int OFF_ITEM = OFF_PATCH + STAGES * 8;  // work item of each stage, -1: no more
+    static constexpr int OFF_MISC = OFF_ITEM + STAGES * 4;   // abort flag + 8 scan slots
     static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;        // s_len[B], s_pre[B + 1]
     static size_t smem_bytes(int B) { return 1024 + OFF_SEQ + (size_t)(2 * B + 1) * 4; }
 };
@@ -102,6 +111,9 @@ struct DecodeParams {
     float* part_o;
     float* part_ml;
     int32_t* err;
+    // item counter and finished-CTA counter (zero before the launch, zero
+    // after it); null: items are dealt out round-robin instead
+    uint32_t* sched;
     int B, Hq, Hkv, MB, P, NP;
     int num_blocks;
     float scale_log2;
@@ -191,13 +203,20 @@ __device__ __forceinline__ bf16 from_d<bf16>(double x) {
 // Fused step: a warp writes the cos/sin table of a position, tab[i] =
 // cos(pos f_i), tab[D/2 + i] = sin(pos f_i), i < D/2: angle in fp64, reduced
 // mod 2pi in fp64, then sine and cosine in fp32 of the reduced angle.
+// Lane i handles i and i + 32; `f` holds theta^(-2i/d) for those.
 template <int D>
-__device__ __forceinline__ void warp_rope_table(double pos, const RopeFreq& fr, float* tab) {
-    for (int i = threadIdx.x & 31; i < D / 2; i += 32) {
-        float sn, cs;
-        sincosf((float)reduce_two_pi(pos * fr.f[i]), &sn, &cs);
-        tab[i] = cs;
-        tab[D / 2 + i] = sn;
+__device__ __forceinline__ void warp_rope_table(double pos, const double (&f)[(D + 63) / 64],
+                                                float* tab) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int u = 0; u < (D + 63) / 64; ++u) {
+        const int i = lane + 32 * u;
+        if (i < D / 2) {
+            float sn, cs;
+            sincosf((float)reduce_two_pi(pos * f[u]), &sn, &cs);
+            tab[i] = cs;
+            tab[D / 2 + i] = sn;
+        }
     }
 }
 
@@ -283,47 +302,89 @@ __device__ void append_only(const DecodeParams& p, const RopeFreq& fr, int b) {
 
 // ---------------------------------------------------------------- producer
 
+// Reads the producer issues before the context lengths are known, for the
+// first item this CTA would get if every sequence had NP partitions (exact
+// for uniform batches; a wrong guess costs the reads and nothing else).
+template <int D>
+struct FirstItemGuess {
+    int b = -1, part = -1;
+    int ent = -1;                 // block-table entry of page `lane` of the item
+    int64_t slot = -1, pos = 0;   // fused step: the sequence's new token
+    double f[(D + 63) / 64];      // fused step: RoPE frequencies of this lane
+};
+
 template <typename T, int D, int G, bool FUSED>
-__device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CUtensorMap* tmk,
-                             const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
-                             uint64_t* empty, uint32_t* masks, volatile int* s_abort,
-                             const int* s_len, const int* s_pre, int W) {
+__device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& guess,
+                             const CUtensorMap* tmk, const CUtensorMap* tmv, uint8_t* base,
+                             uint64_t* full, uint64_t* empty, uint32_t* masks,
+                             volatile int* s_abort, const int* s_len, const int* s_pre, int W) {
     using L = Layout<T, D, G>;
     const int lane = threadIdx.x & 31;
-    int item = blockIdx.x;
-    if (item >= W) return;
+    int* s_item = reinterpret_cast<int*>(base + L::OFF_ITEM);
 
-    auto entry = [&](const Item& it, int page) -> int {
-        if (page >= it.npages) return -1;
-        const int jb = it.t0 / kPageRows + page;
-        const int v = p.block_tables[(size_t)it.b * p.MB + jb];
+    // Work order of this CTA: items blockIdx.x and blockIdx.x + gridDim.x,
+    // then items claimed one at a time from the counter (2 gridDim.x + its
+    // old value), so that CTAs that finish early take more; without a
+    // counter, blockIdx.x + k gridDim.x.  A claim is issued one item before
+    // its result is needed, and nothing touches the returned value until
+    // then (the warp would stall on it).  Claimed values only grow, so once
+    // a CTA sees an item >= W every later claim is past W too and nothing
+    // claimed is lost.
+    int item = blockIdx.x;
+    int item1 = item + (int)gridDim.x;  // the item after `item`
+    uint32_t pend = 0;                  // lane 0: raw counter value of the claim in flight
+    int k_static = 2;
+    auto issue_claim = [&]() {
+        if (p.sched && lane == 0) pend = atomicAdd(p.sched, 1u);
+    };
+    auto take_claim = [&]() -> int {
+        int v;
+        if (p.sched)
+            v = 2 * (int)gridDim.x + (int)__shfl_sync(0xffffffffu, pend, 0);
+        else
+            v = (int)blockIdx.x + k_static * (int)gridDim.x;
+        ++k_static;
+        return v;
+    };
+
+    auto checked = [&](int v) -> int {
         if (v < 0 || v >= p.num_blocks) {
             report_error(p.err, PKV_DEVERR_BLOCK_ID);
             return -1;
         }
         return v;
     };
+    auto entry = [&](const Item& it, int page) -> int {
+        if (page >= it.npages) return -1;
+        const int jb = it.t0 / kPageRows + page;
+        return checked(p.block_tables[(size_t)it.b * p.MB + jb]);
+    };
 
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_parity[8];  // parity of the last issue into each stage
     uint32_t issued_any = 0;
+    bool abort = false;
+    if (item < W) {
+    if (item1 < W) issue_claim();
     Item cur = decode_item(item, p, s_len, s_pre);
     int c0 = 0;
-    int cur_ent = entry(cur, lane);
-    // fused step: the new token's slot and position, read together with the
-    // block table
-    int64_t cur_slot = FUSED ? p.slot_mapping[cur.b] : -1;
-    int64_t cur_pos = FUSED ? p.positions[cur.b] : 0;
+    const bool hit = cur.b == guess.b && cur.part == guess.part;
+    int cur_ent = hit ? (lane < cur.npages ? checked(guess.ent) : -1) : entry(cur, lane);
+    // fused step: the new token's slot and position
+    int64_t cur_slot = -1, cur_pos = 0;
+    if constexpr (FUSED) {
+        cur_slot = hit ? guess.slot : p.slot_mapping[cur.b];
+        cur_pos = hit ? guess.pos : p.positions[cur.b];
+    }
     int* patch = reinterpret_cast<int*>(base + L::OFF_PATCH);
-    bool abort = false;
 
     while (!abort) {
         // prefetch the block-table entries of the next chunk of 32 pages
         int nitem = item, nc0 = c0 + 32;
         Item nxt = cur;
         if (nc0 >= cur.npages) {
-            nitem = item + gridDim.x;
+            nitem = item1;
             nc0 = 0;
             if (nitem < W) nxt = decode_item(nitem, p, s_len, s_pre);
         }
@@ -333,8 +394,8 @@ __device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CU
         const int64_t nxt_pos = new_item ? p.positions[nxt.b] : cur_pos;
 
         const int cend = min(cur.npages, c0 + 32);
-        for (int s0 = c0; s0 < cend; s0 += NW) {
-            const int npg = min(NW, cur.npages - s0);
+        for (int s0 = c0; s0 < cend; s0 += L::STAGE_PAGES) {
+            const int npg = min(L::STAGE_PAGES, cur.npages - s0);
             const int k = lane - (s0 - c0);
             const bool mine = k >= 0 && k < npg && cur_ent >= 0;
             const uint32_t vmask = __ballot_sync(0xffffffffu, mine) >> (s0 - c0);
@@ -346,13 +407,13 @@ __device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CU
                 break;
             }
             uint8_t* kdst = base + stage * L::STAGE_BYTES;
-            uint8_t* vdst = kdst + NW * L::PAGE_BYTES;
+            uint8_t* vdst = kdst + L::STAGE_PAGES * L::PAGE_BYTES;
             const bool first = (s0 == 0);
             // fused step: the sequence's last page gets the new token's row;
             // only when its slot is the one the block table gives that token
             int patch_row = -1, patch_blk = 0;
             if constexpr (FUSED) {
-                if (s0 + NW >= cur.npages && cur.part == cur.np - 1) {
+                if (s0 + L::STAGE_PAGES >= cur.npages && cur.part == cur.np - 1) {
                     const int lastpage = cur.npages - 1;
                     const int phys = __shfl_sync(0xffffffffu, cur_ent, lastpage - c0);
                     const int row = (s_len[cur.b] - 1) % kPageRows;
@@ -366,26 +427,15 @@ __device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CU
                     }
                 }
             }
-            if constexpr (FUSED) {
-                // the rope table rides with the item's first stage and with
-                // the stage that carries the new token
-                if (first || patch_row >= 0) {
-                    warp_rope_table<D>((double)cur_pos, fr,
-                                       reinterpret_cast<float*>(base + L::OFF_ROPE +
-                                                                stage * L::ROPE_BYTES));
-                    __syncwarp();
-                }
-            }
+            // The stage's bytes are announced first and the copies issued at
+            // once; what the producer writes itself (mask, patch, rope table)
+            // follows while the copies are in flight and is published by the
+            // stage's one arrival.
             if (lane == 0) {
-                masks[stage] = vmask;
-                if constexpr (FUSED) {
-                    patch[2 * stage] = patch_row;
-                    patch[2 * stage + 1] = patch_blk;
-                }
                 const uint32_t bytes = __popc(vmask) * 2u * L::PAGE_BYTES +
                                        (first ? (uint32_t)L::Q_COPY : 0u) +
                                        (patch_row >= 0 ? (uint32_t)L::NEWKV_BYTES : 0u);
-                mbar_arrive_expect_tx(&full[stage], bytes);
+                mbar_expect_tx(&full[stage], bytes);
             }
             __syncwarp();
             if (mine) {
@@ -411,6 +461,24 @@ __device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CU
                 bulk_load(nk + L::ROW_COPY, reinterpret_cast<const uint8_t*>(p.v_new) + row_off,
                           L::ROW_COPY, &full[stage]);
             }
+            if constexpr (FUSED) {
+                // the rope table rides with the item's first stage and with
+                // the stage that carries the new token
+                if (first || patch_row >= 0)
+                    warp_rope_table<D>((double)cur_pos, guess.f,
+                                       reinterpret_cast<float*>(base + L::OFF_ROPE +
+                                                                stage * L::ROPE_BYTES));
+            }
+            if (lane == 0) {
+                masks[stage] = vmask;
+                s_item[stage] = item;
+                if constexpr (FUSED) {
+                    patch[2 * stage] = patch_row;
+                    patch[2 * stage + 1] = patch_blk;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[stage]);
             issued_parity[stage] = phase;
             issued_any |= 1u << stage;
             if (++stage == L::STAGES) {
@@ -419,6 +487,10 @@ __device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CU
             }
         }
         if (abort || nitem >= W) break;
+        if (nitem != item) {
+            item1 = take_claim();
+            if (item1 < W) issue_claim();
+        }
         item = nitem;
         c0 = nc0;
         cur = nxt;
@@ -426,6 +498,17 @@ __device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CU
         cur_slot = nxt_slot;
         cur_pos = nxt_pos;
     }
+    }
+    if (!abort && lane == 0) {
+        // no more work: a stage without data whose item is -1 tells the consumers
+        if (mbar_wait(&empty[stage], phase ^ 1) && !*s_abort) {
+            s_item[stage] = -1;
+            mbar_arrive(&full[stage]);
+        } else {
+            abort = true;
+        }
+    }
+    abort = __shfl_sync(0xffffffffu, abort, 0);
     if (abort) {
         *s_abort = 1;
         if (lane == 0) {
@@ -436,24 +519,46 @@ __device__ void run_producer(const DecodeParams& p, const RopeFreq& fr, const CU
         }
         __syncwarp();
     }
+    // This CTA has made its last claim.  The last CTA to get here puts both
+    // counters back to zero for the next launch.
+    if (p.sched && lane == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
+        }
+    }
 }
 
 // ------------------------------------------------------------ item merge
 
-// All consumer warps have written (o, m, l) per head into `mb`; merge them
-// and write the output row or the partition partial.
-template <int D, int G>
+// Row g (head g of the item) of warp w's merge record in stage `st`.
+template <typename T, int D, int G>
+__device__ __forceinline__ float* merge_row(uint8_t* base, int st, int w, int g) {
+    using L = Layout<T, D, G>;
+    uint8_t* kslot = base + st * L::STAGE_BYTES + w * L::PPW * L::PAGE_BYTES;
+    uint8_t* row = g < L::MERGE_ROWS_PER_SLOT
+                       ? kslot + g * L::MERGE_ROW_BYTES
+                       : kslot + L::STAGE_PAGES * L::PAGE_BYTES +
+                             (g - L::MERGE_ROWS_PER_SLOT) * L::MERGE_ROW_BYTES;
+    return reinterpret_cast<float*>(row);
+}
+
+// All consumer warps have written (o, m, l) per head into their merge rows
+// of stage `st`; merge them and write the output row or the partition
+// partial.
+template <typename T, int D, int G>
 __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Item& it,
-                                                const float* mb) {
+                                                uint8_t* base, int st) {
     for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
         const int g = idx / D, dim = idx - (idx / D) * D;
         float M = kNegInf;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, mb[(w * G + g) * (D + 2) + D]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, merge_row<T, D, G>(base, st, w, g)[D]);
         float num = 0.f, den = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-            const float* row = mb + (w * G + g) * (D + 2);
+            const float* row = merge_row<T, D, G>(base, st, w, g);
             const float f = row[D] == kNegInf ? 0.f : fast_exp2(row[D] - M);
             num += f * row[dim];
             den += f * row[D + 1];
@@ -490,7 +595,7 @@ __device__ __forceinline__ bool consumer_sync(const DecodeParams& p, uint64_t* b
 // Fused step, page that holds the sequence's newest token: patch it in.
 template <typename T, int D, int G, bool FUSED>
 __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Item& it, int j,
-                                                int stage, uint8_t* base) {
+                                                int slot, int stage, uint8_t* base) {
     if constexpr (FUSED) {
         using L = Layout<T, D, G>;
         const float* tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
@@ -498,8 +603,8 @@ __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Ite
         if (pt[0] >= 0 && j == it.npages - 1) {
             const int row = pt[0];
             const size_t grow = (((size_t)pt[1] * p.Hkv + it.h) * kPageRows + row) * D;
-            uint8_t* kpage = base + stage * L::STAGE_BYTES + (threadIdx.x >> 5) * L::PAGE_BYTES;
-            patch_new_row<T, D>(kpage, kpage + NW * L::PAGE_BYTES,
+            uint8_t* kpage = base + stage * L::STAGE_BYTES + slot * L::PAGE_BYTES;
+            patch_new_row<T, D>(kpage, kpage + L::STAGE_PAGES * L::PAGE_BYTES,
                                 base + L::OFF_NEWKV + stage * L::NEWKV_BYTES, row, tab,
                                 reinterpret_cast<T*>(p.k_cache) + grow,
                                 reinterpret_cast<T*>(p.v_cache) + grow);
@@ -529,12 +634,19 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
 
     int stage = 0;
     uint32_t phase = 0, mphase = 0;
-    int mbuf = 0;
-    float* merge = reinterpret_cast<float*>(base + L::OFF_MERGE);
     // fused step: the item's rope table, staged by the producer with its first stage
     const float* tab = nullptr;
 
-    for (int item = blockIdx.x; item < W; item += gridDim.x) {
+    const int* s_item = reinterpret_cast<const int*>(base + L::OFF_ITEM);
+    for (;;) {
+        // the item's first stage says which item it is (-1: no more work)
+        if (!mbar_wait(&full[stage], phase) || *s_abort) {
+            *s_abort = 1;
+            if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
+            return;
+        }
+        const int item = s_item[stage];
+        if (item < 0) return;
         const Item it = decode_item(item, p, s_len, s_pre);
         float o[NT][4];
 #pragma unroll
@@ -542,10 +654,11 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
         float m_run = kNegInf, l_run = 0.f;
         uint32_t qa[KS][4];
 
-        const int nst = (it.npages + NW - 1) / NW;
+        const int nst = (it.npages + L::STAGE_PAGES - 1) / L::STAGE_PAGES;
         bool ok = true;
+        int last = stage;
         for (int s = 0; s < nst; ++s) {
-            ok = mbar_wait(&full[stage], phase) && !*s_abort;
+            ok = (s == 0 || mbar_wait(&full[stage], phase)) && !*s_abort;
             if (!ok) break;
             if (s == 0) {
                 tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
@@ -587,92 +700,129 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
                     qa[kk][3] = a3;  // row r+8
                 }
             }
-            const int j = s * NW + warp;
-            if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
-                const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
-                item_patch_page<bf16, D, G, FUSED>(p, it, j, stage, base);
-                const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
-                const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
+            // this warp's PPW consecutive pages of the stage (a page whose
+            // block id was rejected counts as empty)
+            constexpr int PPW = L::PPW;
+            const int j0 = s * L::STAGE_PAGES + warp * PPW;
+            const uint32_t mk = (masks[stage] >> (warp * PPW)) & ((1u << PPW) - 1u);
+            if (j0 < it.npages && mk != 0u) {
+                int valid[PPW];
+#pragma unroll
+                for (int u = 0; u < PPW; ++u) {
+                    const int jj = j0 + u;
+                    valid[u] = (jj < it.npages && ((mk >> u) & 1u))
+                                   ? min(kPageRows, it.t1 - (it.t0 + jj * kPageRows))
+                                   : 0;
+                    if (valid[u] > 0)
+                        item_patch_page<bf16, D, G, FUSED>(p, it, jj, warp * PPW + u, stage, base);
+                }
+                const uint32_t kbase =
+                    smem_addr(base + stage * L::STAGE_BYTES + warp * PPW * L::PAGE_BYTES);
+                const uint32_t vbase = kbase + L::STAGE_PAGES * L::PAGE_BYTES;
                 const int mi = lane >> 3, ri = lane & 7;
 
-                // S^T tile: 16 rows (heads) x 16 tokens, as two n-tiles of 8 tokens
-                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                // S^T tile: 16 rows (heads) x 16 PPW tokens, n-tiles of 8 tokens
+                float sc[2 * PPW][4];
+#pragma unroll
+                for (int n = 0; n < 2 * PPW; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
 #pragma unroll
                 for (int kk = 0; kk < KS; ++kk) {
                     const int tok = ri + ((mi >> 1) << 3);
                     const int ch = 2 * kk + (mi & 1);
-                    uint32_t b00, b01, b10, b11;
-                    ldsm_x4(kbase + chunk_offset<bf16, D>(tok, ch), b00, b01, b10, b11);
-                    mma_bf16_16816(sc[0], qa[kk], b00, b01);
-                    mma_bf16_16816(sc[1], qa[kk], b10, b11);
+#pragma unroll
+                    for (int u = 0; u < PPW; ++u) {
+                        uint32_t b00, b01, b10, b11;
+                        ldsm_x4(kbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch), b00, b01,
+                                b10, b11);
+                        mma_bf16_16816(sc[2 * u], qa[kk], b00, b01);
+                        mma_bf16_16816(sc[2 * u + 1], qa[kk], b10, b11);
+                    }
                 }
                 // online softmax in the log2 domain; rows r carry c0, c1
-                float x[2][2];
+                float x[2 * PPW][2];
 #pragma unroll
-                for (int n = 0; n < 2; ++n)
+                for (int n = 0; n < 2 * PPW; ++n)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int tk = n * 8 + 2 * cq + e;
-                        x[n][e] = tk < valid ? sc[n][e] * p.scale_log2 : kNegInf;
+                        const int tk = (n & 1) * 8 + 2 * cq + e;
+                        x[n][e] = tk < valid[n >> 1] ? sc[n][e] * p.scale_log2 : kNegInf;
                     }
-                float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+                float mx = kNegInf;
+#pragma unroll
+                for (int n = 0; n < 2 * PPW; ++n) mx = fmaxf(mx, fmaxf(x[n][0], x[n][1]));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
                 const float m_new = fmaxf(m_run, mx);
                 const float alpha = fast_exp2(m_run - m_new);
-                float pr[2][2];
+                float pr[2 * PPW][2];
+                float psum = 0.f;
 #pragma unroll
-                for (int n = 0; n < 2; ++n)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) pr[n][e] = fast_exp2(x[n][e] - m_new);
-                l_run = l_run * alpha + ((pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
-                m_run = m_new;
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    o[n][0] *= alpha;
-                    o[n][1] *= alpha;
-                    o[n][2] *= alpha;
-                    o[n][3] *= alpha;
+                for (int n = 0; n < 2 * PPW; ++n) {
+                    pr[n][0] = fast_exp2(x[n][0] - m_new);
+                    pr[n][1] = fast_exp2(x[n][1] - m_new);
+                    psum += pr[n][0] + pr[n][1];
                 }
-                // P as the A operand of the output MMA: two-term bf16 split
-                uint32_t pa[4];
-                {
-                    const uint32_t hi0 = pack_bf16(pr[0][0], pr[0][1]);
-                    const uint32_t hi1 = pack_bf16(pr[1][0], pr[1][1]);
-                    const uint32_t lo0 = pack_bf16(pr[0][0] - bf16lo(hi0), pr[0][1] - bf16hi(hi0));
-                    const uint32_t lo1 = pack_bf16(pr[1][0] - bf16lo(hi1), pr[1][1] - bf16hi(hi1));
-                    if (G == 8) {
-                        pa[0] = hi0;
-                        pa[1] = lo0;
-                        pa[2] = hi1;
-                        pa[3] = lo1;
-                    } else {
-                        pa[0] = row_used ? (row_is_lo ? lo0 : hi0) : 0u;
-                        pa[2] = row_used ? (row_is_lo ? lo1 : hi1) : 0u;
-                        pa[1] = 0u;
-                        pa[3] = 0u;
+                l_run = l_run * alpha + psum;
+                // alpha is exactly 1 in every row whose maximum did not grow;
+                // skip the rescale when that holds for the whole warp
+                if (__any_sync(0xffffffffu, m_new != m_run)) {
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        o[n][0] *= alpha;
+                        o[n][1] *= alpha;
+                        o[n][2] *= alpha;
+                        o[n][3] *= alpha;
                     }
                 }
-                // O += P V over the page's 16 tokens
-                uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
-                if (valid < kPageRows) {
-                    const int k0 = 2 * cq;
-                    vmask_lo = (k0 < valid ? 0x0000ffffu : 0u) | (k0 + 1 < valid ? 0xffff0000u : 0u);
-                    vmask_hi = (k0 + 8 < valid ? 0x0000ffffu : 0u) |
-                               (k0 + 9 < valid ? 0xffff0000u : 0u);
-                }
+                m_run = m_new;
 #pragma unroll
-                for (int c = 0; c < NT; c += 2) {
-                    const int tok = ri + ((mi & 1) << 3);
-                    const int ch = c + (mi >> 1);
-                    uint32_t v0, v1, v2, v3;
-                    ldsm_x4_trans(vbase + chunk_offset<bf16, D>(tok, ch), v0, v1, v2, v3);
-                    mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
-                    mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
+                for (int u = 0; u < PPW; ++u) {
+                    // P of page u as the A operand of the output MMA: two-term bf16 split
+                    uint32_t pa[4];
+                    {
+                        const float(&p0)[2] = pr[2 * u];
+                        const float(&p1)[2] = pr[2 * u + 1];
+                        const uint32_t hi0 = pack_bf16(p0[0], p0[1]);
+                        const uint32_t hi1 = pack_bf16(p1[0], p1[1]);
+                        const uint32_t lo0 = pack_bf16(p0[0] - bf16lo(hi0), p0[1] - bf16hi(hi0));
+                        const uint32_t lo1 = pack_bf16(p1[0] - bf16lo(hi1), p1[1] - bf16hi(hi1));
+                        if (G == 8) {
+                            pa[0] = hi0;
+                            pa[1] = lo0;
+                            pa[2] = hi1;
+                            pa[3] = lo1;
+                        } else {
+                            pa[0] = row_used ? (row_is_lo ? lo0 : hi0) : 0u;
+                            pa[2] = row_used ? (row_is_lo ? lo1 : hi1) : 0u;
+                            pa[1] = 0u;
+                            pa[3] = 0u;
+                        }
+                    }
+                    // O += P V over the page's 16 tokens (rows past `valid` are zeroed:
+                    // they may hold stale or never-written shared memory)
+                    uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
+                    if (valid[u] < kPageRows) {
+                        const int k0 = 2 * cq, vu = valid[u];
+                        vmask_lo = (k0 < vu ? 0x0000ffffu : 0u) | (k0 + 1 < vu ? 0xffff0000u : 0u);
+                        vmask_hi = (k0 + 8 < vu ? 0x0000ffffu : 0u) |
+                                   (k0 + 9 < vu ? 0xffff0000u : 0u);
+                    }
+#pragma unroll
+                    for (int c = 0; c < NT; c += 2) {
+                        const int tok = ri + ((mi & 1) << 3);
+                        const int ch = c + (mi >> 1);
+                        uint32_t v0, v1, v2, v3;
+                        ldsm_x4_trans(vbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch), v0,
+                                      v1, v2, v3);
+                        mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
+                        mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
+                    }
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
+            // the item's last stage stays held: its page slots take the merge
+            last = stage;
+            if (s + 1 < nst && lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == L::STAGES) {
                 stage = 0;
                 phase ^= 1;
@@ -699,9 +849,8 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
         float lsum = l_run;
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-        float* mb = merge + mbuf * L::MERGE_FLOATS;
         if (r < G) {
-            float* row = mb + (warp * G + r) * (D + 2);
+            float* row = merge_row<bf16, D, G>(base, last, warp, r);
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 row[n * 8 + 2 * cq] = of[n][0];
@@ -712,6 +861,9 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
                 row[D + 1] = lsum;
             }
         }
+        // the rows (generic-proxy writes) precede the TMA writes that refill
+        // the stage after its release
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         // every consumer thread arrives once its rows are written; bounded wait
         mbar_arrive(merge_bar);
         if (!mbar_wait(merge_bar, mphase)) {
@@ -720,8 +872,9 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
             return;
         }
         mphase ^= 1;
-        merge_and_store<D, G>(p, it, mb);
-        mbuf ^= 1;
+        merge_and_store<bf16, D, G>(p, it, base, last);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[last]);
     }
 }
 
@@ -743,8 +896,6 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
 
     int stage = 0;
     uint32_t phase = 0, mphase = 0;
-    int mbuf = 0;
-    float* merge = reinterpret_cast<float*>(base + L::OFF_MERGE);
 
     auto load16 = [&](uint32_t addr, float (&f)[EPL]) {
         uint32_t w0, w1, w2, w3;
@@ -764,7 +915,16 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
     // fused step: the item's rope table, staged by the producer with its first stage
     const float* tab = nullptr;
 
-    for (int item = blockIdx.x; item < W; item += gridDim.x) {
+    const int* s_item = reinterpret_cast<const int*>(base + L::OFF_ITEM);
+    for (;;) {
+        // the item's first stage says which item it is (-1: no more work)
+        if (!mbar_wait(&full[stage], phase) || *s_abort) {
+            *s_abort = 1;
+            if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
+            return;
+        }
+        const int item = s_item[stage];
+        if (item < 0) return;
         const Item it = decode_item(item, p, s_len, s_pre);
         float qf[G][EPL], o[G][EPL], m[G], l[G];
 #pragma unroll
@@ -774,10 +934,11 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
 #pragma unroll
             for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
         }
-        const int nst = (it.npages + NW - 1) / NW;
+        const int nst = (it.npages + L::STAGE_PAGES - 1) / L::STAGE_PAGES;
         bool ok = true;
+        int last = stage;
         for (int s = 0; s < nst; ++s) {
-            ok = mbar_wait(&full[stage], phase) && !*s_abort;
+            ok = (s == 0 || mbar_wait(&full[stage], phase)) && !*s_abort;
             if (!ok) break;
             if (s == 0) {
                 tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
@@ -797,12 +958,15 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
                     for (int g = 0; g < G; ++g) load16(qs + g * D * (int)sizeof(T) + c * 16, qf[g]);
                 }
             }
-            const int j = s * NW + warp;
-            if (j < it.npages && ((masks[stage] >> warp) & 1u)) {
+#pragma unroll 1
+            for (int u = 0; u < L::PPW; ++u) {
+            const int slot = warp * L::PPW + u;
+            const int j = s * L::STAGE_PAGES + slot;
+            if (j < it.npages && ((masks[stage] >> slot) & 1u)) {
                 const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
-                item_patch_page<T, D, G, FUSED>(p, it, j, stage, base);
-                const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + warp * L::PAGE_BYTES);
-                const uint32_t vbase = kbase + NW * L::PAGE_BYTES;
+                item_patch_page<T, D, G, FUSED>(p, it, j, slot, stage, base);
+                const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + slot * L::PAGE_BYTES);
+                const uint32_t vbase = kbase + L::STAGE_PAGES * L::PAGE_BYTES;
 #pragma unroll 2
                 for (int ps = 0; ps < PASSES; ++ps) {
                     const int tk = ps * TPW + tg;
@@ -838,8 +1002,11 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
                     }
                 }
             }
+            }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
+            // the item's last stage stays held: its page slots take the merge
+            last = stage;
+            if (s + 1 < nst && lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == L::STAGES) {
                 stage = 0;
                 phase ^= 1;
@@ -869,11 +1036,10 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
                 m[g] = M;
             }
         }
-        float* mb = merge + mbuf * L::MERGE_FLOATS;
         if (tg == 0) {
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float* row = mb + (warp * G + g) * (D + 2);
+                float* row = merge_row<T, D, G>(base, last, warp, g);
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) row[c * EPL + e] = o[g][e];
                 if (c == 0) {
@@ -882,6 +1048,9 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
                 }
             }
         }
+        // the rows (generic-proxy writes) precede the TMA writes that refill
+        // the stage after its release
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         // every consumer thread arrives once its rows are written; bounded wait
         mbar_arrive(merge_bar);
         if (!mbar_wait(merge_bar, mphase)) {
@@ -890,8 +1059,9 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
             return;
         }
         mphase ^= 1;
-        merge_and_store<D, G>(p, it, mb);
-        mbuf ^= 1;
+        merge_and_store<T, D, G>(p, it, base, last);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[last]);
     }
 }
 
@@ -942,15 +1112,27 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     grid_dependency_wait();
     grid_launch_dependents();
 
-    // Warm L2 with the block-table entries of this CTA's first item, guessed
-    // as if every sequence had NP partitions (exact for uniform batches; a
-    // wrong guess only costs a prefetch), while the lengths are scanned.
-    if (warp == NW && lane < 2) {
+    // The producer starts the reads of its first item's block-table entries
+    // (and, in the fused step, of the new token's slot and position) on a
+    // guess, so that they overlap the scan of the context lengths below.
+    FirstItemGuess<D> guess;
+    if (warp == NW) {
         const int j = blockIdx.x / p.Hkv;
         const int bs = j / p.NP, ps = j - (j / p.NP) * p.NP;
-        const int jb = ps * (p.P / kPageRows) + lane * 31;
-        if (bs < p.B && jb < p.MB)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.block_tables + (size_t)bs * p.MB + jb));
+        if (bs < p.B) {
+            const int jb = ps * (p.P / kPageRows) + lane;
+            guess.b = bs;
+            guess.part = ps;
+            guess.ent = jb < p.MB ? p.block_tables[(size_t)bs * p.MB + jb] : -1;
+            if constexpr (FUSED) {
+                guess.slot = p.slot_mapping[bs];
+                guess.pos = p.positions[bs];
+            }
+        }
+        if constexpr (FUSED) {
+#pragma unroll
+            for (int u = 0; u < (D + 63) / 64; ++u) guess.f[u] = fr.f[(lane + 32 * u) % 64];
+        }
     }
 
     // Partition counts per sequence and their exclusive prefix (block scan).
@@ -990,7 +1172,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     const int W = s_pre[B] * p.Hkv;
 
     if (warp == NW) {
-        run_producer<T, D, G, FUSED>(p, fr, &tm_k, &tm_v, base, full, empty, masks, s_abort,
+        run_producer<T, D, G, FUSED>(p, guess, &tm_k, &tm_v, base, full, empty, masks, s_abort,
                                      s_len, s_pre, W);
         return;
     }
@@ -1208,6 +1390,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     p.out = a.out;
     p.part_o = a.part_o;
     p.part_ml = a.part_ml;
+    p.sched = a.sched;
     p.err = a.device_error;
     p.B = (int)a.B;
     p.Hq = (int)a.Hq;

@@ -140,9 +140,14 @@ int32_t auto_partition(int64_t B, int64_t Hkv, int64_t D, int64_t MB, int32_t kv
     return (int32_t)P;
 }
 
+// Workspace: [scheduler counters, kSchedBytes][partial outputs][partial (m, l)].
+// The counters must be zero before the first launch; every launch leaves them zero.
+constexpr size_t kSchedBytes = 256;
+
 struct WorkspacePlan {
     int32_t P;
     int32_t NP;
+    size_t off_o;
     size_t off_ml;
     size_t bytes;
 };
@@ -165,13 +170,14 @@ pkv_status plan_workspace(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t
     }
     out->P = P;
     out->NP = (int32_t)NP;
+    out->off_o = kSchedBytes;
     if (NP <= 1) {
-        out->off_ml = 0;
-        out->bytes = 0;
+        out->off_ml = kSchedBytes;
+        out->bytes = kSchedBytes;
         return PKV_OK;
     }
     const size_t slots = (size_t)B * Hq * NP;
-    out->off_ml = align_up(slots * D * sizeof(float));
+    out->off_ml = out->off_o + align_up(slots * D * sizeof(float));
     out->bytes = out->off_ml + align_up(slots * 2 * sizeof(float));
     return PKV_OK;
 }
@@ -352,9 +358,12 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
         set_last_error("misaligned tensor pointer (16 bytes for q/k/v/caches/out)");
         return PKV_ERR_INVALID_ARG;
     }
-    if (workspace_bytes < w.bytes || (w.bytes > 0 && (!workspace || !aligned16(workspace)))) {
+    // With one partition per sequence the workspace is optional: without it
+    // the work items are dealt out statically instead of claimed.
+    const bool have_ws = workspace && workspace_bytes >= w.bytes;
+    if ((w.NP > 1 && !have_ws) || (have_ws && !aligned16(workspace))) {
         set_last_error("workspace of %zu bytes given, %zu needed (16-byte aligned)",
-                       workspace_bytes, w.bytes);
+                       workspace ? workspace_bytes : (size_t)0, w.bytes);
         return PKV_ERR_WORKSPACE;
     }
     DecodeArgs a = {};
@@ -364,8 +373,10 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
     a.block_tables = block_tables;
     a.context_lens = context_lens;
     a.out = out;
-    a.part_o = w.bytes ? static_cast<float*>(workspace) : nullptr;
-    a.part_ml = w.bytes ? reinterpret_cast<float*>(static_cast<char*>(workspace) + w.off_ml) : nullptr;
+    char* ws = static_cast<char*>(workspace);
+    a.sched = have_ws ? reinterpret_cast<uint32_t*>(ws) : nullptr;
+    a.part_o = (have_ws && w.NP > 1) ? reinterpret_cast<float*>(ws + w.off_o) : nullptr;
+    a.part_ml = (have_ws && w.NP > 1) ? reinterpret_cast<float*>(ws + w.off_ml) : nullptr;
     a.B = num_seqs;
     a.Hq = num_q_heads;
     a.Hkv = num_kv_heads;

@@ -42,6 +42,7 @@ struct DecodeArgs {
     void* out;
     float* part_o;   // [B, Hq, NP, D]
     float* part_ml;  // [B, Hq, NP, 2]
+    uint32_t* sched; // scheduler counters (2 x u32, zero between launches); null: static
     int64_t B, Hq, Hkv, D, num_blocks, MB;
     int32_t kv_dtype, out_dtype;
     int32_t partition_tokens;  // P (resolved, multiple of 16)

@@ -108,6 +108,8 @@ def test_kv_append_rejects_bad_arguments(lib, kw, status):
     (dict(bt=FAKE + 2), INVALID),
     (dict(MB=0), INVALID),
     (dict(P=16, MB=4), WORKSPACE),         # split path needs a workspace
+    (dict(P=16, MB=4, ws=FAKE, wsb=255), WORKSPACE),   # smaller than the plan
+    (dict(P=16, MB=4, ws=FAKE + 4, wsb=1 << 20), WORKSPACE),   # misaligned
     (dict(B=0, q=None, out=None), OK),
 ])
 def test_decode_rejects_bad_arguments(lib, kw, status):
@@ -120,9 +122,10 @@ def test_workspace_size_formula(lib):
     NP = math.ceil(8193 * 16 / 1024)
     slots = 16 * 32 * NP
     a = lambda x: (x + 255) // 256 * 256
-    assert n == a(slots * 128 * 4) + a(slots * 2 * 4)
-    # a single partition needs no workspace
-    assert lib.pkv_decode_workspace_size(4, 8, 2, 64, 4, 16, BF16, 64) == 0
+    # 256 bytes of scheduler counters, then the partial outputs and (m, l) pairs
+    assert n == 256 + a(slots * 128 * 4) + a(slots * 2 * 4)
+    # a single partition needs the counters only
+    assert lib.pkv_decode_workspace_size(4, 8, 2, 64, 4, 16, BF16, 64) == 256
     assert lib.pkv_decode_workspace_size(4, 8, 2, 64, 4, 16, BF16, 24) == 0  # invalid P -> 0
 
 

@@ -260,3 +260,66 @@ def test_fused_step_edge_cases():
     so3 = int(sub.slots[3])
     check_within_one_bf16_ulp(w.k_cache[s3 // bs, :, s3 % bs].cpu(), kc_or[so3 // bs, :, so3 % bs],
                               "appended k of the empty context")
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "one_launch"])
+def test_claimed_work_items_repeat_exactly(fused):
+    """CTAs claim work items from the workspace's counters: three calls that
+    share one workspace give bit-identical outputs (an item's arithmetic does
+    not depend on which CTA runs it), match the oracle, and leave the
+    counters at zero after every call."""
+    lens = [4000, 130, 2500, 17, 3333, 900, 64, 1, 4095, 2048] * 6
+    w = W.build_workload("claims", lens, 32, 8, 64, torch.bfloat16, 5e5, seed=53, device=DEV)
+    seqs = [0, 3, 7, 8, 59]
+    sub = SubProblem(w, seqs)
+    _, _, _, ref = sub.oracle_step()
+    P = 128
+    need = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, partition_tokens=P)
+    ws = pkv.new_workspace(need, DEV)
+    k0, v0 = w.k_cache.clone(), w.v_cache.clone()
+    outs = []
+    for _ in range(3):
+        w.k_cache.copy_(k0)
+        w.v_cache.copy_(v0)
+        q = w.q.clone()
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=DEV)
+        if fused:
+            pkv.decode_step(q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                            w.v_cache, w.block_tables, w.decode_lens, w.rope_theta, w.scale, out,
+                            workspace=ws, partition_tokens=P)
+        else:
+            pkv.kv_append(q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                          w.v_cache, w.rope_theta)
+            pkv.paged_attention_decode(q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
+                                       w.scale, out, workspace=ws, partition_tokens=P)
+        torch.cuda.synchronize()
+        assert not ws[:pkv.SCHED_BYTES].any(), "scheduler counters not back at zero"
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    check_decode(outs[0].cpu()[torch.tensor(seqs)], ref, torch.bfloat16, "claimed items")
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "one_launch"])
+def test_static_schedule_without_workspace(fused):
+    """No workspace (allowed when no context is split): items are dealt out
+    round-robin; same results as the oracle."""
+    lens = [700, 1, 0, 512, 33, 1000, 999, 16]
+    w = W.build_workload("static", lens, 16, 4, 128, torch.bfloat16, 1e4, seed=59, device=DEV)
+    sub = SubProblem(w, list(range(w.B)))
+    q_or, _, _, ref = sub.oracle_step()
+    P = 1024
+    assert pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks,
+                                     partition_tokens=P) == pkv.SCHED_BYTES
+    none = torch.empty(0, dtype=torch.uint8, device=DEV)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=DEV)
+    if fused:
+        pkv.decode_step(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
+                        w.block_tables, w.decode_lens, w.rope_theta, w.scale, out,
+                        workspace=none, partition_tokens=P)
+    else:
+        pkv.kv_append(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
+                      w.rope_theta)
+        pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
+                                   w.scale, out, workspace=none, partition_tokens=P)
+    torch.cuda.synchronize()
+    check_decode(out.cpu(), ref, torch.bfloat16, "static schedule")
