@@ -1503,14 +1503,21 @@ int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_
     size_t smem = 0;
     const int B = (int)num_seqs;
     auto pick = [&](auto tag) { smem = decltype(tag)::smem_bytes(B); };
+    auto by_g = [&](auto t, auto d) {
+        using T = decltype(t);
+        constexpr int Dv = decltype(d)::value;
+        if (G <= 1) pick(Layout<T, Dv, 1>{});
+        else if (G == 2) pick(Layout<T, Dv, 2>{});
+        else if (G == 4) pick(Layout<T, Dv, 4>{});
+        else pick(Layout<T, Dv, 8>{});
+    };
     if (kv_dtype == PKV_DTYPE_F32) {
-        if (D == 64) pick(Layout<float, 64, 8>{});
-        else pick(Layout<float, 128, 8>{});
+        if (D == 64) by_g(float{}, std::integral_constant<int, 64>{});
+        else by_g(float{}, std::integral_constant<int, 128>{});
     } else {
-        if (D == 64) pick(Layout<bf16, 64, 8>{});
-        else pick(Layout<bf16, 128, 8>{});
+        if (D == 64) by_g(bf16{}, std::integral_constant<int, 64>{});
+        else by_g(bf16{}, std::integral_constant<int, 128>{});
     }
-    (void)G;
     (void)simt;
     const size_t per_sm = 228 * 1024;
     int n = (int)(per_sm / (smem + 1024));

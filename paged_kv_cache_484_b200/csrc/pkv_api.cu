@@ -125,16 +125,23 @@ pkv_status check_heads(int64_t Hq, int64_t Hkv, int64_t D, int64_t bs) {
 
 bool valid_dtype(int32_t t) { return t == PKV_DTYPE_F32 || t == PKV_DTYPE_BF16; }
 
-// Partition length: aim for ~16 items per resident CTA if every sequence had
-// the maximum length, in whole stages (64 tokens), at most 1024 tokens, and
-// never more than kMaxPartitions partitions.
-int32_t auto_partition(int64_t B, int64_t Hkv, int64_t D, int64_t MB, int32_t kv_dtype) {
+// Partition length.  A partition should fill whole stages of the ring and be
+// long enough that the per-item work (q fragments, merge, partial store)
+// stays small next to the streaming: at least 128 tokens (one stage of the
+// two-page-per-warp path), and 1024 once there is work for about two items
+// per resident CTA even at that length.  Between the two, the length that
+// gives about two items per resident CTA if every sequence had the maximum
+// length.  Never more than kMaxPartitions partitions.
+int32_t auto_partition(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t MB,
+                       int32_t kv_dtype) {
     const int64_t maxlen = MB * kPageRows;
-    const int64_t resident = (int64_t)device_sm_count() * decode_ctas_per_sm(D, 0, kv_dtype, false, B);
-    const int64_t target_items = 16 * resident;
+    const int64_t G = Hq / std::max<int64_t>(1, Hkv);
+    const int64_t resident =
+        (int64_t)device_sm_count() * decode_ctas_per_sm(D, G, kv_dtype, false, B);
+    const int64_t target_items = 2 * resident;
     int64_t P = ceil_div(std::max<int64_t>(1, maxlen * B * Hkv), target_items);
-    P = ceil_div(P, kStageTokens) * kStageTokens;
-    P = std::max<int64_t>(kStageTokens, std::min<int64_t>(P, 1024));
+    P = ceil_div(P, 128) * 128;
+    P = std::max<int64_t>(128, std::min<int64_t>(P, 1024));
     const int64_t floor_np = ceil_div(ceil_div(maxlen, kMaxPartitions), kStageTokens) * kStageTokens;
     P = std::max(P, floor_np);
     return (int32_t)P;
@@ -156,7 +163,7 @@ pkv_status plan_workspace(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t
                           int32_t kv_dtype, int32_t partition_tokens, WorkspacePlan* out) {
     int32_t P = partition_tokens;
     if (P == 0) {
-        P = auto_partition(B, Hkv, D, MB, kv_dtype);
+        P = auto_partition(B, Hq, Hkv, D, MB, kv_dtype);
     } else if (P < kPageRows || P % kPageRows != 0 || P > PKV_MAX_PARTITION_TOKENS) {
         set_last_error("partition_tokens %d must be a multiple of 16 in [16, %d]", P,
                        PKV_MAX_PARTITION_TOKENS);
