@@ -58,6 +58,10 @@ namespace {
 using bf16 = __nv_bfloat16;
 constexpr int NW = kConsumerWarps;
 constexpr float kNegInf = -__builtin_huge_valf();
+// Batches of at most this many sequences hand out every sequence's last
+// (shortest) partition after all full ones, longest first, so that the
+// work that finishes last is short.
+constexpr int kLptMaxSeqs = 256;
 
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
@@ -99,8 +103,12 @@ struct Layout {
     static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
     static constexpr int OFF_ITEM = OFF_PATCH + STAGES * 8;  // work item of each stage, -1: no more
     static constexpr int OFF_MISC = OFF_ITEM + STAGES * 4;   // abort flag + 8 scan slots
-    static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;        // s_len[B], s_pre[B + 1]
-    static size_t smem_bytes(int B) { return 1024 + OFF_SEQ + (size_t)(2 * B + 1) * 4; }
+    // s_len[B], s_pre[B + 1]; with at most kLptMaxSeqs sequences also
+    // s_rank[B], s_key[B] (the longest-first order of last partitions)
+    static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;
+    static size_t smem_bytes(int B) {
+        return 1024 + OFF_SEQ + (size_t)(2 * B + 1) * 4 + (B <= kLptMaxSeqs ? (size_t)2 * B * 4 : 0);
+    }
 };
 
 struct DecodeParams {
@@ -135,22 +143,35 @@ struct Item {
     int b, h, part, t0, t1, npages, np;
 };
 
+// Item i -> (sequence, kv head, partition).  Items are j * Hkv + h.  Without
+// the longest-first order, j runs over every sequence's partitions in order
+// (s_pre: exclusive prefix of partition counts).  With it (p.B <=
+// kLptMaxSeqs), j < s_pre[B] runs over the partitions before each sequence's
+// last one, and j >= s_pre[B] over the last partitions in the order s_rank.
 __device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const int* s_len,
                                             const int* s_pre) {
     Item it;
     const int j = i / p.Hkv;
     it.h = i - j * p.Hkv;
-    int lo = 0, hi = p.B - 1;  // largest b with s_pre[b] <= j
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_pre[mid] <= j) lo = mid;
-        else hi = mid - 1;
+    const int nfull = s_pre[p.B];
+    if (p.B <= kLptMaxSeqs && j >= nfull) {
+        const int* s_rank = s_pre + p.B + 1;
+        it.b = s_rank[j - nfull];
+        it.np = (s_len[it.b] + p.P - 1) / p.P;
+        it.part = it.np - 1;
+    } else {
+        int lo = 0, hi = p.B - 1;  // largest b with s_pre[b] <= j
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_pre[mid] <= j) lo = mid;
+            else hi = mid - 1;
+        }
+        it.b = lo;
+        it.part = j - s_pre[lo];
+        it.np = (s_len[lo] + p.P - 1) / p.P;
     }
-    it.b = lo;
-    it.part = j - s_pre[lo];
-    it.np = s_pre[lo + 1] - s_pre[lo];
     it.t0 = it.part * p.P;
-    it.t1 = min(s_len[lo], it.t0 + p.P);
+    it.t1 = min(s_len[it.b], it.t0 + p.P);
     it.npages = (it.t1 - it.t0 + kPageRows - 1) / kPageRows;
     return it;
 }
@@ -1117,8 +1138,22 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     // guess, so that they overlap the scan of the context lengths below.
     FirstItemGuess<D> guess;
     if (warp == NW) {
+        // every sequence at the maximum length: NP partitions each
         const int j = blockIdx.x / p.Hkv;
-        const int bs = j / p.NP, ps = j - (j / p.NP) * p.NP;
+        int bs, ps;
+        if (p.B <= kLptMaxSeqs) {
+            const int nf = p.NP - 1;  // full partitions per sequence, then the last ones
+            if (j < p.B * nf) {
+                bs = j / nf;
+                ps = j - bs * nf;
+            } else {
+                bs = j - p.B * nf;
+                ps = nf;
+            }
+        } else {
+            bs = j / p.NP;
+            ps = j - bs * p.NP;
+        }
         if (bs < p.B) {
             const int jb = ps * (p.P / kPageRows) + lane;
             guess.b = bs;
@@ -1135,11 +1170,15 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         }
     }
 
-    // Partition counts per sequence and their exclusive prefix (block scan).
+    // Partition counts per sequence and their exclusive prefix (block scan);
+    // in the longest-first order only the partitions before the last one.
     const int B = p.B;
+    const bool lpt = B <= kLptMaxSeqs;
     const int maxlen = p.MB * kPageRows;
     const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
     const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
+    int* s_rank = s_pre + B + 1;
+    int* s_key = s_rank + B;
     int local = 0;
     for (int b = b0; b < b1; ++b) {
         int Lb = p.context_lens[b];
@@ -1149,8 +1188,10 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         }
         s_len[b] = Lb;
         const int npb = (Lb + p.P - 1) / p.P;
-        s_pre[b] = npb;
-        local += npb;
+        const int cnt = lpt ? max(npb - 1, 0) : npb;
+        if (lpt) s_key[b] = Lb > 0 ? Lb - (npb - 1) * p.P : -1;  // tokens of the last partition
+        s_pre[b] = cnt;
+        local += cnt;
     }
     int incl = local;
 #pragma unroll
@@ -1168,8 +1209,27 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         run += cnt;
     }
     if (tid == kDecodeThreads - 1) s_pre[B] = run;
+    if (lpt) {
+        // rank of each last partition: longer first, then by sequence
+        // (every CTA derives the same order)
+        for (int b = b0; b < b1; ++b) {
+            const int k = s_key[b];
+            if (k < 0) continue;
+            int rank = 0;
+            for (int b2 = 0; b2 < B; ++b2) {
+                const int k2 = s_key[b2];
+                rank += (k2 > k) || (k2 == k && b2 < b);
+            }
+            s_rank[rank] = b;
+        }
+        if (tid == 0) {
+            int ne = 0;
+            for (int b2 = 0; b2 < B; ++b2) ne += s_key[b2] >= 0;
+            s_warp_tot[7] = ne;
+        }
+    }
     __syncthreads();
-    const int W = s_pre[B] * p.Hkv;
+    const int W = (s_pre[B] + (lpt ? s_warp_tot[7] : 0)) * p.Hkv;
 
     if (warp == NW) {
         run_producer<T, D, G, FUSED>(p, guess, &tm_k, &tm_v, base, full, empty, masks, s_abort,
@@ -1224,6 +1284,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_c
     float4* red = smem4;                                        // [G][PG][CH]
     float* w = reinterpret_cast<float*>(smem4 + G * PG * CH);   // [G][NP]
     grid_dependency_wait();
+    // the next launch (the next step's decode) may start its prologue now;
+    // its own wait still orders it after this grid's writes
+    grid_launch_dependents();
     const int b = blockIdx.y, h = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t hq0 = (size_t)b * p.Hq + (size_t)h * G;
