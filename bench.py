@@ -58,6 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--copies", type=int, default=0,
+                    help="device-side copies of the workload (0: enough to exceed L2)")
     ap.add_argument("--simt", action="store_true", help="bf16: CUDA-core decode kernel")
     ap.add_argument("--two-calls", action="store_true",
                     help="time kv_append + paged_attention_decode as two launches instead of "
@@ -331,6 +333,8 @@ def run_ours(args):
     # a step reads or writes), step k on copy k mod n.
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     ncopies = 1 if nbytes >= 2 * l2 else min(1024, math.ceil(2 * l2 / nbytes))
+    if args.copies:
+        ncopies = args.copies
     fields = ("q", "k_new", "v_new", "positions", "slot_mapping", "k_cache", "v_cache",
               "block_tables", "decode_lens")
     copies = [dict((f, getattr(w, f)) for f in fields)]
@@ -339,7 +343,13 @@ def run_ours(args):
     outs = [torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=device) for _ in range(ncopies)]
 
     fused = not args.two_calls
-    kernels_per_decode = 1 + (1 if NP > 1 else 0)      # decode (+ split-context combine)
+    # decode kernel, plus the partition combine unless the split contexts
+    # are merged inside thread-block clusters (the library decides)
+    kernels_per_decode = pkv.decode_launches(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=w.dtype,
+                                             out_dtype=out_dtype, partition_tokens=P,
+                                             force_simt=args.simt, fused=fused)
+    if kernels_per_decode not in (1, 2):
+        raise SystemExit("decode_launches: no answer from the library")
     launches_per_step = kernels_per_decode + (0 if fused else 1)
 
     def append(c):
@@ -513,7 +523,9 @@ def run_ours(args):
                                  "pair of events"},
         "roofline": {"bound": "hbm",
                      "kernel": ("decode_step" if fused else "paged_attention_decode")
-                     + " call: paged_decode_kernel" + (" + combine_kernel" if NP > 1 else ""),
+                     + " call: paged_decode_kernel" + (" + combine_kernel" if kernels_per_decode == 2
+                                                        else (" (partitions merged in thread-block "
+                                                              "clusters)" if NP > 1 else "")),
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "decode_ms": round(decode_ms_max, 5),

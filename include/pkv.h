@@ -95,6 +95,8 @@ typedef enum pkv_dtype {
 /* Decode flags. */
 #define PKV_DECODE_FORCE_SIMT 0x1u  /* bf16: use the CUDA-core kernel instead of the
                                        tensor-core one (same result within tolerance) */
+#define PKV_DECODE_NO_CLUSTER 0x2u  /* never merge split contexts inside a thread-block
+                                       cluster; always partials + combine kernel */
 
 /* Upper limits of one call. */
 #define PKV_MAX_SEQS_PER_CALL 4096
@@ -161,6 +163,20 @@ size_t pkv_decode_workspace_size(int64_t num_seqs, int64_t num_q_heads, int64_t 
                                  int64_t block_size, int32_t kv_dtype, int32_t partition_tokens);
 
 /*
+ * pkv_decode_launches -- how many kernels a decode call with these shapes
+ * makes on the current device: 1 (one decode kernel: no context split, or
+ * split contexts merged inside thread-block clusters) or 2 (the decode
+ * kernel and the partition-combine kernel).  fused != 0 asks about
+ * pkv_decode_step, 0 about pkv_paged_attention_decode.  Queries the current
+ * device's occupancy limits (cached); launches nothing.  Returns 0 for
+ * invalid arguments or when no device answers.
+ */
+int32_t pkv_decode_launches(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                            int64_t head_dim, int64_t max_blocks_per_seq, int64_t block_size,
+                            int32_t kv_dtype, int32_t out_dtype, int32_t partition_tokens,
+                            uint32_t flags, int32_t fused);
+
+/*
  * pkv_decode_partition_tokens -- the partition length P (tokens, a multiple of
  * block_size) that a decode call with these shapes uses when its
  * partition_tokens argument is 0.  Host only.  Returns 0 for invalid
@@ -205,7 +221,14 @@ int32_t pkv_decode_partition_tokens(int64_t num_seqs, int64_t num_q_heads, int64
  *                 into ceil(L / P) partitions that run in parallel and are
  *                 merged by a log-sum-exp combine (any P gives the same
  *                 result up to rounding)
- *   flags         0 or PKV_DECODE_FORCE_SIMT
+ *   flags         0, or PKV_DECODE_FORCE_SIMT and/or PKV_DECODE_NO_CLUSTER.
+ *                 When contexts are split into 2..16 partitions and every
+ *                 (sequence, kv head) can have its own cluster of that many
+ *                 CTAs resident at once (small batches), the partitions of a
+ *                 (sequence, kv head) run as one thread-block cluster and are
+ *                 merged through distributed shared memory, without the
+ *                 workspace partials and the combine kernel (same result
+ *                 within tolerance); PKV_DECODE_NO_CLUSTER turns that off
  *   device_error  device int32 or NULL
  *   stream        cudaStream_t
  * num_seqs == 0 returns PKV_OK and launches nothing; num_seqs is at most

@@ -23,6 +23,7 @@ from ._binding import (  # noqa: F401
     NOALLOC_SCRATCH_BYTES,
     PkvError,
     SCHED_BYTES,
+    decode_launches,
     decode_partition_tokens,
     decode_step,
     decode_workspace_size,

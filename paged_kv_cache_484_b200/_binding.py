@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libpkv.so")
 PKV_DTYPE_F32 = 0
 PKV_DTYPE_BF16 = 1
 PKV_DECODE_FORCE_SIMT = 0x1
+PKV_DECODE_NO_CLUSTER = 0x2
 DEVERR_SLOT = 0x1
 DEVERR_BLOCK_ID = 0x2
 DEVERR_CONTEXT_LEN = 0x4
@@ -55,6 +56,8 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_kv_append.restype = ctypes.c_int
         lib.pkv_decode_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32]
         lib.pkv_decode_workspace_size.restype = ctypes.c_size_t
+        lib.pkv_decode_launches.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32, i32, u32, i32]
+        lib.pkv_decode_launches.restype = i32
         lib.pkv_decode_partition_tokens.argtypes = [i64, i64, i64, i64, i64, i64, i32]
         lib.pkv_decode_partition_tokens.restype = i32
         lib.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
@@ -106,6 +109,10 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     return t.data_ptr()
+
+
+def _flags(force_simt: bool, cluster: bool) -> int:
+    return (PKV_DECODE_FORCE_SIMT if force_simt else 0) | (0 if cluster else PKV_DECODE_NO_CLUSTER)
 
 
 def _stream_ptr(stream, device) -> int:
@@ -162,6 +169,19 @@ def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blo
                                              _dtype_code(kv_dtype), int(partition_tokens)))
 
 
+def decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                    kv_dtype=torch.bfloat16, out_dtype=torch.bfloat16, partition_tokens=0,
+                    force_simt=False, cluster=True, fused=False, block_size=BLOCK_SIZE) -> int:
+    """Kernels one decode call with these shapes launches on the current
+    device: 1 (no split, or split contexts merged inside thread-block
+    clusters) or 2 (decode + partition combine); 0 for invalid arguments."""
+    lib = load_library()
+    return int(lib.pkv_decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                       max_blocks_per_seq, block_size, _dtype_code(kv_dtype),
+                                       _dtype_code(out_dtype), int(partition_tokens),
+                                       _flags(force_simt, cluster), 1 if fused else 0))
+
+
 SCHED_BYTES = 256  # scheduler counters at the head of a decode workspace
 
 
@@ -176,7 +196,7 @@ def new_workspace(nbytes, device) -> torch.Tensor:
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out,
                            stream=None, *, workspace=None, partition_tokens=0, force_simt=False,
-                           device_error=None) -> torch.Tensor:
+                           device_error=None, cluster=True) -> torch.Tensor:
     """Single-query attention over the paged cache; writes and returns ``out``.
 
     q [B, Hq, d] and caches [NB, Hkv, 16, d] share a dtype (float32 or
@@ -208,14 +228,15 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale), int(partition_tokens),
-        PKV_DECODE_FORCE_SIMT if force_simt else 0, err, _stream_ptr(stream, q.device))
+        _flags(force_simt, cluster), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode")
     return out
 
 
 def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
                 context_lens, rope_theta, scale, out, stream=None, *, workspace=None,
-                partition_tokens=0, force_simt=False, device_error=None) -> torch.Tensor:
+                partition_tokens=0, force_simt=False, device_error=None,
+                cluster=True) -> torch.Tensor:
     """``kv_append`` (one new token per sequence) then ``paged_attention_decode``,
     in one launch.  The new token must be the last token of its context
     (context_lens[b] - 1, at the slot block_tables gives it).  q is read only:
@@ -247,7 +268,7 @@ def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, bloc
         _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(rope_theta), float(scale),
-        int(partition_tokens), PKV_DECODE_FORCE_SIMT if force_simt else 0, err,
+        int(partition_tokens), _flags(force_simt, cluster), err,
         _stream_ptr(stream, q.device))
     _raise(st, lib, "decode_step")
     return out
@@ -255,7 +276,7 @@ def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, bloc
 
 def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, out,
                                    stream=None, *, partition_tokens=0, force_simt=False,
-                                   device_error=None) -> torch.Tensor:
+                                   device_error=None, cluster=True) -> torch.Tensor:
     """``paged_attention_decode`` for callers that cannot allocate device memory.
 
     Same arguments and result, but no workspace: the split-context scratch is
@@ -280,7 +301,7 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
         B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(scale),
-        int(partition_tokens), PKV_DECODE_FORCE_SIMT if force_simt else 0, err,
+        int(partition_tokens), _flags(force_simt, cluster), err,
         _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode_noalloc")
     return out

@@ -44,6 +44,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -100,6 +101,10 @@ struct Layout {
     static constexpr int OFF_ROPE = OFF_NEWKV + STAGES * NEWKV_BYTES;
     static constexpr int OFF_BAR = OFF_ROPE + STAGES * ROPE_BYTES;
     static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
+    // Cluster mode: the CTA's merged partial (o[D], m, l per head) sits in the
+    // q / new-row / rope-table slots once the CTA's one item is done.
+    static constexpr int CLUSTER_PART_BYTES = G * (D + 2) * 4;
+    static_assert(OFF_BAR - OFF_Q >= CLUSTER_PART_BYTES, "cluster partial does not fit");
     static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
     static constexpr int OFF_ITEM = OFF_PATCH + STAGES * 8;  // work item of each stage, -1: no more
     static constexpr int OFF_MISC = OFF_ITEM + STAGES * 4;   // abort flag + 8 scan slots
@@ -126,6 +131,10 @@ struct DecodeParams {
     int num_blocks;
     float scale_log2;
     int out_bf16;
+    // cluster mode: CS > 1 CTAs per (sequence, kv head), CTA rank r takes
+    // partition r, and the cluster merges the partials in shared memory
+    // (no workspace partials, no combine kernel); 0 = off
+    int cluster;
     // fused step only: the new token of every sequence
     const void* k_new;            // [B, Hkv, D]
     const void* v_new;            // [B, Hkv, D]
@@ -154,7 +163,7 @@ __device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const 
     const int j = i / p.Hkv;
     it.h = i - j * p.Hkv;
     const int nfull = s_pre[p.B];
-    if (p.B <= kLptMaxSeqs && j >= nfull) {
+    if (p.B <= kLptMaxSeqs && !p.cluster && j >= nfull) {
         const int* s_rank = s_pre + p.B + 1;
         it.b = s_rank[j - nfull];
         it.np = (s_len[it.b] + p.P - 1) / p.P;
@@ -353,6 +362,15 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
     // claimed is lost.
     int item = blockIdx.x;
     int item1 = item + (int)gridDim.x;  // the item after `item`
+    if (p.cluster) {
+        // cluster mode: CTA rank r of the cluster of (sequence, kv head) takes
+        // partition r, if the sequence has one, and nothing else
+        const int CS = p.cluster, cid = blockIdx.x / CS, rank = blockIdx.x - cid * CS;
+        const int b = cid / p.Hkv, h = cid - b * p.Hkv;
+        const int npb = (s_len[b] + p.P - 1) / p.P;
+        item = rank < npb ? (s_pre[b] + rank) * p.Hkv + h : W;
+        item1 = W;
+    }
     uint32_t pend = 0;                  // lane 0: raw counter value of the claim in flight
     int k_static = 2;
     auto issue_claim = [&]() {
@@ -587,7 +605,15 @@ __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Ite
         const size_t hq = (size_t)it.b * p.Hq + (size_t)it.h * G + g;
         // den == 0 only if every page of the item was rejected (bad block ids)
         const float val = den > 0.f ? num / den : 0.f;
-        if (it.np == 1) {
+        if (p.cluster) {
+            // cluster mode: this CTA's partial, merged across the cluster later
+            float* part = reinterpret_cast<float*>(base + Layout<T, D, G>::OFF_Q) + g * (D + 2);
+            part[dim] = val;
+            if (dim == 0) {
+                part[D] = M;
+                part[D + 1] = den;
+            }
+        } else if (it.np == 1) {
             store_out(p.out, hq * D + dim, val, p.out_bf16);
         } else {
             const size_t slot = hq * p.NP + it.part;
@@ -598,6 +624,54 @@ __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Ite
             }
         }
     }
+}
+
+// Cluster mode, after every CTA of the cluster holds its partial in its own
+// shared memory (an empty one, m = -inf and l = 0, when it had no partition
+// or gave up): CTA rank 0 reads all of them through distributed shared
+// memory and writes out[b, h*G .. h*G+G-1, :], the same log-sum-exp merge as
+// the combine kernel.  Every thread of every CTA of the cluster calls this
+// exactly once (it holds the two cluster barriers).
+template <typename T, int D, int G>
+__device__ void cluster_merge(const DecodeParams& p, uint8_t* base) {
+    using L = Layout<T, D, G>;
+    cluster_sync_all();  // all partials written (release / acquire at cluster scope)
+    const int CS = p.cluster;
+    if (cluster_ctarank() == 0 && threadIdx.x < NW * 32) {
+        const int cid = blockIdx.x / CS;
+        const int b = cid / p.Hkv, h = cid - (cid / p.Hkv) * p.Hkv;
+        const float* part = reinterpret_cast<const float*>(base + L::OFF_Q);
+        for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+            const int g = idx / D, dim = idx - (idx / D) * D;
+            const float* row = part + g * (D + 2);
+            // all remote loads first (independent, so they overlap), then the merge
+            float m[kMaxClusterCtas], l[kMaxClusterCtas], v[kMaxClusterCtas];
+#pragma unroll
+            for (int r = 0; r < kMaxClusterCtas; ++r) {
+                m[r] = kNegInf;
+                l[r] = 0.f;
+                v[r] = 0.f;
+                if (r < CS) {
+                    m[r] = ld_dsmem_f32(dsmem_addr(row + D, r));
+                    l[r] = ld_dsmem_f32(dsmem_addr(row + D + 1, r));
+                    v[r] = ld_dsmem_f32(dsmem_addr(row + dim, r));
+                }
+            }
+            float M = kNegInf;
+#pragma unroll
+            for (int r = 0; r < kMaxClusterCtas; ++r) M = fmaxf(M, m[r]);
+            float num = 0.f, den = 0.f;
+#pragma unroll
+            for (int r = 0; r < kMaxClusterCtas; ++r) {
+                const float w = (m[r] == kNegInf || l[r] == 0.f) ? 0.f : l[r] * fast_exp2(m[r] - M);
+                num = fmaf(w, v[r], num);
+                den += w;
+            }
+            const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
+            store_out(p.out, hq * D + dim, den > 0.f ? num / den : 0.f, p.out_bf16);
+        }
+    }
+    cluster_sync_all();  // no CTA leaves while rank 0 may still read its memory
 }
 
 // Bounded barrier of the consumer warps (every consumer thread arrives).
@@ -636,7 +710,7 @@ __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Ite
 // ------------------------------------------------- tensor-core consumer (bf16)
 
 template <int D, int G, bool FUSED>
-__device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
+__device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
                                  uint64_t* full, uint64_t* empty, uint64_t* merge_bar,
                                  const uint32_t* masks, volatile int* s_abort, const int* s_len,
                                  const int* s_pre, int W) {
@@ -653,6 +727,7 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
     const bool row_is_lo = (G < 8) && (r >= G) && (r < 2 * G);
     const bool row_used = (G == 8) || (r < 2 * G);
 
+    int merged = 0;  // items merged (cluster mode: at most one)
     int stage = 0;
     uint32_t phase = 0, mphase = 0;
     // fused step: the item's rope table, staged by the producer with its first stage
@@ -664,10 +739,10 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
         if (!mbar_wait(&full[stage], phase) || *s_abort) {
             *s_abort = 1;
             if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
-            return;
+            return -1;
         }
         const int item = s_item[stage];
-        if (item < 0) return;
+        if (item < 0) return merged;
         const Item it = decode_item(item, p, s_len, s_pre);
         float o[NT][4];
 #pragma unroll
@@ -852,7 +927,7 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
         if (!ok) {
             *s_abort = 1;
             if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
-            return;
+            return -1;
         }
 
         // per-warp result for each real head: add the low-part rows
@@ -890,10 +965,11 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
         if (!mbar_wait(merge_bar, mphase)) {
             *s_abort = 1;
             report_error(p.err, PKV_DEVERR_TIMEOUT);
-            return;
+            return -1;
         }
         mphase ^= 1;
         merge_and_store<bf16, D, G>(p, it, base, last);
+        ++merged;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[last]);
     }
@@ -902,7 +978,7 @@ __device__ void run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint
 // ------------------------------------------------------- CUDA-core consumer
 
 template <typename T, int D, int G, bool FUSED>
-__device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
+__device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
                                   uint64_t* full, uint64_t* empty, uint64_t* merge_bar,
                                   const uint32_t* masks, volatile int* s_abort, const int* s_len,
                                   const int* s_pre, int W) {
@@ -915,6 +991,7 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = lane % TPL, tg = lane / TPL;
 
+    int merged = 0;  // items merged (cluster mode: at most one)
     int stage = 0;
     uint32_t phase = 0, mphase = 0;
 
@@ -942,10 +1019,10 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
         if (!mbar_wait(&full[stage], phase) || *s_abort) {
             *s_abort = 1;
             if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
-            return;
+            return -1;
         }
         const int item = s_item[stage];
-        if (item < 0) return;
+        if (item < 0) return merged;
         const Item it = decode_item(item, p, s_len, s_pre);
         float qf[G][EPL], o[G][EPL], m[G], l[G];
 #pragma unroll
@@ -1036,7 +1113,7 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
         if (!ok) {
             *s_abort = 1;
             if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
-            return;
+            return -1;
         }
         // merge the token groups of this warp
 #pragma unroll
@@ -1077,10 +1154,11 @@ __device__ void run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uin
         if (!mbar_wait(merge_bar, mphase)) {
             *s_abort = 1;
             report_error(p.err, PKV_DEVERR_TIMEOUT);
-            return;
+            return -1;
         }
         mphase ^= 1;
         merge_and_store<T, D, G>(p, it, base, last);
+        ++merged;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[last]);
     }
@@ -1141,7 +1219,11 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         // every sequence at the maximum length: NP partitions each
         const int j = blockIdx.x / p.Hkv;
         int bs, ps;
-        if (p.B <= kLptMaxSeqs) {
+        if (p.cluster) {
+            const int cid = blockIdx.x / p.cluster;
+            bs = cid / p.Hkv;
+            ps = blockIdx.x - cid * p.cluster;
+        } else if (p.B <= kLptMaxSeqs) {
             const int nf = p.NP - 1;  // full partitions per sequence, then the last ones
             if (j < p.B * nf) {
                 bs = j / nf;
@@ -1173,7 +1255,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     // Partition counts per sequence and their exclusive prefix (block scan);
     // in the longest-first order only the partitions before the last one.
     const int B = p.B;
-    const bool lpt = B <= kLptMaxSeqs;
+    const bool lpt = B <= kLptMaxSeqs && !p.cluster;
     const int maxlen = p.MB * kPageRows;
     const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
     const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
@@ -1231,26 +1313,36 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     __syncthreads();
     const int W = (s_pre[B] + (lpt ? s_warp_tot[7] : 0)) * p.Hkv;
 
+    // In cluster mode no thread leaves before the cluster merge below.
     if (warp == NW) {
         run_producer<T, D, G, FUSED>(p, guess, &tm_k, &tm_v, base, full, empty, masks, s_abort,
                                      s_len, s_pre, W);
-        return;
-    }
-    // zero the output of empty contexts (spread over the CTAs); in the fused
-    // step their new token is still appended
-    for (int b = blockIdx.x; b < B; b += gridDim.x) {
-        if (s_len[b] != 0) continue;
-        for (int idx = tid; idx < p.Hq * D; idx += NW * 32)
-            store_out(p.out, (size_t)b * p.Hq * D + idx, 0.f, p.out_bf16);
-        if constexpr (FUSED) append_only<T, D>(p, fr, b);
-    }
-    if constexpr (MMA) {
-        run_consumer_mma<D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks, s_abort, s_len,
-                                      s_pre, W);
+        if (!p.cluster) return;
     } else {
-        run_consumer_simt<T, D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks, s_abort,
-                                          s_len, s_pre, W);
+        // zero the output of empty contexts (spread over the CTAs); in the
+        // fused step their new token is still appended
+        for (int b = blockIdx.x; b < B; b += gridDim.x) {
+            if (s_len[b] != 0) continue;
+            for (int idx = tid; idx < p.Hq * D; idx += NW * 32)
+                store_out(p.out, (size_t)b * p.Hq * D + idx, 0.f, p.out_bf16);
+            if constexpr (FUSED) append_only<T, D>(p, fr, b);
+        }
+        int merged;
+        if constexpr (MMA) {
+            merged = run_consumer_mma<D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks,
+                                                   s_abort, s_len, s_pre, W);
+        } else {
+            merged = run_consumer_simt<T, D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks,
+                                                       s_abort, s_len, s_pre, W);
+        }
+        if (p.cluster && merged <= 0) {
+            // no partition here (or this CTA gave up): an empty partial
+            float* part = reinterpret_cast<float*>(base + L::OFF_Q);
+            for (int idx = tid; idx < G * (D + 2); idx += NW * 32)
+                part[idx] = (idx % (D + 2)) == D ? kNegInf : 0.f;
+        }
     }
+    if (p.cluster) cluster_merge<T, D, G>(p, base);
 }
 
 // ----------------------------------------------------------------- combine
@@ -1413,6 +1505,11 @@ int current_device() {
     return dev;
 }
 
+// Cluster-mode launches ask for this much shared memory per CTA, so that a
+// cluster spreads over one SM per CTA instead of packing three CTAs into an
+// SM (they share its issue slots and load bandwidth otherwise).
+constexpr size_t kClusterCtaSmem = 116 * 1024;
+
 template <typename K>
 cudaError_t prepare_kernel(K kern, size_t smem, int* ctas_per_sm) {
     static std::mutex mu;
@@ -1425,7 +1522,8 @@ cudaError_t prepare_kernel(K kern, size_t smem, int* ctas_per_sm) {
         *ctas_per_sm = it->second;
         return cudaSuccess;
     }
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)std::max(smem, kClusterCtaSmem));
     if (e != cudaSuccess) return e;
     int n = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, smem);
@@ -1433,6 +1531,44 @@ cudaError_t prepare_kernel(K kern, size_t smem, int* ctas_per_sm) {
     if (n < 1) return cudaErrorInvalidConfiguration;
     cache[key] = n;
     *ctas_per_sm = n;
+    return cudaSuccess;
+}
+
+// Clusters of `cs` CTAs of this kernel that can be resident at once (cached).
+template <typename K>
+cudaError_t max_active_clusters(K kern, size_t smem, int cs, int* n) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, size_t, int>, int> cache;
+    const int dev = current_device();
+    const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), dev, smem, cs);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        *n = it->second;
+        return cudaSuccess;
+    }
+    cudaError_t e = cudaSuccess;
+    if (cs > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cs);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    e = cudaOccupancyMaxActiveClusters(&c, kern, &cfg);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // not fatal: no cluster mode for this shape
+        c = 0;
+    }
+    cache[key] = c;
+    *n = c;
     return cudaSuccess;
 }
 
@@ -1475,20 +1611,45 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
 
     const int64_t upper = a.B * a.Hkv * (int64_t)a.max_partitions;
     const int64_t resident = (int64_t)device_sm_count() * occ;
-    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min(upper, resident));
+    unsigned grid = (unsigned)std::max<int64_t>(1, std::min(upper, resident));
+
+    // Cluster mode: when every (sequence, kv head) can have its own cluster of
+    // NP CTAs resident at once, the partitions are merged inside the cluster
+    // and the combine kernel is not needed.
+    int cs = 0;
+    const size_t smem_cl = std::max(smem, kClusterCtaSmem);
+    if (a.allow_cluster && a.max_partitions >= 2 && a.max_partitions <= kMaxClusterCtas) {
+        int nc = 0;
+        e = max_active_clusters(kern, smem_cl, a.max_partitions, &nc);
+        if (e != cudaSuccess) return e;
+        if ((int64_t)nc >= a.B * a.Hkv) cs = a.max_partitions;
+    }
+    p.cluster = cs;
+    if (a.plan_only) {
+        *a.launches = (cs || a.max_partitions <= 1) ? 1 : 2;
+        return cudaSuccess;
+    }
+    if (cs) {
+        p.sched = nullptr;  // one item per CTA, nothing to claim
+        grid = (unsigned)(a.B * a.Hkv * cs);
+    }
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kDecodeThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = cs ? smem_cl : smem;
     cfg.stream = a.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)(cs ? cs : 1);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = cs ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv, fr);
-    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+    if (e != cudaSuccess || a.max_partitions <= 1 || cs) return e;
 
     CombineParams cp;
     cp.context_lens = a.context_lens;
@@ -1553,11 +1714,32 @@ cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_bl
 
 cudaError_t launch_paged_decode(const DecodeArgs& a) {
     CUtensorMap tmk, tmv;
+    if (a.plan_only) {
+        memset(&tmk, 0, sizeof(tmk));
+        memset(&tmv, 0, sizeof(tmv));
+        return a.fused ? dispatch_all<true>(a, tmk, tmv) : dispatch_all<false>(a, tmk, tmv);
+    }
     cudaError_t e = encode_cache_map(&tmk, a.k_cache, a.num_blocks, a.Hkv, a.D, a.kv_dtype);
     if (e != cudaSuccess) return e;
     e = encode_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D, a.kv_dtype);
     if (e != cudaSuccess) return e;
     return a.fused ? dispatch_all<true>(a, tmk, tmv) : dispatch_all<false>(a, tmk, tmv);
+}
+
+int decode_cluster_capacity(int cs) {
+    // Every decode variant runs at one CTA per SM in cluster mode (its
+    // shared-memory request sees to that), so one variant stands for all.
+    auto kern = paged_decode_kernel<bf16, 64, 4, true, false>;
+    int occ = 0, n = 0;
+    if (prepare_kernel(kern, kClusterCtaSmem, &occ) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    if (max_active_clusters(kern, kClusterCtaSmem, cs, &n) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 
 int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_t num_seqs) {

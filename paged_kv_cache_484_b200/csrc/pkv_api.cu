@@ -128,19 +128,36 @@ bool valid_dtype(int32_t t) { return t == PKV_DTYPE_F32 || t == PKV_DTYPE_BF16; 
 // Partition length.  A partition should fill whole stages of the ring and be
 // long enough that the per-item work (q fragments, merge, partial store)
 // stays small next to the streaming: at least 128 tokens (one stage of the
-// two-page-per-warp path), and 1024 once there is work for about two items
-// per resident CTA even at that length.  Between the two, the length that
-// gives about two items per resident CTA if every sequence had the maximum
-// length.  Never more than kMaxPartitions partitions.
+// two-page-per-warp path), at most 1024.  Between the two, the multiple of
+// 128 nearest to the length that would give about six items per resident
+// CTA if every sequence had the maximum length: enough items that the
+// longest-first tail is short.  Never more than kMaxPartitions partitions.
+// Batches too small to fill the GPU even at 128 tokens get one partition per
+// CTA of a thread-block cluster instead (cluster mode, see the decode).
 int32_t auto_partition(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t MB,
                        int32_t kv_dtype) {
     const int64_t maxlen = MB * kPageRows;
     const int64_t G = Hq / std::max<int64_t>(1, Hkv);
     const int64_t resident =
         (int64_t)device_sm_count() * decode_ctas_per_sm(D, G, kv_dtype, false, B);
-    const int64_t target_items = 2 * resident;
+    // Small batches, where even 128-token partitions would not fill one wave
+    // of CTAs: split each (sequence, kv head) into up to kMaxClusterCtas
+    // partitions, one CTA each, merged inside their thread-block cluster.
+    const int64_t pairs = std::max<int64_t>(1, B * Hkv);
+    if (pairs * ceil_div(maxlen, 128) <= resident && maxlen > 128) {
+        // the largest cluster size of which `pairs` clusters fit at once
+        int64_t np = std::min<int64_t>(kMaxClusterCtas, ceil_div(maxlen, kPageRows));
+        while (np >= 2 && decode_cluster_capacity((int)np) < pairs) --np;
+        if (np >= 2) {
+            int64_t Pc = ceil_div(ceil_div(maxlen, np), kPageRows) * kPageRows;
+            const int64_t floor_np =
+                ceil_div(ceil_div(maxlen, kMaxPartitions), kPageRows) * kPageRows;
+            return (int32_t)std::max(Pc, floor_np);
+        }
+    }
+    const int64_t target_items = 6 * resident;
     int64_t P = ceil_div(std::max<int64_t>(1, maxlen * B * Hkv), target_items);
-    P = ceil_div(P, 128) * 128;
+    P = (P + 64) / 128 * 128;
     P = std::max<int64_t>(128, std::min<int64_t>(P, 1024));
     const int64_t floor_np = ceil_div(ceil_div(maxlen, kMaxPartitions), kStageTokens) * kStageTokens;
     P = std::max(P, floor_np);
@@ -285,6 +302,43 @@ size_t pkv_decode_workspace_size(int64_t num_seqs, int64_t num_q_heads, int64_t 
     return w.bytes;
 }
 
+int32_t pkv_decode_launches(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                            int64_t head_dim, int64_t max_blocks_per_seq, int64_t block_size,
+                            int32_t kv_dtype, int32_t out_dtype, int32_t partition_tokens,
+                            uint32_t flags, int32_t fused) {
+    if (num_seqs <= 0 || max_blocks_per_seq <= 0 || !valid_dtype(kv_dtype) ||
+        !valid_dtype(out_dtype) || (flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_NO_CLUSTER)))
+        return 0;
+    if (num_seqs > PKV_MAX_SEQS_PER_CALL) return 0;
+    if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
+    WorkspacePlan w;
+    if (plan_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, kv_dtype,
+                       partition_tokens, &w) != PKV_OK)
+        return 0;
+    DecodeArgs a = {};
+    a.B = num_seqs;
+    a.Hq = num_q_heads;
+    a.Hkv = num_kv_heads;
+    a.D = head_dim;
+    a.num_blocks = 1;
+    a.MB = max_blocks_per_seq;
+    a.kv_dtype = kv_dtype;
+    a.out_dtype = out_dtype;
+    a.partition_tokens = w.P;
+    a.max_partitions = w.NP;
+    a.force_simt = (flags & PKV_DECODE_FORCE_SIMT) != 0;
+    a.allow_cluster = (flags & PKV_DECODE_NO_CLUSTER) == 0;
+    a.fused = fused != 0;
+    a.plan_only = true;
+    int32_t n = 0;
+    a.launches = &n;
+    if (launch_paged_decode(a) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
 }  // extern "C"
 
 namespace {
@@ -316,7 +370,7 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
         set_last_error("kv_dtype/out_dtype unsupported");
         return PKV_ERR_UNSUPPORTED;
     }
-    if ((flags & ~PKV_DECODE_FORCE_SIMT) != 0) {
+    if ((flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_NO_CLUSTER)) != 0) {
         set_last_error("unknown flags 0x%x", flags);
         return PKV_ERR_INVALID_ARG;
     }
@@ -396,6 +450,7 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
     a.max_partitions = w.NP;
     a.scale = scale;
     a.force_simt = (flags & PKV_DECODE_FORCE_SIMT) != 0;
+    a.allow_cluster = (flags & PKV_DECODE_NO_CLUSTER) == 0;
     a.device_error = device_error;
     a.stream = static_cast<cudaStream_t>(stream);
     a.fused = step != nullptr;

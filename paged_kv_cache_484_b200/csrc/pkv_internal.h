@@ -13,6 +13,7 @@ constexpr int kConsumerWarps = 4;  // decode: warps that compute
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kStageTokens = kConsumerWarps * kPageRows;   // one page per consumer warp
 constexpr int kMaxPartitions = 1024;
+constexpr int kMaxClusterCtas = 16;  // cluster-mode limit (non-portable above 8)
 
 // Per-thread detail of the last failing call (returned by pkv_last_error).
 void set_last_error(const char* fmt, ...);
@@ -49,6 +50,11 @@ struct DecodeArgs {
     int32_t max_partitions;    // NP = ceil(MB * 16 / P)
     float scale;
     bool force_simt;
+    bool allow_cluster;  // split contexts may merge inside a thread-block cluster
+    // planning only: launch nothing, store the number of kernels the call
+    // would launch (1 or 2) in *launches
+    bool plan_only;
+    int32_t* launches;
     int32_t* device_error;
     cudaStream_t stream;
     // fused step (append inside the decode kernel); q is rotated in place
@@ -64,5 +70,8 @@ cudaError_t launch_paged_decode(const DecodeArgs& a);
 // Resident decode CTAs per SM for these shapes (occupancy query, cached).
 int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_t num_seqs);
 int device_sm_count();
+// Clusters of `cs` decode CTAs (cluster mode, one CTA per SM) that can be
+// resident at once on the current device; 0 when unknown.
+int decode_cluster_capacity(int cs);
 
 }  // namespace pkv

@@ -129,8 +129,14 @@ def test_workspace_size_formula(lib):
     assert lib.pkv_decode_workspace_size(4, 8, 2, 64, 4, 16, BF16, 24) == 0  # invalid P -> 0
 
 
-def test_auto_partition_is_a_whole_number_of_stages(lib):
+def test_auto_partition_limits(lib):
+    """Whole pages, at most 1024 partitions; batches that fill the GPU get
+    whole 128-token stages.  (Without a device no cluster capacity is known,
+    so small batches get the same rule here; the GPU tests check the
+    cluster-mode choice.)"""
     for (B, MB) in ((1, 129), (64, 257), (256, 2049), (16, 8193), (4096, 3)):
         P = lib.pkv_decode_partition_tokens(B, 32, 8, 64, MB, 16, BF16)
-        assert P % 64 == 0 and 64 <= P
+        assert P % 16 == 0 and 16 <= P
         assert math.ceil(MB * 16 / P) <= 1024
+    for (B, MB) in ((64, 257), (256, 2049), (16, 8193)):
+        assert lib.pkv_decode_partition_tokens(B, 32, 8, 64, MB, 16, BF16) % 128 == 0

@@ -323,3 +323,73 @@ def test_static_schedule_without_workspace(fused):
                                    w.scale, out, workspace=none, partition_tokens=P)
     torch.cuda.synchronize()
     check_decode(out.cpu(), ref, torch.bfloat16, "static schedule")
+
+
+@pytest.mark.parametrize("dtype,d,G", [(torch.bfloat16, 64, 4), (torch.bfloat16, 64, 8),
+                                       (torch.bfloat16, 128, 4), (torch.float32, 64, 2),
+                                       (torch.bfloat16, 64, 1)])
+@pytest.mark.parametrize("P", [304, 1040])
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "one_launch"])
+def test_cluster_merge(dtype, d, G, P, fused):
+    """Small batches: each (sequence, kv head) runs as one thread-block
+    cluster, one partition per CTA, merged through distributed shared memory.
+    The workspace partials stay untouched (no combine), sequences shorter
+    than the cluster leave CTAs idle, and the result matches the oracle; with
+    cluster=False the same call goes through the partials and the combine."""
+    Hkv = 2
+    lens = [2200, 15, 300, 1200]
+    results = {}
+    for cluster in (True, False):
+        w = W.build_workload("cluster", lens, G * Hkv, Hkv, d, dtype, 1e4, seed=200 + d + G,
+                             device=DEV, pool_factor=1.2)
+        if not fused:
+            w.decode_lens[1] = 0  # an empty context: all-zero output
+        NP = -(-w.max_blocks * w.block_size // P)
+        assert 2 <= NP <= 16
+        assert pkv.decode_launches(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=dtype,
+                                   out_dtype=torch.float32, partition_tokens=P, cluster=cluster,
+                                   fused=fused) == (1 if cluster else 2)
+        sub = SubProblem(w, range(w.B))
+        need = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=dtype,
+                                         partition_tokens=P)
+        ws = pkv.new_workspace(need, DEV)
+        ws[pkv.SCHED_BYTES:].fill_(0x7F)
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=DEV)
+        if fused:
+            pkv.decode_step(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                            w.v_cache, w.block_tables, w.decode_lens, w.rope_theta, w.scale, out,
+                            workspace=ws, partition_tokens=P, cluster=cluster)
+        else:
+            pkv.kv_append(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                          w.v_cache, w.rope_theta)
+            pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
+                                       w.scale, out, workspace=ws, partition_tokens=P,
+                                       cluster=cluster)
+        torch.cuda.synchronize()
+        partials_untouched = bool((ws[pkv.SCHED_BYTES:] == 0x7F).all())
+        assert partials_untouched == cluster, f"cluster={cluster}: partials untouched={partials_untouched}"
+        assert not ws[:pkv.SCHED_BYTES].any()
+        _, _, _, ref = sub.oracle_step()
+        if not fused:
+            ref[1].zero_()
+            assert not out[1].any()
+        check_decode(out, ref, dtype, f"{dtype} d{d} G{G} P={P} fused={fused} cluster={cluster}")
+        results[cluster] = out
+    assert (results[True] - results[False]).abs().max().item() < 1e-4
+
+
+def test_batch1_auto_partition_uses_clusters():
+    """The batch-1 Llama-shaped step: the automatic partition cuts each kv
+    head's context into 2..16 partitions that run as one cluster (one
+    launch), and the result matches the oracle."""
+    w = W.make_config(2, device=DEV)
+    P = pkv.decode_partition_tokens(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=w.dtype)
+    NP = -(-w.max_blocks * w.block_size // P)
+    assert 2 <= NP <= 16
+    assert pkv.decode_launches(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=w.dtype,
+                               fused=True) == 1
+    sub = SubProblem(w, range(w.B))
+    out = gpu_step(w, out_dtype=torch.float32, fused=True)
+    torch.cuda.synchronize()
+    _, _, _, ref = sub.oracle_step()
+    check_decode(out, ref, w.dtype, "batch-1 cluster step")
