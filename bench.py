@@ -472,13 +472,30 @@ def run_ours(args):
     e2e = None
     if host_inputs is not None:
         out_host = torch.empty(outs[0].shape, dtype=out_dtype, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for t in host_inputs.values())
+        # the step's inputs packed into one pinned host buffer (16-byte aligned
+        # fields) and copied into one device buffer whose views the call reads:
+        # one H2D copy per step instead of seven
+        offs, size = {}, 0
+        for name, t in host_inputs.items():
+            offs[name] = size
+            size += (t.numel() * t.element_size() + 15) // 16 * 16
+
+        def view(buf, name):
+            t = host_inputs[name]
+            nb = t.numel() * t.element_size()
+            return buf[offs[name]:offs[name] + nb].view(t.dtype).view(t.shape)
+
+        hbuf = torch.zeros(size, dtype=torch.uint8, pin_memory=True)
+        dbuf = torch.empty(size, dtype=torch.uint8, device=device)
+        for name, t in host_inputs.items():
+            view(hbuf, name).copy_(t)
+        dev_in = {name: view(dbuf, name) for name in host_inputs}
+        h2d = size
         d2h = out_host.numel() * out_host.element_size()
 
         def e2e_step(k):
-            c = copies[k % ncopies]
-            for name, t in host_inputs.items():
-                c[name].copy_(t, non_blocking=True)
+            c = dict(copies[k % ncopies], **dev_in)
+            dbuf.copy_(hbuf, non_blocking=True)
             append(c)
             decode(c, outs[k % ncopies])
             out_host.copy_(outs[k % ncopies], non_blocking=True)

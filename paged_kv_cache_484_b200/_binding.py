@@ -102,7 +102,7 @@ def _dtype_code(dt: torch.dtype) -> int:
 def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
+    if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
