@@ -82,7 +82,10 @@ struct Layout {
     static constexpr int PPW = (SWZ && D == 64 && G <= 4) ? 2 : 1;
     static constexpr int STAGE_PAGES = NW * PPW;
     static constexpr int STAGE_BYTES = 2 * STAGE_PAGES * PAGE_BYTES;  // K pages, then V pages
-    static constexpr int STAGES = cmax(2, cmin(6, 65536 / STAGE_BYTES));
+    // 64 KiB of ring (96 KiB for bf16 d = 128, whose CTAs are two per SM
+    // by registers anyway)
+    static constexpr int STAGES =
+        cmax(2, cmin(6, ((D == 128 && SWZ) ? 98304 : 65536) / STAGE_BYTES));
     static constexpr int Q_COPY = G * D * ESZ;
     static constexpr int Q_BYTES = round_up(Q_COPY, 128);
     static constexpr int ROW_COPY = D * ESZ;           // one k or v row

@@ -128,7 +128,7 @@ bool valid_dtype(int32_t t) { return t == PKV_DTYPE_F32 || t == PKV_DTYPE_BF16; 
 // Partition length.  A partition should fill whole stages of the ring and be
 // long enough that the per-item work (q fragments, merge, partial store)
 // stays small next to the streaming: at least 128 tokens (one stage of the
-// two-page-per-warp path), at most 1024.  Between the two, the multiple of
+// two-page-per-warp path), at most 2048.  Between the two, the multiple of
 // 128 nearest to the length that would give about six items per resident
 // CTA if every sequence had the maximum length: enough items that the
 // longest-first tail is short.  Never more than kMaxPartitions partitions.
@@ -158,7 +158,7 @@ int32_t auto_partition(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t MB
     const int64_t target_items = 6 * resident;
     int64_t P = ceil_div(std::max<int64_t>(1, maxlen * B * Hkv), target_items);
     P = (P + 64) / 128 * 128;
-    P = std::max<int64_t>(128, std::min<int64_t>(P, 1024));
+    P = std::max<int64_t>(128, std::min<int64_t>(P, 2048));
     const int64_t floor_np = ceil_div(ceil_div(maxlen, kMaxPartitions), kStageTokens) * kStageTokens;
     P = std::max(P, floor_np);
     return (int32_t)P;
