@@ -68,6 +68,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--prefill", type=int, default=0, metavar="C",
+                    help="time chunked prefill instead: the last C context tokens of every "
+                         "sequence of the workload attend causally to its paged cache")
     return ap.parse_args(argv)
 
 
@@ -575,10 +578,123 @@ def run_ours(args):
     return 0
 
 
+def run_prefill(args):
+    """Chunked prefill on the workload's sequences: queries for the last C
+    tokens of each context (their K/V are the cache's own rows), timed like
+    the decode step: back to back from captured graphs over enough copies of
+    the inputs to exceed L2.  Bytes: every context token's K and V once per
+    kv head, plus q and out."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, local)
+    import paged_kv_cache_484_b200 as pkv
+    from paged_kv_cache_484_b200 import workloads as W
+
+    pkv.load_library()
+    w = W.make_config(args.config, device=device)
+    if w.dtype != torch.bfloat16:
+        raise SystemExit("prefill: bf16 workloads only")
+    C = args.prefill
+    lens = w.cached_lens.clamp(min=C).to(torch.int32)
+    g = torch.Generator(device=device)
+    g.manual_seed(484 + args.config)
+    q = torch.randn((w.B, C, w.Hq, w.d), generator=g, device=device, dtype=torch.bfloat16)
+    out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+    P = args.partition_tokens or pkv.prefill_partition_tokens(w.B, C, w.Hq, w.Hkv, w.d,
+                                                              w.max_blocks)
+    need = pkv.prefill_workspace_size(w.B, C, w.Hq, w.Hkv, w.d, w.max_blocks,
+                                      partition_tokens=P)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    esz_out = 2 if out_dtype == torch.bfloat16 else 4
+    nbytes = int(lens.to(torch.int64).sum().item()) * w.Hkv * w.d * 2 * 2 + \
+        w.B * C * w.Hq * w.d * (2 + esz_out)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    ncopies = args.copies or (1 if nbytes >= 2 * l2 else min(1024, math.ceil(2 * l2 / nbytes)))
+    copies = [dict(q=q, k=w.k_cache, v=w.v_cache, t=w.block_tables, l=lens)]
+    for _ in range(ncopies - 1):
+        copies.append({k: v.clone() for k, v in copies[0].items()})
+    outs = [torch.empty((w.B, C, w.Hq, w.d), dtype=out_dtype, device=device)
+            for _ in range(ncopies)]
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def call(k):
+        c = copies[k % ncopies]
+        pkv.paged_attention_prefill(c["q"], c["k"], c["v"], c["t"], c["l"], w.scale,
+                                    outs[k % ncopies], workspace=ws, partition_tokens=P,
+                                    device_error=err)
+
+    for k in range(max(3, args.warmup, ncopies)):
+        call(k)
+    torch.cuda.synchronize()
+    K = args.steps
+    S = ncopies if ncopies > 1 else min(K, 16)
+
+    def capture(n):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for k in range(n):
+                call(k)
+        return gr
+
+    full = capture(S)
+    tail = capture(K % S) if K % S else None
+    full.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        e0.record(stream)
+        for _ in range(K // S):
+            full.replay()
+        if tail is not None:
+            tail.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world, device)
+    ms = max_over_ranks(e0.elapsed_time(e1) / K, world, device)
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error flag {int(err.item()):#x}")
+    peak, peak_src = load_peak()
+    value = world * nbytes / (ms * 1e-3) / 1e9
+    launches = 1 + (1 if -(-w.max_blocks * 16 // P) > 1 else 0)
+    line = {
+        "metric": "paged chunked-prefill attention achieved HBM GB/s; query tokens/sec",
+        "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "query_tokens_per_s": round(world * w.B * C / (ms * 1e-3), 1),
+        "config": {"workload": W.CONFIG_NAMES[args.config] + f"_prefill_chunk{C}",
+                   "batch_seqs": w.B, "chunk_tokens": C, "q_heads": w.Hq, "kv_heads": w.Hkv,
+                   "head_dim": w.d, "partition_tokens": P,
+                   "l2": f"inputs larger than L2: {ncopies} copies, no flush in the timed region"},
+        "roofline": {"bound": "hbm", "kernel": "paged_prefill_kernel" +
+                     (" + prefill_combine_kernel" if launches == 2 else ""),
+                     "achieved": round(value / world, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(value / world / peak, 4), "peak_source": peak_src,
+                     "traffic": None},
+        "gpu_launches": K * launches,
+        "clocks": clocks.summary(),
+        "device": torch.cuda.get_device_name(device),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.prefill:
+        return run_prefill(args)
     return run_ours(args)
 
 

@@ -331,6 +331,65 @@ pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache
                                               int32_t partition_tokens, uint32_t flags,
                                               int32_t* device_error, void* stream);
 
+/*
+ * pkv_paged_attention_prefill -- chunked prefill: several query tokens per
+ * sequence attend causally to the paged cache.
+ *
+ * Source: "Efficient LLM Inference", KV Caching: Verify Reuse, Positions and
+ * Windows (a prompt computed in chunks over the retained keys and values
+ * must equal the full-prefix forward pass); "llm-inference-from-scratch",
+ * M1 (prefill/decode equivalence); "Inference From Scratch", ch. 8 and
+ * ch. 10 (online softmax; paged attention through block tables).
+ *
+ * The chunk of sequence b is its last C = chunk_tokens context tokens: their
+ * K/V are already in the cache (appended with pkv_kv_append, e.g. with
+ * positions L_b - C .. L_b - 1), and their rotated queries are q[b, 0..C-1].
+ * For b < num_seqs, i < C, h < Hq, with L = context_lens[b], kvh = h / G:
+ *   out[b, i, h, :] = sum_{t <= L-C+i} exp(s_t - max s) V_b[t] / sum_t exp(s_t - max s),
+ *   s_t = scale * <q[b, i, h, :], K_b[t]>,
+ * i.e. pkv_paged_attention_decode of query i with context length L - C + i + 1.
+ * fp32 arithmetic (bf16 inputs widen exactly), P applied as a two-term bf16
+ * split on the tensor cores, the result rounded once to out_dtype.
+ *
+ * Arguments
+ *   q             device, [num_seqs, C, Hq, head_dim] bf16
+ *   k_cache, v_cache  device, [num_blocks, Hkv, block_size, head_dim] bf16
+ *   block_tables  device, [num_seqs, max_blocks_per_seq] int32
+ *   context_lens  device, [num_seqs] int32 in [C, max_blocks_per_seq * block_size],
+ *                 the chunk included (a shorter one sets PKV_DEVERR_CONTEXT_LEN
+ *                 and its rows are not written)
+ *   out           device, [num_seqs, C, Hq, head_dim], f32 or bf16
+ *   workspace     device, >= pkv_prefill_workspace_size(...) bytes (NULL when
+ *                 that is 0); contents need no initialisation
+ *   partition_tokens  0 = library choice (pkv_prefill_partition_tokens), else a
+ *                 multiple of block_size in [block_size, PKV_MAX_PARTITION_TOKENS]
+ * kv_dtype must be PKV_DTYPE_BF16.  num_seqs == 0 returns PKV_OK and launches
+ * nothing.  Errors as for pkv_paged_attention_decode.
+ */
+pkv_status pkv_paged_attention_prefill(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, const int32_t* context_lens,
+                                       void* out, void* workspace, size_t workspace_bytes,
+                                       int64_t num_seqs, int64_t chunk_tokens,
+                                       int64_t num_q_heads, int64_t num_kv_heads,
+                                       int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                                       int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                       int32_t out_dtype, float scale, int32_t partition_tokens,
+                                       int32_t* device_error, void* stream);
+
+/* Bytes of workspace pkv_paged_attention_prefill needs (partition partials:
+ * num_seqs * C * Hq * NP * (head_dim + 2) floats when NP > 1, else 0).  Host
+ * only; 0 also for invalid arguments. */
+size_t pkv_prefill_workspace_size(int64_t num_seqs, int64_t chunk_tokens, int64_t num_q_heads,
+                                  int64_t num_kv_heads, int64_t head_dim,
+                                  int64_t max_blocks_per_seq, int64_t block_size,
+                                  int32_t partition_tokens);
+
+/* The partition length a prefill call with partition_tokens = 0 uses.  Host
+ * only; 0 for invalid arguments. */
+int32_t pkv_prefill_partition_tokens(int64_t num_seqs, int64_t chunk_tokens, int64_t num_q_heads,
+                                     int64_t num_kv_heads, int64_t head_dim,
+                                     int64_t max_blocks_per_seq, int64_t block_size);
+
 /* Short text for a status code (static storage). */
 const char* pkv_status_string(int32_t status);
 

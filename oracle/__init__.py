@@ -11,6 +11,8 @@ Functions (all take and return CPU ``torch`` tensors):
 * ``kv_append``            -- RoPE on q (in place) and k, write k/v into the slot.
 * ``paged_attention_decode`` -- plain two-pass softmax(q K^T scale) V over the
   tokens each block table lists, in fp64.
+* ``paged_chunked_prefill`` -- a chunk of C queries per sequence, each a
+  decode over its own causal prefix of the paged cache.
 * ``contiguous_decode`` / ``causal_prefill`` -- the same definition without
   paging, used only to check the oracle itself.
 * ``rope`` / ``round_bf16`` / ``bf16_to_double`` -- the oracle's building blocks,
@@ -141,6 +143,28 @@ class Oracle:
                                          float(scale), pp, npairs, int(nthreads), _ptr(out)))
         return out
 
+    def paged_chunked_prefill(self, q, k_cache, v_cache, block_tables, context_lens, scale,
+                              nthreads: int = 1) -> torch.Tensor:
+        """fp64 [B, C, Hq, d] output of a prefill chunk: the last C context
+        tokens of each sequence, query i attending to tokens 0 .. L - C + i.
+
+        "Efficient LLM Inference", KV Caching: Verify Reuse, Positions and
+        Windows -- a chunk computed over the retained K/V equals the
+        full-prefix pass, so query i of the chunk is exactly one decode step
+        over the first L - C + i + 1 tokens.  That is how it is computed here:
+        one plain decode per chunk position, with that context length.
+        """
+        _cpu(q)
+        _cpu(context_lens, torch.int32)
+        B, C, Hq, d = q.shape
+        out = torch.empty((B, C, Hq, d), dtype=torch.float64)
+        for i in range(C):
+            lens_i = (context_lens.to(torch.int64) - C + i + 1).clamp(min=0).to(torch.int32)
+            out[:, i] = self.paged_attention_decode(q[:, i].contiguous(), k_cache, v_cache,
+                                                    block_tables, lens_i, scale,
+                                                    nthreads=nthreads)
+        return out
+
     def contiguous_decode(self, q, K, V, scale) -> torch.Tensor:
         """q [Hq, d], K/V [L, Hkv, d] (float64) -> [Hq, d]."""
         q, K, V = (_cpu(t.contiguous(), torch.float64) for t in (q, K, V))
@@ -197,3 +221,4 @@ kv_append = default.kv_append
 paged_attention_decode = default.paged_attention_decode
 contiguous_decode = default.contiguous_decode
 causal_prefill = default.causal_prefill
+paged_chunked_prefill = default.paged_chunked_prefill

@@ -32,5 +32,8 @@ from ._binding import (  # noqa: F401
     new_workspace,
     paged_attention_decode,
     paged_attention_decode_noalloc,
+    paged_attention_prefill,
+    prefill_partition_tokens,
+    prefill_workspace_size,
     version,
 )

@@ -74,6 +74,14 @@ def load_library() -> ctypes.CDLL:
                                                            i32, i32, ctypes.c_float, i32, u32,
                                                            vp, vp]
         lib.pkv_paged_attention_decode_noalloc.restype = ctypes.c_int
+        lib.pkv_paged_attention_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                                     i64, i64, i64, i64, i64, i64, i64, i64,
+                                                     i32, i32, ctypes.c_float, i32, vp, vp]
+        lib.pkv_paged_attention_prefill.restype = ctypes.c_int
+        lib.pkv_prefill_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i64, i32]
+        lib.pkv_prefill_workspace_size.restype = ctypes.c_size_t
+        lib.pkv_prefill_partition_tokens.argtypes = [i64, i64, i64, i64, i64, i64, i64]
+        lib.pkv_prefill_partition_tokens.restype = i32
         lib.pkv_status_string.argtypes = [i32]
         lib.pkv_status_string.restype = ctypes.c_char_p
         lib.pkv_last_error.argtypes = []
@@ -309,3 +317,55 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
 
 def version() -> int:
     return int(load_library().pkv_version())
+
+
+def prefill_workspace_size(num_seqs, chunk_tokens, num_q_heads, num_kv_heads, head_dim,
+                           max_blocks_per_seq, partition_tokens=0,
+                           block_size=BLOCK_SIZE) -> int:
+    """Bytes of workspace ``paged_attention_prefill`` needs (0: none)."""
+    lib = load_library()
+    return int(lib.pkv_prefill_workspace_size(num_seqs, chunk_tokens, num_q_heads, num_kv_heads,
+                                              head_dim, max_blocks_per_seq, block_size,
+                                              int(partition_tokens)))
+
+
+def prefill_partition_tokens(num_seqs, chunk_tokens, num_q_heads, num_kv_heads, head_dim,
+                             max_blocks_per_seq, block_size=BLOCK_SIZE) -> int:
+    """Partition length a prefill call picks when ``partition_tokens`` is 0."""
+    lib = load_library()
+    return int(lib.pkv_prefill_partition_tokens(num_seqs, chunk_tokens, num_q_heads,
+                                                num_kv_heads, head_dim, max_blocks_per_seq,
+                                                block_size))
+
+
+def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                            stream=None, *, workspace=None, partition_tokens=0,
+                            device_error=None) -> torch.Tensor:
+    """Chunked prefill: the last C tokens of every sequence attend causally to
+    its paged context (their K/V already appended).  q [B, C, Hq, d] bf16,
+    caches [NB, Hkv, 16, d] bf16, out [B, C, Hq, d] float32 or bfloat16;
+    writes and returns ``out``.  See include/pkv.h, pkv_paged_attention_prefill.
+    """
+    lib = load_library()
+    if q.dtype != torch.bfloat16 or k_cache.dtype != torch.bfloat16 \
+            or v_cache.dtype != torch.bfloat16:
+        raise TypeError("prefill: q and the caches must be bfloat16")
+    B, C, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, C, Hq, d) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("inconsistent paged_attention_prefill shapes")
+    need = lib.pkv_prefill_workspace_size(B, C, Hq, Hkv, d, MB, bs, int(partition_tokens))
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_paged_attention_prefill(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        B, C, Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16, _dtype_code(out.dtype), float(scale),
+        int(partition_tokens), err, _stream_ptr(stream, q.device))
+    _raise(st, lib, "paged_attention_prefill")
+    return out

@@ -1,0 +1,513 @@
+// paged_prefill.cu -- multi-query (chunked-prefill) attention over a paged KV
+// cache on sm_100a.
+//
+// What it computes ("Efficient LLM Inference", KV Caching: chunked computation
+// over the retained K/V equals the full-prefix pass; "Inference From Scratch",
+// ch. 10 paged attention and ch. 8 online softmax): every sequence b has a
+// chunk of C query tokens, the last C tokens of its context (their K/V
+// already appended to the cache).  Query i sits at position L_b - C + i and
+// attends causally to tokens 0 .. L_b - C + i:
+//   out[b, i, h, :] = softmax_t(scale q[b, i, h] . K_b[t]) V_b[t],  t <= L_b - C + i,
+// with kv head h / G.  That is the decode definition applied to each query
+// with its own context length, which is how the tests check it.
+//
+// Work decomposition.  A work item is (sequence, kv head, row group,
+// partition of P keys).  Its rows are up to 32 (query, head) pairs of the kv
+// head, (query i, head g) -> row i*G + g; each of the four consumer warps
+// owns 8 rows and runs them over every page of the partition, so a K/V page
+// is read once per row group.  One CTA per item (no persistence: the items
+// of a prefill chunk are uniform).  Partitions are merged by a log-sum-exp
+// combine kernel when a sequence has more than one.
+//
+// Inside a CTA: one producer warp turns block-table entries into TMA loads of
+// whole K and V pages (128-byte swizzle) into a ring of stages guarded by
+// mbarriers; the consumer warps compute S = Q K^T and O += P V with
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate).  A warp's 16-row A tile
+// holds its 8 rows twice: rows r carry the high bf16 part of P, rows r + 8
+// the low part (p = hi + lo to ~2^-17 relative).  Each row masks the keys
+// past its own position; a row can have no key in a page or a partition
+// (its softmax state then stays m = -inf, l = 0).  Every wait is bounded.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "pkv_device.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int NWP = 4;                        // consumer warps
+constexpr int kRowsPerWarp = 8;               // (query, head) rows per warp
+constexpr int kThreadsP = (NWP + 1) * 32;     // + one producer warp
+constexpr float kNegInfP = -__builtin_huge_valf();
+
+template <int D>
+struct PLayout {
+    static constexpr int PAGE_BYTES = kPageRows * D * 2;
+    static constexpr int BOXES = D / 64;            // 64-column TMA boxes per page
+    static constexpr int BOX_BYTES = PAGE_BYTES / BOXES;
+    static constexpr int SP = 4;                    // pages per stage
+    static constexpr int STAGE_BYTES = 2 * SP * PAGE_BYTES;  // SP K pages, then SP V pages
+    static constexpr int STAGES = D == 64 ? 4 : 3;  // 64 KiB / 96 KiB of ring
+    static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+    static constexpr int OFF_MASK = OFF_BAR + 2 * STAGES * 8;  // full, empty
+    static constexpr size_t SMEM = 1024 + OFF_MASK + STAGES * 4 + 16;
+};
+
+struct PrefillParams {
+    const bf16* q;              // [B, C, Hq, D]
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    void* out;                  // [B, C, Hq, D]
+    float* part_o;              // [B, C, Hq, NP, D]
+    float* part_ml;             // [B, C, Hq, NP, 2]
+    int32_t* err;
+    int B, C, Hq, Hkv, MB, P, NP, RG, num_blocks;
+    float scale_log2;
+    int out_bf16;
+};
+
+// Byte offset of 16-byte chunk c of token row tok in a 128-byte-swizzled page.
+template <int D>
+__device__ __forceinline__ uint32_t pchunk(int tok, int c) {
+    if constexpr (D == 64) {
+        return tok * 128 + ((c ^ (tok & 7)) << 4);
+    } else {
+        return (c >> 3) * 2048 + tok * 128 + (((c & 7) ^ (tok & 7)) << 4);
+    }
+}
+
+__device__ __forceinline__ void pstore(void* out, size_t idx, float v, int out_bf16) {
+    if (out_bf16)
+        reinterpret_cast<bf16*>(out)[idx] = __float2bfloat16_rn(v);
+    else
+        reinterpret_cast<float*>(out)[idx] = v;
+}
+
+// The item's sequence and key range, from blockIdx.x.
+struct PItem {
+    int b, h, rg, part, L, np, t0, t1, npages;
+};
+
+__device__ __forceinline__ PItem prefill_item(const PrefillParams& p) {
+    PItem it;
+    int x = blockIdx.x;
+    it.part = x % p.NP;
+    x /= p.NP;
+    it.rg = x % p.RG;
+    x /= p.RG;
+    it.h = x % p.Hkv;
+    it.b = x / p.Hkv;
+    int L = p.context_lens[it.b];
+    const int maxlen = p.MB * kPageRows;
+    if (L < p.C || L > maxlen) {
+        // the chunk must lie inside the context
+        if (it.part == 0 && it.rg == 0 && it.h == 0 && threadIdx.x == 0)
+            report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
+        L = L < p.C ? 0 : maxlen;
+    }
+    it.L = L;
+    it.np = (L + p.P - 1) / p.P;
+    it.t0 = it.part * p.P;
+    it.t1 = min(L, it.t0 + p.P);
+    it.npages = it.t1 > it.t0 ? (it.t1 - it.t0 + kPageRows - 1) / kPageRows : 0;
+    return it;
+}
+
+template <int D>
+__device__ void prefill_producer(const PrefillParams& p, const PItem& it, const CUtensorMap* tmk,
+                                 const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
+                                 uint64_t* empty, uint32_t* masks, volatile int* s_abort) {
+    using L = PLayout<D>;
+    const int lane = threadIdx.x & 31;
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_parity[8];
+    uint32_t issued_any = 0;
+    bool abort = false;
+    for (int c0 = 0; c0 < it.npages && !abort; c0 += 32) {
+        int ent = -1;
+        if (c0 + lane < it.npages) {
+            const int v = p.block_tables[(size_t)it.b * p.MB + it.t0 / kPageRows + c0 + lane];
+            if (v < 0 || v >= p.num_blocks)
+                report_error(p.err, PKV_DEVERR_BLOCK_ID);
+            else
+                ent = v;
+        }
+        const int cend = min(it.npages, c0 + 32);
+        for (int s0 = c0; s0 < cend; s0 += L::SP) {
+            const int npg = min(L::SP, it.npages - s0);
+            const int k = lane - (s0 - c0);
+            const bool mine = k >= 0 && k < npg && ent >= 0;
+            const uint32_t vmask = __ballot_sync(0xffffffffu, mine) >> (s0 - c0);
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1) && !*s_abort;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                abort = true;
+                break;
+            }
+            if (lane == 0) {
+                masks[stage] = vmask;
+                mbar_arrive_expect_tx(&full[stage], __popc(vmask) * 2u * L::PAGE_BYTES);
+            }
+            __syncwarp();
+            if (mine) {
+                uint8_t* kdst = base + stage * L::STAGE_BYTES + k * L::PAGE_BYTES;
+                uint8_t* vdst = kdst + L::SP * L::PAGE_BYTES;
+                const int row0 = (ent * p.Hkv + it.h) * kPageRows;
+#pragma unroll
+                for (int bx = 0; bx < L::BOXES; ++bx) {
+                    tma_load_2d(kdst + bx * L::BOX_BYTES, tmk, bx * 64, row0, &full[stage]);
+                    tma_load_2d(vdst + bx * L::BOX_BYTES, tmv, bx * 64, row0, &full[stage]);
+                }
+            }
+            issued_parity[stage] = phase;
+            issued_any |= 1u << stage;
+            if (++stage == L::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+    }
+    if (abort) {
+        *s_abort = 1;
+        if (lane == 0) {
+            report_error(p.err, PKV_DEVERR_TIMEOUT);
+            for (int s = 0; s < L::STAGES; ++s)
+                if (issued_any & (1u << s)) (void)mbar_wait(&full[s], issued_parity[s]);
+        }
+        __syncwarp();
+    }
+}
+
+template <int D, int G>
+__device__ void prefill_consumer(const PrefillParams& p, const PItem& it, uint8_t* base,
+                                 uint64_t* full, uint64_t* empty, const uint32_t* masks,
+                                 volatile int* s_abort) {
+    using L = PLayout<D>;
+    constexpr int KS = D / 16, NT = D / 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, cq = lane & 3;
+    // this lane's row: (query i, head g) of the item's row group
+    const int fr = it.rg * (NWP * kRowsPerWarp) + warp * kRowsPerWarp + r;
+    const bool row_ok = fr < p.C * G;
+    const int qi = row_ok ? fr / G : 0, g = row_ok ? fr % G : 0;
+    const int hq = it.h * G + g;
+    // keys this row may see: 0 .. L - C + qi
+    const int row_len = row_ok ? it.L - p.C + qi + 1 : 0;
+
+    // A fragments of Q: rows r and r + 8 both hold this lane's row
+    uint32_t qa[KS][2];
+    {
+        const uint32_t* qr = reinterpret_cast<const uint32_t*>(
+            p.q + (((size_t)it.b * p.C + qi) * p.Hq + hq) * D);
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const int col = kk * 16 + 2 * cq;
+            qa[kk][0] = row_ok ? qr[col / 2] : 0u;
+            qa[kk][1] = row_ok ? qr[(col + 8) / 2] : 0u;
+        }
+    }
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_run = kNegInfP, l_run = 0.f;
+
+    int stage = 0;
+    uint32_t phase = 0;
+    const int mi = lane >> 3, ri = lane & 7;
+    const int nst = (it.npages + L::SP - 1) / L::SP;
+    bool ok = true;
+    for (int s = 0; s < nst; ++s) {
+        ok = mbar_wait(&full[stage], phase) && !*s_abort;
+        if (!ok) break;
+        const uint32_t msk = masks[stage];
+        for (int u = 0; u < L::SP; ++u) {
+            const int j = s * L::SP + u;
+            if (j >= it.npages || !((msk >> u) & 1u)) continue;
+            const int tbase = it.t0 + j * kPageRows;       // absolute token of page row 0
+            const int in_part = min(kPageRows, it.t1 - tbase);   // rows inside the partition
+            const int row_valid = max(0, min(in_part, row_len - tbase));
+            const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + u * L::PAGE_BYTES);
+            const uint32_t vbase = kbase + L::SP * L::PAGE_BYTES;
+            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int tok = ri + ((mi >> 1) << 3);
+                const int ch = 2 * kk + (mi & 1);
+                uint32_t b00, b01, b10, b11;
+                ldsm_x4(kbase + pchunk<D>(tok, ch), b00, b01, b10, b11);
+                const uint32_t a[4] = {qa[kk][0], qa[kk][0], qa[kk][1], qa[kk][1]};
+                mma_bf16_16816(sc[0], a, b00, b01);
+                mma_bf16_16816(sc[1], a, b10, b11);
+            }
+            float x[2][2];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tk = n * 8 + 2 * cq + e;
+                    x[n][e] = tk < row_valid ? sc[n][e] * p.scale_log2 : kNegInfP;
+                }
+            float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            // a row with no key so far keeps m = -inf: use 0 as the reference
+            const float m_ref = m_new == kNegInfP ? 0.f : m_new;
+            const float alpha = fast_exp2(m_run - m_ref);
+            float pr[2][2];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) pr[n][e] = fast_exp2(x[n][e] - m_ref);
+            l_run = l_run * alpha + ((pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
+            if (__any_sync(0xffffffffu, m_new != m_run)) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    o[n][0] *= alpha;
+                    o[n][1] *= alpha;
+                    o[n][2] *= alpha;
+                    o[n][3] *= alpha;
+                }
+            }
+            m_run = m_new;
+            // P: rows r the high bf16 part, rows r + 8 the low part
+            uint32_t pa[4];
+            {
+                const uint32_t hi0 = pack_bf16(pr[0][0], pr[0][1]);
+                const uint32_t hi1 = pack_bf16(pr[1][0], pr[1][1]);
+                pa[0] = hi0;
+                pa[1] = pack_bf16(pr[0][0] - bf16lo(hi0), pr[0][1] - bf16hi(hi0));
+                pa[2] = hi1;
+                pa[3] = pack_bf16(pr[1][0] - bf16lo(hi1), pr[1][1] - bf16hi(hi1));
+            }
+            // V rows past the partition may hold stale shared memory: zero them
+            uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
+            if (in_part < kPageRows) {
+                const int k0 = 2 * cq;
+                vmask_lo = (k0 < in_part ? 0x0000ffffu : 0u) | (k0 + 1 < in_part ? 0xffff0000u : 0u);
+                vmask_hi = (k0 + 8 < in_part ? 0x0000ffffu : 0u) |
+                           (k0 + 9 < in_part ? 0xffff0000u : 0u);
+            }
+#pragma unroll
+            for (int c = 0; c < NT; c += 2) {
+                const int tok = ri + ((mi & 1) << 3);
+                const int ch = c + (mi >> 1);
+                uint32_t v0, v1, v2, v3;
+                ldsm_x4_trans(vbase + pchunk<D>(tok, ch), v0, v1, v2, v3);
+                mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
+                mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1;
+        }
+    }
+    if (!ok) {
+        *s_abort = 1;
+        if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
+        return;
+    }
+    // row result: high + low rows, row sum over the quad
+    float lsum = l_run;
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+    if (!row_ok) return;
+    const size_t row = ((size_t)it.b * p.C + qi) * p.Hq + hq;
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    if (it.np == 1) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int col = n * 8 + 2 * cq;
+            pstore(p.out, row * D + col, (o[n][0] + o[n][2]) * inv, p.out_bf16);
+            pstore(p.out, row * D + col + 1, (o[n][1] + o[n][3]) * inv, p.out_bf16);
+        }
+    } else {
+        const size_t slot = row * p.NP + it.part;
+        float* po = p.part_o + slot * D;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int col = n * 8 + 2 * cq;
+            *reinterpret_cast<float2*>(po + col) =
+                make_float2((o[n][0] + o[n][2]) * inv, (o[n][1] + o[n][3]) * inv);
+        }
+        if (cq == 0) {
+            p.part_ml[slot * 2] = m_run;
+            p.part_ml[slot * 2 + 1] = lsum;
+        }
+    }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreadsP)
+    paged_prefill_kernel(const __grid_constant__ PrefillParams p,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v) {
+    using L = PLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
+    uint64_t* empty = full + L::STAGES;
+    uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(masks + L::STAGES);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (tid == 0) {
+        for (int s = 0; s < L::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NWP);
+        }
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == NWP && (tid & 31) == 0) {
+        prefetch_tensor_map(&tm_k);
+        prefetch_tensor_map(&tm_v);
+    }
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const PItem it = prefill_item(p);
+    __syncthreads();
+    if (it.part >= it.np) return;  // no keys in this partition (whole CTA leaves)
+    if (warp == NWP)
+        prefill_producer<D>(p, it, &tm_k, &tm_v, base, full, empty, masks, s_abort);
+    else
+        prefill_consumer<D, G>(p, it, base, full, empty, masks, s_abort);
+}
+
+// out[b, i, h, :] from the partials of the sequence's partitions (the same
+// log-sum-exp merge as the decode's combine).  One warp per (b, i, h).
+template <int D>
+__global__ void __launch_bounds__(128) prefill_combine_kernel(const __grid_constant__ PrefillParams p) {
+    grid_dependency_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);  // (b * C + i) * Hq + h
+    if (row >= (int64_t)p.B * p.C * p.Hq) return;
+    const int b = (int)(row / ((int64_t)p.C * p.Hq));
+    int L = p.context_lens[b];
+    const int maxlen = p.MB * kPageRows;
+    L = L < p.C ? 0 : (L > maxlen ? maxlen : L);
+    const int np = (L + p.P - 1) / p.P;
+    if (np <= 1) return;  // written by the attention kernel
+    const float* ml = p.part_ml + row * p.NP * 2;
+    float M = kNegInfP;
+    for (int k = lane; k < np; k += 32) M = fmaxf(M, ml[2 * k]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    constexpr int PER = D / 32;
+    float acc[PER], den = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    for (int k = 0; k < np; ++k) {
+        const float m = ml[2 * k], l = ml[2 * k + 1];
+        const float w = (m == kNegInfP || l == 0.f) ? 0.f : l * fast_exp2(m - M);
+        den += w;
+        const float* po = p.part_o + (row * p.NP + k) * D;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, po[lane + 32 * e], acc[e]);
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) pstore(p.out, row * D + lane + 32 * e, acc[e] * inv, p.out_bf16);
+}
+
+int current_device_p() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+
+template <typename K>
+cudaError_t set_smem_once(K kern, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, size_t> done;
+    const auto key = std::make_pair(reinterpret_cast<const void*>(kern), current_device_p());
+    std::lock_guard<std::mutex> lock(mu);
+    auto f = done.find(key);
+    if (f != done.end() && f->second >= smem) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) done[key] = smem;
+    return e;
+}
+
+template <int D, int G>
+cudaError_t launch_prefill_typed(const PrefillArgs& a, const CUtensorMap& tmk,
+                                 const CUtensorMap& tmv) {
+    using L = PLayout<D>;
+    auto kern = paged_prefill_kernel<D, G>;
+    cudaError_t e = set_smem_once(kern, L::SMEM);
+    if (e != cudaSuccess) return e;
+    PrefillParams p;
+    p.q = static_cast<const bf16*>(a.q);
+    p.block_tables = a.block_tables;
+    p.context_lens = a.context_lens;
+    p.out = a.out;
+    p.part_o = a.part_o;
+    p.part_ml = a.part_ml;
+    p.err = a.device_error;
+    p.B = (int)a.B;
+    p.C = (int)a.C;
+    p.Hq = (int)a.Hq;
+    p.Hkv = (int)a.Hkv;
+    p.MB = (int)a.MB;
+    p.P = a.partition_tokens;
+    p.NP = a.max_partitions;
+    p.RG = (int)((a.C * G + NWP * kRowsPerWarp - 1) / (NWP * kRowsPerWarp));
+    p.num_blocks = (int)a.num_blocks;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.out_bf16 = a.out_dtype == PKV_DTYPE_BF16;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.B * a.Hkv * p.RG * a.max_partitions));
+    cfg.blockDim = dim3(kThreadsP);
+    cfg.dynamicSmemBytes = L::SMEM;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv);
+    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+
+    cudaLaunchConfig_t cc = cfg;
+    const int64_t rows = a.B * a.C * a.Hq;
+    cc.gridDim = dim3((unsigned)((rows + 3) / 4));
+    cc.blockDim = dim3(128);
+    cc.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cc, prefill_combine_kernel<D>, p);
+}
+
+template <int D>
+cudaError_t prefill_dispatch_g(const PrefillArgs& a, const CUtensorMap& k, const CUtensorMap& v) {
+    switch (a.Hq / a.Hkv) {
+        case 1: return launch_prefill_typed<D, 1>(a, k, v);
+        case 2: return launch_prefill_typed<D, 2>(a, k, v);
+        case 4: return launch_prefill_typed<D, 4>(a, k, v);
+        case 8: return launch_prefill_typed<D, 8>(a, k, v);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_paged_prefill(const PrefillArgs& a) {
+    CUtensorMap tmk, tmv;
+    cudaError_t e = encode_cache_map(&tmk, a.k_cache, a.num_blocks, a.Hkv, a.D, PKV_DTYPE_BF16);
+    if (e != cudaSuccess) return e;
+    e = encode_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D, PKV_DTYPE_BF16);
+    if (e != cudaSuccess) return e;
+    return a.D == 64 ? prefill_dispatch_g<64>(a, tmk, tmv) : prefill_dispatch_g<128>(a, tmk, tmv);
+}
+
+}  // namespace pkv

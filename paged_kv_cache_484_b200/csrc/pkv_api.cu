@@ -501,6 +501,177 @@ pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new, const 
                          partition_tokens, flags, device_error, stream, &step);
 }
 
+}  // extern "C"
+
+// ---- chunked prefill ---------------------------------------------------------
+
+namespace pkv {
+namespace {
+constexpr int kPrefillRowsPerItem = 32;  // (query, head) rows one prefill CTA serves
+
+// Partition length of a prefill call: about two items per SM if every
+// sequence had the maximum length, in whole 128-token stages, [128, 2048].
+int32_t prefill_auto_partition(int64_t B, int64_t C, int64_t Hq, int64_t Hkv, int64_t MB) {
+    const int64_t maxlen = MB * kPageRows;
+    const int64_t G = Hq / std::max<int64_t>(1, Hkv);
+    const int64_t rg = ceil_div(C * G, kPrefillRowsPerItem);
+    const int64_t target = 2 * (int64_t)device_sm_count();
+    int64_t P = ceil_div(std::max<int64_t>(1, maxlen * B * Hkv * rg), target);
+    P = ceil_div(P, 128) * 128;
+    P = std::max<int64_t>(128, std::min<int64_t>(P, 2048));
+    const int64_t floor_np = ceil_div(ceil_div(maxlen, kMaxPartitions), kPageRows) * kPageRows;
+    return (int32_t)std::max(P, floor_np);
+}
+
+pkv_status plan_prefill(int64_t B, int64_t C, int64_t Hq, int64_t Hkv, int64_t D, int64_t MB,
+                        int32_t partition_tokens, int32_t* P_out, int32_t* NP_out,
+                        size_t* off_ml, size_t* bytes) {
+    int32_t P = partition_tokens;
+    if (P == 0) {
+        P = prefill_auto_partition(B, C, Hq, Hkv, MB);
+    } else if (P < kPageRows || P % kPageRows != 0 || P > PKV_MAX_PARTITION_TOKENS) {
+        set_last_error("partition_tokens %d must be a multiple of 16 in [16, %d]", P,
+                       PKV_MAX_PARTITION_TOKENS);
+        return PKV_ERR_INVALID_ARG;
+    }
+    const int64_t NP = std::max<int64_t>(1, ceil_div(MB * kPageRows, P));
+    if (NP > kMaxPartitions) {
+        set_last_error("max_blocks_per_seq*16 / partition_tokens = %lld partitions > %d",
+                       (long long)NP, kMaxPartitions);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    *P_out = P;
+    *NP_out = (int32_t)NP;
+    const size_t slots = NP > 1 ? (size_t)B * C * Hq * NP : 0;
+    *off_ml = align_up(slots * D * sizeof(float));
+    *bytes = slots ? *off_ml + align_up(slots * 2 * sizeof(float)) : 0;
+    return PKV_OK;
+}
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+int32_t pkv_prefill_partition_tokens(int64_t num_seqs, int64_t chunk_tokens, int64_t num_q_heads,
+                                     int64_t num_kv_heads, int64_t head_dim,
+                                     int64_t max_blocks_per_seq, int64_t block_size) {
+    if (num_seqs < 0 || chunk_tokens < 1 || max_blocks_per_seq < 0) return 0;
+    if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
+    return prefill_auto_partition(num_seqs, chunk_tokens, num_q_heads, num_kv_heads,
+                                  max_blocks_per_seq);
+}
+
+size_t pkv_prefill_workspace_size(int64_t num_seqs, int64_t chunk_tokens, int64_t num_q_heads,
+                                  int64_t num_kv_heads, int64_t head_dim,
+                                  int64_t max_blocks_per_seq, int64_t block_size,
+                                  int32_t partition_tokens) {
+    if (num_seqs < 0 || chunk_tokens < 1 || max_blocks_per_seq < 0) return 0;
+    if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
+    int32_t P, NP;
+    size_t off_ml, bytes;
+    if (plan_prefill(num_seqs, chunk_tokens, num_q_heads, num_kv_heads, head_dim,
+                     max_blocks_per_seq, partition_tokens, &P, &NP, &off_ml, &bytes) != PKV_OK)
+        return 0;
+    return bytes;
+}
+
+pkv_status pkv_paged_attention_prefill(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, const int32_t* context_lens,
+                                       void* out, void* workspace, size_t workspace_bytes,
+                                       int64_t num_seqs, int64_t chunk_tokens,
+                                       int64_t num_q_heads, int64_t num_kv_heads,
+                                       int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                                       int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                       int32_t out_dtype, float scale, int32_t partition_tokens,
+                                       int32_t* device_error, void* stream) {
+    set_last_error("");
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || chunk_tokens < 1) {
+        set_last_error("negative num_seqs or max_blocks_per_seq, or chunk_tokens < 1");
+        return PKV_ERR_INVALID_ARG;
+    }
+    pkv_status st = check_heads(num_q_heads, num_kv_heads, head_dim, block_size);
+    if (st != PKV_OK) return st;
+    if (kv_dtype != PKV_DTYPE_BF16 || !valid_dtype(out_dtype)) {
+        set_last_error("prefill: kv_dtype must be bf16; out_dtype f32 or bf16");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (num_seqs > PKV_MAX_SEQS_PER_CALL) {
+        set_last_error("num_seqs %lld > %d", (long long)num_seqs, PKV_MAX_SEQS_PER_CALL);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (chunk_tokens > max_blocks_per_seq * kPageRows && num_seqs > 0) {
+        set_last_error("chunk_tokens %lld longer than max_blocks_per_seq * 16",
+                       (long long)chunk_tokens);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (num_blocks <= 0 || num_blocks * num_kv_heads * kPageRows > INT32_MAX) {
+        set_last_error("num_blocks %lld out of range", (long long)num_blocks);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (max_blocks_per_seq * kPageRows > INT32_MAX / 2) {
+        set_last_error("max_blocks_per_seq too large");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) {
+        set_last_error("scale must be finite");
+        return PKV_ERR_INVALID_ARG;
+    }
+    int32_t P, NP;
+    size_t off_ml, need;
+    st = plan_prefill(num_seqs, chunk_tokens, num_q_heads, num_kv_heads, head_dim,
+                      max_blocks_per_seq, partition_tokens, &P, &NP, &off_ml, &need);
+    if (st != PKV_OK) return st;
+    const int64_t grid = num_seqs * num_kv_heads * NP *
+                         ceil_div(chunk_tokens * (num_q_heads / num_kv_heads), kPrefillRowsPerItem);
+    if (grid > INT32_MAX) {
+        set_last_error("prefill: too many work items");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) {
+        set_last_error("null tensor pointer");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (max_blocks_per_seq == 0) {
+        set_last_error("max_blocks_per_seq must be > 0 when num_seqs > 0");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        !aligned4(block_tables) || !aligned4(context_lens) ||
+        (device_error && !aligned4(device_error))) {
+        set_last_error("misaligned tensor pointer (16 bytes for q/caches/out)");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) {
+        set_last_error("workspace of %zu bytes given, %zu needed (16-byte aligned)",
+                       workspace ? workspace_bytes : (size_t)0, need);
+        return PKV_ERR_WORKSPACE;
+    }
+    PrefillArgs a = {};
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.out = out;
+    a.part_o = need ? static_cast<float*>(workspace) : nullptr;
+    a.part_ml = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off_ml) : nullptr;
+    a.B = num_seqs;
+    a.C = chunk_tokens;
+    a.Hq = num_q_heads;
+    a.Hkv = num_kv_heads;
+    a.D = head_dim;
+    a.num_blocks = num_blocks;
+    a.MB = max_blocks_per_seq;
+    a.out_dtype = out_dtype;
+    a.partition_tokens = P;
+    a.max_partitions = NP;
+    a.scale = scale;
+    a.device_error = device_error;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return cuda_status(launch_paged_prefill(a), "prefill launch");
+}
+
 const char* pkv_status_string(int32_t status) {
     switch (status) {
         case PKV_OK: return "ok";

@@ -1,6 +1,7 @@
 // pkv_internal.h -- declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -66,6 +67,29 @@ struct DecodeArgs {
     double theta;
 };
 cudaError_t launch_paged_decode(const DecodeArgs& a);
+
+// The cache [num_blocks, Hkv, 16, D] as a TMA tensor map of 16-row page boxes.
+cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks, int64_t Hkv,
+                             int64_t D, int32_t dtype);
+
+struct PrefillArgs {
+    const void* q;              // [B, C, Hq, D] bf16
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    void* out;                  // [B, C, Hq, D]
+    float* part_o;              // [B, C, Hq, NP, D]
+    float* part_ml;             // [B, C, Hq, NP, 2]
+    int64_t B, C, Hq, Hkv, D, num_blocks, MB;
+    int32_t out_dtype;
+    int32_t partition_tokens;   // P (resolved)
+    int32_t max_partitions;     // NP = ceil(MB * 16 / P)
+    float scale;
+    int32_t* device_error;
+    cudaStream_t stream;
+};
+cudaError_t launch_paged_prefill(const PrefillArgs& a);
 
 // Resident decode CTAs per SM for these shapes (occupancy query, cached).
 int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_t num_seqs);

@@ -140,3 +140,39 @@ def test_auto_partition_limits(lib):
         assert math.ceil(MB * 16 / P) <= 1024
     for (B, MB) in ((64, 257), (256, 2049), (16, 8193)):
         assert lib.pkv_decode_partition_tokens(B, 32, 8, 64, MB, 16, BF16) % 128 == 0
+
+
+def test_prefill_workspace_size_formula(lib):
+    # 4 sequences, chunk 8, 32/8 heads, d 64, contexts up to 129 blocks, P = 256
+    n = lib.pkv_prefill_workspace_size(4, 8, 32, 8, 64, 129, 16, 256)
+    NP = math.ceil(129 * 16 / 256)
+    slots = 4 * 8 * 32 * NP
+    a = lambda x: (x + 255) // 256 * 256
+    assert n == a(slots * 64 * 4) + a(slots * 2 * 4)
+    assert lib.pkv_prefill_workspace_size(4, 8, 32, 8, 64, 16, 16, 256) == 0   # one partition
+    assert lib.pkv_prefill_workspace_size(4, 0, 32, 8, 64, 16, 16, 256) == 0   # no chunk
+
+
+def _prefill(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, out=FAKE, ws=None, wsb=0, B=2, C=4,
+             Hq=8, Hkv=2, d=64, NB=4, bs=16, MB=4, kvdt=BF16, odt=BF16, scale=0.125, P=0,
+             err=None)
+    a.update(kw)
+    return lib.pkv_paged_attention_prefill(a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"],
+                                           a["ws"], a["wsb"], a["B"], a["C"], a["Hq"], a["Hkv"],
+                                           a["d"], a["NB"], a["bs"], a["MB"], a["kvdt"],
+                                           a["odt"], a["scale"], a["P"], a["err"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kvdt=F32), UNSUPPORTED),          # bf16 only
+    (dict(C=0), INVALID),
+    (dict(C=65), INVALID),                  # longer than max_blocks * 16
+    (dict(d=96), UNSUPPORTED),
+    (dict(P=24), INVALID),
+    (dict(q=None), INVALID),
+    (dict(P=16, MB=4), WORKSPACE),          # split: needs a workspace
+    (dict(B=0, q=None, out=None), OK),
+])
+def test_prefill_rejects_bad_arguments(lib, kw, status):
+    assert _prefill(lib, **kw) == status

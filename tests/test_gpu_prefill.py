@@ -1,0 +1,106 @@
+"""Chunked prefill (multi-query attention over the paged cache) vs the fp64
+oracle, through the C ABI (GPU only).
+
+The chunk of each sequence is the last C tokens of its context; query i
+attends to tokens 0 .. L - C + i.  The oracle computes each query as one
+plain decode over that prefix.  Bar: max-abs error <= 2e-3 (bf16 inputs,
+fp32 output), plus half a bf16 ulp when the output itself is bf16.
+"""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_484_b200 as pkv
+from paged_kv_cache_484_b200 import workloads as W
+from tests.parity_util import TOL_BF16, ulp_bf16
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _case(lens, G, Hkv, d, C, seed):
+    w = W.build_workload("prefill", lens, G * Hkv, Hkv, d, torch.bfloat16, 1e4, seed=seed,
+                         device=DEV, pool_factor=1.2)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed + 1)
+    q = torch.randn((w.B, C, w.Hq, d), generator=g, device=DEV, dtype=torch.bfloat16)
+    lens_t = w.cached_lens.clone()
+    return w, q, lens_t
+
+
+def _oracle(w, q, lens_t):
+    return oracle.paged_chunked_prefill(q.cpu(), w.k_cache.cpu(), w.v_cache.cpu(),
+                                        w.block_tables.cpu(), lens_t.cpu(), w.scale, nthreads=8)
+
+
+def _check(got, want, what, bf16_out=False):
+    got = got.double().cpu()
+    tol = torch.full_like(want, TOL_BF16)
+    if bf16_out:
+        tol = tol + 0.5 * ulp_bf16(want)
+    assert torch.isfinite(got).all(), f"{what}: non-finite output"
+    err = (got - want).abs()
+    bad = err > tol
+    assert not bad.any(), f"{what}: max err {err.max().item():.3e} at {bad.nonzero()[0].tolist()}"
+
+
+@pytest.mark.parametrize("d,G", [(64, 1), (64, 4), (64, 8), (128, 2), (128, 4)])
+@pytest.mark.parametrize("C", [1, 7, 16])
+@pytest.mark.parametrize("P", [0, 64, 512])
+def test_prefill_matches_oracle(d, G, C, P):
+    lens = [300, 16, 1000, 47, 2049][: 3 if d == 128 else 5]
+    lens = [max(L, C) for L in lens]
+    w, q, lens_t = _case(lens, G, 2, d, C, seed=300 + d + G + C)
+    out = torch.empty((w.B, C, w.Hq, d), dtype=torch.float32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.paged_attention_prefill(q, w.k_cache, w.v_cache, w.block_tables, lens_t, w.scale, out,
+                                partition_tokens=P, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    _check(out, _oracle(w, q, lens_t), f"d{d} G{G} C{C} P{P}")
+
+
+def test_prefill_many_row_groups_bf16_out():
+    """C*G = 96 rows per kv head (three row groups), bf16 output."""
+    w, q, lens_t = _case([900, 333], 4, 2, 64, 24, seed=41)
+    out = torch.empty((w.B, 24, w.Hq, 64), dtype=torch.bfloat16, device=DEV)
+    pkv.paged_attention_prefill(q, w.k_cache, w.v_cache, w.block_tables, lens_t, w.scale, out,
+                                partition_tokens=128)
+    torch.cuda.synchronize()
+    _check(out, _oracle(w, q, lens_t), "row groups, bf16 out", bf16_out=True)
+
+
+def test_prefill_whole_context_chunk_and_short_context():
+    """A chunk as long as the context (the first prefill of a prompt); a
+    context shorter than the chunk is flagged and its rows left untouched."""
+    w, q, lens_t = _case([64, 40], 4, 2, 64, 40, seed=43)
+    lens_t[0] = 40           # whole context is the chunk
+    lens_t[1] = 39           # shorter than the chunk: invalid
+    out = torch.full((w.B, 40, w.Hq, 64), 7.0, dtype=torch.float32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.paged_attention_prefill(q, w.k_cache, w.v_cache, w.block_tables, lens_t, w.scale, out,
+                                partition_tokens=16, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pkv.DEVERR_CONTEXT_LEN
+    want = _oracle(w, q[:1], lens_t[:1])
+    sub = oracle.paged_chunked_prefill(q[:1].cpu(), w.k_cache.cpu(), w.v_cache.cpu(),
+                                       w.block_tables[:1].cpu(), lens_t[:1].cpu(), w.scale)
+    _check(out[:1], sub, "whole-context chunk")
+    assert torch.equal(out[1].cpu(), torch.full_like(out[1].cpu(), 7.0))
+    del want
+
+
+def test_prefill_last_query_equals_decode():
+    """The chunk's last query sees the whole context: the same numbers as
+    the decode call up to rounding."""
+    w, q, lens_t = _case([1500, 64, 700], 4, 8, 64, 8, seed=47)
+    out = torch.empty((w.B, 8, w.Hq, 64), dtype=torch.float32, device=DEV)
+    pkv.paged_attention_prefill(q, w.k_cache, w.v_cache, w.block_tables, lens_t, w.scale, out)
+    dec = torch.empty((w.B, w.Hq, 64), dtype=torch.float32, device=DEV)
+    pkv.paged_attention_decode(q[:, -1].contiguous(), w.k_cache, w.v_cache, w.block_tables,
+                               lens_t, w.scale, dec)
+    torch.cuda.synchronize()
+    assert (out[:, -1] - dec).abs().max().item() < 1e-4

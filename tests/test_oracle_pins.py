@@ -454,6 +454,30 @@ def pin_append_then_decode_is_causal_last_row(orc: Oracle):
     assert_close(out[0], want, 1e-6, "append+decode vs causal")  # q/k rounded to f32
 
 
+def pin_chunked_prefill_matches_causal_sdpa(orc: Oracle):
+    """A prefill chunk (the last C tokens of each sequence) over the paged
+    cache equals PyTorch's fp64 causal SDPA over the gathered context, rows
+    L-C .. L-1; and a chunk of the whole context equals the oracle's own
+    full-prefix causal pass."""
+    for (Hq, Hkv, d, lens, C, seed) in [(8, 2, 16, [40, 17, 5], 5, 30),
+                                        (4, 4, 8, [33], 33, 31),
+                                        (8, 1, 16, [64, 20], 1, 32)]:
+        kpool, vpool, tables, Ks, Vs = random_paged(lens, Hkv, d, 16, torch.float32, seed)
+        B = len(lens)
+        q = torch.randn(B, C, Hq, d, generator=_gen(seed + 100))
+        scale = 1.0 / math.sqrt(d)
+        got = orc.paged_chunked_prefill(q, kpool, vpool, tables,
+                                        torch.tensor(lens, dtype=torch.int32), scale)
+        for b, L in enumerate(lens):
+            Q_all = torch.zeros(L, Hq, d, dtype=torch.float64)
+            Q_all[L - C:] = q[b].double()
+            want = sdpa(Q_all, Ks[b].double(), Vs[b].double(), scale, causal=True)[L - C:]
+            assert_close(got[b], want, 1e-12, f"chunked prefill vs causal SDPA b={b}")
+            if C == L:
+                full = orc.causal_prefill(q[b].double(), Ks[b].double(), Vs[b].double(), scale)
+                assert_close(got[b], full, 1e-12, "whole-context chunk vs causal pass")
+
+
 PINS = [
     pin_round_bf16_matches_torch_cast,
     pin_round_bf16_single_rounding,
@@ -472,6 +496,7 @@ PINS = [
     pin_append_placement_and_values,
     pin_append_rejects_out_of_range_slot,
     pin_append_then_decode_is_causal_last_row,
+    pin_chunked_prefill_matches_causal_sdpa,
 ]
 
 
