@@ -1,6 +1,6 @@
 """Pins for the fp64 CPU oracle.
 
-The oracle is what the CUDA path is judged against, so it is itself checked
+The oracle is what the CUDA path is checked against, so it is itself checked
 against things it does not compute: library routines that reduce to the same
 definition (PyTorch's fp64 scaled-dot-product attention, Hugging Face's Llama
 RoPE, PyTorch's float32->bf16 cast), closed forms of the softmax, the
