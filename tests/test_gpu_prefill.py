@@ -104,3 +104,65 @@ def test_prefill_last_query_equals_decode():
                                lens_t, w.scale, dec)
     torch.cuda.synchronize()
     assert (out[:, -1] - dec).abs().max().item() < 1e-4
+
+
+def test_prompt_chunks_then_decode_steps():
+    """A small engine loop on one paged cache: a 40-token prompt appended and
+    attended in two chunks (24 then 16 tokens), then three decode steps
+    (fused append + decode), every output against the oracle running the same
+    appends and attention on its own copy of the cache."""
+    Hq, Hkv, d, bs = 8, 2, 64, 16
+    B, NB, steps = 2, 16, 3
+    total = 40 + steps
+    g = torch.Generator()
+    g.manual_seed(53)
+    tables = torch.randperm(NB, generator=g)[: B * 4].view(B, 4).to(torch.int32)
+    kc = torch.randn(NB, Hkv, bs, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(NB, Hkv, bs, d, generator=g).to(torch.bfloat16)
+    q_all = torch.randn(B, total, Hq, d, generator=g).to(torch.bfloat16)
+    k_all = torch.randn(B, total, Hkv, d, generator=g).to(torch.bfloat16)
+    v_all = torch.randn(B, total, Hkv, d, generator=g).to(torch.bfloat16)
+    theta, scale = 1e4, 1 / 8.0
+    kc_g, vc_g, tables_g = kc.to(DEV), vc.to(DEV), tables.to(DEV)
+    kc_o, vc_o = kc.clone(), vc.clone()
+
+    def slots(pos):  # [B] int64 slot of each sequence's token at position pos
+        return (tables[:, pos // bs].to(torch.int64) * bs + pos % bs)
+
+    done = 0
+    for C in (24, 16):
+        pos = torch.arange(done, done + C, dtype=torch.int64)
+        # append the chunk: T = B*C tokens
+        q_tok = q_all[:, done:done + C].reshape(B * C, Hq, d).clone()
+        k_tok = k_all[:, done:done + C].reshape(B * C, Hkv, d).clone()
+        v_tok = v_all[:, done:done + C].reshape(B * C, Hkv, d).clone()
+        positions = pos.repeat(B)
+        slot = torch.stack([slots(p) for p in pos], 1).reshape(-1)
+        q_g = q_tok.to(DEV)
+        pkv.kv_append(q_g, k_tok.to(DEV), v_tok.to(DEV), positions.to(DEV), slot.to(DEV),
+                      kc_g, vc_g, theta)
+        q_o = q_tok.clone()
+        oracle.kv_append(q_o, k_tok.clone(), v_tok.clone(), positions, slot, kc_o, vc_o, theta)
+        done += C
+        lens = torch.full((B,), done, dtype=torch.int32)
+        out = torch.empty((B, C, Hq, d), dtype=torch.float32, device=DEV)
+        pkv.paged_attention_prefill(q_g.view(B, C, Hq, d), kc_g, vc_g, tables_g, lens.to(DEV),
+                                    scale, out, partition_tokens=16)
+        torch.cuda.synchronize()
+        want = oracle.paged_chunked_prefill(q_o.view(B, C, Hq, d), kc_o, vc_o, tables, lens,
+                                            scale)
+        _check(out, want, f"prompt chunk of {C}")
+    for s in range(steps):
+        pos = torch.full((B,), done, dtype=torch.int64)
+        slot = slots(done)
+        q_s, k_s, v_s = (t[:, done].clone() for t in (q_all, k_all, v_all))
+        lens = torch.full((B,), done + 1, dtype=torch.int32)
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=DEV)
+        pkv.decode_step(q_s.to(DEV), k_s.to(DEV), v_s.to(DEV), pos.to(DEV), slot.to(DEV), kc_g,
+                        vc_g, tables_g, lens.to(DEV), theta, scale, out)
+        torch.cuda.synchronize()
+        q_o = q_s.clone()
+        oracle.kv_append(q_o, k_s.clone(), v_s.clone(), pos, slot, kc_o, vc_o, theta)
+        want = oracle.paged_attention_decode(q_o, kc_o, vc_o, tables, lens, scale)
+        _check(out, want, f"decode step {s}")
+        done += 1
