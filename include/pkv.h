@@ -91,6 +91,8 @@ typedef enum pkv_dtype {
 #define PKV_DEVERR_BLOCK_ID 0x2u    /* block table entry outside [0, num_blocks)   */
 #define PKV_DEVERR_CONTEXT_LEN 0x4u /* context_lens[b] < 0 or > max_blocks * bs    */
 #define PKV_DEVERR_TIMEOUT 0x8u     /* a bounded in-kernel wait ran out            */
+#define PKV_DEVERR_PREFIX 0x10u     /* cascade: a group is malformed, or a member's
+                                       shared block ids differ from its group's      */
 
 /* Decode flags. */
 #define PKV_DECODE_FORCE_SIMT 0x1u  /* bf16: use the CUDA-core kernel instead of the
@@ -330,6 +332,59 @@ pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache
                                               int32_t out_dtype, float scale,
                                               int32_t partition_tokens, uint32_t flags,
                                               int32_t* device_error, void* stream);
+
+/*
+ * pkv_paged_attention_decode_cascade -- pkv_paged_attention_decode for batches
+ * whose sequences share prefix blocks (prefix caching): each shared prefix is
+ * read once for its whole group.
+ *
+ * Source: "Inference From Scratch", ch. 11 (prefix caching: requests with a
+ * common prefix reuse its KV blocks) and ch. 10 (paged attention through
+ * block tables, which is what lets several sequences point at the same
+ * physical blocks); ch. 8 (attention over a split context merges exactly
+ * through (max, sum) partials).
+ *
+ * Groups are runs of consecutive sequences: group g is sequences
+ * [group_start[g], group_start[g + 1]).  shared_tokens[b] (rounded down to
+ * whole blocks and clamped to the context) is how many leading tokens of
+ * sequence b lie in blocks its group shares: for j < shared_tokens[b] /
+ * block_size, block_tables[b, j] must equal the entry j of the group member
+ * with the most shared tokens (a mismatch sets PKV_DEVERR_PREFIX; the
+ * shared pass then reads that member's blocks).  Sequences in no group use
+ * shared_tokens[b] = 0 (and may be left out of every group).
+ *
+ * The result is that of pkv_paged_attention_decode on the same arguments
+ * (same definition, up to rounding).  Work: a shared-prefix pass runs one
+ * item per (group, kv head) whose rows are all the group's query heads over
+ * the shared pages; the decode kernel covers each sequence's remaining
+ * tokens; a combine merges both.
+ *
+ * Arguments: as pkv_paged_attention_decode, plus
+ *   group_start   device int32 [num_groups + 1], non-decreasing, <= num_seqs
+ *   shared_tokens device int32 [num_seqs]
+ *   max_group_size  the largest group_start[g + 1] - group_start[g]
+ *   workspace     >= pkv_decode_cascade_workspace_size(...) bytes, first 256
+ *                 bytes zero before its first call (as for the decode)
+ * kv_dtype must be PKV_DTYPE_BF16; num_seqs <= 256; flags 0 or
+ * PKV_DECODE_FORCE_SIMT (for the per-sequence part).  q must already be
+ * rotated (pkv_kv_append).
+ */
+pkv_status pkv_paged_attention_decode_cascade(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* group_start, const int32_t* shared_tokens,
+    void* out, void* workspace, size_t workspace_bytes, int64_t num_seqs, int64_t num_groups,
+    int64_t max_group_size, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+    int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq, int32_t kv_dtype,
+    int32_t out_dtype, float scale, int32_t partition_tokens, uint32_t flags,
+    int32_t* device_error, void* stream);
+
+/* Bytes of workspace pkv_paged_attention_decode_cascade needs: 256 bytes of
+ * scheduler counters, then num_seqs * Hq * (NP + 1) * (head_dim + 2) floats
+ * of partials.  Host only; 0 for invalid arguments. */
+size_t pkv_decode_cascade_workspace_size(int64_t num_seqs, int64_t num_q_heads,
+                                         int64_t num_kv_heads, int64_t head_dim,
+                                         int64_t max_blocks_per_seq, int64_t block_size,
+                                         int32_t kv_dtype, int32_t partition_tokens);
 
 /*
  * pkv_paged_attention_prefill -- chunked prefill: several query tokens per

@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     BLOCK_SIZE,
     DEVERR_BLOCK_ID,
     DEVERR_CONTEXT_LEN,
+    DEVERR_PREFIX,
     DEVERR_SLOT,
     DEVERR_TIMEOUT,
     LIB_PATH,
@@ -31,7 +32,9 @@ from ._binding import (  # noqa: F401
     load_library,
     new_workspace,
     paged_attention_decode,
+    paged_attention_decode_cascade,
     paged_attention_decode_noalloc,
+    decode_cascade_workspace_size,
     paged_attention_prefill,
     prefill_partition_tokens,
     prefill_workspace_size,

@@ -24,6 +24,7 @@ DEVERR_SLOT = 0x1
 DEVERR_BLOCK_ID = 0x2
 DEVERR_CONTEXT_LEN = 0x4
 DEVERR_TIMEOUT = 0x8
+DEVERR_PREFIX = 0x10
 BLOCK_SIZE = 16
 NOALLOC_SCRATCH_BYTES = 16 << 20   # PKV_NOALLOC_SCRATCH_BYTES in include/pkv.h
 
@@ -82,6 +83,12 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_prefill_workspace_size.restype = ctypes.c_size_t
         lib.pkv_prefill_partition_tokens.argtypes = [i64, i64, i64, i64, i64, i64, i64]
         lib.pkv_prefill_partition_tokens.restype = i32
+        lib.pkv_paged_attention_decode_cascade.argtypes = [
+            vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64,
+            i64, i64, i64, i32, i32, ctypes.c_float, i32, u32, vp, vp]
+        lib.pkv_paged_attention_decode_cascade.restype = ctypes.c_int
+        lib.pkv_decode_cascade_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32]
+        lib.pkv_decode_cascade_workspace_size.restype = ctypes.c_size_t
         lib.pkv_status_string.argtypes = [i32]
         lib.pkv_status_string.restype = ctypes.c_char_p
         lib.pkv_last_error.argtypes = []
@@ -368,4 +375,54 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, sca
         B, C, Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16, _dtype_code(out.dtype), float(scale),
         int(partition_tokens), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_prefill")
+    return out
+
+
+def decode_cascade_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                  max_blocks_per_seq, partition_tokens=0,
+                                  block_size=BLOCK_SIZE) -> int:
+    """Bytes of workspace ``paged_attention_decode_cascade`` needs."""
+    lib = load_library()
+    return int(lib.pkv_decode_cascade_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                                                     head_dim, max_blocks_per_seq, block_size,
+                                                     PKV_DTYPE_BF16, int(partition_tokens)))
+
+
+def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, group_start,
+                                   shared_tokens, max_group_size, scale, out, stream=None, *,
+                                   workspace=None, partition_tokens=0, force_simt=False,
+                                   device_error=None) -> torch.Tensor:
+    """``paged_attention_decode`` for groups of sequences that share prefix
+    blocks: group g is sequences [group_start[g], group_start[g+1]) (int32,
+    device), whose first shared_tokens[b] tokens (int32 [B], device) sit in
+    the group's shared blocks.  Same result; each shared prefix is read once
+    per group.  bf16 only; q already rotated.  See include/pkv.h."""
+    lib = load_library()
+    if q.dtype != torch.bfloat16 or k_cache.dtype != torch.bfloat16 \
+            or v_cache.dtype != torch.bfloat16:
+        raise TypeError("cascade: q and the caches must be bfloat16")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    NG = max(0, group_start.numel() - 1)
+    if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, Hq, d) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,) \
+            or shared_tokens.shape != (B,):
+        raise ValueError("inconsistent paged_attention_decode_cascade shapes")
+    need = lib.pkv_decode_cascade_workspace_size(B, Hq, Hkv, d, MB, bs, PKV_DTYPE_BF16,
+                                                 int(partition_tokens))
+    if workspace is None:
+        workspace = new_workspace(int(need), q.device)
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_paged_attention_decode_cascade(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32),
+        _dev(group_start, "group_start", torch.int32) if NG else None,
+        _dev(shared_tokens, "shared_tokens", torch.int32), _dev(out, "out"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        B, NG, int(max_group_size), Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16,
+        _dtype_code(out.dtype), float(scale), int(partition_tokens),
+        _flags(force_simt, True), err, _stream_ptr(stream, q.device))
+    _raise(st, lib, "paged_attention_decode_cascade")
     return out

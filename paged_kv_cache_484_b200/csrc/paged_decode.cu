@@ -63,6 +63,8 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // (shortest) partition after all full ones, longest first, so that the
 // work that finishes last is short.
 constexpr int kLptMaxSeqs = 256;
+// cascade offsets live in the longest-first arrays' shared memory
+static_assert(kCascadeMaxSeqs <= kLptMaxSeqs, "cascade offsets need the rank arrays");
 
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
@@ -138,6 +140,10 @@ struct DecodeParams {
     // partition r, and the cluster merges the partials in shared memory
     // (no workspace partials, no combine kernel); 0 = off
     int cluster;
+    // cascade: the first shared_tokens[b] tokens of sequence b are attended by
+    // the shared-prefix pass (partial slot 0); this kernel takes the rest,
+    // in partitions that start at that offset (slots 1..); null = off
+    const int32_t* shared_tokens;
     // fused step only: the new token of every sequence
     const void* k_new;            // [B, Hkv, D]
     const void* v_new;            // [B, Hkv, D]
@@ -153,6 +159,7 @@ struct RopeFreq {
 
 struct Item {
     int b, h, part, t0, t1, npages, np;
+    int slot0;  // cascade: 1 when the sequence's shared prefix owns partial slot 0
 };
 
 // Item i -> (sequence, kv head, partition).  Items are j * Hkv + h.  Without
@@ -166,7 +173,7 @@ __device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const 
     const int j = i / p.Hkv;
     it.h = i - j * p.Hkv;
     const int nfull = s_pre[p.B];
-    if (p.B <= kLptMaxSeqs && !p.cluster && j >= nfull) {
+    if (p.B <= kLptMaxSeqs && !p.cluster && !p.shared_tokens && j >= nfull) {
         const int* s_rank = s_pre + p.B + 1;
         it.b = s_rank[j - nfull];
         it.np = (s_len[it.b] + p.P - 1) / p.P;
@@ -182,7 +189,15 @@ __device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const 
         it.part = j - s_pre[lo];
         it.np = (s_len[lo] + p.P - 1) / p.P;
     }
-    it.t0 = it.part * p.P;
+    int off = 0;
+    it.slot0 = 0;
+    if (p.shared_tokens) {
+        // cascade: partitions start after the tokens of the shared-prefix pass
+        off = (s_pre + p.B + 1)[it.b];
+        it.np = (s_len[it.b] - off + p.P - 1) / p.P;
+        it.slot0 = off > 0 ? 1 : 0;
+    }
+    it.t0 = off + it.part * p.P;
     it.t1 = min(s_len[it.b], it.t0 + p.P);
     it.npages = (it.t1 - it.t0 + kPageRows - 1) / kPageRows;
     return it;
@@ -616,10 +631,10 @@ __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Ite
                 part[D] = M;
                 part[D + 1] = den;
             }
-        } else if (it.np == 1) {
+        } else if (it.np == 1 && it.slot0 == 0) {
             store_out(p.out, hq * D + dim, val, p.out_bf16);
         } else {
-            const size_t slot = hq * p.NP + it.part;
+            const size_t slot = hq * p.NP + it.slot0 + it.part;
             p.part_o[slot * D + dim] = val;
             if (dim == 0) {
                 p.part_ml[slot * 2] = M;
@@ -1239,7 +1254,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
             bs = j / p.NP;
             ps = j - bs * p.NP;
         }
-        if (bs < p.B) {
+        if (bs < p.B && !p.shared_tokens) {
             const int jb = ps * (p.P / kPageRows) + lane;
             guess.b = bs;
             guess.part = ps;
@@ -1258,7 +1273,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     // Partition counts per sequence and their exclusive prefix (block scan);
     // in the longest-first order only the partitions before the last one.
     const int B = p.B;
-    const bool lpt = B <= kLptMaxSeqs && !p.cluster;
+    const bool lpt = B <= kLptMaxSeqs && !p.cluster && !p.shared_tokens;
     const int maxlen = p.MB * kPageRows;
     const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
     const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
@@ -1272,7 +1287,14 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
             Lb = Lb < 0 ? 0 : maxlen;
         }
         s_len[b] = Lb;
-        const int npb = (Lb + p.P - 1) / p.P;
+        int off = 0;
+        if (p.shared_tokens) {
+            // cascade (at most kLptMaxSeqs sequences): whole pages, within the context
+            off = p.shared_tokens[b];
+            off = off < 0 ? 0 : (off > Lb ? Lb : off) / kPageRows * kPageRows;
+            s_rank[b] = off;
+        }
+        const int npb = (Lb - off + p.P - 1) / p.P;
         const int cnt = lpt ? max(npb - 1, 0) : npb;
         if (lpt) s_key[b] = Lb > 0 ? Lb - (npb - 1) * p.P : -1;  // tokens of the last partition
         s_pre[b] = cnt;
@@ -1352,6 +1374,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
 
 struct CombineParams {
     const int32_t* context_lens;
+    const int32_t* shared_tokens;  // cascade: slot 0 holds the shared-prefix partial
     const float* part_o;
     const float* part_ml;
     void* out;
@@ -1400,8 +1423,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_c
         }
     }
     Lb = Lb < 0 ? 0 : (Lb > maxlen ? maxlen : Lb);
-    const int np = (Lb + p.P - 1) / p.P;
-    if (np <= 1) return;
+    int off = 0;
+    if (p.shared_tokens) {
+        off = p.shared_tokens[b];
+        off = off < 0 ? 0 : (off > Lb ? Lb : off) / kPageRows * kPageRows;
+    }
+    // slots: the shared prefix (cascade, when it has tokens), then the partitions
+    const int np = (off > 0 ? 1 : 0) + (Lb - off + p.P - 1) / p.P;
+    if (np <= 1 && off == 0) return;  // written by the decode kernel
 
     // first partials of this thread, independent of the weights
     const int ch = threadIdx.x % CH, pg = threadIdx.x / CH;
@@ -1593,6 +1622,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     p.part_o = a.part_o;
     p.part_ml = a.part_ml;
     p.sched = a.sched;
+    p.shared_tokens = a.shared_tokens;
     p.err = a.device_error;
     p.B = (int)a.B;
     p.Hq = (int)a.Hq;
@@ -1621,7 +1651,8 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     // and the combine kernel is not needed.
     int cs = 0;
     const size_t smem_cl = std::max(smem, kClusterCtaSmem);
-    if (a.allow_cluster && a.max_partitions >= 2 && a.max_partitions <= kMaxClusterCtas) {
+    if (a.allow_cluster && !a.shared_tokens && a.max_partitions >= 2 &&
+        a.max_partitions <= kMaxClusterCtas) {
         int nc = 0;
         e = max_active_clusters(kern, smem_cl, a.max_partitions, &nc);
         if (e != cudaSuccess) return e;
@@ -1653,6 +1684,10 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     cfg.numAttrs = cs ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv, fr);
     if (e != cudaSuccess || a.max_partitions <= 1 || cs) return e;
+    if (a.launch_between) {
+        e = a.launch_between(a.between_ctx);
+        if (e != cudaSuccess) return e;
+    }
 
     CombineParams cp;
     cp.context_lens = a.context_lens;
@@ -1664,6 +1699,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     cp.P = a.partition_tokens;
     cp.NP = a.max_partitions;
     cp.out_bf16 = p.out_bf16;
+    cp.shared_tokens = a.shared_tokens;
     auto ckern = combine_kernel<D, G>;
     {
         static std::mutex mu;

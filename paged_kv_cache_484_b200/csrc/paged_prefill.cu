@@ -186,27 +186,35 @@ __device__ void prefill_producer(const PrefillParams& p, const PItem& it, const 
     }
 }
 
-template <int D, int G>
-__device__ void prefill_consumer(const PrefillParams& p, const PItem& it, uint8_t* base,
-                                 uint64_t* full, uint64_t* empty, const uint32_t* masks,
-                                 volatile int* s_abort) {
+// One query row of a consumer lane (lanes 4r .. 4r+3 of a warp share row r).
+struct PRow {
+    bool ok;            // the row exists
+    const bf16* q;      // its query vector (D elements)
+    int len;            // it may attend to tokens t < len
+    bool direct;        // write the output row (else a partition partial)
+    void* out;          // direct: the output row (D elements of out_bf16 ? bf16 : f32)
+    float* po;          // partial: o (D floats)
+    float* pml;         // partial: (m, l)
+};
+
+// A consumer warp runs its 8 rows over every page of the item's key range
+// [t0, t1): S = Q K^T and O += P V on the tensor cores, online softmax per
+// row in the log2 domain, keys at t >= row.len masked per row.
+template <int D>
+__device__ void multirow_consumer(float scale_log2, int out_bf16, int32_t* err, const PItem& it,
+                                  const PRow& row, uint8_t* base, uint64_t* full, uint64_t* empty,
+                                  const uint32_t* masks, volatile int* s_abort) {
     using L = PLayout<D>;
     constexpr int KS = D / 16, NT = D / 8;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = lane >> 2, cq = lane & 3;
-    // this lane's row: (query i, head g) of the item's row group
-    const int fr = it.rg * (NWP * kRowsPerWarp) + warp * kRowsPerWarp + r;
-    const bool row_ok = fr < p.C * G;
-    const int qi = row_ok ? fr / G : 0, g = row_ok ? fr % G : 0;
-    const int hq = it.h * G + g;
-    // keys this row may see: 0 .. L - C + qi
-    const int row_len = row_ok ? it.L - p.C + qi + 1 : 0;
+    const int lane = threadIdx.x & 31;
+    const int cq = lane & 3;
+    const bool row_ok = row.ok;
+    const int row_len = row_ok ? row.len : 0;
 
     // A fragments of Q: rows r and r + 8 both hold this lane's row
     uint32_t qa[KS][2];
     {
-        const uint32_t* qr = reinterpret_cast<const uint32_t*>(
-            p.q + (((size_t)it.b * p.C + qi) * p.Hq + hq) * D);
+        const uint32_t* qr = reinterpret_cast<const uint32_t*>(row.q);
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
             const int col = kk * 16 + 2 * cq;
@@ -253,7 +261,7 @@ __device__ void prefill_consumer(const PrefillParams& p, const PItem& it, uint8_
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int tk = n * 8 + 2 * cq + e;
-                    x[n][e] = tk < row_valid ? sc[n][e] * p.scale_log2 : kNegInfP;
+                    x[n][e] = tk < row_valid ? sc[n][e] * scale_log2 : kNegInfP;
                 }
             float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -315,7 +323,7 @@ __device__ void prefill_consumer(const PrefillParams& p, const PItem& it, uint8_
     }
     if (!ok) {
         *s_abort = 1;
-        if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
+        if (lane == 0) report_error(err, PKV_DEVERR_TIMEOUT);
         return;
     }
     // row result: high + low rows, row sum over the quad
@@ -323,27 +331,24 @@ __device__ void prefill_consumer(const PrefillParams& p, const PItem& it, uint8_
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
     if (!row_ok) return;
-    const size_t row = ((size_t)it.b * p.C + qi) * p.Hq + hq;
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    if (it.np == 1) {
+    if (row.direct) {
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const int col = n * 8 + 2 * cq;
-            pstore(p.out, row * D + col, (o[n][0] + o[n][2]) * inv, p.out_bf16);
-            pstore(p.out, row * D + col + 1, (o[n][1] + o[n][3]) * inv, p.out_bf16);
+            pstore(row.out, col, (o[n][0] + o[n][2]) * inv, out_bf16);
+            pstore(row.out, col + 1, (o[n][1] + o[n][3]) * inv, out_bf16);
         }
     } else {
-        const size_t slot = row * p.NP + it.part;
-        float* po = p.part_o + slot * D;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const int col = n * 8 + 2 * cq;
-            *reinterpret_cast<float2*>(po + col) =
+            *reinterpret_cast<float2*>(row.po + col) =
                 make_float2((o[n][0] + o[n][2]) * inv, (o[n][1] + o[n][3]) * inv);
         }
         if (cq == 0) {
-            p.part_ml[slot * 2] = m_run;
-            p.part_ml[slot * 2 + 1] = lsum;
+            row.pml[0] = m_run;
+            row.pml[1] = lsum;
         }
     }
 }
@@ -379,10 +384,26 @@ __global__ void __launch_bounds__(kThreadsP)
     const PItem it = prefill_item(p);
     __syncthreads();
     if (it.part >= it.np) return;  // no keys in this partition (whole CTA leaves)
-    if (warp == NWP)
+    if (warp == NWP) {
         prefill_producer<D>(p, it, &tm_k, &tm_v, base, full, empty, masks, s_abort);
-    else
-        prefill_consumer<D, G>(p, it, base, full, empty, masks, s_abort);
+        return;
+    }
+    // this lane's row: (query i, head g) of the item's row group; query i
+    // sees tokens 0 .. L - C + i
+    PRow row;
+    const int fr = it.rg * (NWP * kRowsPerWarp) + warp * kRowsPerWarp + ((tid & 31) >> 2);
+    row.ok = fr < p.C * G;
+    const int qi = row.ok ? fr / G : 0, hq = it.h * G + (row.ok ? fr % G : 0);
+    const size_t r = ((size_t)it.b * p.C + qi) * p.Hq + hq;
+    row.q = p.q + r * D;
+    row.len = it.L - p.C + qi + 1;
+    row.direct = it.np == 1;
+    row.out = p.out_bf16 ? (void*)(reinterpret_cast<bf16*>(p.out) + r * D)
+                         : (void*)(reinterpret_cast<float*>(p.out) + r * D);
+    row.po = p.part_o ? p.part_o + (r * p.NP + it.part) * D : nullptr;
+    row.pml = p.part_ml ? p.part_ml + (r * p.NP + it.part) * 2 : nullptr;
+    multirow_consumer<D>(p.scale_log2, p.out_bf16, p.err, it, row, base, full, empty, masks,
+                         s_abort);
 }
 
 // out[b, i, h, :] from the partials of the sequence's partitions (the same
@@ -419,6 +440,146 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const __grid_const
     const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) pstore(p.out, row * D + lane + 32 * e, acc[e] * inv, p.out_bf16);
+}
+
+// ---- cascade decode: the shared-prefix pass ----------------------------------
+
+struct CascadeParams {
+    const bf16* q;                  // [B, Hq, D], rotated (kv_append ran before)
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* group_start;     // [NG + 1]: group g = sequences [gs[g], gs[g + 1])
+    const int32_t* shared_tokens;   // [B]
+    float* part_o;                  // decode workspace partials: NPT slots per (b, q head)
+    float* part_ml;
+    int32_t* err;
+    int B, Hq, Hkv, MB, NPT, RG, NG, num_blocks;
+    float scale_log2;
+};
+
+// Shared tokens of sequence b as the decode counts them: whole pages inside
+// its (clamped) context.
+__device__ __forceinline__ int cascade_shared(const CascadeParams& p, int b) {
+    int L = p.context_lens[b];
+    const int maxlen = p.MB * kPageRows;
+    L = L < 0 ? 0 : (L > maxlen ? maxlen : L);
+    int s = p.shared_tokens[b];
+    return s < 0 ? 0 : (s > L ? L : s) / kPageRows * kPageRows;
+}
+
+// One CTA per (group, kv head, row group): the rows are (member, head)
+// pairs, member m of the group and head g -> row m*G + g; every row attends
+// to the first shared_tokens of its own sequence, read once for the group
+// from the pages of the member that shares the most (the others' shared
+// block-table entries must be the same ids: a mismatch sets
+// PKV_DEVERR_PREFIX).  The result goes to partial slot 0 of each member;
+// the decode kernel writes the rest of the sequence to slots 1.. and the
+// combine merges them.  The kernel does not wait for the decode kernel before
+// it starts (it reads nothing the decode writes), so its CTAs fill SMs as the
+// decode's CTAs finish; each CTA waits for the decode grid before it exits,
+// so that the combine, which waits for this grid, also sees the decode's
+// partials.
+template <int D, int G>
+__global__ void __launch_bounds__(kThreadsP)
+    cascade_prefix_kernel(const __grid_constant__ CascadeParams p,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v) {
+    using L = PLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
+    uint64_t* empty = full + L::STAGES;
+    uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(masks + L::STAGES);
+    __shared__ int s_grp[3];  // first member, member count, leader
+    __shared__ int s_len;     // the leader's shared tokens
+    const int tid = threadIdx.x, warp = tid >> 5;
+    grid_launch_dependents();
+    int x = blockIdx.x;
+    const int rg = x % p.RG;
+    x /= p.RG;
+    const int h = x % p.Hkv, g = x / p.Hkv;
+    if (tid == 0) {
+        for (int s = 0; s < L::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NWP);
+        }
+        *s_abort = 0;
+        fence_barrier_init();
+        int gs = p.group_start[g], ge = p.group_start[g + 1];
+        if (gs < 0 || ge < gs || ge > p.B) {
+            report_error(p.err, PKV_DEVERR_PREFIX);
+            gs = ge = 0;
+        }
+        int best = 0, leader = gs;
+        for (int b = gs; b < ge; ++b) {
+            const int sb = cascade_shared(p, b);
+            if (sb > best) {
+                best = sb;
+                leader = b;
+            }
+        }
+        s_grp[0] = gs;
+        s_grp[1] = ge - gs;
+        s_grp[2] = leader;
+        s_len = best;
+    }
+    __syncthreads();
+    const int gs = s_grp[0], nmem = s_grp[1], leader = s_grp[2], S = s_len;
+    if (S > 0) {
+        if (warp == NWP && (tid & 31) == 0) {
+            prefetch_tensor_map(&tm_k);
+            prefetch_tensor_map(&tm_v);
+        }
+        // every member's shared pages must be the leader's (checked once, by row group 0)
+        if (rg == 0 && h == 0) {
+            for (int idx = tid; idx < nmem * (S / kPageRows); idx += kThreadsP) {
+                const int m = idx / (S / kPageRows), j = idx - m * (S / kPageRows);
+                const int b = gs + m;
+                if (j < cascade_shared(p, b) / kPageRows &&
+                    p.block_tables[(size_t)b * p.MB + j] != p.block_tables[(size_t)leader * p.MB + j])
+                    report_error(p.err, PKV_DEVERR_PREFIX);
+            }
+        }
+        PItem it;
+        it.b = leader;
+        it.h = h;
+        it.rg = rg;
+        it.part = 0;
+        it.L = S;
+        it.np = 1;
+        it.t0 = 0;
+        it.t1 = S;
+        it.npages = S / kPageRows;
+        PrefillParams pp;  // the fields the page producer reads
+        pp.block_tables = p.block_tables;
+        pp.err = p.err;
+        pp.MB = p.MB;
+        pp.Hkv = p.Hkv;
+        pp.num_blocks = p.num_blocks;
+        if (warp == NWP) {
+            prefill_producer<D>(pp, it, &tm_k, &tm_v, base, full, empty, masks, s_abort);
+        } else {
+            PRow row;
+            const int fr = rg * (NWP * kRowsPerWarp) + warp * kRowsPerWarp + ((tid & 31) >> 2);
+            const int m = fr / G, hq = h * G + fr % G;
+            const int b = gs + m;
+            row.ok = m < nmem;
+            row.len = row.ok ? cascade_shared(p, b) : 0;
+            row.ok = row.ok && row.len > 0;  // no shared tokens: no slot 0
+            const size_t r = (size_t)(row.ok ? b : 0) * p.Hq + hq;
+            row.q = p.q + r * D;
+            row.direct = false;
+            row.out = nullptr;
+            row.po = p.part_o + (r * p.NPT) * D;
+            row.pml = p.part_ml + (r * p.NPT) * 2;
+            multirow_consumer<D>(p.scale_log2, 0, p.err, it, row, base, full, empty, masks,
+                                 s_abort);
+        }
+    }
+    // do not complete before the decode grid: the combine waits for this one
+    if ((tid & 31) == 0) grid_dependency_wait();
 }
 
 int current_device_p() {
@@ -499,7 +660,66 @@ cudaError_t prefill_dispatch_g(const PrefillArgs& a, const CUtensorMap& k, const
     return cudaErrorInvalidValue;
 }
 
+template <int D, int G>
+cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
+                                 const CUtensorMap& tmv) {
+    using L = PLayout<D>;
+    auto kern = cascade_prefix_kernel<D, G>;
+    cudaError_t e = set_smem_once(kern, L::SMEM);
+    if (e != cudaSuccess) return e;
+    CascadeParams p;
+    p.q = static_cast<const bf16*>(a.q);
+    p.block_tables = a.block_tables;
+    p.context_lens = a.context_lens;
+    p.group_start = a.group_start;
+    p.shared_tokens = a.shared_tokens;
+    p.part_o = a.part_o;
+    p.part_ml = a.part_ml;
+    p.err = a.device_error;
+    p.B = (int)a.B;
+    p.Hq = (int)a.Hq;
+    p.Hkv = (int)a.Hkv;
+    p.MB = (int)a.MB;
+    p.NPT = a.slots_per_row;
+    p.RG = (int)((a.max_group_size * G + NWP * kRowsPerWarp - 1) / (NWP * kRowsPerWarp));
+    p.NG = (int)a.num_groups;
+    p.num_blocks = (int)a.num_blocks;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.num_groups * a.Hkv * p.RG));
+    cfg.blockDim = dim3(kThreadsP);
+    cfg.dynamicSmemBytes = L::SMEM;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv);
+}
+
+template <int D>
+cudaError_t cascade_dispatch_g(const CascadeArgs& a, const CUtensorMap& k, const CUtensorMap& v) {
+    switch (a.Hq / a.Hkv) {
+        case 1: return launch_cascade_typed<D, 1>(a, k, v);
+        case 2: return launch_cascade_typed<D, 2>(a, k, v);
+        case 4: return launch_cascade_typed<D, 4>(a, k, v);
+        case 8: return launch_cascade_typed<D, 8>(a, k, v);
+    }
+    return cudaErrorInvalidValue;
+}
+
 }  // namespace
+
+cudaError_t launch_cascade_prefix(const CascadeArgs& a) {
+    if (a.num_groups <= 0) return cudaSuccess;
+    CUtensorMap tmk, tmv;
+    cudaError_t e = encode_cache_map(&tmk, a.k_cache, a.num_blocks, a.Hkv, a.D, PKV_DTYPE_BF16);
+    if (e != cudaSuccess) return e;
+    e = encode_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D, PKV_DTYPE_BF16);
+    if (e != cudaSuccess) return e;
+    return a.D == 64 ? cascade_dispatch_g<64>(a, tmk, tmv) : cascade_dispatch_g<128>(a, tmk, tmv);
+}
 
 cudaError_t launch_paged_prefill(const PrefillArgs& a) {
     CUtensorMap tmk, tmv;

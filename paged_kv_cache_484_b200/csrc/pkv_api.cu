@@ -503,6 +503,176 @@ pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new, const 
 
 }  // extern "C"
 
+// ---- cascade decode ----------------------------------------------------------
+
+namespace pkv {
+namespace {
+cudaError_t launch_cascade_between(const void* ctx) {
+    return launch_cascade_prefix(*static_cast<const CascadeArgs*>(ctx));
+}
+
+// Workspace of a cascade call: the scheduler counters, then NP + 1 partial
+// slots per (sequence, q head) -- slot 0 for the shared prefix.
+pkv_status plan_cascade(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t MB,
+                        int32_t kv_dtype, int32_t partition_tokens, WorkspacePlan* w,
+                        int32_t* slots_per_row) {
+    pkv_status st = plan_workspace(B, Hq, Hkv, D, MB, kv_dtype, partition_tokens, w);
+    if (st != PKV_OK) return st;
+    if (w->NP + 1 > kMaxPartitions) {
+        set_last_error("cascade: at most %d partitions per sequence", kMaxPartitions - 1);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    *slots_per_row = w->NP + 1;
+    const size_t slots = (size_t)B * Hq * (w->NP + 1);
+    w->off_o = kSchedBytes;
+    w->off_ml = w->off_o + align_up(slots * D * sizeof(float));
+    w->bytes = w->off_ml + align_up(slots * 2 * sizeof(float));
+    return PKV_OK;
+}
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+size_t pkv_decode_cascade_workspace_size(int64_t num_seqs, int64_t num_q_heads,
+                                         int64_t num_kv_heads, int64_t head_dim,
+                                         int64_t max_blocks_per_seq, int64_t block_size,
+                                         int32_t kv_dtype, int32_t partition_tokens) {
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || kv_dtype != PKV_DTYPE_BF16) return 0;
+    if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
+    WorkspacePlan w;
+    int32_t npt;
+    if (plan_cascade(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, kv_dtype,
+                     partition_tokens, &w, &npt) != PKV_OK)
+        return 0;
+    return w.bytes;
+}
+
+pkv_status pkv_paged_attention_decode_cascade(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* group_start, const int32_t* shared_tokens,
+    void* out, void* workspace, size_t workspace_bytes, int64_t num_seqs, int64_t num_groups,
+    int64_t max_group_size, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+    int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq, int32_t kv_dtype,
+    int32_t out_dtype, float scale, int32_t partition_tokens, uint32_t flags,
+    int32_t* device_error, void* stream) {
+    set_last_error("");
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || num_groups < 0) {
+        set_last_error("negative num_seqs, num_groups or max_blocks_per_seq");
+        return PKV_ERR_INVALID_ARG;
+    }
+    pkv_status st = check_heads(num_q_heads, num_kv_heads, head_dim, block_size);
+    if (st != PKV_OK) return st;
+    if (kv_dtype != PKV_DTYPE_BF16 || !valid_dtype(out_dtype)) {
+        set_last_error("cascade: kv_dtype must be bf16; out_dtype f32 or bf16");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if ((flags & ~PKV_DECODE_FORCE_SIMT) != 0) {
+        set_last_error("cascade: unknown flags 0x%x", flags);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (num_seqs > kCascadeMaxSeqs) {
+        set_last_error("cascade: num_seqs %lld > %d", (long long)num_seqs, kCascadeMaxSeqs);
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (num_groups > 0 && (max_group_size < 1 || max_group_size > num_seqs ||
+                           num_groups * num_kv_heads *
+                                   ceil_div(max_group_size * (num_q_heads / num_kv_heads), 32) >
+                               INT32_MAX)) {
+        set_last_error("cascade: max_group_size %lld out of range", (long long)max_group_size);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (num_blocks <= 0 || num_blocks * num_kv_heads * kPageRows > INT32_MAX) {
+        set_last_error("num_blocks %lld out of range", (long long)num_blocks);
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) {
+        set_last_error("scale must be finite");
+        return PKV_ERR_INVALID_ARG;
+    }
+    WorkspacePlan w;
+    int32_t npt;
+    st = plan_cascade(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, kv_dtype,
+                      partition_tokens, &w, &npt);
+    if (st != PKV_OK) return st;
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !shared_tokens ||
+        (num_groups > 0 && !group_start)) {
+        set_last_error("null tensor pointer");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (max_blocks_per_seq == 0) {
+        set_last_error("max_blocks_per_seq must be > 0 when num_seqs > 0");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        !aligned4(block_tables) || !aligned4(context_lens) || !aligned4(shared_tokens) ||
+        (group_start && !aligned4(group_start)) || (device_error && !aligned4(device_error))) {
+        set_last_error("misaligned tensor pointer");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (!workspace || workspace_bytes < w.bytes || !aligned16(workspace)) {
+        set_last_error("workspace of %zu bytes given, %zu needed (16-byte aligned)",
+                       workspace ? workspace_bytes : (size_t)0, w.bytes);
+        return PKV_ERR_WORKSPACE;
+    }
+    char* ws = static_cast<char*>(workspace);
+    CascadeArgs c = {};
+    c.q = q;
+    c.k_cache = k_cache;
+    c.v_cache = v_cache;
+    c.block_tables = block_tables;
+    c.context_lens = context_lens;
+    c.group_start = group_start;
+    c.shared_tokens = shared_tokens;
+    c.part_o = reinterpret_cast<float*>(ws + w.off_o);
+    c.part_ml = reinterpret_cast<float*>(ws + w.off_ml);
+    c.B = num_seqs;
+    c.Hq = num_q_heads;
+    c.Hkv = num_kv_heads;
+    c.D = head_dim;
+    c.num_blocks = num_blocks;
+    c.MB = max_blocks_per_seq;
+    c.num_groups = num_groups;
+    c.max_group_size = max_group_size;
+    c.slots_per_row = npt;
+    c.scale = scale;
+    c.device_error = device_error;
+    c.stream = static_cast<cudaStream_t>(stream);
+
+    DecodeArgs a = {};
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.out = out;
+    a.sched = reinterpret_cast<uint32_t*>(ws);
+    a.part_o = c.part_o;
+    a.part_ml = c.part_ml;
+    a.B = num_seqs;
+    a.Hq = num_q_heads;
+    a.Hkv = num_kv_heads;
+    a.D = head_dim;
+    a.num_blocks = num_blocks;
+    a.MB = max_blocks_per_seq;
+    a.kv_dtype = kv_dtype;
+    a.out_dtype = out_dtype;
+    a.partition_tokens = w.P;
+    a.max_partitions = npt;   // the slot stride: the shared slot, then the partitions
+    a.scale = scale;
+    a.force_simt = (flags & PKV_DECODE_FORCE_SIMT) != 0;
+    a.allow_cluster = false;
+    a.shared_tokens = shared_tokens;
+    a.launch_between = launch_cascade_between;
+    a.between_ctx = &c;
+    a.device_error = device_error;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return cuda_status(launch_paged_decode(a), "cascade decode launch");
+}
+
+}  // extern "C"
+
 // ---- chunked prefill ---------------------------------------------------------
 
 namespace pkv {

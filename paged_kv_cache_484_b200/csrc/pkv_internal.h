@@ -15,6 +15,7 @@ constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;  // + one producer war
 constexpr int kStageTokens = kConsumerWarps * kPageRows;   // one page per consumer warp
 constexpr int kMaxPartitions = 1024;
 constexpr int kMaxClusterCtas = 16;  // cluster-mode limit (non-portable above 8)
+constexpr int kCascadeMaxSeqs = 256;  // cascade decode keeps per-sequence offsets in shared memory
 
 // Per-thread detail of the last failing call (returned by pkv_last_error).
 void set_last_error(const char* fmt, ...);
@@ -52,6 +53,12 @@ struct DecodeArgs {
     float scale;
     bool force_simt;
     bool allow_cluster;  // split contexts may merge inside a thread-block cluster
+    // cascade: tokens of each sequence attended by the shared-prefix pass
+    // (partial slot 0), and that pass's launch, made between the decode
+    // kernel and the combine; null = no cascade
+    const int32_t* shared_tokens;
+    cudaError_t (*launch_between)(const void* ctx);
+    const void* between_ctx;
     // planning only: launch nothing, store the number of kernels the call
     // would launch (1 or 2) in *launches
     bool plan_only;
@@ -90,6 +97,26 @@ struct PrefillArgs {
     cudaStream_t stream;
 };
 cudaError_t launch_paged_prefill(const PrefillArgs& a);
+
+// Cascade decode, shared-prefix pass (launched between the decode kernel and
+// the combine).
+struct CascadeArgs {
+    const void* q;                  // [B, Hq, D] bf16, rotated
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* group_start;     // [num_groups + 1]
+    const int32_t* shared_tokens;   // [B]
+    float* part_o;
+    float* part_ml;
+    int64_t B, Hq, Hkv, D, num_blocks, MB, num_groups, max_group_size;
+    int32_t slots_per_row;          // partial slots per (sequence, q head): 1 + NP
+    float scale;
+    int32_t* device_error;
+    cudaStream_t stream;
+};
+cudaError_t launch_cascade_prefix(const CascadeArgs& a);
 
 // Resident decode CTAs per SM for these shapes (occupancy query, cached).
 int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_t num_seqs);
