@@ -64,6 +64,9 @@ def parse_args(argv=None):
     ap.add_argument("--two-calls", action="store_true",
                     help="time kv_append + paged_attention_decode as two launches instead of "
                          "the single-launch decode_step")
+    ap.add_argument("--cascade", action="store_true",
+                    help="two calls, the decode as paged_attention_decode_cascade over the "
+                         "workload's prefix groups (config 4)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
@@ -345,6 +348,20 @@ def run_ours(args):
         copies.append(dict((f, getattr(w, f).clone()) for f in fields))
     outs = [torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=device) for _ in range(ncopies)]
 
+    cascade = args.cascade
+    if cascade:
+        if w.meta.get("prefix_group", 0) <= 1:
+            raise SystemExit("--cascade needs a workload with prefix groups (config 4)")
+        args.two_calls = True
+        grp = int(w.meta["prefix_group"])
+        group_start = torch.tensor(list(range(0, w.B, grp)) + [w.B], dtype=torch.int32,
+                                   device=device)
+        cached = w.cached_lens.to(torch.int64)
+        shared_tokens = (torch.minimum(cached // 16,
+                                       torch.full_like(cached, w.meta["prefix_tokens"] // 16))
+                         * 16).to(torch.int32)
+        ws = pkv.new_workspace(pkv.decode_cascade_workspace_size(
+            w.B, w.Hq, w.Hkv, w.d, w.max_blocks, partition_tokens=P), device)
     fused = not args.two_calls
     # decode kernel, plus the partition combine unless the split contexts
     # are merged inside thread-block clusters (the library decides)
@@ -353,6 +370,8 @@ def run_ours(args):
                                              force_simt=args.simt, fused=fused)
     if kernels_per_decode not in (1, 2):
         raise SystemExit("decode_launches: no answer from the library")
+    if cascade:
+        kernels_per_decode = 3     # decode, shared-prefix pass, combine
     launches_per_step = kernels_per_decode + (0 if fused else 1)
 
     def append(c):
@@ -366,6 +385,12 @@ def run_ours(args):
                             c["k_cache"], c["v_cache"], c["block_tables"], c["decode_lens"],
                             w.rope_theta, w.scale, out, workspace=ws, partition_tokens=P,
                             force_simt=args.simt, device_error=err)
+        elif cascade:
+            pkv.paged_attention_decode_cascade(c["q"], c["k_cache"], c["v_cache"],
+                                               c["block_tables"], c["decode_lens"], group_start,
+                                               shared_tokens, grp, w.scale, out, workspace=ws,
+                                               partition_tokens=P, force_simt=args.simt,
+                                               device_error=err)
         else:
             pkv.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
                                        c["decode_lens"], w.scale, out, workspace=ws,
@@ -543,6 +568,8 @@ def run_ours(args):
         "pct_of_hbm_peak": round(100.0 * value / (world * peak), 2),
         "seq_steps_per_s": round(world * w.B / (step_ms_max * 1e-3), 1),
         "config": dict(config_block(args.config, w, out_dtype, P, NP, args.simt, args.two_calls),
+                       **({"step": "two calls (kv_append, paged_attention_decode_cascade over "
+                                   "the prefix groups)"} if cascade else {}),
                        l2=(f"inputs larger than L2 ({l2 >> 20} MiB): " +
                            (f"{ncopies} device-side copies of the workload, step k on copy k mod "
                             f"{ncopies} ({nbytes / 1e6:.1f} MB read per step)" if ncopies > 1 else
@@ -555,10 +582,13 @@ def run_ours(args):
                           "how": "L2 flushed before each step, each step between its own "
                                  "pair of events"},
         "roofline": {"bound": "hbm",
-                     "kernel": ("decode_step" if fused else "paged_attention_decode")
-                     + " call: paged_decode_kernel" + (" + combine_kernel" if kernels_per_decode == 2
-                                                        else (" (partitions merged in thread-block "
-                                                              "clusters)" if NP > 1 else "")),
+                     "kernel": ("paged_attention_decode_cascade call: paged_decode_kernel + "
+                                "cascade_prefix_kernel + combine_kernel") if cascade else
+                               (("decode_step" if fused else "paged_attention_decode")
+                                + " call: paged_decode_kernel" +
+                                (" + combine_kernel" if kernels_per_decode == 2
+                                 else (" (partitions merged in thread-block clusters)"
+                                       if NP > 1 else ""))),
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "decode_ms": round(decode_ms_max, 5),
