@@ -445,6 +445,63 @@ int32_t pkv_prefill_partition_tokens(int64_t num_seqs, int64_t chunk_tokens, int
                                      int64_t num_kv_heads, int64_t head_dim,
                                      int64_t max_blocks_per_seq, int64_t block_size);
 
+/*
+ * Block manager: the host side of a paged KV cache -- which physical blocks
+ * each sequence owns, with prefix caching and eviction.
+ *
+ * Source: "Inference From Scratch", ch. 10 (block pool, block tables, slot
+ * mapping) and ch. 11 (prefix caching, hash-based reuse of the KV blocks of
+ * a common prefix); "The Project: Serve Your Own LLM", M13c (a pool smaller
+ * than the worst case, so the engine must preempt).
+ *
+ * A full block (block_size tokens) is published under its tokens and the
+ * blocks before it; a later sequence whose prompt starts with the same
+ * tokens reuses those blocks (exact token comparison: no false sharing).
+ * Blocks are reference counted; a published block nobody uses stays cached
+ * until the pool needs it (least recently released first).  A partial last
+ * block is always private.  Host memory only, no CUDA; not thread safe.
+ * Statuses: PKV_ERR_INVALID_ARG (bad handle, unknown or duplicate sequence,
+ * short output buffer), PKV_ERR_WORKSPACE (out of blocks: free a sequence,
+ * i.e. preempt, and retry; nothing was allocated).
+ */
+typedef struct pkv_block_manager pkv_block_manager;
+
+/* A manager of num_blocks blocks of block_size tokens; NULL on error. */
+pkv_block_manager* pkv_bm_create(int32_t num_blocks, int32_t block_size);
+void pkv_bm_destroy(pkv_block_manager* bm);
+
+/* Admit a sequence with its prompt's token ids (host memory).  Cached blocks
+ * covering the longest run of whole prompt blocks are reused;
+ * *shared_tokens (may be NULL) receives the number of prompt tokens they
+ * hold, whose K/V need not be computed again. */
+pkv_status pkv_bm_add_sequence(pkv_block_manager* bm, int64_t seq_id, const int32_t* tokens,
+                               int64_t num_tokens, int32_t* shared_tokens);
+
+/* Cache slot (block * block_size + row) of every prompt token of seq_id, -1
+ * for tokens in reused blocks (pkv_kv_append skips negative slots). */
+pkv_status pkv_bm_prompt_slots(const pkv_block_manager* bm, int64_t seq_id, int64_t* slots,
+                               int64_t max_tokens);
+
+/* Append one generated token: *slot receives its cache slot (a new block is
+ * taken when the last one is full; a block that becomes full is published). */
+pkv_status pkv_bm_append(pkv_block_manager* bm, int64_t seq_id, int32_t token, int64_t* slot);
+
+/* Release a finished or preempted sequence's blocks. */
+pkv_status pkv_bm_free_sequence(pkv_block_manager* bm, int64_t seq_id);
+
+/* The sequence's block table row (padded with -1 to max_blocks), its block
+ * count and token count; table may be NULL to query the counts. */
+pkv_status pkv_bm_block_table(const pkv_block_manager* bm, int64_t seq_id, int32_t* table,
+                              int32_t max_blocks, int32_t* num_blocks, int64_t* num_tokens);
+
+/* Prompt tokens the sequence found in cached blocks (-1: unknown sequence). */
+int32_t pkv_bm_shared_tokens(const pkv_block_manager* bm, int64_t seq_id);
+
+/* Blocks available to new tokens (free + cached but unused), and cached
+ * (published) blocks; -1 for a NULL handle. */
+int32_t pkv_bm_free_blocks(const pkv_block_manager* bm);
+int32_t pkv_bm_cached_blocks(const pkv_block_manager* bm);
+
 /* Short text for a status code (static storage). */
 const char* pkv_status_string(int32_t status);
 

@@ -15,6 +15,7 @@ first use and its absence is an error, never a fallback.
 """
 from ._binding import (  # noqa: F401
     BLOCK_SIZE,
+    BlockManager,
     DEVERR_BLOCK_ID,
     DEVERR_CONTEXT_LEN,
     DEVERR_PREFIX,

@@ -89,6 +89,26 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_paged_attention_decode_cascade.restype = ctypes.c_int
         lib.pkv_decode_cascade_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32]
         lib.pkv_decode_cascade_workspace_size.restype = ctypes.c_size_t
+        lib.pkv_bm_create.argtypes = [i32, i32]
+        lib.pkv_bm_create.restype = vp
+        lib.pkv_bm_destroy.argtypes = [vp]
+        lib.pkv_bm_destroy.restype = None
+        lib.pkv_bm_add_sequence.argtypes = [vp, i64, vp, i64, vp]
+        lib.pkv_bm_add_sequence.restype = ctypes.c_int
+        lib.pkv_bm_prompt_slots.argtypes = [vp, i64, vp, i64]
+        lib.pkv_bm_prompt_slots.restype = ctypes.c_int
+        lib.pkv_bm_append.argtypes = [vp, i64, i32, vp]
+        lib.pkv_bm_append.restype = ctypes.c_int
+        lib.pkv_bm_free_sequence.argtypes = [vp, i64]
+        lib.pkv_bm_free_sequence.restype = ctypes.c_int
+        lib.pkv_bm_block_table.argtypes = [vp, i64, vp, i32, vp, vp]
+        lib.pkv_bm_block_table.restype = ctypes.c_int
+        lib.pkv_bm_shared_tokens.argtypes = [vp, i64]
+        lib.pkv_bm_shared_tokens.restype = i32
+        lib.pkv_bm_free_blocks.argtypes = [vp]
+        lib.pkv_bm_free_blocks.restype = i32
+        lib.pkv_bm_cached_blocks.argtypes = [vp]
+        lib.pkv_bm_cached_blocks.restype = i32
         lib.pkv_status_string.argtypes = [i32]
         lib.pkv_status_string.restype = ctypes.c_char_p
         lib.pkv_last_error.argtypes = []
@@ -426,3 +446,74 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_le
         _flags(force_simt, True), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode_cascade")
     return out
+
+
+class BlockManager:
+    """Host-side block allocator of a paged KV cache with prefix caching (the
+    library's pkv_bm_* calls; see include/pkv.h).  Not thread safe."""
+
+    def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE):
+        self._lib = load_library()
+        self._h = self._lib.pkv_bm_create(int(num_blocks), int(block_size))
+        if not self._h:
+            raise PkvError(1, f"pkv_bm_create: {self._lib.pkv_last_error().decode()}")
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+
+    def close(self):
+        if self._h:
+            self._lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_sequence(self, seq_id: int, tokens) -> int:
+        """Admit a sequence with its prompt token ids; returns how many of its
+        leading tokens sit in reused (cached) blocks."""
+        t = torch.as_tensor(tokens, dtype=torch.int32).contiguous()
+        shared = ctypes.c_int32(0)
+        _raise(self._lib.pkv_bm_add_sequence(self._h, int(seq_id), t.data_ptr() if t.numel() else None,
+                                             t.numel(), ctypes.byref(shared)),
+               self._lib, "pkv_bm_add_sequence")
+        return int(shared.value)
+
+    def prompt_slots(self, seq_id: int, num_tokens: int) -> torch.Tensor:
+        """int64 [num_tokens] cache slot of each prompt token, -1 when reused."""
+        out = torch.empty(int(num_tokens), dtype=torch.int64)
+        _raise(self._lib.pkv_bm_prompt_slots(self._h, int(seq_id), out.data_ptr(), out.numel()),
+               self._lib, "pkv_bm_prompt_slots")
+        return out
+
+    def append(self, seq_id: int, token: int) -> int:
+        """Cache slot of the sequence's next token."""
+        slot = ctypes.c_int64(0)
+        _raise(self._lib.pkv_bm_append(self._h, int(seq_id), int(token), ctypes.byref(slot)),
+               self._lib, "pkv_bm_append")
+        return int(slot.value)
+
+    def free_sequence(self, seq_id: int) -> None:
+        _raise(self._lib.pkv_bm_free_sequence(self._h, int(seq_id)), self._lib,
+               "pkv_bm_free_sequence")
+
+    def block_table(self, seq_id: int, max_blocks: int) -> tuple[torch.Tensor, int]:
+        """(int32 [max_blocks] table row padded with -1, number of tokens)."""
+        row = torch.empty(int(max_blocks), dtype=torch.int32)
+        nb, nt = ctypes.c_int32(0), ctypes.c_int64(0)
+        _raise(self._lib.pkv_bm_block_table(self._h, int(seq_id), row.data_ptr(), row.numel(),
+                                            ctypes.byref(nb), ctypes.byref(nt)),
+               self._lib, "pkv_bm_block_table")
+        return row, int(nt.value)
+
+    def shared_tokens(self, seq_id: int) -> int:
+        return int(self._lib.pkv_bm_shared_tokens(self._h, int(seq_id)))
+
+    @property
+    def free_blocks(self) -> int:
+        return int(self._lib.pkv_bm_free_blocks(self._h))
+
+    @property
+    def cached_blocks(self) -> int:
+        return int(self._lib.pkv_bm_cached_blocks(self._h))

@@ -1,7 +1,8 @@
 """Build the sm_100a CUDA library ``_lib/libpkv.so`` in the source tree.
 
 nvcc cross-compiles for sm_100a without a GPU, so this runs anywhere the CUDA
-toolkit is installed.  Each ``csrc/*.cu`` file is compiled in parallel to an
+toolkit is installed.  Each ``csrc/*.cu`` file (and the host-only
+``csrc/*.cpp``, through nvcc's host compiler) is compiled in parallel to an
 object under ``_build/`` and the objects are linked into one shared library
 with the CUDA runtime linked statically (the library then depends only on
 the driver).  The build is skipped when the library is newer than every
@@ -37,7 +38,7 @@ def nvcc() -> str:
 
 
 def sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():
@@ -53,9 +54,9 @@ def up_to_date() -> bool:
 
 
 def _compile(src: str, verbose_ptxas: bool) -> str:
-    obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
+    obj = os.path.join(BUILD_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
     cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
-    if verbose_ptxas:
+    if verbose_ptxas and src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     log = os.path.join(BUILD_DIR, os.path.basename(src) + ".log")
