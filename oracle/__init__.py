@@ -15,6 +15,11 @@ Functions (all take and return CPU ``torch`` tensors):
   decode over its own causal prefix of the paged cache.
 * ``contiguous_decode`` / ``causal_prefill`` -- the same definition without
   paging, used only to check the oracle itself.
+* ``kv_append_e4m3`` / ``paged_attention_decode_e4m3`` -- the same append and
+  decode over an 8-bit (E4M3 code x per-tensor scale) cache, whose V pages
+  are stored transposed: k_cache [NB, Hkv, 16, d], v_cache [NB, Hkv, d, 16],
+  both uint8.
+* ``round_e4m3`` / ``e4m3_to_double`` -- the E4M3 rounding and decoding.
 * ``rope`` / ``round_bf16`` / ``bf16_to_double`` -- the oracle's building blocks,
   exposed so that tests can pin them.
 """
@@ -26,7 +31,7 @@ import torch
 
 from . import build as _build
 
-F32, BF16 = 0, 1
+F32, BF16, E4M3 = 0, 1, 2
 _ERRORS = {
     -1: "invalid argument",
     -2: "block id out of range",
@@ -65,10 +70,19 @@ class Oracle:
             lib.orc_paged_decode.argtypes = [i32, i32, vp, vp, vp, vp, vp,
                                              i64, i64, i64, i64, i64, i64, i64, dbl,
                                              vp, i64, i32, vp]
+            lib.orc_paged_decode_e4m3.argtypes = [i32, vp, vp, vp, vp, vp,
+                                                  i64, i64, i64, i64, i64, i64, i64, dbl, dbl,
+                                                  dbl, vp, i64, i32, vp]
+            lib.orc_kv_append_e4m3.argtypes = [i32, vp, vp, vp, vp, vp, vp, vp,
+                                               i64, i64, i64, i64, i64, i64, dbl, dbl, dbl]
+            lib.orc_round_e4m3.argtypes = [vp, vp, i64]
+            lib.orc_e4m3_to_double.argtypes = [vp, vp, i64]
             lib.orc_contiguous_decode.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, vp]
             lib.orc_causal_prefill.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, vp]
             for name in ("orc_round_bf16", "orc_bf16_to_double", "orc_rope", "orc_kv_append",
-                         "orc_paged_decode", "orc_contiguous_decode", "orc_causal_prefill"):
+                         "orc_paged_decode", "orc_contiguous_decode", "orc_causal_prefill",
+                         "orc_paged_decode_e4m3", "orc_kv_append_e4m3", "orc_round_e4m3",
+                         "orc_e4m3_to_double"):
                 getattr(lib, name).restype = ctypes.c_int
             self._lib = lib
         return self._lib
@@ -84,6 +98,20 @@ class Oracle:
         x = _cpu(x.contiguous(), torch.bfloat16)
         out = torch.empty(x.shape, dtype=torch.float64)
         _check(self.lib.orc_bf16_to_double(_ptr(x), _ptr(out), x.numel()))
+        return out
+
+    def round_e4m3(self, x: torch.Tensor) -> torch.Tensor:
+        """uint8 E4M3 codes of float64 values: nearest, ties to even, saturating
+        to +-448 (no binary32 step: that belongs to the cache quantizer)."""
+        x = _cpu(x.contiguous(), torch.float64)
+        out = torch.empty(x.shape, dtype=torch.uint8)
+        _check(self.lib.orc_round_e4m3(_ptr(x), _ptr(out), x.numel()))
+        return out
+
+    def e4m3_to_double(self, c: torch.Tensor) -> torch.Tensor:
+        c = _cpu(c.contiguous(), torch.uint8)
+        out = torch.empty(c.shape, dtype=torch.float64)
+        _check(self.lib.orc_e4m3_to_double(_ptr(c), _ptr(out), c.numel()))
         return out
 
     def rope(self, x: torch.Tensor, positions: torch.Tensor, theta: float) -> torch.Tensor:
@@ -141,6 +169,60 @@ class Oracle:
                                          _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                          _ptr(context_lens), B, Hq, Hkv, d, NB, bs, MB,
                                          float(scale), pp, npairs, int(nthreads), _ptr(out)))
+        return out
+
+    def kv_append_e4m3(self, q, k_new, v_new, positions, slot_mapping, k_cache, v_cache,
+                       rope_theta, k_scale, v_scale):
+        """In-place: rotate q (its own dtype); write the E4M3 codes of rotated
+        k / k_scale and of v / v_scale into the slots.  q, k_new, v_new share
+        one dtype (float32 or bfloat16); k_cache [NB, Hkv, bs, d] and v_cache
+        [NB, Hkv, d, bs] are uint8."""
+        for t in (q, k_new, v_new, k_cache, v_cache):
+            _cpu(t)
+        dt = _storage_code(q)
+        for t in (k_new, v_new):
+            if t.dtype != q.dtype:
+                raise TypeError("q, k_new and v_new share one dtype")
+        for t in (k_cache, v_cache):
+            if t.dtype != torch.uint8:
+                raise TypeError("E4M3 caches are uint8")
+        _cpu(positions, torch.int64)
+        _cpu(slot_mapping, torch.int64)
+        T, Hq, d = q.shape
+        NB, Hkv, bs, _ = k_cache.shape
+        if v_cache.shape != (NB, Hkv, d, bs):
+            raise ValueError("v_cache must be [NB, Hkv, d, bs]")
+        _check(self.lib.orc_kv_append_e4m3(dt, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(positions),
+                                           _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+                                           T, Hq, Hkv, d, NB, bs, float(rope_theta),
+                                           float(k_scale), float(v_scale)))
+
+    def paged_attention_decode_e4m3(self, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                    k_scale, v_scale, pairs=None,
+                                    nthreads: int = 1) -> torch.Tensor:
+        """fp64 [B, Hq, d] decode over an E4M3 cache (k_cache [NB, Hkv, bs, d],
+        v_cache [NB, Hkv, d, bs], uint8); ``pairs`` as in paged_attention_decode."""
+        _cpu(q)
+        _cpu(k_cache, torch.uint8)
+        _cpu(v_cache, torch.uint8)
+        _cpu(block_tables, torch.int32)
+        _cpu(context_lens, torch.int32)
+        B, Hq, d = q.shape
+        NB, Hkv, bs, _ = k_cache.shape
+        if v_cache.shape != (NB, Hkv, d, bs):
+            raise ValueError("v_cache must be [NB, Hkv, d, bs]")
+        MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+        out = torch.full((B, Hq, d), float("nan"), dtype=torch.float64)
+        if pairs is not None:
+            pairs = _cpu(pairs.contiguous(), torch.int64)
+            pp, npairs = _ptr(pairs), pairs.shape[0]
+        else:
+            pp, npairs = None, 0
+        _check(self.lib.orc_paged_decode_e4m3(_storage_code(q), _ptr(q), _ptr(k_cache),
+                                              _ptr(v_cache), _ptr(block_tables),
+                                              _ptr(context_lens), B, Hq, Hkv, d, NB, bs, MB,
+                                              float(scale), float(k_scale), float(v_scale), pp,
+                                              npairs, int(nthreads), _ptr(out)))
         return out
 
     def paged_chunked_prefill(self, q, k_cache, v_cache, block_tables, context_lens, scale,
@@ -222,3 +304,7 @@ paged_attention_decode = default.paged_attention_decode
 contiguous_decode = default.contiguous_decode
 causal_prefill = default.causal_prefill
 paged_chunked_prefill = default.paged_chunked_prefill
+round_e4m3 = default.round_e4m3
+e4m3_to_double = default.e4m3_to_double
+kv_append_e4m3 = default.kv_append_e4m3
+paged_attention_decode_e4m3 = default.paged_attention_decode_e4m3

@@ -14,7 +14,10 @@
  *     plain two-pass definition: no online softmax, no split, no blocking;
  *   - two self-check variants of the same definition: attention over a
  *     contiguous K/V array (orc_contiguous_decode) and full-prefix causal
- *     attention over a whole sequence (orc_causal_prefill).
+ *     attention over a whole sequence (orc_causal_prefill);
+ *   - the same append and decode over an 8-bit floating-point cache
+ *     (orc_kv_append_e4m3, orc_paged_decode_e4m3): each cached element is an
+ *     E4M3 code times a per-tensor scale.
  *
  * Sources:
  *   [BOOK]    "Inference From Scratch" (book intro), "What you will build" and
@@ -31,7 +34,14 @@
  *   [WARP]    "warpllama", Milestones: static KV cache + single-token decode,
  *             fused RoPE kernel.
  *   [EFF]     "Efficient LLM Inference", "KV Caching: Verify Reuse, Positions
- *             and Windows" (chunked computation equals a full-prefix pass).
+ *             and Windows" (chunked computation equals a full-prefix pass);
+ *             "Quantization: From Rounding Errors to Model-quality Limits"
+ *             (values rounded to a small set of levels with a scale) and
+ *             "Verify Exact Execution and Approximate Quality Separately".
+ *   [OFP8]    The E4M3 format itself is not on the pages; it is the public
+ *             OCP 8-bit floating point format: 1 sign bit, 4 exponent bits
+ *             (bias 7), 3 mantissa bits, no infinities, S.1111.111 = NaN,
+ *             largest finite value 448, subnormals m * 2^-9.
  *
  * Readings where the pages are silent (all stated once here):
  *   - RoPE pairs element i with element i + d/2 ("rotate half", the Llama
@@ -44,6 +54,12 @@
  *     s % block_size.  A negative slot means "do not write this token".
  *   - Query head h reads kv head h / (Hq / Hkv) (contiguous groups).
  *   - A context of length 0 produces an all-zero output row.
+ *   - 8-bit cache: one scale per tensor (k_scale, v_scale); the stored code
+ *     of a value x is x / scale (fp64) rounded to binary32, then to the
+ *     nearest E4M3 value, ties to even, saturating to +-448.  The binary32
+ *     step is the precision the GPU takes that decision in.  V pages of this
+ *     cache are stored transposed, [num_blocks][num_kv_heads][head_dim]
+ *     [block_size]; K pages keep the [block_size][head_dim] row layout.
  *
  * Floating point: every input is converted exactly to double; all sums and
  * exponentials are in double.  Build with plain -O2 (no fast-math).
@@ -56,6 +72,7 @@
 
 #define ORC_F32 0
 #define ORC_BF16 1
+#define ORC_E4M3 2
 
 #define ORC_OK 0
 #define ORC_EARG (-1)
@@ -122,6 +139,65 @@ int orc_bf16_to_double(const uint16_t* x, double* out, int64_t n) {
     return ORC_OK;
 }
 
+/* ---- E4M3 ([OFP8]; [EFF] quantization) ---------------------------------- */
+
+/* The value a code stands for, straight from the format's definition. */
+static double e4m3_to_double(uint8_t c) {
+    int neg = c >> 7, E = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (E == 15 && m == 7) return NAN;
+    if (E == 0)
+        v = ldexp((double)m, -9);           /* subnormal: m * 2^-9 */
+    else
+        v = ldexp(1.0 + m / 8.0, E - 7);   /* normal: 1.m * 2^(E-7) */
+    return neg ? -v : v;
+}
+
+/* Nearest E4M3 value of x, ties to even, saturating: like double_to_bf16,
+ * scale by the spacing of the representable values in x's binade (2^-9 for
+ * everything below 2^-5, where subnormals and the first normal binade share
+ * that spacing), round to an integer, scale back; anything that rounds
+ * above 448 (the largest finite value) becomes 448.  NaN maps to S.1111.111. */
+static uint8_t double_to_e4m3(double x) {
+    if (isnan(x)) return (uint8_t)0x7F;
+    uint8_t sign = signbit(x) ? (uint8_t)0x80 : (uint8_t)0;
+    double a = fabs(x);
+    double r = 448.0;
+    if (!isinf(a)) {
+        int e = 0;
+        if (a > 0.0) (void)frexp(a, &e); /* a in [2^(e-1), 2^e) */
+        int spacing_exp = (e - 1) - 3;   /* 3 stored mantissa bits */
+        if (spacing_exp < -9) spacing_exp = -9;
+        r = ldexp(nearbyint(ldexp(a, -spacing_exp)), spacing_exp);
+        if (r > 448.0) r = 448.0;
+    }
+    if (r < ldexp(1.0, -6)) return (uint8_t)(sign | (uint8_t)ldexp(r, 9)); /* 0 .. 7 */
+    int er;
+    double f = frexp(r, &er);                 /* r = f * 2^er, f in [0.5, 1) */
+    int E = er - 1 + 7;                       /* biased exponent, 1 .. 15 */
+    int m = (int)((2.0 * f - 1.0) * 8.0);     /* exact: r has 4 significant bits */
+    return (uint8_t)(sign | (uint8_t)(E << 3) | (uint8_t)m);
+}
+
+/* The stored code of x under `scale`: x / scale rounded to binary32, then to
+ * E4M3 (the binary32 value is exact in double, so the second rounding is the
+ * correctly rounded E4M3 value of that binary32 number). */
+static uint8_t quantize_e4m3(double x, double scale) {
+    return double_to_e4m3((double)(float)(x / scale));
+}
+
+int orc_e4m3_to_double(const uint8_t* c, double* out, int64_t n) {
+    if (n < 0 || (n > 0 && (!c || !out))) return ORC_EARG;
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_double(c[i]);
+    return ORC_OK;
+}
+
+int orc_round_e4m3(const double* x, uint8_t* out, int64_t n) {
+    if (n < 0 || (n > 0 && (!x || !out))) return ORC_EARG;
+    for (int64_t i = 0; i < n; ++i) out[i] = double_to_e4m3(x[i]);
+    return ORC_OK;
+}
+
 /* ---- RoPE ([LIFS] Architecture overview; [WARP] Milestones) ------------- */
 
 /* Rotate one head vector x[0..d) in place for integer position pos:
@@ -156,6 +232,17 @@ int orc_rope(double* x, int64_t n, int64_t d, const int64_t* positions, double t
  *     v_cache[slot / bs, h, slot % bs, :] <- v_new[t, h, :]        (h < Hkv)
  * q, k_new, v_new, k_cache and v_cache all have storage type `dtype`.
  * Every slot is validated before anything is written. */
+/* q[t, h, :] <- round(rope(q[t, h, :], pos)) for every query head h. */
+static void rotate_q_token(void* q, int dtype, int64_t t, int64_t Hq, int64_t d, int64_t pos,
+                           double theta, double* row) {
+    for (int64_t h = 0; h < Hq; ++h) {
+        int64_t base = (t * Hq + h) * d;
+        for (int64_t i = 0; i < d; ++i) row[i] = load_elem(q, dtype, base + i);
+        rope_rotate(row, d, pos, theta);
+        for (int64_t i = 0; i < d; ++i) store_elem(q, dtype, base + i, row[i]);
+    }
+}
+
 int orc_kv_append(int dtype, void* q, const void* k_new, const void* v_new,
                   const int64_t* positions, const int64_t* slot_mapping,
                   void* k_cache, void* v_cache,
@@ -174,12 +261,7 @@ int orc_kv_append(int dtype, void* q, const void* k_new, const void* v_new,
     if (!row) return ORC_ENOMEM;
     for (int64_t t = 0; t < T; ++t) {
         int64_t pos = positions[t];
-        for (int64_t h = 0; h < Hq; ++h) {
-            int64_t base = (t * Hq + h) * d;
-            for (int64_t i = 0; i < d; ++i) row[i] = load_elem(q, dtype, base + i);
-            rope_rotate(row, d, pos, theta);
-            for (int64_t i = 0; i < d; ++i) store_elem(q, dtype, base + i, row[i]);
-        }
+        rotate_q_token(q, dtype, t, Hq, d, pos, theta, row);
         int64_t slot = slot_mapping[t];
         if (slot < 0) continue;
         int64_t blk = slot / bs, off = slot % bs;
@@ -194,6 +276,50 @@ int orc_kv_append(int dtype, void* q, const void* k_new, const void* v_new,
                 memcpy((float*)v_cache + dst, (const float*)v_new + src, (size_t)d * 4);
             else
                 memcpy((uint16_t*)v_cache + dst, (const uint16_t*)v_new + src, (size_t)d * 2);
+        }
+    }
+    free(row);
+    return ORC_OK;
+}
+
+/* The same append into an E4M3 cache ([EFF] quantization; [OFP8]):
+ *   q[t, h, :] <- round(rope(q[t, h, :]))  in q's storage type `dtype`
+ *   if slot >= 0, for h < Hkv and i < d:
+ *     k_cache[blk, h, off, i] <- code(rope(k_new[t, h, :])[i] / k_scale)
+ *     v_cache[blk, h, i, off] <- code(v_new[t, h, i] / v_scale)    (transposed)
+ * where code() is quantize_e4m3 (binary32, then nearest E4M3, saturating). */
+int orc_kv_append_e4m3(int dtype, void* q, const void* k_new, const void* v_new,
+                       const int64_t* positions, const int64_t* slot_mapping,
+                       uint8_t* k_cache, uint8_t* v_cache,
+                       int64_t T, int64_t Hq, int64_t Hkv, int64_t d,
+                       int64_t num_blocks, int64_t bs, double theta,
+                       double k_scale, double v_scale) {
+    if (dtype != ORC_F32 && dtype != ORC_BF16) return ORC_EARG;
+    if (T < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || (d % 2) != 0 || num_blocks <= 0 || bs <= 0)
+        return ORC_EARG;
+    if (!(k_scale > 0.0) || !(v_scale > 0.0) || isinf(k_scale) || isinf(v_scale)) return ORC_EARG;
+    if (T == 0) return ORC_OK;
+    if (!q || !k_new || !v_new || !positions || !slot_mapping || !k_cache || !v_cache)
+        return ORC_EARG;
+    for (int64_t t = 0; t < T; ++t)
+        if (slot_mapping[t] >= num_blocks * bs) return ORC_ESLOT;
+
+    double* row = (double*)malloc((size_t)d * sizeof(double));
+    if (!row) return ORC_ENOMEM;
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t pos = positions[t];
+        rotate_q_token(q, dtype, t, Hq, d, pos, theta, row);
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t blk = slot / bs, r = slot % bs; /* block, row within the page */
+        for (int64_t h = 0; h < Hkv; ++h) {
+            int64_t src = (t * Hkv + h) * d;
+            int64_t page = (blk * Hkv + h) * bs * d;
+            for (int64_t i = 0; i < d; ++i) row[i] = load_elem(k_new, dtype, src + i);
+            rope_rotate(row, d, pos, theta);
+            for (int64_t i = 0; i < d; ++i) k_cache[page + r * d + i] = quantize_e4m3(row[i], k_scale);
+            for (int64_t i = 0; i < d; ++i)
+                v_cache[page + i * bs + r] = quantize_e4m3(load_elem(v_new, dtype, src + i), v_scale);
         }
     }
     free(row);
@@ -215,12 +341,30 @@ typedef struct {
     const int32_t *block_tables, *context_lens;
     int64_t B, Hq, Hkv, d, num_blocks, bs, MB;
     double scale;
+    double k_scale, v_scale; /* E4M3 cache only */
     const int64_t* pairs; /* optional list of (b, h) pairs */
     int64_t npairs;
     double* out;
     int nthreads, tid;
     int status;
 } decode_job;
+
+/* Element i of cached token `row` (block blk, kv head kvh).  K pages are
+ * [bs][d]; V pages are [bs][d] too, except in the E4M3 cache ([d][bs]). */
+static double k_elem(const decode_job* J, int64_t blk, int64_t kvh, int64_t row, int64_t i) {
+    int64_t idx = ((blk * J->Hkv + kvh) * J->bs + row) * J->d + i;
+    if (J->kv_dtype == ORC_E4M3)
+        return e4m3_to_double(((const uint8_t*)J->k_cache)[idx]) * J->k_scale;
+    return load_elem(J->k_cache, J->kv_dtype, idx);
+}
+
+static double v_elem(const decode_job* J, int64_t blk, int64_t kvh, int64_t row, int64_t i) {
+    if (J->kv_dtype == ORC_E4M3) {
+        int64_t idx = ((blk * J->Hkv + kvh) * J->d + i) * J->bs + row;
+        return e4m3_to_double(((const uint8_t*)J->v_cache)[idx]) * J->v_scale;
+    }
+    return load_elem(J->v_cache, J->kv_dtype, ((blk * J->Hkv + kvh) * J->bs + row) * J->d + i);
+}
 
 static int decode_one(const decode_job* J, int64_t b, int64_t h, double* s) {
     const int64_t G = J->Hq / J->Hkv, d = J->d;
@@ -235,11 +379,9 @@ static int decode_one(const decode_job* J, int64_t b, int64_t h, double* s) {
     for (int64_t t = 0; t < L; ++t) {
         int64_t blk = J->block_tables[b * J->MB + t / J->bs];
         if (blk < 0 || blk >= J->num_blocks) return ORC_EBLOCK;
-        int64_t kbase = ((blk * J->Hkv + kvh) * J->bs + t % J->bs) * d;
         double acc = 0.0;
         for (int64_t i = 0; i < d; ++i)
-            acc += load_elem(J->q, J->q_dtype, qbase + i) *
-                   load_elem(J->k_cache, J->kv_dtype, kbase + i);
+            acc += load_elem(J->q, J->q_dtype, qbase + i) * k_elem(J, blk, kvh, t % J->bs, i);
         s[t] = J->scale * acc;
         if (s[t] > M) M = s[t];
     }
@@ -248,8 +390,7 @@ static int decode_one(const decode_job* J, int64_t b, int64_t h, double* s) {
         double w = exp(s[t] - M);
         den += w;
         int64_t blk = J->block_tables[b * J->MB + t / J->bs];
-        int64_t vbase = ((blk * J->Hkv + kvh) * J->bs + t % J->bs) * d;
-        for (int64_t i = 0; i < d; ++i) o[i] += w * load_elem(J->v_cache, J->kv_dtype, vbase + i);
+        for (int64_t i = 0; i < d; ++i) o[i] += w * v_elem(J, blk, kvh, t % J->bs, i);
     }
     for (int64_t i = 0; i < d; ++i) o[i] /= den;
     return ORC_OK;
@@ -272,14 +413,13 @@ static void* decode_worker(void* arg) {
     return NULL;
 }
 
-int orc_paged_decode(int q_dtype, int kv_dtype, const void* q,
-                     const void* k_cache, const void* v_cache,
-                     const int32_t* block_tables, const int32_t* context_lens,
-                     int64_t B, int64_t Hq, int64_t Hkv, int64_t d,
-                     int64_t num_blocks, int64_t bs, int64_t MB, double scale,
-                     const int64_t* pairs, int64_t npairs, int nthreads, double* out) {
-    if ((q_dtype != ORC_F32 && q_dtype != ORC_BF16) || (kv_dtype != ORC_F32 && kv_dtype != ORC_BF16))
-        return ORC_EARG;
+static int run_decode(int q_dtype, int kv_dtype, const void* q,
+                      const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      int64_t B, int64_t Hq, int64_t Hkv, int64_t d,
+                      int64_t num_blocks, int64_t bs, int64_t MB, double scale,
+                      double k_scale, double v_scale,
+                      const int64_t* pairs, int64_t npairs, int nthreads, double* out) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || d <= 0 || bs <= 0 || MB < 0 ||
         num_blocks <= 0 || npairs < 0)
         return ORC_EARG;
@@ -298,8 +438,8 @@ int orc_paged_decode(int q_dtype, int kv_dtype, const void* q,
     if (!jobs || !th) { free(jobs); free(th); return ORC_ENOMEM; }
     for (int i = 0; i < nthreads; ++i) {
         decode_job J = {q_dtype, kv_dtype, q, k_cache, v_cache, block_tables, context_lens,
-                        B, Hq, Hkv, d, num_blocks, bs, MB, scale, pairs, npairs, out,
-                        nthreads, i, ORC_OK};
+                        B, Hq, Hkv, d, num_blocks, bs, MB, scale, k_scale, v_scale, pairs,
+                        npairs, out, nthreads, i, ORC_OK};
         jobs[i] = J;
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, decode_worker, &jobs[i]);
@@ -311,6 +451,35 @@ int orc_paged_decode(int q_dtype, int kv_dtype, const void* q,
     free(jobs);
     free(th);
     return st;
+}
+
+int orc_paged_decode(int q_dtype, int kv_dtype, const void* q,
+                     const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, const int32_t* context_lens,
+                     int64_t B, int64_t Hq, int64_t Hkv, int64_t d,
+                     int64_t num_blocks, int64_t bs, int64_t MB, double scale,
+                     const int64_t* pairs, int64_t npairs, int nthreads, double* out) {
+    if ((q_dtype != ORC_F32 && q_dtype != ORC_BF16) || (kv_dtype != ORC_F32 && kv_dtype != ORC_BF16))
+        return ORC_EARG;
+    return run_decode(q_dtype, kv_dtype, q, k_cache, v_cache, block_tables, context_lens, B, Hq,
+                      Hkv, d, num_blocks, bs, MB, scale, 1.0, 1.0, pairs, npairs, nthreads, out);
+}
+
+/* The decode over an E4M3 cache: the same definition with
+ * K[t][i] = value(k code) * k_scale and V[t][i] = value(v code) * v_scale
+ * (V pages transposed, see k_elem / v_elem). */
+int orc_paged_decode_e4m3(int q_dtype, const void* q,
+                          const uint8_t* k_cache, const uint8_t* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          int64_t B, int64_t Hq, int64_t Hkv, int64_t d,
+                          int64_t num_blocks, int64_t bs, int64_t MB, double scale,
+                          double k_scale, double v_scale,
+                          const int64_t* pairs, int64_t npairs, int nthreads, double* out) {
+    if (q_dtype != ORC_F32 && q_dtype != ORC_BF16) return ORC_EARG;
+    if (!(k_scale > 0.0) || !(v_scale > 0.0) || isinf(k_scale) || isinf(v_scale)) return ORC_EARG;
+    return run_decode(q_dtype, ORC_E4M3, q, k_cache, v_cache, block_tables, context_lens, B, Hq,
+                      Hkv, d, num_blocks, bs, MB, scale, k_scale, v_scale, pairs, npairs, nthreads,
+                      out);
 }
 
 /* ---- self-check variants (same definition, no paging) ------------------ */

@@ -478,6 +478,170 @@ def pin_chunked_prefill_matches_causal_sdpa(orc: Oracle):
                 assert_close(got[b], full, 1e-12, "whole-context chunk vs causal pass")
 
 
+
+# ---------------------------------------------------------------- 8-bit cache
+
+
+def _e4m3_value(codes):
+    """PyTorch's own reading of E4M3 codes (float8_e4m3fn), as float64."""
+    return codes.view(torch.float8_e4m3fn).to(torch.float64)
+
+
+def pin_e4m3_decode_matches_torch(orc: Oracle):
+    """Every one of the 256 codes means what PyTorch's float8_e4m3fn says
+    (the OCP E4M3 format: bias 7, subnormals m * 2^-9, S.1111.111 NaN)."""
+    c = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    got, want = orc.e4m3_to_double(c), _e4m3_value(c)
+    same = (got == want) | (got.isnan() & want.isnan())
+    assert bool(same.all()), f"codes {c[~same].tolist()} decode differently"
+    assert got[0x7E].item() == 448.0 and got[0x01].item() == 2.0 ** -9
+
+
+def pin_e4m3_round_matches_torch_cast(orc: Oracle):
+    """Rounding binary32 values to E4M3 equals PyTorch's float32 -> float8
+    cast (nearest, ties to even) across the range, subnormals and exact
+    midpoints between neighbouring codes included; beyond the range the
+    oracle saturates to +-448."""
+    g = _gen(61)
+    mant = torch.randn(50000, generator=g, dtype=torch.float64)
+    expo = torch.randint(-14, 10, (50000,), generator=g).to(torch.float64)
+    x = (mant * torch.pow(2.0, expo)).to(torch.float32).to(torch.float64)
+    vals = _e4m3_value(torch.arange(0, 0x7E, dtype=torch.int32).to(torch.uint8))
+    mids = (vals[:-1] + vals[1:]) / 2
+    x = torch.cat([x, mids, -mids, vals, -vals]).clamp(-464.0, 464.0)
+    got = orc.round_e4m3(x)
+    want = x.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+    bad = (got != want).nonzero()
+    assert bad.numel() == 0, f"{bad.numel()} mismatches, first at {x[bad[0]].item()!r}"
+    big = torch.tensor([470.0, 1e6, float("inf"), -500.0, -float("inf")], dtype=torch.float64)
+    assert orc.round_e4m3(big).tolist() == [0x7E, 0x7E, 0x7E, 0xFE, 0xFE], "saturation"
+
+
+def pin_e4m3_quantizer_rounds_through_binary32(orc: Oracle):
+    """The cache quantizer decides in binary32: v / v_scale that lies just
+    above the midpoint between 1 and 1.125 in double, but rounds onto it in
+    binary32, goes to 1 (even); rounded from the double directly it would
+    go to 1.125."""
+    x = torch.tensor([1.0625 + 2.0 ** -40], dtype=torch.float64)
+    assert orc.round_e4m3(x).tolist() == [0x39], "double rounding of the rounding itself"
+    T, Hq, Hkv, d, NB, bs = 1, 1, 1, 2, 1, 16
+    q = torch.zeros(T, Hq, d)
+    k = torch.zeros(T, Hkv, d)
+    v = torch.full((T, Hkv, d), 1.0625)
+    kc = torch.zeros(NB, Hkv, bs, d, dtype=torch.uint8)
+    vc = torch.zeros(NB, Hkv, d, bs, dtype=torch.uint8)
+    v_scale = 1.0 - 2.0 ** -40  # v / v_scale = 1.0625 + ~1e-12
+    orc.kv_append_e4m3(q, k, v, torch.tensor([0]), torch.tensor([3]), kc, vc, 1e4, 1.0, v_scale)
+    assert vc[0, 0, :, 3].tolist() == [0x38, 0x38], vc[0, 0, :, 3].tolist()
+
+
+def _random_e4m3_cache(lens, Hkv, d, bs, seed, extra_blocks=3):
+    """Random finite codes in a paged pool (k [NB, Hkv, bs, d], v transposed
+    [NB, Hkv, d, bs]) and the per-sequence code rows [L, Hkv, d]."""
+    g = _gen(seed)
+    need = [max(1, (L + bs - 1) // bs) for L in lens]
+    NB = sum(need) + extra_blocks
+    perm = torch.randperm(NB, generator=g)
+    tables = torch.full((len(lens), max(need)), -1, dtype=torch.int32)
+
+    def codes(*shape):
+        c = torch.randint(0, 256, shape, generator=g, dtype=torch.int32).to(torch.uint8)
+        return torch.where((c & 0x7F) == 0x7F, c ^ 0x01, c)  # no NaN codes
+
+    kc, vc = codes(NB, Hkv, bs, d), codes(NB, Hkv, d, bs)
+    Ks, Vs, c0 = [], [], 0
+    for b, L in enumerate(lens):
+        ids = perm[c0:c0 + need[b]]
+        c0 += need[b]
+        tables[b, :need[b]] = ids.to(torch.int32)
+        K, V = codes(L, Hkv, d), codes(L, Hkv, d)
+        for t in range(L):
+            kc[ids[t // bs], :, t % bs, :] = K[t]
+            vc[ids[t // bs], :, :, t % bs] = V[t]
+        Ks.append(K)
+        Vs.append(V)
+    return kc, vc, tables, Ks, Vs
+
+
+def pin_e4m3_decode_matches_sdpa_over_dequantized(orc: Oracle):
+    """Decode over the 8-bit cache equals PyTorch's fp64 SDPA over the
+    dequantized contiguous K/V (code value x scale); with power-of-two
+    scales it also equals the oracle's own fp32-cache decode over the same
+    values, which are exact in fp32."""
+    for (Hq, Hkv, d, lens, ks, vs, seed) in [(8, 2, 16, [40, 17, 1, 33], 0.0123, 0.0311, 70),
+                                             (4, 4, 8, [5, 16], 0.125, 0.0625, 71)]:
+        kc, vc, tables, Ks, Vs = _random_e4m3_cache(lens, Hkv, d, 16, seed)
+        B = len(lens)
+        q = torch.randn(B, Hq, d, generator=_gen(seed + 1)).to(torch.bfloat16)
+        scale = 1.0 / math.sqrt(d)
+        cl = torch.tensor(lens, dtype=torch.int32)
+        got = orc.paged_attention_decode_e4m3(q, kc, vc, tables, cl, scale, ks, vs)
+        for b in range(B):
+            K = _e4m3_value(Ks[b]) * ks
+            V = _e4m3_value(Vs[b]) * vs
+            want = sdpa(q[b][None].double(), K, V, scale)[0]
+            assert_close(got[b], want, 1e-12, f"e4m3 decode vs SDPA b={b}")
+        if ks == 0.125:
+            kf = (_e4m3_value(kc) * ks).to(torch.float32)
+            vf = (_e4m3_value(vc) * vs).to(torch.float32).transpose(2, 3).contiguous()
+            same = orc.paged_attention_decode(q, kf, vf, tables, cl, scale)
+            assert_close(got, same, 1e-15, "e4m3 decode vs fp32-cache decode")
+
+
+def pin_append_e4m3_placement_and_values(orc: Oracle):
+    """The 8-bit append changes exactly the addressed K rows and V columns
+    (V pages are transposed); the codes are PyTorch's float8 cast of
+    binary32(rope(k) / k_scale) and binary32(v / v_scale); q is rotated and
+    rounded to its own type as in the plain append."""
+    for dtype in (torch.bfloat16, torch.float32):
+        q, k, v, pos, slots, NB, bs = _append_case(dtype, 43)
+        T, Hq, d = q.shape
+        Hkv = k.shape[1]
+        ks, vs = 0.0173, 0.0291
+        kc = torch.full((NB, Hkv, bs, d), 0x7F, dtype=torch.uint8)
+        vc = torch.full((NB, Hkv, d, bs), 0x7F, dtype=torch.uint8)
+        q2 = q.clone()
+        orc.kv_append_e4m3(q2, k.clone(), v.clone(), pos, slots, kc, vc, 5e5, ks, vs)
+        want_k = torch.zeros(NB, Hkv, bs, dtype=torch.bool)
+        for s in slots.tolist():
+            if s >= 0:
+                want_k[s // bs, :, s % bs] = True
+        kchg, vchg = kc != 0x7F, vc != 0x7F
+        assert torch.equal(kchg.any(-1), want_k), "k rows written"
+        assert torch.equal(vchg.any(-2), want_k), "v columns written"
+
+        def rot(x, p):
+            i = torch.arange(d // 2, dtype=torch.float64)
+            z = torch.complex(x[..., : d // 2].double(), x[..., d // 2:].double())
+            z = z * torch.exp(1j * float(p) * 5e5 ** (-2.0 * i / d))
+            return torch.cat([z.real, z.imag], -1)
+
+        def cast(x):
+            return x.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+
+        for t, s in enumerate(slots.tolist()):
+            want_q = orc.round_bf16(rot(q[t], pos[t])) if dtype == torch.bfloat16 \
+                else rot(q[t], pos[t]).to(torch.float32)
+            assert (q2[t].double() - want_q.double()).abs().max().item() <= \
+                (1e-6 if dtype == torch.float32 else 0.0), f"q token {t}"
+            if s < 0:
+                continue
+            kk = rot(k[t], pos[t]) / ks
+            got_k = kc[s // bs, :, s % bs]
+            exact = cast(kk)
+            # the rotation's last fp64 bit may differ from PyTorch's complex
+            # product: allow a neighbouring code only where binary32(kk) sits
+            # within a few binary32 ulps of an E4M3 midpoint
+            near = torch.zeros_like(exact, dtype=torch.bool)
+            for sgn in (-1, 1):
+                nudged = kk.to(torch.float32)
+                for _ in range(3):
+                    nudged = torch.nextafter(nudged, torch.full_like(nudged, sgn * 1e9))
+                near |= cast(nudged.double()) != exact
+            assert bool(((got_k == exact) | near).all()), f"k codes token {t}"
+            assert torch.equal(vc[s // bs, :, :, s % bs], cast(v[t].double() / vs)), f"v codes {t}"
+
+
 PINS = [
     pin_round_bf16_matches_torch_cast,
     pin_round_bf16_single_rounding,
@@ -497,6 +661,11 @@ PINS = [
     pin_append_rejects_out_of_range_slot,
     pin_append_then_decode_is_causal_last_row,
     pin_chunked_prefill_matches_causal_sdpa,
+    pin_e4m3_decode_matches_torch,
+    pin_e4m3_round_matches_torch_cast,
+    pin_e4m3_quantizer_rounds_through_binary32,
+    pin_e4m3_decode_matches_sdpa_over_dequantized,
+    pin_append_e4m3_placement_and_values,
 ]
 
 
@@ -513,10 +682,10 @@ MUTATIONS = [
     ("drop_scale", "s[t] = J->scale * acc;", "s[t] = acc;"),
     ("gqa_modulo", "const int64_t kvh = h / G;\n    const int64_t L = J->context_lens[b];",
      "const int64_t kvh = h % J->Hkv;\n    const int64_t L = J->context_lens[b];"),
-    ("pool_head_major", "int64_t kbase = ((blk * J->Hkv + kvh) * J->bs + t % J->bs) * d;",
-     "int64_t kbase = ((kvh * J->num_blocks + blk) * J->bs + t % J->bs) * d;"),
-    ("row_index", "int64_t kbase = ((blk * J->Hkv + kvh) * J->bs + t % J->bs) * d;",
-     "int64_t kbase = ((blk * J->Hkv + kvh) * J->bs + (t + 1) % J->bs) * d;"),
+    ("pool_head_major", "int64_t idx = ((blk * J->Hkv + kvh) * J->bs + row) * J->d + i;",
+     "int64_t idx = ((kvh * J->num_blocks + blk) * J->bs + row) * J->d + i;"),
+    ("row_index", "int64_t idx = ((blk * J->Hkv + kvh) * J->bs + row) * J->d + i;",
+     "int64_t idx = ((blk * J->Hkv + kvh) * J->bs + (row + 1) % J->bs) * J->d + i;"),
     ("drop_last_token", "for (int64_t t = 0; t < L; ++t) {\n        double w",
      "for (int64_t t = 0; t + 1 < L; ++t) {\n        double w"),
     ("normalise_by_length", "for (int64_t i = 0; i < d; ++i) o[i] /= den;\n    return ORC_OK;",
@@ -534,7 +703,27 @@ MUTATIONS = [
      "for (int64_t i = 0; i < d; ++i) row[i] = load_elem(v_new, dtype, src + i);\n"
      "            rope_rotate(row, d, pos, theta);\n"
      "            for (int64_t i = 0; i < d; ++i) store_elem((void*)v_new, dtype, src + i, row[i]);"),
-    ("skip_q_rotation", "rope_rotate(row, d, pos, theta);\n            for (int64_t i = 0; i < d; ++i) store_elem(q,",
+    ("e4m3_bias", "v = ldexp(1.0 + m / 8.0, E - 7);", "v = ldexp(1.0 + m / 8.0, E - 8);"),
+    ("e4m3_subnormal", "v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    ("e4m3_spacing", "int spacing_exp = (e - 1) - 3;", "int spacing_exp = (e - 1) - 4;"),
+    ("e4m3_no_saturation", "if (r > 448.0) r = 448.0;", ""),
+    ("e4m3_no_binary32_step", "return double_to_e4m3((double)(float)(x / scale));",
+     "return double_to_e4m3(x / scale);"),
+    ("e4m3_scale_multiplies", "return double_to_e4m3((double)(float)(x / scale));",
+     "return double_to_e4m3((double)(float)(x * scale));"),
+    ("e4m3_v_row_major_store", "v_cache[page + i * bs + r] =", "v_cache[page + r * d + i] ="),
+    ("e4m3_slot_offset", "int64_t blk = slot / bs, r = slot % bs;",
+     "int64_t blk = slot / bs, r = (slot + 1) % bs;"),
+    ("e4m3_v_row_major_load", "int64_t idx = ((blk * J->Hkv + kvh) * J->d + i) * J->bs + row;",
+     "int64_t idx = ((blk * J->Hkv + kvh) * J->bs + row) * J->d + i;"),
+    ("e4m3_drop_k_scale", "return e4m3_to_double(((const uint8_t*)J->k_cache)[idx]) * J->k_scale;",
+     "return e4m3_to_double(((const uint8_t*)J->k_cache)[idx]);"),
+    ("e4m3_drop_v_scale", "return e4m3_to_double(((const uint8_t*)J->v_cache)[idx]) * J->v_scale;",
+     "return e4m3_to_double(((const uint8_t*)J->v_cache)[idx]);"),
+    ("e4m3_k_unrotated", "for (int64_t i = 0; i < d; ++i) k_cache[page + r * d + i] =",
+     "for (int64_t i = 0; i < d; ++i) row[i] = load_elem(k_new, dtype, src + i);\n"
+     "            for (int64_t i = 0; i < d; ++i) k_cache[page + r * d + i] ="),
+    ("skip_q_rotation", "rope_rotate(row, d, pos, theta);\n        for (int64_t i = 0; i < d; ++i) store_elem(q,",
      "for (int64_t i = 0; i < d; ++i) store_elem(q,"),
 ]
 
