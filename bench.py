@@ -61,6 +61,9 @@ def parse_args(argv=None):
     ap.add_argument("--copies", type=int, default=0,
                     help="device-side copies of the workload (0: enough to exceed L2)")
     ap.add_argument("--simt", action="store_true", help="bf16: CUDA-core decode kernel")
+    ap.add_argument("--kv-dtype", default="native", choices=["native", "e4m3"],
+                    help="e4m3: the workload's cache as an 8-bit cache (per-tensor scales), "
+                         "stepped as kv_append_e4m3 + paged_attention_decode_e4m3")
     ap.add_argument("--two-calls", action="store_true",
                     help="time kv_append + paged_attention_decode as two launches instead of "
                          "the single-launch decode_step")
@@ -122,9 +125,10 @@ def esize(dt):
 
 def step_bytes(w, out_dtype) -> int:
     """Algorithmic bytes of one decode call: every context token's K and V
-    row once per KV head, plus q read and out written."""
+    row once per KV head (at the cache's element size), plus q read and out
+    written."""
     L = int(w.decode_lens.to(torch.int64).sum().item())
-    kv = L * w.Hkv * w.d * 2 * esize(w.dtype)
+    kv = L * w.Hkv * w.d * 2 * w.k_cache.element_size()
     qo = w.B * w.Hq * w.d * (esize(w.dtype) + esize(out_dtype))
     return kv + qo
 
@@ -147,9 +151,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(cfg: int):
+def recorded_traffic(cfg):
     """DRAM bytes per decode launch from the committed ncu capture, if it was
-    taken on the current kernel sources (else None)."""
+    taken on the current kernel sources (else None).  ``cfg``: the config
+    number, or e.g. "3_e4m3" for its 8-bit cache."""
     path = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
     try:
         with open(path) as f:
@@ -226,6 +231,18 @@ class ClockSampler:
 def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
     from paged_kv_cache_484_b200 import workloads as W
     s = W.config_summary(cfg)
+    if w.k_cache.dtype == torch.uint8:
+        return {
+            "workload": W.CONFIG_NAMES[cfg] + "_e4m3cache",
+            "batch_seqs": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
+            "context": s["ctx"], "tokens_decoded": int(w.decode_lens.to(torch.int64).sum().item()),
+            "block_size": w.block_size, "pool_blocks": w.num_blocks,
+            "kv_dtype": "e4m3 (per-tensor scales: max|x| / 448)",
+            "kv_scales": list(w.meta.get("e4m3_scales", ())),
+            "out_dtype": "bf16" if out_dtype == torch.bfloat16 else "f32",
+            "partition_tokens": P, "max_partitions": NP, "decode_kernel": "mma_f16 (e4m3 pages)",
+            "step": "two calls (kv_append_e4m3, paged_attention_decode_e4m3)",
+        }
     return {
         "workload": W.CONFIG_NAMES[cfg],
         "batch_seqs": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
@@ -242,9 +259,10 @@ def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
 
 # ---------------------------------------------------------------- oracle arm
 
-def time_oracle(w, seconds: float, nthreads: int):
+def time_oracle(w, seconds: float, nthreads: int, e4m3_scales=None):
     """Oracle append + decode of the whole workload (or a bounded subset of
-    sequences for the big ones), repeated until ~``seconds`` of CPU time."""
+    sequences for the big ones), repeated until ~``seconds`` of CPU time
+    (the 8-bit cache's append and decode when ``e4m3_scales`` is given)."""
     import oracle
     from paged_kv_cache_484_b200.workloads import extract_sequences
 
@@ -264,10 +282,17 @@ def time_oracle(w, seconds: float, nthreads: int):
         q = sub.q.clone()
         kc, vc = sub.k_cache.clone(), sub.v_cache.clone()
         t0 = time.perf_counter()
-        oracle.kv_append(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions, sub.slots, kc, vc,
-                         sub.theta)
-        oracle.paged_attention_decode(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
-                                      nthreads=nthreads)
+        if e4m3_scales is not None:
+            ks, vs = e4m3_scales
+            oracle.kv_append_e4m3(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions,
+                                  sub.slots, kc, vc, sub.theta, ks, vs)
+            oracle.paged_attention_decode_e4m3(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
+                                               ks, vs, nthreads=nthreads)
+        else:
+            oracle.kv_append(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions, sub.slots,
+                             kc, vc, sub.theta)
+            oracle.paged_attention_decode(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
+                                          nthreads=nthreads)
         t_total += time.perf_counter() - t0
         reps += 1
     return t_total / reps, seqs, frac_bytes, reps
@@ -318,6 +343,16 @@ def run_ours(args):
     pkv.load_library()
     out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
     w = W.make_config(args.config, device=device)
+    e4m3 = args.kv_dtype == "e4m3"
+    if e4m3:
+        if w.dtype != torch.bfloat16:
+            raise SystemExit("--kv-dtype e4m3 takes a bf16 workload (configs 2-5)")
+        k8, v8, ks8, vs8 = W.e4m3_cache(w)
+        w.k_cache, w.v_cache = k8, v8
+        w.meta["e4m3_scales"] = (ks8, vs8)
+        args.two_calls = True
+        torch.cuda.empty_cache()
+    kv_dt = torch.uint8 if e4m3 else w.dtype
     host_inputs = None
     if not args.no_e2e:
         # pristine copies of the per-step inputs, in pinned host memory
@@ -327,9 +362,9 @@ def run_ours(args):
             decode_lens=w.decode_lens).items()}
 
     P = args.partition_tokens or pkv.decode_partition_tokens(w.B, w.Hq, w.Hkv, w.d, w.max_blocks,
-                                                              kv_dtype=w.dtype)
+                                                              kv_dtype=kv_dt)
     NP = math.ceil(w.max_blocks * w.block_size / P)
-    ws_bytes = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=w.dtype,
+    ws_bytes = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=kv_dt,
                                          partition_tokens=P)
     ws = pkv.new_workspace(ws_bytes, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
@@ -350,6 +385,8 @@ def run_ours(args):
 
     cascade = args.cascade
     if cascade:
+        if e4m3:
+            raise SystemExit("--cascade takes the bf16 cache")
         if w.meta.get("prefix_group", 0) <= 1:
             raise SystemExit("--cascade needs a workload with prefix groups (config 4)")
         args.two_calls = True
@@ -365,7 +402,7 @@ def run_ours(args):
     fused = not args.two_calls
     # decode kernel, plus the partition combine unless the split contexts
     # are merged inside thread-block clusters (the library decides)
-    kernels_per_decode = pkv.decode_launches(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=w.dtype,
+    kernels_per_decode = pkv.decode_launches(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=kv_dt,
                                              out_dtype=out_dtype, partition_tokens=P,
                                              force_simt=args.simt, fused=fused)
     if kernels_per_decode not in (1, 2):
@@ -375,12 +412,21 @@ def run_ours(args):
     launches_per_step = kernels_per_decode + (0 if fused else 1)
 
     def append(c):
-        if not fused:
+        if e4m3:
+            pkv.kv_append_e4m3(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
+                               c["k_cache"], c["v_cache"], w.rope_theta, ks8, vs8,
+                               device_error=err)
+        elif not fused:
             pkv.kv_append(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                           c["k_cache"], c["v_cache"], w.rope_theta, device_error=err)
 
     def decode(c, out):
-        if fused:
+        if e4m3:
+            pkv.paged_attention_decode_e4m3(c["q"], c["k_cache"], c["v_cache"],
+                                            c["block_tables"], c["decode_lens"], w.scale, ks8,
+                                            vs8, out, workspace=ws, partition_tokens=P,
+                                            device_error=err)
+        elif fused:
             pkv.decode_step(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                             c["k_cache"], c["v_cache"], c["block_tables"], c["decode_lens"],
                             w.rope_theta, w.scale, out, workspace=ws, partition_tokens=P,
@@ -467,8 +513,11 @@ def run_ours(args):
     # scheme over the copies
     def append_only(k):
         c = copies[k % ncopies]
-        pkv.kv_append(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
-                      c["k_cache"], c["v_cache"], w.rope_theta, device_error=err)
+        if e4m3:
+            append(c)
+        else:
+            pkv.kv_append(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
+                          c["k_cache"], c["v_cache"], w.rope_theta, device_error=err)
 
     append_g = graphs_for(append_only)
 
@@ -554,7 +603,11 @@ def run_ours(args):
             # big workloads: the oracle reads a bounded subset copied from the device
             wc = w
         nthreads = os.cpu_count() or 1
-        per_step, seqs, frac, reps = time_oracle(wc, args.cpu_seconds, nthreads)
+        if e4m3 and wc is not w:
+            k8c, v8c, _, _ = W.e4m3_cache(wc)
+            wc.k_cache, wc.v_cache = k8c, v8c
+        per_step, seqs, frac, reps = time_oracle(wc, args.cpu_seconds, nthreads,
+                                                 (ks8, vs8) if e4m3 else None)
         cpu = {"value": round(nbytes * frac / per_step / 1e9, 4), "unit": "GB/s",
                "cores": nthreads, "kind": "oracle",
                "sample": f"{len(seqs)} of {w.B} sequences, full append+decode step in fp64, "
@@ -564,7 +617,8 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": max(3, args.warmup), "ms_per_step": round(step_ms_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "dtype": "e4m3" if e4m3 else ("bf16" if w.dtype == torch.bfloat16 else "f32"),
+        "data": "synthetic",
         "pct_of_hbm_peak": round(100.0 * value / (world * peak), 2),
         "seq_steps_per_s": round(world * w.B / (step_ms_max * 1e-3), 1),
         "config": dict(config_block(args.config, w, out_dtype, P, NP, args.simt, args.two_calls),
@@ -592,7 +646,7 @@ def run_ours(args):
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "decode_ms": round(decode_ms_max, 5),
-                     "traffic": recorded_traffic(args.config)},
+                     "traffic": recorded_traffic(f"{args.config}_e4m3" if e4m3 else args.config)},
         "gpu_launches": K * launches_per_step,
         "kv_append_us_per_call": round(append_ms * 1e3, 3),
         "clocks": clocks.summary(),

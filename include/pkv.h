@@ -46,7 +46,8 @@
  *             h / (Hq / Hkv) (contiguous groups).
  * Supported.  head_dim in {64, 128}; block_size 16; Hq / Hkv in {1, 2, 4, 8};
  *             storage dtype fp32 or bf16 (PKV_DTYPE_*), the same for q, the
- *             new k/v and the cache.
+ *             new k/v and the cache; or an 8-bit E4M3 cache with bf16 q (the
+ *             *_e4m3 entry points).
  * Alignment.  q, k_new, v_new, caches, out and workspace: 16-byte aligned.
  * Streams.    `stream` is a cudaStream_t (NULL = legacy default stream).  All
  *             work is enqueued asynchronously on it; a call returns as soon as
@@ -83,7 +84,9 @@ typedef enum pkv_status {
 
 typedef enum pkv_dtype {
     PKV_DTYPE_F32 = 0,
-    PKV_DTYPE_BF16 = 1
+    PKV_DTYPE_BF16 = 1,
+    PKV_DTYPE_E4M3 = 2 /* 8-bit cache only: E4M3 codes x a per-tensor scale, see
+                          pkv_kv_append_e4m3 / pkv_paged_attention_decode_e4m3 */
 } pkv_dtype;
 
 /* Bits OR-ed into *device_error by the kernels. */
@@ -332,6 +335,81 @@ pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache
                                               int32_t out_dtype, float scale,
                                               int32_t partition_tokens, uint32_t flags,
                                               int32_t* device_error, void* stream);
+
+/*
+ * The 8-bit cache.
+ *
+ * Source: "Efficient LLM Inference", "Quantization: From Rounding Errors to
+ * Model-quality Limits" (values rounded to a small set of levels with a
+ * scale) and "Verify Exact Execution and Approximate Quality Separately";
+ * "From KV Elements to Memory Accounting and Admission Budgets" (cache
+ * bytes per token set how many requests fit).  The element format is the
+ * OCP 8-bit floating point E4M3 format (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, no infinities, largest finite 448), which the pages do
+ * not name.  One scale per tensor: the cached value is code x k_scale (K) or
+ * code x v_scale (V).
+ *
+ * Layout (uint8):
+ *   k_cache  [num_blocks, Hkv, block_size, head_dim]   (rows as in the bf16 cache)
+ *   v_cache  [num_blocks, Hkv, head_dim, block_size]   (each page transposed)
+ * The transposed V page lets the decode's tensor-core tile read the four
+ * tokens a lane needs as four consecutive bytes.
+ */
+
+/*
+ * pkv_kv_append_e4m3 -- pkv_kv_append into the 8-bit cache.
+ *
+ * q is rotated in place and rounded to its own dtype exactly as by
+ * pkv_kv_append.  For a token with slot s >= 0 and every kv head h, dim i:
+ *   k_cache[s / bs, h, s % bs, i] <- code(rope(k_new[t, h, :], p)[i] / k_scale)
+ *   v_cache[s / bs, h, i, s % bs] <- code(v_new[t, h, i] / v_scale)
+ * where the division is fp64, its result is rounded to binary32 and code()
+ * is the nearest E4M3 value of that binary32 number, ties to even,
+ * saturating to +-448 (cvt.rn.satfinite).
+ *
+ * Arguments: those of pkv_kv_append, with
+ *   dtype              PKV_DTYPE_F32 or PKV_DTYPE_BF16: q, k_new, v_new
+ *   k_cache, v_cache   device uint8, the layout above
+ *   k_scale, v_scale   finite, > 0
+ */
+pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,
+                              const int64_t* positions, const int64_t* slot_mapping,
+                              void* k_cache, void* v_cache, int64_t num_tokens,
+                              int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                              int64_t num_blocks, int64_t block_size, int32_t dtype,
+                              double rope_theta, float k_scale, float v_scale,
+                              int32_t* device_error, void* stream);
+
+/*
+ * pkv_paged_attention_decode_e4m3 -- pkv_paged_attention_decode over the 8-bit
+ * cache: the same definition with K_b[t][i] = code x k_scale and
+ * V_b[t][i] = code x v_scale.
+ *
+ * The tensor-core tiles run as f16 MMAs: every E4M3 value is exact in f16;
+ * q (bf16) is rounded to f16, which is exact for |q| in [2^-17, 65504] (q
+ * entries must stay below 65504 in magnitude; smaller ones lose at most
+ * 2^-25 absolutely); P is split into two f16 terms; accumulation is fp32.
+ * Workspace, partitioning, cluster merging, flags (except
+ * PKV_DECODE_FORCE_SIMT, which is not supported here) and errors are those of
+ * pkv_paged_attention_decode; size the workspace with kv_dtype
+ * PKV_DTYPE_E4M3.
+ *
+ * Arguments: those of pkv_paged_attention_decode, with
+ *   q                  device, [num_seqs, Hq, head_dim] bf16
+ *   k_cache, v_cache   device uint8, the layout above
+ *   k_scale, v_scale   finite, > 0
+ */
+pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
+                                           const void* v_cache, const int32_t* block_tables,
+                                           const int32_t* context_lens, void* out,
+                                           void* workspace, size_t workspace_bytes,
+                                           int64_t num_seqs, int64_t num_q_heads,
+                                           int64_t num_kv_heads, int64_t head_dim,
+                                           int64_t num_blocks, int64_t block_size,
+                                           int64_t max_blocks_per_seq, int32_t out_dtype,
+                                           float scale, float k_scale, float v_scale,
+                                           int32_t partition_tokens, uint32_t flags,
+                                           int32_t* device_error, void* stream);
 
 /*
  * pkv_paged_attention_decode_cascade -- pkv_paged_attention_decode for batches

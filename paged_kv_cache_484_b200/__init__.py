@@ -30,10 +30,12 @@ from ._binding import (  # noqa: F401
     decode_step,
     decode_workspace_size,
     kv_append,
+    kv_append_e4m3,
     load_library,
     new_workspace,
     paged_attention_decode,
     paged_attention_decode_cascade,
+    paged_attention_decode_e4m3,
     paged_attention_decode_noalloc,
     decode_cascade_workspace_size,
     paged_attention_prefill,

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libpkv.so")
 
 PKV_DTYPE_F32 = 0
 PKV_DTYPE_BF16 = 1
+PKV_DTYPE_E4M3 = 2  # 8-bit cache (uint8 tensors of E4M3 codes)
 PKV_DECODE_FORCE_SIMT = 0x1
 PKV_DECODE_NO_CLUSTER = 0x2
 DEVERR_SLOT = 0x1
@@ -89,6 +90,14 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_paged_attention_decode_cascade.restype = ctypes.c_int
         lib.pkv_decode_cascade_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32]
         lib.pkv_decode_cascade_workspace_size.restype = ctypes.c_size_t
+        lib.pkv_kv_append_e4m3.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                           i64, i32, ctypes.c_double, ctypes.c_float,
+                                           ctypes.c_float, vp, vp]
+        lib.pkv_kv_append_e4m3.restype = ctypes.c_int
+        lib.pkv_paged_attention_decode_e4m3.argtypes = [
+            vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64, i64, i32,
+            ctypes.c_float, ctypes.c_float, ctypes.c_float, i32, u32, vp, vp]
+        lib.pkv_paged_attention_decode_e4m3.restype = ctypes.c_int
         lib.pkv_bm_create.argtypes = [i32, i32]
         lib.pkv_bm_create.restype = vp
         lib.pkv_bm_destroy.argtypes = [vp]
@@ -132,6 +141,13 @@ def _dtype_code(dt: torch.dtype) -> int:
     if dt == torch.bfloat16:
         return PKV_DTYPE_BF16
     raise TypeError(f"unsupported dtype {dt} (float32 or bfloat16)")
+
+
+def _kv_dtype_code(dt: torch.dtype) -> int:
+    """Cache dtype code: float32, bfloat16, or uint8 for the 8-bit cache."""
+    if dt == torch.uint8:
+        return PKV_DTYPE_E4M3
+    return _dtype_code(dt)
 
 
 def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
@@ -191,7 +207,7 @@ def decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, max_b
     lib = load_library()
     return int(lib.pkv_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                                max_blocks_per_seq, block_size,
-                                               _dtype_code(kv_dtype)))
+                                               _kv_dtype_code(kv_dtype)))
 
 
 def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
@@ -201,7 +217,7 @@ def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blo
     lib = load_library()
     return int(lib.pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                              max_blocks_per_seq, block_size,
-                                             _dtype_code(kv_dtype), int(partition_tokens)))
+                                             _kv_dtype_code(kv_dtype), int(partition_tokens)))
 
 
 def decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
@@ -212,7 +228,7 @@ def decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_pe
     clusters) or 2 (decode + partition combine); 0 for invalid arguments."""
     lib = load_library()
     return int(lib.pkv_decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                       max_blocks_per_seq, block_size, _dtype_code(kv_dtype),
+                                       max_blocks_per_seq, block_size, _kv_dtype_code(kv_dtype),
                                        _dtype_code(out_dtype), int(partition_tokens),
                                        _flags(force_simt, cluster), 1 if fused else 0))
 
@@ -265,6 +281,65 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale), int(partition_tokens),
         _flags(force_simt, cluster), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode")
+    return out
+
+
+def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_theta,
+                   k_scale, v_scale, stream=None, *, device_error=None) -> None:
+    """``kv_append`` into the 8-bit cache: q [T, Hq, d] rotated in place (its
+    own dtype, float32 or bfloat16, shared by k_new/v_new [T, Hkv, d]);
+    k_cache uint8 [NB, Hkv, 16, d] gets the E4M3 codes of rope(k) / k_scale,
+    v_cache uint8 [NB, Hkv, d, 16] (pages transposed) those of v / v_scale.
+    See include/pkv.h, pkv_kv_append_e4m3."""
+    lib = load_library()
+    dt = _dtype_code(q.dtype)
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q dtype {q.dtype}")
+    T, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if k_new.shape != (T, Hkv, d) or v_new.shape != (T, Hkv, d) or d2 != d \
+            or v_cache.shape != (NB, Hkv, d, bs) or positions.shape != (T,) \
+            or slot_mapping.shape != (T,):
+        raise ValueError("inconsistent kv_append_e4m3 shapes")
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_kv_append_e4m3(
+        _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+        _dev(positions, "positions", torch.int64), _dev(slot_mapping, "slot_mapping", torch.int64),
+        _dev(k_cache, "k_cache", torch.uint8), _dev(v_cache, "v_cache", torch.uint8),
+        T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), float(k_scale), float(v_scale), err,
+        _stream_ptr(stream, q.device))
+    _raise(st, lib, "kv_append_e4m3")
+
+
+def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale,
+                                v_scale, out, stream=None, *, workspace=None, partition_tokens=0,
+                                device_error=None, cluster=True) -> torch.Tensor:
+    """``paged_attention_decode`` over the 8-bit cache (k_cache uint8
+    [NB, Hkv, 16, d], v_cache uint8 [NB, Hkv, d, 16]); q bfloat16 [B, Hq, d];
+    cached values are code x k_scale / code x v_scale.  Writes and returns
+    ``out`` (float32 or bfloat16).  See include/pkv.h."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if d2 != d or v_cache.shape != (NB, Hkv, d, bs) or out.shape != (B, Hq, d) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("inconsistent paged_attention_decode_e4m3 shapes")
+    need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, PKV_DTYPE_E4M3,
+                                         int(partition_tokens))
+    if workspace is None:
+        workspace = new_workspace(int(need), q.device)
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = lib.pkv_paged_attention_decode_e4m3(
+        _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.uint8),
+        _dev(v_cache, "v_cache", torch.uint8), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        B, Hq, Hkv, d, NB, bs, MB, _dtype_code(out.dtype), float(scale), float(k_scale),
+        float(v_scale), int(partition_tokens), _flags(False, cluster), err,
+        _stream_ptr(stream, q.device))
+    _raise(st, lib, "paged_attention_decode_e4m3")
     return out
 
 

@@ -1,6 +1,8 @@
 // kv_append.cu -- RoPE on the new tokens' q and k, and the k/v write into the
 // paged cache slot ("warpllama", Milestones: static KV cache + single-token
-// decode, fused RoPE; "Inference From Scratch", ch. 10: block tables).
+// decode, fused RoPE; "Inference From Scratch", ch. 10: block tables), into a
+// bf16 / fp32 cache or an 8-bit (E4M3 code x per-tensor scale) one
+// ("Efficient LLM Inference", Quantization: rounding to a small set of levels).
 //
 // One CTA per token; every thread owns one 16-byte chunk of work:
 //   * a q or k chunk pair: elements [c*E, c*E+E) of the low half of a head row
@@ -42,6 +44,7 @@ struct AppendParams {
     int Hq, Hkv;
     int64_t num_slots;
     int32_t* err;
+    double k_scale, v_scale;  // 8-bit cache only
 };
 
 template <typename T>
@@ -183,6 +186,103 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_kernel(
     }
 }
 
+// The same append into the 8-bit cache: q as above; k and v become E4M3
+// codes of binary32(x / scale) (x / scale in fp64, then one rounding to
+// binary32, then cvt.rn.satfinite to E4M3), k rows into the [16][D] K page,
+// v into column `row` of the transposed [D][16] V page.
+template <typename T, int D>
+__global__ void __launch_bounds__(kAppendThreadsMax) kv_append_e4m3_kernel(
+    const __grid_constant__ AppendParams p, const __grid_constant__ RopeFreq fr) {
+    constexpr int E = 16 / (int)sizeof(T);
+    constexpr int HALF = D / 2;
+    constexpr int CPH = HALF / E;
+    __shared__ double s_cos[HALF], s_sin[HALF];
+
+    grid_launch_dependents();
+    grid_dependency_wait();
+
+    const int64_t t = blockIdx.x;
+    const int nq = p.Hq * CPH, nk = p.Hkv * CPH, nv = p.Hkv * 2 * CPH;
+    const int total = nq + nk + nv;
+    const int64_t slot = p.slot_mapping[t];
+    const int64_t pos = p.positions[t];
+    const bool write_kv = slot >= 0 && slot < p.num_slots;
+    if (slot >= p.num_slots && threadIdx.x == 0) report_error(p.err, PKV_DEVERR_SLOT);
+    const int64_t blk = write_kv ? slot / kPageRows : 0;
+    const int row = write_kv ? (int)(slot % kPageRows) : 0;
+    T* q = static_cast<T*>(p.q);
+    const T* kn = static_cast<const T*>(p.k_new);
+    const T* vn = static_cast<const T*>(p.v_new);
+    uint8_t* kc = static_cast<uint8_t*>(p.k_cache);
+    uint8_t* vc = static_cast<uint8_t*>(p.v_cache);
+
+    for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
+        double s, c;
+        sincos(reduce_two_pi((double)pos * fr.f[i]), &s, &c);
+        s_cos[i] = c;
+        s_sin[i] = s;
+    }
+    __syncthreads();
+
+    auto code2 = [](double a, double b, double scale) -> uint32_t {
+        return f32x2_to_e4m3x2(__double2float_rn(a / scale), __double2float_rn(b / scale));
+    };
+    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+        if (idx >= nq && !write_kv) break;
+        if (idx < nq + nk) {
+            // a rotation unit: E pairs (x[c E + e], x[c E + e + D/2])
+            const bool is_q = idx < nq;
+            const int j = is_q ? idx : idx - nq;
+            const int h = j / CPH, c = j % CPH;
+            const T* src = is_q ? q + (t * p.Hq + h) * D : kn + (t * p.Hkv + h) * D;
+            double x0[E], x1[E], y0[E], y1[E];
+            unpack16<T>(*reinterpret_cast<const uint4*>(src + c * E), x0);
+            unpack16<T>(*reinterpret_cast<const uint4*>(src + HALF + c * E), x1);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const double cs = s_cos[c * E + e], sn = s_sin[c * E + e];
+                y0[e] = x0[e] * cs - x1[e] * sn;
+                y1[e] = x1[e] * cs + x0[e] * sn;
+            }
+            if (is_q) {
+                T* dst = q + (t * p.Hq + h) * D;
+                *reinterpret_cast<uint4*>(dst + c * E) = pack16<T>(y0);
+                *reinterpret_cast<uint4*>(dst + HALF + c * E) = pack16<T>(y1);
+            } else {
+                uint8_t* dst = kc + ((blk * p.Hkv + h) * kPageRows + row) * D;
+                uint32_t w0[E / 4], w1[E / 4];
+#pragma unroll
+                for (int k = 0; k < E / 4; ++k) {
+                    w0[k] = code2(y0[4 * k], y0[4 * k + 1], p.k_scale) |
+                            (code2(y0[4 * k + 2], y0[4 * k + 3], p.k_scale) << 16);
+                    w1[k] = code2(y1[4 * k], y1[4 * k + 1], p.k_scale) |
+                            (code2(y1[4 * k + 2], y1[4 * k + 3], p.k_scale) << 16);
+                }
+                if constexpr (E == 8) {
+                    *reinterpret_cast<uint2*>(dst + c * E) = make_uint2(w0[0], w0[1]);
+                    *reinterpret_cast<uint2*>(dst + HALF + c * E) = make_uint2(w1[0], w1[1]);
+                } else {
+                    *reinterpret_cast<uint32_t*>(dst + c * E) = w0[0];
+                    *reinterpret_cast<uint32_t*>(dst + HALF + c * E) = w1[0];
+                }
+            }
+        } else {
+            // a v unit: elements [c E, c E + E) of the row, one byte each into
+            // the transposed page (dim-major, 16 tokens per dim)
+            const int j = idx - nq - nk, h = j / (2 * CPH), c = j % (2 * CPH);
+            double x[E];
+            unpack16<T>(*reinterpret_cast<const uint4*>(vn + (t * p.Hkv + h) * D + c * E), x);
+            uint8_t* dst = vc + (blk * p.Hkv + h) * (int64_t)D * kPageRows + row;
+#pragma unroll
+            for (int e = 0; e < E; e += 2) {
+                const uint32_t w = code2(x[e], x[e + 1], p.v_scale);
+                dst[(c * E + e) * kPageRows] = (uint8_t)(w & 0xFFu);
+                dst[(c * E + e + 1) * kPageRows] = (uint8_t)(w >> 8);
+            }
+        }
+    }
+}
+
 template <typename T, int D>
 cudaError_t launch_typed(const AppendArgs& a) {
     constexpr int E = 16 / (int)sizeof(T);
@@ -201,6 +301,8 @@ cudaError_t launch_typed(const AppendArgs& a) {
     p.Hkv = (int)a.Hkv;
     p.num_slots = a.num_blocks * (int64_t)kPageRows;
     p.err = a.device_error;
+    p.k_scale = (double)a.k_scale;
+    p.v_scale = (double)a.v_scale;
     RopeFreq fr;
     for (int i = 0; i < 64; ++i) fr.f[i] = i < D / 2 ? std::pow(a.theta, -(2.0 * i) / D) : 0.0;
 
@@ -214,6 +316,7 @@ cudaError_t launch_typed(const AppendArgs& a) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (a.e4m3) return cudaLaunchKernelEx(&cfg, kv_append_e4m3_kernel<T, D>, p, fr);
     return cudaLaunchKernelEx(&cfg, kv_append_kernel<T, D>, p, fr);
 }
 

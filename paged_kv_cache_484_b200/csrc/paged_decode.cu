@@ -70,33 +70,48 @@ __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+// Tag for the 8-bit cache: E4M3 codes times a per-tensor scale (q stays
+// bf16).  Its K pages keep the [16 tokens][D] row layout; its V pages are
+// stored transposed, [D][16 tokens], so that the four tokens one lane needs
+// for the output MMA are four consecutive bytes.
+struct e4m3kv {};
+
 template <typename T, int D, int G>
 struct Layout {
-    static constexpr int ESZ = sizeof(T);
+    static constexpr bool F8 = std::is_same<T, e4m3kv>::value;
+    static constexpr int ESZ = F8 ? 1 : (int)sizeof(T);             // cache element bytes
+    static constexpr int QSZ = F8 ? 2 : (int)sizeof(T);             // q element bytes
     static constexpr bool SWZ = std::is_same<T, bf16>::value;  // 128B-swizzled bf16 pages
+    // 8-bit K pages with 128-byte rows are 128B-swizzled too (bank-conflict
+    // free 16-byte row reads); 64-byte rows need no swizzle.
+    static constexpr bool SWZ_K8 = F8 && D == 128;
     static constexpr int ROW_BYTES = D * ESZ;
     static constexpr int PAGE_BYTES = kPageRows * ROW_BYTES;
     static constexpr int BOXES = SWZ ? D / 64 : 1;  // TMA boxes per page
     static constexpr int BOX_BYTES = PAGE_BYTES / BOXES;
-    // Pages each consumer warp takes per stage: two for the d = 64 bf16
-    // tensor-core path with G <= 4 (a 32-token tile: longer independent MMA
-    // chains and half the softmax bookkeeping per token), else one.
-    static constexpr int PPW = (SWZ && D == 64 && G <= 4) ? 2 : 1;
+    // Pages each consumer warp takes per stage: two for the d = 64 tensor-core
+    // paths with G <= 4 (a 32-token tile: longer independent MMA chains and
+    // half the softmax bookkeeping per token; the 8-bit cache at G = 8 too),
+    // else one.
+    static constexpr int PPW = ((SWZ && D == 64 && G <= 4) || (F8 && D == 64)) ? 2 : 1;
     static constexpr int STAGE_PAGES = NW * PPW;
     static constexpr int STAGE_BYTES = 2 * STAGE_PAGES * PAGE_BYTES;  // K pages, then V pages
     // 64 KiB of ring (96 KiB for bf16 d = 128, whose CTAs are two per SM
     // by registers anyway)
     static constexpr int STAGES =
         cmax(2, cmin(6, ((D == 128 && SWZ) ? 98304 : 65536) / STAGE_BYTES));
-    static constexpr int Q_COPY = G * D * ESZ;
+    static constexpr int Q_COPY = G * D * QSZ;
     static constexpr int Q_BYTES = round_up(Q_COPY, 128);
     static constexpr int ROW_COPY = D * ESZ;           // one k or v row
     static constexpr int NEWKV_BYTES = 2 * ROW_COPY;   // fused step: raw new k row, new v row
     // Item merge: each warp leaves (o[D], m, l) per head in its own K and V
-    // page slots of the item's last stage (free once it has read its pages).
+    // page slots of the item's last stage (free once it has read its pages),
+    // or, where those are too small (8-bit d = 128 at G = 8), in a region of
+    // its own.
     static constexpr int MERGE_ROW_BYTES = (D + 2) * 4;
     static constexpr int MERGE_ROWS_PER_SLOT = PPW * PAGE_BYTES / MERGE_ROW_BYTES;
-    static_assert(2 * MERGE_ROWS_PER_SLOT >= G, "merge rows do not fit a warp's page slots");
+    static constexpr bool MERGE_IN_SLOTS = 2 * MERGE_ROWS_PER_SLOT >= G;
+    static constexpr int MERGE_BYTES = MERGE_IN_SLOTS ? 0 : NW * G * MERGE_ROW_BYTES;
     // byte offsets from the 1024-aligned base
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
     static constexpr int OFF_NEWKV = OFF_Q + STAGES * Q_BYTES;
@@ -104,12 +119,13 @@ struct Layout {
     // written by the producer with the item's first stage
     static constexpr int ROPE_BYTES = D * 4;
     static constexpr int OFF_ROPE = OFF_NEWKV + STAGES * NEWKV_BYTES;
-    static constexpr int OFF_BAR = OFF_ROPE + STAGES * ROPE_BYTES;
+    static constexpr int OFF_MERGE = OFF_ROPE + STAGES * ROPE_BYTES;
+    static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
     static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
     // Cluster mode: the CTA's merged partial (o[D], m, l per head) sits in the
     // q / new-row / rope-table slots once the CTA's one item is done.
     static constexpr int CLUSTER_PART_BYTES = G * (D + 2) * 4;
-    static_assert(OFF_BAR - OFF_Q >= CLUSTER_PART_BYTES, "cluster partial does not fit");
+    static_assert(OFF_MERGE - OFF_Q >= CLUSTER_PART_BYTES, "cluster partial does not fit");
     static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
     static constexpr int OFF_ITEM = OFF_PATCH + STAGES * 8;  // work item of each stage, -1: no more
     static constexpr int OFF_MISC = OFF_ITEM + STAGES * 4;   // abort flag + 8 scan slots
@@ -134,7 +150,8 @@ struct DecodeParams {
     uint32_t* sched;
     int B, Hq, Hkv, MB, P, NP;
     int num_blocks;
-    float scale_log2;
+    float scale_log2;  // softmax scale x log2(e) (x k_scale for the 8-bit cache)
+    float v_scale;     // 8-bit cache: V = code x v_scale; 1 otherwise
     int out_bf16;
     // cluster mode: CS > 1 CTAs per (sequence, kv head), CTA rank r takes
     // partition r, and the cluster merges the partials in shared memory
@@ -497,17 +514,24 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             __syncwarp();
             if (mine) {
                 const int row0 = (cur_ent * p.Hkv + cur.h) * kPageRows;
+                if constexpr (L::F8) {
+                    // K: a [16][D] byte box; V (transposed): a [D][16] byte box
+                    tma_load_2d(kdst + k * L::PAGE_BYTES, tmk, 0, row0, &full[stage]);
+                    tma_load_2d(vdst + k * L::PAGE_BYTES, tmv, 0, (cur_ent * p.Hkv + cur.h) * D,
+                                &full[stage]);
+                } else {
 #pragma unroll
-                for (int bx = 0; bx < L::BOXES; ++bx) {
-                    tma_load_2d(kdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmk, bx * 64, row0,
-                                &full[stage]);
-                    tma_load_2d(vdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmv, bx * 64, row0,
-                                &full[stage]);
+                    for (int bx = 0; bx < L::BOXES; ++bx) {
+                        tma_load_2d(kdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmk, bx * 64,
+                                    row0, &full[stage]);
+                        tma_load_2d(vdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmv, bx * 64,
+                                    row0, &full[stage]);
+                    }
                 }
             }
             if (first && lane == 0) {
                 const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
-                                      ((size_t)cur.b * p.Hq + (size_t)cur.h * G) * D * L::ESZ;
+                                      ((size_t)cur.b * p.Hq + (size_t)cur.h * G) * D * L::QSZ;
                 bulk_load(base + L::OFF_Q + stage * L::Q_BYTES, qsrc, L::Q_COPY, &full[stage]);
             }
             if (FUSED && patch_row >= 0 && lane == 1) {
@@ -593,6 +617,8 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
 template <typename T, int D, int G>
 __device__ __forceinline__ float* merge_row(uint8_t* base, int st, int w, int g) {
     using L = Layout<T, D, G>;
+    if constexpr (!L::MERGE_IN_SLOTS)
+        return reinterpret_cast<float*>(base + L::OFF_MERGE + (w * G + g) * L::MERGE_ROW_BYTES);
     uint8_t* kslot = base + st * L::STAGE_BYTES + w * L::PPW * L::PAGE_BYTES;
     uint8_t* row = g < L::MERGE_ROWS_PER_SLOT
                        ? kslot + g * L::MERGE_ROW_BYTES
@@ -622,7 +648,8 @@ __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Ite
         }
         const size_t hq = (size_t)it.b * p.Hq + (size_t)it.h * G + g;
         // den == 0 only if every page of the item was rejected (bad block ids)
-        const float val = den > 0.f ? num / den : 0.f;
+        float val = den > 0.f ? num / den : 0.f;
+        if constexpr (Layout<T, D, G>::F8) val *= p.v_scale;
         if (p.cluster) {
             // cluster mode: this CTA's partial, merged across the cluster later
             float* part = reinterpret_cast<float*>(base + Layout<T, D, G>::OFF_Q) + g * (D + 2);
@@ -725,14 +752,29 @@ __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Ite
     }
 }
 
-// ------------------------------------------------- tensor-core consumer (bf16)
+// ------------------------------------- tensor-core consumer (bf16, 8-bit cache)
+//
+// The 8-bit cache (T = e4m3kv) runs the same tiles as f16 MMAs: E4M3 codes
+// widen to f16 exactly (cvt.rn.f16x2.e4m3x2), q is rounded to f16 (exact for
+// bf16 values of magnitude 2^-17 .. 65504), and P is split into two f16
+// terms.  Its fragments are read with plain shared-memory loads, in an
+// order that lets each lane take whole 16-byte rows or 4-byte runs:
+//   * scores: a lane's four k-values of k-step kk are the four consecutive
+//     dims (D/4) cq + 4 kk .. +3 (the same order for q and K, so q.K is
+//     unchanged), and lane row r of n-tile j reads token
+//     pi(8j + r) = 2r - (r & 1) + 2j of the page, so that the score columns a
+//     lane ends up with are the page's tokens 4 cq .. 4 cq + 3;
+//   * output: those four tokens are the lane's k-values of the P V MMA, four
+//     consecutive bytes of a transposed V row.
 
-template <int D, int G, bool FUSED>
+template <typename T, int D, int G, bool FUSED>
 __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
                                  uint64_t* full, uint64_t* empty, uint64_t* merge_bar,
                                  const uint32_t* masks, volatile int* s_abort, const int* s_len,
                                  const int* s_pre, int W) {
-    using L = Layout<bf16, D, G>;
+    using L = Layout<T, D, G>;
+    constexpr bool F8 = L::F8;
+    static_assert(!(F8 && FUSED), "the fused step takes bf16 or fp32 caches");
     constexpr int KS = D / 16;  // k-steps of the score MMA
     constexpr int NT = D / 8;   // n-tiles of the output MMA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -782,7 +824,17 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                 for (int kk = 0; kk < KS; ++kk) {
                     const int col = kk * 16 + 2 * cq;
                     uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-                    if (FUSED) {
+                    if constexpr (F8) {
+                        // dims (D/4) cq + 4 kk .. +3 of the head, as two f16 pairs
+                        auto quad = [&](int head, uint32_t& lo, uint32_t& hi) {
+                            const uint2 v = *reinterpret_cast<const uint2*>(
+                                qs + (head * D + (D / 4) * cq + 4 * kk) * 2);
+                            lo = pack_f16(bf16lo(v.x), bf16hi(v.x));
+                            hi = pack_f16(bf16lo(v.y), bf16hi(v.y));
+                        };
+                        if (head_a >= 0) quad(head_a, a0, a2);
+                        if (head_b >= 0) quad(head_b, a1, a3);
+                    } else if (FUSED) {
                         // the staged q is the raw (unrotated) input: rotate the
                         // lane's own elements on the way into the fragment
                         auto pair = [&](int head, int c) -> uint32_t {
@@ -803,7 +855,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                         a0 = qr[col / 2];
                         a2 = qr[(col + 8) / 2];
                     }
-                    if (!FUSED && head_b >= 0) {
+                    if (!F8 && !FUSED && head_b >= 0) {
                         const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_b * D * 2);
                         a1 = qr[col / 2];
                         a3 = qr[(col + 8) / 2];
@@ -828,7 +880,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                                    ? min(kPageRows, it.t1 - (it.t0 + jj * kPageRows))
                                    : 0;
                     if (valid[u] > 0)
-                        item_patch_page<bf16, D, G, FUSED>(p, it, jj, warp * PPW + u, stage, base);
+                        item_patch_page<T, D, G, FUSED>(p, it, jj, warp * PPW + u, stage, base);
                 }
                 const uint32_t kbase =
                     smem_addr(base + stage * L::STAGE_BYTES + warp * PPW * L::PAGE_BYTES);
@@ -839,17 +891,48 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                 float sc[2 * PPW][4];
 #pragma unroll
                 for (int n = 0; n < 2 * PPW; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+                if constexpr (F8) {
+                    // lane row r of n-tile j: token pi(8j + r) of the page, its
+                    // bytes (D/4) cq .. (D/4)(cq + 1) - 1, one word per k-step
+                    uint32_t kw[PPW][2][KS];
 #pragma unroll
-                for (int kk = 0; kk < KS; ++kk) {
-                    const int tok = ri + ((mi >> 1) << 3);
-                    const int ch = 2 * kk + (mi & 1);
+                    for (int u = 0; u < PPW; ++u)
 #pragma unroll
-                    for (int u = 0; u < PPW; ++u) {
-                        uint32_t b00, b01, b10, b11;
-                        ldsm_x4(kbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch), b00, b01,
-                                b10, b11);
-                        mma_bf16_16816(sc[2 * u], qa[kk], b00, b01);
-                        mma_bf16_16816(sc[2 * u + 1], qa[kk], b10, b11);
+                        for (int j = 0; j < 2; ++j) {
+                            const int tok = 2 * r - (r & 1) + 2 * j;
+                            const uint32_t row = kbase + u * L::PAGE_BYTES + tok * D;
+                            if constexpr (D == 64) {
+                                ld_shared_v4(row + 16 * cq, kw[u][j][0], kw[u][j][1], kw[u][j][2],
+                                             kw[u][j][3]);
+                            } else {
+                                // 128B swizzle: 16-byte chunk c of the row sits at c ^ (tok & 7)
+                                ld_shared_v4(row + (((2 * cq) ^ (tok & 7)) << 4), kw[u][j][0],
+                                             kw[u][j][1], kw[u][j][2], kw[u][j][3]);
+                                ld_shared_v4(row + (((2 * cq + 1) ^ (tok & 7)) << 4), kw[u][j][4],
+                                             kw[u][j][5], kw[u][j][6], kw[u][j][7]);
+                            }
+                        }
+#pragma unroll
+                    for (int kk = 0; kk < KS; ++kk)
+#pragma unroll
+                        for (int u = 0; u < PPW; ++u)
+#pragma unroll
+                            for (int j = 0; j < 2; ++j)
+                                mma_f16_16816(sc[2 * u + j], qa[kk], e4m3x2_to_f16x2(kw[u][j][kk]),
+                                              e4m3x2_to_f16x2(kw[u][j][kk] >> 16));
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < KS; ++kk) {
+                        const int tok = ri + ((mi >> 1) << 3);
+                        const int ch = 2 * kk + (mi & 1);
+#pragma unroll
+                        for (int u = 0; u < PPW; ++u) {
+                            uint32_t b00, b01, b10, b11;
+                            ldsm_x4(kbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch), b00,
+                                    b01, b10, b11);
+                            mma_bf16_16816(sc[2 * u], qa[kk], b00, b01);
+                            mma_bf16_16816(sc[2 * u + 1], qa[kk], b10, b11);
+                        }
                     }
                 }
                 // online softmax in the log2 domain; rows r carry c0, c1
@@ -858,7 +941,8 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                 for (int n = 0; n < 2 * PPW; ++n)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int tk = (n & 1) * 8 + 2 * cq + e;
+                        // token of the page in this score register
+                        const int tk = F8 ? 4 * cq + 2 * (n & 1) + e : (n & 1) * 8 + 2 * cq + e;
                         x[n][e] = tk < valid[n >> 1] ? sc[n][e] * p.scale_log2 : kNegInf;
                     }
                 float mx = kNegInf;
@@ -896,10 +980,18 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                     {
                         const float(&p0)[2] = pr[2 * u];
                         const float(&p1)[2] = pr[2 * u + 1];
-                        const uint32_t hi0 = pack_bf16(p0[0], p0[1]);
-                        const uint32_t hi1 = pack_bf16(p1[0], p1[1]);
-                        const uint32_t lo0 = pack_bf16(p0[0] - bf16lo(hi0), p0[1] - bf16hi(hi0));
-                        const uint32_t lo1 = pack_bf16(p1[0] - bf16lo(hi1), p1[1] - bf16hi(hi1));
+                        uint32_t hi0, hi1, lo0, lo1;
+                        if constexpr (F8) {
+                            hi0 = pack_f16(p0[0], p0[1]);
+                            hi1 = pack_f16(p1[0], p1[1]);
+                            lo0 = pack_f16(p0[0] - f16lo(hi0), p0[1] - f16hi(hi0));
+                            lo1 = pack_f16(p1[0] - f16lo(hi1), p1[1] - f16hi(hi1));
+                        } else {
+                            hi0 = pack_bf16(p0[0], p0[1]);
+                            hi1 = pack_bf16(p1[0], p1[1]);
+                            lo0 = pack_bf16(p0[0] - bf16lo(hi0), p0[1] - bf16hi(hi0));
+                            lo1 = pack_bf16(p1[0] - bf16lo(hi1), p1[1] - bf16hi(hi1));
+                        }
                         if (G == 8) {
                             pa[0] = hi0;
                             pa[1] = lo0;
@@ -914,22 +1006,36 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                     }
                     // O += P V over the page's 16 tokens (rows past `valid` are zeroed:
                     // they may hold stale or never-written shared memory)
-                    uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
-                    if (valid[u] < kPageRows) {
-                        const int k0 = 2 * cq, vu = valid[u];
-                        vmask_lo = (k0 < vu ? 0x0000ffffu : 0u) | (k0 + 1 < vu ? 0xffff0000u : 0u);
-                        vmask_hi = (k0 + 8 < vu ? 0x0000ffffu : 0u) |
-                                   (k0 + 9 < vu ? 0xffff0000u : 0u);
-                    }
+                    if constexpr (F8) {
+                        // lane (r, cq), n-tile c: dim 8c + r, tokens 4cq .. 4cq + 3
+                        const int rem = valid[u] - 4 * cq;
+                        const uint32_t bm = rem >= 4 ? 0xffffffffu
+                                                     : (rem <= 0 ? 0u : (1u << (8 * rem)) - 1u);
+                        const uint32_t vrow = vbase + u * L::PAGE_BYTES + r * 16 + 4 * cq;
 #pragma unroll
-                    for (int c = 0; c < NT; c += 2) {
-                        const int tok = ri + ((mi & 1) << 3);
-                        const int ch = c + (mi >> 1);
-                        uint32_t v0, v1, v2, v3;
-                        ldsm_x4_trans(vbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch), v0,
-                                      v1, v2, v3);
-                        mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
-                        mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
+                        for (int c = 0; c < NT; ++c) {
+                            const uint32_t w = ld_shared_u32(vrow + c * 128) & bm;
+                            mma_f16_16816(o[c], pa, e4m3x2_to_f16x2(w), e4m3x2_to_f16x2(w >> 16));
+                        }
+                    } else {
+                        uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
+                        if (valid[u] < kPageRows) {
+                            const int k0 = 2 * cq, vu = valid[u];
+                            vmask_lo = (k0 < vu ? 0x0000ffffu : 0u) |
+                                       (k0 + 1 < vu ? 0xffff0000u : 0u);
+                            vmask_hi = (k0 + 8 < vu ? 0x0000ffffu : 0u) |
+                                       (k0 + 9 < vu ? 0xffff0000u : 0u);
+                        }
+#pragma unroll
+                        for (int c = 0; c < NT; c += 2) {
+                            const int tok = ri + ((mi & 1) << 3);
+                            const int ch = c + (mi >> 1);
+                            uint32_t v0, v1, v2, v3;
+                            ldsm_x4_trans(vbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch),
+                                          v0, v1, v2, v3);
+                            mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
+                            mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
+                        }
                     }
                 }
             }
@@ -964,7 +1070,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
         if (r < G) {
-            float* row = merge_row<bf16, D, G>(base, last, warp, r);
+            float* row = merge_row<T, D, G>(base, last, warp, r);
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 row[n * 8 + 2 * cq] = of[n][0];
@@ -986,7 +1092,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
             return -1;
         }
         mphase ^= 1;
-        merge_and_store<bf16, D, G>(p, it, base, last);
+        merge_and_store<T, D, G>(p, it, base, last);
         ++merged;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[last]);
@@ -1354,8 +1460,8 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         }
         int merged;
         if constexpr (MMA) {
-            merged = run_consumer_mma<D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks,
-                                                   s_abort, s_len, s_pre, W);
+            merged = run_consumer_mma<T, D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks,
+                                                      s_abort, s_len, s_pre, W);
         } else {
             merged = run_consumer_simt<T, D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks,
                                                        s_abort, s_len, s_pre, W);
@@ -1631,7 +1737,8 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     p.P = a.partition_tokens;
     p.NP = a.max_partitions;
     p.num_blocks = (int)a.num_blocks;
-    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.scale_log2 = a.scale * 1.4426950408889634f * (L::F8 ? a.k_scale : 1.0f);
+    p.v_scale = L::F8 ? a.v_scale : 1.0f;
     p.out_bf16 = a.out_dtype == PKV_DTYPE_BF16;
     p.k_new = a.k_new;
     p.v_new = a.v_new;
@@ -1734,6 +1841,14 @@ cudaError_t dispatch_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensor
 
 template <bool FUSED>
 cudaError_t dispatch_all(const DecodeArgs& a, const CUtensorMap& tmk, const CUtensorMap& tmv) {
+    if (a.kv_dtype == PKV_DTYPE_E4M3) {
+        if constexpr (FUSED) {
+            return cudaErrorInvalidValue;  // the fused step takes bf16 or fp32 caches
+        } else {
+            return a.D == 64 ? dispatch_g<e4m3kv, 64, true, false>(a, tmk, tmv)
+                             : dispatch_g<e4m3kv, 128, true, false>(a, tmk, tmv);
+        }
+    }
     if (a.kv_dtype == PKV_DTYPE_F32) {
         return a.D == 64 ? dispatch_g<float, 64, false, FUSED>(a, tmk, tmv)
                          : dispatch_g<float, 128, false, FUSED>(a, tmk, tmv);
@@ -1750,6 +1865,8 @@ cudaError_t dispatch_all(const DecodeArgs& a, const CUtensorMap& tmk, const CUte
 
 cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks, int64_t Hkv,
                              int64_t D, int32_t dtype);
+cudaError_t encode_vt_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
+                                int64_t Hkv, int64_t D);
 
 cudaError_t launch_paged_decode(const DecodeArgs& a) {
     CUtensorMap tmk, tmv;
@@ -1760,7 +1877,9 @@ cudaError_t launch_paged_decode(const DecodeArgs& a) {
     }
     cudaError_t e = encode_cache_map(&tmk, a.k_cache, a.num_blocks, a.Hkv, a.D, a.kv_dtype);
     if (e != cudaSuccess) return e;
-    e = encode_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D, a.kv_dtype);
+    e = a.kv_dtype == PKV_DTYPE_E4M3 ? encode_vt_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D)
+                                     : encode_cache_map(&tmv, a.v_cache, a.num_blocks, a.Hkv, a.D,
+                                                        a.kv_dtype);
     if (e != cudaSuccess) return e;
     return a.fused ? dispatch_all<true>(a, tmk, tmv) : dispatch_all<false>(a, tmk, tmv);
 }
@@ -1798,6 +1917,9 @@ int decode_ctas_per_sm(int64_t D, int64_t G, int32_t kv_dtype, bool simt, int64_
     if (kv_dtype == PKV_DTYPE_F32) {
         if (D == 64) by_g(float{}, std::integral_constant<int, 64>{});
         else by_g(float{}, std::integral_constant<int, 128>{});
+    } else if (kv_dtype == PKV_DTYPE_E4M3) {
+        if (D == 64) by_g(e4m3kv{}, std::integral_constant<int, 64>{});
+        else by_g(e4m3kv{}, std::integral_constant<int, 128>{});
     } else {
         if (D == 64) by_g(bf16{}, std::integral_constant<int, 64>{});
         else by_g(bf16{}, std::integral_constant<int, 128>{});

@@ -77,15 +77,37 @@ cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_bl
     auto fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     const bool bf = dtype == PKV_DTYPE_BF16;
+    const bool f8 = dtype == PKV_DTYPE_E4M3;
+    const int esz = f8 ? 1 : (bf ? 2 : 4);
     const cuuint64_t rows = (cuuint64_t)(num_blocks * Hkv * kPageRows);
     cuuint64_t dims[2] = {(cuuint64_t)D, rows};
-    cuuint64_t strides[1] = {(cuuint64_t)(D * (bf ? 2 : 4))};
+    cuuint64_t strides[1] = {(cuuint64_t)(D * esz)};
     cuuint32_t box[2] = {(cuuint32_t)(bf ? 64 : D), (cuuint32_t)kPageRows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-                    const_cast<void*>(cache), dims, strides, box, estr,
+    // bf16 boxes are 128-byte rows, swizzled; 8-bit rows of 128 bytes too
+    const bool swz = bf || (f8 && D == 128);
+    CUresult r = fn(map,
+                    f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                       : (bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32),
+                    2, const_cast<void*>(cache), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    bf ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The 8-bit cache's transposed V pages [num_blocks, Hkv, D, 16] (bytes): rows
+// of 16 tokens, one [D][16] box per page.
+cudaError_t encode_vt_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
+                                int64_t Hkv, int64_t D) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)kPageRows, (cuuint64_t)(num_blocks * Hkv * D)};
+    cuuint64_t strides[1] = {(cuuint64_t)kPageRows};
+    cuuint32_t box[2] = {(cuuint32_t)kPageRows, (cuuint32_t)D};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(cache), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -124,6 +146,8 @@ pkv_status check_heads(int64_t Hq, int64_t Hkv, int64_t D, int64_t bs) {
 }
 
 bool valid_dtype(int32_t t) { return t == PKV_DTYPE_F32 || t == PKV_DTYPE_BF16; }
+// Cache dtypes the planning calls accept (the 8-bit cache included).
+bool valid_kv_dtype(int32_t t) { return valid_dtype(t) || t == PKV_DTYPE_E4M3; }
 
 // Partition length.  A partition should fill whole stages of the ring and be
 // long enough that the per-item work (q fragments, merge, partial store)
@@ -217,14 +241,15 @@ pkv_status cuda_status(cudaError_t e, const char* what) {
 
 using namespace pkv;
 
-extern "C" {
-
-pkv_status pkv_kv_append(void* q, const void* k_new, const void* v_new, const int64_t* positions,
+namespace {
+// Validation and launch shared by pkv_kv_append and pkv_kv_append_e4m3
+// (e4m3: the caches are 8-bit, the scales apply).
+pkv_status append_common(void* q, const void* k_new, const void* v_new, const int64_t* positions,
                          const int64_t* slot_mapping, void* k_cache, void* v_cache,
                          int64_t num_tokens, int64_t num_q_heads, int64_t num_kv_heads,
                          int64_t head_dim, int64_t num_blocks, int64_t block_size, int32_t dtype,
-                         double rope_theta, int32_t* device_error, void* stream) {
-    set_last_error("");
+                         double rope_theta, int32_t* device_error, void* stream, bool e4m3,
+                         float k_scale, float v_scale) {
     if (num_tokens < 0) {
         set_last_error("num_tokens < 0");
         return PKV_ERR_INVALID_ARG;
@@ -258,7 +283,7 @@ pkv_status pkv_kv_append(void* q, const void* k_new, const void* v_new, const in
         set_last_error("misaligned tensor pointer (16 bytes for q/k/v/caches)");
         return PKV_ERR_INVALID_ARG;
     }
-    AppendArgs a;
+    AppendArgs a = {};
     a.q = q;
     a.k_new = k_new;
     a.v_new = v_new;
@@ -275,13 +300,30 @@ pkv_status pkv_kv_append(void* q, const void* k_new, const void* v_new, const in
     a.theta = rope_theta;
     a.device_error = device_error;
     a.stream = static_cast<cudaStream_t>(stream);
+    a.e4m3 = e4m3;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
     return cuda_status(launch_kv_append(a), "kv_append launch");
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_kv_append(void* q, const void* k_new, const void* v_new, const int64_t* positions,
+                         const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                         int64_t num_tokens, int64_t num_q_heads, int64_t num_kv_heads,
+                         int64_t head_dim, int64_t num_blocks, int64_t block_size, int32_t dtype,
+                         double rope_theta, int32_t* device_error, void* stream) {
+    set_last_error("");
+    return append_common(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, num_tokens,
+                         num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, dtype,
+                         rope_theta, device_error, stream, false, 1.f, 1.f);
 }
 
 int32_t pkv_decode_partition_tokens(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
                                     int64_t head_dim, int64_t max_blocks_per_seq,
                                     int64_t block_size, int32_t kv_dtype) {
-    if (num_seqs < 0 || max_blocks_per_seq < 0 || !valid_dtype(kv_dtype)) return 0;
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || !valid_kv_dtype(kv_dtype)) return 0;
     if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
     WorkspacePlan w;
     if (plan_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, kv_dtype,
@@ -293,7 +335,7 @@ int32_t pkv_decode_partition_tokens(int64_t num_seqs, int64_t num_q_heads, int64
 size_t pkv_decode_workspace_size(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
                                  int64_t head_dim, int64_t max_blocks_per_seq, int64_t block_size,
                                  int32_t kv_dtype, int32_t partition_tokens) {
-    if (num_seqs < 0 || max_blocks_per_seq < 0 || !valid_dtype(kv_dtype)) return 0;
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || !valid_kv_dtype(kv_dtype)) return 0;
     if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
     WorkspacePlan w;
     if (plan_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, kv_dtype,
@@ -306,9 +348,10 @@ int32_t pkv_decode_launches(int64_t num_seqs, int64_t num_q_heads, int64_t num_k
                             int64_t head_dim, int64_t max_blocks_per_seq, int64_t block_size,
                             int32_t kv_dtype, int32_t out_dtype, int32_t partition_tokens,
                             uint32_t flags, int32_t fused) {
-    if (num_seqs <= 0 || max_blocks_per_seq <= 0 || !valid_dtype(kv_dtype) ||
+    if (num_seqs <= 0 || max_blocks_per_seq <= 0 || !valid_kv_dtype(kv_dtype) ||
         !valid_dtype(out_dtype) || (flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_NO_CLUSTER)))
         return 0;
+    if (kv_dtype == PKV_DTYPE_E4M3 && (fused || (flags & PKV_DECODE_FORCE_SIMT))) return 0;
     if (num_seqs > PKV_MAX_SEQS_PER_CALL) return 0;
     if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
     WorkspacePlan w;
@@ -359,16 +402,35 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
                          int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq,
                          int32_t kv_dtype, int32_t out_dtype, float scale,
                          int32_t partition_tokens, uint32_t flags, int32_t* device_error,
-                         void* stream, const StepExtras* step) {
+                         void* stream, const StepExtras* step, const float* kv_scales = nullptr) {
     if (num_seqs < 0 || max_blocks_per_seq < 0) {
         set_last_error("negative num_seqs or max_blocks_per_seq");
         return PKV_ERR_INVALID_ARG;
     }
     pkv_status st = check_heads(num_q_heads, num_kv_heads, head_dim, block_size);
     if (st != PKV_OK) return st;
-    if (!valid_dtype(kv_dtype) || !valid_dtype(out_dtype)) {
+    if (kv_dtype == PKV_DTYPE_E4M3 && !kv_scales) {
+        set_last_error("the 8-bit cache is decoded by pkv_paged_attention_decode_e4m3");
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (!valid_kv_dtype(kv_dtype) || !valid_dtype(out_dtype)) {
         set_last_error("kv_dtype/out_dtype unsupported");
         return PKV_ERR_UNSUPPORTED;
+    }
+    if (kv_dtype == PKV_DTYPE_E4M3) {
+        if (step || (flags & PKV_DECODE_FORCE_SIMT)) {
+            set_last_error("the 8-bit cache has no fused step and no CUDA-core kernel");
+            return PKV_ERR_UNSUPPORTED;
+        }
+        for (int i = 0; i < 2; ++i)
+            if (!(kv_scales[i] > 0.f) || kv_scales[i] == INFINITY) {
+                set_last_error("k_scale and v_scale must be finite and > 0");
+                return PKV_ERR_INVALID_ARG;
+            }
+        if (num_blocks * num_kv_heads * head_dim > INT32_MAX) {
+            set_last_error("num_blocks %lld too large for the 8-bit cache", (long long)num_blocks);
+            return PKV_ERR_INVALID_ARG;
+        }
     }
     if ((flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_NO_CLUSTER)) != 0) {
         set_last_error("unknown flags 0x%x", flags);
@@ -446,6 +508,8 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
     a.MB = max_blocks_per_seq;
     a.kv_dtype = kv_dtype;
     a.out_dtype = out_dtype;
+    a.k_scale = kv_scales ? kv_scales[0] : 1.f;
+    a.v_scale = kv_scales ? kv_scales[1] : 1.f;
     a.partition_tokens = w.P;
     a.max_partitions = w.NP;
     a.scale = scale;
@@ -499,6 +563,47 @@ pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new, const 
                          workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
                          num_blocks, block_size, max_blocks_per_seq, kv_dtype, out_dtype, scale,
                          partition_tokens, flags, device_error, stream, &step);
+}
+
+pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
+                                           const void* v_cache, const int32_t* block_tables,
+                                           const int32_t* context_lens, void* out,
+                                           void* workspace, size_t workspace_bytes,
+                                           int64_t num_seqs, int64_t num_q_heads,
+                                           int64_t num_kv_heads, int64_t head_dim,
+                                           int64_t num_blocks, int64_t block_size,
+                                           int64_t max_blocks_per_seq, int32_t out_dtype,
+                                           float scale, float k_scale, float v_scale,
+                                           int32_t partition_tokens, uint32_t flags,
+                                           int32_t* device_error, void* stream) {
+    set_last_error("");
+    const float scales[2] = {k_scale, v_scale};
+    return decode_common(q, k_cache, v_cache, block_tables, context_lens, out, workspace,
+                         workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                         num_blocks, block_size, max_blocks_per_seq, PKV_DTYPE_E4M3, out_dtype,
+                         scale, partition_tokens, flags, device_error, stream, nullptr, scales);
+}
+
+pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,
+                              const int64_t* positions, const int64_t* slot_mapping,
+                              void* k_cache, void* v_cache, int64_t num_tokens,
+                              int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                              int64_t num_blocks, int64_t block_size, int32_t dtype,
+                              double rope_theta, float k_scale, float v_scale,
+                              int32_t* device_error, void* stream) {
+    set_last_error("");
+    if (!(k_scale > 0.f) || k_scale == INFINITY || !(v_scale > 0.f) || v_scale == INFINITY) {
+        set_last_error("k_scale and v_scale must be finite and > 0");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (num_blocks > 0 && num_kv_heads > 0 && head_dim > 0 &&
+        num_blocks * num_kv_heads * head_dim > INT32_MAX) {
+        set_last_error("num_blocks %lld too large for the 8-bit cache", (long long)num_blocks);
+        return PKV_ERR_INVALID_ARG;
+    }
+    return append_common(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, num_tokens,
+                         num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, dtype,
+                         rope_theta, device_error, stream, true, k_scale, v_scale);
 }
 
 }  // extern "C"

@@ -29,10 +29,13 @@ struct AppendArgs {
     void* k_cache;
     void* v_cache;
     int64_t num_tokens, Hq, Hkv, D, num_blocks;
-    int32_t dtype;
+    int32_t dtype;       // of q, k_new, v_new (and of the caches unless e4m3)
     double theta;
     int32_t* device_error;
     cudaStream_t stream;
+    // 8-bit cache: codes of k / k_scale and v / v_scale; V pages transposed
+    bool e4m3;
+    float k_scale, v_scale;
 };
 cudaError_t launch_kv_append(const AppendArgs& a);
 
@@ -47,7 +50,8 @@ struct DecodeArgs {
     float* part_ml;  // [B, Hq, NP, 2]
     uint32_t* sched; // scheduler counters (2 x u32, zero between launches); null: static
     int64_t B, Hq, Hkv, D, num_blocks, MB;
-    int32_t kv_dtype, out_dtype;
+    int32_t kv_dtype, out_dtype;  // kv_dtype PKV_DTYPE_E4M3: q is bf16
+    float k_scale, v_scale;       // 8-bit cache only (1 otherwise)
     int32_t partition_tokens;  // P (resolved, multiple of 16)
     int32_t max_partitions;    // NP = ceil(MB * 16 / P)
     float scale;

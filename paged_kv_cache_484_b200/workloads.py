@@ -234,6 +234,28 @@ class SequenceSubset:
     scale: float
 
 
+def e4m3_cache(w: Workload, chunk_blocks: int = 4096):
+    """The workload's cached K/V as an 8-bit cache: one scale per tensor
+    (max |x| / 448, so the largest value maps to the largest E4M3 number) and
+    PyTorch's float8_e4m3fn cast of x / scale, as uint8 codes; the V pages
+    transposed to [num_blocks, Hkv, d, block_size].  Returns (k_cache,
+    v_cache, k_scale, v_scale); the cast is PyTorch's, not the library's."""
+    def amax(t):
+        return max(float(t[i:i + chunk_blocks].float().abs().max())
+                   for i in range(0, t.shape[0], chunk_blocks))
+
+    ks, vs = amax(w.k_cache) / 448.0, amax(w.v_cache) / 448.0
+    NB, Hkv, bs, d = w.k_cache.shape
+    k8 = torch.empty((NB, Hkv, bs, d), dtype=torch.uint8, device=w.k_cache.device)
+    v8 = torch.empty((NB, Hkv, d, bs), dtype=torch.uint8, device=w.v_cache.device)
+    for i in range(0, NB, chunk_blocks):
+        j = min(NB, i + chunk_blocks)
+        k8[i:j] = (w.k_cache[i:j].float() / ks).to(torch.float8_e4m3fn).view(torch.uint8)
+        v8[i:j] = (w.v_cache[i:j].float() / vs).to(torch.float8_e4m3fn).view(torch.uint8) \
+            .transpose(2, 3)
+    return k8, v8, ks, vs
+
+
 def extract_sequences(w: Workload, seqs) -> SequenceSubset:
     """Copy the inputs of sequences ``seqs`` to the host (read before any step
     modifies the workload's tensors)."""

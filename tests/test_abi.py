@@ -116,6 +116,70 @@ def test_decode_rejects_bad_arguments(lib, kw, status):
     assert _decode(lib, **kw) == status
 
 
+
+E4M3 = 2
+
+
+def _append8(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, slot=FAKE, kc=FAKE, vc=FAKE, T=1, Hq=8, Hkv=2, d=64,
+             NB=4, bs=16, dtype=BF16, theta=1e4, ks=0.05, vs=0.05, err=None)
+    a.update(kw)
+    return lib.pkv_kv_append_e4m3(a["q"], a["k"], a["v"], a["pos"], a["slot"], a["kc"], a["vc"],
+                                  a["T"], a["Hq"], a["Hkv"], a["d"], a["NB"], a["bs"], a["dtype"],
+                                  a["theta"], a["ks"], a["vs"], a["err"], None)
+
+
+def _decode8(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, out=FAKE, ws=None, wsb=0, B=2, Hq=8, Hkv=2,
+             d=64, NB=4, bs=16, MB=4, odt=BF16, scale=0.125, ks=0.05, vs=0.05, P=0, flags=0,
+             err=None)
+    a.update(kw)
+    return lib.pkv_paged_attention_decode_e4m3(
+        a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"], a["ws"], a["wsb"], a["B"], a["Hq"],
+        a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"], a["odt"], a["scale"], a["ks"], a["vs"],
+        a["P"], a["flags"], a["err"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ks=0.0), INVALID),
+    (dict(vs=-1.0), INVALID),
+    (dict(ks=math.inf), INVALID),
+    (dict(vs=math.nan), INVALID),
+    (dict(dtype=E4M3), UNSUPPORTED),       # q / k_new / v_new are float32 or bfloat16
+    (dict(d=96), UNSUPPORTED),
+    (dict(kc=FAKE + 8), INVALID),
+    (dict(NB=1 << 26, Hkv=8, d=128), INVALID),   # byte rows past int32 tensor coordinates
+    (dict(T=0, q=None, k=None), OK),
+])
+def test_kv_append_e4m3_rejects_bad_arguments(lib, kw, status):
+    assert _append8(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ks=0.0), INVALID),
+    (dict(vs=math.nan), INVALID),
+    (dict(flags=0x1), UNSUPPORTED),        # no CUDA-core kernel for the 8-bit cache
+    (dict(odt=E4M3), UNSUPPORTED),
+    (dict(d=96), UNSUPPORTED),
+    (dict(P=16, MB=4), WORKSPACE),
+    (dict(vc=FAKE + 4), INVALID),
+    (dict(B=0, q=None, out=None), OK),
+])
+def test_decode_e4m3_rejects_bad_arguments(lib, kw, status):
+    assert _decode8(lib, **kw) == status
+
+
+def test_e4m3_planning(lib):
+    """The planning calls take the 8-bit cache dtype: the workspace follows
+    the same formula; the fused step and the CUDA-core kernel do not exist
+    for it."""
+    for P in (0, 64, 1024):
+        assert lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, E4M3, P) == \
+            lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, BF16, P)
+    assert lib.pkv_decode_partition_tokens(64, 32, 8, 64, 257, 16, E4M3) > 0
+    assert lib.pkv_decode_launches(4, 32, 8, 64, 16, 16, E4M3, BF16, 0, 0, 1) == 0
+    assert lib.pkv_decode_launches(4, 32, 8, 64, 16, 16, E4M3, BF16, 0, 1, 0) == 0
+
 def test_workspace_size_formula(lib):
     # 16 sequences, 32/8 heads, d 128, contexts up to 8193 blocks, P = 1024
     n = lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, BF16, 1024)
