@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -421,17 +422,22 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
         return v;
     };
 
+    // Block-table entries are loaded a chunk ahead and range-checked only when
+    // their chunk comes up: a check right after the load would stall the warp
+    // on it (the error report is a side effect the compiler cannot defer).
+    constexpr int kNoPage = INT_MIN;  // lane past the item's last page
     auto checked = [&](int v) -> int {
+        if (v == kNoPage) return -1;
         if (v < 0 || v >= p.num_blocks) {
             report_error(p.err, PKV_DEVERR_BLOCK_ID);
             return -1;
         }
         return v;
     };
-    auto entry = [&](const Item& it, int page) -> int {
-        if (page >= it.npages) return -1;
+    auto raw_entry = [&](const Item& it, int page) -> int {
+        if (page >= it.npages) return kNoPage;
         const int jb = it.t0 / kPageRows + page;
-        return checked(p.block_tables[(size_t)it.b * p.MB + jb]);
+        return p.block_tables[(size_t)it.b * p.MB + jb];
     };
 
     int stage = 0;
@@ -444,7 +450,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
     Item cur = decode_item(item, p, s_len, s_pre);
     int c0 = 0;
     const bool hit = cur.b == guess.b && cur.part == guess.part;
-    int cur_ent = hit ? (lane < cur.npages ? checked(guess.ent) : -1) : entry(cur, lane);
+    int cur_ent = hit ? (lane < cur.npages ? checked(guess.ent) : -1) : checked(raw_entry(cur, lane));
     // fused step: the new token's slot and position
     int64_t cur_slot = -1, cur_pos = 0;
     if constexpr (FUSED) {
@@ -462,7 +468,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             nc0 = 0;
             if (nitem < W) nxt = decode_item(nitem, p, s_len, s_pre);
         }
-        const int nxt_ent = (nitem < W) ? entry(nxt, nc0 + lane) : -1;
+        const int nxt_raw = (nitem < W) ? raw_entry(nxt, nc0 + lane) : kNoPage;
         const bool new_item = FUSED && nitem != item && nitem < W;
         const int64_t nxt_slot = new_item ? p.slot_mapping[nxt.b] : cur_slot;
         const int64_t nxt_pos = new_item ? p.positions[nxt.b] : cur_pos;
@@ -575,7 +581,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
         item = nitem;
         c0 = nc0;
         cur = nxt;
-        cur_ent = nxt_ent;
+        cur_ent = checked(nxt_raw);
         cur_slot = nxt_slot;
         cur_pos = nxt_pos;
     }
@@ -917,9 +923,11 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
 #pragma unroll
                         for (int u = 0; u < PPW; ++u)
 #pragma unroll
-                            for (int j = 0; j < 2; ++j)
-                                mma_f16_16816(sc[2 * u + j], qa[kk], e4m3x2_to_f16x2(kw[u][j][kk]),
-                                              e4m3x2_to_f16x2(kw[u][j][kk] >> 16));
+                            for (int j = 0; j < 2; ++j) {
+                                uint32_t b0, b1;
+                                e4m3x4_to_f16x4(kw[u][j][kk], b0, b1);
+                                mma_f16_16816(sc[2 * u + j], qa[kk], b0, b1);
+                            }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < KS; ++kk) {
@@ -1014,8 +1022,9 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                         const uint32_t vrow = vbase + u * L::PAGE_BYTES + r * 16 + 4 * cq;
 #pragma unroll
                         for (int c = 0; c < NT; ++c) {
-                            const uint32_t w = ld_shared_u32(vrow + c * 128) & bm;
-                            mma_f16_16816(o[c], pa, e4m3x2_to_f16x2(w), e4m3x2_to_f16x2(w >> 16));
+                            uint32_t b0, b1;
+                            e4m3x4_to_f16x4(ld_shared_u32(vrow + c * 128) & bm, b0, b1);
+                            mma_f16_16816(o[c], pa, b0, b1);
                         }
                     } else {
                         uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;

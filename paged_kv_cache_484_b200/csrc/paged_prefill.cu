@@ -130,15 +130,19 @@ __device__ void prefill_producer(const PrefillParams& p, const PItem& it, const 
     uint32_t issued_parity[8];
     uint32_t issued_any = 0;
     bool abort = false;
+    // block-table entries of the next 32-page chunk are loaded while this one
+    // is issued, and range-checked when their chunk comes up
+    const int32_t* row_tab = p.block_tables + (size_t)it.b * p.MB + it.t0 / kPageRows;
+    int raw = lane < it.npages ? row_tab[lane] : -1;
     for (int c0 = 0; c0 < it.npages && !abort; c0 += 32) {
         int ent = -1;
         if (c0 + lane < it.npages) {
-            const int v = p.block_tables[(size_t)it.b * p.MB + it.t0 / kPageRows + c0 + lane];
-            if (v < 0 || v >= p.num_blocks)
+            if (raw < 0 || raw >= p.num_blocks)
                 report_error(p.err, PKV_DEVERR_BLOCK_ID);
             else
-                ent = v;
+                ent = raw;
         }
+        raw = c0 + 32 + lane < it.npages ? row_tab[c0 + 32 + lane] : -1;
         const int cend = min(it.npages, c0 + 32);
         for (int s0 = c0; s0 < cend; s0 += L::SP) {
             const int npg = min(L::SP, it.npages - s0);

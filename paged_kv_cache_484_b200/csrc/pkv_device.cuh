@@ -195,13 +195,13 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_
 }
 
 // ---- 8-bit floating point (E4M3) -------------------------------------------
-// Two E4M3 codes (low byte, high byte of `pair`) -> f16 pair, low byte in the
-// low half.  Exact: every E4M3 value is an f16 normal number.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
-    uint32_t r;
-    const uint16_t h = (uint16_t)pair;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
-    return r;
+// Four E4M3 codes (bytes 0..3 of `w`) -> two f16 pairs: `lo` from bytes 0, 1,
+// `hi` from bytes 2, 3 (the halves of `w` feed the conversions directly).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 // Two floats -> E4M3 codes (nearest even, saturating to +-448), `lo` in the
 // low byte of the result.
