@@ -376,11 +376,16 @@ def run_ours(args):
     ncopies = 1 if nbytes >= 2 * l2 else min(1024, math.ceil(2 * l2 / nbytes))
     if args.copies:
         ncopies = args.copies
-    fields = ("q", "k_new", "v_new", "positions", "slot_mapping", "k_cache", "v_cache",
-              "block_tables", "decode_lens")
-    copies = [dict((f, getattr(w, f)) for f in fields)]
+    # Per-layer tensors (q, the new rows, the caches) get their own copy; the
+    # step's metadata (positions, slots, block tables, context lengths) is one
+    # set shared by all copies, as one decode step's metadata is shared by all
+    # layers of a model.
+    layer_fields = ("q", "k_new", "v_new", "k_cache", "v_cache")
+    step_fields = ("positions", "slot_mapping", "block_tables", "decode_lens")
+    copies = [dict((f, getattr(w, f)) for f in layer_fields + step_fields)]
     for _ in range(ncopies - 1):
-        copies.append(dict((f, getattr(w, f).clone()) for f in fields))
+        copies.append(dict([(f, getattr(w, f).clone()) for f in layer_fields] +
+                           [(f, getattr(w, f)) for f in step_fields]))
     outs = [torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=device) for _ in range(ncopies)]
 
     cascade = args.cascade
@@ -625,8 +630,10 @@ def run_ours(args):
                        **({"step": "two calls (kv_append, paged_attention_decode_cascade over "
                                    "the prefix groups)"} if cascade else {}),
                        l2=(f"inputs larger than L2 ({l2 >> 20} MiB): " +
-                           (f"{ncopies} device-side copies of the workload, step k on copy k mod "
-                            f"{ncopies} ({nbytes / 1e6:.1f} MB read per step)" if ncopies > 1 else
+                           (f"{ncopies} device-side copies of the per-layer tensors (q, new rows, "
+                            f"K/V caches; the step's block tables, context lengths, positions "
+                            f"and slots shared, as by the layers of a model), step k on copy k "
+                            f"mod {ncopies} ({nbytes / 1e6:.1f} MB read per step)" if ncopies > 1 else
                             f"the workload reads {nbytes / 1e6:.1f} MB per step") +
                            "; no flush inside the timed region")),
         "isolated_step": {"ms_per_step": round(iso_ms, 5),
@@ -697,9 +704,10 @@ def run_prefill(args):
         w.B * C * w.Hq * w.d * (2 + esz_out)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     ncopies = args.copies or (1 if nbytes >= 2 * l2 else min(1024, math.ceil(2 * l2 / nbytes)))
+    # per-layer q and caches copied; the block tables and lengths shared
     copies = [dict(q=q, k=w.k_cache, v=w.v_cache, t=w.block_tables, l=lens)]
     for _ in range(ncopies - 1):
-        copies.append({k: v.clone() for k, v in copies[0].items()})
+        copies.append({k: (v.clone() if k in ("q", "k", "v") else v) for k, v in copies[0].items()})
     outs = [torch.empty((w.B, C, w.Hq, w.d), dtype=out_dtype, device=device)
             for _ in range(ncopies)]
     err = torch.zeros(1, dtype=torch.int32, device=device)

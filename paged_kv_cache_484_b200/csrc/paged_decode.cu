@@ -123,10 +123,10 @@ struct Layout {
     static constexpr int OFF_MERGE = OFF_ROPE + STAGES * ROPE_BYTES;
     static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
     static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
-    // Cluster mode: the CTA's merged partial (o[D], m, l per head) sits in the
-    // q / new-row / rope-table slots once the CTA's one item is done.
+    // Cluster mode: every CTA of a cluster stores its merged partial (o[D], m,
+    // l per head) into slot `rank` of a landing area in rank 0's shared memory,
+    // past everything else (rank 0 may still be computing when they land).
     static constexpr int CLUSTER_PART_BYTES = G * (D + 2) * 4;
-    static_assert(OFF_MERGE - OFF_Q >= CLUSTER_PART_BYTES, "cluster partial does not fit");
     static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
     static constexpr int OFF_ITEM = OFF_PATCH + STAGES * 8;  // work item of each stage, -1: no more
     static constexpr int OFF_MISC = OFF_ITEM + STAGES * 4;   // abort flag + 8 scan slots
@@ -135,6 +135,13 @@ struct Layout {
     static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;
     static size_t smem_bytes(int B) {
         return 1024 + OFF_SEQ + (size_t)(2 * B + 1) * 4 + (B <= kLptMaxSeqs ? (size_t)2 * B * 4 : 0);
+    }
+    // cluster mode: the landing area (16-byte aligned, after the sequence arrays)
+    __host__ __device__ static constexpr int land_offset(int B) {
+        return round_up(OFF_SEQ + (2 * B + 1) * 4 + (B <= kLptMaxSeqs ? 2 * B * 4 : 0), 16);
+    }
+    static size_t cluster_smem_bytes(int B, int cs) {
+        return 1024 + (size_t)land_offset(B) + (size_t)cs * CLUSTER_PART_BYTES;
     }
 };
 
@@ -633,6 +640,14 @@ __device__ __forceinline__ float* merge_row(uint8_t* base, int st, int w, int g)
     return reinterpret_cast<float*>(row);
 }
 
+// Cluster mode: slot `r` of the landing area (local address; map it to rank 0
+// for a remote store).
+template <typename T, int D, int G>
+__device__ __forceinline__ float* cluster_slot(const DecodeParams& p, uint8_t* base, int r) {
+    using L = Layout<T, D, G>;
+    return reinterpret_cast<float*>(base + L::land_offset(p.B) + r * L::CLUSTER_PART_BYTES);
+}
+
 // All consumer warps have written (o, m, l) per head into their merge rows
 // of stage `st`; merge them and write the output row or the partition
 // partial.
@@ -657,12 +672,13 @@ __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Ite
         float val = den > 0.f ? num / den : 0.f;
         if constexpr (Layout<T, D, G>::F8) val *= p.v_scale;
         if (p.cluster) {
-            // cluster mode: this CTA's partial, merged across the cluster later
-            float* part = reinterpret_cast<float*>(base + Layout<T, D, G>::OFF_Q) + g * (D + 2);
-            part[dim] = val;
+            // cluster mode: this CTA's partial goes straight into its slot of
+            // rank 0's landing area (distributed shared memory)
+            const float* part = cluster_slot<T, D, G>(p, base, cluster_ctarank()) + g * (D + 2);
+            st_dsmem_f32(dsmem_addr(part + dim, 0), val);
             if (dim == 0) {
-                part[D] = M;
-                part[D + 1] = den;
+                st_dsmem_f32(dsmem_addr(part + D, 0), M);
+                st_dsmem_f32(dsmem_addr(part + D + 1, 0), den);
             }
         } else if (it.np == 1 && it.slot0 == 0) {
             store_out(p.out, hq * D + dim, val, p.out_bf16);
@@ -677,52 +693,36 @@ __device__ __forceinline__ void merge_and_store(const DecodeParams& p, const Ite
     }
 }
 
-// Cluster mode, after every CTA of the cluster holds its partial in its own
-// shared memory (an empty one, m = -inf and l = 0, when it had no partition
-// or gave up): CTA rank 0 reads all of them through distributed shared
-// memory and writes out[b, h*G .. h*G+G-1, :], the same log-sum-exp merge as
-// the combine kernel.  Every thread of every CTA of the cluster calls this
-// exactly once (it holds the two cluster barriers).
+// Cluster mode, once every CTA of the cluster has stored its partial into its
+// slot of rank 0's landing area (an empty one, m = -inf and l = 0, when it had
+// no partition or gave up): one cluster barrier (release / acquire, so the
+// remote stores are visible), then rank 0 merges the slots from its own
+// shared memory and writes out[b, h*G .. h*G+G-1, :], the same log-sum-exp
+// merge as the combine kernel.  The other CTAs leave after the barrier:
+// nothing reads their shared memory.  Every thread of every CTA of the
+// cluster calls this exactly once (it holds the cluster barrier).
 template <typename T, int D, int G>
 __device__ void cluster_merge(const DecodeParams& p, uint8_t* base) {
-    using L = Layout<T, D, G>;
-    cluster_sync_all();  // all partials written (release / acquire at cluster scope)
+    cluster_sync_all();
     const int CS = p.cluster;
-    if (cluster_ctarank() == 0 && threadIdx.x < NW * 32) {
-        const int cid = blockIdx.x / CS;
-        const int b = cid / p.Hkv, h = cid - (cid / p.Hkv) * p.Hkv;
-        const float* part = reinterpret_cast<const float*>(base + L::OFF_Q);
-        for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
-            const int g = idx / D, dim = idx - (idx / D) * D;
-            const float* row = part + g * (D + 2);
-            // all remote loads first (independent, so they overlap), then the merge
-            float m[kMaxClusterCtas], l[kMaxClusterCtas], v[kMaxClusterCtas];
-#pragma unroll
-            for (int r = 0; r < kMaxClusterCtas; ++r) {
-                m[r] = kNegInf;
-                l[r] = 0.f;
-                v[r] = 0.f;
-                if (r < CS) {
-                    m[r] = ld_dsmem_f32(dsmem_addr(row + D, r));
-                    l[r] = ld_dsmem_f32(dsmem_addr(row + D + 1, r));
-                    v[r] = ld_dsmem_f32(dsmem_addr(row + dim, r));
-                }
-            }
-            float M = kNegInf;
-#pragma unroll
-            for (int r = 0; r < kMaxClusterCtas; ++r) M = fmaxf(M, m[r]);
-            float num = 0.f, den = 0.f;
-#pragma unroll
-            for (int r = 0; r < kMaxClusterCtas; ++r) {
-                const float w = (m[r] == kNegInf || l[r] == 0.f) ? 0.f : l[r] * fast_exp2(m[r] - M);
-                num = fmaf(w, v[r], num);
-                den += w;
-            }
-            const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
-            store_out(p.out, hq * D + dim, den > 0.f ? num / den : 0.f, p.out_bf16);
+    if (cluster_ctarank() != 0 || threadIdx.x >= NW * 32) return;
+    const int cid = blockIdx.x / CS;
+    const int b = cid / p.Hkv, h = cid - (cid / p.Hkv) * p.Hkv;
+    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+        const int g = idx / D, dim = idx - (idx / D) * D;
+        float M = kNegInf;
+        for (int r = 0; r < CS; ++r) M = fmaxf(M, cluster_slot<T, D, G>(p, base, r)[g * (D + 2) + D]);
+        float num = 0.f, den = 0.f;
+        for (int r = 0; r < CS; ++r) {
+            const float* row = cluster_slot<T, D, G>(p, base, r) + g * (D + 2);
+            const float m = row[D], l = row[D + 1];
+            const float w = (m == kNegInf || l == 0.f) ? 0.f : l * fast_exp2(m - M);
+            num = fmaf(w, row[dim], num);
+            den += w;
         }
+        const size_t hq = (size_t)b * p.Hq + (size_t)h * G + g;
+        store_out(p.out, hq * D + dim, den > 0.f ? num / den : 0.f, p.out_bf16);
     }
-    cluster_sync_all();  // no CTA leaves while rank 0 may still read its memory
 }
 
 // Bounded barrier of the consumer warps (every consumer thread arrives).
@@ -1477,9 +1477,9 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         }
         if (p.cluster && merged <= 0) {
             // no partition here (or this CTA gave up): an empty partial
-            float* part = reinterpret_cast<float*>(base + L::OFF_Q);
+            const float* part = cluster_slot<T, D, G>(p, base, cluster_ctarank());
             for (int idx = tid; idx < G * (D + 2); idx += NW * 32)
-                part[idx] = (idx % (D + 2)) == D ? kNegInf : 0.f;
+                st_dsmem_f32(dsmem_addr(part + idx, 0), (idx % (D + 2)) == D ? kNegInf : 0.f);
         }
     }
     if (p.cluster) cluster_merge<T, D, G>(p, base);
@@ -1669,8 +1669,13 @@ cudaError_t prepare_kernel(K kern, size_t smem, int* ctas_per_sm) {
         *ctas_per_sm = it->second;
         return cudaSuccess;
     }
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)std::max(smem, kClusterCtaSmem));
+    // allow up to the device's opt-in maximum: cluster-mode launches ask for
+    // more than the layout (spreading, plus the landing area of rank 0)
+    int optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    if ((size_t)optin < smem) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e != cudaSuccess) return e;
     int n = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, smem);
@@ -1766,9 +1771,13 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     // NP CTAs resident at once, the partitions are merged inside the cluster
     // and the combine kernel is not needed.
     int cs = 0;
-    const size_t smem_cl = std::max(smem, kClusterCtaSmem);
+    const size_t smem_cl =
+        std::max(L::cluster_smem_bytes((int)a.B, std::max(2, a.max_partitions)), kClusterCtaSmem);
+    int optin = 0;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, current_device());
+    if (e != cudaSuccess) return e;
     if (a.allow_cluster && !a.shared_tokens && a.max_partitions >= 2 &&
-        a.max_partitions <= kMaxClusterCtas) {
+        a.max_partitions <= kMaxClusterCtas && smem_cl <= (size_t)optin) {
         int nc = 0;
         e = max_active_clusters(kern, smem_cl, a.max_partitions, &nc);
         if (e != cudaSuccess) return e;
