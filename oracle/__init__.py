@@ -68,11 +68,11 @@ class Oracle:
             lib.orc_kv_append.argtypes = [i32, vp, vp, vp, vp, vp, vp, vp,
                                           i64, i64, i64, i64, i64, i64, dbl]
             lib.orc_paged_decode.argtypes = [i32, i32, vp, vp, vp, vp, vp,
-                                             i64, i64, i64, i64, i64, i64, i64, dbl,
+                                             i64, i64, i64, i64, i64, i64, i64, dbl, i64,
                                              vp, i64, i32, vp]
             lib.orc_paged_decode_e4m3.argtypes = [i32, vp, vp, vp, vp, vp,
                                                   i64, i64, i64, i64, i64, i64, i64, dbl, dbl,
-                                                  dbl, vp, i64, i32, vp]
+                                                  dbl, i64, vp, i64, i32, vp]
             lib.orc_kv_append_e4m3.argtypes = [i32, vp, vp, vp, vp, vp, vp, vp,
                                                i64, i64, i64, i64, i64, i64, dbl, dbl, dbl]
             lib.orc_round_e4m3.argtypes = [vp, vp, i64]
@@ -143,11 +143,12 @@ class Oracle:
                                       T, Hq, Hkv, d, NB, bs, float(rope_theta)))
 
     def paged_attention_decode(self, q, k_cache, v_cache, block_tables, context_lens, scale,
-                               pairs=None, nthreads: int = 1) -> torch.Tensor:
+                               pairs=None, nthreads: int = 1, window: int = 0) -> torch.Tensor:
         """fp64 [B, Hq, d] output of single-query attention over paged K/V.
 
         ``pairs`` ([n, 2] int64 of (b, h)) restricts the work to those outputs;
-        the other rows of the result are left as NaN.
+        the other rows of the result are left as NaN.  ``window`` > 0: each
+        query attends to the last ``window`` tokens of its context only.
         """
         _cpu(q)
         _cpu(k_cache)
@@ -168,7 +169,8 @@ class Oracle:
         _check(self.lib.orc_paged_decode(_storage_code(q), _storage_code(k_cache), _ptr(q),
                                          _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                          _ptr(context_lens), B, Hq, Hkv, d, NB, bs, MB,
-                                         float(scale), pp, npairs, int(nthreads), _ptr(out)))
+                                         float(scale), int(window), pp, npairs, int(nthreads),
+                                         _ptr(out)))
         return out
 
     def kv_append_e4m3(self, q, k_new, v_new, positions, slot_mapping, k_cache, v_cache,
@@ -198,8 +200,8 @@ class Oracle:
                                            float(k_scale), float(v_scale)))
 
     def paged_attention_decode_e4m3(self, q, k_cache, v_cache, block_tables, context_lens, scale,
-                                    k_scale, v_scale, pairs=None,
-                                    nthreads: int = 1) -> torch.Tensor:
+                                    k_scale, v_scale, pairs=None, nthreads: int = 1,
+                                    window: int = 0) -> torch.Tensor:
         """fp64 [B, Hq, d] decode over an E4M3 cache (k_cache [NB, Hkv, bs, d],
         v_cache [NB, Hkv, d, bs], uint8); ``pairs`` as in paged_attention_decode."""
         _cpu(q)
@@ -221,8 +223,8 @@ class Oracle:
         _check(self.lib.orc_paged_decode_e4m3(_storage_code(q), _ptr(q), _ptr(k_cache),
                                               _ptr(v_cache), _ptr(block_tables),
                                               _ptr(context_lens), B, Hq, Hkv, d, NB, bs, MB,
-                                              float(scale), float(k_scale), float(v_scale), pp,
-                                              npairs, int(nthreads), _ptr(out)))
+                                              float(scale), float(k_scale), float(v_scale),
+                                              int(window), pp, npairs, int(nthreads), _ptr(out)))
         return out
 
     def paged_chunked_prefill(self, q, k_cache, v_cache, block_tables, context_lens, scale,

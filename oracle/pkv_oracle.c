@@ -54,6 +54,10 @@
  *     s % block_size.  A negative slot means "do not write this token".
  *   - Query head h reads kv head h / (Hq / Hkv) (contiguous groups).
  *   - A context of length 0 produces an all-zero output row.
+ *   - Sliding window W > 0 ([EFF] "KV Caching: Verify Reuse, Positions and
+ *     Windows"): the query at the last position of a context of L tokens
+ *     attends to its last min(W, L) tokens, L - W .. L - 1 (itself
+ *     included); W = 0 means no window.
  *   - 8-bit cache: one scale per tensor (k_scale, v_scale); the stored code
  *     of a value x is x / scale (fp64) rounded to binary32, then to the
  *     nearest E4M3 value, ties to even, saturating to +-448.  The binary32
@@ -329,8 +333,9 @@ int orc_kv_append_e4m3(int dtype, void* q, const void* k_new, const void* v_new,
 /* ---- paged decode ([BOOK] ch. 8 and ch. 10; [PROJ] M2, M13b) -----------
  *
  * For sequence b with L = context_lens[b] and query head h (kv head
- * kvh = h / (Hq / Hkv)):
- *   K[t] = k_cache[block_tables[b][t / bs], kvh, t % bs, :]   for t < L
+ * kvh = h / (Hq / Hkv)), over the tokens t0 <= t < L where t0 = 0, or
+ * max(0, L - window) with a sliding window:
+ *   K[t] = k_cache[block_tables[b][t / bs], kvh, t % bs, :]
  *   s_t  = scale * sum_i q[b, h, i] * K[t][i]
  *   M    = max_t s_t ;   w_t = exp(s_t - M)
  *   out[b, h, :] = sum_t w_t V[t] / sum_t w_t          (zeros when L == 0)
@@ -342,6 +347,7 @@ typedef struct {
     int64_t B, Hq, Hkv, d, num_blocks, bs, MB;
     double scale;
     double k_scale, v_scale; /* E4M3 cache only */
+    int64_t window;          /* 0: none */
     const int64_t* pairs; /* optional list of (b, h) pairs */
     int64_t npairs;
     double* out;
@@ -375,8 +381,9 @@ static int decode_one(const decode_job* J, int64_t b, int64_t h, double* s) {
     if (L == 0) return ORC_OK;
 
     const int64_t qbase = (b * J->Hq + h) * d;
+    const int64_t t0 = (J->window > 0 && L > J->window) ? L - J->window : 0;
     double M = -INFINITY;
-    for (int64_t t = 0; t < L; ++t) {
+    for (int64_t t = t0; t < L; ++t) {
         int64_t blk = J->block_tables[b * J->MB + t / J->bs];
         if (blk < 0 || blk >= J->num_blocks) return ORC_EBLOCK;
         double acc = 0.0;
@@ -386,7 +393,7 @@ static int decode_one(const decode_job* J, int64_t b, int64_t h, double* s) {
         if (s[t] > M) M = s[t];
     }
     double den = 0.0;
-    for (int64_t t = 0; t < L; ++t) {
+    for (int64_t t = t0; t < L; ++t) {
         double w = exp(s[t] - M);
         den += w;
         int64_t blk = J->block_tables[b * J->MB + t / J->bs];
@@ -418,8 +425,9 @@ static int run_decode(int q_dtype, int kv_dtype, const void* q,
                       const int32_t* block_tables, const int32_t* context_lens,
                       int64_t B, int64_t Hq, int64_t Hkv, int64_t d,
                       int64_t num_blocks, int64_t bs, int64_t MB, double scale,
-                      double k_scale, double v_scale,
+                      double k_scale, double v_scale, int64_t window,
                       const int64_t* pairs, int64_t npairs, int nthreads, double* out) {
+    if (window < 0) return ORC_EARG;
     if (B < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || d <= 0 || bs <= 0 || MB < 0 ||
         num_blocks <= 0 || npairs < 0)
         return ORC_EARG;
@@ -438,8 +446,8 @@ static int run_decode(int q_dtype, int kv_dtype, const void* q,
     if (!jobs || !th) { free(jobs); free(th); return ORC_ENOMEM; }
     for (int i = 0; i < nthreads; ++i) {
         decode_job J = {q_dtype, kv_dtype, q, k_cache, v_cache, block_tables, context_lens,
-                        B, Hq, Hkv, d, num_blocks, bs, MB, scale, k_scale, v_scale, pairs,
-                        npairs, out, nthreads, i, ORC_OK};
+                        B, Hq, Hkv, d, num_blocks, bs, MB, scale, k_scale, v_scale, window,
+                        pairs, npairs, out, nthreads, i, ORC_OK};
         jobs[i] = J;
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, decode_worker, &jobs[i]);
@@ -457,12 +465,13 @@ int orc_paged_decode(int q_dtype, int kv_dtype, const void* q,
                      const void* k_cache, const void* v_cache,
                      const int32_t* block_tables, const int32_t* context_lens,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t d,
-                     int64_t num_blocks, int64_t bs, int64_t MB, double scale,
+                     int64_t num_blocks, int64_t bs, int64_t MB, double scale, int64_t window,
                      const int64_t* pairs, int64_t npairs, int nthreads, double* out) {
     if ((q_dtype != ORC_F32 && q_dtype != ORC_BF16) || (kv_dtype != ORC_F32 && kv_dtype != ORC_BF16))
         return ORC_EARG;
     return run_decode(q_dtype, kv_dtype, q, k_cache, v_cache, block_tables, context_lens, B, Hq,
-                      Hkv, d, num_blocks, bs, MB, scale, 1.0, 1.0, pairs, npairs, nthreads, out);
+                      Hkv, d, num_blocks, bs, MB, scale, 1.0, 1.0, window, pairs, npairs,
+                      nthreads, out);
 }
 
 /* The decode over an E4M3 cache: the same definition with
@@ -473,13 +482,13 @@ int orc_paged_decode_e4m3(int q_dtype, const void* q,
                           const int32_t* block_tables, const int32_t* context_lens,
                           int64_t B, int64_t Hq, int64_t Hkv, int64_t d,
                           int64_t num_blocks, int64_t bs, int64_t MB, double scale,
-                          double k_scale, double v_scale,
+                          double k_scale, double v_scale, int64_t window,
                           const int64_t* pairs, int64_t npairs, int nthreads, double* out) {
     if (q_dtype != ORC_F32 && q_dtype != ORC_BF16) return ORC_EARG;
     if (!(k_scale > 0.0) || !(v_scale > 0.0) || isinf(k_scale) || isinf(v_scale)) return ORC_EARG;
     return run_decode(q_dtype, ORC_E4M3, q, k_cache, v_cache, block_tables, context_lens, B, Hq,
-                      Hkv, d, num_blocks, bs, MB, scale, k_scale, v_scale, pairs, npairs, nthreads,
-                      out);
+                      Hkv, d, num_blocks, bs, MB, scale, k_scale, v_scale, window, pairs, npairs,
+                      nthreads, out);
 }
 
 /* ---- self-check variants (same definition, no paging) ------------------ */

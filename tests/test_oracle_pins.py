@@ -642,6 +642,41 @@ def pin_append_e4m3_placement_and_values(orc: Oracle):
             assert torch.equal(vc[s // bs, :, :, s % bs], cast(v[t].double() / vs)), f"v codes {t}"
 
 
+
+def pin_sliding_window_decode(orc: Oracle):
+    """A sliding window of W tokens equals attention over the last W tokens
+    of the context (PyTorch fp64 SDPA on that slice), for bf16 and fp32
+    storage, GQA groups and the 8-bit cache; a window at least as long as
+    the context changes nothing; W = 1 returns the last token's V exactly
+    ("Efficient LLM Inference", KV Caching: positions and windows)."""
+    lens = [40, 17, 5, 33]
+    cl = torch.tensor(lens, dtype=torch.int32)
+    for dtype, Hq, Hkv in ((torch.float32, 8, 2), (torch.bfloat16, 4, 4)):
+        kpool, vpool, tables, Ks, Vs = random_paged(lens, Hkv, 16, 16, dtype, 80)
+        q = torch.randn(len(lens), Hq, 16, generator=_gen(81)).to(dtype)
+        full = orc.paged_attention_decode(q, kpool, vpool, tables, cl, 0.25)
+        for W in (1, 7, 16, 17, 33, 100):
+            got = orc.paged_attention_decode(q, kpool, vpool, tables, cl, 0.25, window=W)
+            for b, L in enumerate(lens):
+                if W >= L:
+                    assert torch.equal(got[b], full[b]), f"window {W} >= L {L} changed the result"
+                    continue
+                s0 = L - W
+                want = sdpa(q[b][None].double(), Ks[b][s0:].double(), Vs[b][s0:].double(), 0.25)[0]
+                assert_close(got[b], want, 1e-12, f"window {W} b={b}")
+                if W == 1:
+                    G = Hq // Hkv
+                    last = Vs[b][L - 1].double().repeat_interleave(G, dim=0)
+                    assert torch.equal(got[b], last), "W = 1 is not the last V"
+    kc, vc, tables, Ks, Vs = _random_e4m3_cache(lens, 2, 16, 16, 82)
+    q = torch.randn(len(lens), 8, 16, generator=_gen(83)).to(torch.bfloat16)
+    got = orc.paged_attention_decode_e4m3(q, kc, vc, tables, cl, 0.25, 0.05, 0.07, window=9)
+    for b, L in enumerate(lens):
+        s0 = max(0, L - 9)
+        want = sdpa(q[b][None].double(), _e4m3_value(Ks[b][s0:]) * 0.05,
+                    _e4m3_value(Vs[b][s0:]) * 0.07, 0.25)[0]
+        assert_close(got[b], want, 1e-12, f"e4m3 window b={b}")
+
 PINS = [
     pin_round_bf16_matches_torch_cast,
     pin_round_bf16_single_rounding,
@@ -666,6 +701,7 @@ PINS = [
     pin_e4m3_quantizer_rounds_through_binary32,
     pin_e4m3_decode_matches_sdpa_over_dequantized,
     pin_append_e4m3_placement_and_values,
+    pin_sliding_window_decode,
 ]
 
 
@@ -686,8 +722,8 @@ MUTATIONS = [
      "int64_t idx = ((kvh * J->num_blocks + blk) * J->bs + row) * J->d + i;"),
     ("row_index", "int64_t idx = ((blk * J->Hkv + kvh) * J->bs + row) * J->d + i;",
      "int64_t idx = ((blk * J->Hkv + kvh) * J->bs + (row + 1) % J->bs) * J->d + i;"),
-    ("drop_last_token", "for (int64_t t = 0; t < L; ++t) {\n        double w",
-     "for (int64_t t = 0; t + 1 < L; ++t) {\n        double w"),
+    ("drop_last_token", "for (int64_t t = t0; t < L; ++t) {\n        double w",
+     "for (int64_t t = t0; t + 1 < L; ++t) {\n        double w"),
     ("normalise_by_length", "for (int64_t i = 0; i < d; ++i) o[i] /= den;\n    return ORC_OK;",
      "for (int64_t i = 0; i < d; ++i) o[i] /= (double)L;\n    return ORC_OK;"),
     ("rope_sign", "x[i] = x0 * c - x1 * s;", "x[i] = x0 * c + x1 * s;"),
@@ -723,6 +759,10 @@ MUTATIONS = [
     ("e4m3_k_unrotated", "for (int64_t i = 0; i < d; ++i) k_cache[page + r * d + i] =",
      "for (int64_t i = 0; i < d; ++i) row[i] = load_elem(k_new, dtype, src + i);\n"
      "            for (int64_t i = 0; i < d; ++i) k_cache[page + r * d + i] ="),
+    ("window_start_late", "const int64_t t0 = (J->window > 0 && L > J->window) ? L - J->window : 0;",
+     "const int64_t t0 = (J->window > 0 && L > J->window) ? L - J->window + 1 : 0;"),
+    ("window_start_early", "const int64_t t0 = (J->window > 0 && L > J->window) ? L - J->window : 0;",
+     "const int64_t t0 = (J->window > 0 && L > J->window) ? L - J->window - 1 : 0;"),
     ("skip_q_rotation", "rope_rotate(row, d, pos, theta);\n        for (int64_t i = 0; i < d; ++i) store_elem(q,",
      "for (int64_t i = 0; i < d; ++i) store_elem(q,"),
 ]
