@@ -61,6 +61,8 @@ def parse_args(argv=None):
     ap.add_argument("--copies", type=int, default=0,
                     help="device-side copies of the workload (0: enough to exceed L2)")
     ap.add_argument("--simt", action="store_true", help="bf16: CUDA-core decode kernel")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window: each query attends to the last W tokens (two calls)")
     ap.add_argument("--kv-dtype", default="native", choices=["native", "e4m3"],
                     help="e4m3: the workload's cache as an 8-bit cache (per-tensor scales), "
                          "stepped as kv_append_e4m3 + paged_attention_decode_e4m3")
@@ -123,11 +125,15 @@ def esize(dt):
     return 2 if dt == torch.bfloat16 else 4
 
 
-def step_bytes(w, out_dtype) -> int:
-    """Algorithmic bytes of one decode call: every context token's K and V
-    row once per KV head (at the cache's element size), plus q read and out
-    written."""
-    L = int(w.decode_lens.to(torch.int64).sum().item())
+def step_bytes(w, out_dtype, window=0) -> int:
+    """Algorithmic bytes of one decode call: every attended context token's K
+    and V row once per KV head (at the cache's element size), plus q read and
+    out written.  With a sliding window only the last ``window`` tokens of a
+    context count."""
+    lens = w.decode_lens.to(torch.int64)
+    if window:
+        lens = lens.clamp(max=window)
+    L = int(lens.sum().item())
     kv = L * w.Hkv * w.d * 2 * w.k_cache.element_size()
     qo = w.B * w.Hq * w.d * (esize(w.dtype) + esize(out_dtype))
     return kv + qo
@@ -259,7 +265,7 @@ def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
 
 # ---------------------------------------------------------------- oracle arm
 
-def time_oracle(w, seconds: float, nthreads: int, e4m3_scales=None):
+def time_oracle(w, seconds: float, nthreads: int, e4m3_scales=None, window: int = 0):
     """Oracle append + decode of the whole workload (or a bounded subset of
     sequences for the big ones), repeated until ~``seconds`` of CPU time
     (the 8-bit cache's append and decode when ``e4m3_scales`` is given)."""
@@ -276,7 +282,8 @@ def time_oracle(w, seconds: float, nthreads: int, e4m3_scales=None):
         seqs.append(b)
         tok += lens[b]
     sub = extract_sequences(w, seqs)
-    frac_bytes = sum(lens[b] for b in seqs) / max(1, sum(lens))
+    att = [min(L, window) if window else L for L in lens]  # attended tokens
+    frac_bytes = sum(att[b] for b in seqs) / max(1, sum(att))
     reps, t_total = 0, 0.0
     while t_total < seconds or reps == 0:
         q = sub.q.clone()
@@ -287,12 +294,12 @@ def time_oracle(w, seconds: float, nthreads: int, e4m3_scales=None):
             oracle.kv_append_e4m3(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions,
                                   sub.slots, kc, vc, sub.theta, ks, vs)
             oracle.paged_attention_decode_e4m3(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
-                                               ks, vs, nthreads=nthreads)
+                                               ks, vs, nthreads=nthreads, window=window)
         else:
             oracle.kv_append(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions, sub.slots,
                              kc, vc, sub.theta)
             oracle.paged_attention_decode(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
-                                          nthreads=nthreads)
+                                          nthreads=nthreads, window=window)
         t_total += time.perf_counter() - t0
         reps += 1
     return t_total / reps, seqs, frac_bytes, reps
@@ -368,7 +375,11 @@ def run_ours(args):
                                          partition_tokens=P)
     ws = pkv.new_workspace(ws_bytes, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
-    nbytes = step_bytes(w, out_dtype)
+    nbytes = step_bytes(w, out_dtype, args.window)
+    if args.window:
+        if args.cascade:
+            raise SystemExit("--window and --cascade do not combine")
+        args.two_calls = True
 
     # Inputs larger than L2: device-side copies of the workload (every tensor
     # a step reads or writes), step k on copy k mod n.
@@ -430,7 +441,7 @@ def run_ours(args):
             pkv.paged_attention_decode_e4m3(c["q"], c["k_cache"], c["v_cache"],
                                             c["block_tables"], c["decode_lens"], w.scale, ks8,
                                             vs8, out, workspace=ws, partition_tokens=P,
-                                            device_error=err)
+                                            device_error=err, sliding_window=args.window)
         elif fused:
             pkv.decode_step(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                             c["k_cache"], c["v_cache"], c["block_tables"], c["decode_lens"],
@@ -446,7 +457,7 @@ def run_ours(args):
             pkv.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
                                        c["decode_lens"], w.scale, out, workspace=ws,
                                        partition_tokens=P, force_simt=args.simt,
-                                       device_error=err)
+                                       device_error=err, sliding_window=args.window)
 
     def step(k):
         c = copies[k % ncopies]
@@ -612,7 +623,7 @@ def run_ours(args):
             k8c, v8c, _, _ = W.e4m3_cache(wc)
             wc.k_cache, wc.v_cache = k8c, v8c
         per_step, seqs, frac, reps = time_oracle(wc, args.cpu_seconds, nthreads,
-                                                 (ks8, vs8) if e4m3 else None)
+                                                 (ks8, vs8) if e4m3 else None, args.window)
         cpu = {"value": round(nbytes * frac / per_step / 1e9, 4), "unit": "GB/s",
                "cores": nthreads, "kind": "oracle",
                "sample": f"{len(seqs)} of {w.B} sequences, full append+decode step in fp64, "
@@ -627,6 +638,7 @@ def run_ours(args):
         "pct_of_hbm_peak": round(100.0 * value / (world * peak), 2),
         "seq_steps_per_s": round(world * w.B / (step_ms_max * 1e-3), 1),
         "config": dict(config_block(args.config, w, out_dtype, P, NP, args.simt, args.two_calls),
+                       **({"sliding_window": args.window} if args.window else {}),
                        **({"step": "two calls (kv_append, paged_attention_decode_cascade over "
                                    "the prefix groups)"} if cascade else {}),
                        l2=(f"inputs larger than L2 ({l2 >> 20} MiB): " +

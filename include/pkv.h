@@ -398,6 +398,7 @@ pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,
  *   q                  device, [num_seqs, Hq, head_dim] bf16
  *   k_cache, v_cache   device uint8, the layout above
  *   k_scale, v_scale   finite, > 0
+ *   sliding_window     0, or a window as in pkv_paged_attention_decode_window
  */
 pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
                                            const void* v_cache, const int32_t* block_tables,
@@ -408,8 +409,38 @@ pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
                                            int64_t num_blocks, int64_t block_size,
                                            int64_t max_blocks_per_seq, int32_t out_dtype,
                                            float scale, float k_scale, float v_scale,
-                                           int32_t partition_tokens, uint32_t flags,
-                                           int32_t* device_error, void* stream);
+                                           int32_t sliding_window, int32_t partition_tokens,
+                                           uint32_t flags, int32_t* device_error, void* stream);
+
+/*
+ * pkv_paged_attention_decode_window -- pkv_paged_attention_decode with a
+ * sliding window: each sequence's query attends to the last
+ * min(sliding_window, L) tokens of its context only, tokens
+ * max(0, L - sliding_window) .. L - 1 (itself included).
+ *
+ * Source: "Efficient LLM Inference", "KV Caching: Verify Reuse, Positions and
+ * Windows" (position windows on the cache; the window's exact extent is this
+ * library's reading).  Pages that lie wholly before the window are not read:
+ * a sequence's partitions start at the page of its window's first token, and
+ * the tokens before it in that page are masked.
+ *
+ * Arguments: those of pkv_paged_attention_decode, plus
+ *   sliding_window     >= 0; 0 = the whole context (the plain decode)
+ * The workspace is sized as for pkv_paged_attention_decode (the same shapes
+ * and partition_tokens).
+ */
+pkv_status pkv_paged_attention_decode_window(const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* block_tables,
+                                             const int32_t* context_lens, void* out,
+                                             void* workspace, size_t workspace_bytes,
+                                             int64_t num_seqs, int64_t num_q_heads,
+                                             int64_t num_kv_heads, int64_t head_dim,
+                                             int64_t num_blocks, int64_t block_size,
+                                             int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                             int32_t out_dtype, float scale,
+                                             int32_t sliding_window, int32_t partition_tokens,
+                                             uint32_t flags, int32_t* device_error,
+                                             void* stream);
 
 /*
  * pkv_paged_attention_decode_cascade -- pkv_paged_attention_decode for batches

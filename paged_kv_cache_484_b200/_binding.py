@@ -96,7 +96,11 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_kv_append_e4m3.restype = ctypes.c_int
         lib.pkv_paged_attention_decode_e4m3.argtypes = [
             vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64, i64, i32,
-            ctypes.c_float, ctypes.c_float, ctypes.c_float, i32, u32, vp, vp]
+            ctypes.c_float, ctypes.c_float, ctypes.c_float, i32, i32, u32, vp, vp]
+        lib.pkv_paged_attention_decode_window.argtypes = [
+            vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64, i64, i32,
+            i32, ctypes.c_float, i32, i32, u32, vp, vp]
+        lib.pkv_paged_attention_decode_window.restype = ctypes.c_int
         lib.pkv_paged_attention_decode_e4m3.restype = ctypes.c_int
         lib.pkv_bm_create.argtypes = [i32, i32]
         lib.pkv_bm_create.restype = vp
@@ -247,7 +251,7 @@ def new_workspace(nbytes, device) -> torch.Tensor:
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out,
                            stream=None, *, workspace=None, partition_tokens=0, force_simt=False,
-                           device_error=None, cluster=True) -> torch.Tensor:
+                           device_error=None, cluster=True, sliding_window=0) -> torch.Tensor:
     """Single-query attention over the paged cache; writes and returns ``out``.
 
     q [B, Hq, d] and caches [NB, Hkv, 16, d] share a dtype (float32 or
@@ -256,7 +260,9 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     at least ``decode_workspace_size`` bytes, see ``new_workspace``) is
     allocated from PyTorch's caching allocator when not given; an empty tensor
     passes none, which is allowed when no context is split (the work items
-    are then dealt out round-robin).  See include/pkv.h.
+    are then dealt out round-robin).  ``sliding_window`` > 0: each query
+    attends to the last ``sliding_window`` tokens of its context
+    (pkv_paged_attention_decode_window).  See include/pkv.h.
     """
     lib = load_library()
     kv_dt = _dtype_code(k_cache.dtype)
@@ -273,13 +279,16 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     if workspace is None:
         workspace = new_workspace(int(need), q.device)
     err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
-    st = lib.pkv_paged_attention_decode(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale), int(partition_tokens),
-        _flags(force_simt, cluster), err, _stream_ptr(stream, q.device))
+    args = [_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+            _dev(block_tables, "block_tables", torch.int32),
+            _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale)]
+    tail = [int(partition_tokens), _flags(force_simt, cluster), err, _stream_ptr(stream, q.device)]
+    if sliding_window:
+        st = lib.pkv_paged_attention_decode_window(*args, int(sliding_window), *tail)
+    else:
+        st = lib.pkv_paged_attention_decode(*args, *tail)
     _raise(st, lib, "paged_attention_decode")
     return out
 
@@ -314,7 +323,8 @@ def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, r
 
 def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale,
                                 v_scale, out, stream=None, *, workspace=None, partition_tokens=0,
-                                device_error=None, cluster=True) -> torch.Tensor:
+                                device_error=None, cluster=True,
+                                sliding_window=0) -> torch.Tensor:
     """``paged_attention_decode`` over the 8-bit cache (k_cache uint8
     [NB, Hkv, 16, d], v_cache uint8 [NB, Hkv, d, 16]); q bfloat16 [B, Hq, d];
     cached values are code x k_scale / code x v_scale.  Writes and returns
@@ -337,7 +347,7 @@ def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens,
         _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         B, Hq, Hkv, d, NB, bs, MB, _dtype_code(out.dtype), float(scale), float(k_scale),
-        float(v_scale), int(partition_tokens), _flags(False, cluster), err,
+        float(v_scale), int(sliding_window), int(partition_tokens), _flags(False, cluster), err,
         _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode_e4m3")
     return out

@@ -169,6 +169,9 @@ struct DecodeParams {
     // the shared-prefix pass (partial slot 0); this kernel takes the rest,
     // in partitions that start at that offset (slots 1..); null = off
     const int32_t* shared_tokens;
+    // sliding window: each query attends to the last `window` tokens of its
+    // context (0 = the whole context)
+    int window;
     // fused step only: the new token of every sequence
     const void* k_new;            // [B, Hkv, D]
     const void* v_new;            // [B, Hkv, D]
@@ -185,7 +188,17 @@ struct RopeFreq {
 struct Item {
     int b, h, part, t0, t1, npages, np;
     int slot0;  // cascade: 1 when the sequence's shared prefix owns partial slot 0
+    int lo;     // first token attended (sliding window; 0 otherwise)
 };
+
+// Sliding window: first token a context of Lb tokens attends to, and the
+// start of its page (where the sequence's partitions begin).
+__host__ __device__ __forceinline__ int window_start(int window, int Lb) {
+    return (window > 0 && Lb > window) ? Lb - window : 0;
+}
+__host__ __device__ __forceinline__ int window_page_start(int window, int Lb) {
+    return window_start(window, Lb) / kPageRows * kPageRows;
+}
 
 // Item i -> (sequence, kv head, partition).  Items are j * Hkv + h.  Without
 // the longest-first order, j runs over every sequence's partitions in order
@@ -201,7 +214,7 @@ __device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const 
     if (p.B <= kLptMaxSeqs && !p.cluster && !p.shared_tokens && j >= nfull) {
         const int* s_rank = s_pre + p.B + 1;
         it.b = s_rank[j - nfull];
-        it.np = (s_len[it.b] + p.P - 1) / p.P;
+        it.np = (s_len[it.b] - window_page_start(p.window, s_len[it.b]) + p.P - 1) / p.P;
         it.part = it.np - 1;
     } else {
         int lo = 0, hi = p.B - 1;  // largest b with s_pre[b] <= j
@@ -212,9 +225,11 @@ __device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const 
         }
         it.b = lo;
         it.part = j - s_pre[lo];
-        it.np = (s_len[lo] + p.P - 1) / p.P;
+        it.np = (s_len[lo] - window_page_start(p.window, s_len[lo]) + p.P - 1) / p.P;
     }
-    int off = 0;
+    // sliding window: partitions start at the page of the window's first token
+    int off = window_page_start(p.window, s_len[it.b]);
+    it.lo = window_start(p.window, s_len[it.b]);
     it.slot0 = 0;
     if (p.shared_tokens) {
         // cascade: partitions start after the tokens of the shared-prefix pass
@@ -410,7 +425,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
         // partition r, if the sequence has one, and nothing else
         const int CS = p.cluster, cid = blockIdx.x / CS, rank = blockIdx.x - cid * CS;
         const int b = cid / p.Hkv, h = cid - b * p.Hkv;
-        const int npb = (s_len[b] + p.P - 1) / p.P;
+        const int npb = (s_len[b] - window_page_start(p.window, s_len[b]) + p.P - 1) / p.P;
         item = rank < npb ? (s_pre[b] + rank) * p.Hkv + h : W;
         item1 = W;
     }
@@ -878,13 +893,16 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
             const int j0 = s * L::STAGE_PAGES + warp * PPW;
             const uint32_t mk = (masks[stage] >> (warp * PPW)) & ((1u << PPW) - 1u);
             if (j0 < it.npages && mk != 0u) {
-                int valid[PPW];
+                // tokens first[u] .. valid[u] - 1 of page u are attended (first > 0
+                // only where a sliding window starts inside the page)
+                int valid[PPW], first[PPW];
 #pragma unroll
                 for (int u = 0; u < PPW; ++u) {
                     const int jj = j0 + u;
                     valid[u] = (jj < it.npages && ((mk >> u) & 1u))
                                    ? min(kPageRows, it.t1 - (it.t0 + jj * kPageRows))
                                    : 0;
+                    first[u] = max(0, it.lo - (it.t0 + jj * kPageRows));
                     if (valid[u] > 0)
                         item_patch_page<T, D, G, FUSED>(p, it, jj, warp * PPW + u, stage, base);
                 }
@@ -951,7 +969,8 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                     for (int e = 0; e < 2; ++e) {
                         // token of the page in this score register
                         const int tk = F8 ? 4 * cq + 2 * (n & 1) + e : (n & 1) * 8 + 2 * cq + e;
-                        x[n][e] = tk < valid[n >> 1] ? sc[n][e] * p.scale_log2 : kNegInf;
+                        x[n][e] = (tk < valid[n >> 1] && tk >= first[n >> 1])
+                                      ? sc[n][e] * p.scale_log2 : kNegInf;
                     }
                 float mx = kNegInf;
 #pragma unroll
@@ -1016,9 +1035,14 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                     // they may hold stale or never-written shared memory)
                     if constexpr (F8) {
                         // lane (r, cq), n-tile c: dim 8c + r, tokens 4cq .. 4cq + 3
-                        const int rem = valid[u] - 4 * cq;
-                        const uint32_t bm = rem >= 4 ? 0xffffffffu
-                                                     : (rem <= 0 ? 0u : (1u << (8 * rem)) - 1u);
+                        uint32_t bm = 0xffffffffu;
+                        if (valid[u] < kPageRows || first[u] > 0) {
+                            bm = 0u;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                if (4 * cq + e >= first[u] && 4 * cq + e < valid[u])
+                                    bm |= 0xffu << (8 * e);
+                        }
                         const uint32_t vrow = vbase + u * L::PAGE_BYTES + r * 16 + 4 * cq;
 #pragma unroll
                         for (int c = 0; c < NT; ++c) {
@@ -1028,12 +1052,12 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                         }
                     } else {
                         uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
-                        if (valid[u] < kPageRows) {
-                            const int k0 = 2 * cq, vu = valid[u];
-                            vmask_lo = (k0 < vu ? 0x0000ffffu : 0u) |
-                                       (k0 + 1 < vu ? 0xffff0000u : 0u);
-                            vmask_hi = (k0 + 8 < vu ? 0x0000ffffu : 0u) |
-                                       (k0 + 9 < vu ? 0xffff0000u : 0u);
+                        if (valid[u] < kPageRows || first[u] > 0) {
+                            const int k0 = 2 * cq, vu = valid[u], fu = first[u];
+                            auto in = [&](int k) { return k >= fu && k < vu; };
+                            vmask_lo = (in(k0) ? 0x0000ffffu : 0u) | (in(k0 + 1) ? 0xffff0000u : 0u);
+                            vmask_hi = (in(k0 + 8) ? 0x0000ffffu : 0u) |
+                                       (in(k0 + 9) ? 0xffff0000u : 0u);
                         }
 #pragma unroll
                         for (int c = 0; c < NT; c += 2) {
@@ -1195,6 +1219,7 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
             const int j = s * L::STAGE_PAGES + slot;
             if (j < it.npages && ((masks[stage] >> slot) & 1u)) {
                 const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
+                const int first = max(0, it.lo - (it.t0 + j * kPageRows));  // sliding window
                 item_patch_page<T, D, G, FUSED>(p, it, j, slot, stage, base);
                 const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + slot * L::PAGE_BYTES);
                 const uint32_t vbase = kbase + L::STAGE_PAGES * L::PAGE_BYTES;
@@ -1216,7 +1241,7 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
 #pragma unroll
                         for (int g = 0; g < G; ++g)
                             sdot[g] += __shfl_xor_sync(0xffffffffu, sdot[g], off);
-                    if (tk < valid) {
+                    if (tk < valid && tk >= first) {
                         float vv[EPL];
                         load16(vbase + chunk_offset<T, D>(tk, c), vv);
 #pragma unroll
@@ -1369,7 +1394,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
             bs = j / p.NP;
             ps = j - bs * p.NP;
         }
-        if (bs < p.B && !p.shared_tokens) {
+        if (bs < p.B && !p.shared_tokens && !p.window) {
             const int jb = ps * (p.P / kPageRows) + lane;
             guess.b = bs;
             guess.part = ps;
@@ -1402,7 +1427,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
             Lb = Lb < 0 ? 0 : maxlen;
         }
         s_len[b] = Lb;
-        int off = 0;
+        int off = window_page_start(p.window, Lb);
         if (p.shared_tokens) {
             // cascade (at most kLptMaxSeqs sequences): whole pages, within the context
             off = p.shared_tokens[b];
@@ -1411,7 +1436,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         }
         const int npb = (Lb - off + p.P - 1) / p.P;
         const int cnt = lpt ? max(npb - 1, 0) : npb;
-        if (lpt) s_key[b] = Lb > 0 ? Lb - (npb - 1) * p.P : -1;  // tokens of the last partition
+        if (lpt) s_key[b] = Lb > 0 ? (Lb - off) - (npb - 1) * p.P : -1;  // tokens of the last partition
         s_pre[b] = cnt;
         local += cnt;
     }
@@ -1490,6 +1515,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
 struct CombineParams {
     const int32_t* context_lens;
     const int32_t* shared_tokens;  // cascade: slot 0 holds the shared-prefix partial
+    int window;                    // sliding window (partitions start at its page)
     const float* part_o;
     const float* part_ml;
     void* out;
@@ -1539,12 +1565,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_c
     }
     Lb = Lb < 0 ? 0 : (Lb > maxlen ? maxlen : Lb);
     int off = 0;
+    const int woff = window_page_start(p.window, Lb);
     if (p.shared_tokens) {
         off = p.shared_tokens[b];
         off = off < 0 ? 0 : (off > Lb ? Lb : off) / kPageRows * kPageRows;
     }
     // slots: the shared prefix (cascade, when it has tokens), then the partitions
-    const int np = (off > 0 ? 1 : 0) + (Lb - off + p.P - 1) / p.P;
+    const int np = (off > 0 ? 1 : 0) + (Lb - off - woff + p.P - 1) / p.P;
     if (np <= 1 && off == 0) return;  // written by the decode kernel
 
     // first partials of this thread, independent of the weights
@@ -1743,6 +1770,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     p.part_ml = a.part_ml;
     p.sched = a.sched;
     p.shared_tokens = a.shared_tokens;
+    p.window = a.window;
     p.err = a.device_error;
     p.B = (int)a.B;
     p.Hq = (int)a.Hq;
@@ -1825,6 +1853,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     cp.NP = a.max_partitions;
     cp.out_bf16 = p.out_bf16;
     cp.shared_tokens = a.shared_tokens;
+    cp.window = a.window;
     auto ckern = combine_kernel<D, G>;
     {
         static std::mutex mu;

@@ -402,7 +402,8 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
                          int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq,
                          int32_t kv_dtype, int32_t out_dtype, float scale,
                          int32_t partition_tokens, uint32_t flags, int32_t* device_error,
-                         void* stream, const StepExtras* step, const float* kv_scales = nullptr) {
+                         void* stream, const StepExtras* step, const float* kv_scales = nullptr,
+                         int32_t window = 0) {
     if (num_seqs < 0 || max_blocks_per_seq < 0) {
         set_last_error("negative num_seqs or max_blocks_per_seq");
         return PKV_ERR_INVALID_ARG;
@@ -454,6 +455,10 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
     }
     if (step && !(step->theta > 0.0)) {
         set_last_error("rope_theta must be > 0");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (window < 0) {
+        set_last_error("sliding_window must be >= 0");
         return PKV_ERR_INVALID_ARG;
     }
     WorkspacePlan w;
@@ -517,6 +522,7 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
     a.allow_cluster = (flags & PKV_DECODE_NO_CLUSTER) == 0;
     a.device_error = device_error;
     a.stream = static_cast<cudaStream_t>(stream);
+    a.window = window;
     a.fused = step != nullptr;
     if (step) {
         a.k_new = step->k_new;
@@ -574,14 +580,35 @@ pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
                                            int64_t num_blocks, int64_t block_size,
                                            int64_t max_blocks_per_seq, int32_t out_dtype,
                                            float scale, float k_scale, float v_scale,
-                                           int32_t partition_tokens, uint32_t flags,
-                                           int32_t* device_error, void* stream) {
+                                           int32_t sliding_window, int32_t partition_tokens,
+                                           uint32_t flags, int32_t* device_error, void* stream) {
     set_last_error("");
     const float scales[2] = {k_scale, v_scale};
     return decode_common(q, k_cache, v_cache, block_tables, context_lens, out, workspace,
                          workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
                          num_blocks, block_size, max_blocks_per_seq, PKV_DTYPE_E4M3, out_dtype,
-                         scale, partition_tokens, flags, device_error, stream, nullptr, scales);
+                         scale, partition_tokens, flags, device_error, stream, nullptr, scales,
+                         sliding_window);
+}
+
+pkv_status pkv_paged_attention_decode_window(const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* block_tables,
+                                             const int32_t* context_lens, void* out,
+                                             void* workspace, size_t workspace_bytes,
+                                             int64_t num_seqs, int64_t num_q_heads,
+                                             int64_t num_kv_heads, int64_t head_dim,
+                                             int64_t num_blocks, int64_t block_size,
+                                             int64_t max_blocks_per_seq, int32_t kv_dtype,
+                                             int32_t out_dtype, float scale,
+                                             int32_t sliding_window, int32_t partition_tokens,
+                                             uint32_t flags, int32_t* device_error,
+                                             void* stream) {
+    set_last_error("");
+    return decode_common(q, k_cache, v_cache, block_tables, context_lens, out, workspace,
+                         workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                         num_blocks, block_size, max_blocks_per_seq, kv_dtype, out_dtype, scale,
+                         partition_tokens, flags, device_error, stream, nullptr, nullptr,
+                         sliding_window);
 }
 
 pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,

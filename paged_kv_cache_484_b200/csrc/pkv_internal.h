@@ -61,6 +61,7 @@ struct DecodeArgs {
     // (partial slot 0), and that pass's launch, made between the decode
     // kernel and the combine; null = no cascade
     const int32_t* shared_tokens;
+    int32_t window;  // sliding window, 0 = none (not with shared_tokens)
     cudaError_t (*launch_between)(const void* ctx);
     const void* between_ctx;
     // planning only: launch nothing, store the number of kernels the call

@@ -137,7 +137,7 @@ def _decode8(lib, **kw):
     return lib.pkv_paged_attention_decode_e4m3(
         a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"], a["ws"], a["wsb"], a["B"], a["Hq"],
         a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"], a["odt"], a["scale"], a["ks"], a["vs"],
-        a["P"], a["flags"], a["err"], None)
+        a.get("win", 0), a["P"], a["flags"], a["err"], None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -163,10 +163,28 @@ def test_kv_append_e4m3_rejects_bad_arguments(lib, kw, status):
     (dict(d=96), UNSUPPORTED),
     (dict(P=16, MB=4), WORKSPACE),
     (dict(vc=FAKE + 4), INVALID),
+    (dict(win=-1), INVALID),
     (dict(B=0, q=None, out=None), OK),
 ])
 def test_decode_e4m3_rejects_bad_arguments(lib, kw, status):
     assert _decode8(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(win=-3), INVALID),
+    (dict(win=16, kvdt=5), UNSUPPORTED),
+    (dict(win=16, P=16, MB=4), WORKSPACE),
+    (dict(win=16, B=0, q=None, out=None), OK),
+])
+def test_decode_window_rejects_bad_arguments(lib, kw, status):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, out=FAKE, ws=None, wsb=0, B=2, Hq=8, Hkv=2,
+             d=64, NB=4, bs=16, MB=4, kvdt=BF16, odt=BF16, scale=0.125, P=0, flags=0, err=None)
+    a.update(kw)
+    st = lib.pkv_paged_attention_decode_window(
+        a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"], a["ws"], a["wsb"], a["B"], a["Hq"],
+        a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"], a["kvdt"], a["odt"], a["scale"], a["win"],
+        a["P"], a["flags"], a["err"], None)
+    assert st == status
 
 
 def test_e4m3_planning(lib):

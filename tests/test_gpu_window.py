@@ -1,0 +1,141 @@
+"""Sliding-window decode through the C ABI vs the fp64 oracle (GPU only).
+
+Each query attends to the last W tokens of its context.  The cases cover a
+window that starts inside a page, on a page boundary, inside the first
+partition and beyond the context (no effect), W = 1, every partitioning
+mode (one partition, split with the combine kernel, cluster merge), the
+tensor-core and CUDA-core kernels, bf16 / fp32 caches and the 8-bit cache.
+Pages before the window hold NaN, so a page or token read outside the
+window shows up as a non-finite or wrong output.
+Bars: 1e-5 (fp32 inputs), 2e-3 (bf16 inputs), fp32 output.
+"""
+from __future__ import annotations
+
+import math
+
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_484_b200 as pkv
+from tests.parity_util import TOL_BF16, TOL_F32
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+BS = 16
+LENS = [1, 15, 16, 17, 300, 2049, 64, 0, 5, 1000]
+
+
+def _gen(seed):
+    g = torch.Generator()
+    g.manual_seed(seed)
+    return g
+
+
+def _paged(lens, Hkv, d, dtype, seed, window):
+    """Random pool and tables; every token before a sequence's window is NaN
+    (it must not be read), the rest N(0, 1)."""
+    g = _gen(seed)
+    need = [max(1, math.ceil(L / BS)) for L in lens]
+    NB = sum(need) + 3
+    perm = torch.randperm(NB, generator=g)
+    tables = torch.full((len(lens), max(need)), -1, dtype=torch.int32)
+    kc = torch.randn(NB, Hkv, BS, d, generator=g).to(dtype)
+    vc = torch.randn(NB, Hkv, BS, d, generator=g).to(dtype)
+    c = 0
+    for b, L in enumerate(lens):
+        ids = perm[c:c + need[b]]
+        c += need[b]
+        tables[b, :need[b]] = ids.to(torch.int32)
+        t = torch.arange(max(0, L - window) if window else 0)
+        kc[ids[t // BS], :, t % BS] = float("nan")
+        vc[ids[t // BS], :, t % BS] = float("nan")
+    return kc, vc, tables
+
+
+def _oracle_input(x):
+    """The oracle reads only tokens inside the window; give it zeros where the
+    GPU input holds NaN so that a wrong oracle read would not hide."""
+    return torch.nan_to_num(x, nan=0.0)
+
+
+@pytest.mark.parametrize("dtype,d,G,simt", [
+    (torch.bfloat16, 64, 4, False), (torch.bfloat16, 64, 8, False), (torch.bfloat16, 128, 4, False),
+    (torch.bfloat16, 64, 1, False), (torch.bfloat16, 64, 4, True), (torch.float32, 64, 4, False),
+    (torch.float32, 128, 2, False),
+])
+@pytest.mark.parametrize("W,P,cluster", [
+    (1, 0, True), (15, 0, True), (16, 64, False), (17, 16, False), (100, 0, True),
+    (100, 48, True), (1000, 128, False), (5000, 0, True),
+])
+def test_window_matches_oracle(dtype, d, G, simt, W, P, cluster):
+    Hkv = 2
+    kc, vc, tables = _paged(LENS, Hkv, d, dtype, seed=700 + d + G + W, window=W)
+    q = torch.randn(len(LENS), Hkv * G, d, generator=_gen(701 + W)).to(dtype)
+    cl = torch.tensor(LENS, dtype=torch.int32)
+    out = torch.empty(len(LENS), Hkv * G, d, dtype=torch.float32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.paged_attention_decode(q.to(DEV), kc.to(DEV), vc.to(DEV), tables.to(DEV), cl.to(DEV),
+                               d ** -0.5, out, partition_tokens=P, force_simt=simt,
+                               cluster=cluster, device_error=err, sliding_window=W)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    want = oracle.paged_attention_decode(q, _oracle_input(kc), _oracle_input(vc), tables, cl,
+                                         d ** -0.5, nthreads=8, window=W)
+    got = out.double().cpu()
+    assert torch.isfinite(got).all(), "a token outside the window was read"
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    assert (got - want).abs().max().item() <= tol
+
+
+@pytest.mark.parametrize("d,W,P", [(64, 33, 0), (64, 1000, 64), (128, 17, 0), (64, 1, 16)])
+def test_window_e4m3_matches_oracle(d, W, P):
+    Hkv, G = 2, 4
+    g = _gen(710 + d + W)
+    need = [max(1, math.ceil(L / BS)) for L in LENS]
+    NB = sum(need) + 3
+    perm = torch.randperm(NB, generator=g)
+    tables = torch.full((len(LENS), max(need)), -1, dtype=torch.int32)
+    kc = (torch.randn(NB, Hkv, BS, d, generator=g) * 16).to(torch.float8_e4m3fn).view(torch.uint8)
+    vc = (torch.randn(NB, Hkv, d, BS, generator=g) * 16).to(torch.float8_e4m3fn).view(torch.uint8)
+    kc_gpu, vc_gpu = kc.clone(), vc.clone()
+    c = 0
+    for b, L in enumerate(LENS):
+        ids = perm[c:c + need[b]]
+        c += need[b]
+        tables[b, :need[b]] = ids.to(torch.int32)
+        t = torch.arange(max(0, L - W))        # NaN codes before the window
+        kc_gpu[ids[t // BS], :, t % BS] = 0x7F
+        vc_gpu[ids[t // BS], :, :, t % BS] = 0x7F
+    q = torch.randn(len(LENS), Hkv * G, d, generator=g).to(torch.bfloat16)
+    cl = torch.tensor(LENS, dtype=torch.int32)
+    out = torch.empty(len(LENS), Hkv * G, d, dtype=torch.float32, device=DEV)
+    pkv.paged_attention_decode_e4m3(q.to(DEV), kc_gpu.to(DEV), vc_gpu.to(DEV), tables.to(DEV),
+                                    cl.to(DEV), d ** -0.5, 1 / 16, 1 / 16, out,
+                                    partition_tokens=P, sliding_window=W)
+    torch.cuda.synchronize()
+    want = oracle.paged_attention_decode_e4m3(q, kc, vc, tables, cl, d ** -0.5, 1 / 16, 1 / 16,
+                                              nthreads=8, window=W)
+    got = out.double().cpu()
+    assert torch.isfinite(got).all(), "a token outside the window was read"
+    assert (got - want).abs().max().item() <= TOL_BF16
+
+
+def test_window_on_the_ragged_batch():
+    """64 sequences of U[128, 4096] tokens, 32/8 heads, window 1024, at the
+    partition length the library picks: against the oracle."""
+    g = _gen(720)
+    lens = torch.randint(128, 4097, (64,), generator=g).tolist()
+    kc, vc, tables = _paged(lens, 8, 64, torch.bfloat16, seed=721, window=1024)
+    q = torch.randn(64, 32, 64, generator=g).to(torch.bfloat16)
+    cl = torch.tensor(lens, dtype=torch.int32)
+    out = torch.empty(64, 32, 64, dtype=torch.float32, device=DEV)
+    pkv.paged_attention_decode(q.to(DEV), kc.to(DEV), vc.to(DEV), tables.to(DEV), cl.to(DEV),
+                               0.125, out, sliding_window=1024)
+    torch.cuda.synchronize()
+    want = oracle.paged_attention_decode(q, _oracle_input(kc), _oracle_input(vc), tables, cl,
+                                         0.125, nthreads=16, window=1024)
+    got = out.double().cpu()
+    assert torch.isfinite(got).all()
+    assert (got - want).abs().max().item() <= TOL_BF16
