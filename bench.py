@@ -712,8 +712,12 @@ def run_prefill(args):
                                       partition_tokens=P)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
     esz_out = 2 if out_dtype == torch.bfloat16 else 4
-    nbytes = int(lens.to(torch.int64).sum().item()) * w.Hkv * w.d * 2 * 2 + \
-        w.B * C * w.Hq * w.d * (2 + esz_out)
+    # K/V read per sequence: its whole context, or with a sliding window the
+    # tokens from the chunk's first query's window on
+    read = lens.to(torch.int64)
+    if args.window:
+        read = read.clamp(max=C - 1 + args.window)
+    nbytes = int(read.sum().item()) * w.Hkv * w.d * 2 * 2 + w.B * C * w.Hq * w.d * (2 + esz_out)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     ncopies = args.copies or (1 if nbytes >= 2 * l2 else min(1024, math.ceil(2 * l2 / nbytes)))
     # per-layer q and caches copied; the block tables and lengths shared
@@ -728,7 +732,7 @@ def run_prefill(args):
         c = copies[k % ncopies]
         pkv.paged_attention_prefill(c["q"], c["k"], c["v"], c["t"], c["l"], w.scale,
                                     outs[k % ncopies], workspace=ws, partition_tokens=P,
-                                    device_error=err)
+                                    device_error=err, sliding_window=args.window)
 
     for k in range(max(3, args.warmup, ncopies)):
         call(k)
@@ -774,6 +778,7 @@ def run_prefill(args):
         "query_tokens_per_s": round(world * w.B * C / (ms * 1e-3), 1),
         "config": {"workload": W.CONFIG_NAMES[args.config] + f"_prefill_chunk{C}",
                    "batch_seqs": w.B, "chunk_tokens": C, "q_heads": w.Hq, "kv_heads": w.Hkv,
+                   **({"sliding_window": args.window} if args.window else {}),
                    "head_dim": w.d, "partition_tokens": P,
                    "l2": f"inputs larger than L2: {ncopies} copies, no flush in the timed region"},
         "roofline": {"bound": "hbm", "kernel": "paged_prefill_kernel" +

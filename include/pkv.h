@@ -512,6 +512,9 @@ size_t pkv_decode_cascade_workspace_size(int64_t num_seqs, int64_t num_q_heads,
  *   out[b, i, h, :] = sum_{t <= L-C+i} exp(s_t - max s) V_b[t] / sum_t exp(s_t - max s),
  *   s_t = scale * <q[b, i, h, :], K_b[t]>,
  * i.e. pkv_paged_attention_decode of query i with context length L - C + i + 1.
+ * With sliding_window = W > 0 the sum runs over L-C+i-W < t <= L-C+i only
+ * (query i's last W tokens, as in pkv_paged_attention_decode_window); pages
+ * before the chunk's first window are not read.
  * fp32 arithmetic (bf16 inputs widen exactly), P applied as a two-term bf16
  * split on the tensor cores, the result rounded once to out_dtype.
  *
@@ -525,6 +528,7 @@ size_t pkv_decode_cascade_workspace_size(int64_t num_seqs, int64_t num_q_heads,
  *   out           device, [num_seqs, C, Hq, head_dim], f32 or bf16
  *   workspace     device, >= pkv_prefill_workspace_size(...) bytes (NULL when
  *                 that is 0); contents need no initialisation
+ *   sliding_window  0 (whole causal prefix) or W > 0 (the last W tokens)
  *   partition_tokens  0 = library choice (pkv_prefill_partition_tokens), else a
  *                 multiple of block_size in [block_size, PKV_MAX_PARTITION_TOKENS]
  * kv_dtype must be PKV_DTYPE_BF16.  num_seqs == 0 returns PKV_OK and launches
@@ -537,8 +541,9 @@ pkv_status pkv_paged_attention_prefill(const void* q, const void* k_cache, const
                                        int64_t num_q_heads, int64_t num_kv_heads,
                                        int64_t head_dim, int64_t num_blocks, int64_t block_size,
                                        int64_t max_blocks_per_seq, int32_t kv_dtype,
-                                       int32_t out_dtype, float scale, int32_t partition_tokens,
-                                       int32_t* device_error, void* stream);
+                                       int32_t out_dtype, float scale, int32_t sliding_window,
+                                       int32_t partition_tokens, int32_t* device_error,
+                                       void* stream);
 
 /* Bytes of workspace pkv_paged_attention_prefill needs (partition partials:
  * num_seqs * C * Hq * NP * (head_dim + 2) floats when NP > 1, else 0).  Host

@@ -228,7 +228,7 @@ class Oracle:
         return out
 
     def paged_chunked_prefill(self, q, k_cache, v_cache, block_tables, context_lens, scale,
-                              nthreads: int = 1) -> torch.Tensor:
+                              nthreads: int = 1, window: int = 0) -> torch.Tensor:
         """fp64 [B, C, Hq, d] output of a prefill chunk: the last C context
         tokens of each sequence, query i attending to tokens 0 .. L - C + i.
 
@@ -236,7 +236,8 @@ class Oracle:
         Windows -- a chunk computed over the retained K/V equals the
         full-prefix pass, so query i of the chunk is exactly one decode step
         over the first L - C + i + 1 tokens.  That is how it is computed here:
-        one plain decode per chunk position, with that context length.
+        one plain decode per chunk position, with that context length (and
+        the same sliding ``window``, when > 0).
         """
         _cpu(q)
         _cpu(context_lens, torch.int32)
@@ -246,7 +247,7 @@ class Oracle:
             lens_i = (context_lens.to(torch.int64) - C + i + 1).clamp(min=0).to(torch.int32)
             out[:, i] = self.paged_attention_decode(q[:, i].contiguous(), k_cache, v_cache,
                                                     block_tables, lens_i, scale,
-                                                    nthreads=nthreads)
+                                                    nthreads=nthreads, window=window)
         return out
 
     def contiguous_decode(self, q, K, V, scale) -> torch.Tensor:

@@ -78,7 +78,7 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_paged_attention_decode_noalloc.restype = ctypes.c_int
         lib.pkv_paged_attention_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                                                      i64, i64, i64, i64, i64, i64, i64, i64,
-                                                     i32, i32, ctypes.c_float, i32, vp, vp]
+                                                     i32, i32, ctypes.c_float, i32, i32, vp, vp]
         lib.pkv_paged_attention_prefill.restype = ctypes.c_int
         lib.pkv_prefill_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i64, i32]
         lib.pkv_prefill_workspace_size.restype = ctypes.c_size_t
@@ -452,9 +452,10 @@ def prefill_partition_tokens(num_seqs, chunk_tokens, num_q_heads, num_kv_heads, 
 
 def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, scale, out,
                             stream=None, *, workspace=None, partition_tokens=0,
-                            device_error=None) -> torch.Tensor:
+                            device_error=None, sliding_window=0) -> torch.Tensor:
     """Chunked prefill: the last C tokens of every sequence attend causally to
-    its paged context (their K/V already appended).  q [B, C, Hq, d] bf16,
+    its paged context (their K/V already appended), each to its last
+    ``sliding_window`` tokens when that is > 0.  q [B, C, Hq, d] bf16,
     caches [NB, Hkv, 16, d] bf16, out [B, C, Hq, d] float32 or bfloat16;
     writes and returns ``out``.  See include/pkv.h, pkv_paged_attention_prefill.
     """
@@ -478,7 +479,7 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, sca
         _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         B, C, Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16, _dtype_code(out.dtype), float(scale),
-        int(partition_tokens), err, _stream_ptr(stream, q.device))
+        int(sliding_window), int(partition_tokens), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_prefill")
     return out
 

@@ -70,6 +70,7 @@ struct PrefillParams {
     int B, C, Hq, Hkv, MB, P, NP, RG, num_blocks;
     float scale_log2;
     int out_bf16;
+    int window;                 // sliding window: query at position t sees t - window + 1 .. t
 };
 
 // Byte offset of 16-byte chunk c of token row tok in a 128-byte-swizzled page.
@@ -92,6 +93,7 @@ __device__ __forceinline__ void pstore(void* out, size_t idx, float v, int out_b
 // The item's sequence and key range, from blockIdx.x.
 struct PItem {
     int b, h, rg, part, L, np, t0, t1, npages;
+    int lo;  // sliding window: first token any query of the chunk attends (0 otherwise)
 };
 
 __device__ __forceinline__ PItem prefill_item(const PrefillParams& p) {
@@ -113,8 +115,12 @@ __device__ __forceinline__ PItem prefill_item(const PrefillParams& p) {
     }
     it.L = L;
     it.np = (L + p.P - 1) / p.P;
-    it.t0 = it.part * p.P;
-    it.t1 = min(L, it.t0 + p.P);
+    // sliding window: pages before the chunk's first query's window are not
+    // read (a partition wholly before it has no pages and leaves an empty
+    // partial)
+    it.lo = (p.window > 0 && L - p.C + 1 > p.window) ? L - p.C + 1 - p.window : 0;
+    it.t0 = max(it.part * p.P, it.lo / kPageRows * kPageRows);
+    it.t1 = min(L, it.part * p.P + p.P);
     it.npages = it.t1 > it.t0 ? (it.t1 - it.t0 + kPageRows - 1) / kPageRows : 0;
     return it;
 }
@@ -195,6 +201,7 @@ struct PRow {
     bool ok;            // the row exists
     const bf16* q;      // its query vector (D elements)
     int len;            // it may attend to tokens t < len
+    int lo;             // and t >= lo (sliding window; 0 otherwise)
     bool direct;        // write the output row (else a partition partial)
     void* out;          // direct: the output row (D elements of out_bf16 ? bf16 : f32)
     float* po;          // partial: o (D floats)
@@ -214,6 +221,7 @@ __device__ void multirow_consumer(float scale_log2, int out_bf16, int32_t* err, 
     const int cq = lane & 3;
     const bool row_ok = row.ok;
     const int row_len = row_ok ? row.len : 0;
+    const int row_lo = row.lo;
 
     // A fragments of Q: rows r and r + 8 both hold this lane's row
     uint32_t qa[KS][2];
@@ -246,6 +254,7 @@ __device__ void multirow_consumer(float scale_log2, int out_bf16, int32_t* err, 
             const int tbase = it.t0 + j * kPageRows;       // absolute token of page row 0
             const int in_part = min(kPageRows, it.t1 - tbase);   // rows inside the partition
             const int row_valid = max(0, min(in_part, row_len - tbase));
+            const int row_first = max(0, row_lo - tbase);   // sliding window
             const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + u * L::PAGE_BYTES);
             const uint32_t vbase = kbase + L::SP * L::PAGE_BYTES;
             float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -265,7 +274,8 @@ __device__ void multirow_consumer(float scale_log2, int out_bf16, int32_t* err, 
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int tk = n * 8 + 2 * cq + e;
-                    x[n][e] = tk < row_valid ? sc[n][e] * scale_log2 : kNegInfP;
+                    x[n][e] = (tk < row_valid && tk >= row_first) ? sc[n][e] * scale_log2
+                                                                  : kNegInfP;
                 }
             float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -300,13 +310,15 @@ __device__ void multirow_consumer(float scale_log2, int out_bf16, int32_t* err, 
                 pa[2] = hi1;
                 pa[3] = pack_bf16(pr[1][0] - bf16lo(hi1), pr[1][1] - bf16hi(hi1));
             }
-            // V rows past the partition may hold stale shared memory: zero them
+            // V rows past the partition may hold stale shared memory, and rows
+            // before every query's window are not attended: zero them
             uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
-            if (in_part < kPageRows) {
+            const int v_first = max(0, it.lo - tbase);
+            if (in_part < kPageRows || v_first > 0) {
                 const int k0 = 2 * cq;
-                vmask_lo = (k0 < in_part ? 0x0000ffffu : 0u) | (k0 + 1 < in_part ? 0xffff0000u : 0u);
-                vmask_hi = (k0 + 8 < in_part ? 0x0000ffffu : 0u) |
-                           (k0 + 9 < in_part ? 0xffff0000u : 0u);
+                auto in = [&](int k) { return k >= v_first && k < in_part; };
+                vmask_lo = (in(k0) ? 0x0000ffffu : 0u) | (in(k0 + 1) ? 0xffff0000u : 0u);
+                vmask_hi = (in(k0 + 8) ? 0x0000ffffu : 0u) | (in(k0 + 9) ? 0xffff0000u : 0u);
             }
 #pragma unroll
             for (int c = 0; c < NT; c += 2) {
@@ -401,6 +413,7 @@ __global__ void __launch_bounds__(kThreadsP)
     const size_t r = ((size_t)it.b * p.C + qi) * p.Hq + hq;
     row.q = p.q + r * D;
     row.len = it.L - p.C + qi + 1;
+    row.lo = (p.window > 0 && row.len > p.window) ? row.len - p.window : 0;
     row.direct = it.np == 1;
     row.out = p.out_bf16 ? (void*)(reinterpret_cast<bf16*>(p.out) + r * D)
                          : (void*)(reinterpret_cast<float*>(p.out) + r * D);
@@ -556,6 +569,7 @@ __global__ void __launch_bounds__(kThreadsP)
         it.t0 = 0;
         it.t1 = S;
         it.npages = S / kPageRows;
+        it.lo = 0;
         PrefillParams pp;  // the fields the page producer reads
         pp.block_tables = p.block_tables;
         pp.err = p.err;
@@ -571,6 +585,7 @@ __global__ void __launch_bounds__(kThreadsP)
             const int b = gs + m;
             row.ok = m < nmem;
             row.len = row.ok ? cascade_shared(p, b) : 0;
+            row.lo = 0;
             row.ok = row.ok && row.len > 0;  // no shared tokens: no slot 0
             const size_t r = (size_t)(row.ok ? b : 0) * p.Hq + hq;
             row.q = p.q + r * D;
@@ -631,6 +646,7 @@ cudaError_t launch_prefill_typed(const PrefillArgs& a, const CUtensorMap& tmk,
     p.num_blocks = (int)a.num_blocks;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out_bf16 = a.out_dtype == PKV_DTYPE_BF16;
+    p.window = a.window;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.B * a.Hkv * p.RG * a.max_partitions));

@@ -884,9 +884,14 @@ pkv_status pkv_paged_attention_prefill(const void* q, const void* k_cache, const
                                        int64_t num_q_heads, int64_t num_kv_heads,
                                        int64_t head_dim, int64_t num_blocks, int64_t block_size,
                                        int64_t max_blocks_per_seq, int32_t kv_dtype,
-                                       int32_t out_dtype, float scale, int32_t partition_tokens,
-                                       int32_t* device_error, void* stream) {
+                                       int32_t out_dtype, float scale, int32_t sliding_window,
+                                       int32_t partition_tokens, int32_t* device_error,
+                                       void* stream) {
     set_last_error("");
+    if (sliding_window < 0) {
+        set_last_error("sliding_window must be >= 0");
+        return PKV_ERR_INVALID_ARG;
+    }
     if (num_seqs < 0 || max_blocks_per_seq < 0 || chunk_tokens < 1) {
         set_last_error("negative num_seqs or max_blocks_per_seq, or chunk_tokens < 1");
         return PKV_ERR_INVALID_ARG;
@@ -969,6 +974,7 @@ pkv_status pkv_paged_attention_prefill(const void* q, const void* k_cache, const
     a.partition_tokens = P;
     a.max_partitions = NP;
     a.scale = scale;
+    a.window = sliding_window;
     a.device_error = device_error;
     a.stream = static_cast<cudaStream_t>(stream);
     return cuda_status(launch_paged_prefill(a), "prefill launch");

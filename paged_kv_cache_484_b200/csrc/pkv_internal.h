@@ -98,6 +98,7 @@ struct PrefillArgs {
     int32_t partition_tokens;   // P (resolved)
     int32_t max_partitions;     // NP = ceil(MB * 16 / P)
     float scale;
+    int32_t window;             // sliding window, 0 = none
     int32_t* device_error;
     cudaStream_t stream;
 };

@@ -243,10 +243,12 @@ def _prefill(lib, **kw):
     return lib.pkv_paged_attention_prefill(a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"],
                                            a["ws"], a["wsb"], a["B"], a["C"], a["Hq"], a["Hkv"],
                                            a["d"], a["NB"], a["bs"], a["MB"], a["kvdt"],
-                                           a["odt"], a["scale"], a["P"], a["err"], None)
+                                           a["odt"], a["scale"], a.get("win", 0), a["P"],
+                                           a["err"], None)
 
 
 @pytest.mark.parametrize("kw,status", [
+    (dict(win=-1), INVALID),
     (dict(kvdt=F32), UNSUPPORTED),          # bf16 only
     (dict(C=0), INVALID),
     (dict(C=65), INVALID),                  # longer than max_blocks * 16

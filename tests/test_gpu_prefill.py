@@ -166,3 +166,33 @@ def test_prompt_chunks_then_decode_steps():
         want = oracle.paged_attention_decode(q_o, kc_o, vc_o, tables, lens, scale)
         _check(out, want, f"decode step {s}")
         done += 1
+
+
+@pytest.mark.parametrize("d,G,C,W,P", [
+    (64, 4, 16, 1, 0), (64, 4, 16, 7, 64), (64, 4, 16, 40, 0), (64, 8, 7, 100, 64),
+    (128, 4, 16, 33, 0), (64, 1, 1, 17, 16), (64, 4, 16, 5000, 0), (64, 4, 24, 16, 128),
+])
+def test_prefill_sliding_window(d, G, C, W, P):
+    """Query i of the chunk attends to its last W tokens only.  Keys and
+    values before the chunk's first window are NaN: reading one of them, or
+    not masking it per row, shows up as a non-finite or wrong output."""
+    lens = [300, 16, 1000, 47, 2049][: 3 if d == 128 else 5]
+    lens = [max(L, C) for L in lens]
+    w, q, lens_t = _case(lens, G, 2, d, C, seed=330 + d + G + C + W)
+    want = oracle.paged_chunked_prefill(q.cpu(), w.k_cache.cpu(), w.v_cache.cpu(),
+                                        w.block_tables.cpu(), lens_t.cpu(), w.scale, nthreads=8,
+                                        window=W)
+    tables = w.block_tables.cpu()
+    for b, L in enumerate(lens_t.tolist()):
+        t = torch.arange(max(0, L - C + 1 - W))   # no query of the chunk attends these
+        blk = tables[b, t // 16].to(torch.int64).to(DEV)
+        row = (t % 16).to(DEV)
+        w.k_cache[blk, :, row] = float("nan")
+        w.v_cache[blk, :, row] = float("nan")
+    out = torch.empty((w.B, C, w.Hq, d), dtype=torch.float32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.paged_attention_prefill(q, w.k_cache, w.v_cache, w.block_tables, lens_t, w.scale, out,
+                                partition_tokens=P, device_error=err, sliding_window=W)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    _check(out, want, f"window {W} d{d} G{G} C{C} P{P}")

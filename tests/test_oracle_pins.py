@@ -677,6 +677,30 @@ def pin_sliding_window_decode(orc: Oracle):
                     _e4m3_value(Vs[b][s0:]) * 0.07, 0.25)[0]
         assert_close(got[b], want, 1e-12, f"e4m3 window b={b}")
 
+
+def pin_sliding_window_chunked_prefill(orc: Oracle):
+    """A windowed prefill chunk equals PyTorch's fp64 SDPA over the gathered
+    context with a banded causal mask: query row r attends to keys
+    r - W + 1 .. r."""
+    for (Hq, Hkv, d, lens, C, W, seed) in [(8, 2, 16, [40, 17, 5], 5, 7, 84),
+                                           (4, 4, 8, [33], 33, 16, 85)]:
+        kpool, vpool, tables, Ks, Vs = random_paged(lens, Hkv, d, 16, torch.float32, seed)
+        q = torch.randn(len(lens), C, Hq, d, generator=_gen(seed + 100))
+        got = orc.paged_chunked_prefill(q, kpool, vpool, tables,
+                                        torch.tensor(lens, dtype=torch.int32), 0.25, window=W)
+        for b, L in enumerate(lens):
+            G = Hq // Hkv
+            Kr = Ks[b].double().repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+            Vr = Vs[b].double().repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+            Q = torch.zeros(L, Hq, d, dtype=torch.float64)
+            Q[L - C:] = q[b].double()
+            r = torch.arange(L)[:, None]
+            t = torch.arange(L)[None, :]
+            band = (t <= r) & (t > r - W)
+            want = F.scaled_dot_product_attention(Q.permute(1, 0, 2)[None], Kr, Vr,
+                                                  attn_mask=band, scale=0.25)[0].permute(1, 0, 2)
+            assert_close(got[b], want[L - C:], 1e-12, f"windowed chunk b={b}")
+
 PINS = [
     pin_round_bf16_matches_torch_cast,
     pin_round_bf16_single_rounding,
@@ -702,6 +726,7 @@ PINS = [
     pin_e4m3_decode_matches_sdpa_over_dequantized,
     pin_append_e4m3_placement_and_values,
     pin_sliding_window_decode,
+    pin_sliding_window_chunked_prefill,
 ]
 
 
