@@ -543,10 +543,13 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             if (mine) {
                 const int row0 = (cur_ent * p.Hkv + cur.h) * kPageRows;
                 if constexpr (L::F8) {
-                    // K: a [16][D] byte box; V (transposed): a [D][16] byte box
-                    tma_load_2d(kdst + k * L::PAGE_BYTES, tmk, 0, row0, &full[stage]);
-                    tma_load_2d(vdst + k * L::PAGE_BYTES, tmv, 0, (cur_ent * p.Hkv + cur.h) * D,
+                    // one box per page: K as 4 rows of 256 bytes (d = 64) or 16
+                    // swizzled rows of 128 bytes (d = 128); V (transposed) as
+                    // D / 16 rows of 256 bytes
+                    const int page = cur_ent * p.Hkv + cur.h;
+                    tma_load_2d(kdst + k * L::PAGE_BYTES, tmk, 0, page * (D == 64 ? 4 : kPageRows),
                                 &full[stage]);
+                    tma_load_2d(vdst + k * L::PAGE_BYTES, tmv, 0, page * (D / 16), &full[stage]);
                 } else {
 #pragma unroll
                     for (int bx = 0; bx < L::BOXES; ++bx) {

@@ -79,10 +79,16 @@ cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_bl
     const bool bf = dtype == PKV_DTYPE_BF16;
     const bool f8 = dtype == PKV_DTYPE_E4M3;
     const int esz = f8 ? 1 : (bf ? 2 : 4);
-    const cuuint64_t rows = (cuuint64_t)(num_blocks * Hkv * kPageRows);
-    cuuint64_t dims[2] = {(cuuint64_t)D, rows};
-    cuuint64_t strides[1] = {(cuuint64_t)(D * esz)};
-    cuuint32_t box[2] = {(cuuint32_t)(bf ? 64 : D), (cuuint32_t)kPageRows};
+    // 8-bit d = 64 pages (16 rows of 64 bytes, 1 KiB contiguous) are described
+    // as 4 rows of 256 bytes: the same bytes in the same order in shared
+    // memory, in a quarter of the row requests
+    const bool wide = f8 && D == 64;
+    const int row_bytes = wide ? 256 : (int)(D * esz);
+    const int rows_per_page = wide ? 4 : kPageRows;
+    const cuuint64_t rows = (cuuint64_t)(num_blocks * Hkv * rows_per_page);
+    cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / esz), rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)(bf ? 64 : row_bytes / esz), (cuuint32_t)rows_per_page};
     cuuint32_t estr[2] = {1, 1};
     // bf16 boxes are 128-byte rows, swizzled; 8-bit rows of 128 bytes too
     const bool swz = bf || (f8 && D == 128);
@@ -96,15 +102,18 @@ cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_bl
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// The 8-bit cache's transposed V pages [num_blocks, Hkv, D, 16] (bytes): rows
-// of 16 tokens, one [D][16] box per page.
+// The 8-bit cache's transposed V pages [num_blocks, Hkv, D, 16] (bytes).  A
+// page is 16 D contiguous bytes; it is described as D / 16 rows of 256 bytes
+// (one box per page) rather than D rows of 16 bytes, which would cost a row
+// request per 16 bytes.  Shared memory receives the same bytes in the same
+// order.
 cudaError_t encode_vt_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
                                 int64_t Hkv, int64_t D) {
     auto fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
-    cuuint64_t dims[2] = {(cuuint64_t)kPageRows, (cuuint64_t)(num_blocks * Hkv * D)};
-    cuuint64_t strides[1] = {(cuuint64_t)kPageRows};
-    cuuint32_t box[2] = {(cuuint32_t)kPageRows, (cuuint32_t)D};
+    cuuint64_t dims[2] = {256, (cuuint64_t)(num_blocks * Hkv * D / 16)};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {256, (cuuint32_t)(D / 16)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(cache), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
