@@ -157,6 +157,20 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def software_versions() -> dict:
+    """Versions the numbers were taken with (NVML read only)."""
+    v = {"torch": torch.__version__, "cuda_runtime": torch.version.cuda,
+         "kernel_sources": kernel_source_hash()}
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        d = pynvml.nvmlSystemGetDriverVersion()
+        v["driver"] = d.decode() if isinstance(d, bytes) else d
+    except Exception:
+        pass
+    return v
+
+
 def recorded_traffic(cfg):
     """DRAM bytes per decode launch from the committed ncu capture, if it was
     taken on the current kernel sources (else None).  ``cfg``: the config
@@ -624,8 +638,12 @@ def run_ours(args):
             wc.k_cache, wc.v_cache = k8c, v8c
         per_step, seqs, frac, reps = time_oracle(wc, args.cpu_seconds, nthreads,
                                                  (ks8, vs8) if e4m3 else None, args.window)
+        # the same oracle on one thread, briefly (reported beside the all-cores figure)
+        per1, seqs1, frac1, reps1 = time_oracle(wc, min(2.0, args.cpu_seconds), 1,
+                                                (ks8, vs8) if e4m3 else None, args.window)
         cpu = {"value": round(nbytes * frac / per_step / 1e9, 4), "unit": "GB/s",
                "cores": nthreads, "kind": "oracle",
+               "value_1_thread": round(nbytes * frac1 / per1 / 1e9, 4),
                "sample": f"{len(seqs)} of {w.B} sequences, full append+decode step in fp64, "
                          f"{reps} repetitions ({per_step * 1e3:.1f} ms each)"}
 
@@ -672,6 +690,7 @@ def run_ours(args):
         "e2e": e2e,
         "cpu_baseline": cpu,
         "device": torch.cuda.get_device_name(device),
+        "versions": software_versions(),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
