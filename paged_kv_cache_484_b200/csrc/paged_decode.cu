@@ -112,7 +112,10 @@ struct Layout {
     static constexpr int MERGE_ROW_BYTES = (D + 2) * 4;
     static constexpr int MERGE_ROWS_PER_SLOT = PPW * PAGE_BYTES / MERGE_ROW_BYTES;
     static constexpr bool MERGE_IN_SLOTS = 2 * MERGE_ROWS_PER_SLOT >= G;
-    static constexpr int MERGE_BYTES = MERGE_IN_SLOTS ? 0 : NW * G * MERGE_ROW_BYTES;
+    // With a region of its own the item's last stage goes back to the
+    // producer before the merge, and the warps meet once more after it.
+    static constexpr bool MERGE_SEPARATE = !MERGE_IN_SLOTS;
+    static constexpr int MERGE_BYTES = MERGE_SEPARATE ? NW * G * MERGE_ROW_BYTES : 0;
     // byte offsets from the 1024-aligned base
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
     static constexpr int OFF_NEWKV = OFF_Q + STAGES * Q_BYTES;
@@ -648,7 +651,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
 template <typename T, int D, int G>
 __device__ __forceinline__ float* merge_row(uint8_t* base, int st, int w, int g) {
     using L = Layout<T, D, G>;
-    if constexpr (!L::MERGE_IN_SLOTS)
+    if constexpr (L::MERGE_SEPARATE)
         return reinterpret_cast<float*>(base + L::OFF_MERGE + (w * G + g) * L::MERGE_ROW_BYTES);
     uint8_t* kslot = base + st * L::STAGE_BYTES + w * L::PPW * L::PAGE_BYTES;
     uint8_t* row = g < L::MERGE_ROWS_PER_SLOT
@@ -1078,7 +1081,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
             __syncwarp();
             // the item's last stage stays held: its page slots take the merge
             last = stage;
-            if (s + 1 < nst && lane == 0) mbar_arrive(&empty[stage]);
+            if ((s + 1 < nst || L::MERGE_SEPARATE) && lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == L::STAGES) {
                 stage = 0;
                 phase ^= 1;
@@ -1131,7 +1134,13 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
         merge_and_store<T, D, G>(p, it, base, last);
         ++merged;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[last]);
+        if constexpr (L::MERGE_SEPARATE) {
+            // one merge region for all items: nobody writes the next item's
+            // rows before every warp has read this item's
+            if (!consumer_sync(p, merge_bar, mphase, s_abort)) return -1;
+        } else {
+            if (lane == 0) mbar_arrive(&empty[last]);
+        }
     }
 }
 
@@ -1265,7 +1274,7 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
             __syncwarp();
             // the item's last stage stays held: its page slots take the merge
             last = stage;
-            if (s + 1 < nst && lane == 0) mbar_arrive(&empty[stage]);
+            if ((s + 1 < nst || L::MERGE_SEPARATE) && lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == L::STAGES) {
                 stage = 0;
                 phase ^= 1;
@@ -1321,7 +1330,13 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
         merge_and_store<T, D, G>(p, it, base, last);
         ++merged;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[last]);
+        if constexpr (L::MERGE_SEPARATE) {
+            // one merge region for all items: nobody writes the next item's
+            // rows before every warp has read this item's
+            if (!consumer_sync(p, merge_bar, mphase, s_abort)) return -1;
+        } else {
+            if (lane == 0) mbar_arrive(&empty[last]);
+        }
     }
 }
 
