@@ -126,6 +126,7 @@ def test_kv_append_e4m3_slot_out_of_range():
     (64, 4, 0, True), (64, 4, 64, True), (64, 4, 64, False), (64, 4, 16, False),
     (64, 1, 0, True), (64, 2, 128, False), (64, 8, 0, True), (64, 8, 48, False),
     (128, 4, 0, True), (128, 4, 256, False), (128, 8, 0, True), (128, 1, 64, True),
+    (128, 8, 16, False),  # merge rows in a region of their own, many one-page items
 ])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_decode_e4m3_matches_oracle(d, G, P, cluster, out_dtype):
