@@ -11,6 +11,14 @@
  *                               for every sequence and query head, reading K/V
  *                               through the sequence's block table.
  *
+ * Around them: the two in one launch (pkv_decode_step); a sliding window
+ * (pkv_paged_attention_decode_window); shared-prefix groups read once
+ * (pkv_paged_attention_decode_cascade); chunked prefill
+ * (pkv_paged_attention_prefill); an 8-bit E4M3 cache (pkv_kv_append_e4m3,
+ * pkv_paged_attention_decode_e4m3); a decode without a caller workspace
+ * (pkv_paged_attention_decode_noalloc); and a host-side block manager with
+ * prefix reuse (pkv_bm_*).
+ *
  * Sources (page title, section):
  *   "Inference From Scratch" (book intro), "What you will build" and the
  *     chapter table: ch. 4 KV cache, ch. 8 online softmax / flash attention,
@@ -24,7 +32,11 @@
  *     with RoPE and causal attention; M1 KV cache, prefill/decode
  *     equivalence);
  *   "warpllama", Milestones (static KV cache + single-token decode; fused
- *     RoPE kernel; fused attention hot path in CUDA).
+ *     RoPE kernel; fused attention hot path in CUDA);
+ *   "Efficient LLM Inference", learning route: KV Caching (reuse, positions
+ *     and windows; chunked equals full prefix), KV memory accounting,
+ *     Quantization, and verifying exact execution and approximate quality
+ *     separately.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
