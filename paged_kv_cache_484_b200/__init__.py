@@ -28,6 +28,8 @@ from ._binding import (  # noqa: F401
     decode_launches,
     decode_partition_tokens,
     decode_step,
+    prepare_decode_step,
+    PreparedCall,
     decode_workspace_size,
     kv_append,
     kv_append_e4m3,

@@ -394,6 +394,63 @@ def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, bloc
     return out
 
 
+class PreparedCall:
+    """A library call whose arguments were checked and marshalled once.
+    Calling it launches the same work again on the same stream; the tensors
+    it was prepared with must stay alive and keep their shapes, dtypes and
+    addresses (their contents may change between calls)."""
+
+    __slots__ = ("_lib", "_fn", "_args", "_name", "_keep")
+
+    def __init__(self, lib, fn, args, name, keep):
+        self._lib, self._fn, self._name, self._keep = lib, fn, name, keep
+        types = fn.argtypes
+        # ctypes instances, so that a call converts nothing
+        self._args = tuple(t(a) if a is not None or t is not ctypes.c_void_p else t()
+                           for t, a in zip(types, args))
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st != 0:
+            _raise(st, self._lib, self._name)
+
+
+def prepare_decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
+                        context_lens, rope_theta, scale, out, stream=None, *, workspace,
+                        partition_tokens=0, force_simt=False, device_error=None,
+                        cluster=True) -> PreparedCall:
+    """``decode_step`` checked and marshalled once, for a caller that repeats
+    the same step on the same buffers (a model's layer loop: one prepared call
+    per layer).  ``workspace`` is required; see ``decode_step``."""
+    lib = load_library()
+    kv_dt = _dtype_code(k_cache.dtype)
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("v_cache", v_cache)):
+        if t.dtype != k_cache.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from the cache dtype {k_cache.dtype}")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, Hq, d) \
+            or k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d) \
+            or positions.shape != (B,) or slot_mapping.shape != (B,) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("inconsistent decode_step shapes")
+    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    args = (_dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+            _dev(positions, "positions", torch.int64),
+            _dev(slot_mapping, "slot_mapping", torch.int64),
+            _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+            _dev(block_tables, "block_tables", torch.int32),
+            _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(rope_theta),
+            float(scale), int(partition_tokens), _flags(force_simt, cluster), err,
+            _stream_ptr(stream, q.device))
+    keep = (q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
+            context_lens, out, workspace, device_error)
+    return PreparedCall(lib, lib.pkv_decode_step, args, "decode_step", keep)
+
+
 def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, out,
                                    stream=None, *, partition_tokens=0, force_simt=False,
                                    device_error=None, cluster=True) -> torch.Tensor:

@@ -151,3 +151,16 @@ def test_random_operations_keep_the_invariants():
                 else:
                     where[blk] = (sid, j)
         assert len(where) + bm.free_blocks == NB
+
+
+def test_prepared_call_marshals_once_and_reports_errors():
+    """PreparedCall (the binding's checked-once call) on a host entry point:
+    the first call succeeds, the repeat reports the library's status."""
+    lib = pkv.load_library()
+    bm = pkv.BlockManager(4, BS)
+    bm.add_sequence(9, [1, 2, 3])
+    call = pkv.PreparedCall(lib, lib.pkv_bm_free_sequence, (bm._h, 9), "pkv_bm_free_sequence", bm)
+    call()
+    assert bm.free_blocks == 4
+    with pytest.raises(pkv.PkvError):
+        call()

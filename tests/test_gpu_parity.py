@@ -393,3 +393,36 @@ def test_batch1_auto_partition_uses_clusters():
     torch.cuda.synchronize()
     _, _, _, ref = sub.oracle_step()
     check_decode(out, ref, w.dtype, "batch-1 cluster step")
+
+
+def test_prepared_decode_step_matches_decode_step():
+    """prepare_decode_step marshals once; each call relaunches the step on the
+    buffers' current contents: bit-identical to decode_step, also after q
+    and the new rows change between calls."""
+    w = W.build_workload("prepared", [300, 17, 2048, 64], 32, 8, 64, torch.bfloat16, 5e5,
+                         seed=61, device=DEV)
+    need = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks)
+    ws = pkv.new_workspace(need, DEV)
+    k0, v0 = w.k_cache.clone(), w.v_cache.clone()
+    q = w.q.clone()
+    out_p = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=DEV)
+    step = pkv.prepare_decode_step(q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache,
+                                   w.v_cache, w.block_tables, w.decode_lens, w.rope_theta,
+                                   w.scale, out_p, workspace=ws)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(62)
+    for rep in range(2):
+        if rep:
+            q.copy_(torch.randn(q.shape, generator=g, device=DEV).to(q.dtype))
+        w.k_cache.copy_(k0)
+        w.v_cache.copy_(v0)
+        step()
+        torch.cuda.synchronize()
+        got = out_p.clone()
+        w.k_cache.copy_(k0)
+        w.v_cache.copy_(v0)
+        out = torch.empty_like(out_p)
+        pkv.decode_step(q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
+                        w.block_tables, w.decode_lens, w.rope_theta, w.scale, out, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(got, out), f"prepared call differs (rep {rep})"
