@@ -275,8 +275,8 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
             or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("inconsistent paged_attention_decode shapes")
     out_dt = _dtype_code(out.dtype)
-    need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
     if workspace is None:
+        need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
         workspace = new_workspace(int(need), q.device)
     err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
     args = [_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
@@ -336,9 +336,9 @@ def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens,
     if d2 != d or v_cache.shape != (NB, Hkv, d, bs) or out.shape != (B, Hq, d) \
             or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("inconsistent paged_attention_decode_e4m3 shapes")
-    need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, PKV_DTYPE_E4M3,
-                                         int(partition_tokens))
     if workspace is None:
+        need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, PKV_DTYPE_E4M3,
+                                             int(partition_tokens))
         workspace = new_workspace(int(need), q.device)
     err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
     st = lib.pkv_paged_attention_decode_e4m3(
@@ -353,16 +353,11 @@ def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens,
     return out
 
 
-def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
-                context_lens, rope_theta, scale, out, stream=None, *, workspace=None,
-                partition_tokens=0, force_simt=False, device_error=None,
-                cluster=True) -> torch.Tensor:
-    """``kv_append`` (one new token per sequence) then ``paged_attention_decode``,
-    in one launch.  The new token must be the last token of its context
-    (context_lens[b] - 1, at the slot block_tables gives it).  q is read only:
-    the rotated q is used inside the kernel and not stored.  See include/pkv.h,
-    pkv_decode_step.
-    """
+def _decode_step_args(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
+                      context_lens, rope_theta, scale, out, stream, workspace, partition_tokens,
+                      force_simt, device_error, cluster):
+    """Checked pkv_decode_step arguments (allocating a workspace if none is
+    given), and the tensors they point into."""
     lib = load_library()
     kv_dt = _dtype_code(k_cache.dtype)
     for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("v_cache", v_cache)):
@@ -376,21 +371,40 @@ def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, bloc
             or positions.shape != (B,) or slot_mapping.shape != (B,) \
             or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("inconsistent decode_step shapes")
-    need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
     if workspace is None:
+        need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
         workspace = new_workspace(int(need), q.device)
     err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
-    st = lib.pkv_decode_step(
-        _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
-        _dev(positions, "positions", torch.int64), _dev(slot_mapping, "slot_mapping", torch.int64),
-        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(rope_theta), float(scale),
-        int(partition_tokens), _flags(force_simt, cluster), err,
-        _stream_ptr(stream, q.device))
-    _raise(st, lib, "decode_step")
+    args = (_dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+            _dev(positions, "positions", torch.int64),
+            _dev(slot_mapping, "slot_mapping", torch.int64),
+            _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+            _dev(block_tables, "block_tables", torch.int32),
+            _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(rope_theta),
+            float(scale), int(partition_tokens), _flags(force_simt, cluster), err,
+            _stream_ptr(stream, q.device))
+    keep = (q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
+            context_lens, out, workspace, device_error)
+    return lib, args, keep
+
+
+def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
+                context_lens, rope_theta, scale, out, stream=None, *, workspace=None,
+                partition_tokens=0, force_simt=False, device_error=None,
+                cluster=True) -> torch.Tensor:
+    """``kv_append`` (one new token per sequence) then ``paged_attention_decode``,
+    in one launch.  The new token must be the last token of its context
+    (context_lens[b] - 1, at the slot block_tables gives it).  q is read only:
+    the rotated q is used inside the kernel and not stored.  See include/pkv.h,
+    pkv_decode_step.
+    """
+    lib, args, _ = _decode_step_args(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache,
+                                     block_tables, context_lens, rope_theta, scale, out, stream,
+                                     workspace, partition_tokens, force_simt, device_error,
+                                     cluster)
+    _raise(lib.pkv_decode_step(*args), lib, "decode_step")
     return out
 
 
@@ -422,32 +436,10 @@ def prepare_decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cac
     """``decode_step`` checked and marshalled once, for a caller that repeats
     the same step on the same buffers (a model's layer loop: one prepared call
     per layer).  ``workspace`` is required; see ``decode_step``."""
-    lib = load_library()
-    kv_dt = _dtype_code(k_cache.dtype)
-    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("v_cache", v_cache)):
-        if t.dtype != k_cache.dtype:
-            raise TypeError(f"{name} dtype {t.dtype} differs from the cache dtype {k_cache.dtype}")
-    B, Hq, d = q.shape
-    NB, Hkv, bs, d2 = k_cache.shape
-    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
-    if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, Hq, d) \
-            or k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d) \
-            or positions.shape != (B,) or slot_mapping.shape != (B,) \
-            or block_tables.shape[0] != B or context_lens.shape != (B,):
-        raise ValueError("inconsistent decode_step shapes")
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
-    args = (_dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
-            _dev(positions, "positions", torch.int64),
-            _dev(slot_mapping, "slot_mapping", torch.int64),
-            _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-            _dev(block_tables, "block_tables", torch.int32),
-            _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
-            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-            B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(rope_theta),
-            float(scale), int(partition_tokens), _flags(force_simt, cluster), err,
-            _stream_ptr(stream, q.device))
-    keep = (q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
-            context_lens, out, workspace, device_error)
+    lib, args, keep = _decode_step_args(q, k_new, v_new, positions, slot_mapping, k_cache,
+                                        v_cache, block_tables, context_lens, rope_theta, scale,
+                                        out, stream, workspace, partition_tokens, force_simt,
+                                        device_error, cluster)
     return PreparedCall(lib, lib.pkv_decode_step, args, "decode_step", keep)
 
 
