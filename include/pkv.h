@@ -628,6 +628,27 @@ int32_t pkv_bm_shared_tokens(const pkv_block_manager* bm, int64_t seq_id);
 int32_t pkv_bm_free_blocks(const pkv_block_manager* bm);
 int32_t pkv_bm_cached_blocks(const pkv_block_manager* bm);
 
+/*
+ * KV memory accounting, before any allocation ("Efficient LLM Inference",
+ * From KV Elements to Memory Accounting and Admission Budgets).  Host only.
+ *
+ * pkv_kv_request_bytes: cache bytes a request of `tokens` tokens occupies
+ * over `num_layers` layers: ceil(tokens / block_size) blocks, each
+ * num_layers * 2 (K and V) * num_kv_heads * block_size * head_dim elements
+ * of kv_dtype (PKV_DTYPE_F32 / _BF16 / _E4M3).  E.g. 16 layers, 8 kv heads,
+ * head_dim 64, bf16: 32 KiB per token, 64 MiB for 2048 tokens.
+ *
+ * pkv_kv_admission_capacity: how many such requests fit in `pool_bytes`
+ * (floor).
+ *
+ * Both return -1 for invalid arguments (or an overflowing size).
+ */
+int64_t pkv_kv_request_bytes(int64_t num_layers, int64_t num_kv_heads, int64_t head_dim,
+                             int64_t block_size, int64_t tokens, int32_t kv_dtype);
+int64_t pkv_kv_admission_capacity(int64_t pool_bytes, int64_t num_layers, int64_t num_kv_heads,
+                                  int64_t head_dim, int64_t block_size, int64_t tokens,
+                                  int32_t kv_dtype);
+
 /* Short text for a status code (static storage). */
 const char* pkv_status_string(int32_t status);
 

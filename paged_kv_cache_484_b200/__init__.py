@@ -31,8 +31,10 @@ from ._binding import (  # noqa: F401
     prepare_decode_step,
     PreparedCall,
     decode_workspace_size,
+    kv_admission_capacity,
     kv_append,
     kv_append_e4m3,
+    kv_request_bytes,
     load_library,
     new_workspace,
     paged_attention_decode,

@@ -102,6 +102,10 @@ def load_library() -> ctypes.CDLL:
             i32, ctypes.c_float, i32, i32, u32, vp, vp]
         lib.pkv_paged_attention_decode_window.restype = ctypes.c_int
         lib.pkv_paged_attention_decode_e4m3.restype = ctypes.c_int
+        lib.pkv_kv_request_bytes.argtypes = [i64, i64, i64, i64, i64, i32]
+        lib.pkv_kv_request_bytes.restype = i64
+        lib.pkv_kv_admission_capacity.argtypes = [i64, i64, i64, i64, i64, i64, i32]
+        lib.pkv_kv_admission_capacity.restype = i64
         lib.pkv_bm_create.argtypes = [i32, i32]
         lib.pkv_bm_create.restype = vp
         lib.pkv_bm_destroy.argtypes = [vp]
@@ -581,6 +585,29 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_le
         _flags(force_simt, True), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode_cascade")
     return out
+
+
+def kv_request_bytes(num_layers, num_kv_heads, head_dim, tokens, kv_dtype=torch.bfloat16,
+                     block_size=BLOCK_SIZE) -> int:
+    """Cache bytes a request of ``tokens`` tokens occupies over ``num_layers``
+    layers (whole blocks); see include/pkv.h, pkv_kv_request_bytes."""
+    lib = load_library()
+    n = int(lib.pkv_kv_request_bytes(num_layers, num_kv_heads, head_dim, block_size, tokens,
+                                     _kv_dtype_code(kv_dtype)))
+    if n < 0:
+        raise ValueError("invalid KV accounting arguments")
+    return n
+
+
+def kv_admission_capacity(pool_bytes, num_layers, num_kv_heads, head_dim, tokens,
+                          kv_dtype=torch.bfloat16, block_size=BLOCK_SIZE) -> int:
+    """How many requests of ``tokens`` tokens fit in ``pool_bytes`` of cache."""
+    lib = load_library()
+    n = int(lib.pkv_kv_admission_capacity(int(pool_bytes), num_layers, num_kv_heads, head_dim,
+                                          block_size, tokens, _kv_dtype_code(kv_dtype)))
+    if n < 0:
+        raise ValueError("invalid KV accounting arguments")
+    return n
 
 
 class BlockManager:

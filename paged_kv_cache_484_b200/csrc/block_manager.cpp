@@ -20,6 +20,7 @@
 //
 // The block manager is plain host C++ with no CUDA; it is not thread safe
 // (one owner, as in an engine's scheduler loop).
+#include <climits>
 #include <stdint.h>
 
 #include <algorithm>
@@ -359,6 +360,34 @@ int32_t pkv_bm_cached_blocks(const pkv_block_manager* handle) {
     auto* bm = reinterpret_cast<const BlockManager*>(handle);
     if (!bm) return -1;
     return (int32_t)bm->cache.size();
+}
+
+// KV memory accounting ("Efficient LLM Inference", From KV Elements to Memory
+// Accounting and Admission Budgets): every cached token holds a key and a
+// value vector per kv head per layer, and the paged cache hands out whole
+// blocks, so a request of L tokens occupies ceil(L / block_size) blocks.
+int64_t pkv_kv_request_bytes(int64_t num_layers, int64_t num_kv_heads, int64_t head_dim,
+                             int64_t block_size, int64_t tokens, int32_t kv_dtype) {
+    const int64_t esz = kv_dtype == PKV_DTYPE_F32 ? 4
+                        : kv_dtype == PKV_DTYPE_BF16 ? 2
+                        : kv_dtype == PKV_DTYPE_E4M3 ? 1 : 0;
+    if (esz == 0 || num_layers <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        tokens < 0)
+        return -1;
+    const int64_t blocks = (tokens + block_size - 1) / block_size;
+    const int64_t per_block = num_layers * 2 * num_kv_heads * block_size * head_dim * esz;
+    if (blocks > 0 && per_block > INT64_MAX / blocks) return -1;
+    return blocks * per_block;
+}
+
+int64_t pkv_kv_admission_capacity(int64_t pool_bytes, int64_t num_layers, int64_t num_kv_heads,
+                                  int64_t head_dim, int64_t block_size, int64_t tokens,
+                                  int32_t kv_dtype) {
+    const int64_t per = pkv_kv_request_bytes(num_layers, num_kv_heads, head_dim, block_size,
+                                             tokens, kv_dtype);
+    if (per < 0 || pool_bytes < 0) return -1;
+    if (per == 0) return INT64_MAX;
+    return pool_bytes / per;
 }
 
 }  // extern "C"

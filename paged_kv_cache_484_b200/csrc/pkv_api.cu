@@ -1002,6 +1002,6 @@ const char* pkv_status_string(int32_t status) {
 
 const char* pkv_last_error(void) { return g_last_error; }
 
-int32_t pkv_version(void) { return 100; }
+int32_t pkv_version(void) { return 200; }
 
 }  // extern "C"

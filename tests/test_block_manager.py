@@ -164,3 +164,23 @@ def test_prepared_call_marshals_once_and_reports_errors():
     assert bm.free_blocks == 4
     with pytest.raises(pkv.PkvError):
         call()
+
+
+def test_kv_memory_accounting():
+    """Bytes per request and admission capacity, against the element count
+    written out by hand: every token holds K and V per kv head per layer, in
+    whole 16-token blocks."""
+    # Llama-3.2-1B attention: 16 layers, 8 kv heads, head_dim 64, bf16
+    per_token = 16 * 2 * 8 * 64 * 2
+    assert per_token == 32 * 1024
+    assert pkv.kv_request_bytes(16, 8, 64, 2048) == 2048 * per_token == 64 << 20
+    assert pkv.kv_request_bytes(16, 8, 64, 2049) == 2064 * per_token   # a 129th block
+    assert pkv.kv_request_bytes(16, 8, 64, 0) == 0
+    assert pkv.kv_request_bytes(16, 8, 64, 100, kv_dtype=torch.uint8) == 112 * per_token // 2
+    assert pkv.kv_request_bytes(32, 8, 128, 1, kv_dtype=torch.float32) == 32 * 2 * 8 * 16 * 128 * 4
+    assert pkv.kv_admission_capacity(80 << 30, 16, 8, 64, 2048) == (80 << 30) // (64 << 20)
+    assert pkv.kv_admission_capacity((64 << 20) - 1, 16, 8, 64, 2048) == 0
+    with pytest.raises(ValueError):
+        pkv.kv_request_bytes(0, 8, 64, 10)
+    with pytest.raises(ValueError):
+        pkv.kv_request_bytes(16, 8, 64, -1)
