@@ -125,7 +125,7 @@ struct Layout {
     static constexpr int OFF_ROPE = OFF_NEWKV + STAGES * NEWKV_BYTES;
     static constexpr int OFF_MERGE = OFF_ROPE + STAGES * ROPE_BYTES;
     static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
-    static constexpr int OFF_MASK = OFF_BAR + (2 * STAGES + 1) * 8;  // full, empty, merge
+    static constexpr int OFF_MASK = OFF_BAR + (3 * STAGES + 1) * 8;  // full, empty, q, merge
     // Cluster mode: every CTA of a cluster stores its merged partial (o[D], m,
     // l per head) into slot `rank` of a landing area in rank 0's shared memory,
     // past everything else (rank 0 may still be computing when they land).
@@ -407,7 +407,7 @@ struct FirstItemGuess {
 template <typename T, int D, int G, bool FUSED>
 __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& guess,
                              const CUtensorMap* tmk, const CUtensorMap* tmv, uint8_t* base,
-                             uint64_t* full, uint64_t* empty, uint32_t* masks,
+                             uint64_t* full, uint64_t* empty, uint64_t* qbar, uint32_t* masks,
                              volatile int* s_abort, const int* s_len, const int* s_pre, int W) {
     using L = Layout<T, D, G>;
     const int lane = threadIdx.x & 31;
@@ -469,6 +469,8 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
     uint32_t phase = 0;
     uint32_t issued_parity[8];  // parity of the last issue into each stage
     uint32_t issued_any = 0;
+    // qbar: per stage, the parity of its next phase and whether a q copy was issued
+    uint32_t q_parity = 0, q_issued = 0;
     bool abort = false;
     if (item < W) {
     if (item1 < W) issue_claim();
@@ -538,7 +540,6 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             // stage's one arrival.
             if (lane == 0) {
                 const uint32_t bytes = __popc(vmask) * 2u * L::PAGE_BYTES +
-                                       (first ? (uint32_t)L::Q_COPY : 0u) +
                                        (patch_row >= 0 ? (uint32_t)L::NEWKV_BYTES : 0u);
                 mbar_expect_tx(&full[stage], bytes);
             }
@@ -566,7 +567,8 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             if (first && lane == 0) {
                 const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
                                       ((size_t)cur.b * p.Hq + (size_t)cur.h * G) * D * L::QSZ;
-                bulk_load(base + L::OFF_Q + stage * L::Q_BYTES, qsrc, L::Q_COPY, &full[stage]);
+                mbar_expect_tx(&qbar[stage], L::Q_COPY);
+                bulk_load(base + L::OFF_Q + stage * L::Q_BYTES, qsrc, L::Q_COPY, &qbar[stage]);
             }
             if (FUSED && patch_row >= 0 && lane == 1) {
                 const size_t row_off = ((size_t)cur.b * p.Hkv + cur.h) * L::ROW_COPY;
@@ -593,9 +595,16 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&full[stage]);
+            if (lane == 0) {
+                if (first) mbar_arrive(&qbar[stage]);
+                mbar_arrive(&full[stage]);
+            }
             issued_parity[stage] = phase;
             issued_any |= 1u << stage;
+            if (first) {
+                q_issued |= 1u << stage;
+                q_parity ^= 1u << stage;
+            }
             if (++stage == L::STAGES) {
                 stage = 0;
                 phase ^= 1;
@@ -618,7 +627,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
         // no more work: a stage without data whose item is -1 tells the consumers
         if (mbar_wait(&empty[stage], phase ^ 1) && !*s_abort) {
             s_item[stage] = -1;
-            mbar_arrive(&full[stage]);
+            mbar_arrive(&qbar[stage]);
         } else {
             abort = true;
         }
@@ -631,6 +640,8 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             // let every copy this warp started land before the CTA can exit
             for (int s = 0; s < L::STAGES; ++s)
                 if (issued_any & (1u << s)) (void)mbar_wait(&full[s], issued_parity[s]);
+            for (int s = 0; s < L::STAGES; ++s)
+                if (q_issued & (1u << s)) (void)mbar_wait(&qbar[s], ((q_parity >> s) & 1u) ^ 1u);
         }
         __syncwarp();
     }
@@ -796,7 +807,8 @@ __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Ite
 
 template <typename T, int D, int G, bool FUSED>
 __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
-                                 uint64_t* full, uint64_t* empty, uint64_t* merge_bar,
+                                 uint64_t* full, uint64_t* empty, uint64_t* qbar,
+                                 uint64_t* merge_bar,
                                  const uint32_t* masks, volatile int* s_abort, const int* s_len,
                                  const int* s_pre, int W) {
     using L = Layout<T, D, G>;
@@ -817,17 +829,20 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
     int merged = 0;  // items merged (cluster mode: at most one)
     int stage = 0;
     uint32_t phase = 0, mphase = 0;
+    uint32_t qph = 0;  // per stage, the parity of qbar's next phase
     // fused step: the item's rope table, staged by the producer with its first stage
     const float* tab = nullptr;
 
     const int* s_item = reinterpret_cast<const int*>(base + L::OFF_ITEM);
     for (;;) {
-        // the item's first stage says which item it is (-1: no more work)
-        if (!mbar_wait(&full[stage], phase) || *s_abort) {
+        // the item's first stage says on qbar which item it is (-1: no more
+        // work); its q and rope table are there too, its pages come on full
+        if (!mbar_wait(&qbar[stage], (qph >> stage) & 1u) || *s_abort) {
             *s_abort = 1;
             if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
             return -1;
         }
+        qph ^= 1u << stage;
         const int item = s_item[stage];
         if (item < 0) return merged;
         const Item it = decode_item(item, p, s_len, s_pre);
@@ -836,63 +851,60 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
         for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
         float m_run = kNegInf, l_run = 0.f;
         uint32_t qa[KS][4];
-
+        tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
+        // A fragments of Q: rows = query heads (see head_a/head_b), cols = dims.
+        const uint8_t* qs = base + L::OFF_Q + stage * L::Q_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const int col = kk * 16 + 2 * cq;
+            uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+            if constexpr (F8) {
+                // dims (D/4) cq + 4 kk .. +3 of the head, as two f16 pairs
+                auto quad = [&](int head, uint32_t& lo, uint32_t& hi) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(
+                        qs + (head * D + (D / 4) * cq + 4 * kk) * 2);
+                    lo = pack_f16(bf16lo(v.x), bf16hi(v.x));
+                    hi = pack_f16(bf16lo(v.y), bf16hi(v.y));
+                };
+                if (head_a >= 0) quad(head_a, a0, a2);
+                if (head_b >= 0) quad(head_b, a1, a3);
+            } else if (FUSED) {
+                // the staged q is the raw (unrotated) input: rotate the
+                // lane's own elements on the way into the fragment
+                auto pair = [&](int head, int c) -> uint32_t {
+                    const bf16* row = reinterpret_cast<const bf16*>(qs + head * D * 2);
+                    return pack_bf16(rotated_elem<bf16, D>(row, c, tab),
+                                     rotated_elem<bf16, D>(row, c + 1, tab));
+                };
+                if (head_a >= 0) {
+                    a0 = pair(head_a, col);
+                    a2 = pair(head_a, col + 8);
+                }
+                if (head_b >= 0) {
+                    a1 = pair(head_b, col);
+                    a3 = pair(head_b, col + 8);
+                }
+            } else if (head_a >= 0) {
+                const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_a * D * 2);
+                a0 = qr[col / 2];
+                a2 = qr[(col + 8) / 2];
+            }
+            if (!F8 && !FUSED && head_b >= 0) {
+                const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_b * D * 2);
+                a1 = qr[col / 2];
+                a3 = qr[(col + 8) / 2];
+            }
+            qa[kk][0] = a0;  // row r,   cols col, col+1
+            qa[kk][1] = a1;  // row r+8
+            qa[kk][2] = a2;  // row r,   cols col+8, col+9
+            qa[kk][3] = a3;  // row r+8
+        }
         const int nst = (it.npages + L::STAGE_PAGES - 1) / L::STAGE_PAGES;
         bool ok = true;
         int last = stage;
         for (int s = 0; s < nst; ++s) {
-            ok = (s == 0 || mbar_wait(&full[stage], phase)) && !*s_abort;
+            ok = mbar_wait(&full[stage], phase) && !*s_abort;
             if (!ok) break;
-            if (s == 0) {
-                tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
-                // A fragments of Q: rows = query heads (see head_a/head_b), cols = dims.
-                const uint8_t* qs = base + L::OFF_Q + stage * L::Q_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < KS; ++kk) {
-                    const int col = kk * 16 + 2 * cq;
-                    uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-                    if constexpr (F8) {
-                        // dims (D/4) cq + 4 kk .. +3 of the head, as two f16 pairs
-                        auto quad = [&](int head, uint32_t& lo, uint32_t& hi) {
-                            const uint2 v = *reinterpret_cast<const uint2*>(
-                                qs + (head * D + (D / 4) * cq + 4 * kk) * 2);
-                            lo = pack_f16(bf16lo(v.x), bf16hi(v.x));
-                            hi = pack_f16(bf16lo(v.y), bf16hi(v.y));
-                        };
-                        if (head_a >= 0) quad(head_a, a0, a2);
-                        if (head_b >= 0) quad(head_b, a1, a3);
-                    } else if (FUSED) {
-                        // the staged q is the raw (unrotated) input: rotate the
-                        // lane's own elements on the way into the fragment
-                        auto pair = [&](int head, int c) -> uint32_t {
-                            const bf16* row = reinterpret_cast<const bf16*>(qs + head * D * 2);
-                            return pack_bf16(rotated_elem<bf16, D>(row, c, tab),
-                                             rotated_elem<bf16, D>(row, c + 1, tab));
-                        };
-                        if (head_a >= 0) {
-                            a0 = pair(head_a, col);
-                            a2 = pair(head_a, col + 8);
-                        }
-                        if (head_b >= 0) {
-                            a1 = pair(head_b, col);
-                            a3 = pair(head_b, col + 8);
-                        }
-                    } else if (head_a >= 0) {
-                        const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_a * D * 2);
-                        a0 = qr[col / 2];
-                        a2 = qr[(col + 8) / 2];
-                    }
-                    if (!F8 && !FUSED && head_b >= 0) {
-                        const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_b * D * 2);
-                        a1 = qr[col / 2];
-                        a3 = qr[(col + 8) / 2];
-                    }
-                    qa[kk][0] = a0;  // row r,   cols col, col+1
-                    qa[kk][1] = a1;  // row r+8
-                    qa[kk][2] = a2;  // row r,   cols col+8, col+9
-                    qa[kk][3] = a3;  // row r+8
-                }
-            }
             // this warp's PPW consecutive pages of the stage (a page whose
             // block id was rejected counts as empty)
             constexpr int PPW = L::PPW;
@@ -1148,7 +1160,8 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
 
 template <typename T, int D, int G, bool FUSED>
 __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint8_t* base,
-                                  uint64_t* full, uint64_t* empty, uint64_t* merge_bar,
+                                  uint64_t* full, uint64_t* empty, uint64_t* qbar,
+                                  uint64_t* merge_bar,
                                   const uint32_t* masks, volatile int* s_abort, const int* s_len,
                                   const int* s_pre, int W) {
     using L = Layout<T, D, G>;
@@ -1163,6 +1176,7 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
     int merged = 0;  // items merged (cluster mode: at most one)
     int stage = 0;
     uint32_t phase = 0, mphase = 0;
+    uint32_t qph = 0;  // per stage, the parity of qbar's next phase
 
     auto load16 = [&](uint32_t addr, float (&f)[EPL]) {
         uint32_t w0, w1, w2, w3;
@@ -1184,12 +1198,14 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
 
     const int* s_item = reinterpret_cast<const int*>(base + L::OFF_ITEM);
     for (;;) {
-        // the item's first stage says which item it is (-1: no more work)
-        if (!mbar_wait(&full[stage], phase) || *s_abort) {
+        // the item's first stage says on qbar which item it is (-1: no more
+        // work); its q and rope table are there too, its pages come on full
+        if (!mbar_wait(&qbar[stage], (qph >> stage) & 1u) || *s_abort) {
             *s_abort = 1;
             if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
             return -1;
         }
+        qph ^= 1u << stage;
         const int item = s_item[stage];
         if (item < 0) return merged;
         const Item it = decode_item(item, p, s_len, s_pre);
@@ -1201,30 +1217,28 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
 #pragma unroll
             for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
         }
+        tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
+        if constexpr (FUSED) {
+            // raw q staged: rotate the lane's slice (rounded to T as an
+            // appended q would be)
+            const T* qrow0 = reinterpret_cast<const T*>(base + L::OFF_Q + stage * L::Q_BYTES);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < EPL; ++e)
+                    qf[g][e] = (float)to_d<T>(from_f<T>(
+                        rotated_elem<T, D>(qrow0 + g * D, c * EPL + e, tab)));
+        } else {
+            const uint32_t qs = smem_addr(base + L::OFF_Q + stage * L::Q_BYTES);
+#pragma unroll
+            for (int g = 0; g < G; ++g) load16(qs + g * D * (int)sizeof(T) + c * 16, qf[g]);
+        }
         const int nst = (it.npages + L::STAGE_PAGES - 1) / L::STAGE_PAGES;
         bool ok = true;
         int last = stage;
         for (int s = 0; s < nst; ++s) {
-            ok = (s == 0 || mbar_wait(&full[stage], phase)) && !*s_abort;
+            ok = mbar_wait(&full[stage], phase) && !*s_abort;
             if (!ok) break;
-            if (s == 0) {
-                tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
-                if constexpr (FUSED) {
-                    // raw q staged: rotate the lane's slice (rounded to T as an
-                    // appended q would be)
-                    const T* qrow0 = reinterpret_cast<const T*>(base + L::OFF_Q + stage * L::Q_BYTES);
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-#pragma unroll
-                        for (int e = 0; e < EPL; ++e)
-                            qf[g][e] = (float)to_d<T>(from_f<T>(
-                                rotated_elem<T, D>(qrow0 + g * D, c * EPL + e, tab)));
-                } else {
-                    const uint32_t qs = smem_addr(base + L::OFF_Q + stage * L::Q_BYTES);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) load16(qs + g * D * (int)sizeof(T) + c * 16, qf[g]);
-                }
-            }
 #pragma unroll 1
             for (int u = 0; u < L::PPW; ++u) {
             const int slot = warp * L::PPW + u;
@@ -1360,7 +1374,11 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
     uint64_t* empty = full + L::STAGES;
-    uint64_t* merge_bar = empty + L::STAGES;
+    // an item's first stage publishes its q (and rope table) on qbar before
+    // its pages complete full, so the q fragments are built while the
+    // pages are still in flight
+    uint64_t* qbar = empty + L::STAGES;
+    uint64_t* merge_bar = qbar + L::STAGES;
     uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
     int* misc = reinterpret_cast<int*>(base + L::OFF_MISC);
     volatile int* s_abort = misc;
@@ -1373,6 +1391,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         for (int s = 0; s < L::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], NW);
+            mbar_init(&qbar[s], 1);
         }
         mbar_init(merge_bar, NW * 32);
         *s_abort = 0;
@@ -1498,7 +1517,8 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
 
     // In cluster mode no thread leaves before the cluster merge below.
     if (warp == NW) {
-        run_producer<T, D, G, FUSED>(p, guess, &tm_k, &tm_v, base, full, empty, masks, s_abort,
+        run_producer<T, D, G, FUSED>(p, guess, &tm_k, &tm_v, base, full, empty, qbar, masks,
+                                     s_abort,
                                      s_len, s_pre, W);
         if (!p.cluster) return;
     } else {
@@ -1512,10 +1532,10 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         }
         int merged;
         if constexpr (MMA) {
-            merged = run_consumer_mma<T, D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks,
+            merged = run_consumer_mma<T, D, G, FUSED>(p, fr, base, full, empty, qbar, merge_bar, masks,
                                                       s_abort, s_len, s_pre, W);
         } else {
-            merged = run_consumer_simt<T, D, G, FUSED>(p, fr, base, full, empty, merge_bar, masks,
+            merged = run_consumer_simt<T, D, G, FUSED>(p, fr, base, full, empty, qbar, merge_bar, masks,
                                                        s_abort, s_len, s_pre, W);
         }
         if (p.cluster && merged <= 0) {
