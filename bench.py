@@ -34,6 +34,7 @@ import json
 import math
 import os
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -161,6 +162,14 @@ def software_versions() -> dict:
     """Versions the numbers were taken with (NVML read only)."""
     v = {"torch": torch.__version__, "cuda_runtime": torch.version.cuda,
          "kernel_sources": kernel_source_hash()}
+    try:
+        # the git commit, where the checkout carries its history
+        r = subprocess.run(["git", "-C", ROOT, "rev-parse", "--short", "HEAD"],
+                           capture_output=True, text=True, timeout=10)
+        if r.returncode == 0 and r.stdout.strip():
+            v["commit"] = r.stdout.strip()
+    except Exception:
+        pass
     try:
         import pynvml
         pynvml.nvmlInit()
