@@ -260,3 +260,107 @@ def _prefill(lib, **kw):
 ])
 def test_prefill_rejects_bad_arguments(lib, kw, status):
     assert _prefill(lib, **kw) == status
+
+
+def _step(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, slot=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE,
+             out=FAKE, ws=None, wsb=0, B=2, Hq=8, Hkv=2, d=64, NB=4, bs=16, MB=4, kvdt=BF16,
+             odt=BF16, theta=1e4, scale=0.125, P=0, flags=0, err=None)
+    a.update(kw)
+    return lib.pkv_decode_step(a["q"], a["k"], a["v"], a["pos"], a["slot"], a["kc"], a["vc"],
+                               a["bt"], a["cl"], a["out"], a["ws"], a["wsb"], a["B"], a["Hq"],
+                               a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"], a["kvdt"], a["odt"],
+                               a["theta"], a["scale"], a["P"], a["flags"], a["err"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(theta=0.0), INVALID),
+    (dict(theta=math.nan), INVALID),
+    (dict(kvdt=E4M3), UNSUPPORTED),        # the 8-bit cache has no fused step
+    (dict(d=96), UNSUPPORTED),
+    (dict(Hq=24, Hkv=2), UNSUPPORTED),     # group size 12
+    (dict(flags=0x10), INVALID),
+    (dict(scale=-math.inf), INVALID),
+    (dict(k=None), INVALID),
+    (dict(slot=None), INVALID),
+    (dict(v=FAKE + 8), INVALID),           # new rows 16-byte aligned
+    (dict(pos=FAKE + 4), INVALID),         # int64 arrays 8-byte aligned
+    (dict(P=16, MB=4), WORKSPACE),         # split path needs a workspace
+    (dict(P=16, MB=4, ws=FAKE, wsb=64), WORKSPACE),
+    (dict(B=0, q=None, k=None, out=None), OK),
+])
+def test_decode_step_rejects_bad_arguments(lib, kw, status):
+    assert _step(lib, **kw) == status
+    if status != OK:
+        assert lib.pkv_last_error() != b""
+
+
+def _cascade(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, gs=FAKE, sh=FAKE, out=FAKE, ws=None,
+             wsb=0, B=8, G=1, MG=8, Hq=8, Hkv=2, d=64, NB=64, bs=16, MB=8, kvdt=BF16, odt=BF16,
+             scale=0.125, P=0, flags=0, err=None)
+    a.update(kw)
+    return lib.pkv_paged_attention_decode_cascade(
+        a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["gs"], a["sh"], a["out"], a["ws"], a["wsb"],
+        a["B"], a["G"], a["MG"], a["Hq"], a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"], a["kvdt"],
+        a["odt"], a["scale"], a["P"], a["flags"], a["err"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kvdt=F32), UNSUPPORTED),         # bf16 cache only
+    (dict(odt=E4M3), UNSUPPORTED),
+    (dict(d=80), UNSUPPORTED),
+    (dict(B=257, MG=8), UNSUPPORTED),      # over 256 sequences
+    (dict(flags=0x2), INVALID),            # only the CUDA-core flag applies
+    (dict(G=-1), INVALID),
+    (dict(MG=0), INVALID),                 # a group needs a member
+    (dict(MG=9), INVALID),                 # larger than the batch
+    (dict(scale=math.nan), INVALID),
+    (dict(NB=0), INVALID),
+    (dict(sh=None), INVALID),
+    (dict(gs=None), INVALID),              # groups given, no offsets
+    (dict(gs=FAKE + 2), INVALID),
+    (dict(MB=0), INVALID),
+    (dict(gs=None, G=0), WORKSPACE),       # no groups: only the workspace is missing
+    (dict(ws=FAKE, wsb=255), WORKSPACE),
+    (dict(B=0, G=0, q=None, out=None), OK),
+])
+def test_cascade_rejects_bad_arguments(lib, kw, status):
+    assert _cascade(lib, **kw) == status
+    if status != OK:
+        assert lib.pkv_last_error() != b""
+
+
+def test_cascade_workspace_size_formula(lib):
+    """256 bytes of scheduler counters, then NP + 1 partial slots per
+    (sequence, q head): slot 0 holds the shared-prefix pass."""
+    a = lambda x: (x + 255) // 256 * 256
+    B, Hq, d, MB, P = 64, 32, 64, 2049, 512
+    NP = math.ceil(MB * 16 / P)
+    slots = B * Hq * (NP + 1)
+    assert lib.pkv_decode_cascade_workspace_size(B, Hq, 8, d, MB, 16, BF16, P) == \
+        256 + a(slots * d * 4) + a(slots * 2 * 4)
+    # one partition still keeps the prefix slot
+    slots = 4 * 8 * 2
+    assert lib.pkv_decode_cascade_workspace_size(4, 8, 2, 64, 4, 16, BF16, 64) == \
+        256 + a(slots * 64 * 4) + a(slots * 2 * 4)
+    assert lib.pkv_decode_cascade_workspace_size(4, 8, 2, 64, 4, 16, F32, 64) == 0    # bf16 only
+    assert lib.pkv_decode_cascade_workspace_size(4, 8, 2, 64, 4, 16, BF16, 24) == 0   # bad P
+    assert lib.pkv_decode_cascade_workspace_size(-1, 8, 2, 64, 4, 16, BF16, 64) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), UNSUPPORTED),             # invalid shapes need no scratch: plain checks
+    (dict(kvdt=7), UNSUPPORTED),
+    # 64 x 32 heads x 64 partitions of d=128 partials: more than the 16 MiB scratch
+    (dict(B=64, Hq=32, Hkv=8, d=128, MB=512, P=128), WORKSPACE),
+])
+def test_noalloc_rejects_before_touching_the_device(lib, kw, status):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, out=FAKE, B=2, Hq=8, Hkv=2, d=64, NB=4,
+             bs=16, MB=4, kvdt=BF16, odt=BF16, scale=0.125, P=0, flags=0, err=None)
+    a.update(kw)
+    st = lib.pkv_paged_attention_decode_noalloc(
+        a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"], a["B"], a["Hq"], a["Hkv"], a["d"],
+        a["NB"], a["bs"], a["MB"], a["kvdt"], a["odt"], a["scale"], a["P"], a["flags"], a["err"],
+        None)
+    assert st == status
