@@ -808,3 +808,62 @@ def test_planted_mistake_is_caught(name, old, new, tmp_path):
         except (AssertionError, OracleError):
             caught.append(pin.__name__)
     assert caught, f"no pin catches the planted mistake {name}"
+
+
+# Planted mistakes in the oracle's Python layer (argument marshalling and the
+# chunked prefill built on the decode): the mutated copy of oracle/__init__.py
+# is loaded as its own module over the unmodified C library.
+PY_MUTATIONS = [
+    ("prefill_query_misses_own_token",
+     "lens_i = (context_lens.to(torch.int64) - C + i + 1).clamp(min=0)",
+     "lens_i = (context_lens.to(torch.int64) - C + i).clamp(min=0)"),
+    ("prefill_not_causal_in_chunk",
+     "lens_i = (context_lens.to(torch.int64) - C + i + 1).clamp(min=0)",
+     "lens_i = context_lens.to(torch.int64).clamp(min=0)"),
+    ("prefill_ignores_window",
+     "nthreads=nthreads, window=window)\n        return out\n\n    def contiguous_decode",
+     "nthreads=nthreads, window=0)\n        return out\n\n    def contiguous_decode"),
+    ("e4m3_scales_swapped",
+     "float(scale), float(k_scale), float(v_scale),\n                                              int(window)",
+     "float(scale), float(v_scale), float(k_scale),\n                                              int(window)"),
+    ("e4m3_append_scales_swapped",
+     "T, Hq, Hkv, d, NB, bs, float(rope_theta),\n                                           float(k_scale), float(v_scale))",
+     "T, Hq, Hkv, d, NB, bs, float(rope_theta),\n                                           float(v_scale), float(k_scale))"),
+    ("decode_window_dropped",
+     "float(scale), int(window), pp, npairs, int(nthreads),",
+     "float(scale), 0, pp, npairs, int(nthreads),"),
+]
+
+
+def _oracle_module_copy(name, src):
+    import types
+
+    mod = types.ModuleType(f"oracle._copy_{name}")
+    mod.__package__ = "oracle"
+    mod.__file__ = oracle.__file__
+    exec(compile(src, f"<oracle copy {name}>", "exec"), mod.__dict__)
+    # the copy raises the original error class, which the pins expect
+    mod.OracleError = OracleError
+    return mod
+
+
+def test_unmutated_module_copy_passes_every_pin():
+    """Control for the harness below: loading the module this way changes
+    nothing by itself."""
+    copy = _oracle_module_copy("control", open(oracle.__file__).read()).Oracle()
+    for pin in PINS:
+        pin(copy)
+
+
+@pytest.mark.parametrize("name,old,new", PY_MUTATIONS, ids=[m[0] for m in PY_MUTATIONS])
+def test_planted_marshalling_mistake_is_caught(name, old, new):
+    src = open(oracle.__file__).read()
+    assert src.count(old) == 1, f"mutation {name} does not match the oracle module exactly once"
+    mutant = _oracle_module_copy(name, src.replace(old, new)).Oracle()
+    caught = []
+    for pin in PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, OracleError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name}"
