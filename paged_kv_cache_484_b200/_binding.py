@@ -158,11 +158,15 @@ def _kv_dtype_code(dt: torch.dtype) -> int:
     return _dtype_code(dt)
 
 
-def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+def _dev(t: torch.Tensor, name: str, dtype=None, on=None) -> int:
+    """Device address of a contiguous CUDA tensor.  ``on``: the device of the
+    call (that of q); a kernel may only be handed memory of its own GPU."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if on is not None and t.device != on:
+        raise ValueError(f"{name} is on {t.device}, the call's other tensors on {on}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -191,6 +195,7 @@ def kv_append(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_t
     (slot < 0: skip the write).  See include/pkv.h, pkv_kv_append.
     """
     lib = load_library()
+    dv = q.device
     dt = _dtype_code(q.dtype)
     for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache)):
         if t.dtype != q.dtype:
@@ -200,11 +205,13 @@ def kv_append(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_t
     if k_new.shape != (T, Hkv, d) or v_new.shape != (T, Hkv, d) or v_cache.shape != k_cache.shape \
             or d2 != d or positions.shape != (T,) or slot_mapping.shape != (T,):
         raise ValueError("inconsistent kv_append shapes")
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
     st = lib.pkv_kv_append(
-        _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
-        _dev(positions, "positions", torch.int64), _dev(slot_mapping, "slot_mapping", torch.int64),
-        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
+        _dev(positions, "positions", torch.int64, on=dv),
+        _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
+        _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
         T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "kv_append")
 
@@ -269,6 +276,7 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     (pkv_paged_attention_decode_window).  See include/pkv.h.
     """
     lib = load_library()
+    dv = q.device
     kv_dt = _dtype_code(k_cache.dtype)
     if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
         raise TypeError("q, k_cache and v_cache must share one dtype")
@@ -282,11 +290,12 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     if workspace is None:
         need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
         workspace = new_workspace(int(need), q.device)
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
-    args = [_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-            _dev(block_tables, "block_tables", torch.int32),
-            _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
-            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
+    args = [_dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+            _dev(block_tables, "block_tables", torch.int32, on=dv),
+            _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+            _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
             B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale)]
     tail = [int(partition_tokens), _flags(force_simt, cluster), err, _stream_ptr(stream, q.device)]
     if sliding_window:
@@ -305,6 +314,7 @@ def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, r
     v_cache uint8 [NB, Hkv, d, 16] (pages transposed) those of v / v_scale.
     See include/pkv.h, pkv_kv_append_e4m3."""
     lib = load_library()
+    dv = q.device
     dt = _dtype_code(q.dtype)
     for name, t in (("k_new", k_new), ("v_new", v_new)):
         if t.dtype != q.dtype:
@@ -315,11 +325,13 @@ def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, r
             or v_cache.shape != (NB, Hkv, d, bs) or positions.shape != (T,) \
             or slot_mapping.shape != (T,):
         raise ValueError("inconsistent kv_append_e4m3 shapes")
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
     st = lib.pkv_kv_append_e4m3(
-        _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
-        _dev(positions, "positions", torch.int64), _dev(slot_mapping, "slot_mapping", torch.int64),
-        _dev(k_cache, "k_cache", torch.uint8), _dev(v_cache, "v_cache", torch.uint8),
+        _dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
+        _dev(positions, "positions", torch.int64, on=dv),
+        _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
+        _dev(k_cache, "k_cache", torch.uint8, on=dv), _dev(v_cache, "v_cache", torch.uint8, on=dv),
         T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), float(k_scale), float(v_scale), err,
         _stream_ptr(stream, q.device))
     _raise(st, lib, "kv_append_e4m3")
@@ -334,6 +346,7 @@ def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens,
     cached values are code x k_scale / code x v_scale.  Writes and returns
     ``out`` (float32 or bfloat16).  See include/pkv.h."""
     lib = load_library()
+    dv = q.device
     B, Hq, d = q.shape
     NB, Hkv, bs, d2 = k_cache.shape
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
@@ -344,12 +357,14 @@ def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens,
         need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, PKV_DTYPE_E4M3,
                                              int(partition_tokens))
         workspace = new_workspace(int(need), q.device)
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
     st = lib.pkv_paged_attention_decode_e4m3(
-        _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.uint8),
-        _dev(v_cache, "v_cache", torch.uint8), _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _dev(q, "q", torch.bfloat16, on=dv), _dev(k_cache, "k_cache", torch.uint8, on=dv),
+        _dev(v_cache, "v_cache", torch.uint8, on=dv),
+        _dev(block_tables, "block_tables", torch.int32, on=dv),
+        _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+        _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
         B, Hq, Hkv, d, NB, bs, MB, _dtype_code(out.dtype), float(scale), float(k_scale),
         float(v_scale), int(sliding_window), int(partition_tokens), _flags(False, cluster), err,
         _stream_ptr(stream, q.device))
@@ -363,6 +378,7 @@ def _decode_step_args(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache
     """Checked pkv_decode_step arguments (allocating a workspace if none is
     given), and the tensors they point into."""
     lib = load_library()
+    dv = q.device
     kv_dt = _dtype_code(k_cache.dtype)
     for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("v_cache", v_cache)):
         if t.dtype != k_cache.dtype:
@@ -378,14 +394,15 @@ def _decode_step_args(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache
     if workspace is None:
         need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, kv_dt, int(partition_tokens))
         workspace = new_workspace(int(need), q.device)
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
-    args = (_dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
-            _dev(positions, "positions", torch.int64),
-            _dev(slot_mapping, "slot_mapping", torch.int64),
-            _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-            _dev(block_tables, "block_tables", torch.int32),
-            _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
-            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
+    args = (_dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
+            _dev(positions, "positions", torch.int64, on=dv),
+            _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
+            _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+            _dev(block_tables, "block_tables", torch.int32, on=dv),
+            _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+            _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
             B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(rope_theta),
             float(scale), int(partition_tokens), _flags(force_simt, cluster), err,
             _stream_ptr(stream, q.device))
@@ -459,6 +476,7 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
     See include/pkv.h, pkv_paged_attention_decode_noalloc.
     """
     lib = load_library()
+    dv = q.device
     kv_dt = _dtype_code(k_cache.dtype)
     if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
         raise TypeError("q, k_cache and v_cache must share one dtype")
@@ -468,11 +486,12 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
     if v_cache.shape != k_cache.shape or d2 != d or out.shape != (B, Hq, d) \
             or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("inconsistent paged_attention_decode_noalloc shapes")
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
     st = lib.pkv_paged_attention_decode_noalloc(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
+        _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+        _dev(block_tables, "block_tables", torch.int32, on=dv),
+        _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
         B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(scale),
         int(partition_tokens), _flags(force_simt, cluster), err,
         _stream_ptr(stream, q.device))
@@ -513,6 +532,7 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, sca
     writes and returns ``out``.  See include/pkv.h, pkv_paged_attention_prefill.
     """
     lib = load_library()
+    dv = q.device
     if q.dtype != torch.bfloat16 or k_cache.dtype != torch.bfloat16 \
             or v_cache.dtype != torch.bfloat16:
         raise TypeError("prefill: q and the caches must be bfloat16")
@@ -525,12 +545,13 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, sca
     need = lib.pkv_prefill_workspace_size(B, C, Hq, Hkv, d, MB, bs, int(partition_tokens))
     if workspace is None:
         workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
     st = lib.pkv_paged_attention_prefill(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), _dev(out, "out"),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+        _dev(block_tables, "block_tables", torch.int32, on=dv),
+        _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+        _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
         B, C, Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16, _dtype_code(out.dtype), float(scale),
         int(sliding_window), int(partition_tokens), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_prefill")
@@ -557,6 +578,7 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_le
     the group's shared blocks.  Same result; each shared prefix is read once
     per group.  bf16 only; q already rotated.  See include/pkv.h."""
     lib = load_library()
+    dv = q.device
     if q.dtype != torch.bfloat16 or k_cache.dtype != torch.bfloat16 \
             or v_cache.dtype != torch.bfloat16:
         raise TypeError("cascade: q and the caches must be bfloat16")
@@ -572,14 +594,15 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_le
                                                  int(partition_tokens))
     if workspace is None:
         workspace = new_workspace(int(need), q.device)
-    err = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
     st = lib.pkv_paged_attention_decode_cascade(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32),
-        _dev(group_start, "group_start", torch.int32) if NG else None,
-        _dev(shared_tokens, "shared_tokens", torch.int32), _dev(out, "out"),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+        _dev(block_tables, "block_tables", torch.int32, on=dv),
+        _dev(context_lens, "context_lens", torch.int32, on=dv),
+        _dev(group_start, "group_start", torch.int32, on=dv) if NG else None,
+        _dev(shared_tokens, "shared_tokens", torch.int32, on=dv), _dev(out, "out", on=dv),
+        _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
         B, NG, int(max_group_size), Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16,
         _dtype_code(out.dtype), float(scale), int(partition_tokens),
         _flags(force_simt, True), err, _stream_ptr(stream, q.device))
