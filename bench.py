@@ -1,30 +1,34 @@
 #!/usr/bin/env python3
-"""Benchmark of one paged decode step: kv_append + paged_attention_decode.
+"""Benchmark of the paged decode step: kv_append + paged_attention_decode.
 
-Default workload: the Llama-3.2-1B-shaped single-layer decode step (batch 1,
-32 query / 8 KV heads, head_dim 64, 2048 cached tokens + 1 appended, block
-size 16, 4096-block shuffled pool, bf16).  ``--config N`` picks another of
-the five named workloads.  Metric: achieved HBM GB/s of the step's
-algorithmic bytes (K/V of every context token + q + out), with seq-steps/s
-alongside.
+Default run: one JSON line for the long-context workload (16 sequences x
+131072 cached tokens + 1 appended, 32 query / 8 KV heads, head_dim 128,
+block size 16, bf16, 1 % of key rows x8, split-K with a partition combine:
+8.6 GB of K/V per step), the largest single-GPU workload and the cleanest
+HBM roofline case.  The same line carries, under ``per_config``, the other
+bf16 workloads timed the same way (same K and W): the batch-1 Llama-3.2-1B
+layer step, the ragged batch of 64 and the 256-sequence prefix-sharing mix.
+``--config N`` times workload N alone.  Metric: achieved HBM GB/s of the
+step's algorithmic bytes (K/V of every context token + q + out), with
+seq-steps/s alongside.
 
 Timing: W warm-up steps, then exactly K timed steps back to back between one
-pair of CUDA events on the launch stream (synchronised on both sides); the
+pair of CUDA events on the launch stream (synchronised on both sides).  The
 steps are replays of CUDA graphs that captured the library call(s) of
-consecutive steps, so host-side marshalling does not set the pace.  The
-inputs are larger than L2: when one copy of the workload touches less than
-twice the L2 size per step, the bench holds enough device-side copies (like
-the per-layer caches of a model) and step k runs on copy k mod n, so every
-step reads its K/V from HBM.  ``isolated_step`` in the output is the older,
-pessimistic figure: one step at a time, L2 flushed before it (512 MiB
-written, then 256 MiB read so no dirty line remains), each step between its
-own pair of events (whose own cost, a few microseconds, it includes).
-Under torchrun every rank runs its own copy of the workload (weak scaling,
-no collective on the data path); the step time is the max over ranks.
+consecutive steps, so host-side marshalling does not set the pace; every
+graph the timed region replays has been replayed before it.  The inputs are
+larger than L2: when one copy of the workload touches less than twice the L2
+size per step, the bench holds enough device-side copies (like the per-layer
+caches of a model) that every timed step reads a copy no step of the last
+2 x L2 bytes touched.  ``isolated_step`` is the older, pessimistic figure:
+one step at a time, L2 flushed before it, each step between its own pair of
+events (whose own cost, a few microseconds, it includes).  Under torchrun
+every rank runs its own copy of the workload (weak scaling, no collective on
+the data path); the step time is the max over ranks.
 
-``--impl reference`` times the fp64 CPU oracle on the same workload instead
-(rank 0 only); it is the deliberately slow definition the CUDA path is
-checked against, not an optimised baseline.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only); it is the deliberately slow definition
+the CUDA path is checked against, not an optimised baseline.
 """
 from __future__ import annotations
 
@@ -47,15 +51,25 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode-attention achieved HBM GB/s (% of B200 peak); seq-steps/sec"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 512 << 20
-DEFAULT_CONFIG = 2
+HEADLINE_CONFIG = 5
+SECONDARY_CONFIGS = (2, 3, 4)
+# the oracle's bounded sample: whole sequences while their K/V stay within this
+SAMPLE_KV_BYTES = 1_100_000_000
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5],
+                    help="time this workload alone (default: the long-context workload, "
+                         "with the other bf16 workloads under per_config)")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="default run: leave out the per_config workloads")
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="keep only the first N sequences of the workload (small profiler "
+                         "captures of the same kernel)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--partition-tokens", type=int, default=0)
@@ -75,7 +89,7 @@ def parse_args(argv=None):
                          "workload's prefix groups (config 4)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--prefill", type=int, default=0, metavar="C",
                     help="time chunked prefill instead: the last C context tokens of every "
@@ -183,7 +197,9 @@ def software_versions() -> dict:
 def recorded_traffic(cfg):
     """DRAM bytes per decode launch from the committed ncu capture, if it was
     taken on the current kernel sources (else None).  ``cfg``: the config
-    number, or e.g. "3_e4m3" for its 8-bit cache."""
+    number, or e.g. "3_e4m3" for its 8-bit cache.  A workload captured on a
+    smaller batch of the same kernel is recorded already scaled to the full
+    launch."""
     path = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
     try:
         with open(path) as f:
@@ -198,7 +214,8 @@ def recorded_traffic(cfg):
 
 class ClockSampler:
     """Polls SM clock and throttle reasons through NVML (read only) while the
-    timed region runs."""
+    timed region runs.  The first sample is taken before ``__enter__``
+    returns, so even a region shorter than the polling period has one."""
 
     REASONS = {
         0x0000000000000004: "sw_power_cap",
@@ -208,11 +225,12 @@ class ClockSampler:
         0x0000000000000080: "hw_power_brake_slowdown",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples = []
         self.reasons = set()
         self.max_mhz = None
         self._stop = threading.Event()
+        self._first = threading.Event()
         self._period = period_s
         self._ok = False
         try:
@@ -225,23 +243,29 @@ class ClockSampler:
         except Exception:
             self._ok = False
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self._period)
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
+        self._sample()
+        self._first.set()
+        while not self._stop.wait(self._period):
+            self._sample()
+        self._sample()
 
     def __enter__(self):
         if self._ok:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
+            self._first.wait(5.0)
         return self
 
     def __exit__(self, *exc):
@@ -260,9 +284,10 @@ class ClockSampler:
 def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
     from paged_kv_cache_484_b200 import workloads as W
     s = W.config_summary(cfg)
+    name = w.name if w.name.startswith(W.CONFIG_NAMES[cfg]) else W.CONFIG_NAMES[cfg]
     if w.k_cache.dtype == torch.uint8:
         return {
-            "workload": W.CONFIG_NAMES[cfg] + "_e4m3cache",
+            "workload": name + "_e4m3cache",
             "batch_seqs": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
             "context": s["ctx"], "tokens_decoded": int(w.decode_lens.to(torch.int64).sum().item()),
             "block_size": w.block_size, "pool_blocks": w.num_blocks,
@@ -273,7 +298,7 @@ def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
             "step": "two calls (kv_append_e4m3, paged_attention_decode_e4m3)",
         }
     return {
-        "workload": W.CONFIG_NAMES[cfg],
+        "workload": name,
         "batch_seqs": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
         "context": s["ctx"], "tokens_decoded": int(w.decode_lens.to(torch.int64).sum().item()),
         "block_size": w.block_size, "pool_blocks": w.num_blocks,
@@ -286,70 +311,129 @@ def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
     }
 
 
+# ---------------------------------------------------------------- timing plan
+
+def copies_plan(nbytes: int, l2_bytes: int, K: int, forced: int = 0):
+    """How many device-side copies of the workload the bench holds, and how
+    many consecutive steps one CUDA graph captures (S).
+
+    A step whose inputs exceed twice the L2 size runs on one copy.  Otherwise
+    ``n_min`` copies put 2 x L2 bytes of other steps between two uses of the
+    same copy.  Graphs: one of S steps over copies 0..S-1 and, when S does not
+    divide K, one of the K mod S first steps; the timed region replays the
+    first K // S times, then the second.  When K is small, K extra copies
+    keep even the tail graph's copies out of L2: the warm-up replays of both
+    graphs end with ``n - K >= n_min`` steps on other copies."""
+    if forced:
+        n = forced
+        return n, (n if n > 1 else min(K, 16))
+    n_min = 1 if nbytes >= 2 * l2_bytes else 1 + math.ceil(2 * l2_bytes / nbytes)
+    if n_min == 1:
+        return 1, min(K, 16)
+    n = n_min + K if K <= 4 * n_min else n_min
+    return n, n
+
+
+def replay_order(K: int, S: int):
+    """Graph replays: (warm-up, timed), as lists of graph lengths in steps.
+    The warm-up replays the tail graph (if any) and then the full graph, so
+    every graph the timed region replays has run once (its first launch pays
+    the graph's upload) and the last warm-up steps use the highest copies."""
+    tail = K % S
+    warm = ([tail] if tail else []) + [S]
+    timed = [S] * (K // S) + ([tail] if tail else [])
+    return warm, timed
+
+
 # ---------------------------------------------------------------- oracle arm
 
-def time_oracle(w, seconds: float, nthreads: int, e4m3_scales=None, window: int = 0):
-    """Oracle append + decode of the whole workload (or a bounded subset of
-    sequences for the big ones), repeated until ~``seconds`` of CPU time
-    (the 8-bit cache's append and decode when ``e4m3_scales`` is given)."""
-    import oracle
-    from paged_kv_cache_484_b200.workloads import extract_sequences
-
-    order = list(range(w.B))
-    # bounded sample: whole sequences until the sample holds <= 8M context tokens
+def oracle_sample(w, window: int = 0):
+    """The oracle's bounded sample of a workload: whole sequences, in order,
+    while their K/V stay within SAMPLE_KV_BYTES (at least one).  Returns the
+    sequence indices and the fraction of the step's attended tokens they
+    hold."""
     lens = w.decode_lens.cpu().tolist()
-    seqs, tok = [], 0
-    for b in order:
-        if seqs and tok + lens[b] > 8_000_000:
+    row = w.Hkv * w.d * 2 * w.k_cache.element_size()
+    seqs, kv = [], 0
+    for b in range(w.B):
+        if seqs and kv + lens[b] * row > SAMPLE_KV_BYTES:
             break
         seqs.append(b)
-        tok += lens[b]
-    sub = extract_sequences(w, seqs)
-    att = [min(L, window) if window else L for L in lens]  # attended tokens
-    frac_bytes = sum(att[b] for b in seqs) / max(1, sum(att))
+        kv += lens[b] * row
+    att = [min(L, window) if window else L for L in lens]
+    return seqs, sum(att[b] for b in seqs) / max(1, sum(att))
+
+
+def oracle_step(sub, nthreads: int, e4m3_scales=None, window: int = 0):
+    """One oracle append + decode over the sample; returns its seconds.  The
+    append writes the same rows every time, so only q (rotated in place) is
+    restored between repetitions."""
+    import oracle
+    q = sub.q.clone()
+    t0 = time.perf_counter()
+    if e4m3_scales is not None:
+        ks, vs = e4m3_scales
+        oracle.kv_append_e4m3(q, sub.k_new, sub.v_new, sub.positions, sub.slots, sub.k_cache,
+                              sub.v_cache, sub.theta, ks, vs)
+        oracle.paged_attention_decode_e4m3(q, sub.k_cache, sub.v_cache, sub.tables,
+                                           sub.decode_lens, sub.scale, ks, vs, nthreads=nthreads,
+                                           window=window)
+    else:
+        oracle.kv_append(q, sub.k_new, sub.v_new, sub.positions, sub.slots, sub.k_cache,
+                         sub.v_cache, sub.theta)
+        oracle.paged_attention_decode(q, sub.k_cache, sub.v_cache, sub.tables, sub.decode_lens,
+                                      sub.scale, nthreads=nthreads, window=window)
+    return time.perf_counter() - t0
+
+
+def time_oracle(sub, seconds: float, nthreads: int, e4m3_scales=None, window: int = 0):
+    """Oracle steps over the sample, repeated until ~``seconds`` of CPU time."""
     reps, t_total = 0, 0.0
     while t_total < seconds or reps == 0:
-        q = sub.q.clone()
-        kc, vc = sub.k_cache.clone(), sub.v_cache.clone()
-        t0 = time.perf_counter()
-        if e4m3_scales is not None:
-            ks, vs = e4m3_scales
-            oracle.kv_append_e4m3(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions,
-                                  sub.slots, kc, vc, sub.theta, ks, vs)
-            oracle.paged_attention_decode_e4m3(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
-                                               ks, vs, nthreads=nthreads, window=window)
-        else:
-            oracle.kv_append(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions, sub.slots,
-                             kc, vc, sub.theta)
-            oracle.paged_attention_decode(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
-                                          nthreads=nthreads, window=window)
-        t_total += time.perf_counter() - t0
+        t_total += oracle_step(sub, nthreads, e4m3_scales, window)
         reps += 1
-    return t_total / reps, seqs, frac_bytes, reps
+    return t_total / reps, reps
 
 
 def run_reference(args):
+    """The fp64 oracle, as it stands, on the host cores: W untimed and K timed
+    steps, each one append + decode pass over the bounded sample of the same
+    seeded workload (generated on the GPU when there is one, as the CUDA arm
+    generates it; no library kernel runs)."""
     world, rank, local = dist_env()
     if rank != 0:
         return 0
     from paged_kv_cache_484_b200 import workloads as W
+    cfg = args.config or HEADLINE_CONFIG
     out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
-    w = W.make_config(args.config, device="cpu")
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    w = W.make_config(cfg, device=dev, num_seqs=args.num_seqs)
+    seqs, frac = oracle_sample(w)
+    sub = W.extract_sequences(w, seqs)
+    nbytes = step_bytes(w, out_dtype)
+    del w
+    if dev.type == "cuda":
+        torch.cuda.empty_cache()
     nthreads = os.cpu_count() or 1
-    per_step, seqs, frac, reps = time_oracle(w, max(1.0, min(args.cpu_seconds, 60.0)), nthreads)
-    bytes_sample = step_bytes(w, out_dtype) * frac
-    value = bytes_sample / per_step / 1e9
+    for _ in range(max(0, args.warmup)):
+        oracle_step(sub, nthreads)
+    K = max(1, args.steps)
+    per_step = sum(oracle_step(sub, nthreads) for _ in range(K)) / K
+    value = nbytes * frac / per_step / 1e9
+    B = W.config_summary(cfg)["B"] if args.num_seqs is None else args.num_seqs
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
-        "n_gpus": args.gpus, "steps": reps, "warmup": 0,
+        "n_gpus": args.gpus, "steps": K, "warmup": max(0, args.warmup),
         "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "seq_steps_per_s": round(len(seqs) / per_step, 3),
-        "config": config_block(args.config, w, out_dtype, None, None, False),
+        "config": {"workload": W.CONFIG_NAMES[cfg], **W.config_summary(cfg),
+                   **({"num_seqs": args.num_seqs} if args.num_seqs is not None else {})},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads,
                          "kind": "oracle",
-                         "sample": f"{len(seqs)} of {w.B} sequences, full append+decode step, "
-                                   f"{reps} repetitions"},
+                         "sample": f"sequences {seqs[0]}..{seqs[-1]} ({len(seqs)} of {B}, "
+                                   f"{100 * frac:.1f} % of the step's K/V), one fp64 append + "
+                                   f"decode pass over them per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -359,37 +443,38 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- CUDA arm
 
-def run_ours(args):
-    world, rank, local = dist_env()
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    init_dist(world, local)
-
+def measure(cfg, args, device, world, local, rank, full: bool):
+    """Time workload ``cfg`` as the bench's step.  Returns the JSON fields of
+    its line (``full``: with the end-to-end figure and the CPU baseline)."""
     import paged_kv_cache_484_b200 as pkv
     from paged_kv_cache_484_b200 import workloads as W
 
-    pkv.load_library()
     out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
-    w = W.make_config(args.config, device=device)
+    w = W.make_config(cfg, device=device, num_seqs=args.num_seqs)
     e4m3 = args.kv_dtype == "e4m3"
+    two_calls = args.two_calls
+    ks8 = vs8 = None
     if e4m3:
         if w.dtype != torch.bfloat16:
             raise SystemExit("--kv-dtype e4m3 takes a bf16 workload (configs 2-5)")
         k8, v8, ks8, vs8 = W.e4m3_cache(w)
         w.k_cache, w.v_cache = k8, v8
         w.meta["e4m3_scales"] = (ks8, vs8)
-        args.two_calls = True
+        two_calls = True
         torch.cuda.empty_cache()
     kv_dt = torch.uint8 if e4m3 else w.dtype
     host_inputs = None
-    if not args.no_e2e:
+    if full and not args.no_e2e:
         # pristine copies of the per-step inputs, in pinned host memory
         host_inputs = {k: v.cpu().pin_memory() for k, v in dict(
             q=w.q, k_new=w.k_new, v_new=w.v_new, positions=w.positions,
             slot_mapping=w.slot_mapping, block_tables=w.block_tables,
             decode_lens=w.decode_lens).items()}
+    sample = None
+    if full and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle's bounded sample, copied to the host before any step
+        seqs, frac = oracle_sample(w, args.window)
+        sample = (W.extract_sequences(w, seqs), frac)
 
     P = args.partition_tokens or pkv.decode_partition_tokens(w.B, w.Hq, w.Hkv, w.d, w.max_blocks,
                                                               kv_dtype=kv_dt)
@@ -402,14 +487,12 @@ def run_ours(args):
     if args.window:
         if args.cascade:
             raise SystemExit("--window and --cascade do not combine")
-        args.two_calls = True
+        two_calls = True
 
-    # Inputs larger than L2: device-side copies of the workload (every tensor
-    # a step reads or writes), step k on copy k mod n.
+    K = args.steps
+    Wu = max(3, args.warmup)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    ncopies = 1 if nbytes >= 2 * l2 else min(1024, math.ceil(2 * l2 / nbytes))
-    if args.copies:
-        ncopies = args.copies
+    ncopies, S = copies_plan(nbytes, l2, K, args.copies)
     # Per-layer tensors (q, the new rows, the caches) get their own copy; the
     # step's metadata (positions, slots, block tables, context lengths) is one
     # set shared by all copies, as one decode step's metadata is shared by all
@@ -428,7 +511,7 @@ def run_ours(args):
             raise SystemExit("--cascade takes the bf16 cache")
         if w.meta.get("prefix_group", 0) <= 1:
             raise SystemExit("--cascade needs a workload with prefix groups (config 4)")
-        args.two_calls = True
+        two_calls = True
         grp = int(w.meta["prefix_group"])
         group_start = torch.tensor(list(range(0, w.B, grp)) + [w.B], dtype=torch.int32,
                                    device=device)
@@ -438,7 +521,7 @@ def run_ours(args):
                          * 16).to(torch.int32)
         ws = pkv.new_workspace(pkv.decode_cascade_workspace_size(
             w.B, w.Hq, w.Hkv, w.d, w.max_blocks, partition_tokens=P), device)
-    fused = not args.two_calls
+    fused = not two_calls
     # decode kernel, plus the partition combine unless the split contexts
     # are merged inside thread-block clusters (the library decides)
     kernels_per_decode = pkv.decode_launches(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=kv_dt,
@@ -488,37 +571,35 @@ def run_ours(args):
         decode(c, outs[k % ncopies])
 
     stream = torch.cuda.current_stream(device)
-    Wu = max(3, args.warmup)
     for k in range(max(Wu, ncopies)):
         step(k)
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise SystemExit(f"device error flag {int(err.item()):#x} during warm-up")
 
-    def timed(K, body):
+    def timed(K_, body):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         barrier(world, device)
         torch.cuda.synchronize()
         e0.record(stream)
-        for k in range(K):
+        for k in range(K_):
             body(k)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world, device)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / K
+        return e0.elapsed_time(e1) / K_
 
     # The timed steps are replays of CUDA graphs that captured S consecutive
-    # steps (steps 0..S-1, one per copy when there are copies), launches and
-    # programmatic dependencies as the library issues them: the host's
-    # per-call marshalling (tens of microseconds in Python) then does not set
-    # the pace of a step whose kernels take a few microseconds, and the next
-    # step's decode launches while the current one ends, as consecutive
-    # layers would.  K = q S + r steps are q replays of the S-step graph and
-    # one of an r-step graph.
-    K = args.steps
-    S = ncopies if ncopies > 1 else min(K, 16)
+    # steps (one per copy when there are copies), launches and programmatic
+    # dependencies as the library issues them: the host's per-call
+    # marshalling (tens of microseconds in Python) then does not set the pace
+    # of a step whose kernels take a few microseconds, and the next step's
+    # decode launches while the current one ends, as consecutive layers
+    # would.  K = q S + r steps are q replays of the S-step graph and one of
+    # an r-step graph; both are replayed once before the timed region.
+    warm_order, timed_order = replay_order(K, S)
 
     def capture(body, n):
         g = torch.cuda.CUDAGraph()
@@ -528,28 +609,26 @@ def run_ours(args):
         return g
 
     def graphs_for(body):
-        full = capture(body, S)
-        tail = capture(body, K % S) if K % S else None
+        gs = {n: capture(body, n) for n in set(warm_order + timed_order)}
         torch.cuda.synchronize()
-        return full, tail
+        return gs
 
-    def replay(gt):
+    def warm(gs):
+        for n in warm_order:
+            gs[n].replay()
+        torch.cuda.synchronize()
+
+    def replay(gs):
         def run(_):
-            for _ in range(K // S):
-                gt[0].replay()
-            if gt[1] is not None:
-                gt[1].replay()
+            for n in timed_order:
+                gs[n].replay()
         return run
 
     step_g = graphs_for(step)
     decode_g = step_g if fused else graphs_for(lambda k: decode(copies[k % ncopies],
                                                                 outs[k % ncopies]))
-    for _ in range(max(1, -(-Wu // S))):
-        step_g[0].replay()
-    torch.cuda.synchronize()
 
-    # kv_append alone (not part of the roofline claim): the same graphs-of-S
-    # scheme over the copies
+    # kv_append alone (not part of the roofline claim): the same graph scheme
     def append_only(k):
         c = copies[k % ncopies]
         if e4m3:
@@ -560,15 +639,21 @@ def run_ours(args):
 
     append_g = graphs_for(append_only)
 
+    warm(step_g)
     with ClockSampler(local) as clocks:
         step_ms = timed(1, replay(step_g)) / K
+    decode_ms = step_ms
+    if not fused:
         # the decode call alone (the same call as the step when it is fused)
-        decode_ms = step_ms if fused else timed(1, replay(decode_g)) / K
+        warm(decode_g)
+        decode_ms = timed(1, replay(decode_g)) / K
+    warm(append_g)
     append_ms = max_over_ranks(timed(1, replay(append_g)) / K, world, device)
     step_ms_max = max_over_ranks(step_ms, world, device)
     decode_ms_max = max_over_ranks(decode_ms, world, device)
     if int(err.item()) != 0:
         raise SystemExit(f"device error flag {int(err.item()):#x} during timing")
+    del step_g, decode_g, append_g
 
     value = world * nbytes / (step_ms_max * 1e-3) / 1e9
     peak, peak_src = load_peak()
@@ -651,45 +736,47 @@ def run_ours(args):
                "d2h_bytes_per_step": d2h}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        wc = W.make_config(args.config, device="cpu") if args.config in (1, 2, 3) else None
-        if wc is None:
-            # big workloads: the oracle reads a bounded subset copied from the device
-            wc = w
+    if sample is not None:
+        sub, frac = sample
         nthreads = os.cpu_count() or 1
-        if e4m3 and wc is not w:
-            k8c, v8c, _, _ = W.e4m3_cache(wc)
-            wc.k_cache, wc.v_cache = k8c, v8c
-        per_step, seqs, frac, reps = time_oracle(wc, args.cpu_seconds, nthreads,
-                                                 (ks8, vs8) if e4m3 else None, args.window)
+        scales = (ks8, vs8) if e4m3 else None
+        if e4m3:
+            # the sample's pages as 8-bit codes, cast the same way as the device cache
+            from paged_kv_cache_484_b200.workloads import Workload  # noqa: F401
+            k_c, v_c = sub.k_cache.float(), sub.v_cache.float()
+            sub.k_cache = (k_c / ks8).to(torch.float8_e4m3fn).view(torch.uint8)
+            sub.v_cache = (v_c / vs8).to(torch.float8_e4m3fn).view(torch.uint8) \
+                .transpose(2, 3).contiguous()
+        per_step, reps = time_oracle(sub, args.cpu_seconds, nthreads, scales, args.window)
         # the same oracle on one thread, briefly (reported beside the all-cores figure)
-        per1, seqs1, frac1, reps1 = time_oracle(wc, min(2.0, args.cpu_seconds), 1,
-                                                (ks8, vs8) if e4m3 else None, args.window)
+        per1, reps1 = time_oracle(sub, min(2.0, args.cpu_seconds), 1, scales, args.window)
         cpu = {"value": round(nbytes * frac / per_step / 1e9, 4), "unit": "GB/s",
                "cores": nthreads, "kind": "oracle",
-               "value_1_thread": round(nbytes * frac1 / per1 / 1e9, 4),
-               "sample": f"{len(seqs)} of {w.B} sequences, full append+decode step in fp64, "
-                         f"{reps} repetitions ({per_step * 1e3:.1f} ms each)"}
+               "value_1_thread": round(nbytes * frac / per1 / 1e9, 4),
+               "sample": f"sequences 0..{len(sub.seqs) - 1} ({len(sub.seqs)} of {w.B}, "
+                         f"{100 * frac:.1f} % of the step's K/V), one fp64 append + decode "
+                         f"pass each, {reps} repetitions ({per_step * 1e3:.1f} ms each)"}
 
-    line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
-        "steps": K, "warmup": max(3, args.warmup), "ms_per_step": round(step_ms_max, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3" if e4m3 else ("bf16" if w.dtype == torch.bfloat16 else "f32"),
-        "data": "synthetic",
+    block = dict(config_block(cfg, w, out_dtype, P, NP, args.simt, two_calls),
+                 **({"sliding_window": args.window} if args.window else {}),
+                 **({"step": "two calls (kv_append, paged_attention_decode_cascade over "
+                             "the prefix groups)"} if cascade else {}),
+                 l2=(f"inputs larger than L2 ({l2 >> 20} MiB): " +
+                     (f"{ncopies} device-side copies of the per-layer tensors (q, new rows, "
+                      f"K/V caches; the step's block tables, context lengths, positions "
+                      f"and slots shared, as by the layers of a model); every timed step "
+                      f"reads a copy that no step of the previous 2 x L2 bytes touched "
+                      f"({nbytes / 1e6:.1f} MB read per step)" if ncopies > 1 else
+                      f"the workload reads {nbytes / 1e6:.1f} MB per step") +
+                     "; no flush inside the timed region"))
+    traffic_key = (f"{cfg}_e4m3" if e4m3 else str(cfg)) if args.num_seqs is None else None
+    res = {
+        "value": round(value, 3), "unit": "GB/s", "steps": K, "warmup": Wu,
+        "ms_per_step": round(step_ms_max, 5),
         "pct_of_hbm_peak": round(100.0 * value / (world * peak), 2),
         "seq_steps_per_s": round(world * w.B / (step_ms_max * 1e-3), 1),
-        "config": dict(config_block(args.config, w, out_dtype, P, NP, args.simt, args.two_calls),
-                       **({"sliding_window": args.window} if args.window else {}),
-                       **({"step": "two calls (kv_append, paged_attention_decode_cascade over "
-                                   "the prefix groups)"} if cascade else {}),
-                       l2=(f"inputs larger than L2 ({l2 >> 20} MiB): " +
-                           (f"{ncopies} device-side copies of the per-layer tensors (q, new rows, "
-                            f"K/V caches; the step's block tables, context lengths, positions "
-                            f"and slots shared, as by the layers of a model), step k on copy k "
-                            f"mod {ncopies} ({nbytes / 1e6:.1f} MB read per step)" if ncopies > 1 else
-                            f"the workload reads {nbytes / 1e6:.1f} MB per step") +
-                           "; no flush inside the timed region")),
+        "dtype": "e4m3" if e4m3 else ("bf16" if w.dtype == torch.bfloat16 else "f32"),
+        "config": block,
         "isolated_step": {"ms_per_step": round(iso_ms, 5),
                           "value": round(world * nbytes / (iso_ms * 1e-3) / 1e9, 3),
                           "ms_median": round(iso_each[len(iso_each) // 2], 5),
@@ -707,12 +794,54 @@ def run_ours(args):
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "decode_ms": round(decode_ms_max, 5),
-                     "traffic": recorded_traffic(f"{args.config}_e4m3" if e4m3 else args.config)},
+                     "algorithmic_bytes": nbytes,
+                     "traffic": recorded_traffic(traffic_key) if traffic_key else None},
         "gpu_launches": K * launches_per_step,
         "kv_append_us_per_call": round(append_ms * 1e3, 3),
         "clocks": clocks.summary(),
         "e2e": e2e,
         "cpu_baseline": cpu,
+    }
+    del copies, outs, w, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, local)
+
+    import paged_kv_cache_484_b200 as pkv
+    pkv.load_library()
+    cfg = args.config or HEADLINE_CONFIG
+    head = measure(cfg, args, device, world, local, rank, full=True)
+    per_config = None
+    if args.config is None and not args.no_secondary:
+        per_config = {}
+        for c in SECONDARY_CONFIGS:
+            r = measure(c, args, device, world, local, rank, full=False)
+            per_config[r["config"]["workload"]] = {
+                k: r[k] for k in ("value", "unit", "ms_per_step", "pct_of_hbm_peak",
+                                  "seq_steps_per_s", "steps", "warmup", "roofline", "clocks",
+                                  "isolated_step", "gpu_launches", "kv_append_us_per_call",
+                                  "config")}
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world,
+        "steps": head["steps"], "warmup": head["warmup"], "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": head["dtype"], "data": "synthetic",
+        "pct_of_hbm_peak": head["pct_of_hbm_peak"], "seq_steps_per_s": head["seq_steps_per_s"],
+        "config": head["config"], "isolated_step": head["isolated_step"],
+        "roofline": head["roofline"],
+        "gpu_launches": head["gpu_launches"] + sum(
+            r["gpu_launches"] for r in (per_config or {}).values()),
+        "kv_append_us_per_call": head["kv_append_us_per_call"],
+        "clocks": head["clocks"], "e2e": head["e2e"], "cpu_baseline": head["cpu_baseline"],
+        **({"per_config": per_config} if per_config is not None else {}),
         "device": torch.cuda.get_device_name(device),
         "versions": software_versions(),
     }
@@ -740,13 +869,14 @@ def run_prefill(args):
     from paged_kv_cache_484_b200 import workloads as W
 
     pkv.load_library()
-    w = W.make_config(args.config, device=device)
+    cfg = args.config or 3
+    w = W.make_config(cfg, device=device, num_seqs=args.num_seqs)
     if w.dtype != torch.bfloat16:
         raise SystemExit("prefill: bf16 workloads only")
     C = args.prefill
     lens = w.cached_lens.clamp(min=C).to(torch.int32)
     g = torch.Generator(device=device)
-    g.manual_seed(484 + args.config)
+    g.manual_seed(484 + cfg)
     q = torch.randn((w.B, C, w.Hq, w.d), generator=g, device=device, dtype=torch.bfloat16)
     out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
     P = args.partition_tokens or pkv.prefill_partition_tokens(w.B, C, w.Hq, w.Hkv, w.d,
@@ -762,7 +892,8 @@ def run_prefill(args):
         read = read.clamp(max=C - 1 + args.window)
     nbytes = int(read.sum().item()) * w.Hkv * w.d * 2 * 2 + w.B * C * w.Hq * w.d * (2 + esz_out)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    ncopies = args.copies or (1 if nbytes >= 2 * l2 else min(1024, math.ceil(2 * l2 / nbytes)))
+    K = args.steps
+    ncopies, S = copies_plan(nbytes, l2, K, args.copies)
     # per-layer q and caches copied; the block tables and lengths shared
     copies = [dict(q=q, k=w.k_cache, v=w.v_cache, t=w.block_tables, l=lens)]
     for _ in range(ncopies - 1):
@@ -780,8 +911,6 @@ def run_prefill(args):
     for k in range(max(3, args.warmup, ncopies)):
         call(k)
     torch.cuda.synchronize()
-    K = args.steps
-    S = ncopies if ncopies > 1 else min(K, 16)
 
     def capture(n):
         gr = torch.cuda.CUDAGraph()
@@ -790,9 +919,10 @@ def run_prefill(args):
                 call(k)
         return gr
 
-    full = capture(S)
-    tail = capture(K % S) if K % S else None
-    full.replay()
+    warm_order, timed_order = replay_order(K, S)
+    graphs = {n: capture(n) for n in set(warm_order + timed_order)}
+    for n in warm_order:
+        graphs[n].replay()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -800,10 +930,8 @@ def run_prefill(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         e0.record(stream)
-        for _ in range(K // S):
-            full.replay()
-        if tail is not None:
-            tail.replay()
+        for n in timed_order:
+            graphs[n].replay()
         e1.record(stream)
         torch.cuda.synchronize()
     barrier(world, device)
@@ -819,7 +947,7 @@ def run_prefill(args):
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "query_tokens_per_s": round(world * w.B * C / (ms * 1e-3), 1),
-        "config": {"workload": W.CONFIG_NAMES[args.config] + f"_prefill_chunk{C}",
+        "config": {"workload": w.name + f"_prefill_chunk{C}",
                    "batch_seqs": w.B, "chunk_tokens": C, "q_heads": w.Hq, "kv_heads": w.Hkv,
                    **({"sliding_window": args.window} if args.window else {}),
                    "head_dim": w.d, "partition_tokens": P,

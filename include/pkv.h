@@ -91,7 +91,9 @@ typedef enum pkv_status {
     PKV_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape */
     PKV_ERR_UNSUPPORTED = 2, /* valid, but outside the supported set above */
     PKV_ERR_WORKSPACE = 3,   /* workspace smaller than required */
-    PKV_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+    PKV_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    PKV_ERR_DEVICE = 5       /* pkv_get_device_error: the kernels reported a bad
+                                device-resident value or a wait that ran out */
 } pkv_status;
 
 typedef enum pkv_dtype {
@@ -648,6 +650,47 @@ int64_t pkv_kv_request_bytes(int64_t num_layers, int64_t num_kv_heads, int64_t h
 int64_t pkv_kv_admission_capacity(int64_t pool_bytes, int64_t num_layers, int64_t num_kv_heads,
                                   int64_t head_dim, int64_t block_size, int64_t tokens,
                                   int32_t kv_dtype);
+
+/*
+ * pkv_get_device_error -- wait for a stream and read the device error word.
+ *
+ * Source: "Inference From Scratch", ch. 10 (block tables: every id a kernel
+ * reads comes from the table, so a bad entry must be reported, not followed).
+ *
+ * Waits until all work enqueued on `stream` so far has finished (a
+ * cudaStreamSynchronize: call it between steps, not inside a captured
+ * graph), then copies the word at `device_error` (the int32 device word the
+ * kernels OR their PKV_DEVERR_* bits into) to *code_out.  The word is left as
+ * it is; the caller clears it (e.g. cudaMemsetAsync) when it wants a fresh
+ * one.
+ *
+ * Arguments
+ *   device_error  int32 device word (required).
+ *   stream        cudaStream_t the kernels ran on (NULL = legacy default).
+ *   code_out      HOST int32, receives the word.
+ * Returns PKV_OK when the word is 0, PKV_ERR_DEVICE when it is not (the bits
+ * are in *code_out and named by pkv_last_error), PKV_ERR_INVALID_ARG for a
+ * null pointer, PKV_ERR_CUDA when the copy or the synchronisation fails
+ * (e.g. a fault of earlier work on the stream).
+ */
+pkv_status pkv_get_device_error(const int32_t* device_error, void* stream, int32_t* code_out);
+
+/*
+ * pkv_selftest_bounded_wait -- run the kernels' bounded wait until it gives up.
+ *
+ * A diagnostic with no counterpart in the pages.  Every in-kernel wait of
+ * this library (the page pipeline's shared-memory barriers) gives up after a
+ * bounded time, sets PKV_DEVERR_TIMEOUT and lets the kernel return, so a
+ * stalled copy can never hang a GPU.  This launches one warp that waits, with
+ * that same code, on a barrier nothing ever completes, for `limit_us`
+ * microseconds (1 .. 2 000 000), then ORs PKV_DEVERR_TIMEOUT into
+ * *device_error and, if `waited_ns` is not NULL, stores the waited time
+ * (int64 device word, nanoseconds).  Asynchronous on `stream`.
+ * Returns PKV_ERR_INVALID_ARG for a limit outside the range or a null
+ * device_error, PKV_ERR_CUDA if the launch fails.
+ */
+pkv_status pkv_selftest_bounded_wait(uint32_t limit_us, int32_t* device_error,
+                                     uint64_t* waited_ns, void* stream);
 
 /* Short text for a status code (static storage). */
 const char* pkv_status_string(int32_t status);

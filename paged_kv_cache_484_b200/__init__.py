@@ -31,6 +31,9 @@ from ._binding import (  # noqa: F401
     prepare_decode_step,
     PreparedCall,
     decode_workspace_size,
+    get_device_error,
+    selftest_bounded_wait,
+    PKV_ERR_DEVICE,
     kv_admission_capacity,
     kv_append,
     kv_append_e4m3,

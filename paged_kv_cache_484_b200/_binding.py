@@ -7,6 +7,7 @@ is missing the call raises -- there is no fallback path.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -132,6 +133,10 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_last_error.restype = ctypes.c_char_p
         lib.pkv_version.argtypes = []
         lib.pkv_version.restype = i32
+        lib.pkv_get_device_error.argtypes = [vp, vp, vp]
+        lib.pkv_get_device_error.restype = ctypes.c_int
+        lib.pkv_selftest_bounded_wait.argtypes = [u32, vp, vp, vp]
+        lib.pkv_selftest_bounded_wait.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -174,6 +179,21 @@ def _dev(t: torch.Tensor, name: str, dtype=None, on=None) -> int:
     return t.data_ptr()
 
 
+@contextlib.contextmanager
+def _current(dv: torch.device):
+    """Makes the call's device (that of q) the current CUDA device for one
+    library call: the library plans a launch from the current device's SM
+    count and shared-memory limit, and the allocation-free decode looks up
+    its built-in scratch on the current device, while the kernels run on the
+    stream of the call's device."""
+    if dv.type == "cuda" and torch.cuda.is_available() and \
+            torch.cuda.current_device() != dv.index:
+        with torch.cuda.device(dv):
+            yield
+    else:
+        yield
+
+
 def _flags(force_simt: bool, cluster: bool) -> int:
     return (PKV_DECODE_FORCE_SIMT if force_simt else 0) | (0 if cluster else PKV_DECODE_NO_CLUSTER)
 
@@ -207,12 +227,13 @@ def kv_append(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_t
         raise ValueError("inconsistent kv_append shapes")
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
-    st = lib.pkv_kv_append(
-        _dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
-        _dev(positions, "positions", torch.int64, on=dv),
-        _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
-        _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
-        T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), err, _stream_ptr(stream, q.device))
+    with _current(dv):
+        st = lib.pkv_kv_append(
+            _dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
+            _dev(positions, "positions", torch.int64, on=dv),
+            _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
+            _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+            T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "kv_append")
 
 
@@ -299,9 +320,11 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
             B, Hq, Hkv, d, NB, bs, MB, kv_dt, out_dt, float(scale)]
     tail = [int(partition_tokens), _flags(force_simt, cluster), err, _stream_ptr(stream, q.device)]
     if sliding_window:
-        st = lib.pkv_paged_attention_decode_window(*args, int(sliding_window), *tail)
+        with _current(dv):
+            st = lib.pkv_paged_attention_decode_window(*args, int(sliding_window), *tail)
     else:
-        st = lib.pkv_paged_attention_decode(*args, *tail)
+        with _current(dv):
+            st = lib.pkv_paged_attention_decode(*args, *tail)
     _raise(st, lib, "paged_attention_decode")
     return out
 
@@ -327,13 +350,14 @@ def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, r
         raise ValueError("inconsistent kv_append_e4m3 shapes")
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
-    st = lib.pkv_kv_append_e4m3(
-        _dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
-        _dev(positions, "positions", torch.int64, on=dv),
-        _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
-        _dev(k_cache, "k_cache", torch.uint8, on=dv), _dev(v_cache, "v_cache", torch.uint8, on=dv),
-        T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), float(k_scale), float(v_scale), err,
-        _stream_ptr(stream, q.device))
+    with _current(dv):
+        st = lib.pkv_kv_append_e4m3(
+            _dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
+            _dev(positions, "positions", torch.int64, on=dv),
+            _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
+            _dev(k_cache, "k_cache", torch.uint8, on=dv), _dev(v_cache, "v_cache", torch.uint8, on=dv),
+            T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), float(k_scale), float(v_scale), err,
+            _stream_ptr(stream, q.device))
     _raise(st, lib, "kv_append_e4m3")
 
 
@@ -359,15 +383,16 @@ def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens,
         workspace = new_workspace(int(need), q.device)
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
-    st = lib.pkv_paged_attention_decode_e4m3(
-        _dev(q, "q", torch.bfloat16, on=dv), _dev(k_cache, "k_cache", torch.uint8, on=dv),
-        _dev(v_cache, "v_cache", torch.uint8, on=dv),
-        _dev(block_tables, "block_tables", torch.int32, on=dv),
-        _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
-        _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
-        B, Hq, Hkv, d, NB, bs, MB, _dtype_code(out.dtype), float(scale), float(k_scale),
-        float(v_scale), int(sliding_window), int(partition_tokens), _flags(False, cluster), err,
-        _stream_ptr(stream, q.device))
+    with _current(dv):
+        st = lib.pkv_paged_attention_decode_e4m3(
+            _dev(q, "q", torch.bfloat16, on=dv), _dev(k_cache, "k_cache", torch.uint8, on=dv),
+            _dev(v_cache, "v_cache", torch.uint8, on=dv),
+            _dev(block_tables, "block_tables", torch.int32, on=dv),
+            _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+            _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
+            B, Hq, Hkv, d, NB, bs, MB, _dtype_code(out.dtype), float(scale), float(k_scale),
+            float(v_scale), int(sliding_window), int(partition_tokens), _flags(False, cluster), err,
+            _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode_e4m3")
     return out
 
@@ -425,7 +450,9 @@ def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, bloc
                                      block_tables, context_lens, rope_theta, scale, out, stream,
                                      workspace, partition_tokens, force_simt, device_error,
                                      cluster)
-    _raise(lib.pkv_decode_step(*args), lib, "decode_step")
+    with _current(q.device):
+        st = lib.pkv_decode_step(*args)
+    _raise(st, lib, "decode_step")
     return out
 
 
@@ -435,17 +462,22 @@ class PreparedCall:
     it was prepared with must stay alive and keep their shapes, dtypes and
     addresses (their contents may change between calls)."""
 
-    __slots__ = ("_lib", "_fn", "_args", "_name", "_keep")
+    __slots__ = ("_lib", "_fn", "_args", "_name", "_keep", "_dev")
 
-    def __init__(self, lib, fn, args, name, keep):
+    def __init__(self, lib, fn, args, name, keep, device=None):
         self._lib, self._fn, self._name, self._keep = lib, fn, name, keep
+        self._dev = device
         types = fn.argtypes
         # ctypes instances, so that a call converts nothing
         self._args = tuple(t(a) if a is not None or t is not ctypes.c_void_p else t()
                            for t, a in zip(types, args))
 
     def __call__(self) -> None:
-        st = self._fn(*self._args)
+        if self._dev is not None:
+            with _current(self._dev):
+                st = self._fn(*self._args)
+        else:
+            st = self._fn(*self._args)
         if st != 0:
             _raise(st, self._lib, self._name)
 
@@ -461,7 +493,7 @@ def prepare_decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cac
                                         v_cache, block_tables, context_lens, rope_theta, scale,
                                         out, stream, workspace, partition_tokens, force_simt,
                                         device_error, cluster)
-    return PreparedCall(lib, lib.pkv_decode_step, args, "decode_step", keep)
+    return PreparedCall(lib, lib.pkv_decode_step, args, "decode_step", keep, q.device)
 
 
 def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, out,
@@ -488,15 +520,49 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
         raise ValueError("inconsistent paged_attention_decode_noalloc shapes")
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
-    st = lib.pkv_paged_attention_decode_noalloc(
-        _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
-        _dev(block_tables, "block_tables", torch.int32, on=dv),
-        _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
-        B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(scale),
-        int(partition_tokens), _flags(force_simt, cluster), err,
-        _stream_ptr(stream, q.device))
+    with _current(dv):
+        st = lib.pkv_paged_attention_decode_noalloc(
+            _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+            _dev(block_tables, "block_tables", torch.int32, on=dv),
+            _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+            B, Hq, Hkv, d, NB, bs, MB, kv_dt, _dtype_code(out.dtype), float(scale),
+            int(partition_tokens), _flags(force_simt, cluster), err,
+            _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode_noalloc")
     return out
+
+
+PKV_ERR_DEVICE = 5
+
+
+def get_device_error(device_error, stream=None) -> int:
+    """Wait for ``stream`` (default: the current stream of the word's device)
+    and return the device error word (PKV_DEVERR_* bits; 0 = none).
+    See include/pkv.h, pkv_get_device_error."""
+    lib = load_library()
+    dv = device_error.device
+    code = ctypes.c_int32(0)
+    with _current(dv):
+        st = lib.pkv_get_device_error(_dev(device_error, "device_error", torch.int32),
+                                      _stream_ptr(stream, dv), ctypes.byref(code))
+    if st not in (0, PKV_ERR_DEVICE):
+        _raise(st, lib, "get_device_error")
+    return int(code.value)
+
+
+def selftest_bounded_wait(limit_us, device_error, waited_ns=None, stream=None) -> None:
+    """Run the kernels' bounded wait on a barrier nothing completes, for
+    ``limit_us`` microseconds; it then sets DEVERR_TIMEOUT in ``device_error``
+    and returns.  ``waited_ns``: optional int64 device tensor of one element,
+    receives the waited time.  See include/pkv.h, pkv_selftest_bounded_wait."""
+    lib = load_library()
+    dv = device_error.device
+    wn = _dev(waited_ns, "waited_ns", torch.int64, on=dv) if waited_ns is not None else None
+    with _current(dv):
+        st = lib.pkv_selftest_bounded_wait(int(limit_us),
+                                           _dev(device_error, "device_error", torch.int32),
+                                           wn, _stream_ptr(stream, dv))
+    _raise(st, lib, "selftest_bounded_wait")
 
 
 def version() -> int:
@@ -547,13 +613,14 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, sca
         workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
-    st = lib.pkv_paged_attention_prefill(
-        _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
-        _dev(block_tables, "block_tables", torch.int32, on=dv),
-        _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
-        _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
-        B, C, Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16, _dtype_code(out.dtype), float(scale),
-        int(sliding_window), int(partition_tokens), err, _stream_ptr(stream, q.device))
+    with _current(dv):
+        st = lib.pkv_paged_attention_prefill(
+            _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+            _dev(block_tables, "block_tables", torch.int32, on=dv),
+            _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+            _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
+            B, C, Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16, _dtype_code(out.dtype), float(scale),
+            int(sliding_window), int(partition_tokens), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_prefill")
     return out
 
@@ -596,16 +663,17 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_le
         workspace = new_workspace(int(need), q.device)
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
-    st = lib.pkv_paged_attention_decode_cascade(
-        _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
-        _dev(block_tables, "block_tables", torch.int32, on=dv),
-        _dev(context_lens, "context_lens", torch.int32, on=dv),
-        _dev(group_start, "group_start", torch.int32, on=dv) if NG else None,
-        _dev(shared_tokens, "shared_tokens", torch.int32, on=dv), _dev(out, "out", on=dv),
-        _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
-        B, NG, int(max_group_size), Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16,
-        _dtype_code(out.dtype), float(scale), int(partition_tokens),
-        _flags(force_simt, True), err, _stream_ptr(stream, q.device))
+    with _current(dv):
+        st = lib.pkv_paged_attention_decode_cascade(
+            _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+            _dev(block_tables, "block_tables", torch.int32, on=dv),
+            _dev(context_lens, "context_lens", torch.int32, on=dv),
+            _dev(group_start, "group_start", torch.int32, on=dv) if NG else None,
+            _dev(shared_tokens, "shared_tokens", torch.int32, on=dv), _dev(out, "out", on=dv),
+            _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
+            B, NG, int(max_group_size), Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16,
+            _dtype_code(out.dtype), float(scale), int(partition_tokens),
+            _flags(force_simt, True), err, _stream_ptr(stream, q.device))
     _raise(st, lib, "paged_attention_decode_cascade")
     return out
 

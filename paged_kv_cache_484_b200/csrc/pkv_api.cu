@@ -996,6 +996,7 @@ const char* pkv_status_string(int32_t status) {
         case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
         case PKV_ERR_WORKSPACE: return "workspace too small";
         case PKV_ERR_CUDA: return "CUDA error";
+        case PKV_ERR_DEVICE: return "device error word set by a kernel";
     }
     return "unknown status";
 }

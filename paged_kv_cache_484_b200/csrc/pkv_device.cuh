@@ -79,8 +79,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 // Wait for the phase with the given parity to complete; false if the wait ran
-// out (kWaitLimitNs).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// out (`limit_ns` after the first timer read, taken once the first 256 polls
+// have failed).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t deadline = 0;
     for (uint32_t i = 1;; ++i) {
@@ -88,11 +89,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         if ((i & 255u) == 0) {
             uint64_t now = global_timer_ns();
             if (deadline == 0)
-                deadline = now + kWaitLimitNs;
+                deadline = now + limit_ns;
             else if (now > deadline)
                 return false;
         }
     }
+}
+// The wait every pipeline stage uses: bounded by kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // ---- TMA / bulk copies (no multicast anywhere in this library) ------------

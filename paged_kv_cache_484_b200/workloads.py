@@ -173,10 +173,15 @@ def _uniform_int(g, lo, hi, n):
     return torch.randint(lo, hi + 1, (n,), generator=g, dtype=torch.int64)
 
 
-def make_config(cfg: int, device="cpu") -> Workload:
-    """Workload ``cfg`` (1..5), seeded with 484 + cfg."""
+def make_config(cfg: int, device="cpu", num_seqs: int | None = None) -> Workload:
+    """Workload ``cfg`` (1..5), seeded with 484 + cfg.  ``num_seqs`` keeps only
+    the first that many sequences (the same lengths and layout rules on a
+    smaller batch, e.g. for a profiler capture that must stay small); the
+    pool and values are then drawn for that batch."""
     seed = 484 + cfg
     name = CONFIG_NAMES[cfg]
+    if num_seqs is not None:
+        return _truncated(cfg, device, int(num_seqs))
     if cfg == 1:
         # 1 sequence, 4/4 heads, d 64, 256 cached tokens in a 64-block pool, fp32
         return build_workload(name, [256], 4, 4, 64, torch.float32, 1e4, seed, device,
@@ -201,6 +206,30 @@ def make_config(cfg: int, device="cpu") -> Workload:
         return build_workload(name, [131072] * 16, 32, 8, 128, torch.bfloat16, 5e5, seed,
                               device, hot_key_frac=0.01, hot_key_scale=8.0)
     raise ValueError(f"unknown config {cfg}")
+
+
+def _truncated(cfg: int, device, n: int) -> Workload:
+    full = {1: ([256], dict(pool_blocks=64)), 2: ([2048], dict(pool_blocks=4096))}
+    seed = 484 + cfg
+    if cfg in full:
+        lens, kw = full[cfg]
+        lens = lens[:n]
+    elif cfg == 3:
+        lens, kw = _uniform_int(_gen("cpu", seed + 1), 128, 4096, 64)[:n], dict(pool_factor=1.25)
+    elif cfg == 4:
+        g = _gen("cpu", seed + 1)
+        u = torch.rand(256, generator=g, dtype=torch.float64)
+        lens = torch.floor(torch.exp(math.log(16) + u * (math.log(32768) - math.log(16))))
+        lens = lens.clamp(16, 32768).to(torch.int64)[:n]
+        kw = dict(pool_factor=1.0, prefix_group=8, prefix_tokens=1024)
+    elif cfg == 5:
+        lens, kw = [131072] * min(n, 16), dict(hot_key_frac=0.01, hot_key_scale=8.0)
+    else:
+        raise ValueError(f"unknown config {cfg}")
+    shape = {1: (4, 4, 64, torch.float32, 1e4)}.get(
+        cfg, (32, 8, 128 if cfg == 5 else 64, torch.bfloat16, 5e5))
+    name = f"{CONFIG_NAMES[cfg]}_first{len(lens)}seqs"
+    return build_workload(name, lens, *shape, seed, device, **kw)
 
 
 def config_summary(cfg: int) -> dict:

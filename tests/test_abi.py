@@ -364,3 +364,16 @@ def test_noalloc_rejects_before_touching_the_device(lib, kw, status):
         a["NB"], a["bs"], a["MB"], a["kvdt"], a["odt"], a["scale"], a["P"], a["flags"], a["err"],
         None)
     assert st == status
+
+
+def test_device_error_reader_and_wait_selftest_reject_bad_arguments(lib):
+    """Both diagnostics refuse their bad arguments on the host (no copy, no
+    launch): null pointers, and a self-test limit outside 1 us .. 2 s."""
+    code = ctypes.c_int32(7)
+    assert lib.pkv_get_device_error(None, None, ctypes.byref(code)) == INVALID
+    assert lib.pkv_get_device_error(FAKE, None, None) == INVALID
+    assert code.value == 7
+    assert lib.pkv_selftest_bounded_wait(0, FAKE, None, None) == INVALID
+    assert lib.pkv_selftest_bounded_wait(2_000_001, FAKE, None, None) == INVALID
+    assert lib.pkv_selftest_bounded_wait(1000, None, None, None) == INVALID
+    assert lib.pkv_status_string(5) == b"device error word set by a kernel"

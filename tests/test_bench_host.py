@@ -45,3 +45,47 @@ def test_peak_falls_back_when_no_measured_file(tmp_path, monkeypatch):
     assert bench.load_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6539.5}))
     assert bench.load_peak() == (6539.5, "measured")
+
+
+def _timed_reuse_distance(nbytes, l2, K, warmup):
+    """Replays the bench's warm-up and timed schedule as a list of the copies
+    each step touches; returns, for every timed step, the bytes other steps
+    moved since its copy was last touched (None: first touch)."""
+    n, S = bench.copies_plan(nbytes, l2, K)
+    warm_order, timed_order = bench.replay_order(K, S)
+    uses = [k % n for k in range(max(warmup, n))]            # eager warm-up steps
+    for length in warm_order:
+        uses += [k % n for k in range(length)]
+    t0 = len(uses)
+    for length in timed_order:
+        uses += [k % n for k in range(length)]
+    assert len(uses) - t0 == K                                # exactly K timed steps
+    last, dist = {}, []
+    for i, c in enumerate(uses):
+        if i >= t0:
+            dist.append(None if c not in last else (i - last[c] - 1) * nbytes)
+        last[c] = i
+    return n, S, warm_order, timed_order, dist
+
+
+def test_timed_steps_never_reread_what_l2_holds():
+    """Every timed step reads a copy that at least 2 x L2 bytes of other steps
+    have passed over since it was last used, for short and long timed regions
+    (the driver's --steps 20 included) and small and large workloads."""
+    l2 = 126 << 20
+    for nbytes in (524_800, 4_202_496, 60 << 20, 283_000_000, 8_590_000_000):
+        for K in (1, 3, 20, 50, 64, 65, 200, 2000):
+            n, S, warm, timed, dist = _timed_reuse_distance(nbytes, l2, K, 5)
+            if n == 1:
+                assert nbytes >= 2 * l2
+                continue
+            assert all(d is not None and d >= 2 * l2 for d in dist), (nbytes, K, n, dist[:4])
+
+
+def test_every_timed_graph_is_replayed_before_the_timed_region():
+    for K in (1, 4, 16, 20, 33, 2000):
+        for S in (1, 7, 16, 64, 83):
+            warm, timed = bench.replay_order(K, S)
+            assert sum(timed) == K
+            assert set(timed) <= set(warm)
+            assert warm[-1] == S          # the full graph runs last, over the highest copies

@@ -3,6 +3,9 @@ oracle's plain decode, through the C ABI (GPU only).
 
 The cascade call must give the plain decode's result: the oracle decodes
 every sequence over its own block table, with no knowledge of the groups.
+The oracle's inputs are host copies taken before any GPU call, and the
+oracle performs its own append (RoPE on q and k, the new rows written into
+their slots): no value the CUDA path produced reaches it.
 Bar: max-abs error <= 2e-3 (bf16 inputs, fp32 output).
 """
 from __future__ import annotations
@@ -10,10 +13,9 @@ from __future__ import annotations
 import pytest
 import torch
 
-import oracle
 import paged_kv_cache_484_b200 as pkv
 from paged_kv_cache_484_b200 import workloads as W
-from tests.parity_util import TOL_BF16
+from tests.parity_util import TOL_BF16, SubProblem
 
 pytestmark = pytest.mark.gpu
 
@@ -24,6 +26,8 @@ def _grouped(lens, group, prefix_tokens, G, Hkv, d, seed):
     w = W.build_workload("cascade", lens, G * Hkv, Hkv, d, torch.bfloat16, 1e4, seed=seed,
                          device=DEV, pool_factor=1.2, prefix_group=group,
                          prefix_tokens=prefix_tokens)
+    # the oracle's inputs, copied before the CUDA path touches anything
+    sub = SubProblem(w, range(w.B))
     # rotate q and append the new token the usual way (two calls)
     pkv.kv_append(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
                   w.rope_theta)
@@ -32,13 +36,12 @@ def _grouped(lens, group, prefix_tokens, G, Hkv, d, seed):
     group_start = torch.tensor(starts, dtype=torch.int32, device=DEV)
     cached = w.cached_lens.to(torch.int64)
     shared = torch.minimum(cached // 16, torch.full_like(cached, prefix_tokens // 16)) * 16
-    return w, group_start, shared.to(torch.int32), group
+    return w, sub, group_start, shared.to(torch.int32), group
 
 
-def _oracle(w):
-    return oracle.paged_attention_decode(w.q.cpu(), w.k_cache.cpu(), w.v_cache.cpu(),
-                                         w.block_tables.cpu(), w.decode_lens.cpu(), w.scale,
-                                         nthreads=8)
+def _oracle(sub):
+    """The oracle's own append then plain decode, on the pristine copies."""
+    return sub.oracle_step(nthreads=8)[3]
 
 
 def _check(got, want, what):
@@ -61,11 +64,11 @@ def _run(w, group_start, shared, max_group, P=0, err=None):
                                          (128, 4, 4, 256), (64, 1, 16, 0), (64, 4, 16, 512)])
 def test_cascade_matches_plain_decode(d, G, group, P):
     lens = [1500, 300, 40, 255, 2000, 256, 16, 700, 1024, 77, 900, 260, 2047, 511, 5, 3000]
-    w, gs, shared, group = _grouped(lens, group, 512, G, 2, d, seed=400 + d + G + group)
+    w, sub, gs, shared, group = _grouped(lens, group, 512, G, 2, d, seed=400 + d + G + group)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
     out = _run(w, gs, shared, group, P=P, err=err)
     assert int(err.item()) == 0
-    _check(out, _oracle(w), f"cascade d{d} G{G} group{group} P{P}")
+    _check(out, _oracle(sub), f"cascade d{d} G{G} group{group} P{P}")
     # and the same numbers as the plain decode call, up to rounding
     plain = torch.empty_like(out)
     pkv.paged_attention_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
@@ -80,18 +83,20 @@ def test_cascade_edge_cases():
     context (all-zero row), and a member whose shared block id differs from
     its group's (flagged)."""
     lens = [512, 700, 512, 100, 900, 30, 640, 640]
-    w, gs, shared, _ = _grouped(lens, 4, 512, 4, 2, 64, seed=431)
-    # context 512 of the first sequence is exactly its shared prefix after
-    # the append? its decode length is 513: make it exactly the shared part
+    w, sub, gs, shared, _ = _grouped(lens, 4, 512, 4, 2, 64, seed=431)
+    # the first sequence's decode length is 513 after the append: make its
+    # context exactly the shared part (the oracle's copy likewise)
     w.decode_lens[0] = 512
+    sub.decode_lens[0] = 512
     # group layout: [0, 4) and [4, 6); sequences 6 and 7 in no group
     gs = torch.tensor([0, 4, 5, 6], dtype=torch.int32, device=DEV)   # group of one: [4, 5)
     shared[6:] = 0
     shared[5] = 0                       # in a group, nothing shared
     w.decode_lens[7] = 0                # empty context
+    sub.decode_lens[7] = 0
     out = _run(w, gs, shared, 4)
-    want = _oracle(w)
-    want[7].zero_()
+    want = _oracle(sub)
+    assert not want[7].any()            # the oracle's empty context is a zero row too
     _check(out, want, "cascade edge cases")
     assert not out[7].any()
     # a member whose shared block differs from the group's: flagged
@@ -102,7 +107,7 @@ def test_cascade_edge_cases():
 
 
 def test_cascade_workspace_counters_return_to_zero():
-    w, gs, shared, group = _grouped([800, 600, 1200, 300] * 2, 4, 256, 4, 8, 64, seed=433)
+    w, sub, gs, shared, group = _grouped([800, 600, 1200, 300] * 2, 4, 256, 4, 8, 64, seed=433)
     need = pkv.decode_cascade_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks)
     ws = pkv.new_workspace(need, DEV)
     outs = []
@@ -115,4 +120,4 @@ def test_cascade_workspace_counters_return_to_zero():
         assert not ws[:pkv.SCHED_BYTES].any()
         outs.append(out)
     assert torch.equal(outs[0], outs[1])
-    _check(outs[0], _oracle(w), "cascade, reused workspace")
+    _check(outs[0], _oracle(sub), "cascade, reused workspace")
