@@ -206,10 +206,10 @@ def recorded_traffic(cfg):
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_source_hash") != kernel_source_hash():
-        return None
     ent = rec.get("configs", {}).get(str(cfg))
-    return None if ent is None else ent.get("bytes_per_launch")
+    if ent is None or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
 
 
 class ClockSampler:

@@ -16,9 +16,9 @@ import bench  # noqa: E402
 
 def test_recorded_traffic_is_tied_to_the_kernel_sources(monkeypatch):
     rec = json.load(open(os.path.join(ROOT, "profiles", "decode_dram_traffic.json")))
-    h = rec["kernel_source_hash"]
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: h)
     for key, ent in rec["configs"].items():
+        h = ent["kernel_source_hash"]
+        monkeypatch.setattr(bench, "kernel_source_hash", lambda: h)
         assert bench.recorded_traffic(key) == ent["bytes_per_launch"]
     assert bench.recorded_traffic("no such workload") is None
     # a capture taken on other sources is not reported
