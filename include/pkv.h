@@ -307,6 +307,31 @@ pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new,
                            int32_t partition_tokens, uint32_t flags, int32_t* device_error,
                            void* stream);
 
+/*
+ * pkv_decode_step_window -- pkv_decode_step with a sliding window.
+ *
+ * Source: "Efficient LLM Inference", KV Caching: positions and windows.
+ *
+ * The same single launch as pkv_decode_step (the new token appended inside
+ * the decode kernel), but each query attends only to the last
+ * `sliding_window` tokens of its context, its own new token included, as in
+ * pkv_paged_attention_decode_window: pages wholly before the window are
+ * never read, and keys before it in its first page are masked.
+ * sliding_window = 0 is no window (the call is then pkv_decode_step);
+ * negative values return PKV_ERR_INVALID_ARG.  Every other argument,
+ * precondition and error is pkv_decode_step's.
+ */
+pkv_status pkv_decode_step_window(void* q, const void* k_new, const void* v_new,
+                                  const int64_t* positions, const int64_t* slot_mapping,
+                                  void* k_cache, void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, void* out, void* workspace,
+                                  size_t workspace_bytes, int64_t num_seqs, int64_t num_q_heads,
+                                  int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                                  int64_t block_size, int64_t max_blocks_per_seq,
+                                  int32_t kv_dtype, int32_t out_dtype, double rope_theta,
+                                  float scale, int32_t sliding_window, int32_t partition_tokens,
+                                  uint32_t flags, int32_t* device_error, void* stream);
+
 /* Bytes of the built-in scratch behind pkv_paged_attention_decode_noalloc.
  * Every GPU that loads the library holds this much device memory until the
  * process exits. */

@@ -72,6 +72,11 @@ def load_library() -> ctypes.CDLL:
                                         i32, i32, ctypes.c_double, ctypes.c_float, i32, u32,
                                         vp, vp]
         lib.pkv_decode_step.restype = ctypes.c_int
+        lib.pkv_decode_step_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                               ctypes.c_size_t, i64, i64, i64, i64, i64, i64,
+                                               i64, i32, i32, ctypes.c_double, ctypes.c_float,
+                                               i32, i32, u32, vp, vp]
+        lib.pkv_decode_step_window.restype = ctypes.c_int
         lib.pkv_paged_attention_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp,
                                                            i64, i64, i64, i64, i64, i64, i64,
                                                            i32, i32, ctypes.c_float, i32, u32,
@@ -439,19 +444,24 @@ def _decode_step_args(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache
 def decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, block_tables,
                 context_lens, rope_theta, scale, out, stream=None, *, workspace=None,
                 partition_tokens=0, force_simt=False, device_error=None,
-                cluster=True) -> torch.Tensor:
+                cluster=True, sliding_window=0) -> torch.Tensor:
     """``kv_append`` (one new token per sequence) then ``paged_attention_decode``,
     in one launch.  The new token must be the last token of its context
     (context_lens[b] - 1, at the slot block_tables gives it).  q is read only:
-    the rotated q is used inside the kernel and not stored.  See include/pkv.h,
-    pkv_decode_step.
+    the rotated q is used inside the kernel and not stored.  ``sliding_window``
+    > 0: each query attends to the last ``sliding_window`` tokens of its context
+    (pkv_decode_step_window).  See include/pkv.h, pkv_decode_step.
     """
     lib, args, _ = _decode_step_args(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache,
                                      block_tables, context_lens, rope_theta, scale, out, stream,
                                      workspace, partition_tokens, force_simt, device_error,
                                      cluster)
     with _current(q.device):
-        st = lib.pkv_decode_step(*args)
+        if sliding_window:
+            # pkv_decode_step_window takes the window just before partition_tokens
+            st = lib.pkv_decode_step_window(*args[:-4], int(sliding_window), *args[-4:])
+        else:
+            st = lib.pkv_decode_step(*args)
     _raise(st, lib, "decode_step")
     return out
 

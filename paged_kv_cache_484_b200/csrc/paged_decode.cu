@@ -125,14 +125,16 @@ struct Layout {
     static constexpr int OFF_ROPE = OFF_NEWKV + STAGES * NEWKV_BYTES;
     static constexpr int OFF_MERGE = OFF_ROPE + STAGES * ROPE_BYTES;
     static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
-    static constexpr int OFF_MASK = OFF_BAR + (3 * STAGES + 1) * 8;  // full, empty, q, merge
+    // full, empty, q per stage; merge; rank (the longest-first order is ready)
+    static constexpr int OFF_MASK = OFF_BAR + (3 * STAGES + 2) * 8;
     // Cluster mode: every CTA of a cluster stores its merged partial (o[D], m,
     // l per head) into slot `rank` of a landing area in rank 0's shared memory,
     // past everything else (rank 0 may still be computing when they land).
     static constexpr int CLUSTER_PART_BYTES = G * (D + 2) * 4;
     static constexpr int OFF_PATCH = OFF_MASK + STAGES * 4;  // fused: (row, block) of the new token
     static constexpr int OFF_ITEM = OFF_PATCH + STAGES * 8;  // work item of each stage, -1: no more
-    static constexpr int OFF_MISC = OFF_ITEM + STAGES * 4;   // abort flag + 8 scan slots
+    // abort flag, per-warp counts of non-empty contexts, 8 scan slots
+    static constexpr int OFF_MISC = OFF_ITEM + STAGES * 4;
     // s_len[B], s_pre[B + 1]; with at most kLptMaxSeqs sequences also
     // s_rank[B], s_key[B] (the longest-first order of last partitions)
     static constexpr int OFF_SEQ = OFF_MISC + 16 * 4;
@@ -408,10 +410,24 @@ template <typename T, int D, int G, bool FUSED>
 __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& guess,
                              const CUtensorMap* tmk, const CUtensorMap* tmv, uint8_t* base,
                              uint64_t* full, uint64_t* empty, uint64_t* qbar, uint32_t* masks,
-                             volatile int* s_abort, const int* s_len, const int* s_pre, int W) {
+                             volatile int* s_abort, const int* s_len, const int* s_pre, int W,
+                             uint64_t* rank_bar, bool lpt) {
     using L = Layout<T, D, G>;
     const int lane = threadIdx.x & 31;
     int* s_item = reinterpret_cast<int*>(base + L::OFF_ITEM);
+    // The longest-first order of the last partitions is ranked by the
+    // consumer warps while this warp streams the full partitions, which come
+    // first; before the first item that needs the order this warp waits for
+    // it (false: the wait ran out).
+    bool ranked = !lpt;
+    const int nfull = s_pre[p.B];
+    auto ensure_ranked = [&](int i) -> bool {
+        if (ranked || i / p.Hkv < nfull) return true;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(rank_bar, 0);
+        ranked = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        return ranked;
+    };
 
     // Work order of this CTA: items blockIdx.x and blockIdx.x + gridDim.x,
     // then items claimed one at a time from the counter (2 gridDim.x + its
@@ -472,6 +488,10 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
     // qbar: per stage, the parity of its next phase and whether a q copy was issued
     uint32_t q_parity = 0, q_issued = 0;
     bool abort = false;
+    if (item < W && !ensure_ranked(item)) {
+        abort = true;
+        item = W;
+    }
     if (item < W) {
     if (item1 < W) issue_claim();
     Item cur = decode_item(item, p, s_len, s_pre);
@@ -493,7 +513,14 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
         if (nc0 >= cur.npages) {
             nitem = item1;
             nc0 = 0;
-            if (nitem < W) nxt = decode_item(nitem, p, s_len, s_pre);
+            if (nitem < W) {
+                if (ensure_ranked(nitem)) {
+                    nxt = decode_item(nitem, p, s_len, s_pre);
+                } else {
+                    nitem = W;
+                    abort = true;
+                }
+            }
         }
         const int nxt_raw = (nitem < W) ? raw_entry(nxt, nc0 + lane) : kNoPage;
         const bool new_item = FUSED && nitem != item && nitem < W;
@@ -1379,6 +1406,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     // pages are still in flight
     uint64_t* qbar = empty + L::STAGES;
     uint64_t* merge_bar = qbar + L::STAGES;
+    uint64_t* rank_bar = merge_bar + 1;
     uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
     int* misc = reinterpret_cast<int*>(base + L::OFF_MISC);
     volatile int* s_abort = misc;
@@ -1394,6 +1422,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
             mbar_init(&qbar[s], 1);
         }
         mbar_init(merge_bar, NW * 32);
+        mbar_init(rank_bar, NW * 32);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -1456,7 +1485,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
     const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
     int* s_rank = s_pre + B + 1;
     int* s_key = s_rank + B;
-    int local = 0;
+    int local = 0, local_ne = 0;
     for (int b = b0; b < b1; ++b) {
         int Lb = p.context_lens[b];
         if (Lb < 0 || Lb > maxlen) {
@@ -1476,6 +1505,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         if (lpt) s_key[b] = Lb > 0 ? (Lb - off) - (npb - 1) * p.P : -1;  // tokens of the last partition
         s_pre[b] = cnt;
         local += cnt;
+        local_ne += Lb > 0;
     }
     int incl = local;
 #pragma unroll
@@ -1484,6 +1514,10 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         if (lane >= off) incl += v;
     }
     if (lane == 31) s_warp_tot[warp] = incl;
+    {
+        const int ne_w = __reduce_add_sync(0xffffffffu, local_ne);
+        if (lane == 0) misc[1 + warp] = ne_w;
+    }
     __syncthreads();
     int run = incl - local;
     for (int w = 0; w < warp; ++w) run += s_warp_tot[w];
@@ -1493,35 +1527,39 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         run += cnt;
     }
     if (tid == kDecodeThreads - 1) s_pre[B] = run;
-    if (lpt) {
-        // rank of each last partition: longer first, then by sequence
-        // (every CTA derives the same order)
-        for (int b = b0; b < b1; ++b) {
-            const int k = s_key[b];
-            if (k < 0) continue;
-            int rank = 0;
-            for (int b2 = 0; b2 < B; ++b2) {
-                const int k2 = s_key[b2];
-                rank += (k2 > k) || (k2 == k && b2 < b);
-            }
-            s_rank[rank] = b;
-        }
-        if (tid == 0) {
-            int ne = 0;
-            for (int b2 = 0; b2 < B; ++b2) ne += s_key[b2] >= 0;
-            s_warp_tot[7] = ne;
-        }
-    }
+    int ne = 0;  // contexts with tokens: one last partition each
+    for (int w = 0; w <= NW; ++w) ne += misc[1 + w];
     __syncthreads();
-    const int W = (s_pre[B] + (lpt ? s_warp_tot[7] : 0)) * p.Hkv;
+    const int W = (s_pre[B] + (lpt ? ne : 0)) * p.Hkv;
 
     // In cluster mode no thread leaves before the cluster merge below.
     if (warp == NW) {
         run_producer<T, D, G, FUSED>(p, guess, &tm_k, &tm_v, base, full, empty, qbar, masks,
-                                     s_abort,
-                                     s_len, s_pre, W);
+                                     s_abort, s_len, s_pre, W, rank_bar, lpt);
         if (!p.cluster) return;
     } else {
+        if (lpt) {
+            // rank of each last partition: longer first, then by sequence
+            // (every CTA derives the same order); the producer is already
+            // streaming the full partitions, which come first
+            const int cper = (B + NW * 32 - 1) / (NW * 32);
+            const int c0 = min(B, tid * cper), c1 = min(B, c0 + cper);
+            for (int b = c0; b < c1; ++b) {
+                const int k = s_key[b];
+                if (k < 0) continue;
+                int rank = 0;
+                for (int b2 = 0; b2 < B; ++b2) {
+                    const int k2 = s_key[b2];
+                    rank += (k2 > k) || (k2 == k && b2 < b);
+                }
+                s_rank[rank] = b;
+            }
+            mbar_arrive(rank_bar);
+            if (!mbar_wait(rank_bar, 0)) {
+                *s_abort = 1;
+                report_error(p.err, PKV_DEVERR_TIMEOUT);
+            }
+        }
         // zero the output of empty contexts (spread over the CTAs); in the
         // fused step their new token is still appended
         for (int b = blockIdx.x; b < B; b += gridDim.x) {

@@ -12,21 +12,22 @@
 // with its own context length, which is how the tests check it.
 //
 // Work decomposition.  A work item is (sequence, kv head, row group,
-// partition of P keys).  Its rows are up to 32 (query, head) pairs of the kv
-// head, (query i, head g) -> row i*G + g; each of the four consumer warps
-// owns 8 rows and runs them over every page of the partition, so a K/V page
-// is read once per row group.  One CTA per item (no persistence: the items
-// of a prefill chunk are uniform).  Partitions are merged by a log-sum-exp
-// combine kernel when a sequence has more than one.
+// partition of P keys).  Its rows are up to 128 (query, head) pairs of the kv
+// head, (query i, head g) -> row i*G + g, one tile of a 5th-generation
+// tensor-core MMA, so a K/V page is read once per row group.  One CTA per
+// item, one CTA per SM.  Partitions are merged by a log-sum-exp combine kernel
+// when a sequence has more than one.  The cascade decode's shared-prefix pass
+// (the end of this file) runs its items through the same tile routine.
 //
-// Inside a CTA: one producer warp turns block-table entries into TMA loads of
-// whole K and V pages (128-byte swizzle) into a ring of stages guarded by
-// mbarriers; the consumer warps compute S = Q K^T and O += P V with
-// mma.sync m16n8k16 (bf16 in, fp32 accumulate).  A warp's 16-row A tile
-// holds its 8 rows twice: rows r carry the high bf16 part of P, rows r + 8
-// the low part (p = hi + lo to ~2^-17 relative).  Each row masks the keys
-// past its own position; a row can have no key in a page or a partition
-// (its softmax state then stays m = -inf, l = 0).  Every wait is bounded.
+// Inside a CTA (umma_attend): one producer warp turns block-table entries
+// into TMA loads of whole K and V pages (128-byte swizzle) into a ring of
+// 64-key stages guarded by mbarriers; one lane issues tcgen05 MMAs, S = Q K^T
+// and O += P V, with the accumulators in tensor memory; two softmax
+// warpgroups (one thread per row each) take alternate tiles.  P is split
+// into a high and a low bf16 part (p = hi + lo to ~2^-17 relative).  Each row
+// masks the keys past its own position; a row can have no key in a tile or a
+// partition (its softmax state then stays m = -inf, l = 0).  Every wait is
+// bounded.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -41,23 +42,7 @@ namespace pkv {
 namespace {
 
 using bf16 = __nv_bfloat16;
-constexpr int NWP = 4;                        // consumer warps
-constexpr int kRowsPerWarp = 8;               // (query, head) rows per warp
-constexpr int kThreadsP = (NWP + 1) * 32;     // + one producer warp
 constexpr float kNegInfP = -__builtin_huge_valf();
-
-template <int D>
-struct PLayout {
-    static constexpr int PAGE_BYTES = kPageRows * D * 2;
-    static constexpr int BOXES = D / 64;            // 64-column TMA boxes per page
-    static constexpr int BOX_BYTES = PAGE_BYTES / BOXES;
-    static constexpr int SP = 4;                    // pages per stage
-    static constexpr int STAGE_BYTES = 2 * SP * PAGE_BYTES;  // SP K pages, then SP V pages
-    static constexpr int STAGES = D == 64 ? 4 : 3;  // 64 KiB / 96 KiB of ring
-    static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-    static constexpr int OFF_MASK = OFF_BAR + 2 * STAGES * 8;  // full, empty
-    static constexpr size_t SMEM = 1024 + OFF_MASK + STAGES * 4 + 16;
-};
 
 struct PrefillParams {
     const bf16* q;              // [B, C, Hq, D]
@@ -72,16 +57,6 @@ struct PrefillParams {
     int out_bf16;
     int window;                 // sliding window: query at position t sees t - window + 1 .. t
 };
-
-// Byte offset of 16-byte chunk c of token row tok in a 128-byte-swizzled page.
-template <int D>
-__device__ __forceinline__ uint32_t pchunk(int tok, int c) {
-    if constexpr (D == 64) {
-        return tok * 128 + ((c ^ (tok & 7)) << 4);
-    } else {
-        return (c >> 3) * 2048 + tok * 128 + (((c & 7) ^ (tok & 7)) << 4);
-    }
-}
 
 __device__ __forceinline__ void pstore(void* out, size_t idx, float v, int out_bf16) {
     if (out_bf16)
@@ -125,304 +100,6 @@ __device__ __forceinline__ PItem prefill_item(const PrefillParams& p) {
     return it;
 }
 
-template <int D>
-__device__ void prefill_producer(const PrefillParams& p, const PItem& it, const CUtensorMap* tmk,
-                                 const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
-                                 uint64_t* empty, uint32_t* masks, volatile int* s_abort) {
-    using L = PLayout<D>;
-    const int lane = threadIdx.x & 31;
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued_parity[8];
-    uint32_t issued_any = 0;
-    bool abort = false;
-    // block-table entries of the next 32-page chunk are loaded while this one
-    // is issued, and range-checked when their chunk comes up
-    const int32_t* row_tab = p.block_tables + (size_t)it.b * p.MB + it.t0 / kPageRows;
-    int raw = lane < it.npages ? row_tab[lane] : -1;
-    for (int c0 = 0; c0 < it.npages && !abort; c0 += 32) {
-        int ent = -1;
-        if (c0 + lane < it.npages) {
-            if (raw < 0 || raw >= p.num_blocks)
-                report_error(p.err, PKV_DEVERR_BLOCK_ID);
-            else
-                ent = raw;
-        }
-        raw = c0 + 32 + lane < it.npages ? row_tab[c0 + 32 + lane] : -1;
-        const int cend = min(it.npages, c0 + 32);
-        for (int s0 = c0; s0 < cend; s0 += L::SP) {
-            const int npg = min(L::SP, it.npages - s0);
-            const int k = lane - (s0 - c0);
-            const bool mine = k >= 0 && k < npg && ent >= 0;
-            const uint32_t vmask = __ballot_sync(0xffffffffu, mine) >> (s0 - c0);
-            int ok = 1;
-            if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1) && !*s_abort;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) {
-                abort = true;
-                break;
-            }
-            if (lane == 0) {
-                masks[stage] = vmask;
-                mbar_arrive_expect_tx(&full[stage], __popc(vmask) * 2u * L::PAGE_BYTES);
-            }
-            __syncwarp();
-            if (mine) {
-                uint8_t* kdst = base + stage * L::STAGE_BYTES + k * L::PAGE_BYTES;
-                uint8_t* vdst = kdst + L::SP * L::PAGE_BYTES;
-                const int row0 = (ent * p.Hkv + it.h) * kPageRows;
-#pragma unroll
-                for (int bx = 0; bx < L::BOXES; ++bx) {
-                    tma_load_2d(kdst + bx * L::BOX_BYTES, tmk, bx * 64, row0, &full[stage]);
-                    tma_load_2d(vdst + bx * L::BOX_BYTES, tmv, bx * 64, row0, &full[stage]);
-                }
-            }
-            issued_parity[stage] = phase;
-            issued_any |= 1u << stage;
-            if (++stage == L::STAGES) {
-                stage = 0;
-                phase ^= 1;
-            }
-        }
-    }
-    if (abort) {
-        *s_abort = 1;
-        if (lane == 0) {
-            report_error(p.err, PKV_DEVERR_TIMEOUT);
-            for (int s = 0; s < L::STAGES; ++s)
-                if (issued_any & (1u << s)) (void)mbar_wait(&full[s], issued_parity[s]);
-        }
-        __syncwarp();
-    }
-}
-
-// One query row of a consumer lane (lanes 4r .. 4r+3 of a warp share row r).
-struct PRow {
-    bool ok;            // the row exists
-    const bf16* q;      // its query vector (D elements)
-    int len;            // it may attend to tokens t < len
-    int lo;             // and t >= lo (sliding window; 0 otherwise)
-    bool direct;        // write the output row (else a partition partial)
-    void* out;          // direct: the output row (D elements of out_bf16 ? bf16 : f32)
-    float* po;          // partial: o (D floats)
-    float* pml;         // partial: (m, l)
-};
-
-// A consumer warp runs its 8 rows over every page of the item's key range
-// [t0, t1): S = Q K^T and O += P V on the tensor cores, online softmax per
-// row in the log2 domain, keys at t >= row.len masked per row.
-template <int D>
-__device__ void multirow_consumer(float scale_log2, int out_bf16, int32_t* err, const PItem& it,
-                                  const PRow& row, uint8_t* base, uint64_t* full, uint64_t* empty,
-                                  const uint32_t* masks, volatile int* s_abort) {
-    using L = PLayout<D>;
-    constexpr int KS = D / 16, NT = D / 8;
-    const int lane = threadIdx.x & 31;
-    const int cq = lane & 3;
-    const bool row_ok = row.ok;
-    const int row_len = row_ok ? row.len : 0;
-    const int row_lo = row.lo;
-
-    // A fragments of Q: rows r and r + 8 both hold this lane's row
-    uint32_t qa[KS][2];
-    {
-        const uint32_t* qr = reinterpret_cast<const uint32_t*>(row.q);
-#pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-            const int col = kk * 16 + 2 * cq;
-            qa[kk][0] = row_ok ? qr[col / 2] : 0u;
-            qa[kk][1] = row_ok ? qr[(col + 8) / 2] : 0u;
-        }
-    }
-    float o[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m_run = kNegInfP, l_run = 0.f;
-
-    int stage = 0;
-    uint32_t phase = 0;
-    const int mi = lane >> 3, ri = lane & 7;
-    const int nst = (it.npages + L::SP - 1) / L::SP;
-    bool ok = true;
-    for (int s = 0; s < nst; ++s) {
-        ok = mbar_wait(&full[stage], phase) && !*s_abort;
-        if (!ok) break;
-        const uint32_t msk = masks[stage];
-        for (int u = 0; u < L::SP; ++u) {
-            const int j = s * L::SP + u;
-            if (j >= it.npages || !((msk >> u) & 1u)) continue;
-            const int tbase = it.t0 + j * kPageRows;       // absolute token of page row 0
-            const int in_part = min(kPageRows, it.t1 - tbase);   // rows inside the partition
-            const int row_valid = max(0, min(in_part, row_len - tbase));
-            const int row_first = max(0, row_lo - tbase);   // sliding window
-            const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + u * L::PAGE_BYTES);
-            const uint32_t vbase = kbase + L::SP * L::PAGE_BYTES;
-            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                const int tok = ri + ((mi >> 1) << 3);
-                const int ch = 2 * kk + (mi & 1);
-                uint32_t b00, b01, b10, b11;
-                ldsm_x4(kbase + pchunk<D>(tok, ch), b00, b01, b10, b11);
-                const uint32_t a[4] = {qa[kk][0], qa[kk][0], qa[kk][1], qa[kk][1]};
-                mma_bf16_16816(sc[0], a, b00, b01);
-                mma_bf16_16816(sc[1], a, b10, b11);
-            }
-            float x[2][2];
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int tk = n * 8 + 2 * cq + e;
-                    x[n][e] = (tk < row_valid && tk >= row_first) ? sc[n][e] * scale_log2
-                                                                  : kNegInfP;
-                }
-            float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run, mx);
-            // a row with no key so far keeps m = -inf: use 0 as the reference
-            const float m_ref = m_new == kNegInfP ? 0.f : m_new;
-            const float alpha = fast_exp2(m_run - m_ref);
-            float pr[2][2];
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) pr[n][e] = fast_exp2(x[n][e] - m_ref);
-            l_run = l_run * alpha + ((pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
-            if (__any_sync(0xffffffffu, m_new != m_run)) {
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    o[n][0] *= alpha;
-                    o[n][1] *= alpha;
-                    o[n][2] *= alpha;
-                    o[n][3] *= alpha;
-                }
-            }
-            m_run = m_new;
-            // P: rows r the high bf16 part, rows r + 8 the low part
-            uint32_t pa[4];
-            {
-                const uint32_t hi0 = pack_bf16(pr[0][0], pr[0][1]);
-                const uint32_t hi1 = pack_bf16(pr[1][0], pr[1][1]);
-                pa[0] = hi0;
-                pa[1] = pack_bf16(pr[0][0] - bf16lo(hi0), pr[0][1] - bf16hi(hi0));
-                pa[2] = hi1;
-                pa[3] = pack_bf16(pr[1][0] - bf16lo(hi1), pr[1][1] - bf16hi(hi1));
-            }
-            // V rows past the partition may hold stale shared memory, and rows
-            // before every query's window are not attended: zero them
-            uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
-            const int v_first = max(0, it.lo - tbase);
-            if (in_part < kPageRows || v_first > 0) {
-                const int k0 = 2 * cq;
-                auto in = [&](int k) { return k >= v_first && k < in_part; };
-                vmask_lo = (in(k0) ? 0x0000ffffu : 0u) | (in(k0 + 1) ? 0xffff0000u : 0u);
-                vmask_hi = (in(k0 + 8) ? 0x0000ffffu : 0u) | (in(k0 + 9) ? 0xffff0000u : 0u);
-            }
-#pragma unroll
-            for (int c = 0; c < NT; c += 2) {
-                const int tok = ri + ((mi & 1) << 3);
-                const int ch = c + (mi >> 1);
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_trans(vbase + pchunk<D>(tok, ch), v0, v1, v2, v3);
-                mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
-                mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
-        if (++stage == L::STAGES) {
-            stage = 0;
-            phase ^= 1;
-        }
-    }
-    if (!ok) {
-        *s_abort = 1;
-        if (lane == 0) report_error(err, PKV_DEVERR_TIMEOUT);
-        return;
-    }
-    // row result: high + low rows, row sum over the quad
-    float lsum = l_run;
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-    if (!row_ok) return;
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    if (row.direct) {
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int col = n * 8 + 2 * cq;
-            pstore(row.out, col, (o[n][0] + o[n][2]) * inv, out_bf16);
-            pstore(row.out, col + 1, (o[n][1] + o[n][3]) * inv, out_bf16);
-        }
-    } else {
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int col = n * 8 + 2 * cq;
-            *reinterpret_cast<float2*>(row.po + col) =
-                make_float2((o[n][0] + o[n][2]) * inv, (o[n][1] + o[n][3]) * inv);
-        }
-        if (cq == 0) {
-            row.pml[0] = m_run;
-            row.pml[1] = lsum;
-        }
-    }
-}
-
-template <int D, int G>
-__global__ void __launch_bounds__(kThreadsP)
-    paged_prefill_kernel(const __grid_constant__ PrefillParams p,
-                         const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v) {
-    using L = PLayout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_addr(smem_raw);
-    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
-    uint64_t* empty = full + L::STAGES;
-    uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(masks + L::STAGES);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    if (tid == 0) {
-        for (int s = 0; s < L::STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NWP);
-        }
-        *s_abort = 0;
-        fence_barrier_init();
-    }
-    if (warp == NWP && (tid & 31) == 0) {
-        prefetch_tensor_map(&tm_k);
-        prefetch_tensor_map(&tm_v);
-    }
-    grid_dependency_wait();
-    grid_launch_dependents();
-    const PItem it = prefill_item(p);
-    __syncthreads();
-    if (it.part >= it.np) return;  // no keys in this partition (whole CTA leaves)
-    if (warp == NWP) {
-        prefill_producer<D>(p, it, &tm_k, &tm_v, base, full, empty, masks, s_abort);
-        return;
-    }
-    // this lane's row: (query i, head g) of the item's row group; query i
-    // sees tokens 0 .. L - C + i
-    PRow row;
-    const int fr = it.rg * (NWP * kRowsPerWarp) + warp * kRowsPerWarp + ((tid & 31) >> 2);
-    row.ok = fr < p.C * G;
-    const int qi = row.ok ? fr / G : 0, hq = it.h * G + (row.ok ? fr % G : 0);
-    const size_t r = ((size_t)it.b * p.C + qi) * p.Hq + hq;
-    row.q = p.q + r * D;
-    row.len = it.L - p.C + qi + 1;
-    row.lo = (p.window > 0 && row.len > p.window) ? row.len - p.window : 0;
-    row.direct = it.np == 1;
-    row.out = p.out_bf16 ? (void*)(reinterpret_cast<bf16*>(p.out) + r * D)
-                         : (void*)(reinterpret_cast<float*>(p.out) + r * D);
-    row.po = p.part_o ? p.part_o + (r * p.NP + it.part) * D : nullptr;
-    row.pml = p.part_ml ? p.part_ml + (r * p.NP + it.part) * 2 : nullptr;
-    multirow_consumer<D>(p.scale_log2, p.out_bf16, p.err, it, row, base, full, empty, masks,
-                         s_abort);
-}
-
 // out[b, i, h, :] from the partials of the sequence's partitions (the same
 // log-sum-exp merge as the decode's combine).  One warp per (b, i, h).
 template <int D>
@@ -459,6 +136,590 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const __grid_const
     for (int e = 0; e < PER; ++e) pstore(p.out, row * D + lane + 32 * e, acc[e] * inv, p.out_bf16);
 }
 
+// ---- attention tiles on the 5th-generation tensor cores ----------------------
+//
+// The chunked prefill (and the cascade's shared-prefix pass) run their items
+// through one routine, umma_attend: an item is up to 128 rows -- (query,
+// head) pairs of one kv head, the M of a tcgen05 MMA -- over a key range of
+// one sequence's pages, so a K/V page is read once per 128 rows.  Both
+// contractions run on the tensor cores with their accumulators in tensor
+// memory:
+//   S = Q K^T      (M = 128 rows, N = 64 keys, K = D), fp32
+//   O += P V       (M = 128 rows, N = D, K = 64 keys), fp32
+// P is split into a high and a low bf16 part (p = hi + lo to ~2^-17
+// relative) and both are multiplied into O, as on the warp-level path.
+//
+// Roles (320 threads):
+//   warp 0   producer: block-table entries -> TMA page loads into a ring of
+//            64-key stages; a stage's K pages are stored [64-column block]
+//            [page][16 rows][128 B] (V likewise), so that each 64-column
+//            block of the tile is one uniformly strided swizzled operand;
+//   warp 1   owns the tensor memory; one lane issues the MMAs;
+//   warps 2-5 and 6-9  two softmax warpgroups, one thread per row
+//            (tensor-memory lane).  Warpgroup w takes the tiles j with
+//            j % 2 = w, with its own score buffer S[w], P buffer P[w],
+//            accumulator O[w] and running (max, sum) per row, so the two
+//            overlap; at the end warpgroup 0 merges the two (max, sum, O)
+//            states of its row exactly (log-sum-exp) and stores the row.
+// A warpgroup's reference max only moves when the row max grew by more
+// than 2^8 (then its O row is rescaled in tensor memory): p <= 2^8, exact.
+// Signals: S_j -> sbar[j % 2]; S_j read into registers -> sfree[j % 2] (128
+// arrivals; S_{j+2} may then overwrite the buffer while the warpgroup is
+// still working on tile j); P_j written -> pready[j % 2] (128 arrivals);
+// O[j % 2] += P_j V_j done -> obar[j % 2]; the MMAs of tile j also release
+// its stage (empty).  The MMA lane polls both streams and issues whichever
+// MMA is ready first.  Every wait is bounded; a timeout sets
+// PKV_DEVERR_TIMEOUT and the CTA ends its work (the MMA lane waits for its
+// own MMAs before tensor memory is freed).
+constexpr int kURows = 128;                 // rows of an item: the MMA's M
+constexpr int kUTileKeys = 64;              // keys of one stage
+constexpr int kUTilePages = kUTileKeys / kPageRows;
+constexpr int kUThreads = 10 * 32;
+constexpr float kURescaleLog2 = 8.f;
+
+template <int D>
+struct ULayout {
+    static constexpr int BOX = kPageRows * 128;                 // 16 rows x 64 bf16 columns
+    static constexpr int NB = D / 64;                           // 64-column blocks of a row
+    static constexpr int BLOCK_STRIDE = kUTilePages * BOX;      // between column blocks of a tile
+    static constexpr int KV_BYTES = NB * BLOCK_STRIDE;          // one tile of K (or of V)
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;            // K tile, then V tile
+    static constexpr int STAGES = D == 64 ? 8 : 4;              // 128 KiB of ring
+    static constexpr int Q_BLOCK = kURows * 128;                // one column block of Q
+    static constexpr int P_BYTES = kURows * 128;                // 128 rows x 64 keys bf16
+    static constexpr int OFF_Q = STAGES * STAGE_BYTES;
+    static constexpr int OFF_P = OFF_Q + NB * Q_BLOCK;          // [warpgroup][hi, lo]
+    static constexpr int OFF_XCHG = OFF_P + 4 * P_BYTES;        // (max, sum) of warpgroup 1's rows
+    static constexpr int OFF_BAR = OFF_XCHG + kURows * 8;
+    // full[STAGES], empty[STAGES], sbar[2], sfree[2], pready[2], obar[2], mma_done, xchg, join
+    static constexpr int NBARS = 2 * STAGES + 11;
+    static constexpr int OFF_MASK = OFF_BAR + NBARS * 8;
+    static constexpr int OFF_MISC = OFF_MASK + STAGES * 4;      // abort flag, TMEM base
+    static constexpr size_t SMEM = 1024 + OFF_MISC + 16;
+    static constexpr uint32_t COL_S = 0;                        // + 64 * warpgroup
+    static constexpr uint32_t COL_O = 128;                      // + D * warpgroup
+    static constexpr uint32_t TMEM_COLS = COL_O + 2 * D <= 256 ? 256 : 512;
+    static constexpr uint32_t IDESC_S = umma_idesc_bf16(kURows, kUTileKeys, false);
+    static constexpr uint32_t IDESC_O = umma_idesc_bf16(kURows, D, true);
+};
+
+struct UItem {
+    int b;        // sequence whose block-table row lists the pages
+    int h;        // kv head
+    int t0, t1;   // the item's keys [t0, t1); t0 is page-aligned
+    int npages;   // pages from t0 on that cover [t0, t1)
+    int lo;       // no row reads a key before this one (V rows before it are zeroed)
+};
+
+struct URow {     // a softmax thread's row
+    bool ok;
+    const bf16* q;   // its query vector (D elements)
+    int len, lo;     // it attends keys lo <= t < len
+    void* out;       // the output row (D elements of out_bf16 ? bf16 : f32), or
+    float* po;       // with out == nullptr: a partial, o (D floats) and
+    float* pml;      // (max in log2 units, sum)
+};
+
+struct UArgs {
+    const int32_t* block_tables;
+    int32_t* err;
+    int MB, Hkv, num_blocks, out_bf16;
+    float scale_log2;
+};
+
+// Producer: the item's pages in 64-key stages (pages whose block id is out
+// of range are skipped and reported).
+template <int D>
+__device__ void umma_producer(const UArgs& a, const UItem& it, const CUtensorMap* tmk,
+                              const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
+                              uint64_t* empty, uint32_t* masks, volatile int* s_abort) {
+    using L = ULayout<D>;
+    const int lane = threadIdx.x & 31;
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_parity[L::STAGES];
+    uint32_t issued_any = 0;
+    bool abort = false;
+    const int32_t* row_tab = a.block_tables + (size_t)it.b * a.MB + it.t0 / kPageRows;
+    int raw = lane < it.npages ? row_tab[lane] : -1;
+    for (int c0 = 0; c0 < it.npages && !abort; c0 += 32) {
+        int ent = -1;
+        if (c0 + lane < it.npages) {
+            if (raw < 0 || raw >= a.num_blocks)
+                report_error(a.err, PKV_DEVERR_BLOCK_ID);
+            else
+                ent = raw;
+        }
+        raw = c0 + 32 + lane < it.npages ? row_tab[c0 + 32 + lane] : -1;
+        const int cend = min(it.npages, c0 + 32);
+        for (int s0 = c0; s0 < cend; s0 += kUTilePages) {
+            const int npg = min(kUTilePages, it.npages - s0);
+            const int k = lane - (s0 - c0);
+            const bool mine = k >= 0 && k < npg && ent >= 0;
+            const uint32_t vmask = __ballot_sync(0xffffffffu, mine) >> (s0 - c0);
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1) && !*s_abort;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                abort = true;
+                break;
+            }
+            if (lane == 0) {
+                masks[stage] = vmask;
+                mbar_arrive_expect_tx(&full[stage], __popc(vmask) * 2u * L::NB * L::BOX);
+            }
+            __syncwarp();
+            if (mine) {
+                uint8_t* kdst = base + stage * L::STAGE_BYTES + k * L::BOX;
+                uint8_t* vdst = kdst + L::KV_BYTES;
+                const int row0 = (ent * a.Hkv + it.h) * kPageRows;
+#pragma unroll
+                for (int bx = 0; bx < L::NB; ++bx) {
+                    tma_load_2d(kdst + bx * L::BLOCK_STRIDE, tmk, bx * 64, row0, &full[stage]);
+                    tma_load_2d(vdst + bx * L::BLOCK_STRIDE, tmv, bx * 64, row0, &full[stage]);
+                }
+            }
+            issued_parity[stage] = phase;
+            issued_any |= 1u << stage;
+            if (++stage == L::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+    }
+    if (abort) {
+        *s_abort = 1;
+        if (lane == 0) {
+            report_error(a.err, PKV_DEVERR_TIMEOUT);
+            for (int s = 0; s < L::STAGES; ++s)
+                if (issued_any & (1u << s)) (void)mbar_wait(&full[s], issued_parity[s]);
+        }
+        __syncwarp();
+    }
+}
+
+// The MMA lane.  Returns after its last MMA has completed (or it gave up).
+template <int D>
+__device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* full,
+                            uint64_t* empty, uint64_t* sbar, uint64_t* sfree, uint64_t* pready,
+                            uint64_t* obar, uint64_t* mma_done, volatile int* s_abort,
+                            int32_t* err) {
+    using L = ULayout<D>;
+    const uint32_t sq = smem_addr(base + L::OFF_Q);
+    auto issue_s = [&](int j) {
+        const int stage = j % L::STAGES;
+        const uint32_t sk = smem_addr(base + stage * L::STAGE_BYTES);
+        const uint32_t d = tmem + L::COL_S + 64u * (uint32_t)(j & 1);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+            const uint64_t da = umma_desc_sw128(sq + (s >> 2) * L::Q_BLOCK + (s & 3) * 32, 16, 1024);
+            const uint64_t db =
+                umma_desc_sw128(sk + (s >> 2) * L::BLOCK_STRIDE + (s & 3) * 32, 16, 1024);
+            umma_bf16(d, da, db, L::IDESC_S, s > 0);
+        }
+        umma_commit(&sbar[j & 1]);
+    };
+    auto issue_pv = [&](int j) {
+        const int w = j & 1;
+        const int stage = j % L::STAGES;
+        const uint32_t sv = smem_addr(base + stage * L::STAGE_BYTES + L::KV_BYTES);
+        const uint32_t sp = smem_addr(base + L::OFF_P + w * 2 * L::P_BYTES);
+        const uint32_t o = tmem + L::COL_O + (uint32_t)(w * D);
+#pragma unroll
+        for (int s = 0; s < kUTileKeys / 16; ++s) {
+            const uint64_t db = umma_desc_sw128(sv + s * 16 * 128, L::BLOCK_STRIDE, 1024);
+            const uint64_t hi = umma_desc_sw128(sp + s * 32, 16, 1024);
+            const uint64_t lo = umma_desc_sw128(sp + L::P_BYTES + s * 32, 16, 1024);
+            umma_bf16(o, hi, db, L::IDESC_O, j >= 2 || s > 0);
+            umma_bf16(o, lo, db, L::IDESC_O, true);
+        }
+        umma_commit(&obar[w]);
+        umma_commit(&empty[stage]);  // the stage's K and V are no longer read
+    };
+    // S_j needs its stage loaded and (j >= 2) the buffer's previous scores read;
+    // PV_j needs P_j.  Neither condition can run two phases ahead of this lane
+    // (the warpgroup's next arrivals wait for MMAs only this lane issues), so
+    // each wait is on an unambiguous parity.
+    int js = 0, jp = 0;
+    bool ok = true;
+    uint64_t since = 0;
+    uint32_t idle = 0;
+    while (jp < ntiles) {
+        bool progressed = false;
+        if (js < ntiles && (js < 2 || mbar_test_wait(&sfree[js & 1], (uint32_t)((js - 2) >> 1) & 1u)) &&
+            mbar_test_wait(&full[js % L::STAGES], (uint32_t)(js / L::STAGES) & 1u)) {
+            tc_fence_after();
+            issue_s(js);
+            ++js;
+            progressed = true;
+        }
+        if (jp < js && mbar_test_wait(&pready[jp & 1], (uint32_t)(jp >> 1) & 1u)) {
+            tc_fence_after();
+            issue_pv(jp);
+            ++jp;
+            progressed = true;
+        }
+        if (progressed) {
+            idle = 0;
+            since = 0;
+            continue;
+        }
+        // nothing ready: leave the issue slots of this sub-partition to the
+        // softmax warps that share it for a moment before polling again
+        __nanosleep(64);
+        if ((++idle & 255u) == 0) {
+            if (*s_abort) {
+                ok = false;
+                break;
+            }
+            const uint64_t now = global_timer_ns();
+            if (since == 0) {
+                since = now;
+            } else if (now - since > kWaitLimitNs) {
+                ok = false;
+                break;
+            }
+        }
+    }
+    if (!ok) {
+        *s_abort = 1;
+        report_error(err, PKV_DEVERR_TIMEOUT);
+    }
+    // every MMA this lane issued has completed before tensor memory is freed
+    umma_commit(mma_done);
+    (void)mbar_wait(mma_done, 0);
+}
+
+// One item, run by all kUThreads threads of the CTA (every thread calls it;
+// `row` matters to the softmax warps only).
+template <int D>
+__device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
+                            const CUtensorMap* tmk, const CUtensorMap* tmv, uint8_t* base) {
+    using L = ULayout<D>;
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
+    uint64_t* empty = full + L::STAGES;
+    uint64_t* sbar = empty + L::STAGES;
+    uint64_t* sfree = sbar + 2;
+    uint64_t* pready = sfree + 2;
+    uint64_t* obar = pready + 2;
+    uint64_t* mma_done = obar + 2;
+    uint64_t* xchg_bar = mma_done + 1;
+    uint64_t* join = xchg_bar + 1;
+    uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(base + L::OFF_MISC);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::OFF_MISC + 4);
+    float2* xchg = reinterpret_cast<float2*>(base + L::OFF_XCHG);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ntiles = (it.npages + kUTilePages - 1) / kUTilePages;
+    if (tid == 0) {
+        for (int s = 0; s < L::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sbar[i], 1);
+            mbar_init(&sfree[i], kURows);
+            mbar_init(&pready[i], kURows);
+            mbar_init(&obar[i], 1);
+        }
+        mbar_init(mma_done, 1);
+        mbar_init(xchg_bar, kURows);
+        mbar_init(join, 2 * kURows);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    const int r = 32 * (warp & 3) + lane;  // softmax threads: the row (tensor-memory lane)
+    const int wg = (warp - 2) >> 2;        // softmax threads: the warpgroup
+    if (warp >= 2) {
+        // warpgroup 0 puts the Q rows into the swizzled tile (zeros for rows
+        // past the item); the V halves of the ring start zeroed, so that a
+        // key no row may read never holds a non-finite value when P = 0
+        // multiplies it
+        if (wg == 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(row.q);
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                const uint4 v = row.ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t off = (c >> 3) * L::Q_BLOCK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                *reinterpret_cast<uint4*>(base + L::OFF_Q + off) = v;
+            }
+        }
+        for (int idx = tid - 64; idx < L::STAGES * L::KV_BYTES / 16; idx += 2 * kURows) {
+            const int st = idx / (L::KV_BYTES / 16), w = idx % (L::KV_BYTES / 16);
+            *reinterpret_cast<uint4*>(base + st * L::STAGE_BYTES + L::KV_BYTES + w * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        umma_producer<D>(a, it, tmk, tmv, base, full, empty, masks, s_abort);
+        return;
+    }
+    if (warp == 1) {
+        if (lane == 0) {
+            umma_issuer<D>(ntiles, base, tmem, full, empty, sbar, sfree, pready, obar, mma_done,
+                           s_abort, a.err);
+            (void)mbar_wait(join, 0);  // both warpgroups have read their O
+        }
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+        return;
+    }
+
+    // ---- softmax warpgroup wg: tiles j = wg, wg + 2, ... ----
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t col_s = L::COL_S + 64u * (uint32_t)wg, col_o = L::COL_O + (uint32_t)(wg * D);
+    const int row_len = row.ok ? row.len : 0;
+    float m_used = kNegInfP, l_run = 0.f;
+    bool ok = true;
+    int k = 0;  // tiles this warpgroup has done
+    for (int j = wg; j < ntiles; j += 2, ++k) {
+        const int stage = j % L::STAGES;
+        const bool w_ok = mbar_wait(&sbar[wg], (uint32_t)k & 1u) &&
+                          mbar_wait(&full[stage], (uint32_t)(j / L::STAGES) & 1u) && !*s_abort;
+        ok = __all_sync(0xffffffffu, w_ok);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t msk = masks[stage];
+        float x[kUTileKeys];
+        {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(lane_base + col_s, v0);
+            tmem_ld32(lane_base + col_s + 32, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                x[e] = __uint_as_float(v0[e]);
+                x[32 + e] = __uint_as_float(v1[e]);
+            }
+        }
+        // the score buffer may take S_{j+2} now
+        tc_fence_before();
+        mbar_arrive(&sfree[wg]);
+        const int tile_t0 = it.t0 + j * kUTileKeys;
+        const int k_lo = max(0, row.lo - tile_t0), k_hi = min(kUTileKeys, row_len - tile_t0);
+        // the row maximum as a tree of eight independent chains
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = kNegInfP;
+        if (k_lo == 0 && k_hi == kUTileKeys && msk == (1u << kUTilePages) - 1u) {
+#pragma unroll
+            for (int e = 0; e < kUTileKeys; ++e) {
+                x[e] *= a.scale_log2;
+                mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < kUTileKeys; ++e) {
+                const bool valid = e >= k_lo && e < k_hi && ((msk >> (e / kPageRows)) & 1u);
+                x[e] = valid ? x[e] * a.scale_log2 : kNegInfP;
+                mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
+            }
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_new = fmaxf(m_used, mx);
+        const bool need = m_used != kNegInfP && m_new > m_used + kURescaleLog2;
+        if (m_used == kNegInfP) m_used = m_new;
+        // this warpgroup's previous tile (j - 2) has left P[wg] and O[wg]
+        if (k >= 1) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&obar[wg], (uint32_t)(k - 1) & 1u));
+            if (!ok) break;
+            tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + col_o + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                tmem_st32(lane_base + col_o + c0, v);
+            }
+            tmem_wait_st();
+            if (need) {
+                l_run *= alpha;
+                m_used = m_new;
+            }
+        }
+        const float m_ref = m_used == kNegInfP ? 0.f : m_used;
+        const uint32_t hi_row = smem_addr(base + L::OFF_P + wg * 2 * L::P_BYTES) + r * 128;
+        const uint32_t lo_row = hi_row + L::P_BYTES;
+        float ps8[8];  // the row sum, eight independent chains
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ps8[u] = 0.f;
+#pragma unroll
+        for (int c = 0; c < kUTileKeys / 8; ++c) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float p0 = fast_exp2(x[8 * c + 2 * e] - m_ref);
+                const float p1 = fast_exp2(x[8 * c + 2 * e + 1] - m_ref);
+                ps8[2 * e] += p0;
+                ps8[2 * e + 1] += p1;
+                hw[e] = pack_bf16(p0, p1);
+                lw[e] = pack_bf16(p0 - bf16lo(hw[e]), p1 - bf16hi(hw[e]));
+            }
+            const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
+            st_shared_v4(hi_row + off, hw[0], hw[1], hw[2], hw[3]);
+            st_shared_v4(lo_row + off, lw[0], lw[1], lw[2], lw[3]);
+        }
+        l_run += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        // V rows that no row of the item may read (past the item's last key,
+        // or before the first key any row attends) may hold anything: zero
+        // them before P V reads them
+        const int z_lo = max(0, it.lo - tile_t0), z_hi = min(kUTileKeys, it.t1 - tile_t0);
+        if (z_lo > 0 || z_hi < kUTileKeys) {
+            uint8_t* vt = base + stage * L::STAGE_BYTES + L::KV_BYTES;
+            for (int idx = r; idx < kUTileKeys * L::NB * 8; idx += kURows) {
+                const int key = idx / (L::NB * 8), rest = idx % (L::NB * 8);
+                if (key >= z_lo && key < z_hi) continue;
+                const int nb = rest >> 3, ch = rest & 7;
+                *reinterpret_cast<uint4*>(vt + nb * L::BLOCK_STRIDE + key * 128 + ch * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&pready[wg]);
+    }
+    if (!ok) {
+        *s_abort = 1;
+        if (lane == 0) report_error(a.err, PKV_DEVERR_TIMEOUT);
+    }
+    // this warpgroup's tiles and its last O += P V
+    const int n_mine = ntiles > wg ? (ntiles - wg + 1) / 2 : 0;
+    const bool have_o =
+        ok && n_mine > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&obar[wg], (uint32_t)(n_mine - 1) & 1u));
+    if (wg == 1) {
+        xchg[r] = make_float2(have_o ? m_used : kNegInfP, have_o ? l_run : 0.f);
+        mbar_arrive(xchg_bar);
+        tc_fence_before();
+        mbar_arrive(join);
+        return;
+    }
+    // warpgroup 0: merge the two states of the row, then store it
+    const bool x_ok = __all_sync(0xffffffffu, mbar_wait(xchg_bar, 0));
+    const float2 o1 = x_ok ? xchg[r] : make_float2(kNegInfP, 0.f);
+    const int n1 = ntiles > 1 ? ntiles / 2 : 0;
+    const bool have_o1 = x_ok && n1 > 0 && o1.x != kNegInfP;
+    const float m0 = have_o ? m_used : kNegInfP;
+    const float M = fmaxf(m0, have_o1 ? o1.x : kNegInfP);
+    const float e0 = (have_o && m0 != kNegInfP) ? fast_exp2(m0 - M) : 0.f;
+    const float e1 = have_o1 ? fast_exp2(o1.x - M) : 0.f;
+    const float l_tot = (have_o ? l_run : 0.f) * e0 + (have_o1 ? o1.y : 0.f) * e1;
+    const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+    const float w0 = e0 * inv, w1 = e1 * inv;
+    if (__any_sync(0xffffffffu, have_o || have_o1)) tc_fence_after();
+    const bool any_o = __any_sync(0xffffffffu, have_o), any_o1 = __any_sync(0xffffffffu, have_o1);
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        if (any_o) {
+            uint32_t u[32];
+            tmem_ld32(lane_base + L::COL_O + c0, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = w0 > 0.f ? __uint_as_float(u[e]) * w0 : 0.f;
+        }
+        if (any_o1) {
+            uint32_t u[32];
+            tmem_ld32(lane_base + L::COL_O + D + c0, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                if (w1 > 0.f) v[e] = fmaf(__uint_as_float(u[e]), w1, v[e]);
+        }
+        if (!row.ok) continue;
+        if (row.out && a.out_bf16) {
+            uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(row.out) + c0);
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+                o[e / 8] = make_uint4(pack_bf16(v[e], v[e + 1]), pack_bf16(v[e + 2], v[e + 3]),
+                                      pack_bf16(v[e + 4], v[e + 5]), pack_bf16(v[e + 6], v[e + 7]));
+        } else {
+            float4* o = reinterpret_cast<float4*>(row.out ? reinterpret_cast<float*>(row.out) + c0
+                                                          : row.po + c0);
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) o[e / 4] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+    }
+    if (row.ok && !row.out) {
+        row.pml[0] = l_tot > 0.f ? M : kNegInfP;
+        row.pml[1] = l_tot;
+    }
+    tc_fence_before();
+    mbar_arrive(join);
+}
+
+// Chunked prefill: item (sequence, kv head, row group of 128 rows,
+// partition); row fr of the group is (query fr / G, head fr % G); query i
+// sits at position L - C + i and attends keys up to it.
+template <int D, int G>
+__global__ void __launch_bounds__(kUThreads)
+    paged_prefill_umma_kernel(const __grid_constant__ PrefillParams p,
+                              const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0 && lane == 0) {
+        prefetch_tensor_map(&tm_k);
+        prefetch_tensor_map(&tm_v);
+    }
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const PItem pit = prefill_item(p);
+    if (pit.part >= pit.np) return;  // no keys in this partition (uniform: the whole CTA leaves)
+    UItem it;
+    it.b = pit.b;
+    it.h = pit.h;
+    it.t0 = pit.t0;
+    it.t1 = pit.t1;
+    it.npages = pit.npages;
+    it.lo = pit.lo;
+    URow row = {};
+    if (warp >= 2) {
+        const int fr = pit.rg * kURows + 32 * (warp & 3) + lane;
+        row.ok = fr < p.C * G;
+        const int qi = row.ok ? fr / G : 0, hq = pit.h * G + (row.ok ? fr % G : 0);
+        const size_t grow = ((size_t)pit.b * p.C + qi) * p.Hq + hq;
+        row.q = p.q + grow * D;
+        row.len = row.ok ? pit.L - p.C + qi + 1 : 0;
+        row.lo = (p.window > 0 && row.len > p.window) ? row.len - p.window : 0;
+        if (pit.np == 1) {
+            row.out = p.out_bf16 ? (void*)(reinterpret_cast<bf16*>(p.out) + grow * D)
+                                 : (void*)(reinterpret_cast<float*>(p.out) + grow * D);
+        } else {
+            row.out = nullptr;
+            row.po = p.part_o + (grow * p.NP + pit.part) * D;
+            row.pml = p.part_ml + (grow * p.NP + pit.part) * 2;
+        }
+    }
+    UArgs a;
+    a.block_tables = p.block_tables;
+    a.err = p.err;
+    a.MB = p.MB;
+    a.Hkv = p.Hkv;
+    a.num_blocks = p.num_blocks;
+    a.out_bf16 = p.out_bf16;
+    a.scale_log2 = p.scale_log2;
+    umma_attend<D>(a, it, row, &tm_k, &tm_v, base);
+}
+
 // ---- cascade decode: the shared-prefix pass ----------------------------------
 
 struct CascadeParams {
@@ -484,46 +745,35 @@ __device__ __forceinline__ int cascade_shared(const CascadeParams& p, int b) {
     return s < 0 ? 0 : (s > L ? L : s) / kPageRows * kPageRows;
 }
 
-// One CTA per (group, kv head, row group): the rows are (member, head)
-// pairs, member m of the group and head g -> row m*G + g; every row attends
-// to the first shared_tokens of its own sequence, read once for the group
-// from the pages of the member that shares the most (the others' shared
-// block-table entries must be the same ids: a mismatch sets
-// PKV_DEVERR_PREFIX).  The result goes to partial slot 0 of each member;
-// the decode kernel writes the rest of the sequence to slots 1.. and the
-// combine merges them.  The kernel does not wait for the decode kernel before
-// it starts (it reads nothing the decode writes), so its CTAs fill SMs as the
-// decode's CTAs finish; each CTA waits for the decode grid before it exits,
-// so that the combine, which waits for this grid, also sees the decode's
-// partials.
+// One CTA per (group, kv head, row group of 128 rows): the rows are
+// (member, head) pairs, member m of the group and head g -> row m*G + g;
+// every row attends to the first shared_tokens of its own sequence, read
+// once for the group from the pages of the member that shares the most (the
+// others' shared block-table entries must be the same ids: a mismatch sets
+// PKV_DEVERR_PREFIX).  The tiles run on the tensor cores (umma_attend).  The
+// result goes to partial slot 0 of each member; the decode kernel writes the
+// rest of the sequence to slots 1.. and the combine merges them.  The kernel
+// does not wait for the decode kernel before it starts (it reads nothing the
+// decode writes; q was rotated before the decode began), so its CTAs fill
+// SMs as the decode's CTAs finish; each CTA waits for the decode grid before
+// it exits, so that the combine, which waits for this grid, also sees the
+// decode's partials.
 template <int D, int G>
-__global__ void __launch_bounds__(kThreadsP)
+__global__ void __launch_bounds__(kUThreads)
     cascade_prefix_kernel(const __grid_constant__ CascadeParams p,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v) {
-    using L = PLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
-    uint64_t* empty = full + L::STAGES;
-    uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(masks + L::STAGES);
-    __shared__ int s_grp[3];  // first member, member count, leader
-    __shared__ int s_len;     // the leader's shared tokens
-    const int tid = threadIdx.x, warp = tid >> 5;
+    __shared__ int s_grp[4];  // first member, member count, leader, the leader's shared tokens
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     grid_launch_dependents();
     int x = blockIdx.x;
     const int rg = x % p.RG;
     x /= p.RG;
     const int h = x % p.Hkv, g = x / p.Hkv;
     if (tid == 0) {
-        for (int s = 0; s < L::STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NWP);
-        }
-        *s_abort = 0;
-        fence_barrier_init();
         int gs = p.group_start[g], ge = p.group_start[g + 1];
         if (gs < 0 || ge < gs || ge > p.B) {
             report_error(p.err, PKV_DEVERR_PREFIX);
@@ -540,18 +790,18 @@ __global__ void __launch_bounds__(kThreadsP)
         s_grp[0] = gs;
         s_grp[1] = ge - gs;
         s_grp[2] = leader;
-        s_len = best;
+        s_grp[3] = best;
     }
     __syncthreads();
-    const int gs = s_grp[0], nmem = s_grp[1], leader = s_grp[2], S = s_len;
-    if (S > 0) {
-        if (warp == NWP && (tid & 31) == 0) {
+    const int gs = s_grp[0], nmem = s_grp[1], leader = s_grp[2], S = s_grp[3];
+    if (S > 0 && rg * kURows < nmem * G) {
+        if (warp == 0 && lane == 0) {
             prefetch_tensor_map(&tm_k);
             prefetch_tensor_map(&tm_v);
         }
         // every member's shared pages must be the leader's (checked once, by row group 0)
         if (rg == 0 && h == 0) {
-            for (int idx = tid; idx < nmem * (S / kPageRows); idx += kThreadsP) {
+            for (int idx = tid; idx < nmem * (S / kPageRows); idx += kUThreads) {
                 const int m = idx / (S / kPageRows), j = idx - m * (S / kPageRows);
                 const int b = gs + m;
                 if (j < cascade_shared(p, b) / kPageRows &&
@@ -559,43 +809,36 @@ __global__ void __launch_bounds__(kThreadsP)
                     report_error(p.err, PKV_DEVERR_PREFIX);
             }
         }
-        PItem it;
+        UItem it;
         it.b = leader;
         it.h = h;
-        it.rg = rg;
-        it.part = 0;
-        it.L = S;
-        it.np = 1;
         it.t0 = 0;
         it.t1 = S;
         it.npages = S / kPageRows;
         it.lo = 0;
-        PrefillParams pp;  // the fields the page producer reads
-        pp.block_tables = p.block_tables;
-        pp.err = p.err;
-        pp.MB = p.MB;
-        pp.Hkv = p.Hkv;
-        pp.num_blocks = p.num_blocks;
-        if (warp == NWP) {
-            prefill_producer<D>(pp, it, &tm_k, &tm_v, base, full, empty, masks, s_abort);
-        } else {
-            PRow row;
-            const int fr = rg * (NWP * kRowsPerWarp) + warp * kRowsPerWarp + ((tid & 31) >> 2);
+        URow row = {};
+        if (warp >= 2) {
+            const int fr = rg * kURows + 32 * (warp & 3) + lane;
             const int m = fr / G, hq = h * G + fr % G;
             const int b = gs + m;
-            row.ok = m < nmem;
-            row.len = row.ok ? cascade_shared(p, b) : 0;
+            row.len = m < nmem ? cascade_shared(p, b) : 0;
+            row.ok = row.len > 0;  // no shared tokens: no slot 0
             row.lo = 0;
-            row.ok = row.ok && row.len > 0;  // no shared tokens: no slot 0
             const size_t r = (size_t)(row.ok ? b : 0) * p.Hq + hq;
             row.q = p.q + r * D;
-            row.direct = false;
             row.out = nullptr;
             row.po = p.part_o + (r * p.NPT) * D;
             row.pml = p.part_ml + (r * p.NPT) * 2;
-            multirow_consumer<D>(p.scale_log2, 0, p.err, it, row, base, full, empty, masks,
-                                 s_abort);
         }
+        UArgs a;
+        a.block_tables = p.block_tables;
+        a.err = p.err;
+        a.MB = p.MB;
+        a.Hkv = p.Hkv;
+        a.num_blocks = p.num_blocks;
+        a.out_bf16 = 0;
+        a.scale_log2 = p.scale_log2;
+        umma_attend<D>(a, it, row, &tm_k, &tm_v, base);
     }
     // do not complete before the decode grid: the combine waits for this one
     if ((tid & 31) == 0) grid_dependency_wait();
@@ -620,11 +863,12 @@ cudaError_t set_smem_once(K kern, size_t smem) {
     return e;
 }
 
+// The tensor-core (tcgen05) prefill: one 128-row item per CTA, one CTA per SM.
 template <int D, int G>
-cudaError_t launch_prefill_typed(const PrefillArgs& a, const CUtensorMap& tmk,
-                                 const CUtensorMap& tmv) {
-    using L = PLayout<D>;
-    auto kern = paged_prefill_kernel<D, G>;
+cudaError_t launch_prefill_umma_typed(const PrefillArgs& a, const CUtensorMap& tmk,
+                                      const CUtensorMap& tmv) {
+    using L = ULayout<D>;
+    auto kern = paged_prefill_umma_kernel<D, G>;
     cudaError_t e = set_smem_once(kern, L::SMEM);
     if (e != cudaSuccess) return e;
     PrefillParams p;
@@ -642,7 +886,7 @@ cudaError_t launch_prefill_typed(const PrefillArgs& a, const CUtensorMap& tmk,
     p.MB = (int)a.MB;
     p.P = a.partition_tokens;
     p.NP = a.max_partitions;
-    p.RG = (int)((a.C * G + NWP * kRowsPerWarp - 1) / (NWP * kRowsPerWarp));
+    p.RG = (int)((a.C * G + kURows - 1) / kURows);
     p.num_blocks = (int)a.num_blocks;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out_bf16 = a.out_dtype == PKV_DTYPE_BF16;
@@ -650,7 +894,7 @@ cudaError_t launch_prefill_typed(const PrefillArgs& a, const CUtensorMap& tmk,
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.B * a.Hkv * p.RG * a.max_partitions));
-    cfg.blockDim = dim3(kThreadsP);
+    cfg.blockDim = dim3(kUThreads);
     cfg.dynamicSmemBytes = L::SMEM;
     cfg.stream = a.stream;
     cudaLaunchAttribute attr[1];
@@ -672,10 +916,10 @@ cudaError_t launch_prefill_typed(const PrefillArgs& a, const CUtensorMap& tmk,
 template <int D>
 cudaError_t prefill_dispatch_g(const PrefillArgs& a, const CUtensorMap& k, const CUtensorMap& v) {
     switch (a.Hq / a.Hkv) {
-        case 1: return launch_prefill_typed<D, 1>(a, k, v);
-        case 2: return launch_prefill_typed<D, 2>(a, k, v);
-        case 4: return launch_prefill_typed<D, 4>(a, k, v);
-        case 8: return launch_prefill_typed<D, 8>(a, k, v);
+        case 1: return launch_prefill_umma_typed<D, 1>(a, k, v);
+        case 2: return launch_prefill_umma_typed<D, 2>(a, k, v);
+        case 4: return launch_prefill_umma_typed<D, 4>(a, k, v);
+        case 8: return launch_prefill_umma_typed<D, 8>(a, k, v);
     }
     return cudaErrorInvalidValue;
 }
@@ -683,7 +927,7 @@ cudaError_t prefill_dispatch_g(const PrefillArgs& a, const CUtensorMap& k, const
 template <int D, int G>
 cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
                                  const CUtensorMap& tmv) {
-    using L = PLayout<D>;
+    using L = ULayout<D>;
     auto kern = cascade_prefix_kernel<D, G>;
     cudaError_t e = set_smem_once(kern, L::SMEM);
     if (e != cudaSuccess) return e;
@@ -701,13 +945,13 @@ cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
     p.Hkv = (int)a.Hkv;
     p.MB = (int)a.MB;
     p.NPT = a.slots_per_row;
-    p.RG = (int)((a.max_group_size * G + NWP * kRowsPerWarp - 1) / (NWP * kRowsPerWarp));
+    p.RG = (int)((a.max_group_size * G + kURows - 1) / kURows);
     p.NG = (int)a.num_groups;
     p.num_blocks = (int)a.num_blocks;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.num_groups * a.Hkv * p.RG));
-    cfg.blockDim = dim3(kThreadsP);
+    cfg.blockDim = dim3(kUThreads);
     cfg.dynamicSmemBytes = L::SMEM;
     cfg.stream = a.stream;
     cudaLaunchAttribute attr[1];

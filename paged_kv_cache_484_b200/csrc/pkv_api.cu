@@ -580,6 +580,25 @@ pkv_status pkv_decode_step(void* q, const void* k_new, const void* v_new, const 
                          partition_tokens, flags, device_error, stream, &step);
 }
 
+pkv_status pkv_decode_step_window(void* q, const void* k_new, const void* v_new,
+                                  const int64_t* positions, const int64_t* slot_mapping,
+                                  void* k_cache, void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, void* out, void* workspace,
+                                  size_t workspace_bytes, int64_t num_seqs, int64_t num_q_heads,
+                                  int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                                  int64_t block_size, int64_t max_blocks_per_seq,
+                                  int32_t kv_dtype, int32_t out_dtype, double rope_theta,
+                                  float scale, int32_t sliding_window, int32_t partition_tokens,
+                                  uint32_t flags, int32_t* device_error, void* stream) {
+    set_last_error("");
+    const StepExtras step = {k_new, v_new, positions, slot_mapping, rope_theta};
+    return decode_common(q, k_cache, v_cache, block_tables, context_lens, out, workspace,
+                         workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                         num_blocks, block_size, max_blocks_per_seq, kv_dtype, out_dtype, scale,
+                         partition_tokens, flags, device_error, stream, &step, nullptr,
+                         sliding_window);
+}
+
 pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
                                            const void* v_cache, const int32_t* block_tables,
                                            const int32_t* context_lens, void* out,
@@ -818,18 +837,19 @@ pkv_status pkv_paged_attention_decode_cascade(
 
 namespace pkv {
 namespace {
-constexpr int kPrefillRowsPerItem = 32;  // (query, head) rows one prefill CTA serves
+constexpr int kPrefillRowsPerItem = 128;  // (query, head) rows one prefill CTA serves
 
-// Partition length of a prefill call: about two items per SM if every
-// sequence had the maximum length, in whole 128-token stages, [128, 2048].
+// Partition length of a prefill call: about eight items per SM (one CTA per
+// SM at a time) if every sequence had the maximum length, in whole 64-key
+// tiles, [256, 2048].
 int32_t prefill_auto_partition(int64_t B, int64_t C, int64_t Hq, int64_t Hkv, int64_t MB) {
     const int64_t maxlen = MB * kPageRows;
     const int64_t G = Hq / std::max<int64_t>(1, Hkv);
     const int64_t rg = ceil_div(C * G, kPrefillRowsPerItem);
-    const int64_t target = 2 * (int64_t)device_sm_count();
+    const int64_t target = 8 * (int64_t)device_sm_count();
     int64_t P = ceil_div(std::max<int64_t>(1, maxlen * B * Hkv * rg), target);
-    P = ceil_div(P, 128) * 128;
-    P = std::max<int64_t>(128, std::min<int64_t>(P, 2048));
+    P = ceil_div(P, 64) * 64;
+    P = std::max<int64_t>(256, std::min<int64_t>(P, 2048));
     const int64_t floor_np = ceil_div(ceil_div(maxlen, kMaxPartitions), kPageRows) * kPageRows;
     return (int32_t)std::max(P, floor_np);
 }

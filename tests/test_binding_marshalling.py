@@ -113,6 +113,15 @@ def _cases():
         ["q", "k_new", "v_new", "positions", "slot_mapping", "k_cache", "v_cache",
          "block_tables", "context_lens", "out", "workspace"]))
 
+    a = dict(_step_args(), workspace=ws(), err=err())
+    cases.append(("decode_step window", lambda a=a: B.decode_step(
+        a["q"], a["k_new"], a["v_new"], a["positions"], a["slot_mapping"], a["k_cache"],
+        a["v_cache"], a["block_tables"], a["context_lens"], 1e4, 0.125, a["out"],
+        workspace=a["workspace"], device_error=a["err"], sliding_window=32), a,
+        "pkv_decode_step_window",
+        ["q", "k_new", "v_new", "positions", "slot_mapping", "k_cache", "v_cache",
+         "block_tables", "context_lens", "out", "workspace"]))
+
     a = dict(_decode_args(), err=err())
     cases.append(("paged_attention_decode_noalloc", lambda a=a: B.paged_attention_decode_noalloc(
         a["q"], a["k_cache"], a["v_cache"], a["block_tables"], a["context_lens"], 0.125, a["out"],
@@ -186,3 +195,13 @@ def test_prepared_step_checks_devices_once(rec):
         B.prepare_decode_step(a["q"], a["k_new"], a["v_new"], a["positions"],
                               a["slot_mapping"], a["k_cache"], a["v_cache"], a["block_tables"],
                               a["context_lens"], 1e4, 0.125, a["out"], workspace=a["workspace"])
+
+
+def test_fused_window_step_passes_the_window_before_the_partition_length(rec):
+    a = dict(_step_args(), workspace=_t((4096,), u8))
+    B.decode_step(a["q"], a["k_new"], a["v_new"], a["positions"], a["slot_mapping"],
+                  a["k_cache"], a["v_cache"], a["block_tables"], a["context_lens"], 1e4, 0.125,
+                  a["out"], workspace=a["workspace"], partition_tokens=48, sliding_window=33)
+    args = [c for c in rec.calls if c[0] == "pkv_decode_step_window"][0][1]
+    # ..., rope_theta, scale, sliding_window, partition_tokens, flags, device_error, stream
+    assert args[-7:-3] == (1e4, 0.125, 33, 48)

@@ -139,3 +139,54 @@ def test_window_on_the_ragged_batch():
     got = out.double().cpu()
     assert torch.isfinite(got).all()
     assert (got - want).abs().max().item() <= TOL_BF16
+
+
+@pytest.mark.parametrize("d,G", [(64, 4), (128, 4), (64, 8)])
+@pytest.mark.parametrize("W,P,cluster", [
+    (1, 0, True), (16, 64, False), (17, 0, True), (100, 48, True), (1000, 128, False),
+    (5000, 0, True),
+])
+def test_fused_step_with_window_matches_oracle(d, G, W, P, cluster):
+    """pkv_decode_step_window: the new token appended inside the decode kernel,
+    each query attending to its last W tokens (the new one included).  The
+    oracle appends with its own RoPE, then decodes with the window, on host
+    copies taken before the GPU step; every cached token before a window is
+    NaN on the GPU."""
+    from paged_kv_cache_484_b200 import workloads as W_
+    from tests.parity_util import SubProblem, check_within_one_bf16_ulp
+    lens = [300, 0, 15, 16, 2048, 777, 64, 5]
+    w = W_.build_workload("window-step", lens, G * 2, 2, d, torch.bfloat16, 5e5,
+                          seed=760 + d + G + W, device=DEV, pool_factor=1.2)
+    sub = SubProblem(w, range(w.B))
+    # tokens before every window hold NaN in the GPU cache (never read)
+    tables = w.block_tables.cpu()
+    blks, rows = [], []
+    for b, L in enumerate(w.decode_lens.tolist()):
+        t = torch.arange(max(0, L - W))
+        blks.append(tables[b, t // BS].long())
+        rows.append(t % BS)
+    blks, rows = torch.cat(blks).to(DEV), torch.cat(rows).to(DEV)
+    w.k_cache[blks, :, rows] = float("nan")
+    w.v_cache[blks, :, rows] = float("nan")
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=DEV)
+    pkv.decode_step(w.q, w.k_new, w.v_new, w.positions, w.slot_mapping, w.k_cache, w.v_cache,
+                    w.block_tables, w.decode_lens, w.rope_theta, w.scale, out,
+                    partition_tokens=P, device_error=err, cluster=cluster, sliding_window=W)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    q, kc, vc = sub.q.clone(), sub.k_cache.clone(), sub.v_cache.clone()
+    oracle.kv_append(q, sub.k_new.clone(), sub.v_new.clone(), sub.positions, sub.slots, kc, vc,
+                     sub.theta)
+    want = oracle.paged_attention_decode(q, kc, vc, sub.tables, sub.decode_lens, sub.scale,
+                                         nthreads=8, window=W)
+    got = out.double().cpu()
+    assert torch.isfinite(got).all()
+    assert (got - want).abs().max().item() <= TOL_BF16
+    # the appended rows: within one bf16 ulp of the oracle's
+    slots = w.slot_mapping.cpu()
+    for b in range(w.B):
+        s_g, s_o = int(slots[b]), int(sub.slots[b])
+        check_within_one_bf16_ulp(w.k_cache[s_g // BS, :, s_g % BS].cpu(), kc[s_o // BS, :, s_o % BS],
+                                  f"appended k of sequence {b}")
+        assert torch.equal(w.v_cache[s_g // BS, :, s_g % BS].cpu(), vc[s_o // BS, :, s_o % BS])
