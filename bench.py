@@ -458,7 +458,10 @@ def measure(cfg, args, device, world, local, rank, full: bool):
         if w.dtype != torch.bfloat16:
             raise SystemExit("--kv-dtype e4m3 takes a bf16 workload (configs 2-5)")
         k8, v8, ks8, vs8 = W.e4m3_cache(w)
-        w.k_cache, w.v_cache = k8, v8
+        # the library's 8-bit cache: one [K | V] region per page, one buffer
+        w.k_cache = W.e4m3_pack(k8, v8)
+        w.v_cache = w.k_cache
+        del k8, v8
         w.meta["e4m3_scales"] = (ks8, vs8)
         two_calls = True
         torch.cuda.empty_cache()
@@ -497,12 +500,15 @@ def measure(cfg, args, device, world, local, rank, full: bool):
     # step's metadata (positions, slots, block tables, context lengths) is one
     # set shared by all copies, as one decode step's metadata is shared by all
     # layers of a model.
-    layer_fields = ("q", "k_new", "v_new", "k_cache", "v_cache")
+    layer_fields = ("q", "k_new", "v_new", "k_cache") + (() if e4m3 else ("v_cache",))
     step_fields = ("positions", "slot_mapping", "block_tables", "decode_lens")
     copies = [dict((f, getattr(w, f)) for f in layer_fields + step_fields)]
     for _ in range(ncopies - 1):
         copies.append(dict([(f, getattr(w, f).clone()) for f in layer_fields] +
                            [(f, getattr(w, f)) for f in step_fields]))
+    if e4m3:
+        for c in copies:
+            c["v_cache"] = c["k_cache"]  # the packed 8-bit cache holds both
     outs = [torch.empty((w.B, w.Hq, w.d), dtype=out_dtype, device=device) for _ in range(ncopies)]
 
     cascade = args.cascade
@@ -536,18 +542,17 @@ def measure(cfg, args, device, world, local, rank, full: bool):
     def append(c):
         if e4m3:
             pkv.kv_append_e4m3(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
-                               c["k_cache"], c["v_cache"], w.rope_theta, ks8, vs8,
-                               device_error=err)
+                               c["k_cache"], w.rope_theta, ks8, vs8, device_error=err)
         elif not fused:
             pkv.kv_append(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                           c["k_cache"], c["v_cache"], w.rope_theta, device_error=err)
 
     def decode(c, out):
         if e4m3:
-            pkv.paged_attention_decode_e4m3(c["q"], c["k_cache"], c["v_cache"],
-                                            c["block_tables"], c["decode_lens"], w.scale, ks8,
-                                            vs8, out, workspace=ws, partition_tokens=P,
-                                            device_error=err, sliding_window=args.window)
+            pkv.paged_attention_decode_e4m3(c["q"], c["k_cache"], c["block_tables"],
+                                            c["decode_lens"], w.scale, ks8, vs8, out,
+                                            workspace=ws, partition_tokens=P, device_error=err,
+                                            sliding_window=args.window)
         elif fused:
             pkv.decode_step(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                             c["k_cache"], c["v_cache"], c["block_tables"], c["decode_lens"],
@@ -741,12 +746,9 @@ def measure(cfg, args, device, world, local, rank, full: bool):
         nthreads = os.cpu_count() or 1
         scales = (ks8, vs8) if e4m3 else None
         if e4m3:
-            # the sample's pages as 8-bit codes, cast the same way as the device cache
-            from paged_kv_cache_484_b200.workloads import Workload  # noqa: F401
-            k_c, v_c = sub.k_cache.float(), sub.v_cache.float()
-            sub.k_cache = (k_c / ks8).to(torch.float8_e4m3fn).view(torch.uint8)
-            sub.v_cache = (v_c / vs8).to(torch.float8_e4m3fn).view(torch.uint8) \
-                .transpose(2, 3).contiguous()
+            # the sample's packed 8-bit pages as the oracle's K and transposed V arrays
+            k_h, v_h = W.e4m3_halves(sub.k_cache)
+            sub.k_cache, sub.v_cache = k_h.contiguous(), v_h.contiguous()
         per_step, reps = time_oracle(sub, args.cpu_seconds, nthreads, scales, args.window)
         # the same oracle on one thread, briefly (reported beside the all-cores figure)
         per1, reps1 = time_oracle(sub, min(2.0, args.cpu_seconds), 1, scales, args.window)

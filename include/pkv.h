@@ -388,11 +388,16 @@ pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache
  * not name.  One scale per tensor: the cached value is code x k_scale (K) or
  * code x v_scale (V).
  *
- * Layout (uint8):
- *   k_cache  [num_blocks, Hkv, block_size, head_dim]   (rows as in the bf16 cache)
- *   v_cache  [num_blocks, Hkv, head_dim, block_size]   (each page transposed)
- * The transposed V page lets the decode's tensor-core tile read the four
- * tokens a lane needs as four consecutive bytes.
+ * Layout (uint8): one buffer kv_cache [num_blocks, Hkv, 2, block_size *
+ * head_dim]; each (block, kv head) page is one contiguous region of
+ * 2 x 16 x head_dim bytes:
+ *   K half  [block_size][head_dim]   (rows as in the bf16 cache)
+ *   V half  [head_dim][block_size]   (transposed)
+ * so that one copy fetches a page's K and V (one 2 KiB request at
+ * head_dim 64), and the transposed V half lets the decode's tensor-core tile
+ * read the four tokens a lane needs as four consecutive bytes.  Token t of
+ * block b, kv head h: K at kv_cache + ((b Hkv + h) 2 + 0) 16 d + (t % 16) d,
+ * V dim i at kv_cache + ((b Hkv + h) 2 + 1) 16 d + i 16 + t % 16.
  */
 
 /*
@@ -400,20 +405,20 @@ pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache
  *
  * q is rotated in place and rounded to its own dtype exactly as by
  * pkv_kv_append.  For a token with slot s >= 0 and every kv head h, dim i:
- *   k_cache[s / bs, h, s % bs, i] <- code(rope(k_new[t, h, :], p)[i] / k_scale)
- *   v_cache[s / bs, h, i, s % bs] <- code(v_new[t, h, i] / v_scale)
+ *   K half of page (s / bs, h), row s % bs, byte i  <- code(rope(k_new[t, h, :], p)[i] / k_scale)
+ *   V half of page (s / bs, h), byte i * 16 + s % bs <- code(v_new[t, h, i] / v_scale)
  * where the division is fp64, its result is rounded to binary32 and code()
  * is the nearest E4M3 value of that binary32 number, ties to even,
  * saturating to +-448 (cvt.rn.satfinite).
  *
  * Arguments: those of pkv_kv_append, with
  *   dtype              PKV_DTYPE_F32 or PKV_DTYPE_BF16: q, k_new, v_new
- *   k_cache, v_cache   device uint8, the layout above
+ *   kv_cache           device uint8, the layout above (16-byte aligned)
  *   k_scale, v_scale   finite, > 0
  */
 pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,
                               const int64_t* positions, const int64_t* slot_mapping,
-                              void* k_cache, void* v_cache, int64_t num_tokens,
+                              void* kv_cache, int64_t num_tokens,
                               int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
                               int64_t num_blocks, int64_t block_size, int32_t dtype,
                               double rope_theta, float k_scale, float v_scale,
@@ -435,12 +440,12 @@ pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,
  *
  * Arguments: those of pkv_paged_attention_decode, with
  *   q                  device, [num_seqs, Hq, head_dim] bf16
- *   k_cache, v_cache   device uint8, the layout above
+ *   kv_cache           device uint8, the layout above (16-byte aligned)
  *   k_scale, v_scale   finite, > 0
  *   sliding_window     0, or a window as in pkv_paged_attention_decode_window
  */
-pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
-                                           const void* v_cache, const int32_t* block_tables,
+pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* kv_cache,
+                                           const int32_t* block_tables,
                                            const int32_t* context_lens, void* out,
                                            void* workspace, size_t workspace_bytes,
                                            int64_t num_seqs, int64_t num_q_heads,

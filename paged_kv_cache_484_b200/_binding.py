@@ -96,12 +96,12 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_paged_attention_decode_cascade.restype = ctypes.c_int
         lib.pkv_decode_cascade_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32]
         lib.pkv_decode_cascade_workspace_size.restype = ctypes.c_size_t
-        lib.pkv_kv_append_e4m3.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
+        lib.pkv_kv_append_e4m3.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
                                            i64, i32, ctypes.c_double, ctypes.c_float,
                                            ctypes.c_float, vp, vp]
         lib.pkv_kv_append_e4m3.restype = ctypes.c_int
         lib.pkv_paged_attention_decode_e4m3.argtypes = [
-            vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64, i64, i32,
+            vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64, i64, i32,
             ctypes.c_float, ctypes.c_float, ctypes.c_float, i32, i32, u32, vp, vp]
         lib.pkv_paged_attention_decode_window.argtypes = [
             vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64, i64, i32,
@@ -334,13 +334,13 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     return out
 
 
-def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, rope_theta,
+def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, kv_cache, rope_theta,
                    k_scale, v_scale, stream=None, *, device_error=None) -> None:
     """``kv_append`` into the 8-bit cache: q [T, Hq, d] rotated in place (its
     own dtype, float32 or bfloat16, shared by k_new/v_new [T, Hkv, d]);
-    k_cache uint8 [NB, Hkv, 16, d] gets the E4M3 codes of rope(k) / k_scale,
-    v_cache uint8 [NB, Hkv, d, 16] (pages transposed) those of v / v_scale.
-    See include/pkv.h, pkv_kv_append_e4m3."""
+    kv_cache uint8 [NB, Hkv, 2, 16 * d]: each page's K half [16][d] gets the
+    E4M3 codes of rope(k) / k_scale, its V half [d][16] (transposed) those of
+    v / v_scale.  See include/pkv.h, pkv_kv_append_e4m3."""
     lib = load_library()
     dv = q.device
     dt = _dtype_code(q.dtype)
@@ -348,10 +348,12 @@ def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, r
         if t.dtype != q.dtype:
             raise TypeError(f"{name} dtype {t.dtype} differs from q dtype {q.dtype}")
     T, Hq, d = q.shape
-    NB, Hkv, bs, d2 = k_cache.shape
-    if k_new.shape != (T, Hkv, d) or v_new.shape != (T, Hkv, d) or d2 != d \
-            or v_cache.shape != (NB, Hkv, d, bs) or positions.shape != (T,) \
-            or slot_mapping.shape != (T,):
+    if kv_cache.dim() != 4:
+        raise ValueError("kv_cache must be [num_blocks, Hkv, 2, 16 * head_dim]")
+    NB, Hkv, two, pg = kv_cache.shape
+    bs = BLOCK_SIZE
+    if k_new.shape != (T, Hkv, d) or v_new.shape != (T, Hkv, d) or two != 2 or pg != bs * d \
+            or positions.shape != (T,) or slot_mapping.shape != (T,):
         raise ValueError("inconsistent kv_append_e4m3 shapes")
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
@@ -360,26 +362,30 @@ def kv_append_e4m3(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, r
             _dev(q, "q", on=dv), _dev(k_new, "k_new", on=dv), _dev(v_new, "v_new", on=dv),
             _dev(positions, "positions", torch.int64, on=dv),
             _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
-            _dev(k_cache, "k_cache", torch.uint8, on=dv), _dev(v_cache, "v_cache", torch.uint8, on=dv),
+            _dev(kv_cache, "kv_cache", torch.uint8, on=dv),
             T, Hq, Hkv, d, NB, bs, dt, float(rope_theta), float(k_scale), float(v_scale), err,
             _stream_ptr(stream, q.device))
     _raise(st, lib, "kv_append_e4m3")
 
 
-def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale,
+def paged_attention_decode_e4m3(q, kv_cache, block_tables, context_lens, scale, k_scale,
                                 v_scale, out, stream=None, *, workspace=None, partition_tokens=0,
                                 device_error=None, cluster=True,
                                 sliding_window=0) -> torch.Tensor:
-    """``paged_attention_decode`` over the 8-bit cache (k_cache uint8
-    [NB, Hkv, 16, d], v_cache uint8 [NB, Hkv, d, 16]); q bfloat16 [B, Hq, d];
-    cached values are code x k_scale / code x v_scale.  Writes and returns
-    ``out`` (float32 or bfloat16).  See include/pkv.h."""
+    """``paged_attention_decode`` over the 8-bit cache (kv_cache uint8
+    [NB, Hkv, 2, 16 * d]: per page its K half [16][d], then its V half
+    [d][16]); q bfloat16 [B, Hq, d]; cached values are code x k_scale /
+    code x v_scale.  Writes and returns ``out`` (float32 or bfloat16).  See
+    include/pkv.h."""
     lib = load_library()
     dv = q.device
     B, Hq, d = q.shape
-    NB, Hkv, bs, d2 = k_cache.shape
+    if kv_cache.dim() != 4:
+        raise ValueError("kv_cache must be [num_blocks, Hkv, 2, 16 * head_dim]")
+    NB, Hkv, two, pg = kv_cache.shape
+    bs = BLOCK_SIZE
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
-    if d2 != d or v_cache.shape != (NB, Hkv, d, bs) or out.shape != (B, Hq, d) \
+    if two != 2 or pg != bs * d or out.shape != (B, Hq, d) \
             or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("inconsistent paged_attention_decode_e4m3 shapes")
     if workspace is None:
@@ -390,8 +396,7 @@ def paged_attention_decode_e4m3(q, k_cache, v_cache, block_tables, context_lens,
            if device_error is not None else None)
     with _current(dv):
         st = lib.pkv_paged_attention_decode_e4m3(
-            _dev(q, "q", torch.bfloat16, on=dv), _dev(k_cache, "k_cache", torch.uint8, on=dv),
-            _dev(v_cache, "v_cache", torch.uint8, on=dv),
+            _dev(q, "q", torch.bfloat16, on=dv), _dev(kv_cache, "kv_cache", torch.uint8, on=dv),
             _dev(block_tables, "block_tables", torch.int32, on=dv),
             _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
             _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),

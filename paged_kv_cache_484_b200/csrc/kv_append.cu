@@ -188,8 +188,9 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_kernel(
 
 // The same append into the 8-bit cache: q as above; k and v become E4M3
 // codes of binary32(x / scale) (x / scale in fp64, then one rounding to
-// binary32, then cvt.rn.satfinite to E4M3), k rows into the [16][D] K page,
-// v into column `row` of the transposed [D][16] V page.
+// binary32, then cvt.rn.satfinite to E4M3), k rows into the [16][D] K half
+// of the page, v into column `row` of its transposed [D][16] V half (a page
+// is one [K | V] region of 2 x 16 D bytes).
 template <typename T, int D>
 __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_e4m3_kernel(
     const __grid_constant__ AppendParams p, const __grid_constant__ RopeFreq fr) {
@@ -213,8 +214,7 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_e4m3_kernel(
     T* q = static_cast<T*>(p.q);
     const T* kn = static_cast<const T*>(p.k_new);
     const T* vn = static_cast<const T*>(p.v_new);
-    uint8_t* kc = static_cast<uint8_t*>(p.k_cache);
-    uint8_t* vc = static_cast<uint8_t*>(p.v_cache);
+    uint8_t* page = static_cast<uint8_t*>(p.k_cache);  // [num_blocks, Hkv, 2, 16 D]
 
     for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
         double s, c;
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_e4m3_kernel(
                 *reinterpret_cast<uint4*>(dst + c * E) = pack16<T>(y0);
                 *reinterpret_cast<uint4*>(dst + HALF + c * E) = pack16<T>(y1);
             } else {
-                uint8_t* dst = kc + ((blk * p.Hkv + h) * kPageRows + row) * D;
+                uint8_t* dst = page + (blk * p.Hkv + h) * (int64_t)(2 * kPageRows * D) + row * D;
                 uint32_t w0[E / 4], w1[E / 4];
 #pragma unroll
                 for (int k = 0; k < E / 4; ++k) {
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_e4m3_kernel(
             const int j = idx - nq - nk, h = j / (2 * CPH), c = j % (2 * CPH);
             double x[E];
             unpack16<T>(*reinterpret_cast<const uint4*>(vn + (t * p.Hkv + h) * D + c * E), x);
-            uint8_t* dst = vc + (blk * p.Hkv + h) * (int64_t)D * kPageRows + row;
+            uint8_t* dst = page + (blk * p.Hkv + h) * (int64_t)(2 * kPageRows * D) + kPageRows * D + row;
 #pragma unroll
             for (int e = 0; e < E; e += 2) {
                 const uint32_t w = code2(x[e], x[e + 1], p.v_scale);

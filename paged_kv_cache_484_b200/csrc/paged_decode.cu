@@ -74,7 +74,9 @@ __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / 
 // Tag for the 8-bit cache: E4M3 codes times a per-tensor scale (q stays
 // bf16).  Its K pages keep the [16 tokens][D] row layout; its V pages are
 // stored transposed, [D][16 tokens], so that the four tokens one lane needs
-// for the output MMA are four consecutive bytes.
+// for the output MMA are four consecutive bytes.  A page's K codes and V
+// codes are one contiguous region of the cache ([K | V] per (block, kv
+// head)), which one TMA box fetches at d = 64.
 struct e4m3kv {};
 
 template <typename T, int D, int G>
@@ -96,7 +98,13 @@ struct Layout {
     // else one.
     static constexpr int PPW = ((SWZ && D == 64 && G <= 4) || (F8 && D == 64)) ? 2 : 1;
     static constexpr int STAGE_PAGES = NW * PPW;
-    static constexpr int STAGE_BYTES = 2 * STAGE_PAGES * PAGE_BYTES;  // K pages, then V pages
+    static constexpr int STAGE_BYTES = 2 * STAGE_PAGES * PAGE_BYTES;
+    // Where a stage's pages sit: page k's K at k * KPITCH, its V VOFF past
+    // that.  The 8-bit cache keeps a page's K and V together ([K | V] per
+    // page, as in the cache); the others place a stage's K pages, then its V
+    // pages.
+    static constexpr int KPITCH = F8 ? 2 * PAGE_BYTES : PAGE_BYTES;
+    static constexpr int VOFF = F8 ? PAGE_BYTES : STAGE_PAGES * PAGE_BYTES;
     // 64 KiB of ring (96 KiB for bf16 d = 128, whose CTAs are two per SM
     // by registers anyway)
     static constexpr int STAGES =
@@ -541,7 +549,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
                 break;
             }
             uint8_t* kdst = base + stage * L::STAGE_BYTES;
-            uint8_t* vdst = kdst + L::STAGE_PAGES * L::PAGE_BYTES;
+            uint8_t* vdst = kdst + L::VOFF;
             const bool first = (s0 == 0);
             // fused step: the sequence's last page gets the new token's row;
             // only when its slot is the one the block table gives that token
@@ -574,19 +582,22 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             if (mine) {
                 const int row0 = (cur_ent * p.Hkv + cur.h) * kPageRows;
                 if constexpr (L::F8) {
-                    // one box per page: K as 4 rows of 256 bytes (d = 64) or 16
-                    // swizzled rows of 128 bytes (d = 128); V (transposed) as
-                    // D / 16 rows of 256 bytes
+                    // the page's [K | V] region: at d = 64 one box of 8 rows of
+                    // 256 bytes; at d = 128 its K as 16 swizzled rows of 128
+                    // bytes and its (transposed) V as 8 rows of 256 bytes
                     const int page = cur_ent * p.Hkv + cur.h;
-                    tma_load_2d(kdst + k * L::PAGE_BYTES, tmk, 0, page * (D == 64 ? 4 : kPageRows),
-                                &full[stage]);
-                    tma_load_2d(vdst + k * L::PAGE_BYTES, tmv, 0, page * (D / 16), &full[stage]);
+                    if constexpr (D == 64) {
+                        tma_load_2d(kdst + k * L::KPITCH, tmk, 0, page * 8, &full[stage]);
+                    } else {
+                        tma_load_2d(kdst + k * L::KPITCH, tmk, 0, page * 32, &full[stage]);
+                        tma_load_2d(vdst + k * L::KPITCH, tmv, 0, page * 16 + 8, &full[stage]);
+                    }
                 } else {
 #pragma unroll
                     for (int bx = 0; bx < L::BOXES; ++bx) {
-                        tma_load_2d(kdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmk, bx * 64,
+                        tma_load_2d(kdst + k * L::KPITCH + bx * L::BOX_BYTES, tmk, bx * 64,
                                     row0, &full[stage]);
-                        tma_load_2d(vdst + k * L::PAGE_BYTES + bx * L::BOX_BYTES, tmv, bx * 64,
+                        tma_load_2d(vdst + k * L::KPITCH + bx * L::BOX_BYTES, tmv, bx * 64,
                                     row0, &full[stage]);
                     }
                 }
@@ -691,11 +702,11 @@ __device__ __forceinline__ float* merge_row(uint8_t* base, int st, int w, int g)
     using L = Layout<T, D, G>;
     if constexpr (L::MERGE_SEPARATE)
         return reinterpret_cast<float*>(base + L::OFF_MERGE + (w * G + g) * L::MERGE_ROW_BYTES);
-    uint8_t* kslot = base + st * L::STAGE_BYTES + w * L::PPW * L::PAGE_BYTES;
-    uint8_t* row = g < L::MERGE_ROWS_PER_SLOT
+    uint8_t* kslot = base + st * L::STAGE_BYTES + w * L::PPW * L::KPITCH;
+    // the 8-bit cache: the warp's pages are one region of 2 PPW pages
+    uint8_t* row = (L::F8 || g < L::MERGE_ROWS_PER_SLOT)
                        ? kslot + g * L::MERGE_ROW_BYTES
-                       : kslot + L::STAGE_PAGES * L::PAGE_BYTES +
-                             (g - L::MERGE_ROWS_PER_SLOT) * L::MERGE_ROW_BYTES;
+                       : kslot + L::VOFF + (g - L::MERGE_ROWS_PER_SLOT) * L::MERGE_ROW_BYTES;
     return reinterpret_cast<float*>(row);
 }
 
@@ -808,8 +819,8 @@ __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Ite
         if (pt[0] >= 0 && j == it.npages - 1) {
             const int row = pt[0];
             const size_t grow = (((size_t)pt[1] * p.Hkv + it.h) * kPageRows + row) * D;
-            uint8_t* kpage = base + stage * L::STAGE_BYTES + slot * L::PAGE_BYTES;
-            patch_new_row<T, D>(kpage, kpage + L::STAGE_PAGES * L::PAGE_BYTES,
+            uint8_t* kpage = base + stage * L::STAGE_BYTES + slot * L::KPITCH;
+            patch_new_row<T, D>(kpage, kpage + L::VOFF,
                                 base + L::OFF_NEWKV + stage * L::NEWKV_BYTES, row, tab,
                                 reinterpret_cast<T*>(p.k_cache) + grow,
                                 reinterpret_cast<T*>(p.v_cache) + grow);
@@ -952,8 +963,8 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                         item_patch_page<T, D, G, FUSED>(p, it, jj, warp * PPW + u, stage, base);
                 }
                 const uint32_t kbase =
-                    smem_addr(base + stage * L::STAGE_BYTES + warp * PPW * L::PAGE_BYTES);
-                const uint32_t vbase = kbase + L::STAGE_PAGES * L::PAGE_BYTES;
+                    smem_addr(base + stage * L::STAGE_BYTES + warp * PPW * L::KPITCH);
+                const uint32_t vbase = kbase + L::VOFF;
                 const int mi = lane >> 3, ri = lane & 7;
 
                 // S^T tile: 16 rows (heads) x 16 PPW tokens, n-tiles of 8 tokens
@@ -969,7 +980,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
                             const int tok = 2 * r - (r & 1) + 2 * j;
-                            const uint32_t row = kbase + u * L::PAGE_BYTES + tok * D;
+                            const uint32_t row = kbase + u * L::KPITCH + tok * D;
                             if constexpr (D == 64) {
                                 ld_shared_v4(row + 16 * cq, kw[u][j][0], kw[u][j][1], kw[u][j][2],
                                              kw[u][j][3]);
@@ -999,7 +1010,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
 #pragma unroll
                         for (int u = 0; u < PPW; ++u) {
                             uint32_t b00, b01, b10, b11;
-                            ldsm_x4(kbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch), b00,
+                            ldsm_x4(kbase + u * L::KPITCH + chunk_offset<bf16, D>(tok, ch), b00,
                                     b01, b10, b11);
                             mma_bf16_16816(sc[2 * u], qa[kk], b00, b01);
                             mma_bf16_16816(sc[2 * u + 1], qa[kk], b10, b11);
@@ -1088,7 +1099,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                                 if (4 * cq + e >= first[u] && 4 * cq + e < valid[u])
                                     bm |= 0xffu << (8 * e);
                         }
-                        const uint32_t vrow = vbase + u * L::PAGE_BYTES + r * 16 + 4 * cq;
+                        const uint32_t vrow = vbase + u * L::KPITCH + r * 16 + 4 * cq;
 #pragma unroll
                         for (int c = 0; c < NT; ++c) {
                             uint32_t b0, b1;
@@ -1109,7 +1120,7 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                             const int tok = ri + ((mi & 1) << 3);
                             const int ch = c + (mi >> 1);
                             uint32_t v0, v1, v2, v3;
-                            ldsm_x4_trans(vbase + u * L::PAGE_BYTES + chunk_offset<bf16, D>(tok, ch),
+                            ldsm_x4_trans(vbase + u * L::KPITCH + chunk_offset<bf16, D>(tok, ch),
                                           v0, v1, v2, v3);
                             mma_bf16_16816(o[c], pa, v0 & vmask_lo, v1 & vmask_hi);
                             mma_bf16_16816(o[c + 1], pa, v2 & vmask_lo, v3 & vmask_hi);
@@ -1274,8 +1285,8 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
                 const int valid = min(kPageRows, it.t1 - (it.t0 + j * kPageRows));
                 const int first = max(0, it.lo - (it.t0 + j * kPageRows));  // sliding window
                 item_patch_page<T, D, G, FUSED>(p, it, j, slot, stage, base);
-                const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + slot * L::PAGE_BYTES);
-                const uint32_t vbase = kbase + L::STAGE_PAGES * L::PAGE_BYTES;
+                const uint32_t kbase = smem_addr(base + stage * L::STAGE_BYTES + slot * L::KPITCH);
+                const uint32_t vbase = kbase + L::VOFF;
 #pragma unroll 2
                 for (int ps = 0; ps < PASSES; ++ps) {
                     const int tk = ps * TPW + tg;

@@ -157,8 +157,8 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const __grid_const
 //   warp 1   owns the tensor memory; one lane issues the MMAs;
 //   warps 2-5 and 6-9  two softmax warpgroups, one thread per row
 //            (tensor-memory lane).  Warpgroup w takes the tiles j with
-//            j % 2 = w, with its own score buffer S[w], P buffer P[w],
-//            accumulator O[w] and running (max, sum) per row, so the two
+//            j % 2 = w, with its own score buffer S[w], accumulator O[w] and
+//            running (max, sum) per row (P buffers rotate), so the two
 //            overlap; at the end warpgroup 0 merges the two (max, sum, O)
 //            states of its row exactly (log-sum-exp) and stores the row.
 // A warpgroup's reference max only moves when the row max grew by more
@@ -167,7 +167,10 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const __grid_const
 // arrivals; S_{j+2} may then overwrite the buffer while the warpgroup is
 // still working on tile j); P_j written -> pready[j % 2] (128 arrivals);
 // O[j % 2] += P_j V_j done -> obar[j % 2]; the MMAs of tile j also release
-// its stage (empty).  The MMA lane polls both streams and issues whichever
+// its stage (empty) and P buffer j % PBUFS (pfree).  A warp
+// arrives on pready for its warpgroup's next tile only once that
+// warpgroup's previous O += P V has completed (at most one phase ahead of
+// the MMA lane).  The MMA lane polls both streams and issues whichever
 // MMA is ready first.  Every wait is bounded; a timeout sets
 // PKV_DEVERR_TIMEOUT and the CTA ends its work (the MMA lane waits for its
 // own MMAs before tensor memory is freed).
@@ -188,11 +191,13 @@ struct ULayout {
     static constexpr int Q_BLOCK = kURows * 128;                // one column block of Q
     static constexpr int P_BYTES = kURows * 128;                // 128 rows x 64 keys bf16
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
-    static constexpr int OFF_P = OFF_Q + NB * Q_BLOCK;          // [warpgroup][hi, lo]
-    static constexpr int OFF_XCHG = OFF_P + 4 * P_BYTES;        // (max, sum) of warpgroup 1's rows
+    static constexpr int PBUFS = 2;                             // P buffers, tile j uses j % 2
+    static constexpr int OFF_P = OFF_Q + NB * Q_BLOCK;          // [buffer][hi, lo]
+    static constexpr int OFF_XCHG = OFF_P + PBUFS * 2 * P_BYTES;  // (max, sum) of warpgroup 1's rows
     static constexpr int OFF_BAR = OFF_XCHG + kURows * 8;
-    // full[STAGES], empty[STAGES], sbar[2], sfree[2], pready[2], obar[2], mma_done, xchg, join
-    static constexpr int NBARS = 2 * STAGES + 11;
+    // full[STAGES], empty[STAGES], sbar[2], sfree[2], pready[2], obar[2], pfree[PBUFS],
+    // mma_done, xchg, join
+    static constexpr int NBARS = 2 * STAGES + 11 + PBUFS;
     static constexpr int OFF_MASK = OFF_BAR + NBARS * 8;
     static constexpr int OFF_MISC = OFF_MASK + STAGES * 4;      // abort flag, TMEM base
     static constexpr size_t SMEM = 1024 + OFF_MISC + 16;
@@ -302,8 +307,8 @@ __device__ void umma_producer(const UArgs& a, const UItem& it, const CUtensorMap
 template <int D>
 __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* full,
                             uint64_t* empty, uint64_t* sbar, uint64_t* sfree, uint64_t* pready,
-                            uint64_t* obar, uint64_t* mma_done, volatile int* s_abort,
-                            int32_t* err) {
+                            uint64_t* obar, uint64_t* pfree, uint64_t* mma_done,
+                            volatile int* s_abort, int32_t* err) {
     using L = ULayout<D>;
     const uint32_t sq = smem_addr(base + L::OFF_Q);
     auto issue_s = [&](int j) {
@@ -323,7 +328,7 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
         const int w = j & 1;
         const int stage = j % L::STAGES;
         const uint32_t sv = smem_addr(base + stage * L::STAGE_BYTES + L::KV_BYTES);
-        const uint32_t sp = smem_addr(base + L::OFF_P + w * 2 * L::P_BYTES);
+        const uint32_t sp = smem_addr(base + L::OFF_P + (j % L::PBUFS) * 2 * L::P_BYTES);
         const uint32_t o = tmem + L::COL_O + (uint32_t)(w * D);
 #pragma unroll
         for (int s = 0; s < kUTileKeys / 16; ++s) {
@@ -334,6 +339,7 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
             umma_bf16(o, lo, db, L::IDESC_O, true);
         }
         umma_commit(&obar[w]);
+        umma_commit(&pfree[j % L::PBUFS]);
         umma_commit(&empty[stage]);  // the stage's K and V are no longer read
     };
     // S_j needs its stage loaded and (j >= 2) the buffer's previous scores read;
@@ -390,6 +396,24 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
     (void)mbar_wait(mma_done, 0);
 }
 
+// V rows of tile j that no row of the item may read (past the item's last
+// key, or before the first key any row attends) may hold anything: a
+// warpgroup's 128 threads zero them before P V reads them.
+template <int D>
+__device__ __forceinline__ void umma_zero_v_rows(const UItem& it, int j, int r, uint8_t* vt) {
+    using L = ULayout<D>;
+    const int tile_t0 = it.t0 + j * kUTileKeys;
+    const int z_lo = max(0, it.lo - tile_t0), z_hi = min(kUTileKeys, it.t1 - tile_t0);
+    if (z_lo <= 0 && z_hi >= kUTileKeys) return;
+    for (int idx = r; idx < kUTileKeys * L::NB * 8; idx += kURows) {
+        const int key = idx / (L::NB * 8), rest = idx % (L::NB * 8);
+        if (key >= z_lo && key < z_hi) continue;
+        const int nb = rest >> 3, ch = rest & 7;
+        *reinterpret_cast<uint4*>(vt + nb * L::BLOCK_STRIDE + key * 128 + ch * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
 // One item, run by all kUThreads threads of the CTA (every thread calls it;
 // `row` matters to the softmax warps only).
 template <int D>
@@ -402,7 +426,8 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     uint64_t* sfree = sbar + 2;
     uint64_t* pready = sfree + 2;
     uint64_t* obar = pready + 2;
-    uint64_t* mma_done = obar + 2;
+    uint64_t* pfree = obar + 2;
+    uint64_t* mma_done = pfree + L::PBUFS;
     uint64_t* xchg_bar = mma_done + 1;
     uint64_t* join = xchg_bar + 1;
     uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
@@ -422,6 +447,7 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             mbar_init(&pready[i], kURows);
             mbar_init(&obar[i], 1);
         }
+        for (int i = 0; i < L::PBUFS; ++i) mbar_init(&pfree[i], 1);
         mbar_init(mma_done, 1);
         mbar_init(xchg_bar, kURows);
         mbar_init(join, 2 * kURows);
@@ -463,8 +489,8 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     }
     if (warp == 1) {
         if (lane == 0) {
-            umma_issuer<D>(ntiles, base, tmem, full, empty, sbar, sfree, pready, obar, mma_done,
-                           s_abort, a.err);
+            umma_issuer<D>(ntiles, base, tmem, full, empty, sbar, sfree, pready, obar, pfree,
+                           mma_done, s_abort, a.err);
             (void)mbar_wait(join, 0);  // both warpgroups have read their O
         }
         __syncwarp();
@@ -477,6 +503,11 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t col_s = L::COL_S + 64u * (uint32_t)wg, col_o = L::COL_O + (uint32_t)(wg * D);
     const int row_len = row.ok ? row.len : 0;
+    // a warp whose 32 rows are all padding (past the item's rows) has no
+    // scores to read and no P worth writing: its rows of O are never stored.
+    // It still keeps the tiles' cadence (the same waits and arrivals), so
+    // that it never arrives for a later tile while an earlier one is open.
+    const bool pad_warp = __all_sync(0xffffffffu, !row.ok);
     float m_used = kNegInfP, l_run = 0.f;
     bool ok = true;
     int k = 0;  // tiles this warpgroup has done
@@ -486,6 +517,20 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
                           mbar_wait(&full[stage], (uint32_t)(j / L::STAGES) & 1u) && !*s_abort;
         ok = __all_sync(0xffffffffu, w_ok);
         if (!ok) break;
+        if (pad_warp) {
+            tc_fence_before();
+            mbar_arrive(&sfree[wg]);
+            // one phase ahead of the MMAs at most (see below)
+            if (k >= 1) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&obar[wg], (uint32_t)(k - 1) & 1u));
+                if (!ok) break;
+            }
+            umma_zero_v_rows<D>(it, j, r, base + stage * L::STAGE_BYTES + L::KV_BYTES);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&pready[wg]);
+            continue;
+        }
         tc_fence_after();
         const uint32_t msk = masks[stage];
         float x[kUTileKeys];
@@ -528,13 +573,12 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
         const float m_new = fmaxf(m_used, mx);
         const bool need = m_used != kNegInfP && m_new > m_used + kURescaleLog2;
         if (m_used == kNegInfP) m_used = m_new;
-        // this warpgroup's previous tile (j - 2) has left P[wg] and O[wg]
-        if (k >= 1) {
+        if (__any_sync(0xffffffffu, need)) {
+            // O += P_{j-2} V_{j-2}, this warpgroup's previous tile, has to
+            // land before its O row is rescaled
             ok = __all_sync(0xffffffffu, mbar_wait(&obar[wg], (uint32_t)(k - 1) & 1u));
             if (!ok) break;
             tc_fence_after();
-        }
-        if (__any_sync(0xffffffffu, need)) {
             const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
@@ -552,7 +596,14 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             }
         }
         const float m_ref = m_used == kNegInfP ? 0.f : m_used;
-        const uint32_t hi_row = smem_addr(base + L::OFF_P + wg * 2 * L::P_BYTES) + r * 128;
+        // P buffer j % PBUFS was last read by O += P_{j-PBUFS} V_{j-PBUFS}
+        if (j >= L::PBUFS) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&pfree[j % L::PBUFS],
+                                                   (uint32_t)(j / L::PBUFS - 1) & 1u));
+            if (!ok) break;
+        }
+        const uint32_t hi_row =
+            smem_addr(base + L::OFF_P + (j % L::PBUFS) * 2 * L::P_BYTES) + r * 128;
         const uint32_t lo_row = hi_row + L::P_BYTES;
         float ps8[8];  // the row sum, eight independent chains
 #pragma unroll
@@ -574,21 +625,19 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             st_shared_v4(lo_row + off, lw[0], lw[1], lw[2], lw[3]);
         }
         l_run += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
-        // V rows that no row of the item may read (past the item's last key,
-        // or before the first key any row attends) may hold anything: zero
-        // them before P V reads them
-        const int z_lo = max(0, it.lo - tile_t0), z_hi = min(kUTileKeys, it.t1 - tile_t0);
-        if (z_lo > 0 || z_hi < kUTileKeys) {
-            uint8_t* vt = base + stage * L::STAGE_BYTES + L::KV_BYTES;
-            for (int idx = r; idx < kUTileKeys * L::NB * 8; idx += kURows) {
-                const int key = idx / (L::NB * 8), rest = idx % (L::NB * 8);
-                if (key >= z_lo && key < z_hi) continue;
-                const int nb = rest >> 3, ch = rest & 7;
-                *reinterpret_cast<uint4*>(vt + nb * L::BLOCK_STRIDE + key * 128 + ch * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
+        umma_zero_v_rows<D>(it, j, r, base + stage * L::STAGE_BYTES + L::KV_BYTES);
         fence_proxy_async_smem();
+        // O += P V of this warpgroup's previous tile has completed before
+        // this warp arrives for the next: the warpgroup then runs at most one
+        // phase ahead of the MMA lane, which keeps every parity wait on
+        // pready, obar and pfree unambiguous (two phases ahead, a wait on
+        // obar could mistake an older completed phase for the one it wants,
+        // and a rescale could run under P V updates still in flight).  By now
+        // that MMA has normally long finished.
+        if (k >= 1) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&obar[wg], (uint32_t)(k - 1) & 1u));
+            if (!ok) break;
+        }
         tc_fence_before();
         mbar_arrive(&pready[wg]);
     }
@@ -621,7 +670,8 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
     const float w0 = e0 * inv, w1 = e1 * inv;
     if (__any_sync(0xffffffffu, have_o || have_o1)) tc_fence_after();
-    const bool any_o = __any_sync(0xffffffffu, have_o), any_o1 = __any_sync(0xffffffffu, have_o1);
+    const bool any_o = !pad_warp && __any_sync(0xffffffffu, have_o);
+    const bool any_o1 = !pad_warp && __any_sync(0xffffffffu, have_o1);
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
         float v[32];

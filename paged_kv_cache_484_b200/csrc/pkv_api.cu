@@ -72,6 +72,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // The cache [num_blocks, Hkv, 16, D] viewed as a 2-D tensor of num_blocks*Hkv*16
 // rows of D elements; one box is one 16-row page (bf16: 64 columns per box,
 // 128-byte swizzle; fp32: the whole row, no swizzle).
+//
+// The 8-bit cache is [num_blocks, Hkv, 2, 16 D] bytes: per page its K codes
+// [16][D], then its V codes transposed [D][16].  At D = 64 the page's 2 KiB
+// are one box of 8 rows of 256 bytes (the same bytes in the same order in
+// shared memory, one request per page).  At D = 128 this map covers the
+// cache as rows of 128 bytes (32 per page) and one box is the page's K half,
+// 16 rows, 128-byte swizzled; encode_vt_cache_map gives its V half.
 cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks, int64_t Hkv,
                              int64_t D, int32_t dtype) {
     auto fn = encode_fn();
@@ -79,16 +86,13 @@ cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_bl
     const bool bf = dtype == PKV_DTYPE_BF16;
     const bool f8 = dtype == PKV_DTYPE_E4M3;
     const int esz = f8 ? 1 : (bf ? 2 : 4);
-    // 8-bit d = 64 pages (16 rows of 64 bytes, 1 KiB contiguous) are described
-    // as 4 rows of 256 bytes: the same bytes in the same order in shared
-    // memory, in a quarter of the row requests
-    const bool wide = f8 && D == 64;
-    const int row_bytes = wide ? 256 : (int)(D * esz);
-    const int rows_per_page = wide ? 4 : kPageRows;
+    const int row_bytes = f8 ? (D == 64 ? 256 : 128) : (int)(D * esz);
+    const int rows_per_page = f8 ? (D == 64 ? 8 : 32) : kPageRows;
+    const int box_rows = f8 ? (D == 64 ? 8 : kPageRows) : kPageRows;
     const cuuint64_t rows = (cuuint64_t)(num_blocks * Hkv * rows_per_page);
     cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / esz), rows};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    cuuint32_t box[2] = {(cuuint32_t)(bf ? 64 : row_bytes / esz), (cuuint32_t)rows_per_page};
+    cuuint32_t box[2] = {(cuuint32_t)(bf ? 64 : row_bytes / esz), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     // bf16 boxes are 128-byte rows, swizzled; 8-bit rows of 128 bytes too
     const bool swz = bf || (f8 && D == 128);
@@ -102,18 +106,16 @@ cudaError_t encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_bl
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// The 8-bit cache's transposed V pages [num_blocks, Hkv, D, 16] (bytes).  A
-// page is 16 D contiguous bytes; it is described as D / 16 rows of 256 bytes
-// (one box per page) rather than D rows of 16 bytes, which would cost a row
-// request per 16 bytes.  Shared memory receives the same bytes in the same
-// order.
+// The 8-bit cache at D = 128 as rows of 256 bytes (16 per page); one box is a
+// page's V half, its transposed V codes [128][16] as 8 rows of 256 bytes
+// (page p's V half starts at row 16 p + 8).
 cudaError_t encode_vt_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
                                 int64_t Hkv, int64_t D) {
     auto fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
-    cuuint64_t dims[2] = {256, (cuuint64_t)(num_blocks * Hkv * D / 16)};
+    cuuint64_t dims[2] = {256, (cuuint64_t)(num_blocks * Hkv * (2 * kPageRows * D / 256))};
     cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {256, (cuuint32_t)(D / 16)};
+    cuuint32_t box[2] = {256, (cuuint32_t)(kPageRows * D / 256)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(cache), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -599,8 +601,8 @@ pkv_status pkv_decode_step_window(void* q, const void* k_new, const void* v_new,
                          sliding_window);
 }
 
-pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
-                                           const void* v_cache, const int32_t* block_tables,
+pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* kv_cache,
+                                           const int32_t* block_tables,
                                            const int32_t* context_lens, void* out,
                                            void* workspace, size_t workspace_bytes,
                                            int64_t num_seqs, int64_t num_q_heads,
@@ -612,7 +614,8 @@ pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* k_cache,
                                            uint32_t flags, int32_t* device_error, void* stream) {
     set_last_error("");
     const float scales[2] = {k_scale, v_scale};
-    return decode_common(q, k_cache, v_cache, block_tables, context_lens, out, workspace,
+    // one [K | V] region per page: both halves are reached from kv_cache
+    return decode_common(q, kv_cache, kv_cache, block_tables, context_lens, out, workspace,
                          workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
                          num_blocks, block_size, max_blocks_per_seq, PKV_DTYPE_E4M3, out_dtype,
                          scale, partition_tokens, flags, device_error, stream, nullptr, scales,
@@ -641,7 +644,7 @@ pkv_status pkv_paged_attention_decode_window(const void* q, const void* k_cache,
 
 pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,
                               const int64_t* positions, const int64_t* slot_mapping,
-                              void* k_cache, void* v_cache, int64_t num_tokens,
+                              void* kv_cache, int64_t num_tokens,
                               int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
                               int64_t num_blocks, int64_t block_size, int32_t dtype,
                               double rope_theta, float k_scale, float v_scale,
@@ -656,9 +659,9 @@ pkv_status pkv_kv_append_e4m3(void* q, const void* k_new, const void* v_new,
         set_last_error("num_blocks %lld too large for the 8-bit cache", (long long)num_blocks);
         return PKV_ERR_INVALID_ARG;
     }
-    return append_common(q, k_new, v_new, positions, slot_mapping, k_cache, v_cache, num_tokens,
-                         num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, dtype,
-                         rope_theta, device_error, stream, true, k_scale, v_scale);
+    return append_common(q, k_new, v_new, positions, slot_mapping, kv_cache, kv_cache,
+                         num_tokens, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                         dtype, rope_theta, device_error, stream, true, k_scale, v_scale);
 }
 
 }  // extern "C"

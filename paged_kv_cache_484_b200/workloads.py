@@ -285,6 +285,23 @@ def e4m3_cache(w: Workload, chunk_blocks: int = 4096):
     return k8, v8, ks, vs
 
 
+def e4m3_pack(k8: torch.Tensor, v8: torch.Tensor) -> torch.Tensor:
+    """The 8-bit cache as the library stores it: K codes [NB, Hkv, 16, d] and
+    transposed V codes [NB, Hkv, d, 16] interleaved page by page into one
+    uint8 buffer [NB, Hkv, 2, 16 * d] (each page's K half, then its V half).
+    Pure data movement."""
+    NB, Hkv = k8.shape[:2]
+    return torch.stack((k8.reshape(NB, Hkv, -1), v8.reshape(NB, Hkv, -1)), dim=2).contiguous()
+
+
+def e4m3_halves(kv8: torch.Tensor):
+    """Views of a packed 8-bit cache: (K [NB, Hkv, 16, d], V [NB, Hkv, d, 16]);
+    they alias kv8 and are not contiguous (use .contiguous() for a copy)."""
+    NB, Hkv, _, pg = kv8.shape
+    d = pg // BLOCK_SIZE
+    return kv8[:, :, 0].view(NB, Hkv, BLOCK_SIZE, d), kv8[:, :, 1].view(NB, Hkv, d, BLOCK_SIZE)
+
+
 def extract_sequences(w: Workload, seqs) -> SequenceSubset:
     """Copy the inputs of sequences ``seqs`` to the host (read before any step
     modifies the workload's tensors)."""

@@ -121,21 +121,21 @@ E4M3 = 2
 
 
 def _append8(lib, **kw):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, slot=FAKE, kc=FAKE, vc=FAKE, T=1, Hq=8, Hkv=2, d=64,
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, slot=FAKE, kv=FAKE, T=1, Hq=8, Hkv=2, d=64,
              NB=4, bs=16, dtype=BF16, theta=1e4, ks=0.05, vs=0.05, err=None)
     a.update(kw)
-    return lib.pkv_kv_append_e4m3(a["q"], a["k"], a["v"], a["pos"], a["slot"], a["kc"], a["vc"],
+    return lib.pkv_kv_append_e4m3(a["q"], a["k"], a["v"], a["pos"], a["slot"], a["kv"],
                                   a["T"], a["Hq"], a["Hkv"], a["d"], a["NB"], a["bs"], a["dtype"],
                                   a["theta"], a["ks"], a["vs"], a["err"], None)
 
 
 def _decode8(lib, **kw):
-    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, out=FAKE, ws=None, wsb=0, B=2, Hq=8, Hkv=2,
+    a = dict(q=FAKE, kv=FAKE, bt=FAKE, cl=FAKE, out=FAKE, ws=None, wsb=0, B=2, Hq=8, Hkv=2,
              d=64, NB=4, bs=16, MB=4, odt=BF16, scale=0.125, ks=0.05, vs=0.05, P=0, flags=0,
              err=None)
     a.update(kw)
     return lib.pkv_paged_attention_decode_e4m3(
-        a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["out"], a["ws"], a["wsb"], a["B"], a["Hq"],
+        a["q"], a["kv"], a["bt"], a["cl"], a["out"], a["ws"], a["wsb"], a["B"], a["Hq"],
         a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"], a["odt"], a["scale"], a["ks"], a["vs"],
         a.get("win", 0), a["P"], a["flags"], a["err"], None)
 
@@ -147,7 +147,7 @@ def _decode8(lib, **kw):
     (dict(vs=math.nan), INVALID),
     (dict(dtype=E4M3), UNSUPPORTED),       # q / k_new / v_new are float32 or bfloat16
     (dict(d=96), UNSUPPORTED),
-    (dict(kc=FAKE + 8), INVALID),
+    (dict(kv=FAKE + 8), INVALID),
     (dict(NB=1 << 26, Hkv=8, d=128), INVALID),   # byte rows past int32 tensor coordinates
     (dict(T=0, q=None, k=None), OK),
 ])
@@ -162,7 +162,7 @@ def test_kv_append_e4m3_rejects_bad_arguments(lib, kw, status):
     (dict(odt=E4M3), UNSUPPORTED),
     (dict(d=96), UNSUPPORTED),
     (dict(P=16, MB=4), WORKSPACE),
-    (dict(vc=FAKE + 4), INVALID),
+    (dict(kv=FAKE + 4), INVALID),
     (dict(win=-1), INVALID),
     (dict(B=0, q=None, out=None), OK),
 ])

@@ -128,20 +128,18 @@ def _cases():
         device_error=a["err"]), a, "pkv_paged_attention_decode_noalloc",
         ["q", "k_cache", "v_cache", "block_tables", "context_lens", "out"]))
 
-    a = dict(_step_args(), k_cache=_t((NB, Hkv, 16, D), u8), v_cache=_t((NB, Hkv, D, 16), u8),
-             err=err())
+    a = dict(_step_args(), kv_cache=_t((NB, Hkv, 2, 16 * D), u8), err=err())
     cases.append(("kv_append_e4m3", lambda a=a: B.kv_append_e4m3(
-        a["q"], a["k_new"], a["v_new"], a["positions"], a["slot_mapping"], a["k_cache"],
-        a["v_cache"], 1e4, 0.05, 0.05, device_error=a["err"]), a, "pkv_kv_append_e4m3",
-        ["q", "k_new", "v_new", "positions", "slot_mapping", "k_cache", "v_cache"]))
+        a["q"], a["k_new"], a["v_new"], a["positions"], a["slot_mapping"], a["kv_cache"],
+        1e4, 0.05, 0.05, device_error=a["err"]), a, "pkv_kv_append_e4m3",
+        ["q", "k_new", "v_new", "positions", "slot_mapping", "kv_cache"]))
 
-    a = dict(_decode_args(), k_cache=_t((NB, Hkv, 16, D), u8), v_cache=_t((NB, Hkv, D, 16), u8),
-             workspace=ws(), err=err())
+    a = dict(_decode_args(), kv_cache=_t((NB, Hkv, 2, 16 * D), u8), workspace=ws(), err=err())
     cases.append(("paged_attention_decode_e4m3", lambda a=a: B.paged_attention_decode_e4m3(
-        a["q"], a["k_cache"], a["v_cache"], a["block_tables"], a["context_lens"], 0.125, 0.05,
+        a["q"], a["kv_cache"], a["block_tables"], a["context_lens"], 0.125, 0.05,
         0.05, a["out"], workspace=a["workspace"], device_error=a["err"]), a,
         "pkv_paged_attention_decode_e4m3",
-        ["q", "k_cache", "v_cache", "block_tables", "context_lens", "out", "workspace"]))
+        ["q", "kv_cache", "block_tables", "context_lens", "out", "workspace"]))
 
     a = dict(_decode_args(), q=_t((Bs, C, Hq, D), bf16), out=_t((Bs, C, Hq, D), f32),
              workspace=ws(), err=err())

@@ -134,11 +134,12 @@ def test_decode_e4m3_bad_block_ids():
     tables = _corrupt_tables(w)
     err = _err()
     out = torch.full((w.B, w.Hq, w.d), float("nan"), dtype=torch.float32, device=DEV)
-    pkv.paged_attention_decode_e4m3(w.q, k8, v8, tables, w.cached_lens, w.scale, ks, vs, out,
+    kv8 = W.e4m3_pack(k8, v8)
+    pkv.paged_attention_decode_e4m3(w.q, kv8, tables, w.cached_lens, w.scale, ks, vs, out,
                                     partition_tokens=64, device_error=err)
     assert pkv.get_device_error(err) == pkv.DEVERR_BLOCK_ID
     assert torch.isfinite(out).all()
-    assert torch.equal(k8.cpu(), pristine["k"]) and torch.equal(v8.cpu(), pristine["v"])
+    assert torch.equal(kv8.cpu(), W.e4m3_pack(pristine["k"], pristine["v"]))
     want = oracle.paged_attention_decode_e4m3(pristine["q"], pristine["k"], pristine["v"],
                                               pristine["t"], pristine["l"], w.scale, ks, vs,
                                               nthreads=8)

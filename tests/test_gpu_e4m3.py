@@ -22,6 +22,7 @@ import torch
 
 import oracle
 import paged_kv_cache_484_b200 as pkv
+from paged_kv_cache_484_b200.workloads import e4m3_halves, e4m3_pack
 from tests.parity_util import TOL_BF16, ulp_bf16
 
 pytestmark = pytest.mark.gpu
@@ -93,15 +94,16 @@ def test_kv_append_e4m3_codes_bit_exact(dtype, d):
     kc = torch.full((NB, Hkv, BS, d), 0x7F, dtype=torch.uint8)
     vc = torch.full((NB, Hkv, d, BS), 0x7F, dtype=torch.uint8)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
-    qg, kcg, vcg = q.to(DEV), kc.to(DEV), vc.to(DEV)
-    pkv.kv_append_e4m3(qg, k.to(DEV), v.to(DEV), pos.to(DEV), slots.to(DEV), kcg, vcg, 5e5, ks,
+    qg, kvg = q.to(DEV), e4m3_pack(kc, vc).to(DEV)
+    pkv.kv_append_e4m3(qg, k.to(DEV), v.to(DEV), pos.to(DEV), slots.to(DEV), kvg, 5e5, ks,
                        vs, device_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     qo = q.clone()
     oracle.kv_append_e4m3(qo, k.clone(), v.clone(), pos, slots, kc, vc, 5e5, ks, vs)
-    assert torch.equal(kcg.cpu(), kc), f"k codes differ at {(kcg.cpu() != kc).nonzero()[:4].tolist()}"
-    assert torch.equal(vcg.cpu(), vc), f"v codes differ at {(vcg.cpu() != vc).nonzero()[:4].tolist()}"
+    kcg, vcg = (h.cpu() for h in e4m3_halves(kvg))
+    assert torch.equal(kcg, kc), f"k codes differ at {(kcg != kc).nonzero()[:4].tolist()}"
+    assert torch.equal(vcg, vc), f"v codes differ at {(vcg != vc).nonzero()[:4].tolist()}"
     dq = (qg.cpu().double() - qo.double()).abs()
     bound = ulp_bf16(qo.double()) if dtype == torch.bfloat16 else 1e-6 * qo.double().abs() + 1e-30
     assert (dq <= bound).all(), "rotated q"
@@ -111,15 +113,15 @@ def test_kv_append_e4m3_slot_out_of_range():
     T, Hq, Hkv, d, NB = 2, 8, 2, 64, 4
     q = torch.randn(T, Hq, d, device=DEV).to(torch.bfloat16)
     k = torch.randn(T, Hkv, d, device=DEV).to(torch.bfloat16)
-    kc = torch.zeros(NB, Hkv, BS, d, dtype=torch.uint8, device=DEV)
-    vc = torch.zeros(NB, Hkv, d, BS, dtype=torch.uint8, device=DEV)
+    kv = torch.zeros(NB, Hkv, 2, BS * d, dtype=torch.uint8, device=DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
     slots = torch.tensor([NB * BS, 5], dtype=torch.int64, device=DEV)
     pos = torch.tensor([1, 2], dtype=torch.int64, device=DEV)
-    pkv.kv_append_e4m3(q, k, k.clone(), pos, slots, kc, vc, 1e4, 0.05, 0.05, device_error=err)
+    pkv.kv_append_e4m3(q, k, k.clone(), pos, slots, kv, 1e4, 0.05, 0.05, device_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) & pkv.DEVERR_SLOT
-    assert kc[0, :, 5].any() and not kc[1:].any()
+    kc, vc = e4m3_halves(kv)
+    assert kc[0, :, 5].any() and vc[0, :, :, 5].any() and not kv[1:].any()
 
 
 @pytest.mark.parametrize("d,G,P,cluster", [
@@ -139,9 +141,9 @@ def test_decode_e4m3_matches_oracle(d, G, P, cluster, out_dtype):
     ks, vs, scale = 1 / 16, 1 / 16, 1 / math.sqrt(d)
     out = torch.empty(B, Hkv * G, d, dtype=out_dtype, device=DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
-    pkv.paged_attention_decode_e4m3(q.to(DEV), kc.to(DEV), vc.to(DEV), tables.to(DEV), cl.to(DEV),
-                                    scale, ks, vs, out, partition_tokens=P, cluster=cluster,
-                                    device_error=err)
+    pkv.paged_attention_decode_e4m3(q.to(DEV), e4m3_pack(kc, vc).to(DEV), tables.to(DEV),
+                                    cl.to(DEV), scale, ks, vs, out, partition_tokens=P,
+                                    cluster=cluster, device_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     want = oracle.paged_attention_decode_e4m3(q, kc, vc, tables, cl, scale, ks, vs, nthreads=8)
@@ -155,7 +157,7 @@ def test_decode_e4m3_cluster_modes_agree():
     kc, vc, tables = _cache(lens, Hkv, d, seed=610)
     q = torch.randn(1, Hkv * G, d, generator=_gen(611)).to(torch.bfloat16)
     cl = torch.tensor(lens, dtype=torch.int32)
-    args = [t.to(DEV) for t in (q, kc, vc, tables, cl)]
+    args = [t.to(DEV) for t in (q, e4m3_pack(kc, vc), tables, cl)]
     outs = []
     for cluster in (True, False):
         out = torch.empty(1, Hkv * G, d, dtype=torch.float32, device=DEV)
@@ -185,17 +187,18 @@ def test_e4m3_append_then_decode_ragged_batch():
                          dtype=torch.int64)
     cl = torch.tensor([L + 1 for L in lens], dtype=torch.int32)
     ks, vs, theta, scale = 1 / 16, 1 / 16, 5e5, 0.125
-    qg, kcg, vcg = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    qg, kvg = q.to(DEV), e4m3_pack(kc, vc).to(DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
-    pkv.kv_append_e4m3(qg, kn.to(DEV), vn.to(DEV), pos.to(DEV), slots.to(DEV), kcg, vcg, theta,
+    pkv.kv_append_e4m3(qg, kn.to(DEV), vn.to(DEV), pos.to(DEV), slots.to(DEV), kvg, theta,
                        ks, vs, device_error=err)
     out = torch.empty(B, Hkv * G, d, dtype=torch.float32, device=DEV)
-    pkv.paged_attention_decode_e4m3(qg, kcg, vcg, tables.to(DEV), cl.to(DEV), scale, ks, vs, out,
+    pkv.paged_attention_decode_e4m3(qg, kvg, tables.to(DEV), cl.to(DEV), scale, ks, vs, out,
                                     device_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     qo, kco, vco = q.clone(), kc.clone(), vc.clone()
     oracle.kv_append_e4m3(qo, kn.clone(), vn.clone(), pos, slots, kco, vco, theta, ks, vs)
-    assert torch.equal(kcg.cpu(), kco) and torch.equal(vcg.cpu(), vco), "appended codes"
+    kcg, vcg = (h.cpu() for h in e4m3_halves(kvg))
+    assert torch.equal(kcg, kco) and torch.equal(vcg, vco), "appended codes"
     want = oracle.paged_attention_decode_e4m3(qo, kco, vco, tables, cl, scale, ks, vs, nthreads=16)
     _check(out, want, "ragged batch step")

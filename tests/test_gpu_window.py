@@ -111,7 +111,8 @@ def test_window_e4m3_matches_oracle(d, W, P):
     q = torch.randn(len(LENS), Hkv * G, d, generator=g).to(torch.bfloat16)
     cl = torch.tensor(LENS, dtype=torch.int32)
     out = torch.empty(len(LENS), Hkv * G, d, dtype=torch.float32, device=DEV)
-    pkv.paged_attention_decode_e4m3(q.to(DEV), kc_gpu.to(DEV), vc_gpu.to(DEV), tables.to(DEV),
+    from paged_kv_cache_484_b200.workloads import e4m3_pack
+    pkv.paged_attention_decode_e4m3(q.to(DEV), e4m3_pack(kc_gpu, vc_gpu).to(DEV), tables.to(DEV),
                                     cl.to(DEV), d ** -0.5, 1 / 16, 1 / 16, out,
                                     partition_tokens=P, sliding_window=W)
     torch.cuda.synchronize()
