@@ -77,10 +77,11 @@ def parse_args(argv=None):
                     help="device-side copies of the workload (0: enough to exceed L2)")
     ap.add_argument("--simt", action="store_true", help="bf16: CUDA-core decode kernel")
     ap.add_argument("--window", type=int, default=0,
-                    help="sliding window: each query attends to the last W tokens (two calls)")
+                    help="sliding window: each query attends to the last W tokens")
     ap.add_argument("--kv-dtype", default="native", choices=["native", "e4m3"],
                     help="e4m3: the workload's cache as an 8-bit cache (per-tensor scales), "
-                         "stepped as kv_append_e4m3 + paged_attention_decode_e4m3")
+                         "stepped by decode_step_e4m3 (kv_append_e4m3 + "
+                         "paged_attention_decode_e4m3 with --two-calls)")
     ap.add_argument("--two-calls", action="store_true",
                     help="time kv_append + paged_attention_decode as two launches instead of "
                          "the single-launch decode_step")
@@ -295,7 +296,8 @@ def config_block(cfg, w, out_dtype, P, NP, simt, two_calls=False):
             "kv_scales": list(w.meta.get("e4m3_scales", ())),
             "out_dtype": "bf16" if out_dtype == torch.bfloat16 else "f32",
             "partition_tokens": P, "max_partitions": NP, "decode_kernel": "mma_f16 (e4m3 pages)",
-            "step": "two calls (kv_append_e4m3, paged_attention_decode_e4m3)",
+            "step": "two calls (kv_append_e4m3, paged_attention_decode_e4m3)" if two_calls
+                    else "one launch (decode_step_e4m3: append fused into the decode kernel)",
         }
     return {
         "workload": name,
@@ -463,7 +465,6 @@ def measure(cfg, args, device, world, local, rank, full: bool):
         w.v_cache = w.k_cache
         del k8, v8
         w.meta["e4m3_scales"] = (ks8, vs8)
-        two_calls = True
         torch.cuda.empty_cache()
     kv_dt = torch.uint8 if e4m3 else w.dtype
     host_inputs = None
@@ -487,10 +488,8 @@ def measure(cfg, args, device, world, local, rank, full: bool):
     ws = pkv.new_workspace(ws_bytes, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     nbytes = step_bytes(w, out_dtype, args.window)
-    if args.window:
-        if args.cascade:
-            raise SystemExit("--window and --cascade do not combine")
-        two_calls = True
+    if args.window and args.cascade:
+        raise SystemExit("--window and --cascade do not combine")
 
     K = args.steps
     Wu = max(3, args.warmup)
@@ -540,15 +539,23 @@ def measure(cfg, args, device, world, local, rank, full: bool):
     launches_per_step = kernels_per_decode + (0 if fused else 1)
 
     def append(c):
+        if fused:
+            return
         if e4m3:
             pkv.kv_append_e4m3(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                                c["k_cache"], w.rope_theta, ks8, vs8, device_error=err)
-        elif not fused:
+        else:
             pkv.kv_append(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                           c["k_cache"], c["v_cache"], w.rope_theta, device_error=err)
 
     def decode(c, out):
-        if e4m3:
+        if e4m3 and fused:
+            pkv.decode_step_e4m3(c["q"], c["k_new"], c["v_new"], c["positions"],
+                                 c["slot_mapping"], c["k_cache"], c["block_tables"],
+                                 c["decode_lens"], w.rope_theta, w.scale, ks8, vs8, out,
+                                 workspace=ws, partition_tokens=P, device_error=err,
+                                 sliding_window=args.window)
+        elif e4m3:
             pkv.paged_attention_decode_e4m3(c["q"], c["k_cache"], c["block_tables"],
                                             c["decode_lens"], w.scale, ks8, vs8, out,
                                             workspace=ws, partition_tokens=P, device_error=err,
@@ -557,7 +564,7 @@ def measure(cfg, args, device, world, local, rank, full: bool):
             pkv.decode_step(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                             c["k_cache"], c["v_cache"], c["block_tables"], c["decode_lens"],
                             w.rope_theta, w.scale, out, workspace=ws, partition_tokens=P,
-                            force_simt=args.simt, device_error=err)
+                            force_simt=args.simt, device_error=err, sliding_window=args.window)
         elif cascade:
             pkv.paged_attention_decode_cascade(c["q"], c["k_cache"], c["v_cache"],
                                                c["block_tables"], c["decode_lens"], group_start,
@@ -637,7 +644,8 @@ def measure(cfg, args, device, world, local, rank, full: bool):
     def append_only(k):
         c = copies[k % ncopies]
         if e4m3:
-            append(c)
+            pkv.kv_append_e4m3(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
+                               c["k_cache"], w.rope_theta, ks8, vs8, device_error=err)
         else:
             pkv.kv_append(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                           c["k_cache"], c["v_cache"], w.rope_theta, device_error=err)

@@ -15,7 +15,8 @@
  * (pkv_paged_attention_decode_window); shared-prefix groups read once
  * (pkv_paged_attention_decode_cascade); chunked prefill
  * (pkv_paged_attention_prefill); an 8-bit E4M3 cache (pkv_kv_append_e4m3,
- * pkv_paged_attention_decode_e4m3); a decode without a caller workspace
+ * pkv_paged_attention_decode_e4m3, and the two in one launch,
+ * pkv_decode_step_e4m3); a decode without a caller workspace
  * (pkv_paged_attention_decode_noalloc); and a host-side block manager with
  * prefix reuse (pkv_bm_*).
  *
@@ -272,11 +273,12 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
  * "Inference From Scratch", ch. 4 and ch. 10 (the new token's K/V go into its
  * sequence's cache block, then the token attends to the whole cache).
  *
- * Token b of the append is sequence b's new token.  Every warp of the decode
- * kernel rotates the q elements it feeds to its own MMA fragments, and the
- * CTA that holds a sequence's last cache page rotates the new k, writes k and
- * v into the slot and patches them into the staged page, so no separate
- * append launch and no extra pass over memory is needed.  Here the angle is
+ * Token b of the append is sequence b's new token.  The decode kernel
+ * rotates each work item's staged q once in shared memory before its MMA
+ * fragments are built, and the CTA that holds a sequence's last cache page
+ * rotates the new k, writes k and v into the slot and patches them into the
+ * staged page, so no separate append launch and no extra pass over memory is
+ * needed.  Here the angle is
  * reduced mod 2pi in fp64 but its sine, cosine and the rotation are fp32,
  * rounded once to the storage type: within one storage ulp of the fp64 result
  * pkv_kv_append produces (bit-equal in the vast majority of elements).  q itself is only read:
@@ -455,6 +457,41 @@ pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* kv_cache,
                                            float scale, float k_scale, float v_scale,
                                            int32_t sliding_window, int32_t partition_tokens,
                                            uint32_t flags, int32_t* device_error, void* stream);
+
+/*
+ * pkv_decode_step_e4m3 -- pkv_decode_step over the 8-bit cache: the effect of
+ * pkv_kv_append_e4m3 (one new token per sequence, bf16 inputs) followed by
+ * pkv_paged_attention_decode_e4m3, in ONE launch.
+ *
+ * Source: "warpllama", Milestones (single-token decode with the attention
+ * hot path fused); "Efficient LLM Inference", Quantization (values stored as
+ * a small set of levels times a scale).
+ *
+ * The CTA that holds a sequence's last cache page rotates the new k in fp64
+ * and writes the new k and v codes into the slot and into the staged page
+ * exactly as pkv_kv_append_e4m3 computes them, so the cache bytes after the
+ * step equal those after the two calls.  q is only read: the kernel rotates
+ * its staged copy in fp32 (angle reduced in fp64) and rounds it to bf16, as
+ * the append would store it; the result is within one bf16 ulp of that q.  Preconditions, the handling of slots that differ
+ * from the table's, contexts of length 0 and every error are those of
+ * pkv_decode_step.
+ *
+ * Arguments: those of pkv_decode_step (q, k_new, v_new bf16, read only), with
+ *   kv_cache           device uint8, the layout above (16-byte aligned)
+ *   k_scale, v_scale   finite, > 0
+ *   sliding_window     0, or a window as in pkv_decode_step_window
+ * Size the workspace with kv_dtype PKV_DTYPE_E4M3.
+ */
+pkv_status pkv_decode_step_e4m3(void* q, const void* k_new, const void* v_new,
+                                const int64_t* positions, const int64_t* slot_mapping,
+                                void* kv_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, void* out, void* workspace,
+                                size_t workspace_bytes, int64_t num_seqs, int64_t num_q_heads,
+                                int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                                int64_t block_size, int64_t max_blocks_per_seq, int32_t out_dtype,
+                                double rope_theta, float scale, float k_scale, float v_scale,
+                                int32_t sliding_window, int32_t partition_tokens, uint32_t flags,
+                                int32_t* device_error, void* stream);
 
 /*
  * pkv_paged_attention_decode_window -- pkv_paged_attention_decode with a

@@ -28,7 +28,9 @@ from ._binding import (  # noqa: F401
     decode_launches,
     decode_partition_tokens,
     decode_step,
+    decode_step_e4m3,
     prepare_decode_step,
+    prepare_decode_step_e4m3,
     PreparedCall,
     decode_workspace_size,
     get_device_error,

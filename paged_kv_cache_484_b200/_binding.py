@@ -108,6 +108,11 @@ def load_library() -> ctypes.CDLL:
             i32, ctypes.c_float, i32, i32, u32, vp, vp]
         lib.pkv_paged_attention_decode_window.restype = ctypes.c_int
         lib.pkv_paged_attention_decode_e4m3.restype = ctypes.c_int
+        lib.pkv_decode_step_e4m3.argtypes = [
+            vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64,
+            i64, i64, i32, ctypes.c_double, ctypes.c_float, ctypes.c_float, ctypes.c_float, i32,
+            i32, u32, vp, vp]
+        lib.pkv_decode_step_e4m3.restype = ctypes.c_int
         lib.pkv_kv_request_bytes.argtypes = [i64, i64, i64, i64, i64, i32]
         lib.pkv_kv_request_bytes.restype = i64
         lib.pkv_kv_admission_capacity.argtypes = [i64, i64, i64, i64, i64, i64, i32]
@@ -509,6 +514,77 @@ def prepare_decode_step(q, k_new, v_new, positions, slot_mapping, k_cache, v_cac
                                         out, stream, workspace, partition_tokens, force_simt,
                                         device_error, cluster)
     return PreparedCall(lib, lib.pkv_decode_step, args, "decode_step", keep, q.device)
+
+
+def _decode_step_e4m3_args(q, k_new, v_new, positions, slot_mapping, kv_cache, block_tables,
+                           context_lens, rope_theta, scale, k_scale, v_scale, out, stream,
+                           workspace, partition_tokens, device_error, cluster, sliding_window):
+    """Checked pkv_decode_step_e4m3 arguments (allocating a workspace if none
+    is given), and the tensors they point into."""
+    lib = load_library()
+    dv = q.device
+    B, Hq, d = q.shape
+    if kv_cache.dim() != 4:
+        raise ValueError("kv_cache must be [num_blocks, Hkv, 2, 16 * head_dim]")
+    NB, Hkv, two, pg = kv_cache.shape
+    bs = BLOCK_SIZE
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if two != 2 or pg != bs * d or out.shape != (B, Hq, d) \
+            or k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d) \
+            or positions.shape != (B,) or slot_mapping.shape != (B,) \
+            or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("inconsistent decode_step_e4m3 shapes")
+    if workspace is None:
+        need = lib.pkv_decode_workspace_size(B, Hq, Hkv, d, MB, bs, PKV_DTYPE_E4M3,
+                                             int(partition_tokens))
+        workspace = new_workspace(int(need), q.device)
+    err = (_dev(device_error, "device_error", torch.int32, on=dv)
+           if device_error is not None else None)
+    args = (_dev(q, "q", torch.bfloat16, on=dv), _dev(k_new, "k_new", torch.bfloat16, on=dv),
+            _dev(v_new, "v_new", torch.bfloat16, on=dv),
+            _dev(positions, "positions", torch.int64, on=dv),
+            _dev(slot_mapping, "slot_mapping", torch.int64, on=dv),
+            _dev(kv_cache, "kv_cache", torch.uint8, on=dv),
+            _dev(block_tables, "block_tables", torch.int32, on=dv),
+            _dev(context_lens, "context_lens", torch.int32, on=dv), _dev(out, "out", on=dv),
+            _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
+            B, Hq, Hkv, d, NB, bs, MB, _dtype_code(out.dtype), float(rope_theta), float(scale),
+            float(k_scale), float(v_scale), int(sliding_window), int(partition_tokens),
+            _flags(False, cluster), err, _stream_ptr(stream, q.device))
+    keep = (q, k_new, v_new, positions, slot_mapping, kv_cache, block_tables, context_lens, out,
+            workspace, device_error)
+    return lib, args, keep
+
+
+def decode_step_e4m3(q, k_new, v_new, positions, slot_mapping, kv_cache, block_tables,
+                     context_lens, rope_theta, scale, k_scale, v_scale, out, stream=None, *,
+                     workspace=None, partition_tokens=0, device_error=None, cluster=True,
+                     sliding_window=0) -> torch.Tensor:
+    """``kv_append_e4m3`` (one new token per sequence, bfloat16 q/k_new/v_new)
+    then ``paged_attention_decode_e4m3``, in one launch; the new codes equal
+    the append's.  q is read only.  See include/pkv.h, pkv_decode_step_e4m3."""
+    lib, args, _ = _decode_step_e4m3_args(q, k_new, v_new, positions, slot_mapping, kv_cache,
+                                          block_tables, context_lens, rope_theta, scale, k_scale,
+                                          v_scale, out, stream, workspace, partition_tokens,
+                                          device_error, cluster, sliding_window)
+    with _current(q.device):
+        st = lib.pkv_decode_step_e4m3(*args)
+    _raise(st, lib, "decode_step_e4m3")
+    return out
+
+
+def prepare_decode_step_e4m3(q, k_new, v_new, positions, slot_mapping, kv_cache, block_tables,
+                             context_lens, rope_theta, scale, k_scale, v_scale, out, stream=None,
+                             *, workspace, partition_tokens=0, device_error=None, cluster=True,
+                             sliding_window=0) -> PreparedCall:
+    """``decode_step_e4m3`` checked and marshalled once (see
+    ``prepare_decode_step``)."""
+    lib, args, keep = _decode_step_e4m3_args(q, k_new, v_new, positions, slot_mapping, kv_cache,
+                                             block_tables, context_lens, rope_theta, scale,
+                                             k_scale, v_scale, out, stream, workspace,
+                                             partition_tokens, device_error, cluster,
+                                             sliding_window)
+    return PreparedCall(lib, lib.pkv_decode_step_e4m3, args, "decode_step_e4m3", keep, q.device)
 
 
 def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, out,

@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_e4m3_kernel(
     __syncthreads();
 
     auto code2 = [](double a, double b, double scale) -> uint32_t {
-        return f32x2_to_e4m3x2(__double2float_rn(a / scale), __double2float_rn(b / scale));
+        return e4m3x2_scaled(a, b, scale);
     };
     for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
         if (idx >= nq && !write_kv) break;
@@ -239,11 +239,8 @@ __global__ void __launch_bounds__(kAppendThreadsMax) kv_append_e4m3_kernel(
             unpack16<T>(*reinterpret_cast<const uint4*>(src + c * E), x0);
             unpack16<T>(*reinterpret_cast<const uint4*>(src + HALF + c * E), x1);
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const double cs = s_cos[c * E + e], sn = s_sin[c * E + e];
-                y0[e] = x0[e] * cs - x1[e] * sn;
-                y1[e] = x1[e] * cs + x0[e] * sn;
-            }
+            for (int e = 0; e < E; ++e)
+                rope_rotate_f64(x0[e], x1[e], s_cos[c * E + e], s_sin[c * E + e], y0[e], y1[e]);
             if (is_q) {
                 T* dst = q + (t * p.Hq + h) * D;
                 *reinterpret_cast<uint4*>(dst + c * E) = pack16<T>(y0);

@@ -111,8 +111,10 @@ struct Layout {
         cmax(2, cmin(6, ((D == 128 && SWZ) ? 98304 : 65536) / STAGE_BYTES));
     static constexpr int Q_COPY = G * D * QSZ;
     static constexpr int Q_BYTES = round_up(Q_COPY, 128);
-    static constexpr int ROW_COPY = D * ESZ;           // one k or v row
-    static constexpr int NEWKV_BYTES = 2 * ROW_COPY;   // fused step: raw new k row, new v row
+    static constexpr int ROW_COPY = D * QSZ;           // one new k or v row (q's type)
+    // fused step: the raw new k row and v row, or (8-bit cache) their codes,
+    // computed by the producer
+    static constexpr int NEWKV_BYTES = F8 ? 2 * D : 2 * ROW_COPY;
     // Item merge: each warp leaves (o[D], m, l) per head in its own K and V
     // page slots of the item's last stage (free once it has read its pages),
     // or, where those are too small (8-bit d = 128 at G = 8), in a region of
@@ -173,6 +175,7 @@ struct DecodeParams {
     int num_blocks;
     float scale_log2;  // softmax scale x log2(e) (x k_scale for the 8-bit cache)
     float v_scale;     // 8-bit cache: V = code x v_scale; 1 otherwise
+    float k_scale;     // 8-bit cache: K = code x k_scale (the fused step's new codes)
     int out_bf16;
     // cluster mode: CS > 1 CTAs per (sequence, kv head), CTA rank r takes
     // partition r, and the cluster merges the partials in shared memory
@@ -185,12 +188,12 @@ struct DecodeParams {
     // sliding window: each query attends to the last `window` tokens of its
     // context (0 = the whole context)
     int window;
-    // fused step only: the new token of every sequence
+    // fused step only: the new token of every sequence (q's type)
     const void* k_new;            // [B, Hkv, D]
     const void* v_new;            // [B, Hkv, D]
     const int64_t* positions;     // [B]
     const int64_t* slot_mapping;  // [B]
-    void* k_cache;                // cache bases for the new rows
+    void* k_cache;                // cache bases for the new rows (8-bit: the [K | V] pages)
     void* v_cache;
 };
 
@@ -368,9 +371,58 @@ __device__ void patch_new_row(uint8_t* kpage, uint8_t* vpage, const uint8_t* new
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same for the 8-bit cache, whose codes the producer has computed
+// (k codes at newkv[0, D), v codes at newkv[D, 2D)) and already written to
+// the cache: copy them into row r of the staged K half (128-byte rows are
+// 128B-swizzled at d = 128) and column r of the transposed V half.
+template <int D>
+__device__ __forceinline__ void patch_new_codes(uint8_t* kpage, uint8_t* vpage,
+                                                const uint8_t* newkv, int r) {
+    const int lane = threadIdx.x & 31;
+    if (lane < D / 16) {
+        const int c = D == 128 ? (lane ^ (r & 7)) : lane;
+        *reinterpret_cast<uint4*>(kpage + r * D + c * 16) =
+            *reinterpret_cast<const uint4*>(newkv + lane * 16);
+    }
+    for (int i = lane; i < D; i += 32) vpage[i * kPageRows + r] = newkv[D + i];
+    __syncwarp();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Fused step, context length 0: no attention, but the new token's k (rotated)
 // and v still go into a valid slot, as kv_append would put them.  Run by the
 // consumer threads of one CTA.
+template <int D>
+__device__ void append_only_e4m3(const DecodeParams& p, const RopeFreq& fr, int b) {
+    constexpr int HALF = D / 2;
+    const double pos = (double)p.positions[b];
+    const int64_t slot = p.slot_mapping[b];
+    const int64_t num_slots = (int64_t)p.num_blocks * kPageRows;
+    if (slot >= num_slots && threadIdx.x == 0) report_error(p.err, PKV_DEVERR_SLOT);
+    if (slot < 0 || slot >= num_slots) return;
+    const uint16_t* kn = reinterpret_cast<const uint16_t*>(p.k_new) + (size_t)b * p.Hkv * D;
+    const uint16_t* vn = reinterpret_cast<const uint16_t*>(p.v_new) + (size_t)b * p.Hkv * D;
+    auto bf = [](uint16_t x) { return (double)__uint_as_float((uint32_t)x << 16); };
+    const int64_t blk = slot / kPageRows;
+    const int row = (int)(slot % kPageRows);
+    for (int idx = threadIdx.x; idx < p.Hkv * HALF; idx += NW * 32) {
+        const int h = idx / HALF, i = idx % HALF;
+        uint8_t* pg = reinterpret_cast<uint8_t*>(p.k_cache) + (blk * p.Hkv + h) * (2 * kPageRows * D);
+        double sn, cs, y0, y1;
+        sincos(reduce_two_pi(pos * fr.f[i]), &sn, &cs);
+        rope_rotate_f64(bf(kn[h * D + i]), bf(kn[h * D + i + HALF]), cs, sn, y0, y1);
+        const uint32_t c = e4m3x2_scaled(y0, y1, (double)p.k_scale);
+        pg[row * D + i] = (uint8_t)(c & 0xFFu);
+        pg[row * D + i + HALF] = (uint8_t)(c >> 8);
+    }
+    for (int idx = threadIdx.x; idx < p.Hkv * D; idx += NW * 32) {
+        const int h = idx / D, i = idx % D;
+        uint8_t* pg = reinterpret_cast<uint8_t*>(p.k_cache) + (blk * p.Hkv + h) * (2 * kPageRows * D);
+        pg[kPageRows * D + i * kPageRows + row] =
+            (uint8_t)(e4m3x2_scaled(bf(vn[h * D + i]), 0.0, (double)p.v_scale) & 0xFFu);
+    }
+}
+
 template <typename T, int D>
 __device__ void append_only(const DecodeParams& p, const RopeFreq& fr, int b) {
     constexpr int HALF = D / 2;
@@ -402,6 +454,44 @@ __device__ void append_only(const DecodeParams& p, const RopeFreq& fr, int b) {
 }
 
 // ---------------------------------------------------------------- producer
+
+// Fused step, 8-bit cache: one warp makes the new token's codes of
+// (sequence b, kv head h) exactly as the 8-bit append does (k rotated in
+// fp64, x / scale in fp64 rounded to binary32, nearest E4M3), writes them
+// into row `row` of the cache page `blk` and stages them at nk (k codes in
+// [0, D), v codes in [D, 2D)) for the consumers' patch.
+template <int D>
+__device__ __forceinline__ void make_new_codes(const DecodeParams& p, int b, int h, double pos,
+                                            const double (&f)[(D + 63) / 64], int row, int blk,
+                                            uint8_t* nk) {
+    constexpr int HALF = D / 2;
+    const int lane = threadIdx.x & 31;
+    const uint16_t* kn = reinterpret_cast<const uint16_t*>(p.k_new) + ((size_t)b * p.Hkv + h) * D;
+    const uint16_t* vn = reinterpret_cast<const uint16_t*>(p.v_new) + ((size_t)b * p.Hkv + h) * D;
+    uint8_t* gpage = reinterpret_cast<uint8_t*>(p.k_cache) +
+                     ((size_t)blk * p.Hkv + h) * (size_t)(2 * kPageRows * D);
+    auto bf = [](uint16_t x) { return (double)__uint_as_float((uint32_t)x << 16); };
+#pragma unroll
+    for (int u = 0; u < (D + 63) / 64; ++u) {
+        const int i = lane + 32 * u;
+        if (i < HALF) {
+            double sn, cs, y0, y1;
+            sincos(reduce_two_pi(pos * f[u]), &sn, &cs);
+            rope_rotate_f64(bf(kn[i]), bf(kn[i + HALF]), cs, sn, y0, y1);
+            const uint32_t c = e4m3x2_scaled(y0, y1, (double)p.k_scale);
+            nk[i] = (uint8_t)(c & 0xFFu);
+            nk[i + HALF] = (uint8_t)(c >> 8);
+            gpage[row * D + i] = (uint8_t)(c & 0xFFu);
+            gpage[row * D + i + HALF] = (uint8_t)(c >> 8);
+        }
+    }
+    for (int i = lane; i < D; i += 32) {
+        const uint8_t c = (uint8_t)(e4m3x2_scaled(bf(vn[i]), 0.0, (double)p.v_scale) & 0xFFu);
+        nk[D + i] = c;
+        gpage[kPageRows * D + i * kPageRows + row] = c;
+    }
+}
+
 
 // Reads the producer issues before the context lengths are known, for the
 // first item this CTA would get if every sequence had NP partitions (exact
@@ -575,7 +665,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
             // stage's one arrival.
             if (lane == 0) {
                 const uint32_t bytes = __popc(vmask) * 2u * L::PAGE_BYTES +
-                                       (patch_row >= 0 ? (uint32_t)L::NEWKV_BYTES : 0u);
+                                       ((patch_row >= 0 && !L::F8) ? (uint32_t)L::NEWKV_BYTES : 0u);
                 mbar_expect_tx(&full[stage], bytes);
             }
             __syncwarp();
@@ -608,7 +698,15 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
                 mbar_expect_tx(&qbar[stage], L::Q_COPY);
                 bulk_load(base + L::OFF_Q + stage * L::Q_BYTES, qsrc, L::Q_COPY, &qbar[stage]);
             }
-            if (FUSED && patch_row >= 0 && lane == 1) {
+            if constexpr (FUSED && L::F8) {
+                // 8-bit cache: this warp makes the new token's codes exactly
+                // as the 8-bit append does (k rotated in fp64, x / scale in
+                // fp64 rounded to binary32, nearest E4M3), writes them to the
+                // cache and stages them for the consumers' patch
+                if (patch_row >= 0)
+                    make_new_codes<D>(p, cur.b, cur.h, (double)cur_pos, guess.f, patch_row,
+                                      patch_blk, base + L::OFF_NEWKV + stage * L::NEWKV_BYTES);
+            } else if (FUSED && patch_row >= 0 && lane == 1) {
                 const size_t row_off = ((size_t)cur.b * p.Hkv + cur.h) * L::ROW_COPY;
                 uint8_t* nk = base + L::OFF_NEWKV + stage * L::NEWKV_BYTES;
                 bulk_load(nk, reinterpret_cast<const uint8_t*>(p.k_new) + row_off, L::ROW_COPY,
@@ -617,9 +715,10 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
                           L::ROW_COPY, &full[stage]);
             }
             if constexpr (FUSED) {
-                // the rope table rides with the item's first stage and with
-                // the stage that carries the new token
-                if (first || patch_row >= 0)
+                // the rope table rides with the item's first stage (q) and,
+                // for the bf16 / fp32 caches, with the stage that carries the
+                // new token (its k)
+                if (first || (!L::F8 && patch_row >= 0))
                     warp_rope_table<D>((double)cur_pos, guess.f,
                                        reinterpret_cast<float*>(base + L::OFF_ROPE +
                                                                 stage * L::ROPE_BYTES));
@@ -814,9 +913,19 @@ __device__ __forceinline__ void item_patch_page(const DecodeParams& p, const Ite
                                                 int slot, int stage, uint8_t* base) {
     if constexpr (FUSED) {
         using L = Layout<T, D, G>;
+        // only the last page of a sequence's last partition can carry the
+        // new token: test that (registers) before reading the stage's record
+        if (j != it.npages - 1 || it.part != it.np - 1) return;
         const float* tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
         const int* pt = reinterpret_cast<const int*>(base + L::OFF_PATCH) + 2 * stage;
-        if (pt[0] >= 0 && j == it.npages - 1) {
+        if constexpr (L::F8) {
+            if (pt[0] >= 0) {
+                uint8_t* kpage = base + stage * L::STAGE_BYTES + slot * L::KPITCH;
+                patch_new_codes<D>(kpage, kpage + L::VOFF,
+                                   base + L::OFF_NEWKV + stage * L::NEWKV_BYTES, pt[0]);
+            }
+            return;
+        } else if (pt[0] >= 0) {
             const int row = pt[0];
             const size_t grow = (((size_t)pt[1] * p.Hkv + it.h) * kPageRows + row) * D;
             uint8_t* kpage = base + stage * L::STAGE_BYTES + slot * L::KPITCH;
@@ -851,7 +960,6 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
                                  const int* s_pre, int W) {
     using L = Layout<T, D, G>;
     constexpr bool F8 = L::F8;
-    static_assert(!(F8 && FUSED), "the fused step takes bf16 or fp32 caches");
     constexpr int KS = D / 16;  // k-steps of the score MMA
     constexpr int NT = D / 8;   // n-tiles of the output MMA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -890,8 +998,28 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
         float m_run = kNegInf, l_run = 0.f;
         uint32_t qa[KS][4];
         tab = reinterpret_cast<const float*>(base + L::OFF_ROPE + stage * L::ROPE_BYTES);
-        // A fragments of Q: rows = query heads (see head_a/head_b), cols = dims.
         const uint8_t* qs = base + L::OFF_Q + stage * L::Q_BYTES;
+        if constexpr (FUSED) {
+            // The staged q is the raw input.  The consumer threads rotate it
+            // in place once (thread t takes the pairs t, t + 128, ...), each
+            // element rounded to bf16 as the append would store it, and meet
+            // before any fragment is read.  The rotated q never leaves shared
+            // memory.
+            constexpr int HALF = D / 2;
+            bf16* qrow = reinterpret_cast<bf16*>(base + L::OFF_Q + stage * L::Q_BYTES);
+            for (int idx = warp * 32 + lane; idx < G * HALF; idx += NW * 32) {
+                const int g = idx / HALF, i = idx - g * HALF;
+                bf16* row = qrow + g * D;
+                const float x = __bfloat162float(row[i]), y = __bfloat162float(row[i + HALF]);
+                const float c = tab[i], sn = tab[HALF + i];
+                row[i] = __float2bfloat16_rn(fmaf(x, c, -y * sn));
+                row[i + HALF] = __float2bfloat16_rn(fmaf(y, c, x * sn));
+            }
+            // the buffer's next writer is a bulk copy (async proxy)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (!consumer_sync(p, merge_bar, mphase, s_abort)) return -1;
+        }
+        // A fragments of Q: rows = query heads (see head_a/head_b), cols = dims.
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
             const int col = kk * 16 + 2 * cq;
@@ -899,35 +1027,19 @@ __device__ int run_consumer_mma(const DecodeParams& p, const RopeFreq& fr, uint8
             if constexpr (F8) {
                 // dims (D/4) cq + 4 kk .. +3 of the head, as two f16 pairs
                 auto quad = [&](int head, uint32_t& lo, uint32_t& hi) {
-                    const uint2 v = *reinterpret_cast<const uint2*>(
-                        qs + (head * D + (D / 4) * cq + 4 * kk) * 2);
+                    const int c = (D / 4) * cq + 4 * kk;
+                    const uint2 v = *reinterpret_cast<const uint2*>(qs + (head * D + c) * 2);
                     lo = pack_f16(bf16lo(v.x), bf16hi(v.x));
                     hi = pack_f16(bf16lo(v.y), bf16hi(v.y));
                 };
                 if (head_a >= 0) quad(head_a, a0, a2);
                 if (head_b >= 0) quad(head_b, a1, a3);
-            } else if (FUSED) {
-                // the staged q is the raw (unrotated) input: rotate the
-                // lane's own elements on the way into the fragment
-                auto pair = [&](int head, int c) -> uint32_t {
-                    const bf16* row = reinterpret_cast<const bf16*>(qs + head * D * 2);
-                    return pack_bf16(rotated_elem<bf16, D>(row, c, tab),
-                                     rotated_elem<bf16, D>(row, c + 1, tab));
-                };
-                if (head_a >= 0) {
-                    a0 = pair(head_a, col);
-                    a2 = pair(head_a, col + 8);
-                }
-                if (head_b >= 0) {
-                    a1 = pair(head_b, col);
-                    a3 = pair(head_b, col + 8);
-                }
             } else if (head_a >= 0) {
                 const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_a * D * 2);
                 a0 = qr[col / 2];
                 a2 = qr[(col + 8) / 2];
             }
-            if (!F8 && !FUSED && head_b >= 0) {
+            if (!F8 && head_b >= 0) {
                 const uint32_t* qr = reinterpret_cast<const uint32_t*>(qs + head_b * D * 2);
                 a1 = qr[col / 2];
                 a3 = qr[(col + 8) / 2];
@@ -1396,7 +1508,9 @@ __device__ int run_consumer_simt(const DecodeParams& p, const RopeFreq& fr, uint
 
 // Register budget: the d = 64 tensor-core kernels must fit three CTAs per SM
 // (their shared-memory ring allows it), i.e. at most 128 registers a thread;
-// the others are limited to two CTAs by shared memory anyway.
+// the others run two CTAs per SM, which allows 168: ten warps spread over
+// four SM sub-partitions put three on some, and 3 x 32 x 168 registers fit
+// a sub-partition's 16384 (at 176 they would not, and only one CTA fits).
 template <bool MMA, int D>
 constexpr int decode_max_regs() { return (MMA && D == 64) ? 128 : 168; }
 
@@ -1577,7 +1691,10 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
             if (s_len[b] != 0) continue;
             for (int idx = tid; idx < p.Hq * D; idx += NW * 32)
                 store_out(p.out, (size_t)b * p.Hq * D + idx, 0.f, p.out_bf16);
-            if constexpr (FUSED) append_only<T, D>(p, fr, b);
+            if constexpr (FUSED) {
+                if constexpr (L::F8) append_only_e4m3<D>(p, fr, b);
+                else append_only<T, D>(p, fr, b);
+            }
         }
         int merged;
         if constexpr (MMA) {
@@ -1868,6 +1985,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
     p.num_blocks = (int)a.num_blocks;
     p.scale_log2 = a.scale * 1.4426950408889634f * (L::F8 ? a.k_scale : 1.0f);
     p.v_scale = L::F8 ? a.v_scale : 1.0f;
+    p.k_scale = L::F8 ? a.k_scale : 1.0f;
     p.out_bf16 = a.out_dtype == PKV_DTYPE_BF16;
     p.k_new = a.k_new;
     p.v_new = a.v_new;
@@ -1976,12 +2094,8 @@ cudaError_t dispatch_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensor
 template <bool FUSED>
 cudaError_t dispatch_all(const DecodeArgs& a, const CUtensorMap& tmk, const CUtensorMap& tmv) {
     if (a.kv_dtype == PKV_DTYPE_E4M3) {
-        if constexpr (FUSED) {
-            return cudaErrorInvalidValue;  // the fused step takes bf16 or fp32 caches
-        } else {
-            return a.D == 64 ? dispatch_g<e4m3kv, 64, true, false>(a, tmk, tmv)
-                             : dispatch_g<e4m3kv, 128, true, false>(a, tmk, tmv);
-        }
+        return a.D == 64 ? dispatch_g<e4m3kv, 64, true, FUSED>(a, tmk, tmv)
+                         : dispatch_g<e4m3kv, 128, true, FUSED>(a, tmk, tmv);
     }
     if (a.kv_dtype == PKV_DTYPE_F32) {
         return a.D == 64 ? dispatch_g<float, 64, false, FUSED>(a, tmk, tmv)

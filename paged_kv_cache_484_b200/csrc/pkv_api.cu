@@ -362,7 +362,7 @@ int32_t pkv_decode_launches(int64_t num_seqs, int64_t num_q_heads, int64_t num_k
     if (num_seqs <= 0 || max_blocks_per_seq <= 0 || !valid_kv_dtype(kv_dtype) ||
         !valid_dtype(out_dtype) || (flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_NO_CLUSTER)))
         return 0;
-    if (kv_dtype == PKV_DTYPE_E4M3 && (fused || (flags & PKV_DECODE_FORCE_SIMT))) return 0;
+    if (kv_dtype == PKV_DTYPE_E4M3 && (flags & PKV_DECODE_FORCE_SIMT)) return 0;
     if (num_seqs > PKV_MAX_SEQS_PER_CALL) return 0;
     if (check_heads(num_q_heads, num_kv_heads, head_dim, block_size) != PKV_OK) return 0;
     WorkspacePlan w;
@@ -430,8 +430,8 @@ pkv_status decode_common(const void* q, const void* k_cache, const void* v_cache
         return PKV_ERR_UNSUPPORTED;
     }
     if (kv_dtype == PKV_DTYPE_E4M3) {
-        if (step || (flags & PKV_DECODE_FORCE_SIMT)) {
-            set_last_error("the 8-bit cache has no fused step and no CUDA-core kernel");
+        if (flags & PKV_DECODE_FORCE_SIMT) {
+            set_last_error("the 8-bit cache has no CUDA-core kernel");
             return PKV_ERR_UNSUPPORTED;
         }
         for (int i = 0; i < 2; ++i)
@@ -619,6 +619,26 @@ pkv_status pkv_paged_attention_decode_e4m3(const void* q, const void* kv_cache,
                          workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
                          num_blocks, block_size, max_blocks_per_seq, PKV_DTYPE_E4M3, out_dtype,
                          scale, partition_tokens, flags, device_error, stream, nullptr, scales,
+                         sliding_window);
+}
+
+pkv_status pkv_decode_step_e4m3(void* q, const void* k_new, const void* v_new,
+                                const int64_t* positions, const int64_t* slot_mapping,
+                                void* kv_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, void* out, void* workspace,
+                                size_t workspace_bytes, int64_t num_seqs, int64_t num_q_heads,
+                                int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                                int64_t block_size, int64_t max_blocks_per_seq, int32_t out_dtype,
+                                double rope_theta, float scale, float k_scale, float v_scale,
+                                int32_t sliding_window, int32_t partition_tokens, uint32_t flags,
+                                int32_t* device_error, void* stream) {
+    set_last_error("");
+    const float scales[2] = {k_scale, v_scale};
+    const StepExtras step = {k_new, v_new, positions, slot_mapping, rope_theta};
+    return decode_common(q, kv_cache, kv_cache, block_tables, context_lens, out, workspace,
+                         workspace_bytes, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                         num_blocks, block_size, max_blocks_per_seq, PKV_DTYPE_E4M3, out_dtype,
+                         scale, partition_tokens, flags, device_error, stream, &step, scales,
                          sliding_window);
 }
 

@@ -362,6 +362,22 @@ __device__ __forceinline__ uint16_t double_to_bf16_bits(double x) {
     return r;
 }
 
+// RoPE rotation of one pair (x0, x1) = (x[i], x[i + d/2]) in fp64 by the
+// angle whose cosine and sine are (cs, sn); every product and sum is rounded
+// on its own (no fused multiply-add), as the plain formula states.
+__device__ __forceinline__ void rope_rotate_f64(double x0, double x1, double cs, double sn,
+                                                double& y0, double& y1) {
+    y0 = __dsub_rn(__dmul_rn(x0, cs), __dmul_rn(x1, sn));
+    y1 = __dadd_rn(__dmul_rn(x1, cs), __dmul_rn(x0, sn));
+}
+// 8-bit cache codes of two values: x / scale in fp64, rounded once to
+// binary32, then to the nearest E4M3 code (saturating); the first value's
+// code in bits 0-7, the second's in bits 8-15.
+__device__ __forceinline__ uint32_t e4m3x2_scaled(double a, double b, double scale) {
+    return f32x2_to_e4m3x2(__double2float_rn(__ddiv_rn(a, scale)),
+                           __double2float_rn(__ddiv_rn(b, scale)));
+}
+
 // RoPE angle reduction: x - k*2pi with k = rint(x / 2pi), by Cody and
 // Waite's method with 2pi split into three doubles (2pi = C1 + C2 + C3 to
 // ~160 bits; constants computed here from a high-precision 2pi) and one fused

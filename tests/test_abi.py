@@ -189,14 +189,43 @@ def test_decode_window_rejects_bad_arguments(lib, kw, status):
 
 def test_e4m3_planning(lib):
     """The planning calls take the 8-bit cache dtype: the workspace follows
-    the same formula; the fused step and the CUDA-core kernel do not exist
-    for it."""
+    the same formula; the CUDA-core kernel does not exist for it."""
     for P in (0, 64, 1024):
         assert lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, E4M3, P) == \
             lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, BF16, P)
     assert lib.pkv_decode_partition_tokens(64, 32, 8, 64, 257, 16, E4M3) > 0
-    assert lib.pkv_decode_launches(4, 32, 8, 64, 16, 16, E4M3, BF16, 0, 0, 1) == 0
     assert lib.pkv_decode_launches(4, 32, 8, 64, 16, 16, E4M3, BF16, 0, 1, 0) == 0
+
+
+def _step8(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, slot=FAKE, kv=FAKE, bt=FAKE, cl=FAKE, out=FAKE,
+             ws=None, wsb=0, B=2, Hq=8, Hkv=2, d=64, NB=4, bs=16, MB=4, odt=BF16, theta=1e4,
+             scale=0.125, ks=0.05, vs=0.05, win=0, P=0, flags=0, err=None)
+    a.update(kw)
+    return lib.pkv_decode_step_e4m3(
+        a["q"], a["k"], a["v"], a["pos"], a["slot"], a["kv"], a["bt"], a["cl"], a["out"],
+        a["ws"], a["wsb"], a["B"], a["Hq"], a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"],
+        a["odt"], a["theta"], a["scale"], a["ks"], a["vs"], a["win"], a["P"], a["flags"],
+        a["err"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ks=0.0), INVALID),
+    (dict(vs=math.inf), INVALID),
+    (dict(theta=0.0), INVALID),
+    (dict(flags=0x1), UNSUPPORTED),        # no CUDA-core kernel for the 8-bit cache
+    (dict(odt=E4M3), UNSUPPORTED),
+    (dict(d=96), UNSUPPORTED),
+    (dict(P=16, MB=4), WORKSPACE),
+    (dict(kv=FAKE + 4), INVALID),
+    (dict(k=FAKE + 8), INVALID),
+    (dict(pos=FAKE + 4), INVALID),
+    (dict(slot=None), INVALID),
+    (dict(win=-1), INVALID),
+    (dict(B=0, q=None, out=None), OK),
+])
+def test_decode_step_e4m3_rejects_bad_arguments(lib, kw, status):
+    assert _step8(lib, **kw) == status
 
 def test_workspace_size_formula(lib):
     # 16 sequences, 32/8 heads, d 128, contexts up to 8193 blocks, P = 1024

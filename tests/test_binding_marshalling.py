@@ -141,6 +141,15 @@ def _cases():
         "pkv_paged_attention_decode_e4m3",
         ["q", "kv_cache", "block_tables", "context_lens", "out", "workspace"]))
 
+    a = dict(_step_args(), kv_cache=_t((NB, Hkv, 2, 16 * D), u8), workspace=ws(), err=err())
+    cases.append(("decode_step_e4m3", lambda a=a: B.decode_step_e4m3(
+        a["q"], a["k_new"], a["v_new"], a["positions"], a["slot_mapping"], a["kv_cache"],
+        a["block_tables"], a["context_lens"], 1e4, 0.125, 0.05, 0.05, a["out"],
+        workspace=a["workspace"], device_error=a["err"], sliding_window=48), a,
+        "pkv_decode_step_e4m3",
+        ["q", "k_new", "v_new", "positions", "slot_mapping", "kv_cache", "block_tables",
+         "context_lens", "out", "workspace"]))
+
     a = dict(_decode_args(), q=_t((Bs, C, Hq, D), bf16), out=_t((Bs, C, Hq, D), f32),
              workspace=ws(), err=err())
     cases.append(("paged_attention_prefill", lambda a=a: B.paged_attention_prefill(
@@ -203,3 +212,17 @@ def test_fused_window_step_passes_the_window_before_the_partition_length(rec):
     args = [c for c in rec.calls if c[0] == "pkv_decode_step_window"][0][1]
     # ..., rope_theta, scale, sliding_window, partition_tokens, flags, device_error, stream
     assert args[-7:-3] == (1e4, 0.125, 33, 48)
+
+
+def test_e4m3_step_passes_scales_and_window_in_declared_order(rec):
+    a = dict(_step_args(), kv_cache=_t((NB, Hkv, 2, 16 * D), u8), workspace=_t((4096,), u8))
+    B.decode_step_e4m3(a["q"], a["k_new"], a["v_new"], a["positions"], a["slot_mapping"],
+                       a["kv_cache"], a["block_tables"], a["context_lens"], 5e5, 0.125, 0.25,
+                       0.5, a["out"], workspace=a["workspace"], sliding_window=48,
+                       partition_tokens=64)
+    (name, args), = rec.calls
+    assert name == "pkv_decode_step_e4m3"
+    # ... out, workspace, bytes, B, Hq, Hkv, d, NB, bs, MB, out_dtype, theta, scale,
+    # k_scale, v_scale, window, P, flags, device_error, stream
+    assert list(args[10:]) == [4096, Bs, Hq, Hkv, D, NB, 16, MB, 0, 5e5, 0.125, 0.25, 0.5, 48,
+                               64, 0, None, 0]

@@ -202,3 +202,143 @@ def test_e4m3_append_then_decode_ragged_batch():
     assert torch.equal(kcg, kco) and torch.equal(vcg, vco), "appended codes"
     want = oracle.paged_attention_decode_e4m3(qo, kco, vco, tables, cl, scale, ks, vs, nthreads=16)
     _check(out, want, "ragged batch step")
+
+
+def _step_case(lens, Hkv, G, d, seed):
+    """Inputs of one decode step over the 8-bit cache: context lens[b]
+    includes the new token L - 1, whose slot is the one the table gives it."""
+    kc, vc, tables = _cache(lens, Hkv, d, seed=seed)
+    g = _gen(seed + 1)
+    B = len(lens)
+    q = torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16)
+    kn = (torch.randn(B, Hkv, d, generator=g) * 1.5).to(torch.bfloat16)
+    vn = (torch.randn(B, Hkv, d, generator=g) * 1.5).to(torch.bfloat16)
+    pos = torch.tensor([max(L - 1, 0) + 7 * b for b, L in enumerate(lens)], dtype=torch.int64)
+    slots = torch.tensor([int(tables[b, (L - 1) // BS]) * BS + (L - 1) % BS if L > 0 else -1
+                          for b, L in enumerate(lens)], dtype=torch.int64)
+    cl = torch.tensor(lens, dtype=torch.int32)
+    return kc, vc, tables, q, kn, vn, pos, slots, cl
+
+
+def _oracle_step(kc, vc, tables, q, kn, vn, pos, slots, cl, theta, scale, ks, vs, window=0):
+    qo, kco, vco = q.clone(), kc.clone(), vc.clone()
+    oracle.kv_append_e4m3(qo, kn.clone(), vn.clone(), pos, slots, kco, vco, theta, ks, vs)
+    if window:
+        want = oracle.paged_attention_decode_e4m3(qo, kco, vco, tables, cl, scale, ks, vs,
+                                                  nthreads=8, window=window)
+    else:
+        want = oracle.paged_attention_decode_e4m3(qo, kco, vco, tables, cl, scale, ks, vs,
+                                                  nthreads=8)
+    return kco, vco, want
+
+
+@pytest.mark.parametrize("d,G,P,cluster", [
+    (64, 4, 0, True), (64, 4, 64, False), (64, 1, 16, False), (64, 8, 0, True),
+    (64, 2, 128, False), (128, 4, 0, True), (128, 8, 48, False), (128, 1, 0, True),
+    (128, 2, 256, False),
+])
+def test_decode_step_e4m3_matches_oracle(d, G, P, cluster):
+    """The one-launch step: the new codes in the cache equal the oracle
+    append's bit for bit, q is left as it was, and the output matches the
+    oracle's decode over the appended cache."""
+    lens = [1, 15, 16, 17, 300, 2049, 64, 5, 1000, 33]
+    Hkv = 2
+    kc, vc, tables, q, kn, vn, pos, slots, cl = _step_case(lens, Hkv, G, d, 640 + d + G + P)
+    ks, vs, theta, scale = 1 / 16, 1 / 12, 5e5, 1 / math.sqrt(d)
+    qg, kvg = q.to(DEV), e4m3_pack(kc, vc).to(DEV)
+    out = torch.full((len(lens), Hkv * G, d), float("nan"), device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.decode_step_e4m3(qg, kn.to(DEV), vn.to(DEV), pos.to(DEV), slots.to(DEV), kvg,
+                         tables.to(DEV), cl.to(DEV), theta, scale, ks, vs, out,
+                         partition_tokens=P, cluster=cluster, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    kco, vco, want = _oracle_step(kc, vc, tables, q, kn, vn, pos, slots, cl, theta, scale, ks, vs)
+    kcg, vcg = (h.cpu() for h in e4m3_halves(kvg))
+    assert torch.equal(kcg, kco), f"k codes differ at {(kcg != kco).nonzero()[:4].tolist()}"
+    assert torch.equal(vcg, vco), f"v codes differ at {(vcg != vco).nonzero()[:4].tolist()}"
+    assert torch.equal(qg.cpu(), q), "q must be read only"
+    _check(out, want, f"e4m3 step d{d} G{G} P{P} cluster{cluster}")
+
+
+def test_decode_step_e4m3_equals_two_calls_bytes():
+    """The 64-sequence ragged batch (32/8 heads, d 64, U[128, 4096]): the
+    fused step leaves the same cache bytes as kv_append_e4m3 and its output
+    agrees with the two-call decode within rounding; both match the oracle."""
+    g = _gen(650)
+    B, Hkv, G, d = 64, 8, 4, 64
+    lens = [L + 1 for L in torch.randint(128, 4097, (B,), generator=g).tolist()]
+    kc, vc, tables, q, kn, vn, pos, slots, cl = _step_case(lens, Hkv, G, d, 651)
+    ks, vs, theta, scale = 1 / 16, 1 / 16, 5e5, 0.125
+    dev = [t.to(DEV) for t in (q, kn, vn, pos, slots, tables, cl)]
+    qg, kng, vng, posg, slg, tg, clg = dev
+    kv1, kv2 = e4m3_pack(kc, vc).to(DEV), e4m3_pack(kc, vc).to(DEV)
+    out1 = torch.empty(B, Hkv * G, d, device=DEV)
+    out2 = torch.empty(B, Hkv * G, d, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.decode_step_e4m3(qg, kng, vng, posg, slg, kv1, tg, clg, theta, scale, ks, vs, out1,
+                         device_error=err)
+    q2 = qg.clone()
+    pkv.kv_append_e4m3(q2, kng, vng, posg, slg, kv2, theta, ks, vs, device_error=err)
+    pkv.paged_attention_decode_e4m3(q2, kv2, tg, clg, scale, ks, vs, out2, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(kv1, kv2), "fused and two-call cache bytes differ"
+    kco, vco, want = _oracle_step(kc, vc, tables, q, kn, vn, pos, slots, cl, theta, scale, ks, vs)
+    assert torch.equal(kv1.cpu(), e4m3_pack(kco, vco)), "cache bytes differ from the oracle's"
+    _check(out1, want, "fused ragged batch")
+    _check(out2, want, "two-call ragged batch")
+
+
+def test_decode_step_e4m3_edge_cases():
+    """A padding slot (-1: not appended), a slot that is not the table's
+    (flagged, not appended) and an empty context (zero output, token
+    appended), against the oracle's append + decode of the same intent."""
+    lens = [40, 40, 40, 0, 33]
+    Hkv, G, d = 2, 4, 64
+    kc, vc, tables, q, kn, vn, pos, slots, cl = _step_case(lens, Hkv, G, d, 660)
+    slots_gpu = slots.clone()
+    slots_gpu[0] = -1
+    slots_gpu[1] = int(tables[1, 0]) * BS + 3
+    slots_gpu[3] = int(tables[3, 0]) * BS + 9       # empty context: appended here
+    slots_or = slots_gpu.clone()
+    slots_or[1] = -1                               # the oracle sees "not appended"
+    ks, vs, theta, scale = 1 / 16, 1 / 16, 1e4, 0.125
+    kvg = e4m3_pack(kc, vc).to(DEV)
+    out = torch.full((len(lens), Hkv * G, d), float("nan"), device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.decode_step_e4m3(q.to(DEV), kn.to(DEV), vn.to(DEV), pos.to(DEV), slots_gpu.to(DEV), kvg,
+                         tables.to(DEV), cl.to(DEV), theta, scale, ks, vs, out,
+                         device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == pkv.DEVERR_SLOT
+    kco, vco, want = _oracle_step(kc, vc, tables, q, kn, vn, pos, slots_or, cl, theta, scale,
+                                  ks, vs)
+    want[3].zero_()
+    kcg, vcg = (h.cpu() for h in e4m3_halves(kvg))
+    assert torch.equal(kcg, kco) and torch.equal(vcg, vco), "cache bytes"
+    _check(out, want, "e4m3 step edge cases")
+
+
+@pytest.mark.parametrize("window", [1, 16, 100, 5000])
+def test_decode_step_e4m3_window(window):
+    """The one-launch step with a sliding window: the same bytes as the
+    append, the output of the windowed oracle decode; every byte no query
+    may read is random (NaN codes included) in the pool."""
+    lens = [1, 17, 300, 2049, 1000]
+    Hkv, G, d = 2, 4, 128
+    kc, vc, tables, q, kn, vn, pos, slots, cl = _step_case(lens, Hkv, G, d, 670 + window)
+    ks, vs, theta, scale = 1 / 16, 1 / 16, 5e5, 1 / math.sqrt(d)
+    kvg = e4m3_pack(kc, vc).to(DEV)
+    out = torch.full((len(lens), Hkv * G, d), float("nan"), device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.decode_step_e4m3(q.to(DEV), kn.to(DEV), vn.to(DEV), pos.to(DEV), slots.to(DEV), kvg,
+                         tables.to(DEV), cl.to(DEV), theta, scale, ks, vs, out,
+                         partition_tokens=64, device_error=err, sliding_window=window)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    kco, vco, want = _oracle_step(kc, vc, tables, q, kn, vn, pos, slots, cl, theta, scale, ks, vs,
+                                  window=window)
+    kcg, vcg = (h.cpu() for h in e4m3_halves(kvg))
+    assert torch.equal(kcg, kco) and torch.equal(vcg, vco), "cache bytes"
+    _check(out, want, f"e4m3 step window {window}")
