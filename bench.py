@@ -488,8 +488,6 @@ def measure(cfg, args, device, world, local, rank, full: bool):
     ws = pkv.new_workspace(ws_bytes, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     nbytes = step_bytes(w, out_dtype, args.window)
-    if args.window and args.cascade:
-        raise SystemExit("--window and --cascade do not combine")
 
     K = args.steps
     Wu = max(3, args.warmup)
@@ -570,7 +568,7 @@ def measure(cfg, args, device, world, local, rank, full: bool):
                                                c["block_tables"], c["decode_lens"], group_start,
                                                shared_tokens, grp, w.scale, out, workspace=ws,
                                                partition_tokens=P, force_simt=args.simt,
-                                               device_error=err)
+                                               device_error=err, sliding_window=args.window)
         else:
             pkv.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
                                        c["decode_lens"], w.scale, out, workspace=ws,

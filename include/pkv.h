@@ -568,6 +568,33 @@ pkv_status pkv_paged_attention_decode_cascade(
     int32_t out_dtype, float scale, int32_t partition_tokens, uint32_t flags,
     int32_t* device_error, void* stream);
 
+/*
+ * pkv_paged_attention_decode_cascade_window -- the cascade decode with a
+ * sliding window.
+ *
+ * Source: "Efficient LLM Inference", KV Caching: positions and windows;
+ * "Inference From Scratch", ch. 11 (prefix caching by block reuse).
+ *
+ * The result of pkv_paged_attention_decode_window: each query attends to the
+ * last `sliding_window` tokens of its context.  The shared-prefix pass gives
+ * each member only the shared tokens inside its own window (none when its
+ * window starts past them: its shared slot is then an empty partial), and
+ * reads the group's shared pages from the first page any member's window
+ * reaches; the per-sequence part starts at the later of the shared prefix's
+ * end and the window's page.  sliding_window = 0 is no window (the call is
+ * then pkv_paged_attention_decode_cascade); negative values return
+ * PKV_ERR_INVALID_ARG.  Every other argument, precondition, the workspace and
+ * every error are pkv_paged_attention_decode_cascade's.
+ */
+pkv_status pkv_paged_attention_decode_cascade_window(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* group_start, const int32_t* shared_tokens,
+    void* out, void* workspace, size_t workspace_bytes, int64_t num_seqs, int64_t num_groups,
+    int64_t max_group_size, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+    int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq, int32_t kv_dtype,
+    int32_t out_dtype, float scale, int32_t sliding_window, int32_t partition_tokens,
+    uint32_t flags, int32_t* device_error, void* stream);
+
 /* Bytes of workspace pkv_paged_attention_decode_cascade needs: 256 bytes of
  * scheduler counters, then num_seqs * Hq * (NP + 1) * (head_dim + 2) floats
  * of partials.  Host only; 0 for invalid arguments. */

@@ -94,6 +94,10 @@ def load_library() -> ctypes.CDLL:
             vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64,
             i64, i64, i64, i32, i32, ctypes.c_float, i32, u32, vp, vp]
         lib.pkv_paged_attention_decode_cascade.restype = ctypes.c_int
+        lib.pkv_paged_attention_decode_cascade_window.argtypes = [
+            vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i64, i64, i64, i64, i64, i64,
+            i64, i64, i64, i32, i32, ctypes.c_float, i32, i32, u32, vp, vp]
+        lib.pkv_paged_attention_decode_cascade_window.restype = ctypes.c_int
         lib.pkv_decode_cascade_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32]
         lib.pkv_decode_cascade_workspace_size.restype = ctypes.c_size_t
         lib.pkv_kv_append_e4m3.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
@@ -729,12 +733,14 @@ def decode_cascade_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
 def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, group_start,
                                    shared_tokens, max_group_size, scale, out, stream=None, *,
                                    workspace=None, partition_tokens=0, force_simt=False,
-                                   device_error=None) -> torch.Tensor:
+                                   device_error=None, sliding_window=0) -> torch.Tensor:
     """``paged_attention_decode`` for groups of sequences that share prefix
     blocks: group g is sequences [group_start[g], group_start[g+1]) (int32,
     device), whose first shared_tokens[b] tokens (int32 [B], device) sit in
     the group's shared blocks.  Same result; each shared prefix is read once
-    per group.  bf16 only; q already rotated.  See include/pkv.h."""
+    per group.  bf16 only; q already rotated.  ``sliding_window`` > 0: each
+    query attends to the last ``sliding_window`` tokens of its context
+    (pkv_paged_attention_decode_cascade_window).  See include/pkv.h."""
     lib = load_library()
     dv = q.device
     if q.dtype != torch.bfloat16 or k_cache.dtype != torch.bfloat16 \
@@ -754,17 +760,21 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, block_tables, context_le
         workspace = new_workspace(int(need), q.device)
     err = (_dev(device_error, "device_error", torch.int32, on=dv)
            if device_error is not None else None)
-    with _current(dv):
-        st = lib.pkv_paged_attention_decode_cascade(
-            _dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv), _dev(v_cache, "v_cache", on=dv),
+    head = (_dev(q, "q", on=dv), _dev(k_cache, "k_cache", on=dv),
+            _dev(v_cache, "v_cache", on=dv),
             _dev(block_tables, "block_tables", torch.int32, on=dv),
             _dev(context_lens, "context_lens", torch.int32, on=dv),
             _dev(group_start, "group_start", torch.int32, on=dv) if NG else None,
             _dev(shared_tokens, "shared_tokens", torch.int32, on=dv), _dev(out, "out", on=dv),
             _dev(workspace, "workspace", on=dv), workspace.numel() * workspace.element_size(),
             B, NG, int(max_group_size), Hq, Hkv, d, NB, bs, MB, PKV_DTYPE_BF16,
-            _dtype_code(out.dtype), float(scale), int(partition_tokens),
-            _flags(force_simt, True), err, _stream_ptr(stream, q.device))
+            _dtype_code(out.dtype), float(scale))
+    tail = (int(partition_tokens), _flags(force_simt, True), err, _stream_ptr(stream, q.device))
+    with _current(dv):
+        if sliding_window:
+            st = lib.pkv_paged_attention_decode_cascade_window(*head, int(sliding_window), *tail)
+        else:
+            st = lib.pkv_paged_attention_decode_cascade(*head, *tail)
     _raise(st, lib, "paged_attention_decode_cascade")
     return out
 

@@ -249,9 +249,12 @@ __device__ __forceinline__ Item decode_item(int i, const DecodeParams& p, const 
     it.slot0 = 0;
     if (p.shared_tokens) {
         // cascade: partitions start after the tokens of the shared-prefix pass
-        off = (s_pre + p.B + 1)[it.b];
+        // (or at the window's page, when the window starts past them); slot 0
+        // belongs to the shared prefix whenever it has tokens
+        const int sh = (s_pre + p.B + 1)[it.b];
+        off = max(sh, off);
         it.np = (s_len[it.b] - off + p.P - 1) / p.P;
-        it.slot0 = off > 0 ? 1 : 0;
+        it.slot0 = sh > 0 ? 1 : 0;
     }
     it.t0 = off + it.part * p.P;
     it.t1 = min(s_len[it.b], it.t0 + p.P);
@@ -1621,9 +1624,10 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__((decode_max_regs<M
         int off = window_page_start(p.window, Lb);
         if (p.shared_tokens) {
             // cascade (at most kLptMaxSeqs sequences): whole pages, within the context
-            off = p.shared_tokens[b];
-            off = off < 0 ? 0 : (off > Lb ? Lb : off) / kPageRows * kPageRows;
-            s_rank[b] = off;
+            int sh = p.shared_tokens[b];
+            sh = sh < 0 ? 0 : (sh > Lb ? Lb : sh) / kPageRows * kPageRows;
+            s_rank[b] = sh;
+            off = max(off, sh);
         }
         const int npb = (Lb - off + p.P - 1) / p.P;
         const int cnt = lpt ? max(npb - 1, 0) : npb;
@@ -1774,8 +1778,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_c
         off = p.shared_tokens[b];
         off = off < 0 ? 0 : (off > Lb ? Lb : off) / kPageRows * kPageRows;
     }
-    // slots: the shared prefix (cascade, when it has tokens), then the partitions
-    const int np = (off > 0 ? 1 : 0) + (Lb - off - woff + p.P - 1) / p.P;
+    // slots: the shared prefix (cascade, when it has tokens), then the
+    // partitions, from the later of the prefix's end and the window's page
+    const int np = (off > 0 ? 1 : 0) + (Lb - max(off, woff) + p.P - 1) / p.P;
     if (np <= 1 && off == 0) return;  // written by the decode kernel
 
     // first partials of this thread, independent of the weights

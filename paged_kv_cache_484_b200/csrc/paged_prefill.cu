@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <climits>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -782,22 +783,36 @@ struct CascadeParams {
     float* part_ml;
     int32_t* err;
     int B, Hq, Hkv, MB, NPT, RG, NG, num_blocks;
+    int window;        // sliding window (0: none)
     float scale_log2;
 };
+
+// Context length of sequence b, clamped as the decode clamps it.
+__device__ __forceinline__ int cascade_len(const CascadeParams& p, int b) {
+    const int L = p.context_lens[b];
+    const int maxlen = p.MB * kPageRows;
+    return L < 0 ? 0 : (L > maxlen ? maxlen : L);
+}
 
 // Shared tokens of sequence b as the decode counts them: whole pages inside
 // its (clamped) context.
 __device__ __forceinline__ int cascade_shared(const CascadeParams& p, int b) {
-    int L = p.context_lens[b];
-    const int maxlen = p.MB * kPageRows;
-    L = L < 0 ? 0 : (L > maxlen ? maxlen : L);
-    int s = p.shared_tokens[b];
+    const int L = cascade_len(p, b);
+    const int s = p.shared_tokens[b];
     return s < 0 ? 0 : (s > L ? L : s) / kPageRows * kPageRows;
+}
+
+// First token sequence b's query attends (sliding window; 0 otherwise).
+__device__ __forceinline__ int cascade_lo(const CascadeParams& p, int b) {
+    const int L = cascade_len(p, b);
+    return (p.window > 0 && L > p.window) ? L - p.window : 0;
 }
 
 // One CTA per (group, kv head, row group of 128 rows): the rows are
 // (member, head) pairs, member m of the group and head g -> row m*G + g;
-// every row attends to the first shared_tokens of its own sequence, read
+// every row attends to the first shared_tokens of its own sequence (under a
+// sliding window only those inside its window: a row whose window starts past
+// them leaves an empty partial), read
 // once for the group from the pages of the member that shares the most (the
 // others' shared block-table entries must be the same ids: a mismatch sets
 // PKV_DEVERR_PREFIX).  The tiles run on the tensor cores (umma_attend).  The
@@ -816,7 +831,9 @@ __global__ void __launch_bounds__(kUThreads)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    __shared__ int s_grp[4];  // first member, member count, leader, the leader's shared tokens
+    // first member, member count, leader, the leader's shared tokens, the
+    // first token any row attends
+    __shared__ int s_grp[5];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     grid_launch_dependents();
     int x = blockIdx.x;
@@ -829,21 +846,25 @@ __global__ void __launch_bounds__(kUThreads)
             report_error(p.err, PKV_DEVERR_PREFIX);
             gs = ge = 0;
         }
-        int best = 0, leader = gs;
+        int best = 0, leader = gs, minlo = INT_MAX;
         for (int b = gs; b < ge; ++b) {
-            const int sb = cascade_shared(p, b);
+            const int sb = cascade_shared(p, b), lo = cascade_lo(p, b);
             if (sb > best) {
                 best = sb;
                 leader = b;
             }
+            if (lo < sb) minlo = min(minlo, lo);
         }
         s_grp[0] = gs;
         s_grp[1] = ge - gs;
         s_grp[2] = leader;
         s_grp[3] = best;
+        // no row has a shared token inside its window: one page, all masked
+        s_grp[4] = minlo < best ? minlo : max(best - 1, 0);
     }
     __syncthreads();
     const int gs = s_grp[0], nmem = s_grp[1], leader = s_grp[2], S = s_grp[3];
+    const int first_key = s_grp[4];
     if (S > 0 && rg * kURows < nmem * G) {
         if (warp == 0 && lane == 0) {
             prefetch_tensor_map(&tm_k);
@@ -862,10 +883,11 @@ __global__ void __launch_bounds__(kUThreads)
         UItem it;
         it.b = leader;
         it.h = h;
-        it.t0 = 0;
+        // pages before the page of the first key any row attends are skipped
+        it.t0 = first_key / kPageRows * kPageRows;
         it.t1 = S;
-        it.npages = S / kPageRows;
-        it.lo = 0;
+        it.npages = (S - it.t0) / kPageRows;
+        it.lo = first_key;
         URow row = {};
         if (warp >= 2) {
             const int fr = rg * kURows + 32 * (warp & 3) + lane;
@@ -873,7 +895,7 @@ __global__ void __launch_bounds__(kUThreads)
             const int b = gs + m;
             row.len = m < nmem ? cascade_shared(p, b) : 0;
             row.ok = row.len > 0;  // no shared tokens: no slot 0
-            row.lo = 0;
+            row.lo = m < nmem ? cascade_lo(p, b) : 0;
             const size_t r = (size_t)(row.ok ? b : 0) * p.Hq + hq;
             row.q = p.q + r * D;
             row.out = nullptr;
@@ -995,6 +1017,7 @@ cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
     p.Hkv = (int)a.Hkv;
     p.MB = (int)a.MB;
     p.NPT = a.slots_per_row;
+    p.window = a.window;
     p.RG = (int)((a.max_group_size * G + kURows - 1) / kURows);
     p.NG = (int)a.num_groups;
     p.num_blocks = (int)a.num_blocks;

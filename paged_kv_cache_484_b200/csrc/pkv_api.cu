@@ -731,15 +731,17 @@ size_t pkv_decode_cascade_workspace_size(int64_t num_seqs, int64_t num_q_heads,
     return w.bytes;
 }
 
-pkv_status pkv_paged_attention_decode_cascade(
+}  // extern "C"
+
+namespace {
+pkv_status cascade_common(
     const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
     const int32_t* context_lens, const int32_t* group_start, const int32_t* shared_tokens,
     void* out, void* workspace, size_t workspace_bytes, int64_t num_seqs, int64_t num_groups,
     int64_t max_group_size, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
     int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq, int32_t kv_dtype,
-    int32_t out_dtype, float scale, int32_t partition_tokens, uint32_t flags,
+    int32_t out_dtype, float scale, int32_t window, int32_t partition_tokens, uint32_t flags,
     int32_t* device_error, void* stream) {
-    set_last_error("");
     if (num_seqs < 0 || max_blocks_per_seq < 0 || num_groups < 0) {
         set_last_error("negative num_seqs, num_groups or max_blocks_per_seq");
         return PKV_ERR_INVALID_ARG;
@@ -771,6 +773,10 @@ pkv_status pkv_paged_attention_decode_cascade(
     }
     if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) {
         set_last_error("scale must be finite");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (window < 0) {
+        set_last_error("sliding_window must be >= 0");
         return PKV_ERR_INVALID_ARG;
     }
     WorkspacePlan w;
@@ -819,6 +825,7 @@ pkv_status pkv_paged_attention_decode_cascade(
     c.num_groups = num_groups;
     c.max_group_size = max_group_size;
     c.slots_per_row = npt;
+    c.window = window;
     c.scale = scale;
     c.device_error = device_error;
     c.stream = static_cast<cudaStream_t>(stream);
@@ -847,11 +854,47 @@ pkv_status pkv_paged_attention_decode_cascade(
     a.force_simt = (flags & PKV_DECODE_FORCE_SIMT) != 0;
     a.allow_cluster = false;
     a.shared_tokens = shared_tokens;
+    a.window = window;
     a.launch_between = launch_cascade_between;
     a.between_ctx = &c;
     a.device_error = device_error;
     a.stream = static_cast<cudaStream_t>(stream);
     return cuda_status(launch_paged_decode(a), "cascade decode launch");
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode_cascade(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* group_start, const int32_t* shared_tokens,
+    void* out, void* workspace, size_t workspace_bytes, int64_t num_seqs, int64_t num_groups,
+    int64_t max_group_size, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+    int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq, int32_t kv_dtype,
+    int32_t out_dtype, float scale, int32_t partition_tokens, uint32_t flags,
+    int32_t* device_error, void* stream) {
+    set_last_error("");
+    return cascade_common(q, k_cache, v_cache, block_tables, context_lens, group_start,
+                          shared_tokens, out, workspace, workspace_bytes, num_seqs, num_groups,
+                          max_group_size, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                          block_size, max_blocks_per_seq, kv_dtype, out_dtype, scale, 0,
+                          partition_tokens, flags, device_error, stream);
+}
+
+pkv_status pkv_paged_attention_decode_cascade_window(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* group_start, const int32_t* shared_tokens,
+    void* out, void* workspace, size_t workspace_bytes, int64_t num_seqs, int64_t num_groups,
+    int64_t max_group_size, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+    int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq, int32_t kv_dtype,
+    int32_t out_dtype, float scale, int32_t sliding_window, int32_t partition_tokens,
+    uint32_t flags, int32_t* device_error, void* stream) {
+    set_last_error("");
+    return cascade_common(q, k_cache, v_cache, block_tables, context_lens, group_start,
+                          shared_tokens, out, workspace, workspace_bytes, num_seqs, num_groups,
+                          max_group_size, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                          block_size, max_blocks_per_seq, kv_dtype, out_dtype, scale,
+                          sliding_window, partition_tokens, flags, device_error, stream);
 }
 
 }  // extern "C"

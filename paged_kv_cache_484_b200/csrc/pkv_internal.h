@@ -118,6 +118,7 @@ struct CascadeArgs {
     float* part_ml;
     int64_t B, Hq, Hkv, D, num_blocks, MB, num_groups, max_group_size;
     int32_t slots_per_row;          // partial slots per (sequence, q head): 1 + NP
+    int32_t window;                 // sliding window (0: none)
     float scale;
     int32_t* device_error;
     cudaStream_t stream;

@@ -32,15 +32,16 @@ class SubProblem:
     def __init__(self, w: Workload, seqs):
         self.__dict__.update(vars(extract_sequences(w, seqs)))
 
-    def oracle_step(self, nthreads=8, pairs=None):
-        """Oracle append then decode; returns (q_rot, k_cache, v_cache, out_f64)."""
+    def oracle_step(self, nthreads=8, pairs=None, window=0):
+        """Oracle append then decode (over the last ``window`` tokens when
+        > 0); returns (q_rot, k_cache, v_cache, out_f64)."""
         q = self.q.clone()
         kc = self.k_cache.clone()
         vc = self.v_cache.clone()
         oracle.kv_append(q, self.k_new.clone(), self.v_new.clone(), self.positions, self.slots,
                          kc, vc, self.theta)
         out = oracle.paged_attention_decode(q, kc, vc, self.tables, self.decode_lens, self.scale,
-                                            pairs=pairs, nthreads=nthreads)
+                                            pairs=pairs, nthreads=nthreads, window=window)
         return q, kc, vc, out
 
 

@@ -360,6 +360,25 @@ def test_cascade_rejects_bad_arguments(lib, kw, status):
         assert lib.pkv_last_error() != b""
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(win=-1), INVALID),
+    (dict(win=64, kvdt=F32), UNSUPPORTED),
+    (dict(win=64, MG=9), INVALID),
+    (dict(win=64, ws=FAKE, wsb=255), WORKSPACE),
+    (dict(win=64, B=0, G=0, q=None, out=None), OK),
+])
+def test_cascade_window_rejects_bad_arguments(lib, kw, status):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, gs=FAKE, sh=FAKE, out=FAKE, ws=None,
+             wsb=0, B=8, G=1, MG=8, Hq=8, Hkv=2, d=64, NB=64, bs=16, MB=8, kvdt=BF16, odt=BF16,
+             scale=0.125, win=0, P=0, flags=0, err=None)
+    a.update(kw)
+    st = lib.pkv_paged_attention_decode_cascade_window(
+        a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["gs"], a["sh"], a["out"], a["ws"], a["wsb"],
+        a["B"], a["G"], a["MG"], a["Hq"], a["Hkv"], a["d"], a["NB"], a["bs"], a["MB"], a["kvdt"],
+        a["odt"], a["scale"], a["win"], a["P"], a["flags"], a["err"], None)
+    assert st == status
+
+
 def test_cascade_workspace_size_formula(lib):
     """256 bytes of scheduler counters, then NP + 1 partial slots per
     (sequence, q head): slot 0 holds the shared-prefix pass."""

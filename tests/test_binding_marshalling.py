@@ -165,6 +165,17 @@ def _cases():
         device_error=a["err"]), a, "pkv_paged_attention_decode_cascade",
         ["q", "k_cache", "v_cache", "block_tables", "context_lens", "group_start",
          "shared_tokens", "out", "workspace"]))
+
+    a = dict(_decode_args(), group_start=_t((2,), i32), shared_tokens=_t((Bs,), i32),
+             workspace=ws(), err=err())
+    cases.append(("paged_attention_decode_cascade window",
+                  lambda a=a: B.paged_attention_decode_cascade(
+                      a["q"], a["k_cache"], a["v_cache"], a["block_tables"], a["context_lens"],
+                      a["group_start"], a["shared_tokens"], 2, 0.125, a["out"],
+                      workspace=a["workspace"], device_error=a["err"], sliding_window=64), a,
+                  "pkv_paged_attention_decode_cascade_window",
+                  ["q", "k_cache", "v_cache", "block_tables", "context_lens", "group_start",
+                   "shared_tokens", "out", "workspace"]))
     return cases
 
 

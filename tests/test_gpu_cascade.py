@@ -51,11 +51,12 @@ def _check(got, want, what):
     assert err.max().item() <= TOL_BF16, f"{what}: max err {err.max().item():.3e}"
 
 
-def _run(w, group_start, shared, max_group, P=0, err=None):
+def _run(w, group_start, shared, max_group, P=0, err=None, window=0):
     out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=DEV)
     pkv.paged_attention_decode_cascade(w.q, w.k_cache, w.v_cache, w.block_tables, w.decode_lens,
                                        group_start, shared, max_group, w.scale, out,
-                                       partition_tokens=P, device_error=err)
+                                       partition_tokens=P, device_error=err,
+                                       sliding_window=window)
     torch.cuda.synchronize()
     return out
 
@@ -75,6 +76,47 @@ def test_cascade_matches_plain_decode(d, G, group, P):
                                w.scale, plain, partition_tokens=P)
     torch.cuda.synchronize()
     assert (out - plain).abs().max().item() < 1e-4
+
+
+@pytest.mark.parametrize("window,P", [(1, 0), (16, 64), (100, 0), (300, 128), (600, 0),
+                                      (1100, 256), (5000, 0)])
+def test_cascade_with_window_matches_windowed_decode(window, P):
+    """Each query attends to its last `window` tokens: windows that start past
+    the shared prefix (empty shared slot), inside it, and before it, against
+    the oracle's windowed decode of every sequence over its own table.  The
+    tokens the kernels may skip are NaN in the cache, so a stray read shows
+    up."""
+    lens = [1500, 300, 40, 255, 2000, 256, 16, 700, 1024, 77, 900, 260, 2047, 511, 5, 3000]
+    w, sub, gs, shared, group = _grouped(lens, 4, 512, 4, 2, 64, seed=470 + window)
+    # NaN (in the GPU's cache only) in the tokens no query reads: those of a
+    # sequence's own pages before its window, and those of the group's shared
+    # pages before the first token any member attends.  (Shared tokens from
+    # there on are the group's prompt prefix, finite cache contents, which a
+    # member may skip under its own window while another reads them.)
+    L = w.decode_lens.to(torch.int64).cpu()
+    lo = torch.clamp(L - window, min=0)
+    sh = shared.to(torch.int64).cpu()
+    tables = w.block_tables.to(torch.int64).cpu()
+    nan_k, nan_v = w.k_cache.clone(), w.v_cache.clone()
+    for b in range(w.B):
+        g0 = (b // group) * group
+        members = range(g0, min(g0 + group, w.B))
+        with_keys = [int(lo[m]) for m in members if lo[m] < sh[m]]
+        first_read = min(with_keys) if with_keys else int(max(sh[m] for m in members))
+        t = torch.arange(int(lo[b]))
+        t = t[(t >= sh[b]) | (t < first_read)]
+        if t.numel() == 0:
+            continue
+        blk, row = tables[b, t // 16].to(DEV), (t % 16).to(DEV)
+        nan_k[blk, :, row] = float("nan")
+        nan_v[blk, :, row] = float("nan")
+    w.k_cache.copy_(nan_k)
+    w.v_cache.copy_(nan_v)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = _run(w, gs, shared, group, P=P, err=err, window=window)
+    assert int(err.item()) == 0
+    _check(out, sub.oracle_step(nthreads=8, window=window)[3],
+           f"cascade window {window} P{P}")
 
 
 def test_cascade_edge_cases():
