@@ -164,19 +164,32 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources a decode call's kernels and their launch plan are built from
+# (the chunked prefill and the cascade's shared-prefix pass live elsewhere).
+DECODE_SOURCES = ("paged_decode.cu", "pkv_api.cu", "pkv_device.cuh", "pkv_internal.h")
+
+
+def kernel_source_hash(names=None) -> str:
+    """Hash of the library's CUDA sources (``names``: only those files of
+    csrc/, plus the public header; default: every file)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_484_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        if names is not None and name not in names:
+            continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
+    if names is not None:
+        with open(os.path.join(ROOT, "include", "pkv.h"), "rb") as f:
+            h.update(b"pkv.h" + f.read())
     return h.hexdigest()[:16]
 
 
 def software_versions() -> dict:
     """Versions the numbers were taken with (NVML read only)."""
     v = {"torch": torch.__version__, "cuda_runtime": torch.version.cuda,
-         "kernel_sources": kernel_source_hash()}
+         "kernel_sources": kernel_source_hash(),
+         "decode_sources": kernel_source_hash(DECODE_SOURCES)}
     try:
         # the git commit, where the checkout carries its history
         r = subprocess.run(["git", "-C", ROOT, "rev-parse", "--short", "HEAD"],
@@ -197,7 +210,7 @@ def software_versions() -> dict:
 
 def recorded_traffic(cfg):
     """DRAM bytes per decode launch from the committed ncu capture, if it was
-    taken on the current kernel sources (else None).  ``cfg``: the config
+    taken on the current decode sources (else None).  ``cfg``: the config
     number, or e.g. "3_e4m3" for its 8-bit cache.  A workload captured on a
     smaller batch of the same kernel is recorded already scaled to the full
     launch."""
@@ -208,7 +221,7 @@ def recorded_traffic(cfg):
     except Exception:
         return None
     ent = rec.get("configs", {}).get(str(cfg))
-    if ent is None or ent.get("kernel_source_hash") != kernel_source_hash():
+    if ent is None or ent.get("decode_source_hash") != kernel_source_hash(DECODE_SOURCES):
         return None
     return ent.get("bytes_per_launch")
 

@@ -14,15 +14,15 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-def test_recorded_traffic_is_tied_to_the_kernel_sources(monkeypatch):
+def test_recorded_traffic_is_tied_to_the_decode_sources(monkeypatch):
     rec = json.load(open(os.path.join(ROOT, "profiles", "decode_dram_traffic.json")))
     for key, ent in rec["configs"].items():
-        h = ent["kernel_source_hash"]
-        monkeypatch.setattr(bench, "kernel_source_hash", lambda: h)
+        h = ent["decode_source_hash"]
+        monkeypatch.setattr(bench, "kernel_source_hash", lambda names=None: h)
         assert bench.recorded_traffic(key) == ent["bytes_per_launch"]
     assert bench.recorded_traffic("no such workload") is None
     # a capture taken on other sources is not reported
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda names=None: "0" * 16)
     for key in rec["configs"]:
         assert bench.recorded_traffic(key) is None
 
@@ -32,12 +32,20 @@ def test_kernel_source_hash_covers_every_source_file(tmp_path, monkeypatch):
     csrc.mkdir(parents=True)
     (csrc / "a.cu").write_text("one")
     (csrc / "b.cuh").write_text("two")
+    (tmp_path / "include").mkdir()
+    (tmp_path / "include" / "pkv.h").write_text("api")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h0 = bench.kernel_source_hash()
     (csrc / "b.cuh").write_text("two ")
     assert bench.kernel_source_hash() != h0
     (csrc / "b.cuh").write_text("two")
     assert bench.kernel_source_hash() == h0
+    # the decode hash covers only the named files and the public header
+    d0 = bench.kernel_source_hash(("b.cuh",))
+    (csrc / "a.cu").write_text("one ")
+    assert bench.kernel_source_hash(("b.cuh",)) == d0
+    (tmp_path / "include" / "pkv.h").write_text("api ")
+    assert bench.kernel_source_hash(("b.cuh",)) != d0
 
 
 def test_peak_falls_back_when_no_measured_file(tmp_path, monkeypatch):
