@@ -148,7 +148,10 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const __grid_const
 //   S = Q K^T      (M = 128 rows, N = 64 keys, K = D), fp32
 //   O += P V       (M = 128 rows, N = D, K = 64 keys), fp32
 // P is split into a high and a low bf16 part (p = hi + lo to ~2^-17
-// relative) and both are multiplied into O, as on the warp-level path.
+// relative) and both are multiplied into O, as on the warp-level path.  The
+// softmax threads write P into tensor memory and O += P V reads it from
+// there as its A operand: only V comes from shared memory, which halves the
+// shared-memory reads of that MMA.
 //
 // Roles (320 threads):
 //   warp 0   producer: block-table entries -> TMA page loads into a ring of
@@ -181,6 +184,58 @@ constexpr int kUTilePages = kUTileKeys / kPageRows;
 constexpr int kUThreads = 10 * 32;
 constexpr float kURescaleLog2 = 8.f;
 
+// 16 columns of the warp's 32 tensor-memory lanes (one 32-bit value per
+// lane and column).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] . B[smem]: A read from tensor memory (see COL_P).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+// N consecutive 32-bit columns of the warp's 32 lanes (N = 8 or 16).
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[N]) {
+    static_assert(N == 8 || N == 16, "x8 or x16");
+    if constexpr (N == 8) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                         taddr),
+                     "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                     "r"(v[7])
+                     : "memory");
+    } else {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+            "%13,%14,%15,%16};" ::"r"(taddr),
+            "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+            "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+            "r"(v[15])
+            : "memory");
+    }
+}
+
+// Rows of an item split over T tensor-memory lanes each: an item of at most
+// 128 / T query rows stores each row T times in the 128-row tile, in lane
+// quadrants 4 / T apart, and the copy in quadrant group `part` takes the
+// key columns [part 64 / T, (part + 1) 64 / T) of every tile with a softmax
+// state of its own; the parts are merged at the end.  Half-full tiles then
+// run their softmax on all four SM sub-partitions with half the columns per
+// thread.
+__host__ __device__ constexpr int umma_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
+
 template <int D>
 struct ULayout {
     static constexpr int BOX = kPageRows * 128;                 // 16 rows x 64 bf16 columns
@@ -188,23 +243,26 @@ struct ULayout {
     static constexpr int BLOCK_STRIDE = kUTilePages * BOX;      // between column blocks of a tile
     static constexpr int KV_BYTES = NB * BLOCK_STRIDE;          // one tile of K (or of V)
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;            // K tile, then V tile
-    static constexpr int STAGES = D == 64 ? 8 : 4;              // 128 KiB of ring
+    static constexpr int STAGES = D == 64 ? 8 : 5;              // 128 / 160 KiB of ring
     static constexpr int Q_BLOCK = kURows * 128;                // one column block of Q
-    static constexpr int P_BYTES = kURows * 128;                // 128 rows x 64 keys bf16
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
     static constexpr int PBUFS = 2;                             // P buffers, tile j uses j % 2
-    static constexpr int OFF_P = OFF_Q + NB * Q_BLOCK;          // [buffer][hi, lo]
-    static constexpr int OFF_XCHG = OFF_P + PBUFS * 2 * P_BYTES;  // (max, sum) of warpgroup 1's rows
+    static constexpr int OFF_XCHG = OFF_Q + NB * Q_BLOCK;       // (max, sum) of warpgroup 1's rows
     static constexpr int OFF_BAR = OFF_XCHG + kURows * 8;
     // full[STAGES], empty[STAGES], sbar[2], sfree[2], pready[2], obar[2], pfree[PBUFS],
-    // mma_done, xchg, join
-    static constexpr int NBARS = 2 * STAGES + 11 + PBUFS;
+    // mma_done, xchg, join, parts (split rows: the row's parts are staged)
+    static constexpr int NBARS = 2 * STAGES + 12 + PBUFS;
     static constexpr int OFF_MASK = OFF_BAR + NBARS * 8;
     static constexpr int OFF_MISC = OFF_MASK + STAGES * 4;      // abort flag, TMEM base
     static constexpr size_t SMEM = 1024 + OFF_MISC + 16;
     static constexpr uint32_t COL_S = 0;                        // + 64 * warpgroup
     static constexpr uint32_t COL_O = 128;                      // + D * warpgroup
-    static constexpr uint32_t TMEM_COLS = COL_O + 2 * D <= 256 ? 256 : 512;
+    // P buffer b: bf16 pairs of the hi part in columns [0, 32), of the lo
+    // part in [32, 64) (lane = row, column c = keys 2c and 2c + 1: the A
+    // operand layout of an MMA that reads A from tensor memory)
+    static constexpr uint32_t COL_P = COL_O + 2 * D;            // + 64 * buffer
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(COL_P + 64 * PBUFS <= TMEM_COLS, "tensor memory");
     static constexpr uint32_t IDESC_S = umma_idesc_bf16(kURows, kUTileKeys, false);
     static constexpr uint32_t IDESC_O = umma_idesc_bf16(kURows, D, true);
 };
@@ -311,16 +369,22 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
                             uint64_t* obar, uint64_t* pfree, uint64_t* mma_done,
                             volatile int* s_abort, int32_t* err) {
     using L = ULayout<D>;
-    const uint32_t sq = smem_addr(base + L::OFF_Q);
+    // Descriptors are built once and advanced by constant offsets: the start
+    // address field holds address / 16 in its low bits (shared-memory
+    // addresses stay below 2^18 bytes, so the sum never carries out of it).
+    // One thread issues every MMA, so keeping its instruction chain short
+    // sets how fast the tiles go.
+    const uint64_t q_desc = umma_desc_sw128(smem_addr(base + L::OFF_Q), 16, 1024);
+    const uint64_t k_desc0 = umma_desc_sw128(smem_addr(base), 16, 1024);
+    const uint64_t v_desc0 = umma_desc_sw128(smem_addr(base + L::KV_BYTES), L::BLOCK_STRIDE, 1024);
     auto issue_s = [&](int j) {
         const int stage = j % L::STAGES;
-        const uint32_t sk = smem_addr(base + stage * L::STAGE_BYTES);
+        const uint64_t k_desc = k_desc0 + (uint64_t)((stage * L::STAGE_BYTES) >> 4);
         const uint32_t d = tmem + L::COL_S + 64u * (uint32_t)(j & 1);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
-            const uint64_t da = umma_desc_sw128(sq + (s >> 2) * L::Q_BLOCK + (s & 3) * 32, 16, 1024);
-            const uint64_t db =
-                umma_desc_sw128(sk + (s >> 2) * L::BLOCK_STRIDE + (s & 3) * 32, 16, 1024);
+            const uint64_t da = q_desc + (uint64_t)(((s >> 2) * L::Q_BLOCK + (s & 3) * 32) >> 4);
+            const uint64_t db = k_desc + (uint64_t)(((s >> 2) * L::BLOCK_STRIDE + (s & 3) * 32) >> 4);
             umma_bf16(d, da, db, L::IDESC_S, s > 0);
         }
         umma_commit(&sbar[j & 1]);
@@ -328,16 +392,14 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
     auto issue_pv = [&](int j) {
         const int w = j & 1;
         const int stage = j % L::STAGES;
-        const uint32_t sv = smem_addr(base + stage * L::STAGE_BYTES + L::KV_BYTES);
-        const uint32_t sp = smem_addr(base + L::OFF_P + (j % L::PBUFS) * 2 * L::P_BYTES);
+        const uint64_t v_desc = v_desc0 + (uint64_t)((stage * L::STAGE_BYTES) >> 4);
+        const uint32_t pt = tmem + L::COL_P + (uint32_t)((j % L::PBUFS) * 64);
         const uint32_t o = tmem + L::COL_O + (uint32_t)(w * D);
 #pragma unroll
         for (int s = 0; s < kUTileKeys / 16; ++s) {
-            const uint64_t db = umma_desc_sw128(sv + s * 16 * 128, L::BLOCK_STRIDE, 1024);
-            const uint64_t hi = umma_desc_sw128(sp + s * 32, 16, 1024);
-            const uint64_t lo = umma_desc_sw128(sp + L::P_BYTES + s * 32, 16, 1024);
-            umma_bf16(o, hi, db, L::IDESC_O, j >= 2 || s > 0);
-            umma_bf16(o, lo, db, L::IDESC_O, true);
+            const uint64_t db = v_desc + (uint64_t)((s * 16 * 128) >> 4);
+            umma_bf16_ts(o, pt + 8u * s, db, L::IDESC_O, j >= 2 || s > 0);
+            umma_bf16_ts(o, pt + 32u + 8u * s, db, L::IDESC_O, true);
         }
         umma_commit(&obar[w]);
         umma_commit(&pfree[j % L::PBUFS]);
@@ -346,7 +408,9 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
     // S_j needs its stage loaded and (j >= 2) the buffer's previous scores read;
     // PV_j needs P_j.  Neither condition can run two phases ahead of this lane
     // (the warpgroup's next arrivals wait for MMAs only this lane issues), so
-    // each wait is on an unambiguous parity.
+    // each wait is on an unambiguous parity.  (Measured against this polling
+    // loop: issuing every ready S first, and a fixed order S_{j+2}, PV_j after
+    // each P_j with blocking waits, were both slower.)
     int js = 0, jp = 0;
     bool ok = true;
     uint64_t since = 0;
@@ -416,11 +480,14 @@ __device__ __forceinline__ void umma_zero_v_rows(const UItem& it, int j, int r, 
 }
 
 // One item, run by all kUThreads threads of the CTA (every thread calls it;
-// `row` matters to the softmax warps only).
-template <int D>
+// `row` matters to the softmax warps only).  T: tensor-memory lanes per
+// query row (umma_split): the softmax thread of lane quadrant q takes the key
+// columns of part q / (4 / T).
+template <int D, int T>
 __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
                             const CUtensorMap* tmk, const CUtensorMap* tmv, uint8_t* base) {
     using L = ULayout<D>;
+    constexpr int NC = kUTileKeys / T;  // key columns of a tile per softmax thread
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
     uint64_t* empty = full + L::STAGES;
     uint64_t* sbar = empty + L::STAGES;
@@ -431,6 +498,7 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     uint64_t* mma_done = pfree + L::PBUFS;
     uint64_t* xchg_bar = mma_done + 1;
     uint64_t* join = xchg_bar + 1;
+    uint64_t* parts_bar = join + 1;
     uint32_t* masks = reinterpret_cast<uint32_t*>(base + L::OFF_MASK);
     volatile int* s_abort = reinterpret_cast<volatile int*>(base + L::OFF_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::OFF_MISC + 4);
@@ -452,11 +520,13 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
         mbar_init(mma_done, 1);
         mbar_init(xchg_bar, kURows);
         mbar_init(join, 2 * kURows);
+        mbar_init(parts_bar, kURows);
         *s_abort = 0;
         fence_barrier_init();
     }
     const int r = 32 * (warp & 3) + lane;  // softmax threads: the row (tensor-memory lane)
     const int wg = (warp - 2) >> 2;        // softmax threads: the warpgroup
+    const int part = (warp & 3) / (4 / T);  // softmax threads: the row's part
     if (warp >= 2) {
         // warpgroup 0 puts the Q rows into the swizzled tile (zeros for rows
         // past the item); the V halves of the ring start zeroed, so that a
@@ -483,6 +553,23 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if constexpr (T > 1) {
+        // split rows: a thread writes only its part's columns of its P rows;
+        // the other columns stay zero for the whole item (warpgroup 0 clears
+        // the P buffers of its lanes before any MMA can read them)
+        if (warp >= 2 && warp < 6) {
+            uint32_t z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) z[e] = 0u;
+            const uint32_t lb = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + L::COL_P;
+#pragma unroll
+            for (int c = 0; c < 64 * L::PBUFS; c += 16) tmem_st<16>(lb + (uint32_t)c, z);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
 
     if (warp == 0) {
         umma_producer<D>(a, it, tmk, tmv, base, full, empty, masks, s_abort);
@@ -504,6 +591,7 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t col_s = L::COL_S + 64u * (uint32_t)wg, col_o = L::COL_O + (uint32_t)(wg * D);
     const int row_len = row.ok ? row.len : 0;
+    const int c_first = part * NC;  // this thread's first key column of a tile
     // a warp whose 32 rows are all padding (past the item's rows) has no
     // scores to read and no P worth writing: its rows of O are never stored.
     // It still keeps the tiles' cadence (the same waits and arrivals), so
@@ -533,9 +621,9 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             continue;
         }
         tc_fence_after();
-        const uint32_t msk = masks[stage];
-        float x[kUTileKeys];
-        {
+        const uint32_t msk = masks[stage] >> (c_first / kPageRows);
+        float x[NC];
+        if constexpr (NC == 64) {
             uint32_t v0[32], v1[32];
             tmem_ld32(lane_base + col_s, v0);
             tmem_ld32(lane_base + col_s + 32, v1);
@@ -545,25 +633,38 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
                 x[e] = __uint_as_float(v0[e]);
                 x[32 + e] = __uint_as_float(v1[e]);
             }
+        } else if constexpr (NC == 32) {
+            uint32_t v0[32];
+            tmem_ld32(lane_base + col_s + (uint32_t)c_first, v0);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(v0[e]);
+        } else {
+            uint32_t v0[16];
+            tmem_ld16(lane_base + col_s + (uint32_t)c_first, v0);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v0[e]);
         }
         // the score buffer may take S_{j+2} now
         tc_fence_before();
         mbar_arrive(&sfree[wg]);
-        const int tile_t0 = it.t0 + j * kUTileKeys;
-        const int k_lo = max(0, row.lo - tile_t0), k_hi = min(kUTileKeys, row_len - tile_t0);
+        const int tile_t0 = it.t0 + j * kUTileKeys + c_first;
+        const int k_lo = max(0, row.lo - tile_t0), k_hi = min(NC, row_len - tile_t0);
         // the row maximum as a tree of eight independent chains
         float mx8[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx8[u] = kNegInfP;
-        if (k_lo == 0 && k_hi == kUTileKeys && msk == (1u << kUTilePages) - 1u) {
+        constexpr uint32_t kAllPages = (1u << (NC / kPageRows)) - 1u;
+        if (k_lo == 0 && k_hi == NC && (msk & kAllPages) == kAllPages) {
 #pragma unroll
-            for (int e = 0; e < kUTileKeys; ++e) {
+            for (int e = 0; e < NC; ++e) {
                 x[e] *= a.scale_log2;
                 mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < kUTileKeys; ++e) {
+            for (int e = 0; e < NC; ++e) {
                 const bool valid = e >= k_lo && e < k_hi && ((msk >> (e / kPageRows)) & 1u);
                 x[e] = valid ? x[e] * a.scale_log2 : kNegInfP;
                 mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
@@ -602,29 +703,30 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             ok = __all_sync(0xffffffffu, mbar_wait(&pfree[j % L::PBUFS],
                                                    (uint32_t)(j / L::PBUFS - 1) & 1u));
             if (!ok) break;
+            tc_fence_after();
         }
-        const uint32_t hi_row =
-            smem_addr(base + L::OFF_P + (j % L::PBUFS) * 2 * L::P_BYTES) + r * 128;
-        const uint32_t lo_row = hi_row + L::P_BYTES;
+        // this thread's columns of P buffer j % PBUFS: hi pairs, then lo pairs
+        const uint32_t p_col = lane_base + L::COL_P + (uint32_t)((j % L::PBUFS) * 64 + c_first / 2);
         float ps8[8];  // the row sum, eight independent chains
 #pragma unroll
         for (int u = 0; u < 8; ++u) ps8[u] = 0.f;
+        constexpr int CW = NC / 2 < 16 ? NC / 2 : 16;  // words per tensor-memory store
 #pragma unroll
-        for (int c = 0; c < kUTileKeys / 8; ++c) {
-            uint32_t hw[4], lw[4];
+        for (int c = 0; c < NC / 2; c += CW) {
+            uint32_t hw[CW], lw[CW];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float p0 = fast_exp2(x[8 * c + 2 * e] - m_ref);
-                const float p1 = fast_exp2(x[8 * c + 2 * e + 1] - m_ref);
-                ps8[2 * e] += p0;
-                ps8[2 * e + 1] += p1;
+            for (int e = 0; e < CW; ++e) {
+                const float p0 = fast_exp2(x[2 * (c + e)] - m_ref);
+                const float p1 = fast_exp2(x[2 * (c + e) + 1] - m_ref);
+                ps8[(2 * e) & 7] += p0;
+                ps8[(2 * e + 1) & 7] += p1;
                 hw[e] = pack_bf16(p0, p1);
                 lw[e] = pack_bf16(p0 - bf16lo(hw[e]), p1 - bf16hi(hw[e]));
             }
-            const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
-            st_shared_v4(hi_row + off, hw[0], hw[1], hw[2], hw[3]);
-            st_shared_v4(lo_row + off, lw[0], lw[1], lw[2], lw[3]);
+            tmem_st<CW>(p_col + (uint32_t)c, hw);
+            tmem_st<CW>(p_col + 32u + (uint32_t)c, lw);
         }
+        tmem_wait_st();
         l_run += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
         umma_zero_v_rows<D>(it, j, r, base + stage * L::STAGE_BYTES + L::KV_BYTES);
         fence_proxy_async_smem();
@@ -658,7 +760,8 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
         mbar_arrive(join);
         return;
     }
-    // warpgroup 0: merge the two states of the row, then store it
+    // warpgroup 0: merge the two states of the lane, then (split rows) the
+    // row's parts, then store the row
     const bool x_ok = __all_sync(0xffffffffu, mbar_wait(xchg_bar, 0));
     const float2 o1 = x_ok ? xchg[r] : make_float2(kNegInfP, 0.f);
     const int n1 = ntiles > 1 ? ntiles / 2 : 0;
@@ -673,19 +776,78 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     if (__any_sync(0xffffffffu, have_o || have_o1)) tc_fence_after();
     const bool any_o = !pad_warp && __any_sync(0xffffffffu, have_o);
     const bool any_o1 = !pad_warp && __any_sync(0xffffffffu, have_o1);
+    // split rows: part p > 0 leaves (max, sum) in xchg and its normalised
+    // output in the ring's shared memory (every tile consumed); part 0 waits
+    // for them and merges the parts exactly (log-sum-exp)
+    // the ring's shared memory is free by now (every tile consumed)
+    float* xo = reinterpret_cast<float*>(base);  // [lane][D]
+    float M_all = M, l_all = l_tot;
+    float sp[T];  // part 0: the weight of each part's normalised output
+    sp[0] = 1.f;
+    if constexpr (T > 1) {
+        const bool parts_ok_in = ok && x_ok;
+        if (part > 0) xchg[r] = make_float2(l_tot > 0.f ? M : kNegInfP, l_tot);
+        if (part > 0 && !pad_warp) {  // warp-uniform: the tensor-memory loads are collective
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t u0[32], u1[32];
+                if (any_o) tmem_ld32(lane_base + L::COL_O + c0, u0);
+                if (any_o1) tmem_ld32(lane_base + L::COL_O + D + c0, u1);
+                if (any_o || any_o1) tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    float4 v;
+                    float* vv = reinterpret_cast<float*>(&v);
+#pragma unroll
+                    for (int f = 0; f < 4; ++f) {
+                        float t = any_o && w0 > 0.f ? __uint_as_float(u0[e + f]) * w0 : 0.f;
+                        if (any_o1 && w1 > 0.f) t = fmaf(__uint_as_float(u1[e + f]), w1, t);
+                        vv[f] = t;
+                    }
+                    *reinterpret_cast<float4*>(xo + (size_t)r * D + c0 + e) = v;
+                }
+            }
+        }
+        mbar_arrive(parts_bar);
+        const bool p_ok = __all_sync(0xffffffffu, mbar_wait(parts_bar, 0)) && parts_ok_in;
+        if (part == 0) {
+            float mp[T], lp[T];
+            mp[0] = l_tot > 0.f ? M : kNegInfP;
+            lp[0] = l_tot;
+#pragma unroll
+            for (int q = 1; q < T; ++q) {
+                const float2 st = p_ok ? xchg[r + 32 * q * (4 / T)] : make_float2(kNegInfP, 0.f);
+                mp[q] = st.x;
+                lp[q] = st.y;
+            }
+            M_all = kNegInfP;
+#pragma unroll
+            for (int q = 0; q < T; ++q) M_all = fmaxf(M_all, mp[q]);
+            l_all = 0.f;
+#pragma unroll
+            for (int q = 0; q < T; ++q) {
+                sp[q] = (lp[q] > 0.f && mp[q] != kNegInfP) ? lp[q] * fast_exp2(mp[q] - M_all) : 0.f;
+                l_all += sp[q];
+            }
+            const float inv_all = l_all > 0.f ? 1.f / l_all : 0.f;
+#pragma unroll
+            for (int q = 0; q < T; ++q) sp[q] *= inv_all;
+        }
+    }
+    const bool store = row.ok && part == 0;
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
         float v[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0.f;
-        if (any_o) {
+        if (part == 0 && any_o) {
             uint32_t u[32];
             tmem_ld32(lane_base + L::COL_O + c0, u);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = w0 > 0.f ? __uint_as_float(u[e]) * w0 : 0.f;
         }
-        if (any_o1) {
+        if (part == 0 && any_o1) {
             uint32_t u[32];
             tmem_ld32(lane_base + L::COL_O + D + c0, u);
             tmem_wait_ld();
@@ -693,7 +855,25 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             for (int e = 0; e < 32; ++e)
                 if (w1 > 0.f) v[e] = fmaf(__uint_as_float(u[e]), w1, v[e]);
         }
-        if (!row.ok) continue;
+        if (!store) continue;
+        if constexpr (T > 1) {
+            // the parts' normalised outputs, weighted by their share of the row's sum
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= sp[0];
+#pragma unroll
+            for (int q = 1; q < T; ++q) {
+                if (sp[q] == 0.f) continue;
+                const float* src = xo + (size_t)(r + 32 * q * (4 / T)) * D + c0;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 t = *reinterpret_cast<const float4*>(src + e);
+                    v[e] = fmaf(t.x, sp[q], v[e]);
+                    v[e + 1] = fmaf(t.y, sp[q], v[e + 1]);
+                    v[e + 2] = fmaf(t.z, sp[q], v[e + 2]);
+                    v[e + 3] = fmaf(t.w, sp[q], v[e + 3]);
+                }
+            }
+        }
         if (row.out && a.out_bf16) {
             uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(row.out) + c0);
 #pragma unroll
@@ -707,9 +887,9 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             for (int e = 0; e < 32; e += 4) o[e / 4] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
     }
-    if (row.ok && !row.out) {
-        row.pml[0] = l_tot > 0.f ? M : kNegInfP;
-        row.pml[1] = l_tot;
+    if (store && !row.out) {
+        row.pml[0] = l_all > 0.f ? M_all : kNegInfP;
+        row.pml[1] = l_all;
     }
     tc_fence_before();
     mbar_arrive(join);
@@ -743,8 +923,10 @@ __global__ void __launch_bounds__(kUThreads)
     it.npages = pit.npages;
     it.lo = pit.lo;
     URow row = {};
+    const int T = umma_split(p.C * G);
     if (warp >= 2) {
-        const int fr = pit.rg * kURows + 32 * (warp & 3) + lane;
+        // lane quadrant q holds rows (q mod 4/T) 32 + lane: each row T times
+        const int fr = pit.rg * kURows + ((warp & 3) % (4 / T)) * 32 + lane;
         row.ok = fr < p.C * G;
         const int qi = row.ok ? fr / G : 0, hq = pit.h * G + (row.ok ? fr % G : 0);
         const size_t grow = ((size_t)pit.b * p.C + qi) * p.Hq + hq;
@@ -768,7 +950,9 @@ __global__ void __launch_bounds__(kUThreads)
     a.num_blocks = p.num_blocks;
     a.out_bf16 = p.out_bf16;
     a.scale_log2 = p.scale_log2;
-    umma_attend<D>(a, it, row, &tm_k, &tm_v, base);
+    if (T == 4) umma_attend<D, 4>(a, it, row, &tm_k, &tm_v, base);
+    else if (T == 2) umma_attend<D, 2>(a, it, row, &tm_k, &tm_v, base);
+    else umma_attend<D, 1>(a, it, row, &tm_k, &tm_v, base);
 }
 
 // ---- cascade decode: the shared-prefix pass ----------------------------------
@@ -784,6 +968,7 @@ struct CascadeParams {
     int32_t* err;
     int B, Hq, Hkv, MB, NPT, RG, NG, num_blocks;
     int window;        // sliding window (0: none)
+    int split;         // tensor-memory lanes per row (umma_split of the largest group's rows)
     float scale_log2;
 };
 
@@ -890,7 +1075,7 @@ __global__ void __launch_bounds__(kUThreads)
         it.lo = first_key;
         URow row = {};
         if (warp >= 2) {
-            const int fr = rg * kURows + 32 * (warp & 3) + lane;
+            const int fr = rg * kURows + ((warp & 3) % (4 / p.split)) * 32 + lane;
             const int m = fr / G, hq = h * G + fr % G;
             const int b = gs + m;
             row.len = m < nmem ? cascade_shared(p, b) : 0;
@@ -910,7 +1095,9 @@ __global__ void __launch_bounds__(kUThreads)
         a.num_blocks = p.num_blocks;
         a.out_bf16 = 0;
         a.scale_log2 = p.scale_log2;
-        umma_attend<D>(a, it, row, &tm_k, &tm_v, base);
+        if (p.split == 4) umma_attend<D, 4>(a, it, row, &tm_k, &tm_v, base);
+        else if (p.split == 2) umma_attend<D, 2>(a, it, row, &tm_k, &tm_v, base);
+        else umma_attend<D, 1>(a, it, row, &tm_k, &tm_v, base);
     }
     // do not complete before the decode grid: the combine waits for this one
     if ((tid & 31) == 0) grid_dependency_wait();
@@ -1019,6 +1206,7 @@ cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
     p.NPT = a.slots_per_row;
     p.window = a.window;
     p.RG = (int)((a.max_group_size * G + kURows - 1) / kURows);
+    p.split = umma_split((int)(a.max_group_size * G));
     p.NG = (int)a.num_groups;
     p.num_blocks = (int)a.num_blocks;
     p.scale_log2 = a.scale * 1.4426950408889634f;
