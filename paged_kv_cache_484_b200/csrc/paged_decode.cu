@@ -307,22 +307,34 @@ __device__ __forceinline__ bf16 from_d<bf16>(double x) {
     return *reinterpret_cast<const bf16*>(&b);
 }
 
-// Fused step: a warp writes the cos/sin table of a position, tab[i] =
-// cos(pos f_i), tab[D/2 + i] = sin(pos f_i), i < D/2: angle in fp64, reduced
-// mod 2pi in fp64, then sine and cosine in fp32 of the reduced angle.
-// Lane i handles i and i + 32; `f` holds theta^(-2i/d) for those.
+// Fused step: the cos/sin table of a position, tab[i] = cos(pos f_i),
+// tab[D/2 + i] = sin(pos f_i), i < D/2: angle in fp64, reduced mod 2pi in
+// fp64, then sine and cosine in fp32 of the reduced angle; `f` holds
+// theta^(-2i/d) for the lane's i = lane + 32 u.  A warp computes its lanes'
+// entries into registers (cs[u], sn[u]) ahead of time, and stores them when
+// the stage that carries them is issued.
 template <int D>
-__device__ __forceinline__ void warp_rope_table(double pos, const double (&f)[(D + 63) / 64],
-                                                float* tab) {
+__device__ __forceinline__ void warp_rope_regs(double pos, const double (&f)[(D + 63) / 64],
+                                               float (&cs)[(D + 63) / 64],
+                                               float (&sn)[(D + 63) / 64]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int u = 0; u < (D + 63) / 64; ++u) {
+        cs[u] = 1.f;
+        sn[u] = 0.f;
+        if (lane + 32 * u < D / 2) sincosf((float)reduce_two_pi(pos * f[u]), &sn[u], &cs[u]);
+    }
+}
+template <int D>
+__device__ __forceinline__ void warp_rope_store(const float (&cs)[(D + 63) / 64],
+                                                const float (&sn)[(D + 63) / 64], float* tab) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int u = 0; u < (D + 63) / 64; ++u) {
         const int i = lane + 32 * u;
         if (i < D / 2) {
-            float sn, cs;
-            sincosf((float)reduce_two_pi(pos * f[u]), &sn, &cs);
-            tab[i] = cs;
-            tab[D / 2 + i] = sn;
+            tab[i] = cs[u];
+            tab[D / 2 + i] = sn[u];
         }
     }
 }
@@ -601,9 +613,13 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
     int cur_ent = hit ? (lane < cur.npages ? checked(guess.ent) : -1) : checked(raw_entry(cur, lane));
     // fused step: the new token's slot and position
     int64_t cur_slot = -1, cur_pos = 0;
+    // fused step: the current item's rope table, computed ahead (for the
+    // next item while this one's last stages are in flight)
+    float rope_cs[(D + 63) / 64], rope_sn[(D + 63) / 64];
     if constexpr (FUSED) {
         cur_slot = hit ? guess.slot : p.slot_mapping[cur.b];
         cur_pos = hit ? guess.pos : p.positions[cur.b];
+        warp_rope_regs<D>((double)cur_pos, guess.f, rope_cs, rope_sn);
     }
     int* patch = reinterpret_cast<int*>(base + L::OFF_PATCH);
 
@@ -722,7 +738,7 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
                 // for the bf16 / fp32 caches, with the stage that carries the
                 // new token (its k)
                 if (first || (!L::F8 && patch_row >= 0))
-                    warp_rope_table<D>((double)cur_pos, guess.f,
+                    warp_rope_store<D>(rope_cs, rope_sn,
                                        reinterpret_cast<float*>(base + L::OFF_ROPE +
                                                                 stage * L::ROPE_BYTES));
             }
@@ -754,6 +770,8 @@ __device__ void run_producer(const DecodeParams& p, const FirstItemGuess<D>& gue
         if (nitem != item) {
             item1 = take_claim();
             if (item1 < W) issue_claim();
+            // the next item's table, while this item's stages are in flight
+            if constexpr (FUSED) warp_rope_regs<D>((double)nxt_pos, guess.f, rope_cs, rope_sn);
         }
         item = nitem;
         c0 = nc0;
