@@ -905,17 +905,21 @@ namespace pkv {
 namespace {
 constexpr int kPrefillRowsPerItem = 128;  // (query, head) rows one prefill CTA serves
 
-// Partition length of a prefill call: about eight items per SM (one CTA per
-// SM at a time) if every sequence had the maximum length, in whole 64-key
-// tiles, [256, 2048].
+// Partition length of a prefill call: about two items per SM (one CTA per SM
+// at a time) if every sequence had the maximum length, in whole 64-key tiles,
+// [256, PKV_MAX_PARTITION_TOKENS].  An item pays about 6 us of set-up,
+// pipeline fill and epilogue, so few long items beat many short ones (on the
+// ragged batch at C = 16: 144 us at P = 4096 against 167 us at P = 1792, the
+// earlier choice of eight items per SM); only where the items are then fewer
+// than the SMs do shorter partitions win (batch 1, 2048 tokens: P = 256).
 int32_t prefill_auto_partition(int64_t B, int64_t C, int64_t Hq, int64_t Hkv, int64_t MB) {
     const int64_t maxlen = MB * kPageRows;
     const int64_t G = Hq / std::max<int64_t>(1, Hkv);
     const int64_t rg = ceil_div(C * G, kPrefillRowsPerItem);
-    const int64_t target = 8 * (int64_t)device_sm_count();
+    const int64_t target = 2 * (int64_t)device_sm_count();
     int64_t P = ceil_div(std::max<int64_t>(1, maxlen * B * Hkv * rg), target);
     P = ceil_div(P, 64) * 64;
-    P = std::max<int64_t>(256, std::min<int64_t>(P, 2048));
+    P = std::max<int64_t>(256, std::min<int64_t>(P, PKV_MAX_PARTITION_TOKENS));
     const int64_t floor_np = ceil_div(ceil_div(maxlen, kMaxPartitions), kPageRows) * kPageRows;
     return (int32_t)std::max(P, floor_np);
 }

@@ -300,12 +300,6 @@ __device__ __forceinline__ void tmem_wait_st() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
 // ---- 8-bit floating point (E4M3) -------------------------------------------
 // Four E4M3 codes (bytes 0..3 of `w`) -> two f16 pairs: `lo` from bytes 0, 1,
 // `hi` from bytes 2, 3 (the halves of `w` feed the conversions directly).
