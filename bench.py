@@ -498,6 +498,9 @@ def measure(cfg, args, device, world, local, rank, full: bool):
     NP = math.ceil(w.max_blocks * w.block_size / P)
     ws_bytes = pkv.decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.max_blocks, kv_dtype=kv_dt,
                                          partition_tokens=P)
+    # the calls get the caller's choice: 0 lets the library pick, which under
+    # a sliding window can be shorter than the planned P (the same workspace)
+    P_call = args.partition_tokens
     ws = pkv.new_workspace(ws_bytes, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     nbytes = step_bytes(w, out_dtype, args.window)
@@ -564,28 +567,28 @@ def measure(cfg, args, device, world, local, rank, full: bool):
             pkv.decode_step_e4m3(c["q"], c["k_new"], c["v_new"], c["positions"],
                                  c["slot_mapping"], c["k_cache"], c["block_tables"],
                                  c["decode_lens"], w.rope_theta, w.scale, ks8, vs8, out,
-                                 workspace=ws, partition_tokens=P, device_error=err,
+                                 workspace=ws, partition_tokens=P_call, device_error=err,
                                  sliding_window=args.window)
         elif e4m3:
             pkv.paged_attention_decode_e4m3(c["q"], c["k_cache"], c["block_tables"],
                                             c["decode_lens"], w.scale, ks8, vs8, out,
-                                            workspace=ws, partition_tokens=P, device_error=err,
+                                            workspace=ws, partition_tokens=P_call, device_error=err,
                                             sliding_window=args.window)
         elif fused:
             pkv.decode_step(c["q"], c["k_new"], c["v_new"], c["positions"], c["slot_mapping"],
                             c["k_cache"], c["v_cache"], c["block_tables"], c["decode_lens"],
-                            w.rope_theta, w.scale, out, workspace=ws, partition_tokens=P,
+                            w.rope_theta, w.scale, out, workspace=ws, partition_tokens=P_call,
                             force_simt=args.simt, device_error=err, sliding_window=args.window)
         elif cascade:
             pkv.paged_attention_decode_cascade(c["q"], c["k_cache"], c["v_cache"],
                                                c["block_tables"], c["decode_lens"], group_start,
                                                shared_tokens, grp, w.scale, out, workspace=ws,
-                                               partition_tokens=P, force_simt=args.simt,
+                                               partition_tokens=P_call, force_simt=args.simt,
                                                device_error=err, sliding_window=args.window)
         else:
             pkv.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
                                        c["decode_lens"], w.scale, out, workspace=ws,
-                                       partition_tokens=P, force_simt=args.simt,
+                                       partition_tokens=P_call, force_simt=args.simt,
                                        device_error=err, sliding_window=args.window)
 
     def step(k):
@@ -736,7 +739,7 @@ def measure(cfg, args, device, world, local, rank, full: bool):
                 dev_in["q"], dev_in["k_new"], dev_in["v_new"], dev_in["positions"],
                 dev_in["slot_mapping"], copies[i]["k_cache"], copies[i]["v_cache"],
                 dev_in["block_tables"], dev_in["decode_lens"], w.rope_theta, w.scale, outs[i],
-                workspace=ws, partition_tokens=P, force_simt=args.simt, device_error=err)
+                workspace=ws, partition_tokens=P_call, force_simt=args.simt, device_error=err)
                 for i in range(ncopies)]
 
             def e2e_step(k):

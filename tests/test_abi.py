@@ -190,9 +190,14 @@ def test_decode_window_rejects_bad_arguments(lib, kw, status):
 def test_e4m3_planning(lib):
     """The planning calls take the 8-bit cache dtype: the workspace follows
     the same formula; the CUDA-core kernel does not exist for it."""
-    for P in (0, 64, 1024):
+    for P in (64, 1024):
         assert lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, E4M3, P) == \
             lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, BF16, P)
+    # the automatic partition length depends on how many CTAs of the 8-bit
+    # kernel fit on an SM; the workspace follows the same formula for it
+    P8 = lib.pkv_decode_partition_tokens(16, 32, 8, 128, 8193, 16, E4M3)
+    assert lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, E4M3, 0) == \
+        lib.pkv_decode_workspace_size(16, 32, 8, 128, 8193, 16, BF16, P8)
     assert lib.pkv_decode_partition_tokens(64, 32, 8, 64, 257, 16, E4M3) > 0
     assert lib.pkv_decode_launches(4, 32, 8, 64, 16, 16, E4M3, BF16, 0, 1, 0) == 0
 
