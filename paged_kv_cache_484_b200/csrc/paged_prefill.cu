@@ -227,6 +227,18 @@ __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[N]) 
     }
 }
 
+// N consecutive columns (N = 16 or 32), loaded or stored.
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&v)[N]) {
+    if constexpr (N == 16) tmem_ld16(taddr, v);
+    else tmem_ld32(taddr, v);
+}
+template <int N>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&v)[N]) {
+    if constexpr (N == 16) tmem_st<16>(taddr, v);
+    else tmem_st32(taddr, v);
+}
+
 // Rows of an item split over T tensor-memory lanes each: an item of at most
 // 128 / T query rows stores each row T times in the 128-row tile, in lane
 // quadrants 4 / T apart, and the copy in quadrant group `part` takes the
@@ -236,14 +248,19 @@ __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[N]) 
 // thread.
 __host__ __device__ constexpr int umma_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
 
-template <int D>
+// NARROW (d = 64 only): a layout that lets two CTAs share an SM.  P is
+// written over the scores it came from (tensor memory: 2 score/P buffers and
+// 2 O accumulators, 256 columns) and the ring has 5 stages, so that two CTAs'
+// shared memory and tensor memory fit one SM.
+template <int D, bool NARROW = false>
 struct ULayout {
+    static_assert(!NARROW || D == 64, "the narrow layout is for d = 64");
     static constexpr int BOX = kPageRows * 128;                 // 16 rows x 64 bf16 columns
     static constexpr int NB = D / 64;                           // 64-column blocks of a row
     static constexpr int BLOCK_STRIDE = kUTilePages * BOX;      // between column blocks of a tile
     static constexpr int KV_BYTES = NB * BLOCK_STRIDE;          // one tile of K (or of V)
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;            // K tile, then V tile
-    static constexpr int STAGES = D == 64 ? 8 : 5;              // 128 / 160 KiB of ring
+    static constexpr int STAGES = NARROW ? 5 : (D == 64 ? 8 : 5);  // 80 / 128 / 160 KiB of ring
     static constexpr int Q_BLOCK = kURows * 128;                // one column block of Q
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
     static constexpr int PBUFS = 2;                             // P buffers, tile j uses j % 2
@@ -259,10 +276,11 @@ struct ULayout {
     static constexpr uint32_t COL_O = 128;                      // + D * warpgroup
     // P buffer b: bf16 pairs of the hi part in columns [0, 32), of the lo
     // part in [32, 64) (lane = row, column c = keys 2c and 2c + 1: the A
-    // operand layout of an MMA that reads A from tensor memory)
-    static constexpr uint32_t COL_P = COL_O + 2 * D;            // + 64 * buffer
-    static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(COL_P + 64 * PBUFS <= TMEM_COLS, "tensor memory");
+    // operand layout of an MMA that reads A from tensor memory).  NARROW:
+    // buffer b is score buffer b (tile j's P replaces its scores)
+    static constexpr uint32_t COL_P = NARROW ? COL_S : COL_O + 2 * D;  // + 64 * buffer
+    static constexpr uint32_t TMEM_COLS = NARROW ? 256 : 512;
+    static_assert(COL_O + 2 * D <= TMEM_COLS && COL_P + 64 * PBUFS <= TMEM_COLS, "tensor memory");
     static constexpr uint32_t IDESC_S = umma_idesc_bf16(kURows, kUTileKeys, false);
     static constexpr uint32_t IDESC_O = umma_idesc_bf16(kURows, D, true);
 };
@@ -293,11 +311,11 @@ struct UArgs {
 
 // Producer: the item's pages in 64-key stages (pages whose block id is out
 // of range are skipped and reported).
-template <int D>
+template <int D, bool NARROW>
 __device__ void umma_producer(const UArgs& a, const UItem& it, const CUtensorMap* tmk,
                               const CUtensorMap* tmv, uint8_t* base, uint64_t* full,
                               uint64_t* empty, uint32_t* masks, volatile int* s_abort) {
-    using L = ULayout<D>;
+    using L = ULayout<D, NARROW>;
     const int lane = threadIdx.x & 31;
     int stage = 0;
     uint32_t phase = 0;
@@ -363,12 +381,12 @@ __device__ void umma_producer(const UArgs& a, const UItem& it, const CUtensorMap
 }
 
 // The MMA lane.  Returns after its last MMA has completed (or it gave up).
-template <int D>
+template <int D, bool NARROW>
 __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* full,
                             uint64_t* empty, uint64_t* sbar, uint64_t* sfree, uint64_t* pready,
                             uint64_t* obar, uint64_t* pfree, uint64_t* mma_done,
                             volatile int* s_abort, int32_t* err) {
-    using L = ULayout<D>;
+    using L = ULayout<D, NARROW>;
     // Descriptors are built once and advanced by constant offsets: the start
     // address field holds address / 16 in its low bits (shared-memory
     // addresses stay below 2^18 bytes, so the sum never carries out of it).
@@ -405,8 +423,10 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
         umma_commit(&pfree[j % L::PBUFS]);
         umma_commit(&empty[stage]);  // the stage's K and V are no longer read
     };
-    // S_j needs its stage loaded and (j >= 2) the buffer's previous scores read;
-    // PV_j needs P_j.  Neither condition can run two phases ahead of this lane
+    // S_j needs its stage loaded and (j >= 2) the buffer's previous scores read
+    // (NARROW: O += P_{j-2} V_{j-2} issued, since that P sits where S_j goes;
+    // the MMAs of this thread run in issue order, so P_{j-2} is read before
+    // S_j overwrites it); PV_j needs P_j.  Neither condition can run two phases ahead of this lane
     // (the warpgroup's next arrivals wait for MMAs only this lane issues), so
     // each wait is on an unambiguous parity.  (Measured against this polling
     // loop: issuing every ready S first, and a fixed order S_{j+2}, PV_j after
@@ -417,7 +437,10 @@ __device__ void umma_issuer(int ntiles, uint8_t* base, uint32_t tmem, uint64_t* 
     uint32_t idle = 0;
     while (jp < ntiles) {
         bool progressed = false;
-        if (js < ntiles && (js < 2 || mbar_test_wait(&sfree[js & 1], (uint32_t)((js - 2) >> 1) & 1u)) &&
+        const bool s_buf_free =
+            js < 2 || (NARROW ? jp >= js - 1
+                              : mbar_test_wait(&sfree[js & 1], (uint32_t)((js - 2) >> 1) & 1u));
+        if (js < ntiles && s_buf_free &&
             mbar_test_wait(&full[js % L::STAGES], (uint32_t)(js / L::STAGES) & 1u)) {
             tc_fence_after();
             issue_s(js);
@@ -483,11 +506,13 @@ __device__ __forceinline__ void umma_zero_v_rows(const UItem& it, int j, int r, 
 // `row` matters to the softmax warps only).  T: tensor-memory lanes per
 // query row (umma_split): the softmax thread of lane quadrant q takes the key
 // columns of part q / (4 / T).
-template <int D, int T>
+template <int D, int T, bool NARROW = false>
 __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
                             const CUtensorMap* tmk, const CUtensorMap* tmv, uint8_t* base) {
-    using L = ULayout<D>;
+    using L = ULayout<D, NARROW>;
     constexpr int NC = kUTileKeys / T;  // key columns of a tile per softmax thread
+    // columns per tensor-memory access of O (narrow: half, for registers)
+    constexpr int EC = NARROW ? 16 : 32;
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
     uint64_t* empty = full + L::STAGES;
     uint64_t* sbar = empty + L::STAGES;
@@ -572,12 +597,12 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     }
 
     if (warp == 0) {
-        umma_producer<D>(a, it, tmk, tmv, base, full, empty, masks, s_abort);
+        umma_producer<D, NARROW>(a, it, tmk, tmv, base, full, empty, masks, s_abort);
         return;
     }
     if (warp == 1) {
         if (lane == 0) {
-            umma_issuer<D>(ntiles, base, tmem, full, empty, sbar, sfree, pready, obar, pfree,
+            umma_issuer<D, NARROW>(ntiles, base, tmem, full, empty, sbar, sfree, pready, obar, pfree,
                            mma_done, s_abort, a.err);
             (void)mbar_wait(join, 0);  // both warpgroups have read their O
         }
@@ -683,13 +708,13 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             tc_fence_after();
             const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(lane_base + col_o + c0, v);
+            for (int c0 = 0; c0 < D; c0 += EC) {
+                uint32_t v[EC];
+                tmem_ldn<EC>(lane_base + col_o + c0, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                tmem_st32(lane_base + col_o + c0, v);
+                for (int e = 0; e < EC; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                tmem_stn<EC>(lane_base + col_o + c0, v);
             }
             tmem_wait_st();
             if (need) {
@@ -710,7 +735,8 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
         float ps8[8];  // the row sum, eight independent chains
 #pragma unroll
         for (int u = 0; u < 8; ++u) ps8[u] = 0.f;
-        constexpr int CW = NC / 2 < 16 ? NC / 2 : 16;  // words per tensor-memory store
+        constexpr int CWMAX = NARROW ? 8 : 16;
+        constexpr int CW = NC / 2 < CWMAX ? NC / 2 : CWMAX;  // words per tensor-memory store
 #pragma unroll
         for (int c = 0; c < NC / 2; c += CW) {
             uint32_t hw[CW], lw[CW];
@@ -725,6 +751,21 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
             }
             tmem_st<CW>(p_col + (uint32_t)c, hw);
             tmem_st<CW>(p_col + 32u + (uint32_t)c, lw);
+        }
+        if constexpr (NARROW && T > 1) {
+            // P replaced the scores: the other parts' columns of this lane
+            // still hold scores and must read as zero
+            uint32_t z[CW];
+#pragma unroll
+            for (int e = 0; e < CW; ++e) z[e] = 0u;
+            const uint32_t p_buf = lane_base + L::COL_P + (uint32_t)((j % L::PBUFS) * 64);
+#pragma unroll
+            for (int c = 0; c < 32; c += CW) {
+                // warp-uniform: a warp is one part
+                if (c >= c_first / 2 && c < c_first / 2 + NC / 2) continue;
+                tmem_st<CW>(p_buf + (uint32_t)c, z);
+                tmem_st<CW>(p_buf + 32u + (uint32_t)c, z);
+            }
         }
         tmem_wait_st();
         l_run += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
@@ -789,13 +830,13 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
         if (part > 0) xchg[r] = make_float2(l_tot > 0.f ? M : kNegInfP, l_tot);
         if (part > 0 && !pad_warp) {  // warp-uniform: the tensor-memory loads are collective
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t u0[32], u1[32];
-                if (any_o) tmem_ld32(lane_base + L::COL_O + c0, u0);
-                if (any_o1) tmem_ld32(lane_base + L::COL_O + D + c0, u1);
+            for (int c0 = 0; c0 < D; c0 += EC) {
+                uint32_t u0[EC], u1[EC];
+                if (any_o) tmem_ldn<EC>(lane_base + L::COL_O + c0, u0);
+                if (any_o1) tmem_ldn<EC>(lane_base + L::COL_O + D + c0, u1);
                 if (any_o || any_o1) tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
+                for (int e = 0; e < EC; e += 4) {
                     float4 v;
                     float* vv = reinterpret_cast<float*>(&v);
 #pragma unroll
@@ -836,36 +877,36 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
     }
     const bool store = row.ok && part == 0;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-        float v[32];
+    for (int c0 = 0; c0 < D; c0 += EC) {
+        float v[EC];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        for (int e = 0; e < EC; ++e) v[e] = 0.f;
         if (part == 0 && any_o) {
-            uint32_t u[32];
-            tmem_ld32(lane_base + L::COL_O + c0, u);
+            uint32_t u[EC];
+            tmem_ldn<EC>(lane_base + L::COL_O + c0, u);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = w0 > 0.f ? __uint_as_float(u[e]) * w0 : 0.f;
+            for (int e = 0; e < EC; ++e) v[e] = w0 > 0.f ? __uint_as_float(u[e]) * w0 : 0.f;
         }
         if (part == 0 && any_o1) {
-            uint32_t u[32];
-            tmem_ld32(lane_base + L::COL_O + D + c0, u);
+            uint32_t u[EC];
+            tmem_ldn<EC>(lane_base + L::COL_O + D + c0, u);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
+            for (int e = 0; e < EC; ++e)
                 if (w1 > 0.f) v[e] = fmaf(__uint_as_float(u[e]), w1, v[e]);
         }
         if (!store) continue;
         if constexpr (T > 1) {
             // the parts' normalised outputs, weighted by their share of the row's sum
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= sp[0];
+            for (int e = 0; e < EC; ++e) v[e] *= sp[0];
 #pragma unroll
             for (int q = 1; q < T; ++q) {
                 if (sp[q] == 0.f) continue;
                 const float* src = xo + (size_t)(r + 32 * q * (4 / T)) * D + c0;
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
+                for (int e = 0; e < EC; e += 4) {
                     const float4 t = *reinterpret_cast<const float4*>(src + e);
                     v[e] = fmaf(t.x, sp[q], v[e]);
                     v[e + 1] = fmaf(t.y, sp[q], v[e + 1]);
@@ -877,14 +918,14 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
         if (row.out && a.out_bf16) {
             uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(row.out) + c0);
 #pragma unroll
-            for (int e = 0; e < 32; e += 8)
+            for (int e = 0; e < EC; e += 8)
                 o[e / 8] = make_uint4(pack_bf16(v[e], v[e + 1]), pack_bf16(v[e + 2], v[e + 3]),
                                       pack_bf16(v[e + 4], v[e + 5]), pack_bf16(v[e + 6], v[e + 7]));
         } else {
             float4* o = reinterpret_cast<float4*>(row.out ? reinterpret_cast<float*>(row.out) + c0
                                                           : row.po + c0);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) o[e / 4] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            for (int e = 0; e < EC; e += 4) o[e / 4] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
     }
     if (store && !row.out) {
@@ -897,9 +938,12 @@ __device__ void umma_attend(const UArgs& a, const UItem& it, const URow& row,
 
 // Chunked prefill: item (sequence, kv head, row group of 128 rows,
 // partition); row fr of the group is (query fr / G, head fr % G); query i
-// sits at position L - C + i and attends keys up to it.
-template <int D, int G>
-__global__ void __launch_bounds__(kUThreads)
+// sits at position L - C + i and attends keys up to it.  T = umma_split(C G)
+// tensor-memory lanes per row.  NARROW (d = 64 with split rows, more items
+// than SMs): the narrow layout lets two CTAs share an SM (at most 102
+// registers a thread).
+template <int D, int G, int T, bool NARROW>
+__global__ void __launch_bounds__(kUThreads, NARROW ? 2 : 1)
     paged_prefill_umma_kernel(const __grid_constant__ PrefillParams p,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v) {
@@ -923,7 +967,6 @@ __global__ void __launch_bounds__(kUThreads)
     it.npages = pit.npages;
     it.lo = pit.lo;
     URow row = {};
-    const int T = umma_split(p.C * G);
     if (warp >= 2) {
         // lane quadrant q holds rows (q mod 4/T) 32 + lane: each row T times
         const int fr = pit.rg * kURows + ((warp & 3) % (4 / T)) * 32 + lane;
@@ -950,9 +993,7 @@ __global__ void __launch_bounds__(kUThreads)
     a.num_blocks = p.num_blocks;
     a.out_bf16 = p.out_bf16;
     a.scale_log2 = p.scale_log2;
-    if (T == 4) umma_attend<D, 4>(a, it, row, &tm_k, &tm_v, base);
-    else if (T == 2) umma_attend<D, 2>(a, it, row, &tm_k, &tm_v, base);
-    else umma_attend<D, 1>(a, it, row, &tm_k, &tm_v, base);
+    umma_attend<D, T, NARROW>(a, it, row, &tm_k, &tm_v, base);
 }
 
 // ---- cascade decode: the shared-prefix pass ----------------------------------
@@ -1122,12 +1163,13 @@ cudaError_t set_smem_once(K kern, size_t smem) {
     return e;
 }
 
-// The tensor-core (tcgen05) prefill: one 128-row item per CTA, one CTA per SM.
-template <int D, int G>
-cudaError_t launch_prefill_umma_typed(const PrefillArgs& a, const CUtensorMap& tmk,
+// The tensor-core (tcgen05) prefill: one 128-row item per CTA; one CTA per
+// SM, two with the narrow layout.
+template <int D, int G, int T, bool NARROW>
+cudaError_t launch_prefill_umma_split(const PrefillArgs& a, const CUtensorMap& tmk,
                                       const CUtensorMap& tmv) {
-    using L = ULayout<D>;
-    auto kern = paged_prefill_umma_kernel<D, G>;
+    using L = ULayout<D, NARROW>;
+    auto kern = paged_prefill_umma_kernel<D, G, T, NARROW>;
     cudaError_t e = set_smem_once(kern, L::SMEM);
     if (e != cudaSuccess) return e;
     PrefillParams p;
@@ -1170,6 +1212,25 @@ cudaError_t launch_prefill_umma_typed(const PrefillArgs& a, const CUtensorMap& t
     cc.blockDim = dim3(128);
     cc.dynamicSmemBytes = 0;
     return cudaLaunchKernelEx(&cc, prefill_combine_kernel<D>, p);
+}
+
+// Two CTAs per SM pay where the items outnumber the SMs (at batch 1, 64
+// items on 148 SMs, a shared SM only slows its pair: 16.1 -> 16.9 us).
+template <int D, int G>
+cudaError_t launch_prefill_umma_typed(const PrefillArgs& a, const CUtensorMap& tmk,
+                                      const CUtensorMap& tmv) {
+    const int64_t items =
+        a.B * a.Hkv * ((a.C * G + kURows - 1) / kURows) * (int64_t)a.max_partitions;
+    const bool narrow = D == 64 && items > (int64_t)device_sm_count();
+    switch (umma_split((int)(a.C * G))) {
+        case 4:
+            return narrow ? launch_prefill_umma_split<D, G, 4, (D == 64)>(a, tmk, tmv)
+                          : launch_prefill_umma_split<D, G, 4, false>(a, tmk, tmv);
+        case 2:
+            return narrow ? launch_prefill_umma_split<D, G, 2, (D == 64)>(a, tmk, tmv)
+                          : launch_prefill_umma_split<D, G, 2, false>(a, tmk, tmv);
+        default: return launch_prefill_umma_split<D, G, 1, false>(a, tmk, tmv);
+    }
 }
 
 template <int D>
