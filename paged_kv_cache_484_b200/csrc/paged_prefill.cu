@@ -72,7 +72,8 @@ struct PItem {
     int lo;  // sliding window: first token any query of the chunk attends (0 otherwise)
 };
 
-__device__ __forceinline__ PItem prefill_item(const PrefillParams& p) {
+// order: the sequences longest first (null: in order).
+__device__ __forceinline__ PItem prefill_item(const PrefillParams& p, const int* order) {
     PItem it;
     int x = blockIdx.x;
     it.part = x % p.NP;
@@ -80,7 +81,7 @@ __device__ __forceinline__ PItem prefill_item(const PrefillParams& p) {
     it.rg = x % p.RG;
     x /= p.RG;
     it.h = x % p.Hkv;
-    it.b = x / p.Hkv;
+    it.b = order ? order[x / p.Hkv] : x / p.Hkv;
     int L = p.context_lens[it.b];
     const int maxlen = p.MB * kPageRows;
     if (L < p.C || L > maxlen) {
@@ -957,7 +958,30 @@ __global__ void __launch_bounds__(kUThreads, NARROW ? 2 : 1)
     }
     grid_dependency_wait();
     grid_launch_dependents();
-    const PItem pit = prefill_item(p);
+    // Longest first: CTAs start in blockIdx order, so the items of the
+    // longest contexts go first and the last wave holds the short ones.
+    // Every CTA ranks the lengths (the ring's memory is free until the item
+    // starts).
+    int* s_order = reinterpret_cast<int*>(base);
+    int* s_len = s_order + p.B;
+    const bool lpt = p.B <= kUThreads;
+    if (lpt) {
+        const int t = threadIdx.x;
+        if (t < p.B) s_len[t] = p.context_lens[t];
+        __syncthreads();
+        if (t < p.B) {
+            const int Lt = s_len[t];
+            int rank = 0;
+#pragma unroll 8
+            for (int b2 = 0; b2 < p.B; ++b2) {
+                const int L2 = s_len[b2];
+                rank += (L2 > Lt) || (L2 == Lt && b2 < t);
+            }
+            s_order[rank] = t;
+        }
+        __syncthreads();
+    }
+    const PItem pit = prefill_item(p, lpt ? s_order : nullptr);
     if (pit.part >= pit.np) return;  // no keys in this partition (uniform: the whole CTA leaves)
     UItem it;
     it.b = pit.b;
