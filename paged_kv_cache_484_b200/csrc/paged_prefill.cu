@@ -1072,9 +1072,10 @@ __device__ __forceinline__ int cascade_lo(const CascadeParams& p, int b) {
 // decode writes; q was rotated before the decode began), so its CTAs fill
 // SMs as the decode's CTAs finish; each CTA waits for the decode grid before
 // it exits, so that the combine, which waits for this grid, also sees the
-// decode's partials.
-template <int D, int G>
-__global__ void __launch_bounds__(kUThreads)
+// decode's partials.  T = p.split; NARROW as for the prefill (two CTAs per
+// SM at d = 64 with split rows).
+template <int D, int G, int T, bool NARROW>
+__global__ void __launch_bounds__(kUThreads, NARROW ? 2 : 1)
     cascade_prefix_kernel(const __grid_constant__ CascadeParams p,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v) {
@@ -1160,9 +1161,7 @@ __global__ void __launch_bounds__(kUThreads)
         a.num_blocks = p.num_blocks;
         a.out_bf16 = 0;
         a.scale_log2 = p.scale_log2;
-        if (p.split == 4) umma_attend<D, 4>(a, it, row, &tm_k, &tm_v, base);
-        else if (p.split == 2) umma_attend<D, 2>(a, it, row, &tm_k, &tm_v, base);
-        else umma_attend<D, 1>(a, it, row, &tm_k, &tm_v, base);
+        umma_attend<D, T, NARROW>(a, it, row, &tm_k, &tm_v, base);
     }
     // do not complete before the decode grid: the combine waits for this one
     if ((tid & 31) == 0) grid_dependency_wait();
@@ -1268,11 +1267,11 @@ cudaError_t prefill_dispatch_g(const PrefillArgs& a, const CUtensorMap& k, const
     return cudaErrorInvalidValue;
 }
 
-template <int D, int G>
-cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
+template <int D, int G, int T, bool NARROW>
+cudaError_t launch_cascade_split(const CascadeArgs& a, const CUtensorMap& tmk,
                                  const CUtensorMap& tmv) {
-    using L = ULayout<D>;
-    auto kern = cascade_prefix_kernel<D, G>;
+    using L = ULayout<D, NARROW>;
+    auto kern = cascade_prefix_kernel<D, G, T, NARROW>;
     cudaError_t e = set_smem_once(kern, L::SMEM);
     if (e != cudaSuccess) return e;
     CascadeParams p;
@@ -1306,6 +1305,22 @@ cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, p, tmk, tmv);
+}
+
+template <int D, int G>
+cudaError_t launch_cascade_typed(const CascadeArgs& a, const CUtensorMap& tmk,
+                                 const CUtensorMap& tmv) {
+    const int64_t items = a.num_groups * a.Hkv * ((a.max_group_size * G + kURows - 1) / kURows);
+    const bool narrow = D == 64 && items > (int64_t)device_sm_count();
+    switch (umma_split((int)(a.max_group_size * G))) {
+        case 4:
+            return narrow ? launch_cascade_split<D, G, 4, (D == 64)>(a, tmk, tmv)
+                          : launch_cascade_split<D, G, 4, false>(a, tmk, tmv);
+        case 2:
+            return narrow ? launch_cascade_split<D, G, 2, (D == 64)>(a, tmk, tmv)
+                          : launch_cascade_split<D, G, 2, false>(a, tmk, tmv);
+        default: return launch_cascade_split<D, G, 1, false>(a, tmk, tmv);
+    }
 }
 
 template <int D>
