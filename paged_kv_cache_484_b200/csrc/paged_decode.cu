@@ -1758,10 +1758,16 @@ struct CombineParams {
 //   * every thread owns one float4 column chunk of one partition group and
 //     loads its first partials before the weights are known;
 //   * all heads' column sums meet in shared memory once, then are reduced.
-constexpr int kCombineThreads = 256;
+// Threads per combine CTA: one warp per head for the weights, four warps at
+// least.  At 128 threads (G <= 4) the ragged batch's 512 CTAs are resident at
+// once (at 256 threads and 80 registers three fit an SM, and 68 CTAs waited
+// for the first ones to leave).
+template <int G>
+constexpr int combine_threads() { return G <= 4 ? 128 : 32 * G; }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_constant__ CombineParams p) {
+__global__ void __launch_bounds__(combine_threads<G>()) combine_kernel(const __grid_constant__ CombineParams p) {
+    constexpr int kCombineThreads = combine_threads<G>();
     constexpr int CH = D / 4;                   // float4 chunks per row
     constexpr int PG = kCombineThreads / CH;    // partition groups
     constexpr int kCombineUnroll = G >= 8 ? 1 : 8 / G;  // partitions in flight per head
@@ -1769,9 +1775,6 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_c
     float4* red = smem4;                                        // [G][PG][CH]
     float* w = reinterpret_cast<float*>(smem4 + G * PG * CH);   // [G][NP]
     grid_dependency_wait();
-    // the next launch (the next step's decode) may start its prologue now;
-    // its own wait still orders it after this grid's writes
-    grid_launch_dependents();
     const int b = blockIdx.y, h = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t hq0 = (size_t)b * p.Hq + (size_t)h * G;
@@ -1896,6 +1899,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_c
         store_out(p.out, o + 2, sum.z, p.out_bf16);
         store_out(p.out, o + 3, sum.w, p.out_bf16);
     }
+    // the next launch (the next step's decode) starts once every CTA of this
+    // grid is done or here (a CTA that returned early counts as done), so
+    // that its CTAs find the SMs free; its own wait still orders it after
+    // this grid's writes
+    grid_launch_dependents();
 }
 
 // ------------------------------------------------------------------- host
@@ -2088,17 +2096,17 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, const CUtensorMap& tmk,
         static size_t set_bytes[64] = {0};
         const int dev = current_device();
         std::lock_guard<std::mutex> lock(mu);
-        if (dev >= 0 && dev < 64 && set_bytes[dev] < (size_t)(G * kCombineThreads * 16 + G * kMaxPartitions * 4)) {
+        if (dev >= 0 && dev < 64 && set_bytes[dev] < (size_t)(G * combine_threads<G>() * 16 + G * kMaxPartitions * 4)) {
             e = cudaFuncSetAttribute(ckern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     G * kCombineThreads * 16 + G * kMaxPartitions * 4);
+                                     G * combine_threads<G>() * 16 + G * kMaxPartitions * 4);
             if (e != cudaSuccess) return e;
-            set_bytes[dev] = (size_t)(G * kCombineThreads * 16 + G * kMaxPartitions * 4);
+            set_bytes[dev] = (size_t)(G * combine_threads<G>() * 16 + G * kMaxPartitions * 4);
         }
     }
-    const size_t csmem = (size_t)G * kCombineThreads * 16 + (size_t)G * a.max_partitions * sizeof(float);
+    const size_t csmem = (size_t)G * combine_threads<G>() * 16 + (size_t)G * a.max_partitions * sizeof(float);
     cudaLaunchConfig_t cc = cfg;
     cc.gridDim = dim3((unsigned)a.Hkv, (unsigned)a.B);
-    cc.blockDim = dim3(kCombineThreads);
+    cc.blockDim = dim3(combine_threads<G>());
     cc.dynamicSmemBytes = csmem;
     return cudaLaunchKernelEx(&cc, ckern, cp);
 }

@@ -196,3 +196,30 @@ def test_prefill_sliding_window(d, G, C, W, P):
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     _check(out, want, f"window {W} d{d} G{G} C{C} P{P}")
+
+
+def test_prefill_full_ragged_batch_sampled():
+    """The chunked-prefill workload at full size (the ragged batch of 64
+    sequences, 32/8 heads, d 64, C = 16, the library's partition length, as
+    the benchmark times it: two CTAs per SM, longest contexts first), checked
+    on the longest, a middle and the shortest context against the oracle run
+    on just those sequences."""
+    C = 16
+    w = W.make_config(3, device=DEV)
+    lens = w.cached_lens.clamp(min=C).to(torch.int32)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(487)
+    q = torch.randn((w.B, C, w.Hq, w.d), generator=g, device=DEV, dtype=torch.bfloat16)
+    out = torch.empty((w.B, C, w.Hq, w.d), dtype=torch.float32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.paged_attention_prefill(q, w.k_cache, w.v_cache, w.block_tables, lens, w.scale, out,
+                                device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    order = torch.argsort(lens.cpu(), descending=True).tolist()
+    kc, vc = w.k_cache.cpu(), w.v_cache.cpu()
+    for b in (order[0], order[len(order) // 2], order[-1]):
+        want = oracle.paged_chunked_prefill(q[b:b + 1].cpu(), kc, vc,
+                                            w.block_tables[b:b + 1].cpu(),
+                                            lens[b:b + 1].cpu(), w.scale, nthreads=8)
+        _check(out[b:b + 1], want, f"sequence {b} (context {int(lens[b])})")
