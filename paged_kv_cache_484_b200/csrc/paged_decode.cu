@@ -361,8 +361,11 @@ __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_
 // the staged K and V pages (overwriting what the TMA brought) and into the
 // cache rows in global memory; then orders its shared-memory writes before
 // any later TMA write into the same stage.
+// Out of line: it runs once per sequence, and inlined into the consumers'
+// page loop it cost the fused d = 64 kernel 6 registers and a spill (ragged
+// batch 56.6 -> 55.5 us out of line).
 template <typename T, int D>
-__device__ void patch_new_row(uint8_t* kpage, uint8_t* vpage, const uint8_t* newkv, int r,
+__device__ __noinline__ void patch_new_row(uint8_t* kpage, uint8_t* vpage, const uint8_t* newkv, int r,
                               const float* tab, T* kglob, T* vglob) {
     constexpr int HALF = D / 2, E = 16 / (int)sizeof(T), CH = D * (int)sizeof(T) / 16;
     const int lane = threadIdx.x & 31;
@@ -408,7 +411,7 @@ __device__ __forceinline__ void patch_new_codes(uint8_t* kpage, uint8_t* vpage,
 // and v still go into a valid slot, as kv_append would put them.  Run by the
 // consumer threads of one CTA.
 template <int D>
-__device__ void append_only_e4m3(const DecodeParams& p, const RopeFreq& fr, int b) {
+__device__ __noinline__ void append_only_e4m3(const DecodeParams& p, const RopeFreq& fr, int b) {
     constexpr int HALF = D / 2;
     const double pos = (double)p.positions[b];
     const int64_t slot = p.slot_mapping[b];
@@ -439,7 +442,7 @@ __device__ void append_only_e4m3(const DecodeParams& p, const RopeFreq& fr, int 
 }
 
 template <typename T, int D>
-__device__ void append_only(const DecodeParams& p, const RopeFreq& fr, int b) {
+__device__ __noinline__ void append_only(const DecodeParams& p, const RopeFreq& fr, int b) {
     constexpr int HALF = D / 2;
     const double pos = (double)p.positions[b];
     const int64_t slot = p.slot_mapping[b];
